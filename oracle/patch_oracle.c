@@ -1,0 +1,467 @@
+/*
+ * patch_oracle.c -- plain, slow, obviously-correct CPU oracle for the
+ * tile-hybrid (dense / 2:4) Wanda-masked linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path
+ * (the CUDA library and its Python binding) never calls it, and this file
+ * shares no code, header, table or constant generator with the CUDA path.
+ *
+ * Arithmetic is IEEE fp64 throughout.  Build with -ffp-contract=off so that
+ * no multiply-add is fused: every sum below is a chain of separately rounded
+ * additions in the order written.  OpenMP splits work only across
+ * independent output rows / columns, so the per-element order, and therefore
+ * every bit of every result, is independent of the thread count.
+ *
+ * What is computed, and where it comes from:
+ *   - Wanda importance |W_ij| * ||X_:,j||_2 over calibration tokens:
+ *     "SparseGPT vs Wanda: one-shot LLM pruning without retraining",
+ *     section "Wanda: simplicity of activation-aware pruning" (the page says
+ *     the weight magnitude times the input activation of that channel; the
+ *     activation term is read as the l2 norm over calibration tokens).
+ *   - 2:4 groups (keep 2 of every 4 consecutive input channels) and the six
+ *     possible keep patterns: "PATCH: Learnable Tile-level Hybrid Sparsity
+ *     for LLMs", section 1 (problem statement, semi-structured 2:4) and
+ *     section 2 (methodology, pattern choice among 6 permutations).
+ *   - tiles of b1 x b2, each either dense (0% sparse) or 2:4 (50% sparse):
+ *     same PATCH page, section 2, core mechanism.
+ *   - the per-tile choice is learned in PATCH; here it is either given by the
+ *     caller or taken as the tiles whose 2:4 pruning loses the least Wanda
+ *     score (a data-free stand-in for the learned map; PATCH-Tile, section 2
+ *     variants, freezes 2:4 patterns from a one-shot method).
+ *   - compressed storage is required for any speedup: SparseGPT-vs-Wanda
+ *     page, section on structured vs unstructured sparsity.  The packed
+ *     layout itself is this library's own format (documented in
+ *     include/patch.h); pack/unpack here are an independent restatement.
+ *
+ * Parity pins for every function live in tests/test_oracle.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ */
+/* bf16 helpers                                                        */
+/* ------------------------------------------------------------------ */
+
+/* Exact widening of a bf16 bit pattern to double (bf16 is the top half of
+ * an IEEE binary32). */
+static double bf16_bits_to_f64(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* |w| taken on the bits: clear the sign, so -0 becomes +0. */
+static double bf16_abs_to_f64(uint16_t b) {
+    return bf16_bits_to_f64((uint16_t)(b & 0x7FFFu));
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 1: column sum of squares of the calibration activations         */
+/* ------------------------------------------------------------------ */
+
+/*
+ * s[j] = sum over calibration tokens t of x[t,j]^2, in this fixed order:
+ *   tokens are cut into consecutive chunks of `chunk` tokens (the last
+ *   chunk may be short); inside a chunk the squares are added one token
+ *   after another, starting from 0.0; the chunk partials are then added one
+ *   chunk after another, starting from 0.0.
+ * A bf16 value squared is exact in fp64, so only the additions round.
+ * Xcal is [T, K] row-major bf16 bits.
+ */
+void oracle_colsq(const uint16_t *Xcal, int64_t T, int64_t K, int64_t chunk,
+                  double *s) {
+    double *part = (double *)malloc(sizeof(double) * (size_t)K);
+    for (int64_t j = 0; j < K; ++j) s[j] = 0.0;
+    for (int64_t c0 = 0; c0 < T; c0 += chunk) {
+        int64_t c1 = c0 + chunk < T ? c0 + chunk : T;
+        for (int64_t j = 0; j < K; ++j) part[j] = 0.0;
+        for (int64_t t = c0; t < c1; ++t) {
+            const uint16_t *row = Xcal + t * K;
+#pragma omp parallel for schedule(static)
+            for (int64_t j = 0; j < K; ++j) {
+                double x = bf16_bits_to_f64(row[j]);
+                part[j] = part[j] + x * x;
+            }
+        }
+        for (int64_t j = 0; j < K; ++j) s[j] = s[j] + part[j];
+    }
+    free(part);
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 2: Wanda scores                                                 */
+/* ------------------------------------------------------------------ */
+
+/*
+ * score[i,j] = |W[i,j]| * sqrt(s[j]).  sqrt is the correctly rounded IEEE
+ * square root; the product is one rounded fp64 multiply.
+ */
+void oracle_wanda_scores(const uint16_t *W, const double *s, int64_t N,
+                         int64_t K, double *score) {
+    double *norm = (double *)malloc(sizeof(double) * (size_t)K);
+    for (int64_t j = 0; j < K; ++j) norm[j] = sqrt(s[j]);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i)
+        for (int64_t j = 0; j < K; ++j)
+            score[i * K + j] = bf16_abs_to_f64(W[i * K + j]) * norm[j];
+    free(norm);
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 3: top-2-of-4 selection and its 4-bit code                      */
+/* ------------------------------------------------------------------ */
+
+/*
+ * For row i and group g (columns 4g..4g+3) keep the two candidates that come
+ * first when ordered by (score descending, column index ascending): the
+ * highest scores win and a tie goes to the lower index.  With idx0 < idx1 the
+ * kept positions inside the group, the code is idx0 | (idx1 << 2).  Group g
+ * of row i is stored in bits 4*(g%8) .. 4*(g%8)+3 of meta[i, g/8] (K/32 words
+ * per row).
+ */
+static unsigned select_group(const double *sc) {
+    /* first pick: the largest score, lowest index on ties (strict >) */
+    int a = 0;
+    for (int q = 1; q < 4; ++q)
+        if (sc[q] > sc[a]) a = q;
+    /* second pick: the largest among the other three, lowest index on ties */
+    int b = -1;
+    for (int q = 0; q < 4; ++q) {
+        if (q == a) continue;
+        if (b < 0 || sc[q] > sc[b]) b = q;
+    }
+    int lo = a < b ? a : b, hi = a < b ? b : a;
+    return (unsigned)(lo | (hi << 2));
+}
+
+void oracle_select_2of4(const double *score, int64_t N, int64_t K,
+                        uint32_t *meta) {
+    int64_t words = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+        for (int64_t w = 0; w < words; ++w) {
+            uint32_t word = 0;
+            for (int g8 = 0; g8 < 8; ++g8) {
+                int64_t col = w * 32 + g8 * 4;
+                unsigned code = select_group(score + i * K + col);
+                word |= (uint32_t)code << (4 * g8);
+            }
+            meta[i * words + w] = word;
+        }
+    }
+}
+
+/* Is column j of row i kept by the 2:4 code in meta? */
+static int kept(const uint32_t *meta, int64_t K, int64_t i, int64_t j) {
+    uint32_t word = meta[i * (K / 32) + j / 32];
+    unsigned code = (word >> (4 * ((j % 32) / 4))) & 0xFu;
+    unsigned pos = (unsigned)(j % 4);
+    return pos == (code & 3u) || pos == (code >> 2);
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 4: per-tile loss of 2:4 pruning                                  */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Tiles are tn x tk, numbered row-major: t = (i/tn)*(K/tk) + (j/tk).
+ * loss[t] = the Wanda score that 2:4 pruning would remove from tile t:
+ * every row of the tile sums its pruned scores left to right from 0.0, then
+ * the row sums are added top to bottom from 0.0.
+ */
+void oracle_tile_loss(const double *score, const uint32_t *meta, int64_t N,
+                      int64_t K, int64_t tn, int64_t tk, double *loss) {
+    int64_t tiles_k = K / tk, tiles_n = N / tn;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < tiles_n * tiles_k; ++t) {
+        int64_t i0 = (t / tiles_k) * tn, j0 = (t % tiles_k) * tk;
+        double total = 0.0;
+        for (int64_t i = i0; i < i0 + tn; ++i) {
+            double row = 0.0;
+            for (int64_t j = j0; j < j0 + tk; ++j)
+                if (!kept(meta, K, i, j)) row = row + score[i * K + j];
+            total = total + row;
+        }
+        loss[t] = total;
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 5: tile map                                                      */
+/* ------------------------------------------------------------------ */
+
+/* Number of 2:4 tiles for a target fraction f: floor(f * n_tiles). */
+int64_t oracle_n_sparse(double f, int64_t n_tiles) {
+    return (int64_t)floor(f * (double)n_tiles);
+}
+
+typedef struct { double loss; int64_t t; } keyed_tile;
+
+static int cmp_keyed(const void *pa, const void *pb) {
+    const keyed_tile *a = (const keyed_tile *)pa, *b = (const keyed_tile *)pb;
+    if (a->loss < b->loss) return -1;
+    if (a->loss > b->loss) return 1;
+    return a->t < b->t ? -1 : (a->t > b->t ? 1 : 0);
+}
+
+/*
+ * Order the tiles by (loss ascending, tile index ascending) and mark the
+ * first n_sparse as 2:4.  Bit t%32 of map[t/32] is 1 for a 2:4 tile.
+ */
+void oracle_select_map(const double *loss, int64_t n_tiles, int64_t n_sparse,
+                       uint32_t *map) {
+    keyed_tile *kt = (keyed_tile *)malloc(sizeof(keyed_tile) * (size_t)n_tiles);
+    for (int64_t t = 0; t < n_tiles; ++t) { kt[t].loss = loss[t]; kt[t].t = t; }
+    qsort(kt, (size_t)n_tiles, sizeof(keyed_tile), cmp_keyed);
+    for (int64_t w = 0; w < (n_tiles + 31) / 32; ++w) map[w] = 0;
+    for (int64_t r = 0; r < n_sparse && r < n_tiles; ++r)
+        map[kt[r].t / 32] |= 1u << (kt[r].t % 32);
+    free(kt);
+}
+
+static int tile_is_sparse(const uint32_t *map, int64_t t) {
+    return (int)((map[t / 32] >> (t % 32)) & 1u);
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 6: effective weight                                              */
+/* ------------------------------------------------------------------ */
+
+/*
+ * W_eff = W on dense tiles; on 2:4 tiles the kept entries of W and +0
+ * elsewhere.  Output is bf16 bits.
+ */
+void oracle_weff(const uint16_t *W, const uint32_t *meta, const uint32_t *map,
+                 int64_t N, int64_t K, int64_t tn, int64_t tk, uint16_t *weff) {
+    int64_t tiles_k = K / tk;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i)
+        for (int64_t j = 0; j < K; ++j) {
+            int64_t t = (i / tn) * tiles_k + j / tk;
+            uint16_t w = W[i * K + j];
+            if (tile_is_sparse(map, t) && !kept(meta, K, i, j)) w = 0;
+            weff[i * K + j] = w;
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 7: the packed layout, restated independently                    */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Packed layout (this library's own format; the header include/patch.h is
+ * its normative statement).  Geometry: bands of 128 rows, k-steps of 64
+ * columns, k-pairs of 128 columns.
+ *   - A k-step (band b, step c) is stored 2:4-compressed iff every tile of
+ *     the map that overlaps rows [128b, 128b+128) x cols [64c, 64c+64) is a
+ *     2:4 tile; otherwise it is stored dense, holding W_eff.
+ *   - Bands are stored one after another; inside a band, k-steps in order.
+ *   - dense k-step: 16384 bytes, element (r, k), r<128, k<64 at byte
+ *       (r/8)*1024 + (r%8)*128 + (((k/8) ^ (r%8)) * 16) + (k%8)*2.
+ *   - 2:4 k-step: 8192 bytes of kept values.  Kept value v (v<32, in
+ *     increasing column order; two per group of 4) of row r at byte
+ *       (r/8)*512 + (r%8)*64 + (((v/8) ^ ((r%8)/2)) * 16) + (v%8)*2.
+ *   - metadata block: 2048 bytes per (band, k-pair) that holds at least one
+ *     2:4 k-step, stored directly before the values of the first 2:4 k-step
+ *     of that pair.  For row m = m0 + 8*m1 + 16*m2 (m0<8, m1<2, m2<8) and
+ *     pair column k = k0 + 16*k1 + 32*k2 (k0<16, k1<2, k2<4), the code bit of
+ *     logical column k lives in 16-byte line (m0 + 8*k1 + 16*m2) at bit
+ *     (32*k2 + 16*m1 + k0); a group's 4-bit code occupies its four columns'
+ *     bits, least significant bit first.  Bits of dense k-steps are zero.
+ *   - table[b*(K/64) + c] (uint64): bits 0..47 byte offset of the k-step's
+ *     data (values for 2:4, the matrix for dense); bit 62 set for 2:4;
+ *     bit 63 set when the pair's metadata block sits right before it.
+ */
+#define BAND 128
+#define KSTEP 64
+
+static int kstep_sparse(const uint32_t *map, int64_t K, int64_t tn, int64_t tk,
+                        int64_t b, int64_t c) {
+    int64_t tiles_k = K / tk;
+    for (int64_t ti = (b * BAND) / tn; ti <= (b * BAND + BAND - 1) / tn; ++ti)
+        for (int64_t tj = (c * KSTEP) / tk; tj <= (c * KSTEP + KSTEP - 1) / tk;
+             ++tj)
+            if (!tile_is_sparse(map, ti * tiles_k + tj)) return 0;
+    return 1;
+}
+
+/* Total packed bytes for this map. */
+int64_t oracle_pack_bytes(const uint32_t *map, int64_t N, int64_t K, int64_t tn,
+                          int64_t tk) {
+    int64_t total = 0, steps = K / KSTEP;
+    for (int64_t b = 0; b < N / BAND; ++b)
+        for (int64_t c = 0; c < steps; ++c) {
+            if (kstep_sparse(map, K, tn, tk, b, c)) {
+                int first_in_pair = (c % 2 == 0) ||
+                                    !kstep_sparse(map, K, tn, tk, b, c - 1);
+                total += 8192 + (first_in_pair ? 2048 : 0);
+            } else {
+                total += 16384;
+            }
+        }
+    return total;
+}
+
+void oracle_pack(const uint16_t *W, const uint32_t *meta, const uint32_t *map,
+                 int64_t N, int64_t K, int64_t tn, int64_t tk, uint8_t *out,
+                 uint64_t *table) {
+    int64_t steps = K / KSTEP, off = 0;
+    for (int64_t b = 0; b < N / BAND; ++b) {
+        int64_t e_off = -1; /* metadata block of the current pair */
+        for (int64_t c = 0; c < steps; ++c) {
+            int sp = kstep_sparse(map, K, tn, tk, b, c);
+            if (c % 2 == 0) e_off = -1;
+            uint64_t entry = 0;
+            if (!sp) {
+                uint8_t *blk = out + off;
+                for (int64_t r = 0; r < BAND; ++r)
+                    for (int64_t k = 0; k < KSTEP; ++k) {
+                        int64_t i = b * BAND + r, j = c * KSTEP + k;
+                        int64_t t = (i / tn) * (K / tk) + j / tk;
+                        uint16_t w = W[i * K + j];
+                        if (tile_is_sparse(map, t) && !kept(meta, K, i, j)) w = 0;
+                        int64_t byte = (r / 8) * 1024 + (r % 8) * 128 +
+                                       (((k / 8) ^ (r % 8)) * 16) + (k % 8) * 2;
+                        memcpy(blk + byte, &w, 2);
+                    }
+                entry = (uint64_t)off;
+                off += 16384;
+            } else {
+                if (e_off < 0) {
+                    e_off = off;
+                    memset(out + off, 0, 2048);
+                    off += 2048;
+                    entry |= 1ull << 63;
+                }
+                /* metadata bits for this k-step's half of the pair */
+                uint8_t *eb = out + e_off;
+                for (int64_t m = 0; m < BAND; ++m)
+                    for (int64_t k = 0; k < KSTEP; ++k) {
+                        int64_t kp = (c % 2) * KSTEP + k; /* column in pair */
+                        int64_t i = b * BAND + m, j = c * KSTEP + k;
+                        uint32_t word = meta[i * (K / 32) + j / 32];
+                        unsigned code = (word >> (4 * ((j % 32) / 4))) & 0xFu;
+                        unsigned bit = (code >> (j % 4)) & 1u;
+                        int64_t m0 = m % 8, m1 = (m / 8) % 2, m2 = m / 16;
+                        int64_t k0 = kp % 16, k1 = (kp / 16) % 2, k2 = kp / 32;
+                        int64_t line = m0 + 8 * k1 + 16 * m2;
+                        int64_t pos = 32 * k2 + 16 * m1 + k0;
+                        if (bit) eb[line * 16 + pos / 8] |= (uint8_t)(1u << (pos % 8));
+                    }
+                /* kept values, two per group, in column order */
+                uint8_t *blk = out + off;
+                for (int64_t r = 0; r < BAND; ++r) {
+                    int64_t i = b * BAND + r;
+                    int v = 0;
+                    for (int64_t k = 0; k < KSTEP; ++k) {
+                        int64_t j = c * KSTEP + k;
+                        if (!kept(meta, K, i, j)) continue;
+                        uint16_t w = W[i * K + j];
+                        int64_t byte = (r / 8) * 512 + (r % 8) * 64 +
+                                       (((v / 8) ^ ((r % 8) / 2)) * 16) + (v % 8) * 2;
+                        memcpy(blk + byte, &w, 2);
+                        ++v;
+                    }
+                }
+                entry |= (uint64_t)off | (1ull << 62);
+                off += 8192;
+            }
+            table[b * steps + c] = entry;
+        }
+    }
+}
+
+/*
+ * Inverse of oracle_pack: rebuild W_eff (bf16 bits, [N,K]) from the packed
+ * bytes and the table alone.
+ */
+void oracle_unpack(const uint8_t *packed, const uint64_t *table, int64_t N,
+                   int64_t K, uint16_t *weff) {
+    int64_t steps = K / KSTEP;
+    for (int64_t b = 0; b < N / BAND; ++b) {
+        int64_t e_off = -1;
+        for (int64_t c = 0; c < steps; ++c) {
+            uint64_t entry = table[b * steps + c];
+            int64_t off = (int64_t)(entry & ((1ull << 48) - 1));
+            if (c % 2 == 0) e_off = -1;
+            if (!(entry >> 62 & 1)) {
+                for (int64_t r = 0; r < BAND; ++r)
+                    for (int64_t k = 0; k < KSTEP; ++k) {
+                        int64_t byte = (r / 8) * 1024 + (r % 8) * 128 +
+                                       (((k / 8) ^ (r % 8)) * 16) + (k % 8) * 2;
+                        memcpy(&weff[(b * BAND + r) * K + c * KSTEP + k],
+                               packed + off + byte, 2);
+                    }
+                continue;
+            }
+            if (entry >> 63) e_off = off - 2048;
+            for (int64_t r = 0; r < BAND; ++r) {
+                int v = 0;
+                for (int64_t k = 0; k < KSTEP; ++k) {
+                    int64_t kp = (c % 2) * KSTEP + k;
+                    int64_t m0 = r % 8, m1 = (r / 8) % 2, m2 = r / 16;
+                    int64_t k0 = kp % 16, k1 = (kp / 16) % 2, k2 = kp / 32;
+                    int64_t line = m0 + 8 * k1 + 16 * m2;
+                    int64_t pos = 32 * k2 + 16 * m1 + k0;
+                    /* the group's code: its four bits starting at the group's
+                     * first column */
+                    int64_t gpos = pos - (k0 % 4);
+                    unsigned code = 0;
+                    for (int q = 0; q < 4; ++q) {
+                        int64_t p = gpos + q;
+                        code |= ((packed[e_off + line * 16 + p / 8] >> (p % 8)) & 1u) << q;
+                    }
+                    unsigned here = (unsigned)(k % 4);
+                    uint16_t w = 0;
+                    if (here == (code & 3u) || here == (code >> 2)) {
+                        int64_t byte = (r / 8) * 512 + (r % 8) * 64 +
+                                       (((v / 8) ^ ((r % 8) / 2)) * 16) + (v % 8) * 2;
+                        memcpy(&w, packed + off + byte, 2);
+                        ++v;
+                    }
+                    weff[(b * BAND + r) * K + c * KSTEP + k] = w;
+                }
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 8: the product                                                   */
+/* ------------------------------------------------------------------ */
+
+/*
+ * y[m,n] = sum_k X[m,k] * W_eff[n,k]: a naive triple loop, fp64 products of
+ * the exact bf16 values, accumulated from 0.0 in increasing k.  The product
+ * of two bf16 values is exact in fp64.
+ */
+void oracle_gemm(const uint16_t *X, const uint16_t *Weff, int64_t M, int64_t N,
+                 int64_t K, double *y) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc = acc + bf16_bits_to_f64(X[m * K + k]) *
+                                bf16_bits_to_f64(Weff[n * K + k]);
+            y[m * N + n] = acc;
+        }
+}
+
+/* The same sum for a list of (m, n) output positions only. */
+void oracle_gemm_at(const uint16_t *X, const uint16_t *Weff, int64_t K,
+                    const int64_t *ms, const int64_t *ns, int64_t count,
+                    double *y) {
+#pragma omp parallel for schedule(static)
+    for (int64_t q = 0; q < count; ++q) {
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+            acc = acc + bf16_bits_to_f64(X[ms[q] * K + k]) *
+                            bf16_bits_to_f64(Weff[ns[q] * K + k]);
+        y[q] = acc;
+    }
+}

@@ -1,0 +1,403 @@
+"""Pins of the CPU oracle to facts fixed outside the oracle itself.
+
+Each oracle step is checked against something other than its own formula:
+closed forms, exact rational brute force, invariants of 2:4 / tile sparsity,
+hand-worked golden fixtures (tests/golden/, each citing its page), and library
+routines (numpy fp64 matmul / sum) for the special cases that reduce to them.
+The checks are chosen so that a dropped term, a swapped kept/pruned set, a
+wrong tie rule, a transposed operand or a wrong tile index fails at least one.
+"""
+import os
+from fractions import Fraction
+from itertools import combinations
+
+import numpy as np
+import pytest
+import torch
+
+from tests.conftest import bf16_bits
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+ALLOWED_CODES = {4, 8, 12, 9, 13, 14}
+
+
+def to_bits(values, shape=None):
+    t = torch.tensor(np.asarray(values, dtype=np.float32))
+    if shape is not None:
+        t = t.reshape(shape)
+    return bf16_bits(t.to(torch.bfloat16))
+
+
+def codes_of(meta):
+    """Unpack uint32 meta words into per-group 4-bit codes [N, K/4]."""
+    meta = np.asarray(meta, dtype=np.uint32)
+    shifts = (np.arange(8, dtype=np.uint32) * 4)
+    c = (meta[..., None] >> shifts) & 0xF
+    return c.reshape(meta.shape[0], -1)
+
+
+def read_golden(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+# ----------------------------------------------------------------------------
+# column sum of squares
+# ----------------------------------------------------------------------------
+
+def test_colsq_constant_ones_ragged(oracle_mod):
+    # X == 1 -> s_j = T exactly, with a ragged last chunk (300 = 2*128 + 44)
+    x = to_bits(np.ones((300, 40)))
+    s = oracle_mod.colsq(x)
+    assert np.all(s == 300.0)
+
+
+def test_colsq_one_hot(oracle_mod):
+    x = np.zeros((257, 16), dtype=np.float32)
+    x[200, 5] = 3.0
+    x[0, 7] = -0.5
+    s = oracle_mod.colsq(to_bits(x))
+    expect = np.zeros(16)
+    expect[5] = 9.0
+    expect[7] = 0.25
+    assert np.array_equal(s, expect)
+
+
+def test_colsq_integer_exact(oracle_mod):
+    rng = np.random.default_rng(0)
+    xi = rng.integers(-8, 9, size=(1000, 64))
+    s = oracle_mod.colsq(to_bits(xi.astype(np.float32)))
+    assert np.array_equal(s, (xi.astype(np.int64) ** 2).sum(axis=0).astype(np.float64))
+
+
+def test_colsq_matches_numpy_sum(oracle_mod):
+    g = torch.Generator().manual_seed(3)
+    x = (torch.randn(777, 96, generator=g) * 5).to(torch.bfloat16)
+    s = oracle_mod.colsq(bf16_bits(x))
+    ref = (x.double() ** 2).sum(0).numpy()
+    np.testing.assert_allclose(s, ref, rtol=1e-13, atol=0)
+
+
+# ----------------------------------------------------------------------------
+# scores
+# ----------------------------------------------------------------------------
+
+def test_scores_hand_values(oracle_mod):
+    # -0.5, 1.5, -0.0, 2.0 as bf16 bit patterns
+    w = np.array([[0xBF00, 0x3FC0, 0x8000, 0x4000]], dtype=np.uint16)
+    s = np.array([4.0, 9.0, 0.25, 0.0])
+    sc = oracle_mod.wanda_scores(w, s)
+    assert np.array_equal(sc, [[1.0, 4.5, 0.0, 0.0]])
+    assert not np.signbit(sc[0, 2]), "|w| of -0 must be +0"
+
+
+def test_golden_activation_outranks_magnitude(oracle_mod):
+    rows = {r[0]: r[1:] for r in read_golden("wanda_activation_outranks_magnitude.txt")}
+    w = to_bits([float(v) for v in rows["w"]], (1, 4))
+    w = np.concatenate([w, np.zeros((1, 28), np.uint16)], axis=1)  # one 32-wide word
+    s = np.concatenate([np.array([float(v) for v in rows["s"]]), np.ones(28)])
+    sc = oracle_mod.wanda_scores(w, s)
+    assert np.array_equal(sc[0, :4], [float(v) for v in rows["score"]])
+    code = codes_of(oracle_mod.select_2of4(sc))[0, 0]
+    assert code == int(rows["code"][0])
+    # dropping the activation term (all norms 1) gives the magnitude-only code
+    code_mag = codes_of(oracle_mod.select_2of4(oracle_mod.wanda_scores(w, np.ones(32))))[0, 0]
+    assert code_mag == int(rows["magnitude_only_code"][0])
+
+
+# ----------------------------------------------------------------------------
+# top-2-of-4 selection
+# ----------------------------------------------------------------------------
+
+def brute_force_code(sc4):
+    """Best of the 6 patterns by exact kept sum; ties -> lexicographically smallest pair."""
+    best = None
+    for pair in combinations(range(4), 2):  # already in lexicographic order
+        total = Fraction(sc4[pair[0]]) + Fraction(sc4[pair[1]])
+        if best is None or total > best[0]:
+            best = (total, pair)
+    a, b = best[1]
+    return a | (b << 2)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_select_equals_bruteforce_with_ties(oracle_mod, seed):
+    rng = np.random.default_rng(seed)
+    # few distinct values -> many exact ties
+    sc = rng.choice([0.0, 0.5, 1.0, 1.5, 2.0], size=(64, 64)).astype(np.float64)
+    codes = codes_of(oracle_mod.select_2of4(sc))
+    for i in range(sc.shape[0]):
+        for g in range(sc.shape[1] // 4):
+            assert codes[i, g] == brute_force_code(sc[i, 4 * g:4 * g + 4]), (i, g)
+
+
+def test_select_equals_bruteforce_random(oracle_mod):
+    rng = np.random.default_rng(11)
+    sc = np.abs(rng.standard_normal((32, 256)))
+    codes = codes_of(oracle_mod.select_2of4(sc))
+    for i in range(sc.shape[0]):
+        for g in range(sc.shape[1] // 4):
+            assert codes[i, g] == brute_force_code(sc[i, 4 * g:4 * g + 4])
+
+
+@pytest.mark.parametrize("group,code", [((1, 1, 1, 1), 0x4), ((1, 3, 2, 0), 0x9),
+                                        ((0, 0, 0, 1), 0xC), ((5, 1, 1, 5), 0xC),
+                                        ((0, 2, 2, 2), 0x9), ((1, 0, 0, 1), 0xC),
+                                        ((0, 0, 1, 1), 0xE), ((2, 0, 2, 0), 0x8)])
+def test_select_special_cases(oracle_mod, group, code):
+    sc = np.zeros((1, 32))
+    sc[0, :4] = group
+    assert codes_of(oracle_mod.select_2of4(sc))[0, 0] == code
+
+
+def test_golden_patterns_all_reachable(oracle_mod):
+    rows = read_golden("two_four_patterns.txt")
+    assert len(rows) == 6
+    seen = {}
+    for idx0, idx1, code in rows:
+        sc = np.zeros((1, 32))
+        sc[0, int(idx0)] = 2.0
+        sc[0, int(idx1)] = 1.0
+        got = codes_of(oracle_mod.select_2of4(sc))[0, 0]
+        assert got == int(code)
+        seen[int(code)] = True
+    assert set(seen) == ALLOWED_CODES
+
+
+def test_select_dominance_and_alphabet(oracle_mod):
+    rng = np.random.default_rng(5)
+    sc = np.abs(rng.standard_normal((16, 128))).round(1)
+    codes = codes_of(oracle_mod.select_2of4(sc))
+    assert set(np.unique(codes)) <= ALLOWED_CODES
+    for i in range(16):
+        for g in range(32):
+            c = codes[i, g]
+            keep = {c & 3, c >> 2}
+            grp = sc[i, 4 * g:4 * g + 4]
+            for k in keep:
+                for d in set(range(4)) - keep:
+                    # kept beats dropped in the order (score desc, index asc)
+                    assert grp[k] > grp[d] or (grp[k] == grp[d] and k < d)
+
+
+# ----------------------------------------------------------------------------
+# tile loss
+# ----------------------------------------------------------------------------
+
+def pruned_mask(codes, K):
+    N = codes.shape[0]
+    keep = np.zeros((N, K), dtype=bool)
+    for g in range(K // 4):
+        c = codes[:, g]
+        for pos in range(4):
+            keep[:, 4 * g + pos] = ((c & 3) == pos) | ((c >> 2) == pos)
+    return ~keep
+
+
+def test_tile_loss_exact_dyadic(oracle_mod):
+    # dyadic scores with small magnitude: every partial sum is exact in fp64,
+    # so the loss must equal the exact rational sum of the pruned scores.
+    rng = np.random.default_rng(7)
+    N, K, tn, tk = 128, 192, 64, 64
+    sc = rng.integers(0, 4096, size=(N, K)) / 8.0
+    meta = oracle_mod.select_2of4(sc)
+    loss = oracle_mod.tile_loss(sc, meta, tn, tk)
+    pm = pruned_mask(codes_of(meta), K)
+    tiles_k = K // tk
+    for t in range(len(loss)):
+        i0, j0 = (t // tiles_k) * tn, (t % tiles_k) * tk
+        blk = sc[i0:i0 + tn, j0:j0 + tk][pm[i0:i0 + tn, j0:j0 + tk]]
+        assert Fraction(loss[t]) == sum(Fraction(v) for v in blk)
+        # exactly half of every tile is pruned
+        assert blk.size == tn * tk // 2
+
+
+def test_tile_loss_plus_kept_is_total(oracle_mod):
+    rng = np.random.default_rng(9)
+    N, K, tn, tk = 256, 256, 128, 128
+    sc = np.abs(rng.standard_normal((N, K)))
+    meta = oracle_mod.select_2of4(sc)
+    loss = oracle_mod.tile_loss(sc, meta, tn, tk)
+    pm = pruned_mask(codes_of(meta), K)
+    for t in range(4):
+        i0, j0 = (t // 2) * tn, (t % 2) * tk
+        blk = sc[i0:i0 + tn, j0:j0 + tk]
+        kept_sum = blk[~pm[i0:i0 + tn, j0:j0 + tk]].sum()
+        np.testing.assert_allclose(loss[t] + kept_sum, blk.sum(), rtol=1e-12)
+        assert loss[t] <= kept_sum  # the kept half is the larger half
+
+
+# ----------------------------------------------------------------------------
+# map selection
+# ----------------------------------------------------------------------------
+
+def test_n_sparse_floor(oracle_mod):
+    assert oracle_mod.n_sparse(0.6, 1024) == 614
+    assert oracle_mod.n_sparse(0.6, 2752) == 1651
+    assert oracle_mod.n_sparse(0.5, 16) == 8
+    assert oracle_mod.n_sparse(1.0, 4320) == 4320
+    assert oracle_mod.n_sparse(0.0, 4320) == 0
+    assert oracle_mod.n_sparse(0.999, 10) == 9
+
+
+def popcount(words):
+    return int(sum(bin(int(w)).count("1") for w in np.asarray(words, dtype=np.uint32)))
+
+
+def bits_of(words, n):
+    words = np.asarray(words, dtype=np.uint32)
+    return np.array([(int(words[t // 32]) >> (t % 32)) & 1 for t in range(n)], dtype=bool)
+
+
+def test_map_invariants(oracle_mod):
+    rng = np.random.default_rng(1)
+    loss = rng.standard_normal(1000).round(2)  # with ties
+    for ns in [0, 1, 313, 999, 1000]:
+        m = oracle_mod.select_map(loss, ns)
+        b = bits_of(m, 1000)
+        assert b.sum() == ns == popcount(m)
+        if 0 < ns < 1000:
+            assert loss[b].max() <= loss[~b].min()
+            # on the boundary value, lower indices were taken first
+            v = loss[b].max()
+            chosen = np.where(b & (loss == v))[0]
+            left = np.where(~b & (loss == v))[0]
+            if len(left):
+                assert chosen.max() < left.min()
+
+
+def test_map_all_ties_take_lowest_indices(oracle_mod):
+    m = oracle_mod.select_map(np.full(70, 3.0), 33)
+    b = bits_of(m, 70)
+    assert b[:33].all() and not b[33:].any()
+
+
+# ----------------------------------------------------------------------------
+# effective weight and product
+# ----------------------------------------------------------------------------
+
+def rand_problem(seed, N, K, M=8):
+    g = torch.Generator().manual_seed(seed)
+    w = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    xc = torch.randn(32, K, generator=g).to(torch.bfloat16)
+    return bf16_bits(w), bf16_bits(x), bf16_bits(xc)
+
+
+def full_map(n_tiles, value):
+    words = np.zeros((n_tiles + 31) // 32, dtype=np.uint32)
+    if value:
+        for t in range(n_tiles):
+            words[t // 32] |= np.uint32(1 << (t % 32))
+    return words
+
+
+def test_all_dense_is_plain_gemm(oracle_mod):
+    w, x, xc = rand_problem(0, 128, 256)
+    r = oracle_mod.score_mask(w, xc, 64, 64, tile_map=full_map(8, False))
+    weff = oracle_mod.weff(w, r["meta"], r["map"], 64, 64)
+    assert np.array_equal(weff, w)
+    y = oracle_mod.gemm(x, weff)
+    xf, wf = oracle_mod.bf16_bits_to_f64(x), oracle_mod.bf16_bits_to_f64(w)
+    bound = 1e-12 * (np.abs(xf) @ np.abs(wf).T)
+    assert np.all(np.abs(y - xf @ wf.T) <= bound)
+    # a transposed operand would not match
+    assert not np.allclose(y, xf @ wf[:, ::-1].T)
+
+
+def test_all_sparse_is_masked_gemm(oracle_mod):
+    w, x, xc = rand_problem(1, 128, 256)
+    r = oracle_mod.score_mask(w, xc, 64, 64, tile_map=full_map(8, True))
+    weff = oracle_mod.weff(w, r["meta"], r["map"], 64, 64)
+    # mask from brute-force selection on the same scores
+    sc = r["score"]
+    wf = oracle_mod.bf16_bits_to_f64(w)
+    masked = wf.copy()
+    for i in range(128):
+        for g in range(64):
+            c = brute_force_code(sc[i, 4 * g:4 * g + 4])
+            for pos in range(4):
+                if pos not in (c & 3, c >> 2):
+                    masked[i, 4 * g + pos] = 0.0
+    assert np.array_equal(oracle_mod.bf16_bits_to_f64(weff), masked)
+    y = oracle_mod.gemm(x, weff)
+    xf = oracle_mod.bf16_bits_to_f64(x)
+    bound = 1e-12 * (np.abs(xf) @ np.abs(masked).T)
+    assert np.all(np.abs(y - xf @ masked.T) <= bound)
+
+
+def test_gemm_integer_exact_and_sampled(oracle_mod):
+    rng = np.random.default_rng(4)
+    xi = rng.integers(-4, 5, size=(5, 96))
+    wi = rng.integers(-4, 5, size=(7, 96))
+    y = oracle_mod.gemm(to_bits(xi), to_bits(wi))
+    assert np.array_equal(y, (xi @ wi.T).astype(np.float64))
+    ms, ns = np.array([0, 4, 2]), np.array([6, 0, 3])
+    assert np.array_equal(oracle_mod.gemm_at(to_bits(xi), to_bits(wi), ms, ns), y[ms, ns])
+
+
+@pytest.mark.parametrize("f_line", read_golden("tile_sparsity_endpoints.txt"))
+def test_golden_achieved_sparsity(oracle_mod, f_line):
+    f, s_expect = float(f_line[0]), float(f_line[1])
+    N, K, tn, tk = 256, 512, 64, 64
+    n_tiles = (N // tn) * (K // tk)
+    w = np.full((N, K), 0x3F80, dtype=np.uint16)  # all ones: nothing is zero by chance
+    sc = np.abs(np.random.default_rng(2).standard_normal((N, K)))
+    meta = oracle_mod.select_2of4(sc)
+    loss = oracle_mod.tile_loss(sc, meta, tn, tk)
+    m = oracle_mod.select_map(loss, oracle_mod.n_sparse(f, n_tiles))
+    weff = oracle_mod.weff(w, meta, m, tn, tk)
+    achieved = np.count_nonzero(weff == 0) / weff.size
+    assert achieved == s_expect
+    # every 4-group of a 2:4 tile has exactly two nonzeros
+    b = bits_of(m, n_tiles)
+    for t in np.where(b)[0][:4]:
+        i0, j0 = (t // (K // tk)) * tn, (t % (K // tk)) * tk
+        blk = weff[i0:i0 + tn, j0:j0 + tk].reshape(tn, tk // 4, 4)
+        assert np.all(np.count_nonzero(blk, axis=2) == 2)
+
+
+# ----------------------------------------------------------------------------
+# packed layout
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("tn,tk", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("frac", [0.0, 0.3, 0.5, 1.0])
+def test_pack_round_trip(oracle_mod, tn, tk, frac):
+    N, K = 256, 384
+    w, x, xc = rand_problem(int(frac * 10) + tn, N, K)
+    n_tiles = (N // tn) * (K // tk)
+    g = np.random.default_rng(tn + tk)
+    chosen = g.permutation(n_tiles)[:int(frac * n_tiles)]
+    m = np.zeros((n_tiles + 31) // 32, dtype=np.uint32)
+    for t in chosen:
+        m[t // 32] |= np.uint32(1 << (int(t) % 32))
+    r = oracle_mod.score_mask(w, xc, tn, tk, tile_map=m)
+    weff = oracle_mod.weff(w, r["meta"], m, tn, tk)
+    packed, table = oracle_mod.pack(w, r["meta"], m, tn, tk)
+    assert np.array_equal(oracle_mod.unpack(packed, table, N, K), weff)
+
+
+@pytest.mark.parametrize("frac", [0.0, 0.25, 0.5, 0.75, 1.0])
+def test_pack_bytes_closed_form(oracle_mod, frac):
+    # 128x128 tiles: dense 32768 B, 2:4 16384 + 2048 B -> ratio 1 - 0.4375 f
+    N, K = 512, 1024
+    n_tiles = (N // 128) * (K // 128)
+    ns = int(frac * n_tiles)
+    m = np.zeros((n_tiles + 31) // 32, dtype=np.uint32)
+    for t in range(ns):
+        m[t // 32] |= np.uint32(1 << (t % 32))
+    nbytes = oracle_mod.pack_bytes(m, N, K, 128, 128)
+    assert nbytes == int(2 * N * K * (1 - 0.4375 * frac))
+    w = np.zeros((N, K), dtype=np.uint16)
+    meta = np.full((N, K // 32), 0x44444444, dtype=np.uint32)
+    packed, table = oracle_mod.pack(w, meta, m, 128, 128)
+    assert packed.size == nbytes
+    sparse_steps = int(((table >> np.uint64(62)) & np.uint64(1)).sum())
+    e_blocks = int((table >> np.uint64(63)).sum())
+    assert sparse_steps == 2 * ns and e_blocks == ns
