@@ -1,0 +1,586 @@
+"""Benchmark of the tile-hybrid (dense / 2:4) Wanda-masked linear layer on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input,
+for every weight matrix of the workload:
+  column norms of the calibration set -> Wanda scores / 2:4 codes / tile loss
+  -> tile map (least-loss tiles become 2:4) -> pack -> hybrid GEMM for every
+  token count of the workload.
+Default workload: Llama-7B-shaped decode (W 4096x4096 and 11008x4096, 128x128
+tiles, half the tiles 2:4 chosen by least Wanda tile loss, calibration
+2048x4096 with 1% outlier channels x20, M in {1, 4, 16}).
+
+Metric: dense-equivalent GEMM TFLOP/s = sum over the step's GEMMs of 2*M*N*K,
+divided by the step's device time (mask build and pack included).  Also
+reported: tokens/s, per-call times, the roofline of the dominant call, an
+isolated decode-GEMM and prefill-GEMM measurement (speedup over the same
+kernel with an all-dense map), end-to-end time with host buffers, and the CPU
+oracle timed on the host cores.
+
+Launch: ``python bench.py [--gpus N --steps K --warmup W]``; for N > 1 under
+``torch.distributed.run`` one rank per GPU, each rank running the step on its
+own independent matrices (weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_gemm_wanda_b200 import inputs  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- utilities
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        top = max(sm)
+        loaded = [s for s in sm if s >= 0.5 * top] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+class L2Flusher:
+    def __init__(self, nbytes: int = 512 << 20):
+        self.buf = torch.empty(nbytes // 4, dtype=torch.int32, device="cuda")
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+class CallTimer:
+    """CUDA events around each ABI call on the launching stream."""
+
+    def __init__(self):
+        self.open = []
+        self.enabled = False
+
+    def wrap(self, name, fn, *a, **kw):
+        if not self.enabled:
+            return fn(*a, **kw)
+        s = torch.cuda.current_stream()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        out = fn(*a, **kw)
+        e1.record(s)
+        self.open.append((name, e0, e1))
+        return out
+
+    def summary(self):
+        torch.cuda.synchronize()
+        agg = {}
+        for name, e0, e1 in self.open:
+            agg.setdefault(name, []).append(e0.elapsed_time(e1))
+        return {k: {"launches": len(v), "mean_ms": sum(v) / len(v), "total_ms": sum(v)}
+                for k, v in agg.items()}
+
+
+# ----------------------------------------------------------------- workload
+def make_tensors(wl, rank: int, device="cpu"):
+    """Synthetic weights, calibration and inputs of a workload (per-rank seed)."""
+    seed = wl.seed + 1009 * rank
+    mats = []
+    outl = {}
+    calib = {}
+    for mi, m in enumerate(wl.matrices):
+        if m.K not in outl:
+            outl[m.K] = inputs.outlier_channels(m.K, seed, wl.outlier_count)
+            if wl.calib_tokens:
+                calib[m.K] = inputs.activations(wl.calib_tokens, m.K, seed, outl[m.K], role=0)
+        w = inputs.weight(m.N, m.K, seed + 17 * (mi + 1))
+        xs = {M: inputs.activations(M, m.K, seed, outl[m.K], role=1 + mi * 100 + M)
+              for M in wl.tokens}
+        mats.append({"name": m.name, "N": m.N, "K": m.K, "W": w.to(device),
+                     "X": {M: x.to(device) for M, x in xs.items()}})
+    return mats, {K: x.to(device) for K, x in calib.items()}
+
+
+def gemm_flops(mats, tokens):
+    return sum(2.0 * M * m["N"] * m["K"] for m in mats for M in tokens)
+
+
+def run_step(P, wl, mats, calib, timer: CallTimer, keep=None):
+    """The hot path once for every matrix; returns the GEMM outputs."""
+    outs = []
+    colsq_cache = {}
+    for m in mats:
+        K = m["K"]
+        cin = colsq_cache.get(K)
+        r = timer.wrap("score_mask", P.patch_score_mask, m["W"], calib[K] if cin is None else None,
+                       tile_n=wl.tile_n, tile_k=wl.tile_k, fraction=wl.fractions[0],
+                       colsq_in=cin, want_colsq=cin is None)
+        if cin is None:
+            colsq_cache[K] = r["colsq"]
+        pk = timer.wrap("pack", P.patch_pack, m["W"], r["meta"], r["map"], tile_n=wl.tile_n,
+                        tile_k=wl.tile_k)
+        for M in wl.tokens:
+            outs.append(timer.wrap(f"gemm_m{M}" if M <= 16 else "gemm_prefill",
+                                   P.patch_hybrid_gemm, pk, m["X"][M]))
+        if keep is not None:
+            keep.append((m, r, pk))
+        else:
+            pk.close()
+    return outs
+
+
+def algorithmic_bytes(name, wl, mats, packed_bytes):
+    """Bytes each call must move at minimum (roofline section)."""
+    total = 0.0
+    count = 0
+    seen_k = set()
+    for m, pb in zip(mats, packed_bytes):
+        N, K = m["N"], m["K"]
+        nt = (N // wl.tile_n) * (K // wl.tile_k)
+        if name == "score_mask":
+            b = 2 * N * K + N * K / 8 + 8 * nt + (nt + 31) // 32 * 4
+            if K not in seen_k and wl.calib_tokens:
+                b += 2 * wl.calib_tokens * K + 8 * K
+                seen_k.add(K)
+            total += b
+            count += 1
+        elif name == "pack":
+            total += 2 * N * K + N * K / 8 + pb + 8 * (N // 128) * (K // 64)
+            count += 1
+        elif name.startswith("gemm_m"):
+            M = int(name[6:])
+            total += pb + 8 * (N // 128) * (K // 64) + 2 * M * K + 2 * M * N
+            count += 1
+    return total / max(count, 1)
+
+
+def traffic_for(kernel_key: str):
+    """dram read+write bytes per launch from the committed ncu summary, if the
+    kernel source is unchanged since the capture; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        d = json.load(fh)
+    ent = d.get(kernel_key)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, ent["source"])
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if h != ent.get("source_sha256_16"):
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------- isolated GEMMs
+def isolated_gemm(P, wl, W, M, frac_map, X, flush, reps=20, seed=0):
+    """Time one GEMM configuration with L2 flushed before every call."""
+    N, K = W.shape
+    nt = (N // wl.tile_n) * (K // wl.tile_k)
+    tmap = inputs.random_map(nt, int(round(frac_map * nt)), seed).cuda()
+    r = P.patch_score_mask(W, X, tile_n=wl.tile_n, tile_k=wl.tile_k, map_in=tmap)
+    pk = P.patch_pack(W, r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        P.patch_hybrid_gemm(pk, X, out=Y)
+    ts = []
+    s = torch.cuda.current_stream()
+    for _ in range(reps):
+        flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        P.patch_hybrid_gemm(pk, X, out=Y)
+        e1.record(s)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    nbytes = pk.packed_bytes
+    pk.close()
+    return statistics.median(ts), nbytes
+
+
+# -------------------------------------------------------------- CPU oracle
+def cpu_oracle_sample(wl, rows=512, reps=1):
+    """The oracle as it stands on a bounded sample: the first `rows` rows of every
+    matrix through every step (full calibration set).  Returns (seconds, flops)."""
+    import numpy as np
+    import oracle
+    mats, calib = make_tensors(wl, 0)
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    t0 = time.perf_counter()
+    flops = 0.0
+    for _ in range(reps):
+        colsq = {}
+        for m in mats:
+            K = m["K"]
+            if K not in colsq:
+                colsq[K] = oracle.colsq(bits(calib[K]))
+            w = bits(m["W"][:rows])
+            sc = oracle.wanda_scores(w, colsq[K])
+            meta = oracle.select_2of4(sc)
+            loss = oracle.tile_loss(sc, meta, wl.tile_n, wl.tile_k)
+            tmap = oracle.select_map(loss, oracle.n_sparse(wl.fractions[0], loss.shape[0]))
+            oracle.pack(w, meta, tmap, wl.tile_n, wl.tile_k)
+            weff = oracle.weff(w, meta, tmap, wl.tile_n, wl.tile_k)
+            for M in wl.tokens:
+                oracle.gemm(bits(m["X"][M]), weff)
+                flops += 2.0 * M * rows * K
+    return time.perf_counter() - t0, flops
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# --------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama7b-decode")
+    ap.add_argument("--no-extras", action="store_true", help="skip isolated GEMM / oracle legs")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = inputs.workloads()[args.workload]
+
+    if args.impl == "reference":
+        return main_reference(args, wl, world, rank)
+
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    from sparse_gemm_wanda_b200 import patch as P
+    P.load_library()
+
+    mats, calib = make_tensors(wl, rank, device="cuda")
+    flops = gemm_flops(mats, wl.tokens)
+    tokens = sum(wl.tokens) * len(mats)
+    flush = L2Flusher()
+    timer = CallTimer()
+
+    for _ in range(args.warmup):
+        run_step(P, wl, mats, calib, timer)
+    torch.cuda.synchronize()
+
+    # ------------------------------------------------------------ timed steps
+    clocks = ClockSampler(torch.cuda.current_device())
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    timer.enabled = True
+    s = torch.cuda.current_stream()
+    step_ms = []
+    events = []
+    for _ in range(args.steps):
+        flush()  # between timed steps, outside the events
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        run_step(P, wl, mats, calib, timer)
+        e1.record(s)
+        events.append((e0, e1))
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    timer.enabled = False
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in events]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    calls = timer.summary()
+
+    # packed sizes, for algorithmic bytes
+    keep = []
+    run_step(P, wl, mats, calib, CallTimer(), keep=keep)
+    packed_bytes = [pk.packed_bytes for _, _, pk in keep]
+    for _, _, pk in keep:
+        pk.close()
+    torch.cuda.synchronize()
+
+    peaks, peak_kind = load_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    dominant = max(calls, key=lambda k: calls[k]["total_ms"])
+    roof = None
+    if dominant.startswith("gemm_prefill"):
+        fl = sum(2.0 * M * m["N"] * m["K"] for m in mats for M in wl.tokens if M > 16) / \
+            max(1, calls[dominant]["launches"] // args.steps)
+        ach = fl / (calls[dominant]["mean_ms"] * 1e-3) / 1e12
+        pk_ = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        roof = {"bound": "tensor", "achieved": ach, "peak": pk_, "unit": "TFLOP/s",
+                "frac": ach / pk_, "traffic": None, "kernel": dominant,
+                "peak_source": peak_kind}
+    else:
+        bpl = algorithmic_bytes(dominant, wl, mats, packed_bytes)
+        ach = bpl / (calls[dominant]["mean_ms"] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+                "frac": ach / hbm_peak, "traffic": traffic_for(dominant), "kernel": dominant,
+                "algorithmic_bytes_per_launch": bpl, "peak_source": peak_kind}
+    per_call = {}
+    for k, v in calls.items():
+        ent = {"launches_per_step": v["launches"] / args.steps, "mean_us": v["mean_ms"] * 1e3,
+               "share": v["total_ms"] / max(sum(c["total_ms"] for c in calls.values()), 1e-9)}
+        if not k.startswith("gemm_prefill"):
+            b = algorithmic_bytes(k, wl, mats, packed_bytes)
+            ent["algorithmic_bytes"] = b
+            ent["achieved_gbs"] = b / (v["mean_ms"] * 1e-3) / 1e9
+        per_call[k] = ent
+
+    # ------------------------------------------------------- end to end
+    e2e = None
+    if rank == 0 or world > 1:
+        host = {"W": [m["W"].cpu().pin_memory() for m in mats],
+                "X": [{M: x.cpu().pin_memory() for M, x in m["X"].items()} for m in mats],
+                "C": {K: c.cpu().pin_memory() for K, c in calib.items()}}
+        h2d = sum(t.numel() * 2 for t in host["W"]) + sum(c.numel() * 2 for c in host["C"].values()) \
+            + sum(x.numel() * 2 for d in host["X"] for x in d.values())
+        d2h = sum(m["N"] * M * 2 for m in mats for M in wl.tokens)
+        e2e_events = []
+        for it in range(args.warmup + args.steps):
+            flush()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            dm = []
+            for mi, m in enumerate(mats):
+                dm.append({"name": m["name"], "N": m["N"], "K": m["K"],
+                           "W": host["W"][mi].to("cuda", non_blocking=True),
+                           "X": {M: x.to("cuda", non_blocking=True) for M, x in host["X"][mi].items()}})
+            dc = {K: c.to("cuda", non_blocking=True) for K, c in host["C"].items()}
+            outs = run_step(P, wl, dm, dc, CallTimer())
+            hy = [o.to("cpu", non_blocking=True) for o in outs]
+            e1.record(s)
+            e1.synchronize()
+            del hy
+            if it >= args.warmup:
+                e2e_events.append(e0.elapsed_time(e1))
+        e2e_ms = sum(e2e_events) / len(e2e_events)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # --------------------------------------------- isolated GEMM measurements
+    extras = {}
+    if not args.no_extras and rank == 0:
+        W0 = mats[-1]["W"]  # the MLP-shaped matrix
+        dec = {}
+        for M in wl.tokens:
+            if M > 16:
+                continue
+            X = mats[-1]["X"][M]
+            t_ms, nb = isolated_gemm(P, wl, W0, M, wl.fractions[0], X, flush, seed=M)
+            b = nb + 8 * (W0.shape[0] // 128) * (W0.shape[1] // 64) + 2 * M * W0.shape[1] + 2 * M * W0.shape[0]
+            dec[f"m{M}"] = {"us": t_ms * 1e3, "compressed_bytes": b,
+                            "achieved_gbs": b / (t_ms * 1e-3) / 1e9,
+                            "frac_of_hbm": b / (t_ms * 1e-3) / 1e9 / hbm_peak}
+        extras["decode_gemm_isolated"] = {"matrix": f"{W0.shape[0]}x{W0.shape[1]}",
+                                          "fraction_2to4_tiles": wl.fractions[0],
+                                          "by_m": dec, "l2": "flushed before every call"}
+        # prefill: Llama-7B MLP up projection at M = 2048, f in {0, 0.5, 1}
+        g = torch.Generator().manual_seed(4242)
+        Wp = (torch.randn(11008, 4096, generator=g) * 0.02).to(torch.bfloat16).cuda()
+        Xp = torch.randn(2048, 4096, generator=g).to(torch.bfloat16).cuda()
+        pre = {}
+        base = None
+        for f in (0.0, 0.5, 1.0):
+            t_ms, _ = isolated_gemm(P, wl, Wp, 2048, f, Xp, flush, seed=7)
+            fl = 2.0 * 2048 * 11008 * 4096
+            eff = fl / (t_ms * 1e-3) / 1e12
+            useful = fl * (1 - f / 2) / (t_ms * 1e-3) / 1e12
+            if f == 0.0:
+                base = t_ms
+            pre[f"f{f}"] = {"us": t_ms * 1e3, "effective_tflops": eff,
+                            "useful_tflops": useful, "speedup_vs_all_dense": base / t_ms,
+                            "frac_of_dense_peak_useful": useful / float(peaks["bf16_tflops"])}
+        extras["prefill_gemm_isolated"] = {"shape": "M=2048 N=11008 K=4096", "by_fraction": pre,
+                                           "peak_tflops": float(peaks["bf16_tflops"]),
+                                           "peak_source": peak_kind}
+        del Wp, Xp
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        secs, fl = cpu_oracle_sample(wl)
+        cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
+               "kind": "oracle",
+               "sample": "first 512 rows of each matrix through every step, full calibration "
+                         f"set, M in {wl.tokens}; {secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": "hybrid-sparse GEMM effective TFLOP/s (dense-equivalent 2*M*N*K over the "
+                      "whole step: mask build + pack + GEMMs)",
+            "value": flops * world / (ms_per_step * 1e-3) / 1e12,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded Llama-shaped weights N(0,0.02); activations N(0,1) with "
+                    "1% outlier channels x20)",
+            "config": {"workload": wl.name, "matrices": [f"{m['N']}x{m['K']}" for m in mats],
+                       "tiles": f"{wl.tile_n}x{wl.tile_k}", "fraction_2to4_tiles": wl.fractions[0],
+                       "map": "least Wanda tile loss" if wl.map_rule == "loss" else "seeded random",
+                       "calibration_tokens": wl.calib_tokens, "tokens": wl.tokens,
+                       "l2": "flushed (512 MB write) between timed steps",
+                       "parallelism": f"independent matrices per rank x{world}"},
+            "tokens_per_s": tokens * world / (ms_per_step * 1e-3),
+            "e2e": e2e,
+            "gpu_launches": gpu_launches(wl, mats) * args.steps,
+            "roofline": roof,
+            "calls": per_call,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def gpu_launches(wl, mats):
+    """Kernels this library launches per step (see the launch list in profiles/)."""
+    n = 0
+    seen = set()
+    for m in mats:
+        first = m["K"] not in seen
+        seen.add(m["K"])
+        n += (2 if first else 1) + 1 + 2  # norms, score, rank + map
+        n += 1  # pack
+        for M in wl.tokens:
+            n += 2 if M <= 16 else 1  # GEMM (+ split-K reduce)
+    return n
+
+
+def main_reference(args, wl, world, rank):
+    """The oracle as it stands on the host cores, on a bounded sample per step."""
+    if rank != 0:
+        return
+    rows = 256
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, rows=rows)
+    tot_s, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        sec, fl = cpu_oracle_sample(wl, rows=rows)
+        tot_s += sec
+        tot_f += fl
+    v = tot_f / tot_s / 1e12
+    line = {
+        "impl": "reference",
+        "metric": "hybrid-sparse GEMM effective TFLOP/s (dense-equivalent 2*M*N*K over the whole "
+                  "step: mask build + pack + GEMMs)",
+        "value": v, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": wl.name,
+                                        "sample": f"first {rows} rows of each matrix"},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"first {rows} rows of each matrix, full calibration set, "
+                                   f"M in {wl.tokens}"},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,214 @@
+/*
+ * patch.h -- C ABI of the B200 (sm_100a) tile-hybrid sparse linear layer.
+ *
+ * A weight matrix W[N,K] is cut into tile_n x tile_k tiles.  A per-tile map
+ * marks each tile dense or 2:4-sparse, so the overall sparsity is anywhere
+ * between 0% and 50% ("PATCH: Learnable Tile-level Hybrid Sparsity for LLMs",
+ * section 2, core mechanism).  Inside a 2:4 tile every group of 4 consecutive
+ * input channels keeps the 2 weights with the highest Wanda score
+ * |W_ij| * ||X_:,j||_2 over calibration tokens ("SparseGPT vs Wanda: one-shot
+ * LLM pruning without retraining", section on Wanda), ties going to the lower
+ * index.  The product Y = X * W_eff^T then runs as one kernel over the mixed
+ * tiles (PATCH page, section 2, inference and deployment: dense tiles on the
+ * dense tensor-core path, 2:4 tiles on the sparse one).
+ *
+ * Conventions for every call:
+ *   - All array pointers are DEVICE pointers on the current CUDA device,
+ *     unless a comment says otherwise.  The caller owns them.
+ *   - bf16 arrays are row-major with the last index contiguous.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued on it; no call synchronises the host except
+ *     where its comment says so.
+ *   - Errors are returned, never thrown.  An asynchronous kernel fault
+ *     surfaces as PATCH_ERR_CUDA on a later call.  Calls on different
+ *     handles may run concurrently; calls on one handle must not.
+ *
+ * Layouts:
+ *   meta  uint32 [N, K/32]: group g of row i (columns 4g..4g+3) is the 4-bit
+ *         code idx0 | (idx1 << 2) of its two kept positions (idx0 < idx1), at
+ *         bits 4*(g%8) of word [i, g/8].  Codes are written for every group,
+ *         dense tiles included (dense tiles simply ignore them).
+ *   map   uint32 [ceil(n_tiles/32)]: tile t = (i/tile_n)*(K/tile_k) + j/tile_k
+ *         is 2:4 iff bit t%32 of word t/32 is 1.  Unused high bits are 0.
+ *   colsq fp64 [K]: s_j = sum_t x_tj^2 over calibration tokens, added in a
+ *         fixed order: chunks of 128 consecutive tokens, each summed token
+ *         by token from 0.0, then the chunk sums added chunk by chunk from
+ *         0.0.  The result is therefore bit-reproducible.
+ *   tile_loss fp64 [n_tiles]: Wanda score removed by 2:4 pruning of the tile;
+ *         each row of the tile sums its pruned scores left to right, then the
+ *         row sums are added top to bottom.
+ */
+#ifndef PATCH_B200_H
+#define PATCH_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PATCH_OK = 0,
+    PATCH_ERR_INVALID_ARG = 1, /* null pointer, misalignment, bad shape     */
+    PATCH_ERR_UNSUPPORTED = 2, /* tile size not in {64,128}, not sm_100     */
+    PATCH_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed          */
+    PATCH_ERR_OOM = 4,         /* device allocation failed                   */
+    PATCH_ERR_TIMEOUT = 5      /* a bounded device wait ran out (see below)  */
+} patch_status;
+
+typedef struct {
+    int64_t N;      /* output features (rows of W)                          */
+    int64_t K;      /* input features (columns of W)                        */
+    int32_t tile_n; /* tile rows, 64 or 128                                 */
+    int32_t tile_k; /* tile columns, 64 or 128                              */
+} patch_shape;
+
+/* Opaque packed weight, owned by the library (patch_pack / patch_free). */
+typedef struct patch_packed patch_packed;
+
+/*
+ * Wanda 2:4 mask builder and tile map.
+ *
+ * Follows the Wanda criterion (SparseGPT-vs-Wanda page, section on Wanda:
+ * weight magnitude times the activation of its input channel, lowest
+ * pruned) restricted to 2:4 groups (PATCH page, section 1: semi-structured
+ * 2:4, two nonzeros per four; section 2: one of six patterns per group),
+ * plus the per-tile dense / 2:4 decision (PATCH page, section 2, core
+ * mechanism).  PATCH learns that decision; this call either takes it from
+ * `map_in` or, when `map_in` is NULL, marks as 2:4 the floor(f * n_tiles)
+ * tiles of least tile_loss (ties to the lower tile index).
+ *
+ *   W_bf16      [N,K] bf16, 16-byte aligned.
+ *   Xcal_bf16   [T,K] bf16 calibration activations, 16-byte aligned; may be
+ *               NULL when colsq_in is given.
+ *   T           calibration tokens (>= 1 when Xcal_bf16 is used).
+ *   colsq_in    optional [K] fp64 sums of squares to reuse (matrices that
+ *               share an input, e.g. q/k/v); NULL = compute from Xcal.
+ *   shp         N % tile_n == 0, K % tile_k == 0; tiles in {64,128}.
+ *   sparse_tile_fraction  f in [0,1], used only when map_in is NULL.
+ *   map_in      optional caller map (copied to map_out).
+ *   meta_out    [N, K/32] uint32 (written).
+ *   map_out     [ceil(n_tiles/32)] uint32 (written).
+ *   colsq_out   optional [K] fp64 (written when non-NULL).
+ *   tile_loss_out optional [n_tiles] fp64 (written when non-NULL).
+ *
+ * Temporary device memory (chunk partials of the column sums, 8*K*ceil(T/128)
+ * bytes, plus 8*K bytes of norms) is taken from the stream-ordered pool and
+ * released on the same stream.  Errors: INVALID_ARG for null/misaligned
+ * pointers or bad shapes; UNSUPPORTED for other tile sizes; OOM; CUDA.
+ */
+patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t T,
+                              const double *colsq_in, patch_shape shp,
+                              double sparse_tile_fraction, const uint32_t *map_in,
+                              uint32_t *meta_out, uint32_t *map_out, double *colsq_out,
+                              double *tile_loss_out, void *stream);
+
+/*
+ * Compressor: lay the dense tiles and the 2:4-compressed tiles (kept values +
+ * metadata) out for the hybrid GEMM.  Compressed storage is what turns
+ * zeros into speed (SparseGPT-vs-Wanda page, section on structured vs
+ * unstructured sparsity); the layout is this library's own.
+ *
+ *   W_bf16  [N,K] bf16 (16-byte aligned); meta, map as produced above.
+ *   shp     as above, and additionally N % 128 == 0 and K % 128 == 0.
+ *   max_decode_m  largest M (1..16) the handle will run through the split-K
+ *           decode path; sizes the handle's fp32 split-K workspace.  0 = 16.
+ *   out     receives the new handle (host pointer to a library object).
+ *   packed_bytes  optional host pointer: compressed weight bytes (values +
+ *           metadata, excluding the k-step table).
+ *
+ * Packed format (normative).  Geometry: bands of 128 rows, k-steps of 64
+ * columns, k-pairs of 128 columns.
+ *   - k-step (band b, step c) is stored 2:4-compressed iff every map tile
+ *     overlapping rows [128b,128b+128) x cols [64c,64c+64) is 2:4; otherwise
+ *     dense, holding W_eff (W with pruned entries of 2:4 tiles set to +0).
+ *   - bands one after another; inside a band, k-steps in order.
+ *   - dense k-step: 16384 bytes; element (r,k), r<128, k<64, at byte
+ *     (r/8)*1024 + (r%8)*128 + ((k/8) ^ (r%8))*16 + (k%8)*2
+ *     (the tensor-core K-major 128-byte-swizzled layout).
+ *   - 2:4 k-step: 8192 bytes of kept values; kept value v (v<32, column
+ *     order, two per group) of row r at byte
+ *     (r/8)*512 + (r%8)*64 + ((v/8) ^ ((r%8)/2))*16 + (v%8)*2
+ *     (K-major 64-byte-swizzled).
+ *   - metadata block: 2048 bytes per (band, k-pair) holding at least one 2:4
+ *     k-step, placed right before the values of the pair's first 2:4
+ *     k-step.  Row m = m0+8*m1+16*m2 (m0<8,m1<2,m2<8), pair column
+ *     k = k0+16*k1+32*k2 (k0<16,k1<2,k2<4): the code bit of column k is in
+ *     16-byte line m0+8*k1+16*m2 at bit 32*k2+16*m1+k0 (a group's 4-bit code
+ *     over its four columns, least significant bit first).  Bits of a dense
+ *     k-step are 0.  This is the tensor-memory metadata layout of the
+ *     sm_100 sparse MMA for 16-bit inputs, one 16-byte line per TMEM lane.
+ *   - table[b*(K/64)+c] (uint64): bits 0..47 byte offset of the k-step's
+ *     data, bit 62 = 2:4, bit 63 = the pair's metadata block precedes it.
+ *
+ * Synchronises the stream once: the map is read back to plan the layout and
+ * size the allocation exactly.
+ * Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA.
+ */
+patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
+                        patch_shape shp, int32_t max_decode_m, patch_packed **out,
+                        size_t *packed_bytes, void *stream);
+
+/*
+ * Hybrid product Y[M,N] = X[M,K] * W_eff^T with fp32 accumulation in tensor
+ * memory and one rounding at the end (PATCH page, section 2, inference and
+ * deployment: one kernel over mixed dense / 2:4 tiles).  Dense k-steps issue
+ * the dense tcgen05 MMA, 2:4 k-steps the sparse tcgen05 MMA, into one
+ * accumulator.  M <= 16 (and M <= the handle's max_decode_m) runs the split-K
+ * decode configuration; larger M the prefill configuration.
+ *
+ *   Wp      handle from patch_pack.
+ *   X_bf16  [M,K] bf16, 16-byte aligned.
+ *   M       tokens, >= 0 (any value; a ragged last token tile is masked;
+ *           M == 0 returns PATCH_OK without touching X or Y).
+ *   Y       [M,N]: bf16 (y_is_fp32 = 0) or fp32 (y_is_fp32 = 1), 16-byte
+ *           aligned.
+ *
+ * Every device wait inside the kernel is bounded; a wait that runs out sets
+ * the handle's status word and the kernel returns early (Y undefined).
+ * Errors: INVALID_ARG, CUDA; PATCH_ERR_TIMEOUT is reported by
+ * patch_get_status, not here (the call does not synchronise).
+ */
+patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
+                               int32_t y_is_fp32, void *stream);
+
+/* Release a handle's device memory (stream-ordered on `stream`).  NULL ok. */
+void patch_free(patch_packed *Wp, void *stream);
+
+/*
+ * Read the handle's device status word (synchronises the device).
+ * PATCH_OK, PATCH_ERR_TIMEOUT (a bounded wait ran out in an earlier
+ * patch_hybrid_gemm), or PATCH_ERR_CUDA / INVALID_ARG.
+ */
+patch_status patch_get_status(const patch_packed *Wp);
+
+/* Read-only view of a handle, for inspection and tests. */
+typedef struct {
+    const void *packed;     /* device: packed bytes                         */
+    const uint64_t *table;  /* device: k-step table, (N/128)*(K/64) entries */
+    size_t packed_bytes;    /* bytes at `packed`                            */
+    int64_t N, K;
+    int32_t tile_n, tile_k;
+    int64_t sparse_ksteps;  /* k-steps stored 2:4                           */
+    int64_t meta_blocks;    /* 2048-byte metadata blocks                    */
+} patch_packed_view;
+
+patch_status patch_packed_info(const patch_packed *Wp, patch_packed_view *view);
+
+/*
+ * Copy a handle's packed bytes (view.packed_bytes) and k-step table
+ * ((N/128)*(K/64) uint64) into caller-owned DEVICE buffers, stream-ordered.
+ * Either destination may be NULL to skip it.  For inspection and tests.
+ */
+patch_status patch_packed_export(const patch_packed *Wp, void *packed_dst, uint64_t *table_dst,
+                                 void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *patch_status_string(patch_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PATCH_B200_H */

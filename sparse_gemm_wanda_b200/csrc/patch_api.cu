@@ -1,0 +1,309 @@
+// C ABI of the tile-hybrid sparse linear layer: argument checks, planning of
+// the packed layout, device memory of the packed handle, kernel launches.
+// Declarations and the normative description of every call: include/patch.h.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "patch.h"
+#include "patch_common.cuh"
+#include "patch_internal.h"
+
+struct patch_packed {
+    int device;
+    patch_shape shp;
+    uint8_t *packed;           // packed k-steps
+    size_t packed_bytes;
+    uint64_t *table;           // (N/128) * (K/64) entries
+    int64_t sparse_ksteps;
+    int64_t meta_blocks;
+    float *workspace;          // split-K partials for the decode configuration
+    int64_t workspace_floats;
+    int32_t max_decode_m;
+    uint32_t *status;          // device status word
+    int num_sms;
+};
+
+namespace {
+
+using patchk::kBand;
+using patchk::kStep;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool tile_ok(int32_t t) { return t == 64 || t == 128; }
+
+patch_status check_shape(const patch_shape &s) {
+    if (s.N <= 0 || s.K <= 0) return PATCH_ERR_INVALID_ARG;
+    if (!tile_ok(s.tile_n) || !tile_ok(s.tile_k)) return PATCH_ERR_UNSUPPORTED;
+    if (s.N % s.tile_n != 0 || s.K % s.tile_k != 0) return PATCH_ERR_INVALID_ARG;
+    if (s.K % 64 != 0) return PATCH_ERR_INVALID_ARG;
+    if (s.N > (int64_t(1) << 31) || s.K > (int64_t(1) << 31)) return PATCH_ERR_INVALID_ARG;
+    return PATCH_OK;
+}
+
+patch_status check_device(int *num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PATCH_ERR_CUDA;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return PATCH_ERR_CUDA;
+    if (major != 10 || minor != 0) return PATCH_ERR_UNSUPPORTED;
+    if (num_sms &&
+        cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return PATCH_ERR_CUDA;
+    return PATCH_OK;
+}
+
+patch_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return PATCH_OK;
+    if (e == cudaErrorMemoryAllocation) return PATCH_ERR_OOM;
+    return PATCH_ERR_CUDA;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+const char *patch_status_string(patch_status s) {
+    switch (s) {
+        case PATCH_OK: return "ok";
+        case PATCH_ERR_INVALID_ARG: return "invalid argument";
+        case PATCH_ERR_UNSUPPORTED: return "unsupported";
+        case PATCH_ERR_CUDA: return "cuda error";
+        case PATCH_ERR_OOM: return "out of device memory";
+        case PATCH_ERR_TIMEOUT: return "bounded device wait ran out";
+    }
+    return "unknown status";
+}
+
+patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t T,
+                              const double *colsq_in, patch_shape shp,
+                              double sparse_tile_fraction, const uint32_t *map_in,
+                              uint32_t *meta_out, uint32_t *map_out, double *colsq_out,
+                              double *tile_loss_out, void *stream_v) {
+    patch_status st = check_shape(shp);
+    if (st != PATCH_OK) return st;
+    if (!W_bf16 || !meta_out || !map_out || !aligned16(W_bf16)) return PATCH_ERR_INVALID_ARG;
+    if (!colsq_in && (!Xcal_bf16 || T < 1 || !aligned16(Xcal_bf16))) return PATCH_ERR_INVALID_ARG;
+    if (!map_in && !(sparse_tile_fraction >= 0.0 && sparse_tile_fraction <= 1.0))
+        return PATCH_ERR_INVALID_ARG;
+    st = check_device(nullptr);
+    if (st != PATCH_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+
+    const int64_t N = shp.N, K = shp.K;
+    const int64_t n_tiles = (N / shp.tile_n) * (K / shp.tile_k);
+    const int64_t chunks = colsq_in ? 0 : (T + 127) / 128;
+
+    // one stream-ordered scratch allocation: chunk partials, norms, loss, rank
+    size_t off_partial = 0;
+    size_t off_norm = round_up(off_partial + sizeof(double) * chunks * K, 256);
+    size_t off_loss = round_up(off_norm + sizeof(double) * K, 256);
+    size_t off_rank = round_up(off_loss + (tile_loss_out ? 0 : sizeof(double) * n_tiles), 256);
+    size_t total = round_up(off_rank + (map_in ? 0 : sizeof(int32_t) * n_tiles), 256);
+    uint8_t *scratch = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&scratch), total, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    double *partial = reinterpret_cast<double *>(scratch + off_partial);
+    double *norm = reinterpret_cast<double *>(scratch + off_norm);
+    double *loss = tile_loss_out ? tile_loss_out : reinterpret_cast<double *>(scratch + off_loss);
+    int32_t *rank = reinterpret_cast<int32_t *>(scratch + off_rank);
+
+    if (colsq_in)
+        e = patchk::launch_norms_from_colsq(colsq_in, K, colsq_out, norm, stream);
+    else
+        e = patchk::launch_colsq(Xcal_bf16, T, K, partial, colsq_out, norm, stream);
+    if (e == cudaSuccess)
+        e = patchk::launch_score_mask(W_bf16, norm, N, K, shp.tile_n, shp.tile_k, meta_out, loss,
+                                      stream);
+    if (e == cudaSuccess) {
+        if (map_in) {
+            e = cudaMemcpyAsync(map_out, map_in, sizeof(uint32_t) * ((n_tiles + 31) / 32),
+                                cudaMemcpyDeviceToDevice, stream);
+        } else {
+            const int64_t n_sp =
+                static_cast<int64_t>(floor(sparse_tile_fraction * static_cast<double>(n_tiles)));
+            e = patchk::launch_select_map(loss, n_tiles, n_sp, rank, map_out, stream);
+        }
+    }
+    cudaError_t e2 = cudaFreeAsync(scratch, stream);
+    return from_cuda(e != cudaSuccess ? e : e2);
+}
+
+patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
+                        patch_shape shp, int32_t max_decode_m, patch_packed **out,
+                        size_t *packed_bytes, void *stream_v) {
+    if (!out) return PATCH_ERR_INVALID_ARG;
+    *out = nullptr;
+    patch_status st = check_shape(shp);
+    if (st != PATCH_OK) return st;
+    if (shp.N % kBand != 0 || shp.K % (2 * kStep) != 0) return PATCH_ERR_INVALID_ARG;
+    if (!W_bf16 || !meta || !map || !aligned16(W_bf16)) return PATCH_ERR_INVALID_ARG;
+    if (max_decode_m < 0 || max_decode_m > 16) return PATCH_ERR_INVALID_ARG;
+    if (max_decode_m == 0) max_decode_m = 16;
+    int num_sms = 0;
+    st = check_device(&num_sms);
+    if (st != PATCH_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+
+    const int64_t N = shp.N, K = shp.K, tn = shp.tile_n, tk = shp.tile_k;
+    const int64_t tiles_k = K / tk, n_tiles = (N / tn) * tiles_k;
+    const int64_t bands = N / kBand, nsteps = K / kStep;
+
+    // the map is read back once to plan the layout
+    std::vector<uint32_t> hmap(static_cast<size_t>((n_tiles + 31) / 32));
+    cudaError_t e = cudaMemcpyAsync(hmap.data(), map, sizeof(uint32_t) * hmap.size(),
+                                    cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    auto tile_sparse = [&](int64_t t) { return ((hmap[t / 32] >> (t % 32)) & 1u) != 0; };
+
+    std::vector<uint64_t> table(static_cast<size_t>(bands * nsteps));
+    std::vector<uint8_t> sparse(static_cast<size_t>(nsteps));
+    uint64_t offset = 0;
+    int64_t n_sparse = 0, n_meta = 0;
+    for (int64_t b = 0; b < bands; ++b) {
+        for (int64_t c = 0; c < nsteps; ++c) {
+            bool all = true;
+            for (int64_t ti = (b * kBand) / tn; ti <= (b * kBand + kBand - 1) / tn; ++ti)
+                for (int64_t tj = (c * kStep) / tk; tj <= (c * kStep + kStep - 1) / tk; ++tj)
+                    all = all && tile_sparse(ti * tiles_k + tj);
+            sparse[c] = all;
+        }
+        for (int64_t c = 0; c < nsteps; ++c) {
+            uint64_t entry = 0;
+            if (sparse[c]) {
+                const bool first_of_pair = (c % 2 == 0) || !sparse[c - 1];
+                if (first_of_pair) {
+                    offset += patchk::kMetaBlockBytes;
+                    entry |= patchk::kEntryMeta;
+                    ++n_meta;
+                }
+                entry |= offset | patchk::kEntrySparse;
+                offset += patchk::kSparseStepBytes;
+                ++n_sparse;
+            } else {
+                entry = offset;
+                offset += patchk::kDenseStepBytes;
+            }
+            table[static_cast<size_t>(b * nsteps + c)] = entry;
+        }
+    }
+
+    patch_packed *h = new (std::nothrow) patch_packed();
+    if (!h) return PATCH_ERR_OOM;
+    cudaGetDevice(&h->device);
+    h->shp = shp;
+    h->packed_bytes = static_cast<size_t>(offset);
+    h->sparse_ksteps = n_sparse;
+    h->meta_blocks = n_meta;
+    h->max_decode_m = max_decode_m;
+    h->num_sms = num_sms;
+    const int splits = patchk::decode_splits(N, K, num_sms);
+    h->workspace_floats = static_cast<int64_t>(splits) * max_decode_m * N;
+
+    e = cudaMallocAsync(reinterpret_cast<void **>(&h->packed), h->packed_bytes ? h->packed_bytes : 16, stream);
+    if (e == cudaSuccess)
+        e = cudaMallocAsync(reinterpret_cast<void **>(&h->table), sizeof(uint64_t) * table.size(), stream);
+    if (e == cudaSuccess)
+        e = cudaMallocAsync(reinterpret_cast<void **>(&h->workspace),
+                            sizeof(float) * static_cast<size_t>(h->workspace_floats), stream);
+    if (e == cudaSuccess)
+        e = cudaMallocAsync(reinterpret_cast<void **>(&h->status), sizeof(uint32_t) * 4, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(h->status, 0, sizeof(uint32_t) * 4, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(h->table, table.data(), sizeof(uint64_t) * table.size(),
+                            cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess)
+        e = patchk::launch_pack(W_bf16, meta, map, N, K, static_cast<int>(tn), static_cast<int>(tk),
+                                h->table, h->packed, stream);
+    if (e != cudaSuccess) {
+        patch_free(h, stream_v);
+        return from_cuda(e);
+    }
+    if (packed_bytes) *packed_bytes = h->packed_bytes;
+    *out = h;
+    return PATCH_OK;
+}
+
+patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
+                               int32_t y_is_fp32, void *stream_v) {
+    if (!Wp || M < 0) return PATCH_ERR_INVALID_ARG;
+    if (M == 0) return PATCH_OK;  // empty batch: nothing to do
+    if (!X_bf16 || !Y) return PATCH_ERR_INVALID_ARG;
+    if (!aligned16(X_bf16) || !aligned16(Y)) return PATCH_ERR_INVALID_ARG;
+    if (y_is_fp32 != 0 && y_is_fp32 != 1) return PATCH_ERR_INVALID_ARG;
+    if (M > (int64_t(1) << 31)) return PATCH_ERR_INVALID_ARG;
+    patchk::GemmLaunch g;
+    g.packed = Wp->packed;
+    g.table = Wp->table;
+    g.N = Wp->shp.N;
+    g.K = Wp->shp.K;
+    g.X = X_bf16;
+    g.M = M;
+    g.Y = Y;
+    g.y_fp32 = y_is_fp32;
+    g.workspace = (M <= Wp->max_decode_m) ? Wp->workspace : nullptr;
+    g.workspace_floats = Wp->workspace_floats;
+    g.status = Wp->status;
+    g.num_sms = Wp->num_sms;
+    return from_cuda(patchk::launch_hybrid_gemm(g, static_cast<cudaStream_t>(stream_v)));
+}
+
+void patch_free(patch_packed *Wp, void *stream_v) {
+    if (!Wp) return;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    if (Wp->packed) cudaFreeAsync(Wp->packed, stream);
+    if (Wp->table) cudaFreeAsync(Wp->table, stream);
+    if (Wp->workspace) cudaFreeAsync(Wp->workspace, stream);
+    if (Wp->status) cudaFreeAsync(Wp->status, stream);
+    delete Wp;
+}
+
+patch_status patch_get_status(const patch_packed *Wp) {
+    if (!Wp) return PATCH_ERR_INVALID_ARG;
+    uint32_t word = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(&word, Wp->status, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return from_cuda(e);
+    return (word & patchk::kStatusTimeout) ? PATCH_ERR_TIMEOUT : PATCH_OK;
+}
+
+patch_status patch_packed_info(const patch_packed *Wp, patch_packed_view *view) {
+    if (!Wp || !view) return PATCH_ERR_INVALID_ARG;
+    view->packed = Wp->packed;
+    view->table = Wp->table;
+    view->packed_bytes = Wp->packed_bytes;
+    view->N = Wp->shp.N;
+    view->K = Wp->shp.K;
+    view->tile_n = Wp->shp.tile_n;
+    view->tile_k = Wp->shp.tile_k;
+    view->sparse_ksteps = Wp->sparse_ksteps;
+    view->meta_blocks = Wp->meta_blocks;
+    return PATCH_OK;
+}
+
+patch_status patch_packed_export(const patch_packed *Wp, void *packed_dst, uint64_t *table_dst,
+                                 void *stream_v) {
+    if (!Wp) return PATCH_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    cudaError_t e = cudaSuccess;
+    if (packed_dst && Wp->packed_bytes)
+        e = cudaMemcpyAsync(packed_dst, Wp->packed, Wp->packed_bytes, cudaMemcpyDeviceToDevice,
+                            stream);
+    if (e == cudaSuccess && table_dst)
+        e = cudaMemcpyAsync(table_dst, Wp->table,
+                            sizeof(uint64_t) * (Wp->shp.N / kBand) * (Wp->shp.K / kStep),
+                            cudaMemcpyDeviceToDevice, stream);
+    return from_cuda(e);
+}
+
+}  // extern "C"

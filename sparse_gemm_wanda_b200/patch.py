@@ -1,0 +1,206 @@
+"""Thin ctypes binding of ``libpatch_b200.so`` (include/patch.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  PyTorch provides device memory and the current stream.  If the
+library is missing or cannot be loaded, every call raises ``PatchLibraryError``;
+there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpatch_b200.so")
+
+PATCH_OK = 0
+STATUS_NAMES = {0: "PATCH_OK", 1: "PATCH_ERR_INVALID_ARG", 2: "PATCH_ERR_UNSUPPORTED",
+                3: "PATCH_ERR_CUDA", 4: "PATCH_ERR_OOM", 5: "PATCH_ERR_TIMEOUT"}
+
+# every symbol include/patch.h declares
+EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
+           "patch_get_status", "patch_packed_info", "patch_packed_export",
+           "patch_status_string")
+
+
+class PatchLibraryError(RuntimeError):
+    pass
+
+
+class PatchError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+class PatchShape(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("tile_n", ctypes.c_int32), ("tile_k", ctypes.c_int32)]
+
+
+class PatchPackedView(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("table", ctypes.c_void_p),
+                ("packed_bytes", ctypes.c_size_t), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("tile_n", ctypes.c_int32), ("tile_k", ctypes.c_int32),
+                ("sparse_ksteps", ctypes.c_int64), ("meta_blocks", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises PatchLibraryError when it is absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise PatchLibraryError(
+            f"{path} is missing: build it with `python -m sparse_gemm_wanda_b200.build`")
+    try:
+        lib = ctypes.CDLL(path)
+    except OSError as exc:
+        raise PatchLibraryError(f"cannot load {path}: {exc}") from exc
+    vp, i64, i32, dbl = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+    lib.patch_score_mask.argtypes = [vp, vp, i64, vp, PatchShape, dbl, vp, vp, vp, vp, vp, vp]
+    lib.patch_pack.argtypes = [vp, vp, vp, PatchShape, i32, ctypes.POINTER(vp),
+                               ctypes.POINTER(ctypes.c_size_t), vp]
+    lib.patch_hybrid_gemm.argtypes = [vp, vp, i64, vp, i32, vp]
+    lib.patch_free.argtypes = [vp, vp]
+    lib.patch_free.restype = None
+    lib.patch_get_status.argtypes = [vp]
+    lib.patch_packed_info.argtypes = [vp, ctypes.POINTER(PatchPackedView)]
+    lib.patch_packed_export.argtypes = [vp, vp, vp, vp]
+    lib.patch_status_string.argtypes = [ctypes.c_int]
+    lib.patch_status_string.restype = ctypes.c_char_p
+    for name in ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_get_status",
+                 "patch_packed_info", "patch_packed_export"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, code: int):
+    if code != PATCH_OK:
+        raise PatchError(fn, code)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def n_tiles(N: int, K: int, tile_n: int, tile_k: int) -> int:
+    return (N // tile_n) * (K // tile_k)
+
+
+def patch_score_mask(W: torch.Tensor, Xcal: torch.Tensor | None = None, *, tile_n: int = 128,
+                     tile_k: int = 128, fraction: float = 0.0, map_in: torch.Tensor | None = None,
+                     colsq_in: torch.Tensor | None = None, want_colsq: bool = False,
+                     want_loss: bool = False, stream=None) -> dict:
+    """Wanda 2:4 codes, tile map (and optionally colsq, tile loss) for W[N,K] bf16."""
+    lib = load_library()
+    N, K = W.shape
+    nt = n_tiles(N, K, tile_n, tile_k)
+    dev = W.device
+    meta = torch.empty((N, K // 32), dtype=torch.int32, device=dev)
+    tmap = torch.empty(((nt + 31) // 32,), dtype=torch.int32, device=dev)
+    colsq = torch.empty((K,), dtype=torch.float64, device=dev) if want_colsq else None
+    loss = torch.empty((nt,), dtype=torch.float64, device=dev) if want_loss else None
+    T = Xcal.shape[0] if Xcal is not None else 0
+    code = lib.patch_score_mask(
+        _dptr(W, torch.bfloat16, "W"), _dptr(Xcal, torch.bfloat16, "Xcal"), T,
+        _dptr(colsq_in, torch.float64, "colsq_in"), PatchShape(N, K, tile_n, tile_k),
+        float(fraction), _dptr(map_in, (torch.int32, torch.uint32), "map_in"), _dptr(meta),
+        _dptr(tmap), _dptr(colsq), _dptr(loss), _stream(stream))
+    _check("patch_score_mask", code)
+    return {"meta": meta, "map": tmap, "colsq": colsq, "loss": loss}
+
+
+class PackedWeight:
+    """Owns a patch_packed handle; released by patch_free on close / deletion."""
+
+    def __init__(self, handle: int, shape: tuple, packed_bytes: int):
+        self.handle = ctypes.c_void_p(handle)
+        self.N, self.K, self.tile_n, self.tile_k = shape
+        self.packed_bytes = packed_bytes
+
+    def view(self) -> PatchPackedView:
+        v = PatchPackedView()
+        _check("patch_packed_info", load_library().patch_packed_info(self.handle, ctypes.byref(v)))
+        return v
+
+    def export(self, stream=None):
+        """Copies of the packed bytes (uint8) and the k-step table (int64) as CUDA tensors."""
+        v = self.view()
+        packed = torch.empty((v.packed_bytes,), dtype=torch.uint8, device="cuda")
+        table = torch.empty(((self.N // 128) * (self.K // 64),), dtype=torch.int64, device="cuda")
+        _check("patch_packed_export", load_library().patch_packed_export(
+            self.handle, _dptr(packed), _dptr(table), _stream(stream)))
+        return packed, table
+
+    def close(self, stream=None):
+        if self.handle and self.handle.value:
+            load_library().patch_free(self.handle, _stream(stream))
+            self.handle = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def patch_pack(W: torch.Tensor, meta: torch.Tensor, tile_map: torch.Tensor, *, tile_n: int = 128,
+               tile_k: int = 128, max_decode_m: int = 16, stream=None) -> PackedWeight:
+    """Compress W (dense tiles + 2:4 tiles) into a library-owned handle."""
+    lib = load_library()
+    N, K = W.shape
+    out = ctypes.c_void_p(0)
+    nbytes = ctypes.c_size_t(0)
+    code = lib.patch_pack(_dptr(W, torch.bfloat16, "W"), _dptr(meta, (torch.int32, torch.uint32), "meta"),
+                          _dptr(tile_map, (torch.int32, torch.uint32), "map"),
+                          PatchShape(N, K, tile_n, tile_k), int(max_decode_m), ctypes.byref(out),
+                          ctypes.byref(nbytes), _stream(stream))
+    _check("patch_pack", code)
+    return PackedWeight(out.value, (N, K, tile_n, tile_k), nbytes.value)
+
+
+def patch_hybrid_gemm(packed: PackedWeight, X: torch.Tensor, out: torch.Tensor | None = None,
+                      out_fp32: bool = False, stream=None) -> torch.Tensor:
+    """Y[M,N] = X[M,K] @ W_eff^T on the tensor cores (bf16 out, or fp32 out)."""
+    lib = load_library()
+    M, K = X.shape
+    if K != packed.K:
+        raise ValueError(f"X has {K} columns, the packed weight {packed.K}")
+    if out is None:
+        out = torch.empty((M, packed.N), dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                          device=X.device)
+    want = torch.float32 if out_fp32 else torch.bfloat16
+    code = lib.patch_hybrid_gemm(packed.handle, _dptr(X, torch.bfloat16, "X"), M,
+                                 _dptr(out, want, "out"), 1 if out_fp32 else 0, _stream(stream))
+    _check("patch_hybrid_gemm", code)
+    return out
+
+
+def patch_free(packed: PackedWeight, stream=None) -> None:
+    packed.close(stream)
+
+
+def patch_get_status(packed: PackedWeight) -> int:
+    """0 (ok) or 5 (a bounded device wait ran out); synchronises the device."""
+    return int(load_library().patch_get_status(packed.handle))

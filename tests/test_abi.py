@@ -1,0 +1,111 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+symbol include/patch.h declares, and rejects bad arguments before touching the
+device.  No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "patch.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_gemm_wanda_b200 import build, patch
+    build.build()
+    return patch.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(patch_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from sparse_gemm_wanda_b200 import patch
+    names = declared_functions()
+    assert set(names) == set(patch.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    assert lib.patch_status_string(0) == b"ok"
+    assert lib.patch_status_string(5) == b"bounded device wait ran out"
+
+
+def test_gemm_rejects_null_handle(lib):
+    assert lib.patch_hybrid_gemm(None, None, 1, None, 0, None) == 1
+    assert lib.patch_hybrid_gemm(None, None, -1, None, 0, None) == 1
+
+
+def test_score_mask_argument_checks(lib):
+    from sparse_gemm_wanda_b200.patch import PatchShape
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: checks fail first
+    # unsupported tile size
+    assert lib.patch_score_mask(fake, fake, 8, None, PatchShape(256, 256, 32, 64), 0.5, None,
+                                fake, fake, None, None, None) == 2
+    # N not a multiple of the tile
+    assert lib.patch_score_mask(fake, fake, 8, None, PatchShape(200, 256, 64, 64), 0.5, None,
+                                fake, fake, None, None, None) == 1
+    # null weight
+    assert lib.patch_score_mask(None, fake, 8, None, PatchShape(256, 256, 64, 64), 0.5, None,
+                                fake, fake, None, None, None) == 1
+    # misaligned weight
+    assert lib.patch_score_mask(ctypes.c_void_p(0x1002), fake, 8, None,
+                                PatchShape(256, 256, 64, 64), 0.5, None, fake, fake, None, None,
+                                None) == 1
+    # no calibration and no colsq
+    assert lib.patch_score_mask(fake, None, 8, None, PatchShape(256, 256, 64, 64), 0.5, None,
+                                fake, fake, None, None, None) == 1
+    # fraction out of range without a map
+    assert lib.patch_score_mask(fake, fake, 8, None, PatchShape(256, 256, 64, 64), 1.5, None,
+                                fake, fake, None, None, None) == 1
+    # T < 1
+    assert lib.patch_score_mask(fake, fake, 0, None, PatchShape(256, 256, 64, 64), 0.5, None,
+                                fake, fake, None, None, None) == 1
+
+
+def test_pack_argument_checks(lib):
+    from sparse_gemm_wanda_b200.patch import PatchShape
+    fake = ctypes.c_void_p(0x1000)
+    out = ctypes.c_void_p(0)
+    assert lib.patch_pack(fake, fake, fake, PatchShape(256, 256, 64, 64), 16, None, None,
+                          None) == 1
+    # N not a multiple of 128 (64-row tiles allow N=192, the packed bands do not)
+    assert lib.patch_pack(fake, fake, fake, PatchShape(192, 256, 64, 64), 16, ctypes.byref(out),
+                          None, None) == 1
+    # K not a multiple of 128
+    assert lib.patch_pack(fake, fake, fake, PatchShape(256, 192, 64, 64), 16, ctypes.byref(out),
+                          None, None) == 1
+    assert lib.patch_pack(fake, fake, fake, PatchShape(256, 256, 64, 64), 17, ctypes.byref(out),
+                          None, None) == 1
+    assert out.value is None
+
+
+def test_handle_calls_reject_null(lib):
+    assert lib.patch_get_status(None) == 1
+    assert lib.patch_packed_info(None, None) == 1
+    assert lib.patch_packed_export(None, None, None, None) == 1
+    lib.patch_free(None, None)  # no-op
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from sparse_gemm_wanda_b200 import patch
+    with pytest.raises(patch.PatchLibraryError):
+        # a fresh loader pointed at a missing file must raise, not fall back
+        saved = patch._lib
+        try:
+            patch._lib = None
+            patch.load_library(str(tmp_path / "missing.so"))
+        finally:
+            patch._lib = saved

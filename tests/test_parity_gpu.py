@@ -1,0 +1,263 @@
+"""GPU path vs the CPU oracle, element by element, through the C ABI.
+
+Bit-exact: column sums of squares, 2:4 codes, tile losses, tile maps, packed
+bytes and k-step tables.  GEMM: fp32-output mode within the literal bound
+max|y - y_ref| <= 1e-2 * RMS(y_ref); bf16-output mode per element within
+1e-2 * RMS(y_ref) + half a bf16 ulp of max(|y|, |y_ref|) (the output rounding
+alone can exceed the literal bound at |y| > ~2.6 RMS).
+"""
+import numpy as np
+import pytest
+import torch
+
+from sparse_gemm_wanda_b200 import inputs
+from tests.conftest import bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU machines, skipped there
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+
+@pytest.fixture(scope="module")
+def P():
+    from sparse_gemm_wanda_b200 import build, patch
+    build.build()
+    patch.load_library()
+    return patch
+
+
+def u32(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def rel_rms_check(y, yref_f64, fp32_mode):
+    y = y.double().cpu().numpy()
+    rms = float(np.sqrt(np.mean(yref_f64 ** 2))) if yref_f64.size else 0.0
+    err = np.abs(y - yref_f64)
+    if fp32_mode:
+        assert err.max() <= 1e-2 * rms, (err.max(), rms)
+    else:
+        mag = np.maximum(np.abs(y), np.abs(yref_f64))
+        ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-30))) - 7)
+        bad = err > 1e-2 * rms + 0.5 * ulp
+        assert not bad.any(), (int(bad.sum()), float(err.max()), rms)
+    return float(err.max()), rms
+
+
+def make_problem(N, K, T, M, seed, outliers=None):
+    w = inputs.weight(N, K, seed)
+    o = inputs.outlier_channels(K, seed, outliers)
+    xc = inputs.activations(T, K, seed, o, role=0) if T else None
+    x = inputs.activations(M, K, seed, o, role=1)
+    return w, xc, x
+
+
+def oracle_mask(oracle_mod, w, xc, tn, tk, frac=None, tmap=None):
+    return oracle_mod.score_mask(bf16_bits(w), bf16_bits(xc), tn, tk,
+                                 fraction=frac if frac is not None else 0.0,
+                                 tile_map=tmap)
+
+
+# ---------------------------------------------------------------- mask builder
+
+@pytest.mark.parametrize("N,K,T,tn,tk,frac", [
+    (256, 256, 64, 64, 64, 0.5),        # tiny config shape
+    (256, 512, 300, 128, 128, 0.5),     # ragged calibration chunk
+    (512, 384, 129, 64, 128, 0.3),
+    (384, 256, 1, 128, 64, 1.0),        # single calibration token
+    (256, 256, 64, 64, 64, 0.0),
+    (4096, 4096, 2048, 128, 128, 0.5),  # decode config, attention-shaped
+    (11008, 4096, 2048, 128, 128, 0.5), # decode config, MLP-shaped
+])
+def test_mask_builder_bit_exact(P, oracle_mod, N, K, T, tn, tk, frac):
+    w, xc, _ = make_problem(N, K, T, 1, seed=N + K + T, outliers=3 if K == 256 else None)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), tile_n=tn, tile_k=tk, fraction=frac,
+                           want_colsq=True, want_loss=True)
+    torch.cuda.synchronize()
+    ref = oracle_mask(oracle_mod, w, xc, tn, tk, frac=frac)
+    assert np.array_equal(r["colsq"].cpu().numpy(), ref["colsq"])
+    assert np.array_equal(u32(r["meta"]), ref["meta"])
+    assert np.array_equal(r["loss"].cpu().numpy(), ref["loss"])
+    assert np.array_equal(u32(r["map"]), ref["map"])
+
+
+def test_mask_builder_given_map_and_colsq(P, oracle_mod):
+    N, K, tn, tk = 512, 512, 128, 64
+    w, xc, _ = make_problem(N, K, 200, 1, seed=7)
+    nt = (N // tn) * (K // tk)
+    tmap = inputs.random_map(nt, nt // 3, seed=7)
+    ref = oracle_mask(oracle_mod, w, xc, tn, tk, tmap=tmap.numpy().view(np.uint32))
+    colsq = torch.from_numpy(ref["colsq"]).cuda()
+    r = P.patch_score_mask(w.cuda(), None, tile_n=tn, tile_k=tk, map_in=tmap.cuda(),
+                           colsq_in=colsq, want_colsq=True, want_loss=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(u32(r["meta"]), ref["meta"])
+    assert np.array_equal(u32(r["map"]), ref["map"])
+    assert np.array_equal(r["colsq"].cpu().numpy(), ref["colsq"])
+    assert np.array_equal(r["loss"].cpu().numpy(), ref["loss"])
+
+
+def test_mask_builder_ties(P, oracle_mod):
+    # zero and duplicated calibration columns: exact score ties everywhere
+    N, K = 256, 256
+    w, xc, _ = make_problem(N, K, 64, 1, seed=3)
+    xc = xc.clone()
+    xc[:, 0:64] = 0
+    xc[:, 64:128] = xc[:, 128:192]
+    w = w.clone()
+    w[:, 200:256] = w[:, 200:201]  # equal magnitudes along rows
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), tile_n=64, tile_k=64, fraction=0.5,
+                           want_colsq=True, want_loss=True)
+    torch.cuda.synchronize()
+    ref = oracle_mask(oracle_mod, w, xc, 64, 64, frac=0.5)
+    assert np.array_equal(u32(r["meta"]), ref["meta"])
+    assert np.array_equal(u32(r["map"]), ref["map"])
+    assert np.array_equal(r["loss"].cpu().numpy(), ref["loss"])
+
+
+# ----------------------------------------------------------------------- pack
+
+@pytest.mark.parametrize("tn,tk", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("frac", [0.0, 0.3, 0.5, 1.0])
+def test_pack_bit_exact(P, oracle_mod, tn, tk, frac):
+    N, K = 512, 768
+    w, xc, _ = make_problem(N, K, 64, 1, seed=tn + tk + int(frac * 100))
+    nt = (N // tn) * (K // tk)
+    tmap = inputs.random_map(nt, int(frac * nt), seed=tn * 3 + tk)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), tile_n=tn, tile_k=tk, map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"], tile_n=tn, tile_k=tk)
+    packed, table = pk.export()
+    torch.cuda.synchronize()
+    ref_meta = oracle_mask(oracle_mod, w, xc, tn, tk, tmap=tmap.numpy().view(np.uint32))["meta"]
+    ref_packed, ref_table = oracle_mod.pack(bf16_bits(w), ref_meta, tmap.numpy().view(np.uint32),
+                                            tn, tk)
+    assert pk.packed_bytes == ref_packed.size
+    assert np.array_equal(table.cpu().numpy().view(np.uint64), ref_table)
+    assert np.array_equal(packed.cpu().numpy(), ref_packed)
+    pk.close()
+
+
+# ----------------------------------------------------------------------- GEMM
+
+def run_case(P, oracle_mod, N, K, M, tn, tk, frac, seed, fp32_mode, sample=None):
+    w, xc, x = make_problem(N, K, 64, M, seed)
+    nt = (N // tn) * (K // tk)
+    tmap = inputs.random_map(nt, int(round(frac * nt)), seed=seed)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), tile_n=tn, tile_k=tk, map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"], tile_n=tn, tile_k=tk)
+    y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=fp32_mode)
+    torch.cuda.synchronize()
+    assert P.patch_get_status(pk) == 0
+    meta = u32(r["meta"])
+    weff = oracle_mod.weff(bf16_bits(w), meta, tmap.numpy().view(np.uint32), tn, tk)
+    if sample is None:
+        yref = oracle_mod.gemm(bf16_bits(x), weff)
+        out = rel_rms_check(y, yref, fp32_mode)
+    else:
+        g = np.random.default_rng(seed)
+        ms = g.integers(0, M, sample)
+        ns = g.integers(0, N, sample)
+        yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
+        # RMS of the reference over the sample stands in for the full matrix
+        out = rel_rms_check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref,
+                            fp32_mode)
+    pk.close()
+    return out
+
+
+@pytest.mark.parametrize("fp32_mode", [True, False])
+@pytest.mark.parametrize("M", [1, 3, 8, 16, 17, 64, 100, 128, 200, 256, 300])
+def test_gemm_small_shapes(P, oracle_mod, M, fp32_mode):
+    run_case(P, oracle_mod, 384, 512, M, 128, 128, 0.5, seed=M, fp32_mode=fp32_mode)
+
+
+@pytest.mark.parametrize("tn,tk", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
+@pytest.mark.parametrize("M", [8, 160])
+def test_gemm_tiles_and_fractions(P, oracle_mod, tn, tk, frac, M):
+    run_case(P, oracle_mod, 256, 512, M, tn, tk, frac, seed=tn + tk + M, fp32_mode=True)
+
+
+def test_gemm_tiny_config(P, oracle_mod):
+    # W 256x256, 64x64 tiles, 8 of 16 tiles 2:4, Xcal 64x256, X 8x256, 3 outlier channels
+    wl = inputs.workloads()["tiny"]
+    s = wl.seed
+    w = inputs.weight(256, 256, s)
+    o = inputs.outlier_channels(256, s, 3)
+    xc = inputs.activations(64, 256, s, o, role=0)
+    x = inputs.activations(8, 256, s, o, role=1)
+    tmap = inputs.random_map(16, 8, s)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), tile_n=64, tile_k=64, map_in=tmap.cuda(),
+                           want_colsq=True, want_loss=True)
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"], tile_n=64, tile_k=64)
+    y32 = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    y16 = P.patch_hybrid_gemm(pk, x.cuda())
+    torch.cuda.synchronize()
+    ref = oracle_mask(oracle_mod, w, xc, 64, 64, tmap=tmap.numpy().view(np.uint32))
+    assert np.array_equal(u32(r["meta"]), ref["meta"])
+    assert np.array_equal(r["colsq"].cpu().numpy(), ref["colsq"])
+    weff = oracle_mod.weff(bf16_bits(w), ref["meta"], ref["map"], 64, 64)
+    yref = oracle_mod.gemm(bf16_bits(x), weff)
+    rel_rms_check(y32, yref, True)
+    rel_rms_check(y16, yref, False)
+    # achieved sparsity: 8 of 16 tiles 2:4 -> 25%
+    w_eff = oracle_mod.bf16_bits_to_f64(weff)
+    assert abs(np.mean(w_eff == 0) - 0.25) < 1e-3
+
+
+def test_gemm_all_dense_matches_cublas(P):
+    N, K, M = 1024, 2048, 512
+    w, xc, x = make_problem(N, K, 64, M, seed=99)
+    nt = (N // 128) * (K // 128)
+    tmap = torch.zeros(((nt + 31) // 32,), dtype=torch.int32)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    ref = x.cuda().float() @ w.cuda().float().t()  # fp32 library GEMM of the same operands
+    torch.cuda.synchronize()
+    err = (y - ref).abs().max().item()
+    rms = ref.pow(2).mean().sqrt().item()
+    assert err <= 1e-2 * rms
+    pk.close()
+
+
+def test_gemm_empty_batch(P, oracle_mod):
+    w, xc, x = make_problem(256, 256, 64, 4, seed=5)
+    nt = 4
+    tmap = inputs.random_map(nt, 2, seed=5)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    y = P.patch_hybrid_gemm(pk, x.cuda()[:0])
+    assert y.shape == (0, 256)
+    pk.close()
+
+
+@pytest.mark.parametrize("N", [4096, 11008])
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_gemm_decode_config_full(P, oracle_mod, N, M):
+    # Llama-7B decode shapes, map by least Wanda tile loss at f = 0.5
+    K = 4096
+    seed = inputs.BASE_SEED + 1
+    w = inputs.weight(N, K, seed + N)
+    o = inputs.outlier_channels(K, seed)
+    xc = inputs.activations(2048, K, seed, o, role=0)
+    x = inputs.activations(M, K, seed, o, role=1 + M)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), fraction=0.5)
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    y16 = P.patch_hybrid_gemm(pk, x.cuda())
+    y32 = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), u32(r["map"]), 128, 128)
+    yref = oracle_mod.gemm(bf16_bits(x), weff)
+    rel_rms_check(y32, yref, True)
+    rel_rms_check(y16, yref, False)
+    pk.close()
+
+
+@pytest.mark.parametrize("N,K", [(11008, 4096), (4096, 11008)])
+@pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
+def test_gemm_prefill_config_sampled(P, oracle_mod, N, K, frac):
+    # Llama-7B prefill shapes at M = 2048, seeded random maps; sampled outputs
+    run_case(P, oracle_mod, N, K, 2048, 128, 128, frac, seed=N + int(frac * 4),
+             fp32_mode=False, sample=4000)
