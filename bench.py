@@ -320,7 +320,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b-decode")
     ap.add_argument("--no-extras", action="store_true", help="skip isolated GEMM / oracle legs")
+    ap.add_argument("--case", choices=["gemm", "mask", "pack"], default=None,
+                    help="run one operation a few times and exit (profiling aid, no JSON)")
+    ap.add_argument("--N", type=int, default=11008)
+    ap.add_argument("--K", type=int, default=4096)
+    ap.add_argument("--M", type=int, default=2048)
+    ap.add_argument("--frac", type=float, default=0.5)
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
+    if args.case:
+        return run_case(args)
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -550,6 +559,36 @@ def gpu_launches(wl, mats):
         for M in wl.tokens:
             n += 2 if M <= 16 else 1  # GEMM (+ split-K reduce)
     return n
+
+
+def run_case(args):
+    """One operation on seeded inputs, `reps` times (for profiler captures)."""
+    from sparse_gemm_wanda_b200 import patch as P
+    torch.cuda.set_device(0)
+    P.load_library()
+    g = torch.Generator().manual_seed(4242)
+    W = (torch.randn(args.N, args.K, generator=g) * 0.02).to(torch.bfloat16).cuda()
+    X = torch.randn(args.M, args.K, generator=g).to(torch.bfloat16).cuda()
+    Xcal = torch.randn(2048, args.K, generator=g).to(torch.bfloat16).cuda()
+    nt = (args.N // 128) * (args.K // 128)
+    tmap = inputs.random_map(nt, int(round(args.frac * nt)), 7).cuda()
+    if args.case == "mask":
+        for _ in range(args.reps):
+            P.patch_score_mask(W, Xcal, fraction=args.frac)
+    else:
+        r = P.patch_score_mask(W, Xcal, map_in=tmap)
+        if args.case == "pack":
+            for _ in range(args.reps):
+                P.patch_pack(W, r["meta"], r["map"]).close()
+        else:
+            pk = P.patch_pack(W, r["meta"], r["map"])
+            for _ in range(args.reps):
+                P.patch_hybrid_gemm(pk, X)
+            torch.cuda.synchronize()
+            assert P.patch_get_status(pk) == 0
+            pk.close()
+    torch.cuda.synchronize()
+    print(f"case {args.case} N={args.N} K={args.K} M={args.M} frac={args.frac} ok")
 
 
 def main_reference(args, wl, world, rank):

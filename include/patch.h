@@ -112,8 +112,6 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
  *
  *   W_bf16  [N,K] bf16 (16-byte aligned); meta, map as produced above.
  *   shp     as above, and additionally N % 128 == 0 and K % 128 == 0.
- *   max_decode_m  largest M (1..16) the handle will run through the split-K
- *           decode path; sizes the handle's fp32 split-K workspace.  0 = 16.
  *   out     receives the new handle (host pointer to a library object).
  *   packed_bytes  optional host pointer: compressed weight bytes (values +
  *           metadata, excluding the k-step table).
@@ -147,8 +145,8 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
  * Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA.
  */
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
-                        patch_shape shp, int32_t max_decode_m, patch_packed **out,
-                        size_t *packed_bytes, void *stream);
+                        patch_shape shp, patch_packed **out, size_t *packed_bytes,
+                        void *stream);
 
 /*
  * Hybrid product Y[M,N] = X[M,K] * W_eff^T with fp32 accumulation in tensor
@@ -165,10 +163,14 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
  *   Y       [M,N]: bf16 (y_is_fp32 = 0) or fp32 (y_is_fp32 = 1), 16-byte
  *           aligned.
  *
- * Every device wait inside the kernel is bounded; a wait that runs out sets
- * the handle's status word and the kernel returns early (Y undefined).
+ * Every device wait inside the kernel is bounded (2 s); a wait that runs out
+ * sets the handle's status word and the kernel returns early (Y undefined);
+ * while the word is set, later calls on the handle skip their work.
  * Errors: INVALID_ARG, CUDA; PATCH_ERR_TIMEOUT is reported by
  * patch_get_status, not here (the call does not synchronise).
+ * Test hook: with the environment variable PATCH_B200_TEST_STALL=1 the first
+ * CTA never loads its first k-step, which makes that wait run out on purpose
+ * (the failure-detection test); leave it unset in normal use.
  */
 patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
                                int32_t y_is_fp32, void *stream);
@@ -177,7 +179,7 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
 void patch_free(patch_packed *Wp, void *stream);
 
 /*
- * Read the handle's device status word (synchronises the device).
+ * Read and clear the handle's device status word (synchronises the device).
  * PATCH_OK, PATCH_ERR_TIMEOUT (a bounded wait ran out in an earlier
  * patch_hybrid_gemm), or PATCH_ERR_CUDA / INVALID_ARG.
  */

@@ -4,23 +4,31 @@
 // (inference and deployment): dense tiles run on the dense tensor-core path,
 // 2:4 tiles on the sparse one, inside one kernel over the mixed tiles.  The
 // page's kernels came from a Triton autotuner on Ampere-class GPUs; this is a
-// hand-written Blackwell design:
+// hand-written Blackwell design.
 //
-//   * one CTA = one 128-row band of W x one tile of BN tokens (x one split-K
-//     slice for decode).  D^T[128 x BN] lives in tensor memory (fp32).
-//   * warp 0 (one thread): producer.  Per 64-column k-step it reads the
-//     k-step's table entry and moves the packed weights with ONE bulk copy
-//     (16 KB dense, or 8 KB kept values + the 2 KB metadata block of the pair
-//     when it starts there) and the activations X with one TMA tensor load
-//     (128-byte swizzle), all completing on the stage's mbarrier.
-//   * warp 1 (one thread): MMA issuer.  Dense k-step: 4 x tcgen05.mma
+// Work.  An output tile is one 128-row band of W x BN tokens; D^T[128 x BN]
+// accumulates in tensor memory (fp32).  CTAs are persistent.  Two schedules:
+//   * whole tiles: tile c, c + P, c + 2P, ... (many tiles per CTA);
+//   * stream-K: the (tile, k-pair) units are cut into P contiguous, equal
+//     ranges, one per CTA.  A tile covered by several CTAs leaves fp32
+//     partials; the last of its CTAs to finish (an atomic ticket) adds them in
+//     CTA order and stores Y, so the result does not depend on timing.
+//     No CTA ever waits for another.
+//
+// Roles (192 threads):
+//   * warp 0, one thread: producer.  Per 64-column k-step it reads the table
+//     entry and moves the packed weights with ONE bulk copy (16 KB dense, or
+//     8 KB kept values, plus the 2 KB metadata block where a pair starts) and
+//     the activations X with one TMA tensor load (128-byte swizzle), all
+//     completing on the stage's mbarrier.
+//   * warp 1, one thread: MMA issuer.  Dense k-step: 4 x tcgen05.mma kind::f16
 //     (M128 N=BN K16).  2:4 k-step: tcgen05.cp of the metadata block into 4
 //     TMEM columns when the pair starts, then 2 x tcgen05.mma.sp (M128 N=BN
-//     K32).  Both accumulate into the same TMEM accumulator.  tcgen05.commit
-//     frees the stage.
-//   * warps 2..5: epilogue.  tcgen05.ld of the accumulator (each warp its
-//     32-lane quarter), one rounding to bf16 (or fp32 out), stores to Y, or
-//     fp32 split-K partials that a second kernel adds in slice order.
+//     K32).  Both accumulate into the same accumulator; two accumulators
+//     alternate between consecutive tiles so the epilogue of one overlaps the
+//     main loop of the next.
+//   * warps 2..5: epilogue.  tcgen05.ld (each warp its 32-lane quarter), one
+//     rounding to bf16 (or fp32 out), stores to Y, or partials.
 //
 // Every mbarrier wait is bounded by %globaltimer; when one runs out the CTA
 // raises the status word, drains its copies in flight and returns.
@@ -29,6 +37,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "patch_common.cuh"
@@ -45,25 +54,79 @@ struct GemmCfg {
     static constexpr int kBBytes = BN * kStep * 2;   // BN tokens x 64 columns
     static constexpr int kEBytes = kMetaBlockBytes;
     static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
-    static constexpr int kTmemCols = (BN + 4 <= 32) ? 32 : (BN + 4 <= 64) ? 64
-                                     : (BN + 4 <= 128) ? 128 : (BN + 4 <= 256) ? 256 : 512;
-    static constexpr int kEcol = BN;  // metadata columns follow the accumulator
-    static constexpr int kBarBytes = 8 * (2 * STAGES + 1) + 16;
+    static constexpr int kCols = 2 * BN + 4;         // two accumulators + metadata
+    static constexpr int kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128
+                                     : kCols <= 256 ? 256 : 512;
+    static constexpr int kEcol = 2 * BN;
+    static constexpr int kBarBytes = 8 * (2 * STAGES + 4) + 32;
     static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 + kBarBytes;
     static_assert(kBBytes % 1024 == 0, "stage regions must stay 1024-B aligned");
+    static_assert(kCols <= 512, "tensor memory holds 512 columns");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128");
 };
 
 struct GemmParams {
     const uint8_t *packed;
     const uint64_t *table;
     int64_t N, K, M;
-    int nsteps;            // K / 64
-    int steps_per_split;   // even, so a split never starts inside a k-pair
+    int nsteps;      // K / 64
+    int bands;       // N / 128
+    int ttiles;      // ceil(M / BN)
+    int stream_k;    // 0: whole tiles, 1: stream-K units
+    int64_t units;   // stream-K: tiles * pairs
     void *Y;
     int y_fp32;
-    float *partial;        // [splits][M][N] when gridDim.z > 1
+    float *partial;  // stream-K: [2 * gridDim.x][BN][128]
+    int *tickets;    // stream-K: one per (tile, 32-row quarter), zero between calls
     uint32_t *status;
+    int stall_first_kstep;  // failure-detection test hook: CTA 0 never loads its first k-step
 };
+
+// One piece of work of a CTA: k-steps [ks0, ks1) of tile (band, ttile).
+struct Segment {
+    int tile, band, ttile, ks0, ks1;
+    int nsegs;   // CTAs sharing the tile (1 = store Y directly)
+    int slot;    // partial slot of this CTA for this tile
+};
+
+__device__ __forceinline__ int64_t sk_u0(int64_t c, int64_t units, int64_t P) {
+    return (c * units) / P;
+}
+// CTA whose unit range holds unit x: the largest c with floor(c*U/P) <= x.
+__device__ __forceinline__ int64_t sk_cta_of(int64_t x, int64_t units, int64_t P) {
+    return ((x + 1) * P - 1) / units;
+}
+
+__device__ __forceinline__ bool get_segment(const GemmParams &p, int c, int i, Segment &s) {
+    const int P = gridDim.x;
+    const int tiles = p.bands * p.ttiles;
+    if (!p.stream_k) {
+        const int64_t t = static_cast<int64_t>(c) + static_cast<int64_t>(i) * P;
+        if (t >= tiles) return false;
+        s.tile = static_cast<int>(t);
+        s.ks0 = 0;
+        s.ks1 = p.nsteps;
+        s.nsegs = 1;
+        s.slot = -1;
+    } else {
+        const int Q = p.nsteps / 2;
+        const int64_t u0 = sk_u0(c, p.units, P), u1 = sk_u0(c + 1, p.units, P);
+        if (u0 >= u1) return false;
+        const int64_t t0 = u0 / Q;
+        const int64_t t = t0 + i;
+        if (t * Q >= u1) return false;
+        const int64_t a = max(u0, t * Q), b = min(u1, (t + 1) * Q);
+        s.tile = static_cast<int>(t);
+        s.ks0 = static_cast<int>(2 * (a - t * Q));
+        s.ks1 = static_cast<int>(2 * (b - t * Q));
+        const int64_t cf = sk_cta_of(t * Q, p.units, P), cl = sk_cta_of((t + 1) * Q - 1, p.units, P);
+        s.nsegs = static_cast<int>(cl - cf + 1);
+        s.slot = 2 * c + (t == t0 ? 0 : 1);
+    }
+    s.band = s.tile / p.ttiles;
+    s.ttile = s.tile % p.ttiles;
+    return true;
+}
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -74,24 +137,24 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::kStageBytes);
     uint64_t *empty = full + STAGES;
-    uint64_t *accf = empty + STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accf + 1);
-    volatile uint32_t *abort_flag = tmem_slot + 1;   // raised by any role that gives up
-    volatile uint32_t *never_flag = tmem_slot + 2;   // stays 0: time-only bounded waits
+    uint64_t *acc_full = empty + STAGES;   // [2]
+    uint64_t *acc_empty = acc_full + 2;    // [2]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    volatile uint32_t *abort_flag = tmem_slot + 1;  // raised by any role that gives up
+    volatile uint32_t *never_flag = tmem_slot + 2;  // stays 0: time-only bounded waits
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int band = blockIdx.x, ttile = blockIdx.y, split = blockIdx.z;
-    const int ks_begin = split * p.steps_per_split;
-    const int ks_end = min(p.nsteps, ks_begin + p.steps_per_split);
-    const int nks = ks_end - ks_begin;
-    const uint64_t *tab = p.table + static_cast<int64_t>(band) * p.nsteps + ks_begin;
+    const int cta = blockIdx.x;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accf, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
         *never_flag = 0u;
         *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
         fence_mbar_init();
@@ -105,30 +168,36 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const bool skip = (*abort_flag != 0) || nks <= 0;
+    const bool skip = *abort_flag != 0;
 
     if (warp == 0) {
         if (lane == 0 && !skip) {
             // ------------------------------------------------------ producer
-            int issued = 0;
+            int it = 0;  // k-steps issued so far (stage ring position)
             bool ok = true;
-            for (int i = 0; i < nks; ++i) {
-                const int s = i % STAGES;
-                const uint32_t ph = (i / STAGES) & 1u;
-                if (i >= STAGES && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
-                    ok = false;
-                    break;
+            Segment sg;
+            for (int i = 0; ok && get_segment(p, cta, i, sg); ++i) {
+                const uint64_t *tab = p.table + static_cast<int64_t>(sg.band) * p.nsteps;
+                for (int ks = sg.ks0; ks < sg.ks1; ++ks, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (it >= STAGES &&
+                        !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    if (p.stall_first_kstep && cta == 0 && it == 0) continue;  // never lands
+                    const uint64_t e = tab[ks];
+                    const bool sp = (e & kEntrySparse) != 0, has_e = (e & kEntryMeta) != 0;
+                    const uint32_t a_bytes = sp ? kSparseStepBytes : kDenseStepBytes;
+                    uint8_t *st = smem + s * C::kStageBytes;
+                    const uint8_t *src = p.packed + (e & kEntryOffsetMask);
+                    mbar_arrive_expect_tx(&full[s], a_bytes + C::kBBytes + (has_e ? C::kEBytes : 0));
+                    bulk_g2s(st, src, a_bytes, &full[s]);
+                    if (has_e)
+                        bulk_g2s(st + C::kABytes + C::kBBytes, src - C::kEBytes, C::kEBytes, &full[s]);
+                    tma_load_2d(st + C::kABytes, &tmap_x, ks * kStep, sg.ttile * BN, &full[s]);
                 }
-                const uint64_t e = tab[i];
-                const bool sp = (e & kEntrySparse) != 0, has_e = (e & kEntryMeta) != 0;
-                const uint32_t a_bytes = sp ? kSparseStepBytes : kDenseStepBytes;
-                uint8_t *st = smem + s * C::kStageBytes;
-                const uint8_t *src = p.packed + (e & kEntryOffsetMask);
-                mbar_arrive_expect_tx(&full[s], a_bytes + C::kBBytes + (has_e ? C::kEBytes : 0));
-                bulk_g2s(st, src, a_bytes, &full[s]);
-                if (has_e) bulk_g2s(st + C::kABytes + C::kBBytes, src - C::kEBytes, C::kEBytes, &full[s]);
-                tma_load_2d(st + C::kABytes, &tmap_x, (ks_begin + i) * kStep, ttile * BN, &full[s]);
-                ++issued;
             }
             if (!ok) {
                 *abort_flag = 1u;
@@ -136,117 +205,170 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
             }
             // Drain: the last phase issued on every stage must have landed
             // before the CTA exits (a no-op when the MMA thread consumed all).
-            for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-                mbar_wait_bounded(&full[i % STAGES], (i / STAGES) & 1u, never_flag,
-                                  kWaitLimitNs / 4);
+            for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j) {
+                if (p.stall_first_kstep && cta == 0 && j == 0) continue;  // never issued
+                mbar_wait_bounded(&full[j % STAGES], (j / STAGES) & 1u, never_flag, kWaitLimitNs / 4);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0 && !skip) {
             // ---------------------------------------------------------- MMA
-            const uint32_t d_tmem = tmem_base;
             const uint32_t e_tmem = tmem_base + C::kEcol;
             constexpr uint32_t kIdescDense = idesc_bf16(BN, false);
+            int it = 0;
             bool ok = true;
-            for (int i = 0; i < nks; ++i) {
-                const int s = i % STAGES;
-                const uint32_t ph = (i / STAGES) & 1u;
-                if (!mbar_wait_bounded(&full[s], ph, abort_flag, kWaitLimitNs)) {
+            Segment sg;
+            for (int i = 0; ok && get_segment(p, cta, i, sg); ++i) {
+                const int buf = i & 1;
+                if (i >= 2 && !mbar_wait_bounded(&acc_empty[buf], ((i >> 1) & 1u) ^ 1u, abort_flag,
+                                                 kWaitLimitNs)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t e = tab[i];
-                uint8_t *st = smem + s * C::kStageBytes;
-                const uint32_t a_addr = smem_u32(st), b_addr = smem_u32(st + C::kABytes);
-                if (e & kEntrySparse) {
-                    if (e & kEntryMeta)
-                        tmem_cp_128x128b(e_tmem, smem_desc(smem_u32(st + C::kABytes + C::kBBytes),
-                                                           16, 128, kSwizzleNone));
-                    const uint32_t half = static_cast<uint32_t>((ks_begin + i) & 1);
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const uint64_t ad = smem_desc(a_addr + j * 32, 16, 512, kSwizzle64B);
-                        const uint64_t bd = smem_desc(b_addr + j * 64, 16, 1024, kSwizzle128B);
-                        mma_sparse(d_tmem, ad, bd, e_tmem + 2 * half, idesc_bf16(BN, true, j),
-                                   (i > 0 || j > 0) ? 1u : 0u);
+                const uint32_t d_tmem = tmem_base + buf * BN;
+                const uint64_t *tab = p.table + static_cast<int64_t>(sg.band) * p.nsteps;
+                for (int ks = sg.ks0; ks < sg.ks1; ++ks, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1u;
+                    if (!mbar_wait_bounded(&full[s], ph, abort_flag, kWaitLimitNs)) {
+                        ok = false;
+                        break;
                     }
-                } else {
+                    tc_fence_after();
+                    const uint64_t e = tab[ks];
+                    uint8_t *st = smem + s * C::kStageBytes;
+                    const uint32_t a_addr = smem_u32(st), b_addr = smem_u32(st + C::kABytes);
+                    const bool first = ks == sg.ks0;
+                    if (e & kEntrySparse) {
+                        if (e & kEntryMeta)
+                            tmem_cp_128x128b(e_tmem, smem_desc(smem_u32(st + C::kABytes + C::kBBytes),
+                                                               16, 128, kSwizzleNone));
+                        const uint32_t half = static_cast<uint32_t>(ks & 1);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint64_t ad = smem_desc(a_addr + j * 32, 16, 1024, kSwizzle128B);
-                        const uint64_t bd = smem_desc(b_addr + j * 32, 16, 1024, kSwizzle128B);
-                        mma_dense(d_tmem, ad, bd, kIdescDense, (i > 0 || j > 0) ? 1u : 0u);
+                        for (int j = 0; j < 2; ++j) {
+                            const uint64_t ad = smem_desc(a_addr + j * 32, 16, 512, kSwizzle64B);
+                            const uint64_t bd = smem_desc(b_addr + j * 64, 16, 1024, kSwizzle128B);
+                            mma_sparse(d_tmem, ad, bd, e_tmem + 2 * half, idesc_bf16(BN, true, j),
+                                       (first && j == 0) ? 0u : 1u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint64_t ad = smem_desc(a_addr + j * 32, 16, 1024, kSwizzle128B);
+                            const uint64_t bd = smem_desc(b_addr + j * 32, 16, 1024, kSwizzle128B);
+                            mma_dense(d_tmem, ad, bd, kIdescDense, (first && j == 0) ? 0u : 1u);
+                        }
                     }
+                    tc_commit(&empty[s]);
                 }
-                tc_commit(&empty[s]);
+                // fires once every MMA of this tile has completed (also after a
+                // failure, so the epilogue never deallocates under a running MMA)
+                tc_commit(&acc_full[buf]);
             }
             if (!ok) {
                 *abort_flag = 1u;
                 atomicOr(p.status, kStatusTimeout);
             }
-            tc_commit(accf);  // fires once every MMA issued above has completed
         }
     } else if (!skip) {
         // ------------------------------------------------------- epilogue
-        // The MMA thread always commits accf, also when it gave up, so this
-        // wait is bounded by time only: no MMA may be in flight at dealloc.
-        const bool ok = mbar_wait_bounded(accf, 0u, never_flag, kWaitLimitNs);
-        tc_fence_after();
-        if (!ok) {
-            *abort_flag = 1u;
-            atomicOr(p.status, kStatusTimeout);
-        } else if (*abort_flag == 0) {
-            const int quad = warp % 4;  // TMEM lanes 32*quad .. 32*quad+31
-            const int64_t n = static_cast<int64_t>(band) * kBand + quad * 32 + lane;
-            const int64_t m_base = static_cast<int64_t>(ttile) * BN;
+        const int quad = warp % 4;  // TMEM lanes 32*quad .. 32*quad+31
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+        Segment sg;
+        for (int i = 0; get_segment(p, cta, i, sg); ++i) {
+            const int buf = i & 1;
+            // bounded by time only: the MMA thread commits acc_full even when
+            // it gave up, so no MMA can be in flight at deallocation
+            const bool ok = mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1u, never_flag, kWaitLimitNs);
+            tc_fence_after();
+            if (!ok) {
+                *abort_flag = 1u;
+                atomicOr(p.status, kStatusTimeout);
+                break;
+            }
+            const bool live = *abort_flag == 0;
+            const int64_t n = static_cast<int64_t>(sg.band) * kBand + row;
+            const int64_t m_base = static_cast<int64_t>(sg.ttile) * BN;
+            const int m_valid = static_cast<int>(min(static_cast<int64_t>(BN), p.M - m_base));
+            float *part = (sg.nsegs > 1) ? p.partial + static_cast<int64_t>(sg.slot) * BN * kBand
+                                         : nullptr;
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 16) {
                 uint32_t r[16];
-                tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c0, r);
+                tmem_ld_32x32b_x16(lane_base + buf * BN + c0, r);
                 tmem_ld_wait();
-                if (gridDim.z > 1) {
-                    float *dst = p.partial + static_cast<int64_t>(split) * p.M * p.N;
+                if (!live) continue;
+                if (part) {
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int64_t m = m_base + c0 + q;
-                        if (m < p.M) dst[m * p.N + n] = __uint_as_float(r[q]);
-                    }
+                    for (int q = 0; q < 16; ++q)
+                        if (c0 + q < m_valid) part[(c0 + q) * kBand + row] = __uint_as_float(r[q]);
                 } else if (p.y_fp32) {
                     float *y = static_cast<float *>(p.Y);
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int64_t m = m_base + c0 + q;
-                        if (m < p.M) y[m * p.N + n] = __uint_as_float(r[q]);
-                    }
+                    for (int q = 0; q < 16; ++q)
+                        if (c0 + q < m_valid) y[(m_base + c0 + q) * p.N + n] = __uint_as_float(r[q]);
                 } else {
                     __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(p.Y);
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int64_t m = m_base + c0 + q;
-                        if (m < p.M) y[m * p.N + n] = __float2bfloat16_rn(__uint_as_float(r[q]));
-                    }
+                    for (int q = 0; q < 16; ++q)
+                        if (c0 + q < m_valid)
+                            y[(m_base + c0 + q) * p.N + n] = __float2bfloat16_rn(__uint_as_float(r[q]));
                 }
             }
+            // the accumulator may be reused as soon as every lane has read it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (!part) continue;
+
+            // Stream-K fix-up, per warp (each warp owns 32 rows of the tile, so
+            // no barrier between warps is needed): the last CTA to finish this
+            // tile's quarter adds the partials of all its CTAs in CTA order and
+            // stores Y.
+            __threadfence();
+            __syncwarp();
+            int ticket = 0;
+            if (lane == 0) ticket = atomicAdd(p.tickets + sg.tile * 4 + quad, 1);
+            ticket = __shfl_sync(0xFFFFFFFFu, ticket, 0);
+            if (ticket != sg.nsegs - 1) continue;
+            __threadfence();
+            const int Q = p.nsteps / 2;
+            const int64_t P = gridDim.x;
+            const int64_t t = sg.tile;
+            const int64_t cf = sk_cta_of(t * Q, p.units, P);
+            for (int c0 = 0; c0 < m_valid; c0 += 16) {
+                float acc[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) acc[q] = 0.0f;
+                for (int64_t cc = cf; cc < cf + sg.nsegs; ++cc) {
+                    const int64_t t0 = sk_u0(cc, p.units, P) / Q;
+                    const int64_t slot = 2 * cc + (t == t0 ? 0 : 1);
+                    const float *src = p.partial + slot * BN * kBand;
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        if (c0 + q < m_valid)
+                            acc[q] = __fadd_rn(acc[q], __ldcg(src + (c0 + q) * kBand + row));
+                }
+                if (!live) continue;
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    if (c0 + q >= m_valid) continue;
+                    const int64_t yi = (m_base + c0 + q) * p.N + n;
+                    if (p.y_fp32)
+                        static_cast<float *>(p.Y)[yi] = acc[q];
+                    else
+                        static_cast<__nv_bfloat16 *>(p.Y)[yi] = __float2bfloat16_rn(acc[q]);
+                }
+            }
+            if (lane == 0) p.tickets[sg.tile * 4 + quad] = 0;  // ready for the next call
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
-}
-
-// Y[m,n] = sum over split slices s (in order) of partial[s][m][n].
-__global__ void splitk_reduce_kernel(const float *__restrict__ partial, int splits, int64_t M,
-                                     int64_t N, void *Y, int y_fp32) {
-    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t total = M * N;
-    if (idx >= total) return;
-    float acc = 0.0f;
-    for (int s = 0; s < splits; ++s) acc = __fadd_rn(acc, __ldg(partial + s * total + idx));
-    if (y_fp32)
-        static_cast<float *>(Y)[idx] = acc;
-    else
-        static_cast<__nv_bfloat16 *>(Y)[idx] = __float2bfloat16_rn(acc);
 }
 
 // ------------------------------------------------------------------- host
@@ -287,7 +409,7 @@ bool make_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K, int bn) {
 }
 
 template <int BN, int STAGES>
-cudaError_t run(const GemmLaunch &g, int splits, int steps_per_split, cudaStream_t stream) {
+cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     using C = GemmCfg<BN, STAGES>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -305,50 +427,54 @@ cudaError_t run(const GemmLaunch &g, int splits, int steps_per_split, cudaStream
     p.K = g.K;
     p.M = g.M;
     p.nsteps = static_cast<int>(g.K / kStep);
-    p.steps_per_split = steps_per_split;
+    p.bands = static_cast<int>(g.N / kBand);
+    p.ttiles = static_cast<int>((g.M + BN - 1) / BN);
     p.Y = g.Y;
     p.y_fp32 = g.y_fp32;
-    p.partial = splits > 1 ? g.workspace : nullptr;
     p.status = g.status;
-    dim3 grid(static_cast<unsigned>(g.N / kBand), static_cast<unsigned>((g.M + BN - 1) / BN),
-              static_cast<unsigned>(splits));
-    hybrid_gemm_kernel<BN, STAGES><<<grid, kGemmThreads, C::kSmemBytes, stream>>>(map, p);
+    p.tickets = g.tickets;
+    p.stall_first_kstep = g.stall_first_kstep;
+    const int64_t tiles = static_cast<int64_t>(p.bands) * p.ttiles;
+    const int64_t slots = static_cast<int64_t>(g.num_sms) * ctas_per_sm;
+    // whole tiles when there are at least two waves of them (or no room for
+    // the stream-K tickets), stream-K otherwise
+    const bool sk = tiles < 2 * slots && tiles <= g.max_tickets && g.tickets != nullptr;
+    p.stream_k = sk ? 1 : 0;
+    p.units = tiles * (p.nsteps / 2);
+    const int64_t grid = sk ? std::min<int64_t>(slots, p.units) : std::min<int64_t>(slots, tiles);
+    float *ws = nullptr;
+    if (sk) {
+        const size_t bytes = sizeof(float) * static_cast<size_t>(2 * grid) * BN * kBand;
+        if (g.workspace && bytes <= g.workspace_bytes) {
+            ws = g.workspace;
+        } else {
+            cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), bytes, g.pool, stream);
+            if (e != cudaSuccess) return e;
+        }
+    }
+    p.partial = ws;
+    hybrid_gemm_kernel<BN, STAGES>
+        <<<static_cast<unsigned>(grid), kGemmThreads, C::kSmemBytes, stream>>>(map, p);
     cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess || splits == 1) return err;
-    const int64_t total = g.M * g.N;
-    splitk_reduce_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
-        g.workspace, splits, g.M, g.N, g.Y, g.y_fp32);
-    return cudaGetLastError();
+    if (ws && ws != g.workspace) {
+        cudaError_t e2 = cudaFreeAsync(ws, stream);
+        if (err == cudaSuccess) err = e2;
+    }
+    return err;
 }
 
 }  // namespace
 
-int decode_splits(int64_t N, int64_t K, int num_sms) {
-    const int64_t bands = N / kBand;
-    const int64_t pairs = K / (2 * kStep);
-    // aim at two resident CTAs per SM
-    int64_t s = (2 * static_cast<int64_t>(num_sms) + bands - 1) / bands;
-    if (s > pairs) s = pairs;
-    if (s > 16) s = 16;
-    if (s < 1) s = 1;
-    // balance: slices of ceil(pairs / s) pairs, drop empty trailing slices
-    const int64_t per = (pairs + s - 1) / s;
-    return static_cast<int>((pairs + per - 1) / per);
+size_t decode_workspace_bytes(int num_sms) {
+    // stream-K partials of the M <= 16 configuration: 2 slots per CTA, two CTAs per SM
+    return sizeof(float) * static_cast<size_t>(2 * 2 * num_sms) * 16 * kBand;
 }
 
 cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
-    const int nsteps = static_cast<int>(g.K / kStep);
-    if (g.M <= 16 && g.workspace != nullptr) {
-        int splits = decode_splits(g.N, g.K, g.num_sms);
-        const int pairs = nsteps / 2;
-        const int per_pairs = (pairs + splits - 1) / splits;
-        if (static_cast<int64_t>(splits) * g.M * g.N > g.workspace_floats) splits = 1;
-        const int steps = splits > 1 ? 2 * per_pairs : nsteps;
-        return run<16, 5>(g, splits, steps, stream);
-    }
-    if (g.M <= 64) return run<64, 6>(g, 1, nsteps, stream);
-    if (g.M <= 128) return run<128, 6>(g, 1, nsteps, stream);
-    return run<256, 4>(g, 1, nsteps, stream);
+    if (g.M <= 16) return run<16, 4>(g, 2, stream);
+    if (g.M <= 64) return run<64, 8>(g, 1, stream);
+    if (g.M <= 128) return run<128, 6>(g, 1, stream);
+    return run<240, 4>(g, 1, stream);
 }
 
 }  // namespace patchk

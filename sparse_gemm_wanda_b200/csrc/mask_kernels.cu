@@ -202,7 +202,7 @@ score_mask_kernel(const uint16_t *__restrict__ W, const double *__restrict__ nor
 
 // ------------------------------------------------------------- tile ranking
 constexpr int kRankThreads = 128;
-constexpr int kRankSlice = 1024;
+constexpr int kRankSlice = 256;
 
 // rank[t] += #{u in this block's slice : (L_u, u) < (L_t, t)}.  Integer
 // counts, so the accumulated rank does not depend on the order of atomics.

@@ -4,8 +4,11 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
+#include <map>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -21,11 +24,13 @@ struct patch_packed {
     uint64_t *table;           // (N/128) * (K/64) entries
     int64_t sparse_ksteps;
     int64_t meta_blocks;
-    float *workspace;          // split-K partials for the decode configuration
-    int64_t workspace_floats;
-    int32_t max_decode_m;
+    float *workspace;          // stream-K partials of the M <= 16 configuration
+    size_t workspace_bytes;
+    int *tickets;              // stream-K tickets (4 per tile), zero between calls
+    int max_tickets;           // tiles covered by `tickets`
     uint32_t *status;          // device status word
     int num_sms;
+    cudaMemPool_t pool;
 };
 
 namespace {
@@ -68,7 +73,40 @@ patch_status from_cuda(cudaError_t e) {
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+constexpr int kMaxTicketTiles = 1024;
+
 }  // namespace
+
+namespace patchk {
+
+cudaError_t device_pool(cudaMemPool_t *pool) {
+    static std::mutex mu;
+    static std::map<int, cudaMemPool_t> pools;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = pools.find(dev);
+    if (it != pools.end()) {
+        *pool = it->second;
+        return cudaSuccess;
+    }
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    e = cudaMemPoolCreate(&p, &props);
+    if (e != cudaSuccess) return e;
+    uint64_t keep = UINT64_MAX;  // keep freed blocks cached across synchronisations
+    e = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) return e;
+    pools[dev] = p;
+    *pool = p;
+    return cudaSuccess;
+}
+
+}  // namespace patchk
 
 extern "C" {
 
@@ -109,8 +147,11 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
     size_t off_loss = round_up(off_norm + sizeof(double) * K, 256);
     size_t off_rank = round_up(off_loss + (tile_loss_out ? 0 : sizeof(double) * n_tiles), 256);
     size_t total = round_up(off_rank + (map_in ? 0 : sizeof(int32_t) * n_tiles), 256);
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = patchk::device_pool(&pool);
+    if (e != cudaSuccess) return from_cuda(e);
     uint8_t *scratch = nullptr;
-    cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&scratch), total, stream);
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&scratch), total, pool, stream);
     if (e != cudaSuccess) return from_cuda(e);
     double *partial = reinterpret_cast<double *>(scratch + off_partial);
     double *norm = reinterpret_cast<double *>(scratch + off_norm);
@@ -139,7 +180,7 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
 }
 
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
-                        patch_shape shp, int32_t max_decode_m, patch_packed **out,
+                        patch_shape shp, patch_packed **out,
                         size_t *packed_bytes, void *stream_v) {
     if (!out) return PATCH_ERR_INVALID_ARG;
     *out = nullptr;
@@ -147,8 +188,6 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     if (st != PATCH_OK) return st;
     if (shp.N % kBand != 0 || shp.K % (2 * kStep) != 0) return PATCH_ERR_INVALID_ARG;
     if (!W_bf16 || !meta || !map || !aligned16(W_bf16)) return PATCH_ERR_INVALID_ARG;
-    if (max_decode_m < 0 || max_decode_m > 16) return PATCH_ERR_INVALID_ARG;
-    if (max_decode_m == 0) max_decode_m = 16;
     int num_sms = 0;
     st = check_device(&num_sms);
     if (st != PATCH_OK) return st;
@@ -205,19 +244,21 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     h->packed_bytes = static_cast<size_t>(offset);
     h->sparse_ksteps = n_sparse;
     h->meta_blocks = n_meta;
-    h->max_decode_m = max_decode_m;
     h->num_sms = num_sms;
-    const int splits = patchk::decode_splits(N, K, num_sms);
-    h->workspace_floats = static_cast<int64_t>(splits) * max_decode_m * N;
+    h->workspace_bytes = patchk::decode_workspace_bytes(num_sms);
+    h->max_tickets = kMaxTicketTiles;
 
-    e = cudaMallocAsync(reinterpret_cast<void **>(&h->packed), h->packed_bytes ? h->packed_bytes : 16, stream);
+    e = patchk::device_pool(&h->pool);
+    auto alloc = [&](void **ptr, size_t bytes) {
+        if (e == cudaSuccess) e = cudaMallocFromPoolAsync(ptr, bytes, h->pool, stream);
+    };
+    alloc(reinterpret_cast<void **>(&h->packed), h->packed_bytes ? h->packed_bytes : 16);
+    alloc(reinterpret_cast<void **>(&h->table), sizeof(uint64_t) * table.size());
+    alloc(reinterpret_cast<void **>(&h->workspace), h->workspace_bytes);
+    alloc(reinterpret_cast<void **>(&h->tickets), sizeof(int) * 4 * kMaxTicketTiles);
+    alloc(reinterpret_cast<void **>(&h->status), sizeof(uint32_t) * 4);
     if (e == cudaSuccess)
-        e = cudaMallocAsync(reinterpret_cast<void **>(&h->table), sizeof(uint64_t) * table.size(), stream);
-    if (e == cudaSuccess)
-        e = cudaMallocAsync(reinterpret_cast<void **>(&h->workspace),
-                            sizeof(float) * static_cast<size_t>(h->workspace_floats), stream);
-    if (e == cudaSuccess)
-        e = cudaMallocAsync(reinterpret_cast<void **>(&h->status), sizeof(uint32_t) * 4, stream);
+        e = cudaMemsetAsync(h->tickets, 0, sizeof(int) * 4 * kMaxTicketTiles, stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(h->status, 0, sizeof(uint32_t) * 4, stream);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(h->table, table.data(), sizeof(uint64_t) * table.size(),
@@ -251,10 +292,18 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.M = M;
     g.Y = Y;
     g.y_fp32 = y_is_fp32;
-    g.workspace = (M <= Wp->max_decode_m) ? Wp->workspace : nullptr;
-    g.workspace_floats = Wp->workspace_floats;
+    g.workspace = Wp->workspace;
+    g.workspace_bytes = Wp->workspace_bytes;
+    g.tickets = Wp->tickets;
+    g.max_tickets = Wp->max_tickets;
+    g.pool = Wp->pool;
     g.status = Wp->status;
     g.num_sms = Wp->num_sms;
+    // Failure-detection test hook: with PATCH_B200_TEST_STALL=1 in the
+    // environment, CTA 0 never loads its first k-step, so its bounded wait runs
+    // out, the kernel returns early and patch_get_status reports the timeout.
+    const char *stall = getenv("PATCH_B200_TEST_STALL");
+    g.stall_first_kstep = (stall && stall[0] == '1') ? 1 : 0;
     return from_cuda(patchk::launch_hybrid_gemm(g, static_cast<cudaStream_t>(stream_v)));
 }
 
@@ -264,6 +313,7 @@ void patch_free(patch_packed *Wp, void *stream_v) {
     if (Wp->packed) cudaFreeAsync(Wp->packed, stream);
     if (Wp->table) cudaFreeAsync(Wp->table, stream);
     if (Wp->workspace) cudaFreeAsync(Wp->workspace, stream);
+    if (Wp->tickets) cudaFreeAsync(Wp->tickets, stream);
     if (Wp->status) cudaFreeAsync(Wp->status, stream);
     delete Wp;
 }
@@ -273,6 +323,7 @@ patch_status patch_get_status(const patch_packed *Wp) {
     uint32_t word = 0;
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess) e = cudaMemcpy(&word, Wp->status, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && word != 0) e = cudaMemset(Wp->status, 0, sizeof(uint32_t));
     if (e != cudaSuccess) return from_cuda(e);
     return (word & patchk::kStatusTimeout) ? PATCH_ERR_TIMEOUT : PATCH_OK;
 }

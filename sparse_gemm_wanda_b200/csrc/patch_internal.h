@@ -27,17 +27,24 @@ struct GemmLaunch {
     int64_t M;
     void *Y;
     int y_fp32;
-    float *workspace;         // split-K partials [splits][M][N] (fp32)
-    int64_t workspace_floats; // capacity of `workspace`
+    float *workspace;        // stream-K partials owned by the handle (may be null)
+    size_t workspace_bytes;  // capacity of `workspace`
+    int *tickets;            // stream-K tickets, 4 per tile, zero between calls
+    int max_tickets;         // tiles the ticket array covers
+    cudaMemPool_t pool;      // for larger stream-K partials
     uint32_t *status;
     int num_sms;
+    int stall_first_kstep;   // failure-detection test hook (see patch_hybrid_gemm)
 };
 
-// Picks the configuration (token tile, split-K) for M and launches.
+// Picks the configuration (token tile, schedule) for M and launches.
 cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream);
 
-// Number of split-K slices the decode configuration uses for N rows and K
-// columns (k-pairs per slice are balanced; always >= 1).
-int decode_splits(int64_t N, int64_t K, int num_sms);
+// Bytes of stream-K partials the M <= 16 configuration needs at most.
+size_t decode_workspace_bytes(int num_sms);
+
+// The library's stream-ordered memory pool for the current device (cached
+// memory is kept, not returned to the system between calls).
+cudaError_t device_pool(cudaMemPool_t *pool);
 
 }  // namespace patchk

@@ -64,7 +64,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         raise PatchLibraryError(f"cannot load {path}: {exc}") from exc
     vp, i64, i32, dbl = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double
     lib.patch_score_mask.argtypes = [vp, vp, i64, vp, PatchShape, dbl, vp, vp, vp, vp, vp, vp]
-    lib.patch_pack.argtypes = [vp, vp, vp, PatchShape, i32, ctypes.POINTER(vp),
+    lib.patch_pack.argtypes = [vp, vp, vp, PatchShape, ctypes.POINTER(vp),
                                ctypes.POINTER(ctypes.c_size_t), vp]
     lib.patch_hybrid_gemm.argtypes = [vp, vp, i64, vp, i32, vp]
     lib.patch_free.argtypes = [vp, vp]
@@ -166,7 +166,7 @@ class PackedWeight:
 
 
 def patch_pack(W: torch.Tensor, meta: torch.Tensor, tile_map: torch.Tensor, *, tile_n: int = 128,
-               tile_k: int = 128, max_decode_m: int = 16, stream=None) -> PackedWeight:
+               tile_k: int = 128, stream=None) -> PackedWeight:
     """Compress W (dense tiles + 2:4 tiles) into a library-owned handle."""
     lib = load_library()
     N, K = W.shape
@@ -174,7 +174,7 @@ def patch_pack(W: torch.Tensor, meta: torch.Tensor, tile_map: torch.Tensor, *, t
     nbytes = ctypes.c_size_t(0)
     code = lib.patch_pack(_dptr(W, torch.bfloat16, "W"), _dptr(meta, (torch.int32, torch.uint32), "meta"),
                           _dptr(tile_map, (torch.int32, torch.uint32), "map"),
-                          PatchShape(N, K, tile_n, tile_k), int(max_decode_m), ctypes.byref(out),
+                          PatchShape(N, K, tile_n, tile_k), ctypes.byref(out),
                           ctypes.byref(nbytes), _stream(stream))
     _check("patch_pack", code)
     return PackedWeight(out.value, (N, K, tile_n, tile_k), nbytes.value)

@@ -79,15 +79,16 @@ def test_pack_argument_checks(lib):
     from sparse_gemm_wanda_b200.patch import PatchShape
     fake = ctypes.c_void_p(0x1000)
     out = ctypes.c_void_p(0)
-    assert lib.patch_pack(fake, fake, fake, PatchShape(256, 256, 64, 64), 16, None, None,
+    assert lib.patch_pack(fake, fake, fake, PatchShape(256, 256, 64, 64), None, None,
                           None) == 1
     # N not a multiple of 128 (64-row tiles allow N=192, the packed bands do not)
-    assert lib.patch_pack(fake, fake, fake, PatchShape(192, 256, 64, 64), 16, ctypes.byref(out),
+    assert lib.patch_pack(fake, fake, fake, PatchShape(192, 256, 64, 64), ctypes.byref(out),
                           None, None) == 1
     # K not a multiple of 128
-    assert lib.patch_pack(fake, fake, fake, PatchShape(256, 192, 64, 64), 16, ctypes.byref(out),
+    assert lib.patch_pack(fake, fake, fake, PatchShape(256, 192, 64, 64), ctypes.byref(out),
                           None, None) == 1
-    assert lib.patch_pack(fake, fake, fake, PatchShape(256, 256, 64, 64), 17, ctypes.byref(out),
+    # null map
+    assert lib.patch_pack(fake, fake, None, PatchShape(256, 256, 64, 64), ctypes.byref(out),
                           None, None) == 1
     assert out.value is None
 

@@ -261,3 +261,42 @@ def test_gemm_prefill_config_sampled(P, oracle_mod, N, K, frac):
     # Llama-7B prefill shapes at M = 2048, seeded random maps; sampled outputs
     run_case(P, oracle_mod, N, K, 2048, 128, 128, frac, seed=N + int(frac * 4),
              fp32_mode=False, sample=4000)
+
+
+def test_gemm_repeated_calls_reset_tickets(P, oracle_mod):
+    # stream-K tiles shared by several CTAs: every call must find its tickets at zero
+    N, K, M = 1024, 2048, 5
+    w, xc, _ = make_problem(N, K, 64, M, seed=31)
+    nt = (N // 128) * (K // 128)
+    tmap = inputs.random_map(nt, nt // 2, seed=31)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
+    for rep in range(3):
+        x = inputs.activations(M, K, 100 + rep, None)
+        y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+        torch.cuda.synchronize()
+        rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), weff), True)
+    assert P.patch_get_status(pk) == 0
+    pk.close()
+
+
+def test_gemm_bounded_wait_reports_timeout(P, oracle_mod, monkeypatch):
+    # Failure detection without a GPU fault: the first CTA never receives its
+    # first k-step; its bounded wait runs out, the kernel returns, the status
+    # word reports the timeout, and the handle works again once cleared.
+    N, K, M = 256, 256, 4
+    w, xc, x = make_problem(N, K, 64, M, seed=41)
+    tmap = inputs.random_map(4, 2, seed=41)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    monkeypatch.setenv("PATCH_B200_TEST_STALL", "1")
+    P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    monkeypatch.delenv("PATCH_B200_TEST_STALL")
+    assert P.patch_get_status(pk) == 5  # PATCH_ERR_TIMEOUT, read and cleared
+    assert P.patch_get_status(pk) == 0
+    y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
+    rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), weff), True)
+    pk.close()
