@@ -34,9 +34,11 @@
  *         fixed order: chunks of 128 consecutive tokens, each summed token
  *         by token from 0.0, then the chunk sums added chunk by chunk from
  *         0.0.  The result is therefore bit-reproducible.
- *   tile_loss fp64 [n_tiles]: Wanda score removed by 2:4 pruning of the tile;
- *         each row of the tile sums its pruned scores left to right, then the
- *         row sums are added top to bottom.
+ *   tile_loss fp64 [n_tiles]: Wanda score removed by 2:4 pruning of the tile,
+ *         added in a fixed order: inside each 32-column word of a row the
+ *         pruned scores left to right; the row's words left to right; the
+ *         tile's row sums as a balanced binary tree ((0,1), (2,3), ..., then
+ *         pairs of those, ...).
  */
 #ifndef PATCH_B200_H
 #define PATCH_B200_H
@@ -111,7 +113,8 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
  * unstructured sparsity); the layout is this library's own.
  *
  *   W_bf16  [N,K] bf16 (16-byte aligned); meta, map as produced above.
- *   shp     as above, and additionally N % 128 == 0 and K % 128 == 0.
+ *   shp     as above, and additionally N % 128 == 0, K % 128 == 0 and
+ *           K <= 28672.
  *   out     receives the new handle (host pointer to a library object).
  *   packed_bytes  optional host pointer: compressed weight bytes (values +
  *           metadata, excluding the k-step table).

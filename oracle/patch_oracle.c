@@ -169,24 +169,41 @@ static int kept(const uint32_t *meta, int64_t K, int64_t i, int64_t j) {
 
 /*
  * Tiles are tn x tk, numbered row-major: t = (i/tn)*(K/tk) + (j/tk).
- * loss[t] = the Wanda score that 2:4 pruning would remove from tile t:
- * every row of the tile sums its pruned scores left to right from 0.0, then
- * the row sums are added top to bottom from 0.0.
+ * loss[t] = the Wanda score that 2:4 pruning would remove from tile t, added
+ * in this fixed order (the pages fix none):
+ *   - word sum: inside each 32-column word of a row, the pruned scores are
+ *     added left to right, starting from 0.0;
+ *   - row sum: the word sums of the row's tk/32 words inside the tile are
+ *     added left to right, starting from 0.0;
+ *   - tile sum: the tn row sums are added as a balanced binary tree: row
+ *     sums (0,1), (2,3), ... are added pairwise, then those results
+ *     pairwise, and so on until one value is left (tn is a power of two).
  */
+static double word_pruned_sum(const double *score, const uint32_t *meta, int64_t K,
+                              int64_t i, int64_t j0) {
+    double w = 0.0;
+    for (int64_t j = j0; j < j0 + 32; ++j)
+        if (!kept(meta, K, i, j)) w = w + score[i * K + j];
+    return w;
+}
+
 void oracle_tile_loss(const double *score, const uint32_t *meta, int64_t N,
                       int64_t K, int64_t tn, int64_t tk, double *loss) {
     int64_t tiles_k = K / tk, tiles_n = N / tn;
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < tiles_n * tiles_k; ++t) {
         int64_t i0 = (t / tiles_k) * tn, j0 = (t % tiles_k) * tk;
-        double total = 0.0;
-        for (int64_t i = i0; i < i0 + tn; ++i) {
+        double *rows = (double *)malloc(sizeof(double) * (size_t)tn);
+        for (int64_t r = 0; r < tn; ++r) {
             double row = 0.0;
-            for (int64_t j = j0; j < j0 + tk; ++j)
-                if (!kept(meta, K, i, j)) row = row + score[i * K + j];
-            total = total + row;
+            for (int64_t w = j0; w < j0 + tk; w += 32)
+                row = row + word_pruned_sum(score, meta, K, i0 + r, w);
+            rows[r] = row;
         }
-        loss[t] = total;
+        for (int64_t n = tn; n > 1; n /= 2)
+            for (int64_t q = 0; q < n / 2; ++q) rows[q] = rows[2 * q] + rows[2 * q + 1];
+        loss[t] = rows[0];
+        free(rows);
     }
 }
 

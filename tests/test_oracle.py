@@ -201,7 +201,8 @@ def pruned_mask(codes, K):
 
 def test_tile_loss_exact_dyadic(oracle_mod):
     # dyadic scores with small magnitude: every partial sum is exact in fp64,
-    # so the loss must equal the exact rational sum of the pruned scores.
+    # so the loss must equal the exact rational sum of the pruned scores,
+    # whatever the order.
     rng = np.random.default_rng(7)
     N, K, tn, tk = 128, 192, 64, 64
     sc = rng.integers(0, 4096, size=(N, K)) / 8.0
@@ -215,6 +216,24 @@ def test_tile_loss_exact_dyadic(oracle_mod):
         assert Fraction(loss[t]) == sum(Fraction(v) for v in blk)
         # exactly half of every tile is pruned
         assert blk.size == tn * tk // 2
+
+
+def test_tile_loss_order_is_the_stated_tree(oracle_mod):
+    # Row sums chosen so that fp64 rounding depends on the order: the stated
+    # order (rows added as a balanced pairwise tree) must be the one used, not
+    # a plain top-to-bottom sum.
+    N, K, tn, tk = 4, 32, 4, 32
+    sc = np.zeros((N, K))
+    sc[:, 0::4] = 1e30        # positions 0 and 1 of every group are kept
+    sc[:, 1::4] = 1e30
+    r = [1.0, 2.0 ** 53, 1.0, 1.0]
+    sc[:, 2] = r              # the only nonzero pruned score of each row
+    meta = oracle_mod.select_2of4(sc)
+    loss = oracle_mod.tile_loss(sc, meta, tn, tk)[0]
+    tree = (r[0] + r[1]) + (r[2] + r[3])
+    top_to_bottom = ((r[0] + r[1]) + r[2]) + r[3]
+    assert tree != top_to_bottom  # 2**53 + 2 vs 2**53
+    assert loss == tree
 
 
 def test_tile_loss_plus_kept_is_total(oracle_mod):
