@@ -152,6 +152,16 @@ class CallTimer:
                 for k, v in agg.items()}
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest value over all ranks (the job's time is its slowest rank's)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------- workload
 def make_tensors(wl, rank: int, device="cpu"):
     """Synthetic weights, calibration and inputs of a workload (per-rank seed)."""
@@ -384,11 +394,7 @@ def main():
     timer.enabled = False
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in events]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), "cuda")
     ms_per_step = total_ms / args.steps
     calls = timer.summary()
 
@@ -456,11 +462,7 @@ def main():
             del hy
             if it >= args.warmup:
                 e2e_events.append(e0.elapsed_time(e1))
-        e2e_ms = sum(e2e_events) / len(e2e_events)
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(sum(e2e_events) / len(e2e_events), "cuda")
         e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 

@@ -46,23 +46,31 @@
 namespace patchk {
 
 constexpr int kGemmThreads = 192;
+// k-steps of one segment whose table entries are staged in shared memory
+// (K <= 28672)
+constexpr int kMaxTableSteps = 448;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 template <int BN, int STAGES>
 struct GemmCfg {
-    static constexpr int kABytes = kDenseStepBytes;  // room for a dense k-step
-    static constexpr int kBBytes = BN * kStep * 2;   // BN tokens x 64 columns
-    static constexpr int kEBytes = kMetaBlockBytes;
-    static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
-    static constexpr int kCols = 2 * BN + 4;         // two accumulators + metadata
+    // One stage = one k-pair (128 columns): the pair's packed weights (at most
+    // two dense k-steps, 32 KB; the metadata block travels inside) and the two
+    // 64-column X tiles.
+    static constexpr int kABytes = 2 * kDenseStepBytes;
+    static constexpr int kBTileBytes = BN * kStep * 2;  // BN tokens x 64 columns
+    static constexpr int kBBytes = 2 * kBTileBytes;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kCols = 2 * BN + 4;            // two accumulators + metadata
     static constexpr int kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128
                                      : kCols <= 256 ? 256 : 512;
     static constexpr int kEcol = 2 * BN;
-    static constexpr int kBarBytes = 8 * (2 * STAGES + 4) + 32;
-    static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 + kBarBytes;
-    static_assert(kBBytes % 1024 == 0, "stage regions must stay 1024-B aligned");
+    static constexpr int kBarBytes = 8 * (2 * STAGES + 6) + 32 + 24 * STAGES;
+    static constexpr int kTabBytes = 2 * kMaxTableSteps * 8;  // two segments of table entries
+    static constexpr int kSmemBytes = STAGES * kStageBytes + kTabBytes + 1024 + kBarBytes;
+    static_assert(kBTileBytes % 1024 == 0, "stage regions must stay 1024-B aligned");
     static_assert(kCols <= 512, "tensor memory holds 512 columns");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
 
 struct GemmParams {
@@ -77,7 +85,6 @@ struct GemmParams {
     void *Y;
     int y_fp32;
     float *partial;  // stream-K: [2 * gridDim.x][BN][128]
-    int *tickets;    // stream-K: one per (tile, 32-row quarter), zero between calls
     uint32_t *status;
     int stall_first_kstep;  // failure-detection test hook: CTA 0 never loads its first k-step
 };
@@ -135,13 +142,18 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::kStageBytes);
+    uint64_t *tab_buf = reinterpret_cast<uint64_t *>(smem + STAGES * C::kStageBytes);  // [2][kMaxTableSteps]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::kStageBytes + C::kTabBytes);
     uint64_t *empty = full + STAGES;
     uint64_t *acc_full = empty + STAGES;   // [2]
     uint64_t *acc_empty = acc_full + 2;    // [2]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *tab_full = acc_empty + 2;    // [2]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tab_full + 2);
     volatile uint32_t *abort_flag = tmem_slot + 1;  // raised by any role that gives up
     volatile uint32_t *never_flag = tmem_slot + 2;  // stays 0: time-only bounded waits
+    // per stage, written by the producer before it arms the stage: the pair's two
+    // table entries and the stream offset of its first byte
+    uint64_t *stage_info = reinterpret_cast<uint64_t *>(tmem_slot + 4);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int cta = blockIdx.x;
@@ -154,6 +166,7 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 4);
+            mbar_init(&tab_full[b], 1);
         }
         *never_flag = 0u;
         *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
@@ -173,32 +186,69 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
     if (warp == 0) {
         if (lane == 0 && !skip) {
             // ------------------------------------------------------ producer
-            int it = 0;  // k-steps issued so far (stage ring position)
+            int it = 0;  // k-pairs issued so far (stage ring position)
             bool ok = true;
-            Segment sg;
-            for (int i = 0; ok && get_segment(p, cta, i, sg); ++i) {
-                const uint64_t *tab = p.table + static_cast<int64_t>(sg.band) * p.nsteps;
-                for (int ks = sg.ks0; ks < sg.ks1; ++ks, ++it) {
+            // The table entries of a segment reach shared memory through one
+            // bulk copy issued a whole segment ahead (two buffers), so no table
+            // read waits behind the weight stream in the memory queues.
+            Segment sg, nx;
+            auto fetch_table = [&](const Segment &g, int buf) {
+                const uint32_t nbytes = static_cast<uint32_t>(g.ks1 - g.ks0) * 8u;
+                mbar_arrive_expect_tx(&tab_full[buf], nbytes);
+                bulk_g2s(tab_buf + buf * kMaxTableSteps,
+                         p.table + static_cast<int64_t>(g.band) * p.nsteps + g.ks0, nbytes, &tab_full[buf]);
+            };
+            bool have = get_segment(p, cta, 0, sg);
+            if (have) fetch_table(sg, 0);
+            bool have_nx = have && get_segment(p, cta, 1, nx);
+            if (have_nx) fetch_table(nx, 1);
+            int tabs_issued = (have ? 1 : 0) + (have_nx ? 1 : 0);
+            for (int i = 0; ok && have; ++i) {
+                const int buf = i & 1;
+                if (!mbar_wait_bounded(&tab_full[buf], (i >> 1) & 1u, abort_flag, kWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                const uint64_t *tab = tab_buf + buf * kMaxTableSteps;
+                for (int pr = sg.ks0 / 2; pr < sg.ks1 / 2; ++pr) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1u;
-                    if (it >= STAGES &&
-                        !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
+                    if (it >= STAGES && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
                         ok = false;
                         break;
                     }
-                    if (p.stall_first_kstep && cta == 0 && it == 0) continue;  // never lands
-                    const uint64_t e = tab[ks];
-                    const bool sp = (e & kEntrySparse) != 0, has_e = (e & kEntryMeta) != 0;
-                    const uint32_t a_bytes = sp ? kSparseStepBytes : kDenseStepBytes;
+                    const uint64_t c0 = tab[2 * pr - sg.ks0], c1 = tab[2 * pr + 1 - sg.ks0];
+                    const uint64_t first = (c0 & kEntryOffsetMask) - ((c0 & kEntryMeta) ? kMetaBlockBytes : 0);
+                    const uint64_t end = (c1 & kEntryOffsetMask) +
+                                         ((c1 & kEntrySparse) ? kSparseStepBytes : kDenseStepBytes);
+                    const uint32_t bytes = static_cast<uint32_t>(end - first);
+                    stage_info[3 * s + 0] = c0;
+                    stage_info[3 * s + 1] = c1;
+                    stage_info[3 * s + 2] = first;
+                    ++it;
+                    if (p.stall_first_kstep && cta == 0 && it == 1) continue;  // never lands
                     uint8_t *st = smem + s * C::kStageBytes;
-                    const uint8_t *src = p.packed + (e & kEntryOffsetMask);
-                    mbar_arrive_expect_tx(&full[s], a_bytes + C::kBBytes + (has_e ? C::kEBytes : 0));
-                    bulk_g2s(st, src, a_bytes, &full[s]);
-                    if (has_e)
-                        bulk_g2s(st + C::kABytes + C::kBBytes, src - C::kEBytes, C::kEBytes, &full[s]);
-                    tma_load_2d(st + C::kABytes, &tmap_x, ks * kStep, sg.ttile * BN, &full[s]);
+                    mbar_arrive_expect_tx(&full[s], bytes + C::kBBytes);
+                    bulk_g2s(st, p.packed + first, bytes, &full[s]);
+                    tma_load_3d(st + C::kABytes, &tmap_x, 0, sg.ttile * BN, 2 * pr, &full[s]);
+                }
+                // this buffer is free again: fetch the table of segment i + 2
+                sg = nx;
+                have = have_nx;
+                if (have) {
+                    Segment n2;
+                    have_nx = get_segment(p, cta, i + 2, n2);
+                    if (have_nx) {
+                        fetch_table(n2, buf);
+                        ++tabs_issued;
+                        nx = n2;
+                    }
                 }
             }
+            // table copies still in flight must land before the CTA exits (the
+            // latest phase of each buffer)
+            for (int j = (tabs_issued > 2 ? tabs_issued - 2 : 0); j < tabs_issued; ++j)
+                mbar_wait_bounded(&tab_full[j & 1], (j >> 1) & 1u, never_flag, kWaitLimitNs / 4);
             if (!ok) {
                 *abort_flag = 1u;
                 atomicOr(p.status, kStatusTimeout);
@@ -227,8 +277,7 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * BN;
-                const uint64_t *tab = p.table + static_cast<int64_t>(sg.band) * p.nsteps;
-                for (int ks = sg.ks0; ks < sg.ks1; ++ks, ++it) {
+                for (int pr = sg.ks0 / 2; pr < sg.ks1 / 2; ++pr, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1u;
                     if (!mbar_wait_bounded(&full[s], ph, abort_flag, kWaitLimitNs)) {
@@ -236,28 +285,33 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t e = tab[ks];
+                    const uint64_t first = stage_info[3 * s + 2];
                     uint8_t *st = smem + s * C::kStageBytes;
-                    const uint32_t a_addr = smem_u32(st), b_addr = smem_u32(st + C::kABytes);
-                    const bool first = ks == sg.ks0;
-                    if (e & kEntrySparse) {
-                        if (e & kEntryMeta)
-                            tmem_cp_128x128b(e_tmem, smem_desc(smem_u32(st + C::kABytes + C::kBBytes),
-                                                               16, 128, kSwizzleNone));
-                        const uint32_t half = static_cast<uint32_t>(ks & 1);
 #pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const uint64_t ad = smem_desc(a_addr + j * 32, 16, 512, kSwizzle64B);
-                            const uint64_t bd = smem_desc(b_addr + j * 64, 16, 1024, kSwizzle128B);
-                            mma_sparse(d_tmem, ad, bd, e_tmem + 2 * half, idesc_bf16(BN, true, j),
-                                       (first && j == 0) ? 0u : 1u);
-                        }
-                    } else {
+                    for (int h = 0; h < 2; ++h) {
+                        const uint64_t e = stage_info[3 * s + h];
+                        const uint32_t a_addr =
+                            smem_u32(st + static_cast<uint32_t>((e & kEntryOffsetMask) - first));
+                        const uint32_t b_addr = smem_u32(st + C::kABytes + h * C::kBTileBytes);
+                        const bool first_step = (pr == sg.ks0 / 2) && h == 0;
+                        if (e & kEntrySparse) {
+                            if (e & kEntryMeta)
+                                tmem_cp_128x128b(e_tmem, smem_desc(a_addr - kMetaBlockBytes, 16, 128,
+                                                                   kSwizzleNone));
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint64_t ad = smem_desc(a_addr + j * 32, 16, 1024, kSwizzle128B);
-                            const uint64_t bd = smem_desc(b_addr + j * 32, 16, 1024, kSwizzle128B);
-                            mma_dense(d_tmem, ad, bd, kIdescDense, (first && j == 0) ? 0u : 1u);
+                            for (int j = 0; j < 2; ++j) {
+                                const uint64_t ad = smem_desc(a_addr + j * 32, 16, 512, kSwizzle64B);
+                                const uint64_t bd = smem_desc(b_addr + j * 64, 16, 1024, kSwizzle128B);
+                                mma_sparse(d_tmem, ad, bd, e_tmem + 2 * h, idesc_bf16(BN, true, j),
+                                           (first_step && j == 0) ? 0u : 1u);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const uint64_t ad = smem_desc(a_addr + j * 32, 16, 1024, kSwizzle128B);
+                                const uint64_t bd = smem_desc(b_addr + j * 32, 16, 1024, kSwizzle128B);
+                                mma_dense(d_tmem, ad, bd, kIdescDense, (first_step && j == 0) ? 0u : 1u);
+                            }
                         }
                     }
                     tc_commit(&empty[s]);
@@ -321,54 +375,62 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
-            if (!part) continue;
-
-            // Stream-K fix-up, per warp (each warp owns 32 rows of the tile, so
-            // no barrier between warps is needed): the last CTA to finish this
-            // tile's quarter adds the partials of all its CTAs in CTA order and
-            // stores Y.
-            __threadfence();
-            __syncwarp();
-            int ticket = 0;
-            if (lane == 0) ticket = atomicAdd(p.tickets + sg.tile * 4 + quad, 1);
-            ticket = __shfl_sync(0xFFFFFFFFu, ticket, 0);
-            if (ticket != sg.nsegs - 1) continue;
-            __threadfence();
-            const int Q = p.nsteps / 2;
-            const int64_t P = gridDim.x;
-            const int64_t t = sg.tile;
-            const int64_t cf = sk_cta_of(t * Q, p.units, P);
-            for (int c0 = 0; c0 < m_valid; c0 += 16) {
-                float acc[16];
-#pragma unroll
-                for (int q = 0; q < 16; ++q) acc[q] = 0.0f;
-                for (int64_t cc = cf; cc < cf + sg.nsegs; ++cc) {
-                    const int64_t t0 = sk_u0(cc, p.units, P) / Q;
-                    const int64_t slot = 2 * cc + (t == t0 ? 0 : 1);
-                    const float *src = p.partial + slot * BN * kBand;
-#pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        if (c0 + q < m_valid)
-                            acc[q] = __fadd_rn(acc[q], __ldcg(src + (c0 + q) * kBand + row));
-                }
-                if (!live) continue;
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    if (c0 + q >= m_valid) continue;
-                    const int64_t yi = (m_base + c0 + q) * p.N + n;
-                    if (p.y_fp32)
-                        static_cast<float *>(p.Y)[yi] = acc[q];
-                    else
-                        static_cast<__nv_bfloat16 *>(p.Y)[yi] = __float2bfloat16_rn(acc[q]);
-                }
-            }
-            if (lane == 0) p.tickets[sg.tile * 4 + quad] = 0;  // ready for the next call
         }
     }
+    // let a dependent launch (the stream-K reduction) get scheduled
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// Stream-K fix-up: for every tile shared by several CTAs, Y = the partials of
+// its CTAs added in CTA order (fixed order: the result does not depend on
+// timing).  Launched as a programmatic dependent of the GEMM; waits for it.
+template <int BN>
+__global__ void __launch_bounds__(256)
+streamk_reduce_kernel(const float *__restrict__ partial, int64_t units, int P, int Q, int ttiles,
+                      int64_t M, int64_t N, void *Y, int y_fp32) {
+    // block (tile t, chunk): one output per thread, 256 outputs per block
+    __shared__ int slots[64];
+    __shared__ int nslots;
+    const int64_t t = blockIdx.y;
+    if (threadIdx.x == 0) {
+        const int64_t cf = sk_cta_of(t * Q, units, P), cl = sk_cta_of((t + 1) * Q - 1, units, P);
+        int n = 0;
+        if (cf != cl) {  // a tile with one CTA was stored directly
+            for (int64_t cc = cf; cc <= cl && n < 64; ++cc)
+                slots[n++] = static_cast<int>(2 * cc + ((sk_u0(cc, units, P) / Q == t) ? 0 : 1));
+        }
+        nslots = n;
+    }
+    __syncthreads();
+    const int ns = nslots;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (ns == 0) return;
+    const int band = static_cast<int>(t / ttiles), ttile = static_cast<int>(t % ttiles);
+    const int64_t m_base = static_cast<int64_t>(ttile) * BN;
+    const int m_valid = static_cast<int>(min(static_cast<int64_t>(BN), M - m_base));
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= m_valid * kBand) return;
+    const int m = e / kBand, row = e % kBand;
+    const float *src = partial + m * kBand + row;
+    float acc = 0.0f;
+    for (int j0 = 0; j0 < ns; j0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            v[q] = (j0 + q < ns) ? __ldcg(src + static_cast<int64_t>(slots[j0 + q]) * BN * kBand) : 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (j0 + q < ns) acc = __fadd_rn(acc, v[q]);
+    }
+    const int64_t yi = (m_base + m) * N + static_cast<int64_t>(band) * kBand + row;
+    if (y_fp32)
+        static_cast<float *>(Y)[yi] = acc;
+    else
+        static_cast<__nv_bfloat16 *>(Y)[yi] = __float2bfloat16_rn(acc);
 }
 
 // ------------------------------------------------------------------- host
@@ -393,16 +455,18 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// X [M,K] bf16 row-major, box = 64 columns x BN rows, 128-byte swizzle;
-// rows past M read as zero.
+// X [M,K] bf16 row-major viewed as (64 columns, M rows, K/64 k-steps); one box
+// = both 64-column tiles of a k-pair for BN rows, 128-byte swizzle; rows past
+// M read as zero.
 bool make_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K, int bn) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kStep), static_cast<cuuint32_t>(bn)};
-    const cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(X), dims, strides, box,
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kStep), static_cast<cuuint64_t>(M),
+                                static_cast<cuuint64_t>(K / kStep)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, static_cast<cuuint64_t>(kStep) * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kStep), static_cast<cuuint32_t>(bn), 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(X), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -432,16 +496,17 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     p.Y = g.Y;
     p.y_fp32 = g.y_fp32;
     p.status = g.status;
-    p.tickets = g.tickets;
     p.stall_first_kstep = g.stall_first_kstep;
     const int64_t tiles = static_cast<int64_t>(p.bands) * p.ttiles;
     const int64_t slots = static_cast<int64_t>(g.num_sms) * ctas_per_sm;
     // whole tiles when there are at least two waves of them (or no room for
     // the stream-K tickets), stream-K otherwise
-    const bool sk = tiles < 2 * slots && tiles <= g.max_tickets && g.tickets != nullptr;
+    const bool sk = tiles < 2 * slots;
     p.stream_k = sk ? 1 : 0;
     p.units = tiles * (p.nsteps / 2);
-    const int64_t grid = sk ? std::min<int64_t>(slots, p.units) : std::min<int64_t>(slots, tiles);
+    // stream-K: at most 62 CTAs per tile, so a tile's partials fit the reducer's slot list
+    const int64_t grid = sk ? std::min<int64_t>(std::min<int64_t>(slots, p.units), 62 * tiles)
+                            : std::min<int64_t>(slots, tiles);
     float *ws = nullptr;
     if (sk) {
         const size_t bytes = sizeof(float) * static_cast<size_t>(2 * grid) * BN * kBand;
@@ -456,6 +521,21 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     hybrid_gemm_kernel<BN, STAGES>
         <<<static_cast<unsigned>(grid), kGemmThreads, C::kSmemBytes, stream>>>(map, p);
     cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess && sk) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>((BN * kBand + 255) / 256), static_cast<unsigned>(tiles));
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelEx(&cfg, streamk_reduce_kernel<BN>, static_cast<const float *>(ws),
+                                 p.units, static_cast<int>(grid), p.nsteps / 2, p.ttiles, p.M, p.N,
+                                 p.Y, p.y_fp32);
+    }
     if (ws && ws != g.workspace) {
         cudaError_t e2 = cudaFreeAsync(ws, stream);
         if (err == cudaSuccess) err = e2;
@@ -466,15 +546,15 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
 }  // namespace
 
 size_t decode_workspace_bytes(int num_sms) {
-    // stream-K partials of the M <= 16 configuration: 2 slots per CTA, two CTAs per SM
-    return sizeof(float) * static_cast<size_t>(2 * 2 * num_sms) * 16 * kBand;
+    // stream-K partials of the M <= 16 configuration: 2 slots per CTA, one CTA per SM
+    return sizeof(float) * static_cast<size_t>(2 * num_sms) * 16 * kBand;
 }
 
 cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
-    if (g.M <= 16) return run<16, 4>(g, 2, stream);
-    if (g.M <= 64) return run<64, 8>(g, 1, stream);
-    if (g.M <= 128) return run<128, 6>(g, 1, stream);
-    return run<240, 4>(g, 1, stream);
+    if (g.M <= 16) return run<16, 5>(g, 1, stream);   // 36 KB stages
+    if (g.M <= 64) return run<64, 4>(g, 1, stream);   // 48 KB stages
+    if (g.M <= 128) return run<128, 3>(g, 1, stream); // 64 KB stages
+    return run<160, 3>(g, 1, stream);                 // 72 KB stages
 }
 
 }  // namespace patchk

@@ -26,8 +26,6 @@ struct patch_packed {
     int64_t meta_blocks;
     float *workspace;          // stream-K partials of the M <= 16 configuration
     size_t workspace_bytes;
-    int *tickets;              // stream-K tickets (4 per tile), zero between calls
-    int max_tickets;           // tiles covered by `tickets`
     uint32_t *status;          // device status word
     int num_sms;
     cudaMemPool_t pool;
@@ -72,8 +70,6 @@ patch_status from_cuda(cudaError_t e) {
 }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
-constexpr int kMaxTicketTiles = 1024;
 
 }  // namespace
 
@@ -187,6 +183,7 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     patch_status st = check_shape(shp);
     if (st != PATCH_OK) return st;
     if (shp.N % kBand != 0 || shp.K % (2 * kStep) != 0) return PATCH_ERR_INVALID_ARG;
+    if (shp.K > 28672) return PATCH_ERR_INVALID_ARG;  // one segment's table must fit on chip
     if (!W_bf16 || !meta || !map || !aligned16(W_bf16)) return PATCH_ERR_INVALID_ARG;
     int num_sms = 0;
     st = check_device(&num_sms);
@@ -246,7 +243,6 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     h->meta_blocks = n_meta;
     h->num_sms = num_sms;
     h->workspace_bytes = patchk::decode_workspace_bytes(num_sms);
-    h->max_tickets = kMaxTicketTiles;
 
     e = patchk::device_pool(&h->pool);
     auto alloc = [&](void **ptr, size_t bytes) {
@@ -255,10 +251,7 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     alloc(reinterpret_cast<void **>(&h->packed), h->packed_bytes ? h->packed_bytes : 16);
     alloc(reinterpret_cast<void **>(&h->table), sizeof(uint64_t) * table.size());
     alloc(reinterpret_cast<void **>(&h->workspace), h->workspace_bytes);
-    alloc(reinterpret_cast<void **>(&h->tickets), sizeof(int) * 4 * kMaxTicketTiles);
     alloc(reinterpret_cast<void **>(&h->status), sizeof(uint32_t) * 4);
-    if (e == cudaSuccess)
-        e = cudaMemsetAsync(h->tickets, 0, sizeof(int) * 4 * kMaxTicketTiles, stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(h->status, 0, sizeof(uint32_t) * 4, stream);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(h->table, table.data(), sizeof(uint64_t) * table.size(),
@@ -294,8 +287,6 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.y_fp32 = y_is_fp32;
     g.workspace = Wp->workspace;
     g.workspace_bytes = Wp->workspace_bytes;
-    g.tickets = Wp->tickets;
-    g.max_tickets = Wp->max_tickets;
     g.pool = Wp->pool;
     g.status = Wp->status;
     g.num_sms = Wp->num_sms;
@@ -313,7 +304,6 @@ void patch_free(patch_packed *Wp, void *stream_v) {
     if (Wp->packed) cudaFreeAsync(Wp->packed, stream);
     if (Wp->table) cudaFreeAsync(Wp->table, stream);
     if (Wp->workspace) cudaFreeAsync(Wp->workspace, stream);
-    if (Wp->tickets) cudaFreeAsync(Wp->tickets, stream);
     if (Wp->status) cudaFreeAsync(Wp->status, stream);
     delete Wp;
 }

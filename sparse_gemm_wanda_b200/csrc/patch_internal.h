@@ -29,8 +29,6 @@ struct GemmLaunch {
     int y_fp32;
     float *workspace;        // stream-K partials owned by the handle (may be null)
     size_t workspace_bytes;  // capacity of `workspace`
-    int *tickets;            // stream-K tickets, 4 per tile, zero between calls
-    int max_tickets;         // tiles the ticket array covers
     cudaMemPool_t pool;      // for larger stream-K partials
     uint32_t *status;
     int num_sms;
