@@ -9,8 +9,8 @@
 // Work.  An output tile is one 128-row band of W x BN tokens; D^T[128 x BN]
 // accumulates in tensor memory (fp32).  CTAs are persistent.  Two schedules:
 //   * whole tiles: tile c, c + P, c + 2P, ... (many tiles per CTA);
-//   * stream-K: the (tile, k-pair) units are cut into P contiguous, equal
-//     ranges, one per CTA.  A tile covered by several CTAs leaves fp32
+//   * stream-K: the (tile, k-pair) units are cut into P contiguous ranges of
+//     (nearly) equal bytes, one per CTA.  A tile covered by several CTAs leaves fp32
 //     partials; the last of its CTAs to finish (an atomic ticket) adds them in
 //     CTA order and stores Y, so the result does not depend on timing.
 //     No CTA ever waits for another.
@@ -39,6 +39,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "patch_common.cuh"
 #include "patch_internal.h"
@@ -49,6 +50,8 @@ constexpr int kGemmThreads = 192;
 // k-steps of one segment whose table entries are staged in shared memory
 // (K <= 28672)
 constexpr int kMaxTableSteps = 448;
+// stream-K CTAs whose unit boundaries travel in the kernel parameters
+constexpr int kMaxStreamKCtas = 256;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 template <int BN, int STAGES>
@@ -87,6 +90,7 @@ struct GemmParams {
     float *partial;  // stream-K: [2 * gridDim.x][BN][128]
     uint32_t *status;
     int stall_first_kstep;  // failure-detection test hook: CTA 0 never loads its first k-step
+    int32_t u0[kMaxStreamKCtas + 1];  // stream-K: first unit of every CTA (u0[P] = units)
 };
 
 // One piece of work of a CTA: k-steps [ks0, ks1) of tile (band, ttile).
@@ -96,12 +100,14 @@ struct Segment {
     int slot;    // partial slot of this CTA for this tile
 };
 
-__device__ __forceinline__ int64_t sk_u0(int64_t c, int64_t units, int64_t P) {
-    return (c * units) / P;
-}
-// CTA whose unit range holds unit x: the largest c with floor(c*U/P) <= x.
-__device__ __forceinline__ int64_t sk_cta_of(int64_t x, int64_t units, int64_t P) {
-    return ((x + 1) * P - 1) / units;
+// CTA whose unit range holds unit x: the largest c with u0[c] <= x.
+__device__ __forceinline__ int sk_cta_of(const int32_t *u0, int P, int64_t x) {
+    int lo = 0, hi = P - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (u0[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
 }
 
 __device__ __forceinline__ bool get_segment(const GemmParams &p, int c, int i, Segment &s) {
@@ -117,7 +123,7 @@ __device__ __forceinline__ bool get_segment(const GemmParams &p, int c, int i, S
         s.slot = -1;
     } else {
         const int Q = p.nsteps / 2;
-        const int64_t u0 = sk_u0(c, p.units, P), u1 = sk_u0(c + 1, p.units, P);
+        const int64_t u0 = p.u0[c], u1 = p.u0[c + 1];
         if (u0 >= u1) return false;
         const int64_t t0 = u0 / Q;
         const int64_t t = t0 + i;
@@ -126,7 +132,7 @@ __device__ __forceinline__ bool get_segment(const GemmParams &p, int c, int i, S
         s.tile = static_cast<int>(t);
         s.ks0 = static_cast<int>(2 * (a - t * Q));
         s.ks1 = static_cast<int>(2 * (b - t * Q));
-        const int64_t cf = sk_cta_of(t * Q, p.units, P), cl = sk_cta_of((t + 1) * Q - 1, p.units, P);
+        const int64_t cf = sk_cta_of(p.u0, P, t * Q), cl = sk_cta_of(p.u0, P, (t + 1) * Q - 1);
         s.nsegs = static_cast<int>(cl - cf + 1);
         s.slot = 2 * c + (t == t0 ? 0 : 1);
     }
@@ -137,7 +143,7 @@ __device__ __forceinline__ bool get_segment(const GemmParams &p, int c, int i, S
 
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams p) {
+hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmParams p) {
     using C = GemmCfg<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -171,6 +177,16 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
         *never_flag = 0u;
         *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
         fence_mbar_init();
+        // the first two segments' table entries start moving before anything else
+        if (!*abort_flag) {
+            Segment g0;
+            for (int i = 0; i < 2 && get_segment(p, cta, i, g0); ++i) {
+                const uint32_t nbytes = static_cast<uint32_t>(g0.ks1 - g0.ks0) * 8u;
+                mbar_arrive_expect_tx(&tab_full[i], nbytes);
+                bulk_g2s(tab_buf + i * kMaxTableSteps,
+                         p.table + static_cast<int64_t>(g0.band) * p.nsteps + g0.ks0, nbytes, &tab_full[i]);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, C::kTmemCols);
@@ -198,10 +214,8 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
                 bulk_g2s(tab_buf + buf * kMaxTableSteps,
                          p.table + static_cast<int64_t>(g.band) * p.nsteps + g.ks0, nbytes, &tab_full[buf]);
             };
-            bool have = get_segment(p, cta, 0, sg);
-            if (have) fetch_table(sg, 0);
+            bool have = get_segment(p, cta, 0, sg);  // tables 0 and 1 were fetched at start
             bool have_nx = have && get_segment(p, cta, 1, nx);
-            if (have_nx) fetch_table(nx, 1);
             int tabs_issued = (have ? 1 : 0) + (have_nx ? 1 : 0);
             for (int i = 0; ok && have; ++i) {
                 const int buf = i & 1;
@@ -390,18 +404,22 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams 
 // timing).  Launched as a programmatic dependent of the GEMM; waits for it.
 template <int BN>
 __global__ void __launch_bounds__(256)
-streamk_reduce_kernel(const float *__restrict__ partial, int64_t units, int P, int Q, int ttiles,
-                      int64_t M, int64_t N, void *Y, int y_fp32) {
+streamk_reduce_kernel(const float *__restrict__ partial, const __grid_constant__ GemmParams p,
+                      int P) {
+    const int Q = p.nsteps / 2, ttiles = p.ttiles;
+    const int64_t M = p.M, N = p.N;
+    void *Y = p.Y;
+    const int y_fp32 = p.y_fp32;
     // block (tile t, chunk): one output per thread, 256 outputs per block
     __shared__ int slots[64];
     __shared__ int nslots;
     const int64_t t = blockIdx.y;
     if (threadIdx.x == 0) {
-        const int64_t cf = sk_cta_of(t * Q, units, P), cl = sk_cta_of((t + 1) * Q - 1, units, P);
+        const int64_t cf = sk_cta_of(p.u0, P, t * Q), cl = sk_cta_of(p.u0, P, (t + 1) * Q - 1);
         int n = 0;
         if (cf != cl) {  // a tile with one CTA was stored directly
             for (int64_t cc = cf; cc <= cl && n < 64; ++cc)
-                slots[n++] = static_cast<int>(2 * cc + ((sk_u0(cc, units, P) / Q == t) ? 0 : 1));
+                slots[n++] = static_cast<int>(2 * cc + ((p.u0[cc] / Q == t) ? 0 : 1));
         }
         nslots = n;
     }
@@ -472,6 +490,46 @@ bool make_x_map(CUtensorMap *map, const void *X, int64_t M, int64_t K, int bn) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Stream-K boundaries: unit u = tile * Q + pair (tile = band * ttiles + ttile)
+// costs its packed bytes plus the bytes of its two X tiles; CTA c starts at the
+// first unit whose cumulative cost reaches c / P of the total.
+void streamk_bounds(const GemmLaunch &g, GemmParams &p, int bn, int P) {
+    const int Q = p.nsteps / 2;
+    const int64_t tiles = static_cast<int64_t>(p.bands) * p.ttiles;
+    const int64_t xb = 2LL * bn * kStep * 2;  // X bytes per pair
+    if (!g.pair_prefix) {  // equal unit counts
+        for (int c = 0; c <= P; ++c) p.u0[c] = static_cast<int32_t>((c * p.units) / P);
+        return;
+    }
+    auto pair_cum = [&](int band, int q) {  // cost of pairs [0, q) of a band
+        return g.pair_prefix[static_cast<int64_t>(band) * (Q + 1) + q] + xb * q;
+    };
+    std::vector<int64_t> tile_cum(static_cast<size_t>(tiles + 1), 0);
+    for (int64_t t = 0; t < tiles; ++t)
+        tile_cum[t + 1] = tile_cum[t] + pair_cum(static_cast<int>(t / p.ttiles), Q);
+    const int64_t total = tile_cum[tiles];
+    p.u0[0] = 0;
+    p.u0[P] = static_cast<int32_t>(p.units);
+    for (int c = 1; c < P; ++c) {
+        const int64_t target = (total * c) / P;
+        // the tile holding the target, then the first pair boundary at or past it
+        int64_t t = std::upper_bound(tile_cum.begin(), tile_cum.end(), target) - tile_cum.begin() - 1;
+        if (t >= tiles) t = tiles - 1;
+        const int band = static_cast<int>(t / p.ttiles);
+        int q = 0;
+        while (q < Q && tile_cum[t] + pair_cum(band, q) < target) ++q;
+        int64_t u = t * Q + q;
+        if (u < p.u0[c - 1]) u = p.u0[c - 1];
+        p.u0[c] = static_cast<int32_t>(u);
+    }
+    // every CTA keeps at least one unit (P <= units)
+    for (int c = 1; c < P; ++c)
+        if (p.u0[c] <= p.u0[c - 1]) p.u0[c] = p.u0[c - 1] + 1;
+    p.u0[P] = static_cast<int32_t>(p.units);
+    for (int c = P - 1; c >= 1; --c)
+        if (p.u0[c] >= p.u0[c + 1]) p.u0[c] = p.u0[c + 1] - 1;
+}
+
 template <int BN, int STAGES>
 cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     using C = GemmCfg<BN, STAGES>;
@@ -505,8 +563,11 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     p.stream_k = sk ? 1 : 0;
     p.units = tiles * (p.nsteps / 2);
     // stream-K: at most 62 CTAs per tile, so a tile's partials fit the reducer's slot list
-    const int64_t grid = sk ? std::min<int64_t>(std::min<int64_t>(slots, p.units), 62 * tiles)
+    const int64_t grid = sk ? std::min<int64_t>(std::min<int64_t>(std::min<int64_t>(slots, p.units),
+                                                                   62 * tiles),
+                                                kMaxStreamKCtas)
                             : std::min<int64_t>(slots, tiles);
+    if (sk) streamk_bounds(g, p, BN, static_cast<int>(grid));
     float *ws = nullptr;
     if (sk) {
         const size_t bytes = sizeof(float) * static_cast<size_t>(2 * grid) * BN * kBand;
@@ -532,9 +593,8 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        err = cudaLaunchKernelEx(&cfg, streamk_reduce_kernel<BN>, static_cast<const float *>(ws),
-                                 p.units, static_cast<int>(grid), p.nsteps / 2, p.ttiles, p.M, p.N,
-                                 p.Y, p.y_fp32);
+        err = cudaLaunchKernelEx(&cfg, streamk_reduce_kernel<BN>, static_cast<const float *>(ws), p,
+                                 static_cast<int>(grid));
     }
     if (ws && ws != g.workspace) {
         cudaError_t e2 = cudaFreeAsync(ws, stream);

@@ -7,8 +7,8 @@
 //      n_j = sqrt(s_j) (IEEE round-to-nearest).
 //   2. score_mask: per tile, Wanda scores |W_ij| * n_j (one fp64 multiply),
 //      top-2-of-4 per group (score descending, lower index on ties), the 4-bit
-//      code idx0 | idx1 << 2, and the tile's pruned-score loss (rows left to
-//      right, then rows top to bottom).
+//      code idx0 | idx1 << 2, and the tile's pruned-score loss (32-column words
+//      left to right, a row's words left to right, rows as a pairwise tree).
 //   3. select_map: tiles ranked by (loss ascending, index ascending); the
 //      first floor(f * n_tiles) become 2:4.
 //
@@ -33,43 +33,36 @@ constexpr int kColsqUnroll = 16;
 __device__ __forceinline__ double bf16_lo_to_f64(uint32_t v) {
     return static_cast<double>(__uint_as_float(v << 16));
 }
-__device__ __forceinline__ double bf16_hi_to_f64(uint32_t v) {
-    return static_cast<double>(__uint_as_float(v & 0xFFFF0000u));
-}
 
-// One thread = two adjacent columns x one 128-token chunk.  Reads are 4-byte
-// per thread, 128 contiguous bytes per warp and row.
+// One thread = one column x one 128-token chunk (the chunk's tokens in order).
+// A warp reads 64 contiguous bytes of each token row.
 __global__ void __launch_bounds__(kColsqThreads)
-colsq_partial_kernel(const uint32_t *__restrict__ X2, int64_t T, int64_t K,
+colsq_partial_kernel(const uint16_t *__restrict__ X, int64_t T, int64_t K,
                      double *__restrict__ partial) {
-    const int64_t pairs = K / 2;
-    const int64_t p = static_cast<int64_t>(blockIdx.x) * kColsqThreads + threadIdx.x;
-    if (p >= pairs) return;
+    const int64_t j = static_cast<int64_t>(blockIdx.x) * kColsqThreads + threadIdx.x;
+    if (j >= K) return;
     const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kColsqChunk;
     const int64_t t1 = min(T, t0 + kColsqChunk);
-    const uint32_t *src = X2 + t0 * pairs + p;
-    double a = 0.0, b = 0.0;
+    const uint16_t *src = X + t0 * K + j;
+    double a = 0.0;
     int64_t t = t0;
     for (; t + kColsqUnroll <= t1; t += kColsqUnroll) {
-        uint32_t v[kColsqUnroll];
+        uint16_t v[kColsqUnroll];
 #pragma unroll
-        for (int u = 0; u < kColsqUnroll; ++u) v[u] = __ldg(src + u * pairs);
+        for (int u = 0; u < kColsqUnroll; ++u) v[u] = __ldg(src + u * K);
 #pragma unroll
         for (int u = 0; u < kColsqUnroll; ++u) {
-            const double x0 = bf16_lo_to_f64(v[u]), x1 = bf16_hi_to_f64(v[u]);
-            a = __dadd_rn(a, __dmul_rn(x0, x0));
-            b = __dadd_rn(b, __dmul_rn(x1, x1));
+            const double x = bf16_lo_to_f64(v[u]);
+            a = __dadd_rn(a, __dmul_rn(x, x));
         }
-        src += kColsqUnroll * pairs;
+        src += kColsqUnroll * K;
     }
     for (; t < t1; ++t) {
-        const uint32_t v = __ldg(src);
-        const double x0 = bf16_lo_to_f64(v), x1 = bf16_hi_to_f64(v);
-        a = __dadd_rn(a, __dmul_rn(x0, x0));
-        b = __dadd_rn(b, __dmul_rn(x1, x1));
-        src += pairs;
+        const double x = bf16_lo_to_f64(__ldg(src));
+        a = __dadd_rn(a, __dmul_rn(x, x));
+        src += K;
     }
-    reinterpret_cast<double2 *>(partial + blockIdx.y * K)[p] = make_double2(a, b);
+    partial[blockIdx.y * K + j] = a;
 }
 
 // s_j = chunk sums added in chunk order; n_j = sqrt(s_j).
@@ -105,8 +98,6 @@ __global__ void norms_from_colsq_kernel(const double *__restrict__ colsq_in, int
 }
 
 // ----------------------------------------------------------------- scoring
-constexpr int kScoreThreads = 128;
-
 // Select the two kept positions of one group: q is kept iff fewer than two
 // other candidates come before it in the order (score desc, index asc).
 __device__ __forceinline__ uint32_t top2_code(const double s[4]) {
@@ -124,79 +115,99 @@ __device__ __forceinline__ uint32_t top2_code(const double s[4]) {
     return lo | (hi << 2);
 }
 
-// One CTA per tile.  The tile is staged in shared memory with coalesced 16-B
-// loads (rows padded by 16 B); then thread r owns row r of the tile, so the
-// row's pruned-score sum runs left to right in one thread.
-template <int TN, int TK>
-__global__ void __launch_bounds__(kScoreThreads)
-score_mask_kernel(const uint16_t *__restrict__ W, const double *__restrict__ norm, int64_t N,
-                  int64_t K, uint32_t *__restrict__ meta, double *__restrict__ loss) {
-    constexpr int kRowElems = TK + 8;       // padded row (bf16 elements)
-    constexpr int kChunksPerRow = TK / 8;   // 16-byte chunks per tile row
-    constexpr int kWordsPerRow = TK / 32;   // meta words per tile row
-    __shared__ __align__(16) uint16_t ws[TN * kRowElems];
-    __shared__ double ns[TK];
-    __shared__ double rows[TN];
-    __shared__ uint32_t ms[TN * kWordsPerRow];
+// |w| of a bf16 bit pattern, exactly, as a double (sign cleared: -0 -> +0).
+// Normal values are rebuilt with integer operations (exponent rebias 127 ->
+// 1023, mantissa moved up); zero and subnormals take the conversion path.
+__device__ __forceinline__ double bf16_abs_f64(uint32_t bits16) {
+    const uint32_t e8 = (bits16 >> 7) & 0xFFu, m7 = bits16 & 0x7Fu;
+    if (e8 != 0u) return __hiloint2double(static_cast<int>(((e8 + 896u) << 20) | (m7 << 13)), 0);
+    return static_cast<double>(__uint_as_float((bits16 & 0x7FFFu) << 16));
+}
 
+// One CTA per tile, one thread per (row, 32-column word) of the tile.  A
+// thread reads its 64 bytes of W with coalesced 16-byte loads (a warp covers
+// whole rows), scores its 8 groups, writes the meta word and the word's
+// pruned-score sum (left to right).  The CTA then adds each row's words left
+// to right and the rows as a balanced pairwise tree.
+template <int TN, int TK>
+__global__ void __launch_bounds__(TN *(TK / 32))
+score_mask_kernel(const uint16_t *__restrict__ W, const double *__restrict__ norm, int64_t N,
+                  int64_t K, uint32_t *__restrict__ meta, double *__restrict__ loss,
+                  int32_t *__restrict__ rank, uint32_t *__restrict__ done) {
+    constexpr int WPR = TK / 32;      // words per tile row
+    constexpr int kNormStride = 33;   // padded: the words' norms sit in different banks
+    constexpr int kWarps = TN / 32;   // warps holding the tile's row sums
+    __shared__ double ns[WPR * kNormStride];
+    __shared__ double wsum[TN * WPR];
+    __shared__ double warp_sum[kWarps];
     const int64_t tiles_k = K / TK;
     const int64_t t = blockIdx.x;
     const int64_t i0 = (t / tiles_k) * TN, j0 = (t % tiles_k) * TK;
     const int tid = threadIdx.x;
+    const int r = tid / WPR, w = tid % WPR;
 
-    for (int u = tid; u < TN * kChunksPerRow; u += kScoreThreads) {
-        const int r = u / kChunksPerRow, c = u % kChunksPerRow;
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(W + (i0 + r) * K + j0) + c);
-        *reinterpret_cast<uint4 *>(ws + r * kRowElems + c * 8) = v;
-    }
-    for (int u = tid; u < TK; u += kScoreThreads) ns[u] = __ldg(norm + j0 + u);
+    for (int u = tid; u < TK; u += TN * WPR) ns[(u / 32) * kNormStride + u % 32] = __ldg(norm + j0 + u);
+    const uint4 *src = reinterpret_cast<const uint4 *>(W + (i0 + r) * K + j0 + 32 * w);
+    uint4 v[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) v[h] = __ldg(src + h);
     __syncthreads();
 
-    if (tid < TN) {
-        const uint16_t *row = ws + tid * kRowElems;
-        double rsum = 0.0;
-#pragma unroll 1
-        for (int w = 0; w < kWordsPerRow; ++w) {
-            uint32_t word = 0;
+    const double *nw = ns + w * kNormStride;
+    double acc = 0.0;
+    uint32_t word = 0;
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {  // 4 x 8 columns = one 32-column word
-                const uint4 v = *reinterpret_cast<const uint4 *>(row + w * 32 + h * 8);
-                const uint32_t e[4] = {v.x, v.y, v.z, v.w};
+    for (int h = 0; h < 4; ++h) {
+        const uint32_t e[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
 #pragma unroll
-                for (int gg = 0; gg < 2; ++gg) {
-                    const int col = w * 32 + h * 8 + gg * 4;
-                    double s[4];
+        for (int gg = 0; gg < 2; ++gg) {
+            const int col = h * 8 + gg * 4;
+            double sc[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t pairbits = e[gg * 2 + q / 2];
-                        const uint32_t bits = (q & 1) ? (pairbits >> 16) : (pairbits & 0xFFFFu);
-                        const double mag = static_cast<double>(__uint_as_float((bits & 0x7FFFu) << 16));
-                        s[q] = __dmul_rn(mag, ns[col + q]);
-                    }
-                    const uint32_t code = top2_code(s);
-                    const uint32_t lo = code & 3u, hi = code >> 2;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        if (q != static_cast<int>(lo) && q != static_cast<int>(hi))
-                            rsum = __dadd_rn(rsum, s[q]);
-                    word |= code << (4 * (h * 2 + gg));
-                }
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t pairbits = e[gg * 2 + q / 2];
+                const uint32_t bits = (q & 1) ? (pairbits >> 16) : (pairbits & 0xFFFFu);
+                sc[q] = __dmul_rn(bf16_abs_f64(bits), nw[col + q]);
             }
-            ms[tid * kWordsPerRow + w] = word;
+            const uint32_t code = top2_code(sc);
+            const int lo = static_cast<int>(code & 3u), hi = static_cast<int>(code >> 2);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (q != lo && q != hi) acc = __dadd_rn(acc, sc[q]);
+            word |= code << (4 * (h * 2 + gg));
         }
-        rows[tid] = rsum;
+    }
+    meta[(i0 + r) * (K / 32) + j0 / 32 + w] = word;
+    wsum[tid] = acc;
+    __syncthreads();
+    if (tid < TN) {
+        // row sum: the row's words left to right
+        double row = 0.0;
+#pragma unroll
+        for (int q = 0; q < WPR; ++q) row = __dadd_rn(row, wsum[tid * WPR + q]);
+        // balanced pairwise tree over rows: levels 1..5 inside the warp (node q
+        // of level k lives in lane q * 2^k), then across the warps
+#pragma unroll
+        for (int off = 1; off < 32; off *= 2) {
+            const double other = __shfl_down_sync(0xFFFFFFFFu, row, off);
+            row = __dadd_rn(row, other);
+        }
+        if ((tid & 31) == 0) warp_sum[tid / 32] = row;
     }
     __syncthreads();
-
-    const int64_t words_k = K / 32;
-    for (int u = tid; u < TN * kWordsPerRow; u += kScoreThreads) {
-        const int r = u / kWordsPerRow, w = u % kWordsPerRow;
-        meta[(i0 + r) * words_k + j0 / 32 + w] = ms[u];
+    if (tid == 0 && rank) {  // counters of the ranking step that follows
+        rank[t] = 0;
+        if (t == 0) *done = 0u;
     }
     if (tid == 0) {
-        double total = 0.0;
-        for (int r = 0; r < TN; ++r) total = __dadd_rn(total, rows[r]);
-        loss[t] = total;
+        double x[kWarps];
+#pragma unroll
+        for (int q = 0; q < kWarps; ++q) x[q] = warp_sum[q];
+#pragma unroll
+        for (int n = kWarps; n > 1; n /= 2)
+#pragma unroll
+            for (int q = 0; q < n / 2; ++q) x[q] = __dadd_rn(x[2 * q], x[2 * q + 1]);
+        loss[t] = x[0];
     }
 }
 
@@ -206,43 +217,51 @@ constexpr int kRankSlice = 256;
 
 // rank[t] += #{u in this block's slice : (L_u, u) < (L_t, t)}.  Integer
 // counts, so the accumulated rank does not depend on the order of atomics.
+// The last block to finish writes the bitmap: bit t set iff rank[t] < n_sparse.
 __global__ void __launch_bounds__(kRankThreads)
-rank_tiles_kernel(const double *__restrict__ loss, int64_t n_tiles, int32_t *__restrict__ rank) {
+rank_tiles_kernel(const double *__restrict__ loss, int64_t n_tiles, int64_t n_sparse,
+                  int32_t *__restrict__ rank, uint32_t *__restrict__ done, uint32_t *__restrict__ map) {
     __shared__ double sl[kRankSlice];
+    __shared__ bool last;
     const int64_t t = static_cast<int64_t>(blockIdx.x) * kRankThreads + threadIdx.x;
     const int64_t u0 = static_cast<int64_t>(blockIdx.y) * kRankSlice;
     const int64_t u1 = min(n_tiles, u0 + kRankSlice);
     for (int64_t u = u0 + threadIdx.x; u < u1; u += kRankThreads) sl[u - u0] = loss[u];
     __syncthreads();
-    if (t >= n_tiles) return;
-    const double lt = loss[t];
-    int32_t r = 0;
-    for (int64_t u = u0; u < u1; ++u) {
-        const double lu = sl[u - u0];
-        r += (lu < lt) || (lu == lt && u < t);
+    if (t < n_tiles) {
+        const double lt = loss[t];
+        int32_t r = 0;
+        for (int64_t u = u0; u < u1; ++u) {
+            const double lu = sl[u - u0];
+            r += (lu < lt) || (lu == lt && u < t);
+        }
+        atomicAdd(rank + t, r);
     }
-    atomicAdd(rank + t, r);
-}
-
-// Bit t of the map is set iff rank[t] < n_sparse.  One warp per 32 tiles.
-__global__ void map_from_rank_kernel(const int32_t *__restrict__ rank, int64_t n_tiles,
-                                     int64_t n_sparse, uint32_t *__restrict__ map) {
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+        last = atomicAdd(done, 1u) == gridDim.x * gridDim.y - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
     const int64_t words = (n_tiles + 31) / 32;
-    if (t / 32 >= words) return;
-    const bool bit = t < n_tiles && rank[t] < n_sparse;
-    const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, bit);
-    if ((threadIdx.x & 31) == 0) map[t / 32] = ballot;
+    for (int64_t wd = threadIdx.x; wd < words; wd += kRankThreads) {
+        uint32_t bits = 0;
+        for (int q = 0; q < 32; ++q) {
+            const int64_t tt = wd * 32 + q;
+            if (tt < n_tiles && __ldcg(rank + tt) < n_sparse) bits |= 1u << q;
+        }
+        map[wd] = bits;
+    }
 }
 
 // ------------------------------------------------------------------ launch
 cudaError_t launch_colsq(const void *Xcal, int64_t T, int64_t K, double *partial,
                          double *colsq_out, double *norm_out, cudaStream_t stream) {
     const int64_t chunks = (T + kColsqChunk - 1) / kColsqChunk;
-    const int64_t pairs = K / 2;
-    dim3 grid(static_cast<unsigned>((pairs + kColsqThreads - 1) / kColsqThreads),
+    dim3 grid(static_cast<unsigned>((K + kColsqThreads - 1) / kColsqThreads),
               static_cast<unsigned>(chunks));
-    colsq_partial_kernel<<<grid, kColsqThreads, 0, stream>>>(static_cast<const uint32_t *>(Xcal), T,
+    colsq_partial_kernel<<<grid, kColsqThreads, 0, stream>>>(static_cast<const uint16_t *>(Xcal), T,
                                                              K, partial);
     colsq_final_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, stream>>>(
         partial, chunks, K, colsq_out, norm_out);
@@ -257,34 +276,29 @@ cudaError_t launch_norms_from_colsq(const double *colsq_in, int64_t K, double *c
 }
 
 cudaError_t launch_score_mask(const void *W, const double *norm, int64_t N, int64_t K, int tn,
-                              int tk, uint32_t *meta, double *loss, cudaStream_t stream) {
+                              int tk, uint32_t *meta, double *loss, int32_t *rank, uint32_t *done,
+                              cudaStream_t stream) {
     const int64_t n_tiles = (N / tn) * (K / tk);
     const uint16_t *w = static_cast<const uint16_t *>(W);
     const unsigned g = static_cast<unsigned>(n_tiles);
     if (tn == 128 && tk == 128)
-        score_mask_kernel<128, 128><<<g, kScoreThreads, 0, stream>>>(w, norm, N, K, meta, loss);
+        score_mask_kernel<128, 128><<<g, 512, 0, stream>>>(w, norm, N, K, meta, loss, rank, done);
     else if (tn == 128 && tk == 64)
-        score_mask_kernel<128, 64><<<g, kScoreThreads, 0, stream>>>(w, norm, N, K, meta, loss);
+        score_mask_kernel<128, 64><<<g, 256, 0, stream>>>(w, norm, N, K, meta, loss, rank, done);
     else if (tn == 64 && tk == 128)
-        score_mask_kernel<64, 128><<<g, kScoreThreads, 0, stream>>>(w, norm, N, K, meta, loss);
+        score_mask_kernel<64, 128><<<g, 256, 0, stream>>>(w, norm, N, K, meta, loss, rank, done);
     else if (tn == 64 && tk == 64)
-        score_mask_kernel<64, 64><<<g, kScoreThreads, 0, stream>>>(w, norm, N, K, meta, loss);
+        score_mask_kernel<64, 64><<<g, 128, 0, stream>>>(w, norm, N, K, meta, loss, rank, done);
     else
         return cudaErrorInvalidValue;
     return cudaGetLastError();
 }
 
 cudaError_t launch_select_map(const double *loss, int64_t n_tiles, int64_t n_sparse, int32_t *rank,
-                              uint32_t *map, cudaStream_t stream) {
-    cudaError_t err = cudaMemsetAsync(rank, 0, sizeof(int32_t) * n_tiles, stream);
-    if (err != cudaSuccess) return err;
+                              uint32_t *done, uint32_t *map, cudaStream_t stream) {
     dim3 grid(static_cast<unsigned>((n_tiles + kRankThreads - 1) / kRankThreads),
               static_cast<unsigned>((n_tiles + kRankSlice - 1) / kRankSlice));
-    rank_tiles_kernel<<<grid, kRankThreads, 0, stream>>>(loss, n_tiles, rank);
-    const int64_t words = (n_tiles + 31) / 32;
-    const int64_t threads = words * 32;
-    map_from_rank_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
-        rank, n_tiles, n_sparse, map);
+    rank_tiles_kernel<<<grid, kRankThreads, 0, stream>>>(loss, n_tiles, n_sparse, rank, done, map);
     return cudaGetLastError();
 }
 

@@ -19,79 +19,78 @@ namespace patchk {
 
 constexpr int kPackThreads = 128;
 
-// One CTA per (band, k-step).  The 128 x 64 block of W is staged in shared
-// memory with coalesced loads, thread r rewrites row r, and the result leaves
-// through coalesced 16-byte stores in the swizzled order.
+// Keep the two entries of each group that its 4-bit code names, zero the
+// others, for 8 consecutive bf16 values (two groups) held in a uint4.
+__device__ __forceinline__ uint4 mask_two_groups(uint4 v, uint32_t codes8) {
+    uint32_t e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        const uint32_t code = (codes8 >> (4 * g)) & 0xFu;
+        const uint32_t lo = code & 3u, hi = code >> 2;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (q == static_cast<int>(lo) || q == static_cast<int>(hi)) continue;
+            e[2 * g + q / 2] &= (q & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+        }
+    }
+    return make_uint4(e[0], e[1], e[2], e[3]);
+}
+
+// The two kept values of one group (4 bf16 in the 32-bit words a, b) as one
+// 32-bit word, lower position first.
+__device__ __forceinline__ uint32_t kept_pair(uint32_t a, uint32_t b, uint32_t code) {
+    const uint32_t w0 = a & 0xFFFFu, w1 = a >> 16, w2 = b & 0xFFFFu, w3 = b >> 16;
+    const uint32_t lo = code & 3u, hi = code >> 2;  // lo in {0,1,2}, hi in {1,2,3}
+    const uint32_t x0 = lo == 0 ? w0 : (lo == 1 ? w1 : w2);
+    const uint32_t x1 = hi == 3 ? w3 : (hi == 2 ? w2 : w1);
+    return x0 | (x1 << 16);
+}
+
+// One CTA per (band, k-step); every thread writes whole 16-byte chunks of the
+// swizzled output straight from global W (no shared-memory staging).
 __global__ void __launch_bounds__(kPackThreads)
 pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
             const uint32_t *__restrict__ map, int64_t N, int64_t K, int tn, int tk,
             const uint64_t *__restrict__ table, uint8_t *__restrict__ out) {
-    constexpr int kRow = kStep + 8;  // padded smem row (bf16)
-    __shared__ __align__(16) uint16_t ws[kBand * kRow];
-    __shared__ __align__(16) uint16_t cs[kBand * 40];  // compressed rows (32 used)
-    __shared__ uint32_t ms[kBand * 2];
-
     const int64_t nsteps = K / kStep;
     const int64_t b = blockIdx.x / nsteps, c = blockIdx.x % nsteps;
     const uint64_t entry = table[blockIdx.x];
     const int64_t off = static_cast<int64_t>(entry & kEntryOffsetMask);
-    const bool sparse = (entry & kEntrySparse) != 0;
     const int tid = threadIdx.x;
     const int64_t row0 = b * kBand, col0 = c * kStep;
     const int64_t words_k = K / 32;
 
-    for (int u = tid; u < kBand * 8; u += kPackThreads) {
-        const int r = u / 8, q = u % 8;
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(W + (row0 + r) * K + col0) + q);
-        *reinterpret_cast<uint4 *>(ws + r * kRow + q * 8) = v;
-    }
-    for (int u = tid; u < kBand * 2; u += kPackThreads) {
-        const int r = u / 2, q = u % 2;
-        ms[u] = __ldg(meta + (row0 + r) * words_k + col0 / 32 + q);
-    }
-    __syncthreads();
-
-    {
-        const int r = tid;
-        uint16_t *row = ws + r * kRow;
-        const uint32_t m0 = ms[2 * r], m1 = ms[2 * r + 1];
-        if (!sparse) {
-            // Dense storage: W_eff, i.e. W with pruned entries of 2:4 tiles at +0
-            // (a k-step falls in exactly one tile column since tk >= 64).
-            const int64_t tile = ((row0 + r) / tn) * (K / tk) + col0 / tk;
-            if ((__ldg(map + tile / 32) >> (tile % 32)) & 1u) {
-                for (int g = 0; g < 16; ++g) {
-                    const uint32_t code = ((g < 8 ? m0 : m1) >> (4 * (g % 8))) & 0xFu;
-                    for (int q = 0; q < 4; ++q)
-                        if (q != static_cast<int>(code & 3u) && q != static_cast<int>(code >> 2))
-                            row[4 * g + q] = 0;
-                }
-            }
-        } else {
-            uint16_t *crow = cs + r * 40;
-            for (int g = 0; g < 16; ++g) {
-                const uint32_t code = ((g < 8 ? m0 : m1) >> (4 * (g % 8))) & 0xFu;
-                crow[2 * g] = row[4 * g + (code & 3u)];
-                crow[2 * g + 1] = row[4 * g + (code >> 2)];
-            }
-        }
-    }
-    __syncthreads();
-
-    if (!sparse) {
-        // output 16-B chunk u = r*8 + ((k/8) ^ (r%8))
+    if (!(entry & kEntrySparse)) {
+        // dense: chunk u = r*8 + ((k/8) ^ (r%8)); W_eff, i.e. pruned entries of
+        // a 2:4 tile (64-row tiles sharing a band with a dense tile) are zeroed
+#pragma unroll 4
         for (int u = tid; u < kBand * 8; u += kPackThreads) {
-            const int r = u / 8, cc = u % 8, src = cc ^ (r % 8);
-            const uint4 v = *reinterpret_cast<const uint4 *>(ws + r * kRow + src * 8);
+            const int r = u / 8, k8 = (u % 8) ^ (r % 8);
+            const int64_t i = row0 + r, j = col0 + 8 * k8;
+            uint4 v = __ldg(reinterpret_cast<const uint4 *>(W + i * K + j));
+            const int64_t tile = (i / tn) * (K / tk) + j / tk;
+            if ((__ldg(map + tile / 32) >> (tile % 32)) & 1u) {
+                const uint32_t mw = __ldg(meta + i * words_k + j / 32);
+                v = mask_two_groups(v, mw >> (4 * ((j % 32) / 4)));
+            }
             reinterpret_cast<uint4 *>(out + off)[u] = v;
         }
         return;
     }
-    // output 16-B chunk u = r*4 + ((v/8) ^ ((r%8)/2))
+    // 2:4: chunk u = r*4 + ((v/8) ^ ((r%8)/2)) holds the kept values of groups
+    // 4*(v/8) .. 4*(v/8)+3 of the row, two per group in column order
+#pragma unroll 4
     for (int u = tid; u < kBand * 4; u += kPackThreads) {
-        const int r = u / 4, cc = u % 4, src = cc ^ ((r % 8) / 2);
-        const uint4 v = *reinterpret_cast<const uint4 *>(cs + r * 40 + src * 8);
-        reinterpret_cast<uint4 *>(out + off)[u] = v;
+        const int r = u / 4, v8 = (u % 4) ^ ((r % 8) / 2);
+        const int64_t i = row0 + r, j = col0 + 16 * v8;
+        const uint4 *src = reinterpret_cast<const uint4 *>(W + i * K + j);
+        const uint4 a = __ldg(src), bq = __ldg(src + 1);
+        const uint32_t e[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+        const uint32_t codes = __ldg(meta + i * words_k + j / 32) >> (4 * ((j % 32) / 4));
+        uint32_t o[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) o[g] = kept_pair(e[2 * g], e[2 * g + 1], (codes >> (4 * g)) & 0xFu);
+        reinterpret_cast<uint4 *>(out + off)[u] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (entry & kEntryMeta) {
         // The metadata block of k-pair p: line l = m0 + 8*k1 + 16*m2 holds, in
@@ -102,6 +101,7 @@ pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
         const int m0i = l % 8, k1 = (l / 8) % 2, m2 = l / 16;
         const int64_t ra = row0 + m0i + 16 * m2, rb = ra + 8;
         uint32_t wv[4];
+#pragma unroll
         for (int k2 = 0; k2 < 4; ++k2) {
             const int64_t ks = 2 * p + k2 / 2;
             const bool sp = (table[b * nsteps + ks] & kEntrySparse) != 0;

@@ -7,6 +7,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <map>
 #include <mutex>
 #include <new>
@@ -18,6 +19,7 @@
 
 struct patch_packed {
     int device;
+    uint8_t *base;             // one pool allocation holding all device arrays below
     patch_shape shp;
     uint8_t *packed;           // packed k-steps
     size_t packed_bytes;
@@ -29,6 +31,7 @@ struct patch_packed {
     uint32_t *status;          // device status word
     int num_sms;
     cudaMemPool_t pool;
+    std::vector<int64_t> pair_prefix;  // per band: cumulative packed bytes of its k-pairs
 };
 
 namespace {
@@ -49,18 +52,72 @@ patch_status check_shape(const patch_shape &s) {
     return PATCH_OK;
 }
 
+struct DevInfo {
+    int major = 0, minor = 0, sms = 0;
+};
+
+// Compute capability and SM count of the current device (queried once).
 patch_status check_device(int *num_sms) {
+    static std::mutex mu;
+    static std::map<int, DevInfo> cache;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return PATCH_ERR_CUDA;
-    int major = 0, minor = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-        return PATCH_ERR_CUDA;
-    if (major != 10 || minor != 0) return PATCH_ERR_UNSUPPORTED;
-    if (num_sms &&
-        cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return PATCH_ERR_CUDA;
+    DevInfo info;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(dev);
+        if (it != cache.end()) {
+            info = it->second;
+        } else {
+            if (cudaDeviceGetAttribute(&info.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&info.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return PATCH_ERR_CUDA;
+            cache[dev] = info;
+        }
+    }
+    if (info.major != 10 || info.minor != 0) return PATCH_ERR_UNSUPPORTED;
+    if (num_sms) *num_sms = info.sms;
     return PATCH_OK;
+}
+
+// A reusable page-locked staging buffer per device for small host-to-device
+// uploads (the k-step table): the copy is asynchronous, and the next user
+// waits on the event recorded after it before overwriting the buffer.
+struct PinnedStage {
+    void *buf = nullptr;
+    size_t cap = 0;
+    cudaEvent_t done = nullptr;
+};
+
+cudaError_t upload_via_pinned(void *dst, const void *src, size_t bytes, cudaStream_t stream) {
+    static std::mutex mu;
+    static std::map<int, PinnedStage> stages;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    PinnedStage &st = stages[dev];
+    if (!st.done) {
+        e = cudaEventCreateWithFlags(&st.done, cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+    } else {
+        e = cudaEventSynchronize(st.done);  // the previous upload has left the buffer
+        if (e != cudaSuccess) return e;
+    }
+    if (st.cap < bytes) {
+        if (st.buf) cudaFreeHost(st.buf);
+        st.buf = nullptr;
+        st.cap = 0;
+        const size_t cap = std::max<size_t>(bytes, 1 << 20);
+        e = cudaMallocHost(&st.buf, cap);
+        if (e != cudaSuccess) return e;
+        st.cap = cap;
+    }
+    memcpy(st.buf, src, bytes);
+    e = cudaMemcpyAsync(dst, st.buf, bytes, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaEventRecord(st.done, stream);
+    return e;
 }
 
 patch_status from_cuda(cudaError_t e) {
@@ -142,7 +199,8 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
     size_t off_norm = round_up(off_partial + sizeof(double) * chunks * K, 256);
     size_t off_loss = round_up(off_norm + sizeof(double) * K, 256);
     size_t off_rank = round_up(off_loss + (tile_loss_out ? 0 : sizeof(double) * n_tiles), 256);
-    size_t total = round_up(off_rank + (map_in ? 0 : sizeof(int32_t) * n_tiles), 256);
+    size_t off_done = round_up(off_rank + (map_in ? 0 : sizeof(int32_t) * n_tiles), 256);
+    size_t total = off_done + 256;
     cudaMemPool_t pool = nullptr;
     cudaError_t e = patchk::device_pool(&pool);
     if (e != cudaSuccess) return from_cuda(e);
@@ -152,7 +210,8 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
     double *partial = reinterpret_cast<double *>(scratch + off_partial);
     double *norm = reinterpret_cast<double *>(scratch + off_norm);
     double *loss = tile_loss_out ? tile_loss_out : reinterpret_cast<double *>(scratch + off_loss);
-    int32_t *rank = reinterpret_cast<int32_t *>(scratch + off_rank);
+    int32_t *rank = map_in ? nullptr : reinterpret_cast<int32_t *>(scratch + off_rank);
+    uint32_t *done = reinterpret_cast<uint32_t *>(scratch + off_done);
 
     if (colsq_in)
         e = patchk::launch_norms_from_colsq(colsq_in, K, colsq_out, norm, stream);
@@ -160,7 +219,7 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
         e = patchk::launch_colsq(Xcal_bf16, T, K, partial, colsq_out, norm, stream);
     if (e == cudaSuccess)
         e = patchk::launch_score_mask(W_bf16, norm, N, K, shp.tile_n, shp.tile_k, meta_out, loss,
-                                      stream);
+                                      rank, done, stream);
     if (e == cudaSuccess) {
         if (map_in) {
             e = cudaMemcpyAsync(map_out, map_in, sizeof(uint32_t) * ((n_tiles + 31) / 32),
@@ -168,7 +227,7 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
         } else {
             const int64_t n_sp =
                 static_cast<int64_t>(floor(sparse_tile_fraction * static_cast<double>(n_tiles)));
-            e = patchk::launch_select_map(loss, n_tiles, n_sp, rank, map_out, stream);
+            e = patchk::launch_select_map(loss, n_tiles, n_sp, rank, done, map_out, stream);
         }
     }
     cudaError_t e2 = cudaFreeAsync(scratch, stream);
@@ -202,28 +261,33 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     if (e != cudaSuccess) return from_cuda(e);
     auto tile_sparse = [&](int64_t t) { return ((hmap[t / 32] >> (t % 32)) & 1u) != 0; };
 
+    patch_packed *h = new (std::nothrow) patch_packed();
+    if (!h) return PATCH_ERR_OOM;
+    // k-step (b, c) is 2:4 iff the one or two tiles covering its 128 rows (one
+    // tile column, since tk >= 64) are 2:4
+    const int64_t Q = nsteps / 2;
     std::vector<uint64_t> table(static_cast<size_t>(bands * nsteps));
-    std::vector<uint8_t> sparse(static_cast<size_t>(nsteps));
+    h->pair_prefix.assign(static_cast<size_t>(bands * (Q + 1)), 0);
+    const int64_t rows_tiles = kBand / tn;  // 1 or 2
     uint64_t offset = 0;
     int64_t n_sparse = 0, n_meta = 0;
     for (int64_t b = 0; b < bands; ++b) {
+        const int64_t ti0 = (b * kBand) / tn;
+        const uint64_t band_start = offset;
+        bool prev_sparse = false;
         for (int64_t c = 0; c < nsteps; ++c) {
-            bool all = true;
-            for (int64_t ti = (b * kBand) / tn; ti <= (b * kBand + kBand - 1) / tn; ++ti)
-                for (int64_t tj = (c * kStep) / tk; tj <= (c * kStep + kStep - 1) / tk; ++tj)
-                    all = all && tile_sparse(ti * tiles_k + tj);
-            sparse[c] = all;
-        }
-        for (int64_t c = 0; c < nsteps; ++c) {
-            uint64_t entry = 0;
-            if (sparse[c]) {
-                const bool first_of_pair = (c % 2 == 0) || !sparse[c - 1];
-                if (first_of_pair) {
+            const int64_t tj = (c * kStep) / tk;
+            bool sp = tile_sparse(ti0 * tiles_k + tj);
+            if (rows_tiles == 2) sp = sp && tile_sparse((ti0 + 1) * tiles_k + tj);
+            uint64_t entry;
+            if (sp) {
+                entry = patchk::kEntrySparse;
+                if (c % 2 == 0 || !prev_sparse) {  // first 2:4 k-step of its pair
                     offset += patchk::kMetaBlockBytes;
                     entry |= patchk::kEntryMeta;
                     ++n_meta;
                 }
-                entry |= offset | patchk::kEntrySparse;
+                entry |= offset;
                 offset += patchk::kSparseStepBytes;
                 ++n_sparse;
             } else {
@@ -231,11 +295,13 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
                 offset += patchk::kDenseStepBytes;
             }
             table[static_cast<size_t>(b * nsteps + c)] = entry;
+            prev_sparse = sp;
+            if (c % 2 == 1)  // cumulative bytes of the band's pairs, for stream-K balancing
+                h->pair_prefix[static_cast<size_t>(b * (Q + 1) + c / 2 + 1)] =
+                    static_cast<int64_t>(offset - band_start);
         }
     }
 
-    patch_packed *h = new (std::nothrow) patch_packed();
-    if (!h) return PATCH_ERR_OOM;
     cudaGetDevice(&h->device);
     h->shp = shp;
     h->packed_bytes = static_cast<size_t>(offset);
@@ -244,18 +310,24 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     h->num_sms = num_sms;
     h->workspace_bytes = patchk::decode_workspace_bytes(num_sms);
 
-    e = patchk::device_pool(&h->pool);
-    auto alloc = [&](void **ptr, size_t bytes) {
-        if (e == cudaSuccess) e = cudaMallocFromPoolAsync(ptr, bytes, h->pool, stream);
-    };
-    alloc(reinterpret_cast<void **>(&h->packed), h->packed_bytes ? h->packed_bytes : 16);
-    alloc(reinterpret_cast<void **>(&h->table), sizeof(uint64_t) * table.size());
-    alloc(reinterpret_cast<void **>(&h->workspace), h->workspace_bytes);
-    alloc(reinterpret_cast<void **>(&h->status), sizeof(uint32_t) * 4);
-    if (e == cudaSuccess) e = cudaMemsetAsync(h->status, 0, sizeof(uint32_t) * 4, stream);
-    if (e == cudaSuccess)
-        e = cudaMemcpyAsync(h->table, table.data(), sizeof(uint64_t) * table.size(),
-                            cudaMemcpyHostToDevice, stream);
+    // one pool allocation: packed bytes | table | stream-K workspace | status
+    const size_t off_table = round_up(std::max<size_t>(h->packed_bytes, 16), 256);
+    const size_t off_ws = round_up(off_table + sizeof(uint64_t) * table.size(), 256);
+    const size_t off_status = round_up(off_ws + h->workspace_bytes, 256);
+    const size_t total = off_status + 256;
+    cudaError_t e2 = patchk::device_pool(&h->pool);
+    if (e2 == cudaSuccess)
+        e2 = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->base), total, h->pool, stream);
+    if (e2 == cudaSuccess) {
+        h->packed = h->base;
+        h->table = reinterpret_cast<uint64_t *>(h->base + off_table);
+        h->workspace = reinterpret_cast<float *>(h->base + off_ws);
+        h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
+        e2 = cudaMemsetAsync(h->status, 0, sizeof(uint32_t) * 4, stream);
+    }
+    if (e2 == cudaSuccess)
+        e2 = upload_via_pinned(h->table, table.data(), sizeof(uint64_t) * table.size(), stream);
+    e = e2;
     if (e == cudaSuccess)
         e = patchk::launch_pack(W_bf16, meta, map, N, K, static_cast<int>(tn), static_cast<int>(tk),
                                 h->table, h->packed, stream);
@@ -290,6 +362,7 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.pool = Wp->pool;
     g.status = Wp->status;
     g.num_sms = Wp->num_sms;
+    g.pair_prefix = Wp->pair_prefix.data();
     // Failure-detection test hook: with PATCH_B200_TEST_STALL=1 in the
     // environment, CTA 0 never loads its first k-step, so its bounded wait runs
     // out, the kernel returns early and patch_get_status reports the timeout.
@@ -300,11 +373,7 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
 
 void patch_free(patch_packed *Wp, void *stream_v) {
     if (!Wp) return;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
-    if (Wp->packed) cudaFreeAsync(Wp->packed, stream);
-    if (Wp->table) cudaFreeAsync(Wp->table, stream);
-    if (Wp->workspace) cudaFreeAsync(Wp->workspace, stream);
-    if (Wp->status) cudaFreeAsync(Wp->status, stream);
+    if (Wp->base) cudaFreeAsync(Wp->base, static_cast<cudaStream_t>(stream_v));
     delete Wp;
 }
 

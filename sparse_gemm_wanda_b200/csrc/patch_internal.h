@@ -10,10 +10,13 @@ cudaError_t launch_colsq(const void *Xcal, int64_t T, int64_t K, double *partial
                          double *colsq_out, double *norm_out, cudaStream_t stream);
 cudaError_t launch_norms_from_colsq(const double *colsq_in, int64_t K, double *colsq_out,
                                     double *norm_out, cudaStream_t stream);
+// `rank` / `done` (may be null when no map is selected) are zeroed here for
+// launch_select_map, which must follow on the same stream.
 cudaError_t launch_score_mask(const void *W, const double *norm, int64_t N, int64_t K, int tn,
-                              int tk, uint32_t *meta, double *loss, cudaStream_t stream);
+                              int tk, uint32_t *meta, double *loss, int32_t *rank, uint32_t *done,
+                              cudaStream_t stream);
 cudaError_t launch_select_map(const double *loss, int64_t n_tiles, int64_t n_sparse, int32_t *rank,
-                              uint32_t *map, cudaStream_t stream);
+                              uint32_t *done, uint32_t *map, cudaStream_t stream);
 
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                         int64_t K, int tn, int tk, const uint64_t *table, uint8_t *out,
@@ -33,6 +36,7 @@ struct GemmLaunch {
     uint32_t *status;
     int num_sms;
     int stall_first_kstep;   // failure-detection test hook (see patch_hybrid_gemm)
+    const int64_t *pair_prefix;  // host: per band, cumulative packed bytes of its k-pairs
 };
 
 // Picks the configuration (token tile, schedule) for M and launches.

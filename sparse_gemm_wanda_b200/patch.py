@@ -88,7 +88,7 @@ def _check(fn: str, code: int):
 
 def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
-        stream = torch.cuda.current_stream()
+        return ctypes.c_void_p(torch._C._cuda_getCurrentRawStream(torch.cuda.current_device()))
     return ctypes.c_void_p(stream.cuda_stream)
 
 
