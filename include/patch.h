@@ -107,6 +107,43 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
                               double *tile_loss_out, void *stream);
 
 /*
+ * Allocation-free variant of patch_score_mask.  The pages have no
+ * counterpart: this entry point exists for callers that may not allocate
+ * device memory at all, e.g. code running inside a framework whose caching
+ * allocator owns the whole GPU (a cudaMalloc behind its back would fail or
+ * fragment its pool), embedded runtimes that reserve every byte up front, or
+ * paths with hard latency limits where an allocation (which can synchronise
+ * the device) is not allowed.
+ *
+ * Same arguments, outputs and results as patch_score_mask.  The temporary
+ * values (chunk partials of the column sums, norms, and the loss / rank
+ * counters when the caller does not ask for them) live in one fixed array of
+ * device memory inside this library, 16 MiB per device
+ * (patch_score_mask_noalloc_capacity()), held by every device that loads the
+ * library until the process exits.  A call needs
+ * 8*K*ceil(T/128) + 8*K + 8*n_tiles + 4*n_tiles bytes of it (plus alignment;
+ * the last two terms only when tile_loss_out is NULL / map_in is NULL);
+ * larger problems return PATCH_ERR_UNSUPPORTED without launching anything.
+ * It calls no cudaMalloc / cudaFree / pool allocation.
+ *
+ * All calls on a device share the array and it keeps what the last call left
+ * in it; each call writes every value before reading it.  Calls whose GPU
+ * work overlaps (different streams without ordering between them) race on the
+ * array and give wrong results: order them on one stream or with events.
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture begins.
+ */
+patch_status patch_score_mask_noalloc(const void *W_bf16, const void *Xcal_bf16, int64_t T,
+                                      const double *colsq_in, patch_shape shp,
+                                      double sparse_tile_fraction, const uint32_t *map_in,
+                                      uint32_t *meta_out, uint32_t *map_out, double *colsq_out,
+                                      double *tile_loss_out, void *stream);
+
+/* Bytes of the fixed scratch array patch_score_mask_noalloc works in. */
+size_t patch_score_mask_noalloc_capacity(void);
+
+/*
  * Compressor: lay the dense tiles and the 2:4-compressed tiles (kept values +
  * metadata) out for the hybrid GEMM.  Compressed storage is what turns
  * zeros into speed (SparseGPT-vs-Wanda page, section on structured vs

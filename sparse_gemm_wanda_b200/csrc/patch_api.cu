@@ -234,6 +234,91 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
     return from_cuda(e != cudaSuccess ? e : e2);
 }
 
+// ------------------------------------------------------ allocation-free mask
+// Scratch of patch_score_mask_noalloc: a fixed array in device memory that
+// every device loading this library holds until the process exits.  Host code
+// must not pass the symbol itself to a kernel (on the host it is only a
+// stand-in); its device address is looked up once per device below.
+constexpr size_t kNoallocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
+
+static cudaError_t noalloc_scratch_address(uint8_t **ptr) {
+    static std::mutex mu;
+    static std::map<int, uint8_t *> addr;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = addr.find(dev);
+    if (it != addr.end()) {
+        *ptr = it->second;
+        return cudaSuccess;
+    }
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // with `dev` current
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<uint8_t *>(p);
+    *ptr = static_cast<uint8_t *>(p);
+    return cudaSuccess;
+}
+
+patch_status patch_score_mask_noalloc(const void *W_bf16, const void *Xcal_bf16, int64_t T,
+                                      const double *colsq_in, patch_shape shp,
+                                      double sparse_tile_fraction, const uint32_t *map_in,
+                                      uint32_t *meta_out, uint32_t *map_out, double *colsq_out,
+                                      double *tile_loss_out, void *stream_v) {
+    patch_status st = check_shape(shp);
+    if (st != PATCH_OK) return st;
+    if (!W_bf16 || !meta_out || !map_out || !aligned16(W_bf16)) return PATCH_ERR_INVALID_ARG;
+    if (!colsq_in && (!Xcal_bf16 || T < 1 || !aligned16(Xcal_bf16))) return PATCH_ERR_INVALID_ARG;
+    if (!map_in && !(sparse_tile_fraction >= 0.0 && sparse_tile_fraction <= 1.0))
+        return PATCH_ERR_INVALID_ARG;
+    const int64_t N = shp.N, K = shp.K;
+    const int64_t n_tiles = (N / shp.tile_n) * (K / shp.tile_k);
+    const int64_t chunks = colsq_in ? 0 : (T + 127) / 128;
+    // same scratch layout as patch_score_mask, inside the fixed array
+    const size_t off_norm = round_up(sizeof(double) * static_cast<size_t>(chunks * K), 256);
+    const size_t off_loss = round_up(off_norm + sizeof(double) * K, 256);
+    const size_t off_rank = round_up(off_loss + (tile_loss_out ? 0 : sizeof(double) * n_tiles), 256);
+    const size_t off_done = round_up(off_rank + (map_in ? 0 : sizeof(int32_t) * n_tiles), 256);
+    const size_t total = off_done + 256;
+    if (total > kNoallocScratchBytes) return PATCH_ERR_UNSUPPORTED;  // beyond the fixed scratch
+    st = check_device(nullptr);
+    if (st != PATCH_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    uint8_t *scratch = nullptr;
+    cudaError_t e = noalloc_scratch_address(&scratch);
+    if (e != cudaSuccess) return from_cuda(e);
+    double *partial = reinterpret_cast<double *>(scratch);
+    double *norm = reinterpret_cast<double *>(scratch + off_norm);
+    double *loss = tile_loss_out ? tile_loss_out : reinterpret_cast<double *>(scratch + off_loss);
+    int32_t *rank = map_in ? nullptr : reinterpret_cast<int32_t *>(scratch + off_rank);
+    uint32_t *done = reinterpret_cast<uint32_t *>(scratch + off_done);
+    // every scratch value is written before it is read in this call (the
+    // score kernel zeroes the rank counters), so leftovers of the previous
+    // call do not matter
+    if (colsq_in)
+        e = patchk::launch_norms_from_colsq(colsq_in, K, colsq_out, norm, stream);
+    else
+        e = patchk::launch_colsq(Xcal_bf16, T, K, partial, colsq_out, norm, stream);
+    if (e == cudaSuccess)
+        e = patchk::launch_score_mask(W_bf16, norm, N, K, shp.tile_n, shp.tile_k, meta_out, loss,
+                                      rank, done, stream);
+    if (e == cudaSuccess) {
+        if (map_in) {
+            e = cudaMemcpyAsync(map_out, map_in, sizeof(uint32_t) * ((n_tiles + 31) / 32),
+                                cudaMemcpyDeviceToDevice, stream);
+        } else {
+            const int64_t n_sp =
+                static_cast<int64_t>(floor(sparse_tile_fraction * static_cast<double>(n_tiles)));
+            e = patchk::launch_select_map(loss, n_tiles, n_sp, rank, done, map_out, stream);
+        }
+    }
+    return from_cuda(e);
+}
+
+size_t patch_score_mask_noalloc_capacity(void) { return kNoallocScratchBytes; }
+
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
                         patch_shape shp, patch_packed **out,
                         size_t *packed_bytes, void *stream_v) {

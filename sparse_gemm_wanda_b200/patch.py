@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "PATCH_OK", 1: "PATCH_ERR_INVALID_ARG", 2: "PATCH_ERR_UNSUPPO
 # every symbol include/patch.h declares
 EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
            "patch_get_status", "patch_packed_info", "patch_packed_export",
-           "patch_status_string")
+           "patch_status_string", "patch_score_mask_noalloc",
+           "patch_score_mask_noalloc_capacity")
 
 
 class PatchLibraryError(RuntimeError):
@@ -64,6 +65,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         raise PatchLibraryError(f"cannot load {path}: {exc}") from exc
     vp, i64, i32, dbl = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double
     lib.patch_score_mask.argtypes = [vp, vp, i64, vp, PatchShape, dbl, vp, vp, vp, vp, vp, vp]
+    lib.patch_score_mask_noalloc.argtypes = [vp, vp, i64, vp, PatchShape, dbl, vp, vp, vp, vp, vp,
+                                             vp]
+    lib.patch_score_mask_noalloc.restype = ctypes.c_int
+    lib.patch_score_mask_noalloc_capacity.argtypes = []
+    lib.patch_score_mask_noalloc_capacity.restype = ctypes.c_size_t
     lib.patch_pack.argtypes = [vp, vp, vp, PatchShape, ctypes.POINTER(vp),
                                ctypes.POINTER(ctypes.c_size_t), vp]
     lib.patch_hybrid_gemm.argtypes = [vp, vp, i64, vp, i32, vp]
@@ -129,6 +135,38 @@ def patch_score_mask(W: torch.Tensor, Xcal: torch.Tensor | None = None, *, tile_
         _dptr(tmap), _dptr(colsq), _dptr(loss), _stream(stream))
     _check("patch_score_mask", code)
     return {"meta": meta, "map": tmap, "colsq": colsq, "loss": loss}
+
+
+def patch_score_mask_noalloc(W: torch.Tensor, Xcal: torch.Tensor | None = None, *,
+                             tile_n: int = 128, tile_k: int = 128, fraction: float = 0.0,
+                             map_in: torch.Tensor | None = None,
+                             colsq_in: torch.Tensor | None = None, out: dict | None = None,
+                             stream=None) -> dict:
+    """patch_score_mask without any device allocation inside the library.
+
+    For callers that cannot allocate device memory while they run (the
+    library's scratch is a fixed 16 MiB array per device; see patch.h).  The
+    outputs are the caller's: pass them in `out` (keys "meta", "map" and
+    optionally "colsq", "loss", shaped as patch_score_mask returns them) to
+    keep this call free of allocations on the Python side too.
+    """
+    lib = load_library()
+    N, K = W.shape
+    nt = n_tiles(N, K, tile_n, tile_k)
+    if out is None:
+        dev = W.device
+        out = {"meta": torch.empty((N, K // 32), dtype=torch.int32, device=dev),
+               "map": torch.empty(((nt + 31) // 32,), dtype=torch.int32, device=dev),
+               "colsq": None, "loss": None}
+    T = Xcal.shape[0] if Xcal is not None else 0
+    code = lib.patch_score_mask_noalloc(
+        _dptr(W, torch.bfloat16, "W"), _dptr(Xcal, torch.bfloat16, "Xcal"), T,
+        _dptr(colsq_in, torch.float64, "colsq_in"), PatchShape(N, K, tile_n, tile_k),
+        float(fraction), _dptr(map_in, (torch.int32, torch.uint32), "map_in"),
+        _dptr(out["meta"]), _dptr(out["map"]), _dptr(out.get("colsq")), _dptr(out.get("loss")),
+        _stream(stream))
+    _check("patch_score_mask_noalloc", code)
+    return out
 
 
 class PackedWeight:
