@@ -246,6 +246,13 @@ patch_status patch_packed_info(const patch_packed *Wp, patch_packed_view *view);
 patch_status patch_packed_export(const patch_packed *Wp, void *packed_dst, uint64_t *table_dst,
                                  void *stream);
 
+/*
+ * Number of kernels this library has enqueued in this process, on any stream
+ * and device (a monotonically increasing count; read it before and after a
+ * region to count that region's launches).  Diagnostics only; no device work.
+ */
+uint64_t patch_launch_count(void);
+
 /* Human-readable name of a status code (static string). */
 const char *patch_status_string(patch_status s);
 

@@ -582,6 +582,7 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     hybrid_gemm_kernel<BN, STAGES>
         <<<static_cast<unsigned>(grid), kGemmThreads, C::kSmemBytes, stream>>>(map, p);
     cudaError_t err = cudaGetLastError();
+    if (err == cudaSuccess) note_launches(1);
     if (err == cudaSuccess && sk) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>((BN * kBand + 255) / 256), static_cast<unsigned>(tiles));
@@ -595,6 +596,7 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
         cfg.numAttrs = 1;
         err = cudaLaunchKernelEx(&cfg, streamk_reduce_kernel<BN>, static_cast<const float *>(ws), p,
                                  static_cast<int>(grid));
+        if (err == cudaSuccess) note_launches(1);
     }
     if (ws && ws != g.workspace) {
         cudaError_t e2 = cudaFreeAsync(ws, stream);

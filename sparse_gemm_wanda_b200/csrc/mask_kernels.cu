@@ -265,6 +265,7 @@ cudaError_t launch_colsq(const void *Xcal, int64_t T, int64_t K, double *partial
                                                              K, partial);
     colsq_final_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, stream>>>(
         partial, chunks, K, colsq_out, norm_out);
+    note_launches(2);
     return cudaGetLastError();
 }
 
@@ -272,6 +273,7 @@ cudaError_t launch_norms_from_colsq(const double *colsq_in, int64_t K, double *c
                                     double *norm_out, cudaStream_t stream) {
     norms_from_colsq_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, stream>>>(
         colsq_in, K, colsq_out, norm_out);
+    note_launches(1);
     return cudaGetLastError();
 }
 
@@ -291,6 +293,7 @@ cudaError_t launch_score_mask(const void *W, const double *norm, int64_t N, int6
         score_mask_kernel<64, 64><<<g, 128, 0, stream>>>(w, norm, N, K, meta, loss, rank, done);
     else
         return cudaErrorInvalidValue;
+    note_launches(1);
     return cudaGetLastError();
 }
 
@@ -299,6 +302,7 @@ cudaError_t launch_select_map(const double *loss, int64_t n_tiles, int64_t n_spa
     dim3 grid(static_cast<unsigned>((n_tiles + kRankThreads - 1) / kRankThreads),
               static_cast<unsigned>((n_tiles + kRankSlice - 1) / kRankSlice));
     rank_tiles_kernel<<<grid, kRankThreads, 0, stream>>>(loss, n_tiles, n_sparse, rank, done, map);
+    note_launches(1);
     return cudaGetLastError();
 }
 

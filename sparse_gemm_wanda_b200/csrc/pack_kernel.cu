@@ -120,6 +120,7 @@ cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map
     const int64_t blocks = (N / kBand) * (K / kStep);
     pack_kernel<<<static_cast<unsigned>(blocks), kPackThreads, 0, stream>>>(
         static_cast<const uint16_t *>(W), meta, map, N, K, tn, tk, table, out);
+    note_launches(1);
     return cudaGetLastError();
 }
 

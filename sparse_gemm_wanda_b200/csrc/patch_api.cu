@@ -1,6 +1,7 @@
 // C ABI of the tile-hybrid sparse linear layer: argument checks, planning of
 // the packed layout, device memory of the packed handle, kernel launches.
 // Declarations and the normative description of every call: include/patch.h.
+#include <atomic>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -161,6 +162,13 @@ cudaError_t device_pool(cudaMemPool_t *pool) {
 
 }  // namespace patchk
 
+namespace patchk {
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+void note_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+}  // namespace patchk
+
 extern "C" {
 
 const char *patch_status_string(patch_status s) {
@@ -318,6 +326,8 @@ patch_status patch_score_mask_noalloc(const void *W_bf16, const void *Xcal_bf16,
 }
 
 size_t patch_score_mask_noalloc_capacity(void) { return kNoallocScratchBytes; }
+
+uint64_t patch_launch_count(void) { return patchk::g_launches.load(std::memory_order_relaxed); }
 
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
                         patch_shape shp, patch_packed **out,

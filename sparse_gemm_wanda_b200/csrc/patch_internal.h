@@ -6,6 +6,9 @@
 
 namespace patchk {
 
+// Counts kernels enqueued by the library (exported as patch_launch_count).
+void note_launches(int n);
+
 cudaError_t launch_colsq(const void *Xcal, int64_t T, int64_t K, double *partial,
                          double *colsq_out, double *norm_out, cudaStream_t stream);
 cudaError_t launch_norms_from_colsq(const double *colsq_in, int64_t K, double *colsq_out,

@@ -50,6 +50,23 @@ def activations(T: int, K: int, seed: int, outliers: torch.Tensor | None,
     return x.to(torch.bfloat16)
 
 
+def activations_chunked(T: int, K: int, seed: int, outliers: torch.Tensor | None,
+                        role: int = 0, chunk: int = 16384, out: torch.Tensor | None = None
+                        ) -> torch.Tensor:
+    """Large activation sets drawn in blocks of ``chunk`` tokens.
+
+    Block c is ``activations(rows, K, seed, outliers, role + 100000 * c)``, so
+    the first block of a set equals the unchunked draw of the same role and
+    peak host memory stays at one fp32 block.
+    """
+    if out is None:
+        out = torch.empty((T, K), dtype=torch.bfloat16)
+    for c, t0 in enumerate(range(0, T, chunk)):
+        rows = min(chunk, T - t0)
+        out[t0:t0 + rows] = activations(rows, K, seed, outliers, role=role + 100000 * c)
+    return out
+
+
 def random_map(n_tiles: int, n_sparse: int, seed: int) -> torch.Tensor:
     """Bitmap words (int32 holding the uint32 bit patterns) with exactly n_sparse bits set.
 
@@ -65,9 +82,16 @@ def random_map(n_tiles: int, n_sparse: int, seed: int) -> torch.Tensor:
 
 @dataclass
 class Matrix:
+    """One linear layer W[N, K]; layers with the same ``group`` read the same
+    input activations (q/k/v share one input, gate/up another)."""
     name: str
     N: int
     K: int
+    group: str = ""
+
+    @property
+    def input_group(self) -> str:
+        return self.group or f"in{self.K}"
 
 
 @dataclass
@@ -93,9 +117,10 @@ class Workload:
 
 def workloads() -> dict:
     """The five named workloads (tiny check, decode, prefill sweep, 13B prefill, block)."""
-    L7 = [Matrix("q", 4096, 4096), Matrix("k", 4096, 4096), Matrix("v", 4096, 4096),
-          Matrix("o", 4096, 4096), Matrix("gate", 11008, 4096), Matrix("up", 11008, 4096),
-          Matrix("down", 4096, 11008)]
+    L7 = [Matrix("q", 4096, 4096, "attn_in"), Matrix("k", 4096, 4096, "attn_in"),
+          Matrix("v", 4096, 4096, "attn_in"), Matrix("o", 4096, 4096, "attn_out"),
+          Matrix("gate", 11008, 4096, "mlp_in"), Matrix("up", 11008, 4096, "mlp_in"),
+          Matrix("down", 4096, 11008, "mlp_mid")]
     return {
         "tiny": Workload("tiny", 0, [Matrix("w", 256, 256)], 64, 64, 64, [8], [0.5], "random",
                          outlier_count=3,

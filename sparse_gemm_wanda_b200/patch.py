@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "PATCH_OK", 1: "PATCH_ERR_INVALID_ARG", 2: "PATCH_ERR_UNSUPPO
 EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
            "patch_get_status", "patch_packed_info", "patch_packed_export",
            "patch_status_string", "patch_score_mask_noalloc",
-           "patch_score_mask_noalloc_capacity")
+           "patch_score_mask_noalloc_capacity", "patch_launch_count")
 
 
 class PatchLibraryError(RuntimeError):
@@ -70,6 +70,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.patch_score_mask_noalloc.restype = ctypes.c_int
     lib.patch_score_mask_noalloc_capacity.argtypes = []
     lib.patch_score_mask_noalloc_capacity.restype = ctypes.c_size_t
+    lib.patch_launch_count.argtypes = []
+    lib.patch_launch_count.restype = ctypes.c_uint64
     lib.patch_pack.argtypes = [vp, vp, vp, PatchShape, ctypes.POINTER(vp),
                                ctypes.POINTER(ctypes.c_size_t), vp]
     lib.patch_hybrid_gemm.argtypes = [vp, vp, i64, vp, i32, vp]
@@ -85,6 +87,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued so far in this process."""
+    return int(load_library().patch_launch_count())
 
 
 def _check(fn: str, code: int):

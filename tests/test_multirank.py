@@ -29,7 +29,7 @@ def _worker(rank, world, port, out):
         mats, calib = bench.make_tensors(wl, rank)
         w = mats[0]["W"].float()
         digest = torch.tensor([w.sum().item(), w.abs().sum().item(),
-                               calib[256].float().sum().item()], dtype=torch.float64)
+                               calib["in256"].float().sum().item()], dtype=torch.float64)
         gathered = [torch.zeros(3, dtype=torch.float64) for _ in range(world)]
         dist.all_gather(gathered, digest)
         mx = bench.max_over_ranks(1.5 + rank, "cpu")

@@ -1,0 +1,192 @@
+"""Full-size parity for the 13B-shaped prefill and the whole 7B-shaped block.
+
+Both run at the sizes the benchmark uses, through the C ABI, against the
+oracle on the same seeded inputs:
+
+* 13B prefill: W 13824x5120 and 5120x13824, 128x128 tiles, every tile 2:4
+  (50 % sparsity) and a seeded random map with 75 % of the tiles 2:4 (37.5 %);
+  2:4 patterns from Wanda with the input X (4096 tokens) as calibration set.
+  Codes, map, packed bytes and k-step table bit-exact; GEMM on sampled
+  outputs the oracle computes one dot product at a time.
+* block: q, k, v, o (4096x4096), gate, up (11008x4096), down (4096x11008);
+  Wanda masks from 128 x 2048 = 262144 calibration tokens per distinct layer
+  input (q/k/v share one, gate/up another); per-matrix map of the 2:4 tiles
+  with the least pruned-score loss at 30 % target sparsity (60 % of tiles);
+  GEMM at M in {1, 8, 64, 512, 4096} (M <= 16 takes the split-K path).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_gemm_wanda_b200 import inputs
+from tests.conftest import bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU machines, skipped there
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+TOL_NOTE = "fp32: max err <= 1e-2 RMS; bf16: + half an ulp of the output per element"
+
+
+@pytest.fixture(scope="module")
+def P():
+    from sparse_gemm_wanda_b200 import build, patch
+    build.build()
+    oracle.build()
+    patch.load_library()
+    return patch
+
+
+def u32(t):
+    return t.cpu().numpy().view(np.uint32)
+
+
+def check_close(y, yref, fp32_mode):
+    y = y.double().cpu().numpy()
+    rms = float(np.sqrt(np.mean(yref ** 2)))
+    err = np.abs(y - yref)
+    if fp32_mode:
+        assert err.max() <= 1e-2 * rms, (float(err.max()), rms, TOL_NOTE)
+    else:
+        mag = np.maximum(np.abs(y), np.abs(yref))
+        ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-30))) - 7)
+        bad = err > 1e-2 * rms + 0.5 * ulp
+        assert not bad.any(), (int(bad.sum()), float(err.max()), rms, TOL_NOTE)
+
+
+def sampled_check(y, x_bits, weff, n_samples, seed, fp32_mode):
+    M, N = y.shape
+    g = np.random.default_rng(seed)
+    ms = g.integers(0, M, n_samples)
+    ns = g.integers(0, N, n_samples)
+    # always include the four corners: first/last token and output channel
+    ms = np.concatenate([ms, [0, 0, M - 1, M - 1]])
+    ns = np.concatenate([ns, [0, N - 1, 0, N - 1]])
+    yref = oracle.gemm_at(x_bits, weff, ms, ns)
+    ys = y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()]
+    check_close(ys, yref, fp32_mode)
+
+
+def check_pack(pk, w_bits, meta, tmap, tn, tk):
+    packed, table = pk.export()
+    torch.cuda.synchronize()
+    ref_packed, ref_table = oracle.pack(w_bits, meta, tmap, tn, tk)
+    assert pk.packed_bytes == ref_packed.size
+    assert np.array_equal(table.cpu().numpy().view(np.uint64), ref_table)
+    assert np.array_equal(packed.cpu().numpy(), ref_packed)
+
+
+# ------------------------------------------------------------- 13B prefill
+
+@pytest.mark.parametrize("N,K", [(13824, 5120), (5120, 13824)])
+@pytest.mark.parametrize("frac", [1.0, 0.75])
+def test_13b_prefill_config(P, N, K, frac):
+    wl = inputs.workloads()["llama13b-prefill"]
+    seed = wl.seed + N
+    M = 4096
+    w = inputs.weight(N, K, seed)
+    o = inputs.outlier_channels(K, wl.seed)
+    x = inputs.activations(M, K, wl.seed, o, role=1)
+    nt = (N // 128) * (K // 128)
+    tmap = inputs.random_map(nt, inputs.n_sparse_tiles(frac, nt), seed)
+    wd, xd = w.cuda(), x.cuda()
+    r = P.patch_score_mask(wd, xd, map_in=tmap.cuda(), want_colsq=True, want_loss=True)
+    pk = P.patch_pack(wd, r["meta"], r["map"])
+    y = P.patch_hybrid_gemm(pk, xd)
+    torch.cuda.synchronize()
+    assert P.patch_get_status(pk) == 0
+
+    wb, xb = bf16_bits(w), bf16_bits(x)
+    tm = tmap.numpy().view(np.uint32)
+    ref = oracle.score_mask(wb, xb, 128, 128, tile_map=tm)
+    assert np.array_equal(r["colsq"].cpu().numpy(), ref["colsq"])
+    assert np.array_equal(u32(r["meta"]), ref["meta"])
+    assert np.array_equal(r["loss"].cpu().numpy(), ref["loss"])
+    assert np.array_equal(u32(r["map"]), ref["map"])
+    check_pack(pk, wb, ref["meta"], tm, 128, 128)
+    # achieved sparsity of W_eff is half the fraction of 2:4 tiles
+    weff = oracle.weff(wb, ref["meta"], tm, 128, 128)
+    zero = float(np.mean(weff == 0))
+    assert abs(zero - frac / 2) < 2e-3, zero
+    sampled_check(y, xb, weff, 6000, seed, fp32_mode=False)
+    pk.close()
+
+
+# -------------------------------------------------------------------- block
+
+@pytest.fixture(scope="module")
+def block():
+    """Weights, calibration sets and inputs of the 7B-shaped decoder block,
+    drawn once for the module (about 12 GB of calibration tokens)."""
+    wl = inputs.workloads()["llama7b-block"]
+    seed = wl.seed
+    outl = {}
+    calib = {}
+    mats = []
+    for mi, m in enumerate(wl.matrices):
+        if m.K not in outl:
+            outl[m.K] = inputs.outlier_channels(m.K, seed)
+        g = m.input_group
+        if g not in calib:
+            buf = torch.empty((wl.calib_tokens, m.K), dtype=torch.bfloat16)
+            inputs.activations_chunked(wl.calib_tokens, m.K, seed, outl[m.K],
+                                       role=10 * len(calib), out=buf)
+            calib[g] = buf
+        mats.append((m, inputs.weight(m.N, m.K, seed + 17 * (mi + 1))))
+    return wl, mats, calib, outl
+
+
+def test_block_config(P, block):
+    wl, mats, calib, outl = block
+    frac = wl.fractions[0]
+    colsq_dev = {}
+    colsq_ref = {}
+    for mi, (m, w) in enumerate(mats):
+        g = m.input_group
+        wd = w.cuda()
+        first = g not in colsq_dev
+        if first:
+            xc = calib[g].cuda()
+            r = P.patch_score_mask(wd, xc, fraction=frac, want_colsq=True, want_loss=True)
+            colsq_dev[g] = r["colsq"]
+            del xc
+            colsq_ref[g] = oracle.colsq(bf16_bits(calib[g]))
+        else:
+            # later layers of the group reuse the column norms of the first
+            r = P.patch_score_mask(wd, None, fraction=frac, colsq_in=colsq_dev[g],
+                                   want_loss=True)
+        pk = P.patch_pack(wd, r["meta"], r["map"])
+        torch.cuda.synchronize()
+
+        wb = bf16_bits(w)
+        if first:
+            assert np.array_equal(r["colsq"].cpu().numpy(), colsq_ref[g]), m.name
+        sc = oracle.wanda_scores(wb, colsq_ref[g])
+        meta = oracle.select_2of4(sc)
+        loss = oracle.tile_loss(sc, meta, 128, 128)
+        nt = loss.shape[0]
+        tmap = oracle.select_map(loss, oracle.n_sparse(frac, nt))
+        assert np.array_equal(u32(r["meta"]), meta), m.name
+        assert np.array_equal(r["loss"].cpu().numpy(), loss), m.name
+        assert np.array_equal(u32(r["map"]), tmap), m.name
+        # 30 % target sparsity: floor(0.6 * tiles) tiles 2:4
+        assert sum(bin(int(v)).count("1") for v in tmap) == oracle.n_sparse(frac, nt)
+        check_pack(pk, wb, meta, tmap, 128, 128)
+
+        weff = oracle.weff(wb, meta, tmap, 128, 128)
+        for M in wl.tokens:
+            x = inputs.activations(M, m.K, wl.seed, outl[m.K], role=1 + mi * 100 + M)
+            xb = bf16_bits(x)
+            y = P.patch_hybrid_gemm(pk, x.cuda())
+            torch.cuda.synchronize()
+            if M <= 8:
+                check_close(y, oracle.gemm(xb, weff), fp32_mode=False)
+                y32 = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+                torch.cuda.synchronize()
+                check_close(y32, oracle.gemm(xb, weff), fp32_mode=True)
+            else:
+                sampled_check(y, xb, weff, 3000, seed=M + mi, fp32_mode=False)
+        assert P.patch_get_status(pk) == 0
+        pk.close()
