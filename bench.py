@@ -536,7 +536,7 @@ def main():
         ach = b_call / (ms_call * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
                 "frac": ach / hbm_peak, "traffic": traffic_for("hybrid_gemm_decode"),
-                "kernel": "hybrid_gemm_kernel<16,5> (+ stream-K reduce)",
+                "kernel": "decode_gemm_kernel (+ decode_reduce_kernel)",
                 "algorithmic_bytes_per_launch": b_call, "launch_us": ms_call * 1e3,
                 "launches_per_call": l_call,
                 "timing": f"CUDA events around a graph of the step's decode GEMMs cycling "

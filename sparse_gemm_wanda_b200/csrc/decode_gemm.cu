@@ -1,0 +1,527 @@
+// Split-K hybrid GEMV for decode (M <= 16 tokens) on the sm_100a tensor cores.
+//
+// Same product as the prefill kernel, Y = X * W_eff^T with dense k-steps on
+// tcgen05.mma and 2:4 k-steps on tcgen05.mma.sp ("PATCH: Learnable Tile-level
+// Hybrid Sparsity for LLMs", section 2, inference and deployment), shaped for
+// the case where the weights are read once and the run is bound by HBM.
+//
+// Work.  Every 128-row band of W is cut into chunks of `cp` consecutive
+// k-pairs (128 input columns each).  CTA c first runs chunk c, then claims
+// further chunks from an atomic counter, so SMs that stream faster take more
+// chunks and no CTA's static share decides the end of the kernel.  Each
+// chunk leaves its 16 x 128 fp32 partial in its own slot; a fix-up kernel adds
+// the chunks of a band in chunk order, so Y does not depend on which CTA ran
+// which chunk.  No CTA ever waits for another.
+//
+// Copies.  A chunk's pairs are contiguous in the packed buffer; the chunk
+// descriptor (byte offset + the 2:4 flags of its k-steps) is enough to place
+// every k-step, so no table is read: the descriptors of the CTAs' first
+// chunks travel in the kernel parameters and the first copies start at once.
+// One bulk copy per pair (16-32 KB) and one 3-D TMA load of the pair's X
+// tiles (16 rows, rows past M read as zero) complete on the stage mbarrier.
+//
+// Launch.  A programmatic dependent of the previous kernel: once the packer's
+// ready flag is seen, the first chunk's weight copies are issued before
+// `griddepcontrol.wait`; X, Y, the partials and the chunk counter are touched
+// only after it.  The fix-up kernel resets the counter for the next call.
+//
+// Roles (192 threads): warp 0 lane 0 producer, warp 1 lane 0 MMA issuer,
+// warps 2..5 epilogue (tcgen05.ld of the 16-column accumulator, fp32 partial
+// stores).  Two accumulators alternate between consecutive chunks.  Every
+// mbarrier wait is bounded by %globaltimer.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "patch_common.cuh"
+#include "patch_internal.h"
+
+namespace patchk {
+
+namespace {
+
+constexpr int kDecThreads = 192;
+constexpr int kDecBN = 16;                                // token rows of the MMA (N = 16)
+constexpr int kDecStages = 5;
+constexpr int kDecABytes = 2 * kDenseStepBytes;           // a pair of packed k-steps, at most
+constexpr int kDecBBytes = 2 * kDecBN * kStep * 2;        // the pair's two X tiles
+constexpr int kDecStageBytes = kDecABytes + kDecBBytes;   // 36864
+constexpr int kDecTmemCols = 64;                          // 2 x 16 accumulator + 4 metadata
+constexpr uint32_t kDecEcol = 2 * kDecBN;
+constexpr int kDecSmemBytes = kDecStages * kDecStageBytes + 1024 + 512;
+constexpr uint64_t kDecWaitLimitNs = 2000000000ull;       // 2 s per wait
+
+constexpr uint32_t kTagDone = 1u << 31;   // no more work
+constexpr uint32_t kTagFirst = 1u << 30;  // first pair of its chunk
+constexpr uint32_t kTagLast = 1u << 29;   // last pair of its chunk
+constexpr uint32_t kTagChunk = (1u << 29) - 1;
+
+// chunk descriptor: first byte (40 bits) | 2:4 flag of each k-step (16) | pairs (4)
+constexpr uint64_t kDescOffsetMask = (1ull << 40) - 1;
+constexpr int kDescFlagsShift = 40;
+constexpr int kDescPairsShift = 56;
+constexpr int kDecMaxChunkPairs = 8;
+
+struct DecodeParams {
+    const uint8_t *packed;
+    const uint64_t *chunk_desc;  // [nchunks]
+    int64_t N, K, M;
+    int cpb;      // chunks per band
+    int cp;       // k-pairs per chunk (the last chunk of a band may hold fewer)
+    int nchunks;
+    void *Y;
+    int y_fp32;
+    float *partial;     // [nchunks][16][128]
+    uint32_t *counter;  // chunks claimed beyond the first gridDim.x; zero between calls
+    uint32_t *status;
+    const uint32_t *ready;
+    int stall_first_kstep;  // failure-detection test hook
+    uint64_t first_desc[kDecMaxCtas];  // chunk_desc[c] for c < gridDim.x
+};
+
+// Place pair i of a chunk: its table-equivalent entries, first byte and size.
+// Mirrors the packer: a 2 KB metadata block precedes the first 2:4 k-step of
+// every k-pair.
+__device__ __forceinline__ void chunk_pair(uint64_t &cur, uint32_t flags, int i, uint64_t &e0,
+                                           uint64_t &e1, uint64_t &first, uint32_t &bytes) {
+    const bool s0 = (flags >> (2 * i)) & 1u, s1 = (flags >> (2 * i + 1)) & 1u;
+    first = cur;
+    if (s0) {
+        cur += kMetaBlockBytes;
+        e0 = kEntrySparse | kEntryMeta | cur;
+        cur += kSparseStepBytes;
+    } else {
+        e0 = cur;
+        cur += kDenseStepBytes;
+    }
+    if (s1) {
+        uint64_t m = 0;
+        if (!s0) {
+            cur += kMetaBlockBytes;
+            m = kEntryMeta;
+        }
+        e1 = kEntrySparse | m | cur;
+        cur += kSparseStepBytes;
+    } else {
+        e1 = cur;
+        cur += kDenseStepBytes;
+    }
+    bytes = static_cast<uint32_t>(cur - first);
+}
+
+__device__ __forceinline__ void store_out(const DecodeParams &p, int64_t idx, float v) {
+    if (p.y_fp32)
+        static_cast<float *>(p.Y)[idx] = v;
+    else
+        static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
+}
+
+__global__ void __launch_bounds__(kDecThreads, 1)
+decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ DecodeParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kDecStages * kDecStageBytes);
+    uint64_t *empty = full + kDecStages;
+    uint64_t *acc_full = empty + kDecStages;  // [2] MMA commit + the MMA thread's arrive
+    uint64_t *acc_empty = acc_full + 2;       // [2] one arrive per epilogue warp
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    volatile uint32_t *abort_flag = tmem_slot + 1;  // raised by any role that gives up
+    volatile uint32_t *never_flag = tmem_slot + 2;  // stays 0: time-only bounded waits
+    volatile int32_t *acc_chunk = reinterpret_cast<volatile int32_t *>(tmem_slot + 4);  // [2]
+    uint64_t *stage_info = reinterpret_cast<uint64_t *>(tmem_slot + 8);                 // [STAGES][3]
+    uint32_t *stage_tag = reinterpret_cast<uint32_t *>(stage_info + 3 * kDecStages);    // [STAGES]
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    bool waited = true;  // thread 0: past griddepcontrol.wait
+
+    if (threadIdx.x == 0) {
+        pdl_trigger();
+        // the packed bytes are final once the ready flag is seen; otherwise
+        // (the packer may be the kernel just before) wait first
+        if (ld_acquire_gpu(p.ready) == 0u) pdl_wait();
+        else waited = false;
+        for (int s = 0; s < kDecStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 2);
+            mbar_init(&acc_empty[b], 4);
+        }
+        *never_flag = 0u;
+        *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kDecTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) prefetch_tmap(&tmap_x);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+
+    if (warp == 0) {
+        if (lane == 0 && !skip) {
+            // ------------------------------------------------------ producer
+            int it = 0;  // pairs armed so far (stage ring position)
+            bool ok = true;
+            int pend_s[kDecStages], pend_pr[kDecStages];  // X tiles of stages armed before the wait
+            int npend = 0;
+            auto flush_x = [&]() {
+                pdl_wait();
+                waited = true;
+                for (int q = 0; q < npend; ++q)
+                    tma_load_3d(smem + pend_s[q] * kDecStageBytes + kDecABytes, &tmap_x, 0, 0,
+                                2 * pend_pr[q], &full[pend_s[q]]);
+                npend = 0;
+            };
+            // the next two claimed chunks (claimed only past the wait)
+            int ja = 0, jb = 0;
+            uint64_t da = 0, db = 0;
+            auto claim = [&](int &jj, uint64_t &dd) {
+                jj = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(p.counter, 1u));
+                dd = (jj < p.nchunks) ? __ldcg(p.chunk_desc + jj) : 0ull;
+            };
+            bool claimed = false;
+            if (waited) {
+                claim(ja, da);
+                claim(jb, db);
+                claimed = true;
+            }
+            int j = blockIdx.x;
+            uint64_t d = p.first_desc[blockIdx.x];
+            while (ok && j < p.nchunks) {
+                const int pr0 = (j % p.cpb) * p.cp;
+                const int np = static_cast<int>((d >> kDescPairsShift) & 0xFu);
+                const uint32_t flags = static_cast<uint32_t>((d >> kDescFlagsShift) & 0xFFFFu);
+                uint64_t cur = d & kDescOffsetMask;
+                for (int i = 0; i < np; ++i) {
+                    const int s = it % kDecStages;
+                    const uint32_t ph = (it / kDecStages) & 1u;
+                    if (!waited && it >= kDecStages) flush_x();
+                    if (it >= kDecStages &&
+                        !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kDecWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    uint64_t e0, e1, first;
+                    uint32_t bytes;
+                    chunk_pair(cur, flags, i, e0, e1, first, bytes);
+                    stage_info[3 * s + 0] = e0;
+                    stage_info[3 * s + 1] = e1;
+                    stage_info[3 * s + 2] = first;
+                    stage_tag[s] = static_cast<uint32_t>(j) | (i == 0 ? kTagFirst : 0u) |
+                                   (i == np - 1 ? kTagLast : 0u);
+                    ++it;
+                    if (p.stall_first_kstep && blockIdx.x == 0 && it == 1) continue;  // never lands
+                    uint8_t *st = smem + s * kDecStageBytes;
+                    mbar_arrive_expect_tx(&full[s], bytes + kDecBBytes);
+                    bulk_g2s(st, p.packed + first, bytes, &full[s]);
+                    if (waited) {
+                        tma_load_3d(st + kDecABytes, &tmap_x, 0, 0, 2 * (pr0 + i), &full[s]);
+                    } else {
+                        pend_s[npend] = s;
+                        pend_pr[npend] = pr0 + i;
+                        ++npend;
+                    }
+                }
+                if (!ok) break;
+                if (!waited) flush_x();
+                if (!claimed) {
+                    claim(ja, da);
+                    claim(jb, db);
+                    claimed = true;
+                }
+                j = ja;
+                d = da;
+                ja = jb;
+                da = db;
+                if (j < p.nchunks) claim(jb, db);
+            }
+            if (!waited) flush_x();
+            if (ok) {
+                // no more chunks: a stage carrying the done tag (plain arrive)
+                const int s = it % kDecStages;
+                const uint32_t ph = (it / kDecStages) & 1u;
+                if (it >= kDecStages &&
+                    !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kDecWaitLimitNs)) {
+                    ok = false;
+                } else {
+                    stage_tag[s] = kTagDone;
+                    mbar_arrive(&full[s]);
+                    ++it;
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1u;
+                atomicOr(p.status, kStatusTimeout);
+            }
+            // Drain: the last phase armed on every stage must have landed
+            // before the CTA exits (a no-op when the MMA thread consumed all).
+            for (int q = (it > kDecStages ? it - kDecStages : 0); q < it; ++q) {
+                if (p.stall_first_kstep && blockIdx.x == 0 && q == 0) continue;  // never armed
+                mbar_wait_bounded(&full[q % kDecStages], (q / kDecStages) & 1u, never_flag,
+                                  kDecWaitLimitNs / 4);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && !skip) {
+            // ---------------------------------------------------------- MMA
+            const uint32_t e_tmem = tmem_base + kDecEcol;
+            constexpr uint32_t kIdescDense = idesc_bf16(kDecBN, false);
+            int it = 0, ci = 0;  // stages consumed, chunks finished
+            bool ok = true;
+            for (;;) {
+                const int s = it % kDecStages;
+                const uint32_t ph = (it / kDecStages) & 1u;
+                if (!mbar_wait_bounded(&full[s], ph, abort_flag, kDecWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t tag = stage_tag[s];
+                if (tag & kTagDone) break;
+                const int buf = ci & 1;
+                if ((tag & kTagFirst) && ci >= 2 &&
+                    !mbar_wait_bounded(&acc_empty[buf], ((ci >> 1) & 1u) ^ 1u, abort_flag,
+                                       kDecWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + buf * kDecBN;
+                const uint64_t first = stage_info[3 * s + 2];
+                uint8_t *st = smem + s * kDecStageBytes;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint64_t e = stage_info[3 * s + h];
+                    const uint32_t a_addr =
+                        smem_u32(st + static_cast<uint32_t>((e & kEntryOffsetMask) - first));
+                    const uint32_t b_addr = smem_u32(st + kDecABytes + h * (kDecBBytes / 2));
+                    const bool fresh = (tag & kTagFirst) && h == 0;
+                    if (e & kEntrySparse) {
+                        if (e & kEntryMeta)
+                            tmem_cp_128x128b(e_tmem, smem_desc(a_addr - kMetaBlockBytes, 16, 128,
+                                                               kSwizzleNone));
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const uint64_t ad = smem_desc(a_addr + q * 32, 16, 512, kSwizzle64B);
+                            const uint64_t bd = smem_desc(b_addr + q * 64, 16, 1024, kSwizzle128B);
+                            mma_sparse(d_tmem, ad, bd, e_tmem + 2 * h, idesc_bf16(kDecBN, true, q),
+                                       (fresh && q == 0) ? 0u : 1u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint64_t ad = smem_desc(a_addr + q * 32, 16, 1024, kSwizzle128B);
+                            const uint64_t bd = smem_desc(b_addr + q * 32, 16, 1024, kSwizzle128B);
+                            mma_dense(d_tmem, ad, bd, kIdescDense, (fresh && q == 0) ? 0u : 1u);
+                        }
+                    }
+                }
+                tc_commit(&empty[s]);
+                if (tag & kTagLast) {
+                    acc_chunk[buf] = static_cast<int32_t>(tag & kTagChunk);
+                    tc_commit(&acc_full[buf]);
+                    mbar_arrive(&acc_full[buf]);  // publishes acc_chunk
+                    ++ci;
+                }
+                ++it;
+            }
+            if (!ok) {
+                *abort_flag = 1u;
+                atomicOr(p.status, kStatusTimeout);
+            }
+            // End of work for the epilogue: a phase whose chunk is -1.  Its
+            // commit fires once every MMA issued has completed, so TMEM is
+            // never freed under a running MMA.
+            const int buf = ci & 1;
+            if (ci >= 2)
+                mbar_wait_bounded(&acc_empty[buf], ((ci >> 1) & 1u) ^ 1u, never_flag, kDecWaitLimitNs);
+            acc_chunk[buf] = -1;
+            tc_commit(&acc_full[buf]);
+            mbar_arrive(&acc_full[buf]);
+        }
+    } else if (!skip) {
+        // ------------------------------------------------------- epilogue
+        pdl_wait();  // the partial slots may still be read by an earlier fix-up
+        const int quad = warp % 4;  // TMEM lanes 32*quad .. 32*quad+31
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+        for (int ci = 0;; ++ci) {
+            const int buf = ci & 1;
+            const bool ok = mbar_wait_bounded(&acc_full[buf], (ci >> 1) & 1u, never_flag, kDecWaitLimitNs);
+            tc_fence_after();
+            if (!ok) {
+                *abort_flag = 1u;
+                atomicOr(p.status, kStatusTimeout);
+                break;
+            }
+            const int j = acc_chunk[buf];
+            if (j < 0) break;
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(lane_base + buf * kDecBN, r);
+            tmem_ld_wait();
+            if (*abort_flag == 0) {
+                float *part = p.partial + static_cast<int64_t>(j) * kDecBN * kBand + row;
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    if (q < p.M) part[q * kBand] = __uint_as_float(r[q]);
+            }
+            // the accumulator may be reused as soon as every lane has read it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kDecTmemCols);
+}
+
+// Fix-up: Y[m, band*128 + row] = the band's chunk partials added in chunk
+// order.  Block (band, m), one thread per row.  Launched as a programmatic
+// dependent of the GEMM; resets the chunk counter once the GEMM is complete.
+__global__ void __launch_bounds__(kBand)
+decode_reduce_kernel(const __grid_constant__ DecodeParams p) {
+    if (threadIdx.x == 0) pdl_trigger();  // the next GEMM may start its prologue
+    pdl_wait();
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.counter = 0u;
+    const int band = blockIdx.x, m = blockIdx.y, row = threadIdx.x;
+    const float *src = p.partial + (static_cast<int64_t>(band) * p.cpb * kDecBN + m) * kBand + row;
+    float acc = 0.0f;
+    for (int c0 = 0; c0 < p.cpb; c0 += 8) {
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            v[q] = (c0 + q < p.cpb) ? __ldcg(src + static_cast<int64_t>(c0 + q) * kDecBN * kBand) : 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            if (c0 + q < p.cpb) acc = __fadd_rn(acc, v[q]);
+    }
+    store_out(p, static_cast<int64_t>(m) * p.N + static_cast<int64_t>(band) * kBand + row, acc);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+}  // namespace
+
+void plan_decode_chunks(int64_t bands, int64_t nsteps, int num_sms, int *cp, int *cpb, int *nchunks) {
+    const int64_t Q = nsteps / 2;
+    // four k-pairs (about 100 KB at half 2:4) per chunk: measured on B200
+    // against 1, 2, 6 and 8 for the Llama-7B shapes; smaller chunks cost more
+    // partials and claims than they gain in balance, larger ones lose balance
+    (void)num_sms;
+    const int64_t c = std::min<int64_t>(std::min<int64_t>(4, kDecMaxChunkPairs), Q);
+    *cp = static_cast<int>(c);
+    *cpb = static_cast<int>((Q + c - 1) / c);
+    *nchunks = static_cast<int>(bands * *cpb);
+}
+
+uint64_t decode_chunk_desc(const uint64_t *band_table, int64_t nsteps, int pr0, int np) {
+    const uint64_t e = band_table[2 * pr0];
+    const uint64_t off = (e & kEntryOffsetMask) - ((e & kEntryMeta) ? kMetaBlockBytes : 0);
+    uint64_t flags = 0;
+    for (int i = 0; i < 2 * np; ++i)
+        if (band_table[2 * pr0 + i] & kEntrySparse) flags |= 1ull << i;
+    (void)nsteps;
+    return (off & kDescOffsetMask) | (flags << kDescFlagsShift) |
+           (static_cast<uint64_t>(np) << kDescPairsShift);
+}
+
+size_t decode_workspace_bytes(int nchunks) {
+    return sizeof(float) * static_cast<size_t>(nchunks) * kDecBN * kBand;
+}
+
+cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(decode_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kDecSmemBytes);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorInvalidValue;
+    // X [M,K] viewed as (64 columns, M rows, K/64 k-steps); box = one k-pair
+    // of 16 rows, 128-byte swizzle, rows past M read as zero
+    CUtensorMap map;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kStep), static_cast<cuuint64_t>(g.M),
+                                static_cast<cuuint64_t>(g.K / kStep)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.K) * 2, static_cast<cuuint64_t>(kStep) * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kStep), static_cast<cuuint32_t>(kDecBN), 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(g.X), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    if (!g.chunk_desc || !g.chunk_desc_host || !g.workspace || !g.counter) return cudaErrorInvalidValue;
+    if (decode_workspace_bytes(g.dec_nchunks) > g.workspace_bytes) return cudaErrorInvalidValue;
+
+    DecodeParams p;
+    p.packed = g.packed;
+    p.chunk_desc = g.chunk_desc;
+    p.N = g.N;
+    p.K = g.K;
+    p.M = g.M;
+    p.cpb = g.dec_cpb;
+    p.cp = g.dec_cp;
+    p.nchunks = g.dec_nchunks;
+    p.Y = g.Y;
+    p.y_fp32 = g.y_fp32;
+    p.partial = g.workspace;
+    p.counter = g.counter;
+    p.status = g.status;
+    p.ready = g.ready;
+    p.stall_first_kstep = g.stall_first_kstep;
+    const int grid = std::min(std::min(g.num_sms, g.dec_nchunks), kDecMaxCtas);
+    for (int c = 0; c < kDecMaxCtas; ++c) p.first_desc[c] = c < grid ? g.chunk_desc_host[c] : 0ull;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = kDecSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gemm_kernel, map, p);
+    if (err != cudaSuccess) return err;
+    note_launches(1);
+    cfg.gridDim = dim3(static_cast<unsigned>(g.N / kBand), static_cast<unsigned>(g.M));
+    cfg.blockDim = dim3(kBand);
+    cfg.dynamicSmemBytes = 0;
+    err = cudaLaunchKernelEx(&cfg, decode_reduce_kernel, p);
+    if (err == cudaSuccess) note_launches(1);
+    return err;
+}
+
+}  // namespace patchk

@@ -11,9 +11,18 @@
 //   * whole tiles: tile c, c + P, c + 2P, ... (many tiles per CTA);
 //   * stream-K: the (tile, k-pair) units are cut into P contiguous ranges of
 //     (nearly) equal bytes, one per CTA.  A tile covered by several CTAs leaves fp32
-//     partials; the last of its CTAs to finish (an atomic ticket) adds them in
-//     CTA order and stores Y, so the result does not depend on timing.
+//     partials; a fix-up kernel, launched as a programmatic dependent, adds
+//     them in CTA order and stores Y, so the result does not depend on timing.
 //     No CTA ever waits for another.
+//
+// Launch.  The kernel is launched as a programmatic dependent of the previous
+// kernel of the stream and lets its own successor be scheduled at once.
+// Before `griddepcontrol.wait` it touches only what no earlier kernel can be
+// writing: once the packer has published the handle's ready flag (release /
+// acquire at device scope), the k-step table and the first STAGES pairs of
+// packed weights are fetched ahead of the wait, so the weight stream of one
+// GEMM overlaps the tail of the kernel before it.  X, Y and the partials are
+// touched only after the wait.
 //
 // Roles (192 threads):
 //   * warp 0, one thread: producer.  Per 64-column k-step it reads the table
@@ -89,6 +98,7 @@ struct GemmParams {
     int y_fp32;
     float *partial;  // stream-K: [2 * gridDim.x][BN][128]
     uint32_t *status;
+    const uint32_t *ready;  // set (release) by the packer once the packed bytes are final
     int stall_first_kstep;  // failure-detection test hook: CTA 0 never loads its first k-step
     int32_t u0[kMaxStreamKCtas + 1];  // stream-K: first unit of every CTA (u0[P] = units)
 };
@@ -141,6 +151,13 @@ __device__ __forceinline__ bool get_segment(const GemmParams &p, int c, int i, S
     return true;
 }
 
+__device__ __forceinline__ void store_y(const GemmParams &p, int64_t idx, float v) {
+    if (p.y_fp32)
+        static_cast<float *>(p.Y)[idx] = v;
+    else
+        static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
+}
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmParams p) {
@@ -163,8 +180,15 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int cta = blockIdx.x;
+    // thread 0 (the producer) knows whether it has passed griddepcontrol.wait
+    bool waited = true;
 
     if (threadIdx.x == 0) {
+        pdl_trigger();
+        // the packed weights and table are final once the ready flag is seen;
+        // otherwise (the packer may be the kernel just before) wait first
+        if (ld_acquire_gpu(p.ready) == 0u) pdl_wait();
+        else waited = false;
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -217,6 +241,17 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             bool have = get_segment(p, cta, 0, sg);  // tables 0 and 1 were fetched at start
             bool have_nx = have && get_segment(p, cta, 1, nx);
             int tabs_issued = (have ? 1 : 0) + (have_nx ? 1 : 0);
+            // X tiles of the stages armed before griddepcontrol.wait
+            int pend_s[STAGES], pend_t[STAGES], pend_pr[STAGES];
+            int npend = 0;
+            auto flush_pending = [&]() {
+                pdl_wait();
+                waited = true;
+                for (int j = 0; j < npend; ++j)
+                    tma_load_3d(smem + pend_s[j] * C::kStageBytes + C::kABytes, &tmap_x, 0,
+                                pend_t[j] * BN, 2 * pend_pr[j], &full[pend_s[j]]);
+                npend = 0;
+            };
             for (int i = 0; ok && have; ++i) {
                 const int buf = i & 1;
                 if (!mbar_wait_bounded(&tab_full[buf], (i >> 1) & 1u, abort_flag, kWaitLimitNs)) {
@@ -227,6 +262,7 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                 for (int pr = sg.ks0 / 2; pr < sg.ks1 / 2; ++pr) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1u;
+                    if (!waited && it >= STAGES) flush_pending();
                     if (it >= STAGES && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kWaitLimitNs)) {
                         ok = false;
                         break;
@@ -244,7 +280,14 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     uint8_t *st = smem + s * C::kStageBytes;
                     mbar_arrive_expect_tx(&full[s], bytes + C::kBBytes);
                     bulk_g2s(st, p.packed + first, bytes, &full[s]);
-                    tma_load_3d(st + C::kABytes, &tmap_x, 0, sg.ttile * BN, 2 * pr, &full[s]);
+                    if (waited) {
+                        tma_load_3d(st + C::kABytes, &tmap_x, 0, sg.ttile * BN, 2 * pr, &full[s]);
+                    } else {
+                        pend_s[npend] = s;
+                        pend_t[npend] = sg.ttile;
+                        pend_pr[npend] = pr;
+                        ++npend;
+                    }
                 }
                 // this buffer is free again: fetch the table of segment i + 2
                 sg = nx;
@@ -259,6 +302,7 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     }
                 }
             }
+            if (!waited) flush_pending();
             // table copies still in flight must land before the CTA exits (the
             // latest phase of each buffer)
             for (int j = (tabs_issued > 2 ? tabs_issued - 2 : 0); j < tabs_issued; ++j)
@@ -341,6 +385,7 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         }
     } else if (!skip) {
         // ------------------------------------------------------- epilogue
+        pdl_wait();  // Y and the partials may still be in use by earlier kernels
         const int quad = warp % 4;  // TMEM lanes 32*quad .. 32*quad+31
         const int row = quad * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
@@ -372,17 +417,11 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
 #pragma unroll
                     for (int q = 0; q < 16; ++q)
                         if (c0 + q < m_valid) part[(c0 + q) * kBand + row] = __uint_as_float(r[q]);
-                } else if (p.y_fp32) {
-                    float *y = static_cast<float *>(p.Y);
-#pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        if (c0 + q < m_valid) y[(m_base + c0 + q) * p.N + n] = __uint_as_float(r[q]);
                 } else {
-                    __nv_bfloat16 *y = static_cast<__nv_bfloat16 *>(p.Y);
 #pragma unroll
                     for (int q = 0; q < 16; ++q)
                         if (c0 + q < m_valid)
-                            y[(m_base + c0 + q) * p.N + n] = __float2bfloat16_rn(__uint_as_float(r[q]));
+                            store_y(p, (m_base + c0 + q) * p.N + n, __uint_as_float(r[q]));
                 }
             }
             // the accumulator may be reused as soon as every lane has read it
@@ -391,8 +430,6 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
     }
-    // let a dependent launch (the stream-K reduction) get scheduled
-    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -425,7 +462,8 @@ streamk_reduce_kernel(const float *__restrict__ partial, const __grid_constant__
     }
     __syncthreads();
     const int ns = nslots;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (threadIdx.x == 0) pdl_trigger();  // the next GEMM may start its prologue
+    pdl_wait();
     if (ns == 0) return;
     const int band = static_cast<int>(t / ttiles), ttile = static_cast<int>(t % ttiles);
     const int64_t m_base = static_cast<int64_t>(ttile) * BN;
@@ -554,15 +592,15 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     p.Y = g.Y;
     p.y_fp32 = g.y_fp32;
     p.status = g.status;
+    p.ready = g.ready;
     p.stall_first_kstep = g.stall_first_kstep;
     const int64_t tiles = static_cast<int64_t>(p.bands) * p.ttiles;
     const int64_t slots = static_cast<int64_t>(g.num_sms) * ctas_per_sm;
-    // whole tiles when there are at least two waves of them (or no room for
-    // the stream-K tickets), stream-K otherwise
+    // whole tiles when there are at least two waves of them, stream-K otherwise
     const bool sk = tiles < 2 * slots;
     p.stream_k = sk ? 1 : 0;
     p.units = tiles * (p.nsteps / 2);
-    // stream-K: at most 62 CTAs per tile, so a tile's partials fit the reducer's slot list
+    // stream-K: at most 62 CTAs per tile, so a tile's partials fit the fix-up's slot list
     const int64_t grid = sk ? std::min<int64_t>(std::min<int64_t>(std::min<int64_t>(slots, p.units),
                                                                    62 * tiles),
                                                 kMaxStreamKCtas)
@@ -579,21 +617,25 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
         }
     }
     p.partial = ws;
-    hybrid_gemm_kernel<BN, STAGES>
-        <<<static_cast<unsigned>(grid), kGemmThreads, C::kSmemBytes, stream>>>(map, p);
-    cudaError_t err = cudaGetLastError();
+    // programmatic dependent launch: the prologue and the first weight copies
+    // overlap the previous kernel (see the kernel's comment on what it reads
+    // before griddepcontrol.wait)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, hybrid_gemm_kernel<BN, STAGES>, map, p);
     if (err == cudaSuccess) note_launches(1);
     if (err == cudaSuccess && sk) {
-        cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>((BN * kBand + 255) / 256), static_cast<unsigned>(tiles));
         cfg.blockDim = dim3(256);
         cfg.dynamicSmemBytes = 0;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
         err = cudaLaunchKernelEx(&cfg, streamk_reduce_kernel<BN>, static_cast<const float *>(ws), p,
                                  static_cast<int>(grid));
         if (err == cudaSuccess) note_launches(1);
@@ -607,13 +649,8 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
 
 }  // namespace
 
-size_t decode_workspace_bytes(int num_sms) {
-    // stream-K partials of the M <= 16 configuration: 2 slots per CTA, one CTA per SM
-    return sizeof(float) * static_cast<size_t>(2 * num_sms) * 16 * kBand;
-}
-
 cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
-    if (g.M <= 16) return run<16, 5>(g, 1, stream);   // 36 KB stages
+    if (g.M <= 16) return launch_decode_gemm(g, stream);  // split-K GEMV, csrc/decode_gemm.cu
     if (g.M <= 64) return run<64, 4>(g, 1, stream);   // 48 KB stages
     if (g.M <= 128) return run<128, 3>(g, 1, stream); // 64 KB stages
     return run<160, 3>(g, 1, stream);                 // 72 KB stages

@@ -51,7 +51,8 @@ __device__ __forceinline__ uint32_t kept_pair(uint32_t a, uint32_t b, uint32_t c
 __global__ void __launch_bounds__(kPackThreads)
 pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
             const uint32_t *__restrict__ map, int64_t N, int64_t K, int tn, int tk,
-            const uint64_t *__restrict__ table, uint8_t *__restrict__ out) {
+            const uint64_t *__restrict__ table, uint8_t *__restrict__ out,
+            uint32_t *__restrict__ done, uint32_t *__restrict__ ready) {
     const int64_t nsteps = K / kStep;
     const int64_t b = blockIdx.x / nsteps, c = blockIdx.x % nsteps;
     const uint64_t entry = table[blockIdx.x];
@@ -75,51 +76,63 @@ pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
             }
             reinterpret_cast<uint4 *>(out + off)[u] = v;
         }
-        return;
-    }
-    // 2:4: chunk u = r*4 + ((v/8) ^ ((r%8)/2)) holds the kept values of groups
-    // 4*(v/8) .. 4*(v/8)+3 of the row, two per group in column order
+    } else {
+        // 2:4: chunk u = r*4 + ((v/8) ^ ((r%8)/2)) holds the kept values of groups
+        // 4*(v/8) .. 4*(v/8)+3 of the row, two per group in column order
 #pragma unroll 4
-    for (int u = tid; u < kBand * 4; u += kPackThreads) {
-        const int r = u / 4, v8 = (u % 4) ^ ((r % 8) / 2);
-        const int64_t i = row0 + r, j = col0 + 16 * v8;
-        const uint4 *src = reinterpret_cast<const uint4 *>(W + i * K + j);
-        const uint4 a = __ldg(src), bq = __ldg(src + 1);
-        const uint32_t e[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
-        const uint32_t codes = __ldg(meta + i * words_k + j / 32) >> (4 * ((j % 32) / 4));
-        uint32_t o[4];
+        for (int u = tid; u < kBand * 4; u += kPackThreads) {
+            const int r = u / 4, v8 = (u % 4) ^ ((r % 8) / 2);
+            const int64_t i = row0 + r, j = col0 + 16 * v8;
+            const uint4 *src = reinterpret_cast<const uint4 *>(W + i * K + j);
+            const uint4 a = __ldg(src), bq = __ldg(src + 1);
+            const uint32_t e[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+            const uint32_t codes = __ldg(meta + i * words_k + j / 32) >> (4 * ((j % 32) / 4));
+            uint32_t o[4];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) o[g] = kept_pair(e[2 * g], e[2 * g + 1], (codes >> (4 * g)) & 0xFu);
-        reinterpret_cast<uint4 *>(out + off)[u] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-    if (entry & kEntryMeta) {
-        // The metadata block of k-pair p: line l = m0 + 8*k1 + 16*m2 holds, in
-        // 32-bit word k2, the 16 code bits of rows (m0 + 16*m2) [low half] and
-        // (m0 + 8 + 16*m2) [high half] for pair columns 32*k2 + 16*k1 + [0,16).
-        const int64_t p = c / 2;
-        const int l = tid;
-        const int m0i = l % 8, k1 = (l / 8) % 2, m2 = l / 16;
-        const int64_t ra = row0 + m0i + 16 * m2, rb = ra + 8;
-        uint32_t wv[4];
-#pragma unroll
-        for (int k2 = 0; k2 < 4; ++k2) {
-            const int64_t ks = 2 * p + k2 / 2;
-            const bool sp = (table[b * nsteps + ks] & kEntrySparse) != 0;
-            const uint32_t lo = (__ldg(meta + ra * words_k + 4 * p + k2) >> (16 * k1)) & 0xFFFFu;
-            const uint32_t hi = (__ldg(meta + rb * words_k + 4 * p + k2) >> (16 * k1)) & 0xFFFFu;
-            wv[k2] = sp ? (lo | (hi << 16)) : 0u;
+            for (int g = 0; g < 4; ++g) o[g] = kept_pair(e[2 * g], e[2 * g + 1], (codes >> (4 * g)) & 0xFu);
+            reinterpret_cast<uint4 *>(out + off)[u] = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        reinterpret_cast<uint4 *>(out + off - kMetaBlockBytes)[l] =
-            make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        if (entry & kEntryMeta) {
+            // The metadata block of k-pair p: line l = m0 + 8*k1 + 16*m2 holds, in
+            // 32-bit word k2, the 16 code bits of rows (m0 + 16*m2) [low half] and
+            // (m0 + 8 + 16*m2) [high half] for pair columns 32*k2 + 16*k1 + [0,16).
+            const int64_t p = c / 2;
+            const int l = tid;
+            const int m0i = l % 8, k1 = (l / 8) % 2, m2 = l / 16;
+            const int64_t ra = row0 + m0i + 16 * m2, rb = ra + 8;
+            uint32_t wv[4];
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) {
+                const int64_t ks = 2 * p + k2 / 2;
+                const bool sp = (table[b * nsteps + ks] & kEntrySparse) != 0;
+                const uint32_t lo = (__ldg(meta + ra * words_k + 4 * p + k2) >> (16 * k1)) & 0xFFFFu;
+                const uint32_t hi = (__ldg(meta + rb * words_k + 4 * p + k2) >> (16 * k1)) & 0xFFFFu;
+                wv[k2] = sp ? (lo | (hi << 16)) : 0u;
+            }
+            reinterpret_cast<uint4 *>(out + off - kMetaBlockBytes)[l] =
+                make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+    }
+    // completion: every thread's stores are ordered before the block's ticket;
+    // the last block publishes the ready flag the GEMM reads before its
+    // griddepcontrol.wait
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const uint32_t v = atomicAdd(done, 1u);
+        if (v == gridDim.x - 1) {
+            __threadfence();
+            st_release_gpu(ready, 1u);
+        }
     }
 }
 
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                         int64_t K, int tn, int tk, const uint64_t *table, uint8_t *out,
-                        cudaStream_t stream) {
+                        uint32_t *done, uint32_t *ready, cudaStream_t stream) {
     const int64_t blocks = (N / kBand) * (K / kStep);
     pack_kernel<<<static_cast<unsigned>(blocks), kPackThreads, 0, stream>>>(
-        static_cast<const uint16_t *>(W), meta, map, N, K, tn, tk, table, out);
+        static_cast<const uint16_t *>(W), meta, map, N, K, tn, tk, table, out, done, ready);
     note_launches(1);
     return cudaGetLastError();
 }

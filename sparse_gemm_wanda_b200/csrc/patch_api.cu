@@ -27,9 +27,12 @@ struct patch_packed {
     uint64_t *table;           // (N/128) * (K/64) entries
     int64_t sparse_ksteps;
     int64_t meta_blocks;
-    float *workspace;          // stream-K partials of the M <= 16 configuration
+    float *workspace;          // decode partials (one slot per chunk); reused by stream-K
     size_t workspace_bytes;
-    uint32_t *status;          // device status word
+    uint64_t *chunk_desc;      // device: decode chunk descriptors
+    std::vector<uint64_t> chunk_desc_host;
+    int dec_cp, dec_cpb, dec_nchunks;
+    uint32_t *status;          // device: status word, pack counter, ready flag
     int num_sms;
     cudaMemPool_t pool;
     std::vector<int64_t> pair_prefix;  // per band: cumulative packed bytes of its k-pairs
@@ -400,32 +403,52 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     cudaGetDevice(&h->device);
     h->shp = shp;
     h->packed_bytes = static_cast<size_t>(offset);
+    if (offset >= (1ull << 40)) {  // chunk descriptors hold 40-bit offsets
+        delete h;
+        return PATCH_ERR_UNSUPPORTED;
+    }
     h->sparse_ksteps = n_sparse;
     h->meta_blocks = n_meta;
     h->num_sms = num_sms;
-    h->workspace_bytes = patchk::decode_workspace_bytes(num_sms);
+    // decode GEMV chunks: descriptors from the table just planned
+    patchk::plan_decode_chunks(bands, nsteps, num_sms, &h->dec_cp, &h->dec_cpb, &h->dec_nchunks);
+    h->chunk_desc_host.resize(static_cast<size_t>(h->dec_nchunks));
+    for (int64_t b = 0; b < bands; ++b)
+        for (int c = 0; c < h->dec_cpb; ++c) {
+            const int pr0 = c * h->dec_cp;
+            const int np = static_cast<int>(std::min<int64_t>(h->dec_cp, Q - pr0));
+            h->chunk_desc_host[static_cast<size_t>(b * h->dec_cpb + c)] =
+                patchk::decode_chunk_desc(table.data() + b * nsteps, nsteps, pr0, np);
+        }
+    h->workspace_bytes = patchk::decode_workspace_bytes(h->dec_nchunks);
 
-    // one pool allocation: packed bytes | table | stream-K workspace | status
+    // one pool allocation: packed bytes | table | chunk descriptors | workspace | status
     const size_t off_table = round_up(std::max<size_t>(h->packed_bytes, 16), 256);
-    const size_t off_ws = round_up(off_table + sizeof(uint64_t) * table.size(), 256);
+    const size_t off_chunks = off_table + sizeof(uint64_t) * table.size();  // uploaded with the table
+    const size_t off_ws = round_up(off_chunks + sizeof(uint64_t) * h->chunk_desc_host.size(), 256);
     const size_t off_status = round_up(off_ws + h->workspace_bytes, 256);
-    const size_t total = off_status + 256;
+    const size_t status_bytes = 256;
+    const size_t total = off_status + status_bytes;
     cudaError_t e2 = patchk::device_pool(&h->pool);
     if (e2 == cudaSuccess)
         e2 = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->base), total, h->pool, stream);
     if (e2 == cudaSuccess) {
         h->packed = h->base;
         h->table = reinterpret_cast<uint64_t *>(h->base + off_table);
+        h->chunk_desc = reinterpret_cast<uint64_t *>(h->base + off_chunks);
         h->workspace = reinterpret_cast<float *>(h->base + off_ws);
+        // status word | pack completion counter | ready flag | decode chunk counter
         h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
-        e2 = cudaMemsetAsync(h->status, 0, sizeof(uint32_t) * 4, stream);
+        e2 = cudaMemsetAsync(h->status, 0, status_bytes, stream);
     }
-    if (e2 == cudaSuccess)
+    if (e2 == cudaSuccess) {
+        table.insert(table.end(), h->chunk_desc_host.begin(), h->chunk_desc_host.end());
         e2 = upload_via_pinned(h->table, table.data(), sizeof(uint64_t) * table.size(), stream);
+    }
     e = e2;
     if (e == cudaSuccess)
         e = patchk::launch_pack(W_bf16, meta, map, N, K, static_cast<int>(tn), static_cast<int>(tk),
-                                h->table, h->packed, stream);
+                                h->table, h->packed, h->status + 1, h->status + 2, stream);
     if (e != cudaSuccess) {
         patch_free(h, stream_v);
         return from_cuda(e);
@@ -456,6 +479,13 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.workspace_bytes = Wp->workspace_bytes;
     g.pool = Wp->pool;
     g.status = Wp->status;
+    g.ready = Wp->status + 2;
+    g.counter = Wp->status + 3;
+    g.chunk_desc = Wp->chunk_desc;
+    g.chunk_desc_host = Wp->chunk_desc_host.data();
+    g.dec_cp = Wp->dec_cp;
+    g.dec_cpb = Wp->dec_cpb;
+    g.dec_nchunks = Wp->dec_nchunks;
     g.num_sms = Wp->num_sms;
     g.pair_prefix = Wp->pair_prefix.data();
     // Failure-detection test hook: with PATCH_B200_TEST_STALL=1 in the
@@ -478,6 +508,8 @@ patch_status patch_get_status(const patch_packed *Wp) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess) e = cudaMemcpy(&word, Wp->status, sizeof(word), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && word != 0) e = cudaMemset(Wp->status, 0, sizeof(uint32_t));
+    // a call that gave up may have left decode chunks claimed
+    if (e == cudaSuccess && word != 0) e = cudaMemset(Wp->status + 3, 0, sizeof(uint32_t));
     if (e != cudaSuccess) return from_cuda(e);
     return (word & patchk::kStatusTimeout) ? PATCH_ERR_TIMEOUT : PATCH_OK;
 }

@@ -21,9 +21,15 @@ cudaError_t launch_score_mask(const void *W, const double *norm, int64_t N, int6
 cudaError_t launch_select_map(const double *loss, int64_t n_tiles, int64_t n_sparse, int32_t *rank,
                               uint32_t *done, uint32_t *map, cudaStream_t stream);
 
+// `done` (a zeroed counter) and `ready` (zeroed) live in the handle: the last
+// block to finish publishes ready = 1 with release semantics.
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                         int64_t K, int tn, int tk, const uint64_t *table, uint8_t *out,
-                        cudaStream_t stream);
+                        uint32_t *done, uint32_t *ready, cudaStream_t stream);
+
+// Decode (M <= 16) GEMV: CTAs whose first chunk travels in the kernel
+// parameters, at most.
+constexpr int kDecMaxCtas = 160;
 
 struct GemmLaunch {
     const uint8_t *packed;
@@ -37,6 +43,12 @@ struct GemmLaunch {
     size_t workspace_bytes;  // capacity of `workspace`
     cudaMemPool_t pool;      // for larger stream-K partials
     uint32_t *status;
+    const uint32_t *ready;   // set by the pack kernel when the packed bytes are final
+    // decode chunking (see plan_decode_chunks)
+    const uint64_t *chunk_desc;       // device [dec_nchunks]
+    const uint64_t *chunk_desc_host;  // host copy
+    int dec_cp, dec_cpb, dec_nchunks;
+    uint32_t *counter;                // device: chunks claimed, zero between calls
     int num_sms;
     int stall_first_kstep;   // failure-detection test hook (see patch_hybrid_gemm)
     const int64_t *pair_prefix;  // host: per band, cumulative packed bytes of its k-pairs
@@ -45,8 +57,16 @@ struct GemmLaunch {
 // Picks the configuration (token tile, schedule) for M and launches.
 cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream);
 
-// Bytes of stream-K partials the M <= 16 configuration needs at most.
-size_t decode_workspace_bytes(int num_sms);
+// Decode GEMV for M <= 16 (csrc/decode_gemm.cu).
+cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream);
+// Chunking of a packed matrix for the decode GEMV: `cp` k-pairs per chunk,
+// `cpb` chunks per band.
+void plan_decode_chunks(int64_t bands, int64_t nsteps, int num_sms, int *cp, int *cpb, int *nchunks);
+// Descriptor of the chunk holding pairs [pr0, pr0 + np) of a band whose
+// k-step table starts at `band_table`: first byte | 2:4 flags << 40 | np << 56.
+uint64_t decode_chunk_desc(const uint64_t *band_table, int64_t nsteps, int pr0, int np);
+// fp32 partial bytes of the decode GEMV (one 16 x 128 slot per chunk).
+size_t decode_workspace_bytes(int nchunks);
 
 // The library's stream-ordered memory pool for the current device (cached
 // memory is kept, not returned to the system between calls).

@@ -300,3 +300,39 @@ def test_gemm_bounded_wait_reports_timeout(P, oracle_mod, monkeypatch):
     weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
     rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), weff), True)
     pk.close()
+
+
+def test_gemm_chain_overlapped_matches_serialised(P, oracle_mod):
+    # A layer chain where each GEMM reads the previous one's output as its X:
+    # back to back on one stream, each GEMM may start (prologue and first
+    # weight copies) while its predecessor still runs, and must still read X
+    # only after it finished.  The chained results must equal the same calls
+    # with a device synchronisation between them, bit for bit, for decode and
+    # prefill token counts; the first GEMM is checked against the oracle.
+    shapes = [(1024, 512), (768, 1024), (512, 768)]  # (N, K): K of each = N of the previous
+    pks, weffs = [], []
+    for i, (N, K) in enumerate(shapes):
+        w, xc, _ = make_problem(N, K, 64, 1, seed=700 + i)
+        nt = (N // 128) * (K // 128)
+        tmap = inputs.random_map(nt, nt // 2, seed=700 + i)
+        r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+        pks.append(P.patch_pack(w.cuda(), r["meta"], r["map"]))
+        weffs.append(oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32),
+                                     128, 128))
+    for M in (3, 16, 200):
+        x0 = inputs.activations(M, shapes[0][1], 800 + M, None)
+        xs = x0.cuda()
+        chained = []
+        for pk in pks:
+            xs = P.patch_hybrid_gemm(pk, xs)
+            chained.append(xs)
+        torch.cuda.synchronize()
+        xs = x0.cuda()
+        for i, pk in enumerate(pks):
+            xs = P.patch_hybrid_gemm(pk, xs)
+            torch.cuda.synchronize()
+            assert torch.equal(xs, chained[i]), (M, i)
+        rel_rms_check(chained[0], oracle_mod.gemm(bf16_bits(x0), weffs[0]), False)
+    for pk in pks:
+        assert P.patch_get_status(pk) == 0
+        pk.close()
