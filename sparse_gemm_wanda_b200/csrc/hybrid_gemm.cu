@@ -653,6 +653,16 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     if (g.M <= 16) return launch_decode_gemm(g, stream);  // split-K GEMV, csrc/decode_gemm.cu
     if (g.M <= 64) return run<64, 4>(g, 1, stream);   // 48 KB stages
     if (g.M <= 128) return run<128, 3>(g, 1, stream); // 64 KB stages
+    // larger token counts: the band-pair kernel (two bands share each X tile)
+    // unless its items fall into so few waves that this kernel's finer tiles
+    // finish first.  Both estimated per k-step from shared-memory traffic
+    // (copies in + tensor-core operand reads at 128 B per cycle): a 160-token
+    // one-band item moves 72 KB per dense k-step, 576 cycles.
+    const PairPlan pp = plan_pair_gemm(g.N, g.M, g.num_sms);
+    const int64_t items1 = (g.N / kBand) * ((g.M + 159) / 160);
+    const int64_t waves1 = (items1 + g.num_sms - 1) / g.num_sms;
+    if (pp.cost <= static_cast<double>(waves1) * 576.0 && g.K / kStep <= 448)
+        return launch_pair_gemm(g, pp, stream);
     return run<160, 3>(g, 1, stream);                 // 72 KB stages
 }
 

@@ -57,6 +57,23 @@ struct GemmLaunch {
 // Picks the configuration (token tile, schedule) for M and launches.
 cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream);
 
+// Band-pair prefill GEMM (csrc/prefill_gemm.cu): token tile, grid and
+// shared-memory plan for a matrix of N rows and M tokens.
+struct PairPlan {
+    int bn;           // tokens per tile (multiple of 16, 128..240)
+    int ttiles;       // ceil(M / bn)
+    int items;        // band pairs x token tiles
+    int waves;        // ceil(items / SMs)
+    int stages;       // k-steps in flight
+    int stage_bytes;
+    int smem;         // dynamic shared memory per CTA
+    double cost;      // waves x estimated cycles per k-step of an item
+};
+// Estimated cycles of one dense k-step of a band-pair item with BN tokens.
+double pair_kstep_cycles(int bn);
+PairPlan plan_pair_gemm(int64_t N, int64_t M, int num_sms);
+cudaError_t launch_pair_gemm(const GemmLaunch &g, const PairPlan &plan, cudaStream_t stream);
+
 // Decode GEMV for M <= 16 (csrc/decode_gemm.cu).
 cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream);
 // Chunking of a packed matrix for the decode GEMV: `cp` k-pairs per chunk,

@@ -336,3 +336,42 @@ def test_gemm_chain_overlapped_matches_serialised(P, oracle_mod):
     for pk in pks:
         assert P.patch_get_status(pk) == 0
         pk.close()
+
+
+@pytest.mark.parametrize("N,K,M,tn,tk,frac", [
+    (4096, 512, 1300, 128, 128, 0.5),   # band-pair kernel, 160-token tiles, ragged last tile
+    (3968, 512, 1300, 128, 128, 1.0),   # odd band count: the last pair holds one band
+    (4096, 1024, 2000, 128, 128, 0.0),  # all dense, 224-token tiles
+    (4096, 512, 1300, 64, 64, 0.5),     # 64x64 tiles: mixed 64-row tiles inside a band
+])
+@pytest.mark.parametrize("fp32_mode", [True, False])
+def test_gemm_band_pair_kernel(P, oracle_mod, N, K, M, tn, tk, frac, fp32_mode):
+    # token counts whose one-band tiling takes two or more waves of SMs take
+    # the band-pair kernel (two bands per CTA sharing each X tile)
+    run_case(P, oracle_mod, N, K, M, tn, tk, frac, seed=N + M + tn, fp32_mode=fp32_mode,
+             sample=6000)
+
+
+def test_gemm_band_pair_kernel_bounded_wait(P, oracle_mod, monkeypatch):
+    # the failure-detection hook on the band-pair kernel: CTA 0's first stage
+    # never lands, its waits run out, the status reports the timeout and the
+    # handle computes correctly once the status is read
+    N, K, M = 4096, 512, 1300
+    w, xc, x = make_problem(N, K, 64, M, seed=43)
+    nt = (N // 128) * (K // 128)
+    tmap = inputs.random_map(nt, nt // 2, seed=43)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    monkeypatch.setenv("PATCH_B200_TEST_STALL", "1")
+    P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    monkeypatch.delenv("PATCH_B200_TEST_STALL")
+    assert P.patch_get_status(pk) == 5
+    assert P.patch_get_status(pk) == 0
+    y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
+    g = np.random.default_rng(43)
+    ms, ns = g.integers(0, M, 3000), g.integers(0, N, 3000)
+    yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
+    rel_rms_check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, True)
+    pk.close()
