@@ -661,7 +661,13 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     const PairPlan pp = plan_pair_gemm(g.N, g.M, g.num_sms);
     const int64_t items1 = (g.N / kBand) * ((g.M + 159) / 160);
     const int64_t waves1 = (items1 + g.num_sms - 1) / g.num_sms;
-    if (pp.cost <= static_cast<double>(waves1) * 576.0 && g.K / kStep <= 448)
+    const double t_one = static_cast<double>(waves1) * 576.0;
+    if (g.duo_ok && g.K / kStep <= 448) {
+        // two-SM MMA when the matrix allows it and its estimate is lowest
+        const DuoPlan dp = plan_duo_gemm(g.N, g.M, g.num_sms);
+        if (dp.bn > 0 && dp.cost <= pp.cost && dp.cost <= t_one) return launch_duo_gemm(g, dp, stream);
+    }
+    if (pp.cost <= t_one && g.K / kStep <= 448)
         return launch_pair_gemm(g, pp, stream);
     return run<160, 3>(g, 1, stream);                 // 72 KB stages
 }

@@ -32,6 +32,7 @@ struct patch_packed {
     uint64_t *chunk_desc;      // device: decode chunk descriptors
     std::vector<uint64_t> chunk_desc_host;
     int dec_cp, dec_cpb, dec_nchunks;
+    int duo_ok;                // bands 2p, 2p+1 agree in type at every k-step
     uint32_t *status;          // device: status word, pack counter, ready flag
     int num_sms;
     cudaMemPool_t pool;
@@ -421,6 +422,15 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
                 patchk::decode_chunk_desc(table.data() + b * nsteps, nsteps, pr0, np);
         }
     h->workspace_bytes = patchk::decode_workspace_bytes(h->dec_nchunks);
+    // the two-SM prefill kernel pairs bands 2p and 2p+1 in one instruction
+    h->duo_ok = (bands % 2 == 0) ? 1 : 0;
+    for (int64_t b = 0; h->duo_ok && b < bands; b += 2)
+        for (int64_t c = 0; c < nsteps; ++c)
+            if ((table[static_cast<size_t>(b * nsteps + c)] & patchk::kEntrySparse) !=
+                (table[static_cast<size_t>((b + 1) * nsteps + c)] & patchk::kEntrySparse)) {
+                h->duo_ok = 0;
+                break;
+            }
 
     // one pool allocation: packed bytes | table | chunk descriptors | workspace | status
     const size_t off_table = round_up(std::max<size_t>(h->packed_bytes, 16), 256);
@@ -486,6 +496,8 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.dec_cp = Wp->dec_cp;
     g.dec_cpb = Wp->dec_cpb;
     g.dec_nchunks = Wp->dec_nchunks;
+    g.packed_rows = Wp->packed_bytes / 128;
+    g.duo_ok = Wp->duo_ok;
     g.num_sms = Wp->num_sms;
     g.pair_prefix = Wp->pair_prefix.data();
     // Failure-detection test hook: with PATCH_B200_TEST_STALL=1 in the

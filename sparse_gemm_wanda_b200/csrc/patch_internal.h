@@ -49,6 +49,8 @@ struct GemmLaunch {
     const uint64_t *chunk_desc_host;  // host copy
     int dec_cp, dec_cpb, dec_nchunks;
     uint32_t *counter;                // device: chunks claimed, zero between calls
+    uint64_t packed_rows;             // packed bytes / 128
+    int duo_ok;                       // bands 2p, 2p+1 agree in type at every k-step
     int num_sms;
     int stall_first_kstep;   // failure-detection test hook (see patch_hybrid_gemm)
     const int64_t *pair_prefix;  // host: per band, cumulative packed bytes of its k-pairs
@@ -73,6 +75,19 @@ struct PairPlan {
 double pair_kstep_cycles(int bn);
 PairPlan plan_pair_gemm(int64_t N, int64_t M, int num_sms);
 cudaError_t launch_pair_gemm(const GemmLaunch &g, const PairPlan &plan, cudaStream_t stream);
+
+// Two-SM prefill GEMM (csrc/prefill_duo.cu) for matrices whose bands 2p and
+// 2p+1 agree in tile type at every k-step.
+struct DuoPlan {
+    int bn;           // tokens per tile (each CTA of the pair holds bn / 2)
+    int ttiles, items;
+    int clusters;     // CTA pairs launched
+    int stages, stage_bytes, smem;
+    double cost;      // waves x estimated cycles per k-step of an item
+};
+DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms);
+cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream_t stream);
+double duo_kstep_cycles(int bn);
 
 // Decode GEMV for M <= 16 (csrc/decode_gemm.cu).
 cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream);

@@ -1,0 +1,619 @@
+// Two-SM hybrid GEMM for prefill: tcgen05 with cta_group::2 (sm_100a).
+//
+// Same product as the other GEMM paths, Y = X * W_eff^T ("PATCH: Learnable
+// Tile-level Hybrid Sparsity for LLMs", section 2, inference and deployment),
+// for matrices whose paired bands agree in tile type at every k-step (every
+// tile dense, every tile 2:4, or any map whose bands 2p and 2p+1 match).
+//
+// Why.  The tensor core reads its operands from shared memory and the copies
+// write there too, about 128 B per cycle per SM in all.  With one CTA per MMA
+// every SM must hold the whole token tile; with cta_group::2 a CTA pair runs
+// M = 256 MMAs (one 128-row band per SM) and each SM holds HALF of the token
+// tile: per dense 64-column k-step an SM moves 32 KB + 128 B per token
+// (copies in + operand reads) for 2 x BN MMA cycles, about 97 % of the MMA rate
+// at BN = 240, and a 2:4 k-step about 64 % of the sparse rate.  Both bands of
+// an instruction must be of one kind, hence the matching requirement.
+//
+// Work item = (band pair, token tile of BN tokens); clusters of two CTAs take
+// items c, c + C, ...; CTA rank r owns band 2p + r and tokens
+// [r BN/2, (r+1) BN/2) of the tile.  Stage = one k-pair (128 columns): this
+// SM's band (ONE TMA load of the pair's 18-32 KB, through tensor maps over
+// the packed buffer in 2 KB rows) and its half of the X tile for both k-steps
+// (ONE 3-D TMA load, 128-byte swizzle, rows past M zero).  Few, large copies:
+// a copy costs ~0.16 us of issue-to-issue time whatever its size up to 16 KB.  All loads of both CTAs complete on the
+// leader's stage mbarrier (TMA .cta_group::2); the weights and the X tiles
+// are issued by two threads in different warps, since the copies one thread
+// issues are processed largely one after another.  The leader's single MMA thread
+// issues tcgen05.mma(.sp).cta_group::2 M256 x BN; tcgen05.commit with a CTA
+// mask frees the stage in both CTAs and hands the accumulator to both
+// epilogues.  Each SM holds its band's 128 x BN fp32 accumulator; two
+// accumulators alternate between items (2 x 240 + 4 metadata columns).
+//
+// Every mbarrier wait is bounded by %globaltimer; a CTA that gives up raises
+// its own and its peer's abort flag, drains its copies and still meets its
+// peer at the final cluster barrier, so both CTAs free tensor memory together.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "patch_common.cuh"
+#include "patch_internal.h"
+
+namespace patchk {
+
+namespace {
+
+constexpr int kDuoThreads = 224;   // + warp 6: the X-tile producer
+constexpr int kDuoMaxStages = 8;
+constexpr int kDuoTabSteps = 448;                      // k-steps per band (K <= 28672)
+constexpr int kDuoTabBytes = 2 * kDuoTabSteps * 8;     // two items of one band
+constexpr int kDuoAslot = 2 * kDenseStepBytes;  // one k-pair of weights, at most
+constexpr int kDuoTmemCols = 512;
+constexpr int kDuoSmemLimit = 232448;
+constexpr int kDuoTailBytes = 1024 + kDuoTabBytes + 512;
+constexpr uint64_t kDuoWaitLimitNs = 2000000000ull;
+
+// ------------------------------------------------------------ cluster PTX
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(const void *p, uint32_t rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
+    return out;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void fence_mbar_init_cluster() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// 2-D / 3-D TMA loads into this CTA's shared memory, completing on an
+// mbarrier that may live in the peer CTA (cluster address)
+__device__ __forceinline__ void tma2d_pair(void *dst, const void *tmap, int32_t x, int32_t y,
+                                           uint32_t mbar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(mbar_cluster)
+        : "memory");
+}
+__device__ __forceinline__ void tma3d_pair(void *dst, const void *tmap, int32_t x, int32_t y, int32_t z,
+                                           uint32_t mbar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(mbar_cluster)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+// commit: arrive on the mbarrier at this offset in both CTAs of the pair
+// once every tcgen05 operation issued so far has completed
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+__device__ __forceinline__ void mma_dense_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_sparse_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_cp_pair_128x128b(uint32_t taddr, uint64_t s_desc) {
+    asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
+}
+// instruction descriptor: bf16 x bf16 -> fp32, K-major A and B, M = 256
+__host__ __device__ constexpr uint32_t idesc_pair(int n, bool sparse, uint32_t id2 = 0) {
+    return (id2 & 3u) | (sparse ? (1u << 2) : 0u) | (1u << 4) | (1u << 7) | (1u << 10) |
+           (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
+}
+
+struct DuoParams {
+    const uint64_t *table;
+    int64_t N, K, M;
+    int nsteps, bands, ttiles, items;
+    int bn, half, stages, stage_bytes;
+    void *Y;
+    int y_fp32;
+    uint32_t *status;
+    const uint32_t *ready;
+    int stall_first_kstep;  // failure-detection test hook
+};
+
+__device__ __forceinline__ void store_y(const DuoParams &p, int64_t idx, float v) {
+    if (p.y_fp32)
+        static_cast<float *>(p.Y)[idx] = v;
+    else
+        static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
+}
+
+// Tensor maps over the packed buffer viewed as rows of 2 KB (256 x 8-byte
+// elements); the box is one packed k-pair: 16 rows (two dense k-steps), 13
+// (one dense + metadata + one 2:4) or 9 (metadata + two 2:4).  X is viewed
+// as (64 columns, M rows, K/64 k-steps) with a box of both k-steps of a pair.
+struct DuoMaps {
+    CUtensorMap x, a_dd, a_mixed, a_ss;
+};
+
+__global__ void __launch_bounds__(kDuoThreads, 1)
+duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ DuoParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int S = p.stages;
+    uint64_t *tab_buf = reinterpret_cast<uint64_t *>(smem + S * p.stage_bytes);  // [2][448]
+    uint64_t *full = tab_buf + 2 * kDuoTabSteps;  // leader: all loads of both CTAs
+    uint64_t *empty = full + kDuoMaxStages;        // both: freed by the leader's commit
+    uint64_t *acc_full = empty + kDuoMaxStages;    // [2] both
+    uint64_t *acc_empty = acc_full + 2;            // [2] leader: 4 warps x 2 CTAs
+    uint64_t *tab_full = acc_empty + 2;            // [2] own table copies
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tab_full + 2);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+    volatile uint32_t *never_flag = tmem_slot + 2;
+    uint64_t *stage_info = reinterpret_cast<uint64_t *>(tmem_slot + 4);  // [S][2]: the pair's entries
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_rank();
+    const int cl = blockIdx.x / 2, C = gridDim.x / 2;
+    const int bn = p.bn, half = p.half;
+
+    auto fetch_table = [&](int item, int buf) {
+        const int band = 2 * (item / p.ttiles) + static_cast<int>(rank);
+        const uint32_t nb = static_cast<uint32_t>(p.nsteps) * 8u;
+        mbar_arrive_expect_tx(&tab_full[buf], nb);
+        bulk_g2s(tab_buf + buf * kDuoTabSteps, p.table + static_cast<int64_t>(band) * p.nsteps, nb,
+                 &tab_full[buf]);
+    };
+    auto give_up = [&]() {
+        *abort_flag = 1u;
+        st_cluster_u32(map_to_rank(const_cast<uint32_t *>(abort_flag), rank ^ 1u), 1u);
+        atomicOr(p.status, kStatusTimeout);
+    };
+
+    if (threadIdx.x == 0) {
+        pdl_trigger();
+        // weights are final once the packer's ready flag is seen; otherwise
+        // (the packer may be the kernel just before) wait first
+        if (ld_acquire_gpu(p.ready) == 0u) pdl_wait();
+        for (int s = 0; s < kDuoMaxStages; ++s) {
+            mbar_init(&full[s], 2);  // the leader's weight and X producers
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);
+            mbar_init(&tab_full[b], 1);
+        }
+        *never_flag = 0u;
+        *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
+        fence_mbar_init_cluster();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, kDuoTmemCols);
+        tmem_relinquish_pair();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&maps.x);
+        prefetch_tmap(&maps.a_dd);
+        prefetch_tmap(&maps.a_mixed);
+        prefetch_tmap(&maps.a_ss);
+    }
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs' barriers and tensor memory exist from here on
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    // a CTA that starts with its status raised skips all work but still meets
+    // its peer at the end; the peer's waits then run out and it does the same
+    const bool skip = *abort_flag != 0;
+    if (threadIdx.x == 0 && !skip) {
+        for (int i = 0; i < 2 && cl + i * C < p.items; ++i) fetch_table(cl + i * C, i);
+    }
+
+    if (warp == 0) {
+        if (lane == 0 && !skip) {
+            // ------------------------------------------------------ producer
+            // (both CTAs; every load completes on the LEADER's stage barrier)
+            int it = 0;
+            bool ok = true;
+            int tabs = 0;
+            for (int i = 0; i < 2 && cl + i * C < p.items; ++i) ++tabs;
+            // weights need no wait once the packer's ready flag was seen;
+            // otherwise thread 0 already passed griddepcontrol.wait
+            for (int i = 0; ok; ++i) {
+                const int item = cl + i * C;
+                if (item >= p.items) break;
+                const int buf = i & 1;
+                if (!mbar_wait_bounded(&tab_full[buf], (i >> 1) & 1u, abort_flag, kDuoWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                const uint64_t *tab = tab_buf + buf * kDuoTabSteps;
+                for (int pr = 0; pr < p.nsteps / 2; ++pr) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (it >= S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kDuoWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint64_t e0 = tab[2 * pr], e1 = tab[2 * pr + 1];
+                    const uint64_t first = (e0 & kEntryOffsetMask) - ((e0 & kEntryMeta) ? kMetaBlockBytes : 0);
+                    const uint64_t end = (e1 & kEntryOffsetMask) +
+                                         ((e1 & kEntrySparse) ? kSparseStepBytes : kDenseStepBytes);
+                    const uint32_t a_bytes = static_cast<uint32_t>(end - first);  // 32, 26 or 18 KB
+                    stage_info[2 * s + 0] = e0;
+                    stage_info[2 * s + 1] = e1;
+                    ++it;
+                    if (p.stall_first_kstep && blockIdx.x == 0 && it == 1) continue;  // never lands
+                    // the two bands of a pair agree in kind and metadata placement,
+                    // so the leader arms the barrier for both CTAs' weight bytes
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * a_bytes);
+                    const CUtensorMap *am = a_bytes == 2u * kDenseStepBytes ? &maps.a_dd
+                                          : (a_bytes == 2u * kSparseStepBytes + kMetaBlockBytes ? &maps.a_ss
+                                                                                               : &maps.a_mixed);
+                    tma2d_pair(smem + s * p.stage_bytes, am, 0, static_cast<int32_t>(first / 2048),
+                               map_to_rank(&full[s], 0));
+                }
+                if (ok && cl + (i + 2) * C < p.items) {
+                    fetch_table(cl + (i + 2) * C, buf);
+                    ++tabs;
+                }
+            }
+            for (int q = (tabs > 2 ? tabs - 2 : 0); q < tabs; ++q)
+                mbar_wait_bounded(&tab_full[q & 1], (q >> 1) & 1u, never_flag, kDuoWaitLimitNs / 4);
+            if (!ok) give_up();
+            // Drain.  The leader waits for the last phase of every stage (its
+            // barrier counts both CTAs' loads); the peer waits until the
+            // leader's MMA has released each of its stages, or gives up.
+            for (int q = (it > S ? it - S : 0); q < it; ++q) {
+                if (p.stall_first_kstep && blockIdx.x == 0 && q == 0) continue;  // never armed
+                if (rank == 0)
+                    mbar_wait_bounded(&full[q % S], (q / S) & 1u, never_flag, kDuoWaitLimitNs / 4);
+                else
+                    mbar_wait_bounded(&empty[q % S], (q / S) & 1u, never_flag, kDuoWaitLimitNs / 4);
+            }
+        }
+    } else if (warp == 6) {
+        if (lane == 0 && !skip) {
+            // ------------------------------------------------ X producer
+            // (both CTAs; a second issuing thread: copies from one thread
+            // are processed largely one after another)
+            pdl_wait();  // X may still be written by the kernel before
+            const uint32_t x_bytes = 2u * 2u * static_cast<uint32_t>(half) * kStep * 2u;  // both CTAs, 2 k-steps
+            int it = 0;
+            bool ok = true;
+            for (int i = 0; ok; ++i) {
+                const int item = cl + i * C;
+                if (item >= p.items) break;
+                const int tt = item % p.ttiles;
+                for (int pr = 0; pr < p.nsteps / 2; ++pr) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (it >= S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kDuoWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    ++it;
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], x_bytes);
+                    tma3d_pair(smem + s * p.stage_bytes + kDuoAslot, &maps.x, 0,
+                               tt * bn + static_cast<int>(rank) * half, 2 * pr, map_to_rank(&full[s], 0));
+                }
+            }
+            if (!ok) give_up();
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && !skip && rank == 0) {
+            // ------------------------------------------------- MMA (leader)
+            const uint32_t e_tmem = tmem_base + static_cast<uint32_t>(2 * bn);
+            const uint32_t idesc_dense = idesc_pair(bn, false);
+            int it = 0;
+            bool ok = true;
+            for (int i = 0; ok; ++i) {
+                const int item = cl + i * C;
+                if (item >= p.items) break;
+                const int buf = i & 1;
+                if (i >= 2 &&
+                    !mbar_wait_bounded(&acc_empty[buf], ((i >> 1) & 1u) ^ 1u, abort_flag, kDuoWaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * bn);
+                for (int pr = 0; pr < p.nsteps / 2; ++pr, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait_bounded(&full[s], ph, abort_flag, kDuoWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t slot = smem_u32(smem + s * p.stage_bytes);
+                    const uint64_t e0 = stage_info[2 * s];
+                    const uint64_t first = (e0 & kEntryOffsetMask) - ((e0 & kEntryMeta) ? kMetaBlockBytes : 0);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint64_t e = stage_info[2 * s + h];
+                        const uint32_t a_addr = slot + static_cast<uint32_t>((e & kEntryOffsetMask) - first);
+                        const uint32_t b_addr = slot + kDuoAslot + static_cast<uint32_t>(h * half * kStep * 2);
+                        const bool fresh = pr == 0 && h == 0;
+                        if (e & kEntrySparse) {
+                            if (e & kEntryMeta)
+                                tmem_cp_pair_128x128b(e_tmem, smem_desc(a_addr - kMetaBlockBytes, 16, 128, kSwizzleNone));
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const uint64_t ad = smem_desc(a_addr + q * 32, 16, 512, kSwizzle64B);
+                                const uint64_t bd = smem_desc(b_addr + q * 64, 16, 1024, kSwizzle128B);
+                                mma_sparse_pair(d_tmem, ad, bd, e_tmem + 2 * h, idesc_pair(bn, true, q),
+                                                (fresh && q == 0) ? 0u : 1u);
+                            }
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const uint64_t ad = smem_desc(a_addr + q * 32, 16, 1024, kSwizzle128B);
+                                const uint64_t bd = smem_desc(b_addr + q * 32, 16, 1024, kSwizzle128B);
+                                mma_dense_pair(d_tmem, ad, bd, idesc_dense, (fresh && q == 0) ? 0u : 1u);
+                            }
+                        }
+                    }
+                    tc_commit_pair(&empty[s]);
+                }
+                // fires once every MMA of the item has completed (also after a
+                // failure, so no epilogue frees tensor memory under a running MMA)
+                tc_commit_pair(&acc_full[buf]);
+            }
+            if (!ok) give_up();
+        }
+    } else if (!skip) {
+        // ---------------------------------------------- epilogue (both CTAs)
+        pdl_wait();  // Y may still be read by an earlier kernel
+        const int quad = warp % 4;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+        for (int i = 0;; ++i) {
+            const int item = cl + i * C;
+            if (item >= p.items) break;
+            const int bp = item / p.ttiles, tt = item % p.ttiles;
+            const int buf = i & 1;
+            const bool ok = mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1u, never_flag, kDuoWaitLimitNs);
+            tc_fence_after();
+            if (!ok) {
+                give_up();
+                break;
+            }
+            const int64_t n = static_cast<int64_t>(2 * bp + static_cast<int>(rank)) * kBand + row;
+            const int64_t m_base = static_cast<int64_t>(tt) * bn;
+            const int m_valid = static_cast<int>(min(static_cast<int64_t>(bn), p.M - m_base));
+            if (*abort_flag == 0) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < m_valid; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(buf * bn + c0), r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        if (c0 + q < m_valid) store_y(p, (m_base + c0 + q) * p.N + n, __uint_as_float(r[q]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(map_to_rank(&acc_empty[buf], 0));
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all();  // the peer's MMAs and remote arrivals are all done
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, kDuoTmemCols);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// the packed buffer as rows of 2 KB (256 x 8-byte elements), box of `box_rows`
+bool encode_rows(EncodeTiledFn enc, CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {256, rows};
+    const cuuint64_t strides[1] = {2048};
+    const cuuint32_t box[2] = {256, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t ensure_duo_attributes() {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(duo_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kDuoSmemLimit);
+    });
+    return attr_err;
+}
+
+// clusters of two CTAs that fit on the device at once with `smem` bytes each
+int duo_max_clusters(int smem) {
+    if (ensure_duo_attributes() != cudaSuccess) return 0;
+    static std::mutex mu;
+    static int cached_smem = -1, cached = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached_smem == smem) return cached;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(kDuoThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, duo_gemm_kernel, &cfg) != cudaSuccess) n = 0;
+    cached_smem = smem;
+    cached = n;
+    return n;
+}
+
+}  // namespace
+
+double duo_kstep_cycles(int bn) {
+    // per SM per dense k-step: max(MMA 2 BN cycles, shared-memory traffic
+    // (16 KB + 64 B per token in, the same again read) at 128 B per cycle)
+    return std::max(2.0 * bn, 256.0 + bn);
+}
+
+DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms) {
+    DuoPlan best{};
+    const int64_t bpairs = (N / kBand) / 2;
+    // shared memory per stage: 16 KB of weights + BN/2 tokens x 128 B
+    auto smem_for = [](int bn, int *stages, int *stage_bytes) {
+        *stage_bytes = kDuoAslot + 2 * (bn / 2) * kStep * 2;
+        *stages = std::min(kDuoMaxStages, (kDuoSmemLimit - kDuoTailBytes) / *stage_bytes);
+        return *stages * *stage_bytes + kDuoTailBytes;
+    };
+    int st = 0, sb = 0;
+    const int clusters_cap = duo_max_clusters(smem_for(240, &st, &sb));
+    if (clusters_cap < 1) return best;  // bn = 0: not usable
+    const int clusters = std::min(clusters_cap, num_sms / 2);
+    double best_cost = 0;
+    for (int bn = 240; bn >= 128; bn -= 16) {
+        const int64_t tt = (M + bn - 1) / bn;
+        const int64_t items = bpairs * tt;
+        const int64_t waves = (items + clusters - 1) / clusters;
+        const double cost = static_cast<double>(waves) * duo_kstep_cycles(bn);
+        if (best.bn == 0 || cost < best_cost) {
+            best_cost = cost;
+            best.bn = bn;
+            best.ttiles = static_cast<int>(tt);
+            best.items = static_cast<int>(items);
+            best.clusters = static_cast<int>(std::min<int64_t>(clusters, items));
+        }
+    }
+    best.smem = smem_for(best.bn, &best.stages, &best.stage_bytes);
+    // the same work in per-SM units as the band-pair kernel's estimate: a
+    // cluster item covers two SMs, so compare per-SM cycles
+    best.cost = best_cost;
+    return best;
+}
+
+cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream_t stream) {
+    const cudaError_t attr_err = ensure_duo_attributes();
+    if (attr_err != cudaSuccess) return attr_err;
+    if (plan.stages < 2 || plan.smem > kDuoSmemLimit || plan.clusters < 1) return cudaErrorInvalidValue;
+    if ((g.N / kBand) % 2 != 0 || g.K / kStep > kDuoTabSteps || !g.packed_rows) return cudaErrorInvalidValue;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorInvalidValue;
+    DuoMaps maps;
+    // X [M,K] as (64 columns, M rows, K/64 k-steps); box = this CTA's half of
+    // the token tile for both k-steps of a pair; rows past M read as zero
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kStep), static_cast<cuuint64_t>(g.M),
+                                static_cast<cuuint64_t>(g.K / kStep)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.K) * 2, static_cast<cuuint64_t>(kStep) * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kStep), static_cast<cuuint32_t>(plan.bn / 2), 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(g.X), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const uint64_t rows = g.packed_rows / 16;  // 2 KB rows
+    if (!encode_rows(enc, &maps.a_dd, g.packed, rows, 2 * kDenseStepBytes / 2048) ||
+        !encode_rows(enc, &maps.a_mixed, g.packed, rows,
+                     (kDenseStepBytes + kMetaBlockBytes + kSparseStepBytes) / 2048) ||
+        !encode_rows(enc, &maps.a_ss, g.packed, rows, (kMetaBlockBytes + 2 * kSparseStepBytes) / 2048))
+        return cudaErrorInvalidValue;
+    DuoParams p;
+    p.table = g.table;
+    p.N = g.N;
+    p.K = g.K;
+    p.M = g.M;
+    p.nsteps = static_cast<int>(g.K / kStep);
+    p.bands = static_cast<int>(g.N / kBand);
+    p.ttiles = plan.ttiles;
+    p.items = plan.items;
+    p.bn = plan.bn;
+    p.half = plan.bn / 2;
+    p.stages = plan.stages;
+    p.stage_bytes = plan.stage_bytes;
+    p.Y = g.Y;
+    p.y_fp32 = g.y_fp32;
+    p.status = g.status;
+    p.ready = g.ready;
+    p.stall_first_kstep = g.stall_first_kstep;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * plan.clusters));
+    cfg.blockDim = dim3(kDuoThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, duo_gemm_kernel, maps, p);
+    if (err == cudaSuccess) note_launches(1);
+    return err;
+}
+
+}  // namespace patchk

@@ -22,11 +22,13 @@
 // metadata block + 8 KB kept values) and one 2-D TMA load of the X tile
 // (128-byte swizzle, rows past M read as zero).
 //
-// Roles (320 threads): warp 0 lane 0 producer, warp 1 lane 0 MMA issuer,
-// warps 2..9 epilogue (warps 2..5 drain band 0, warps 6..9 band 1; each warp
-// its 32-lane TMEM quarter).  Launched as a programmatic dependent: with the
-// packer's ready flag seen, the table and the first stages' weights are
-// fetched before `griddepcontrol.wait`; X and Y only after it.  Every mbarrier
+// Roles (352 threads): warp 0 lane 0 weight producer, warp 10 lane 0 X
+// producer (copies one thread issues are processed largely one after another,
+// so the two streams get a thread each), warp 1 lane 0 MMA issuer, warps 2..9
+// epilogue (warps 2..5 drain band 0, warps 6..9 band 1; each warp its 32-lane
+// TMEM quarter).  Launched as a programmatic dependent: with the packer's
+// ready flag seen, the table and the weights are fetched before
+// `griddepcontrol.wait`; X and Y only after it.  Every mbarrier
 // wait is bounded by %globaltimer.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -43,7 +45,7 @@ namespace patchk {
 
 namespace {
 
-constexpr int kPgThreads = 320;
+constexpr int kPgThreads = 352;   // + warp 10: the X-tile producer
 constexpr int kPgEpiWarps = 8;
 constexpr int kPgMaxStages = 6;
 constexpr int kPgTabSteps = 448;                 // k-steps per band (K <= 28672)
@@ -98,7 +100,6 @@ pair_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int cta = blockIdx.x, P = gridDim.x;
-    bool waited = true;  // thread 0: past griddepcontrol.wait
 
     auto item_bands = [&](int item, int &bp, int &tt, bool &two) {
         bp = item / p.ttiles;
@@ -120,10 +121,11 @@ pair_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
 
     if (threadIdx.x == 0) {
         pdl_trigger();
+        // weights are final once the packer's ready flag is seen; otherwise
+        // (the packer may be the kernel just before) wait first
         if (ld_acquire_gpu(p.ready) == 0u) pdl_wait();
-        else waited = false;
         for (int s = 0; s < kPgMaxStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 2);  // weight producer + X producer
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
@@ -156,16 +158,6 @@ pair_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
             bool ok = true;
             int tabs = 0;  // table copies issued
             for (int i = 0; i < 2 && cta + i * P < p.items; ++i) ++tabs;
-            int pend_s[kPgMaxStages], pend_c[kPgMaxStages], pend_t[kPgMaxStages];
-            int npend = 0;
-            auto flush_x = [&]() {
-                pdl_wait();
-                waited = true;
-                for (int q = 0; q < npend; ++q)
-                    tma_load_2d_x(smem + pend_s[q] * p.stage_bytes + 2 * kPgAslot, &tmap_x,
-                                  pend_c[q] * kStep, pend_t[q] * bn, &full[pend_s[q]]);
-                npend = 0;
-            };
             for (int i = 0; ok; ++i) {
                 const int item = cta + i * P;
                 if (item >= p.items) break;
@@ -181,7 +173,6 @@ pair_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
                 for (int c = 0; c < p.nsteps; ++c) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
-                    if (!waited && it >= S) flush_x();
                     if (it >= S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kPgWaitLimitNs)) {
                         ok = false;
                         break;
@@ -192,7 +183,7 @@ pair_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
                     stage_info[2 * s + 1] = e1;
                     ++it;
                     if (p.stall_first_kstep && cta == 0 && it == 1) continue;  // never lands
-                    uint32_t bytes = static_cast<uint32_t>(bn) * kStep * 2;
+                    uint32_t bytes = 0;
                     uint64_t f0 = 0, f1 = 0;
                     uint32_t b0 = 0, b1 = 0;
                     {
@@ -211,14 +202,6 @@ pair_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
                     mbar_arrive_expect_tx(&full[s], bytes);
                     bulk_g2s(st, p.packed + f0, b0, &full[s]);
                     if (two) bulk_g2s(st + kPgAslot, p.packed + f1, b1, &full[s]);
-                    if (waited) {
-                        tma_load_2d_x(st + 2 * kPgAslot, &tmap_x, c * kStep, tt * bn, &full[s]);
-                    } else {
-                        pend_s[npend] = s;
-                        pend_c[npend] = c;
-                        pend_t[npend] = tt;
-                        ++npend;
-                    }
                 }
                 // this table buffer is free again: fetch the table of item i + 2
                 if (ok && cta + (i + 2) * P < p.items) {
@@ -226,7 +209,6 @@ pair_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
                     ++tabs;
                 }
             }
-            if (!waited) flush_x();
             for (int q = (tabs > 2 ? tabs - 2 : 0); q < tabs; ++q)
                 mbar_wait_bounded(&tab_full[q & 1], (q >> 1) & 1u, never_flag, kPgWaitLimitNs / 4);
             if (!ok) {
@@ -237,6 +219,40 @@ pair_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
                 if (p.stall_first_kstep && cta == 0 && q == 0) continue;  // never armed
                 mbar_wait_bounded(&full[q % S], (q / S) & 1u, never_flag, kPgWaitLimitNs / 4);
             }
+        }
+    } else if (warp == 10) {
+        if (lane == 0 && !skip) {
+            // ---------------------------------------------------- X producer
+            // a second issuing thread: copies one thread issues are processed
+            // largely one after another
+            pdl_wait();  // X may still be written by the kernel before
+            const uint32_t x_bytes = static_cast<uint32_t>(bn) * kStep * 2u;
+            int it = 0;
+            bool ok = true;
+            for (int i = 0; ok; ++i) {
+                const int item = cta + i * P;
+                if (item >= p.items) break;
+                const int tt = item % p.ttiles;
+                for (int c = 0; c < p.nsteps; ++c) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (it >= S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kPgWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    ++it;
+                    mbar_arrive_expect_tx(&full[s], x_bytes);
+                    tma_load_2d_x(smem + s * p.stage_bytes + 2 * kPgAslot, &tmap_x, c * kStep, tt * bn,
+                                  &full[s]);
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1u;
+                atomicOr(p.status, kStatusTimeout);
+            }
+            // drain: the last phase of every stage this thread armed
+            for (int q = (it > S ? it - S : 0); q < it; ++q)
+                mbar_wait_bounded(&full[q % S], (q / S) & 1u, never_flag, kPgWaitLimitNs / 4);
         }
     } else if (warp == 1) {
         if (lane == 0 && !skip) {

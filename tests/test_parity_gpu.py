@@ -375,3 +375,76 @@ def test_gemm_band_pair_kernel_bounded_wait(P, oracle_mod, monkeypatch):
     yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
     rel_rms_check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, True)
     pk.close()
+
+
+def band_aligned_map(n_rows_tiles, n_col_tiles, seed):
+    """A map whose tile rows 2p and 2p+1 (bands 2p, 2p+1 for 128-row tiles)
+    share one random dense / 2:4 pattern along K."""
+    g = np.random.default_rng(seed)
+    words = [0] * ((n_rows_tiles * n_col_tiles + 31) // 32)
+    for rp in range(n_rows_tiles // 2):
+        pat = g.integers(0, 2, n_col_tiles)
+        for r in (2 * rp, 2 * rp + 1):
+            for k in range(n_col_tiles):
+                if pat[k]:
+                    t = r * n_col_tiles + k
+                    words[t // 32] |= 1 << (t % 32)
+    return torch.from_numpy(np.array(words, dtype=np.uint32).view(np.int32))
+
+
+@pytest.mark.parametrize("N,K,M,tn,frac", [
+    (4096, 512, 1300, 128, 1.0),   # two-SM kernel: every tile 2:4, 160-token tiles, ragged
+    (4096, 1024, 2000, 128, 0.0),  # every tile dense
+    (4096, 512, 1300, 64, 1.0),    # 64x64 tiles, every tile 2:4
+])
+@pytest.mark.parametrize("fp32_mode", [True, False])
+def test_gemm_two_sm_kernel(P, oracle_mod, N, K, M, tn, frac, fp32_mode):
+    # maps whose bands 2p and 2p+1 agree in type at every k-step take the
+    # cta_group::2 kernel (one band per SM of a CTA pair, M = 256 MMAs)
+    run_case(P, oracle_mod, N, K, M, tn, tn, frac, seed=N + M + 7 * tn, fp32_mode=fp32_mode,
+             sample=6000)
+
+
+@pytest.mark.parametrize("fp32_mode", [True, False])
+def test_gemm_two_sm_kernel_band_aligned_mixed_map(P, oracle_mod, fp32_mode):
+    # dense and 2:4 k-steps alternate along K inside one item; both bands of
+    # every instruction agree
+    N, K, M = 4096, 1024, 1300
+    w, xc, x = make_problem(N, K, 64, M, seed=91)
+    tmap = band_aligned_map(N // 128, K // 128, seed=91)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=fp32_mode)
+    torch.cuda.synchronize()
+    assert P.patch_get_status(pk) == 0
+    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
+    g = np.random.default_rng(91)
+    ms, ns = g.integers(0, M, 6000), g.integers(0, N, 6000)
+    yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
+    rel_rms_check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, fp32_mode)
+    pk.close()
+
+
+def test_gemm_two_sm_kernel_bounded_wait(P, oracle_mod, monkeypatch):
+    # the failure-detection hook on the two-SM kernel: the first CTA never
+    # arms its first stage; both CTAs of its pair give up within their bounds,
+    # meet at the final cluster barrier, and the handle works afterwards
+    N, K, M = 4096, 512, 1300
+    w, xc, x = make_problem(N, K, 64, M, seed=47)
+    nt = (N // 128) * (K // 128)
+    tmap = inputs.random_map(nt, nt, seed=47)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    monkeypatch.setenv("PATCH_B200_TEST_STALL", "1")
+    P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    monkeypatch.delenv("PATCH_B200_TEST_STALL")
+    assert P.patch_get_status(pk) == 5
+    assert P.patch_get_status(pk) == 0
+    y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
+    g = np.random.default_rng(47)
+    ms, ns = g.integers(0, M, 3000), g.integers(0, N, 3000)
+    yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
+    rel_rms_check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, True)
+    pk.close()
