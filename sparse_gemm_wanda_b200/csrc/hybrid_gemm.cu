@@ -664,7 +664,7 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     const double t_one = static_cast<double>(waves1) * 576.0;
     if (g.duo_ok && g.K / kStep <= 448) {
         // two-SM MMA when the matrix allows it and its estimate is lowest
-        const DuoPlan dp = plan_duo_gemm(g.N, g.M, g.num_sms);
+        const DuoPlan dp = plan_duo_gemm(g.N, g.M, g.num_sms, g.max_pair_bytes);
         if (dp.bn > 0 && dp.cost <= pp.cost && dp.cost <= t_one) return launch_duo_gemm(g, dp, stream);
     }
     if (pp.cost <= t_one && g.K / kStep <= 448)

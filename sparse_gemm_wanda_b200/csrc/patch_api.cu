@@ -33,6 +33,7 @@ struct patch_packed {
     std::vector<uint64_t> chunk_desc_host;
     int dec_cp, dec_cpb, dec_nchunks;
     int duo_ok;                // bands 2p, 2p+1 agree in type at every k-step
+    int max_pair_bytes;        // largest packed k-pair
     uint32_t *status;          // device: status word, pack counter, ready flag
     int num_sms;
     cudaMemPool_t pool;
@@ -422,6 +423,13 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
                 patchk::decode_chunk_desc(table.data() + b * nsteps, nsteps, pr0, np);
         }
     h->workspace_bytes = patchk::decode_workspace_bytes(h->dec_nchunks);
+    h->max_pair_bytes = 0;
+    for (int64_t b = 0; b < bands; ++b)
+        for (int64_t q = 0; q < Q; ++q) {
+            const int64_t pb = h->pair_prefix[static_cast<size_t>(b * (Q + 1) + q + 1)] -
+                               h->pair_prefix[static_cast<size_t>(b * (Q + 1) + q)];
+            h->max_pair_bytes = std::max<int>(h->max_pair_bytes, static_cast<int>(pb));
+        }
     // the two-SM prefill kernel pairs bands 2p and 2p+1 in one instruction
     h->duo_ok = (bands % 2 == 0) ? 1 : 0;
     for (int64_t b = 0; h->duo_ok && b < bands; b += 2)
@@ -498,6 +506,7 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.dec_nchunks = Wp->dec_nchunks;
     g.packed_rows = Wp->packed_bytes / 128;
     g.duo_ok = Wp->duo_ok;
+    g.max_pair_bytes = Wp->max_pair_bytes;
     g.num_sms = Wp->num_sms;
     g.pair_prefix = Wp->pair_prefix.data();
     // Failure-detection test hook: with PATCH_B200_TEST_STALL=1 in the

@@ -51,6 +51,7 @@ struct GemmLaunch {
     uint32_t *counter;                // device: chunks claimed, zero between calls
     uint64_t packed_rows;             // packed bytes / 128
     int duo_ok;                       // bands 2p, 2p+1 agree in type at every k-step
+    int max_pair_bytes;               // largest packed k-pair of the matrix
     int num_sms;
     int stall_first_kstep;   // failure-detection test hook (see patch_hybrid_gemm)
     const int64_t *pair_prefix;  // host: per band, cumulative packed bytes of its k-pairs
@@ -83,9 +84,10 @@ struct DuoPlan {
     int ttiles, items;
     int clusters;     // CTA pairs launched
     int stages, stage_bytes, smem;
+    int aslot;        // weight slot of a stage (the largest k-pair, rounded to 1 KB)
     double cost;      // waves x estimated cycles per k-step of an item
 };
-DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms);
+DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms, int max_pair_bytes);
 cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream_t stream);
 double duo_kstep_cycles(int bn);
 

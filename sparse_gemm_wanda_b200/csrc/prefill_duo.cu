@@ -51,7 +51,7 @@ constexpr int kDuoThreads = 224;   // + warp 6: the X-tile producer
 constexpr int kDuoMaxStages = 8;
 constexpr int kDuoTabSteps = 448;                      // k-steps per band (K <= 28672)
 constexpr int kDuoTabBytes = 2 * kDuoTabSteps * 8;     // two items of one band
-constexpr int kDuoAslot = 2 * kDenseStepBytes;  // one k-pair of weights, at most
+constexpr int kDuoAslotMax = 2 * kDenseStepBytes;  // one k-pair of weights, at most
 constexpr int kDuoTmemCols = 512;
 constexpr int kDuoSmemLimit = 232448;
 constexpr int kDuoTailBytes = 1024 + kDuoTabBytes + 512;
@@ -153,6 +153,7 @@ struct DuoParams {
     int64_t N, K, M;
     int nsteps, bands, ttiles, items;
     int bn, half, stages, stage_bytes;
+    int aslot;  // bytes of a stage's weight slot: the largest k-pair of this matrix
     void *Y;
     int y_fp32;
     uint32_t *status;
@@ -335,7 +336,7 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
                     }
                     ++it;
                     if (rank == 0) mbar_arrive_expect_tx(&full[s], x_bytes);
-                    tma3d_pair(smem + s * p.stage_bytes + kDuoAslot, &maps.x, 0,
+                    tma3d_pair(smem + s * p.stage_bytes + p.aslot, &maps.x, 0,
                                tt * bn + static_cast<int>(rank) * half, 2 * pr, map_to_rank(&full[s], 0));
                 }
             }
@@ -374,7 +375,7 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
                     for (int h = 0; h < 2; ++h) {
                         const uint64_t e = stage_info[2 * s + h];
                         const uint32_t a_addr = slot + static_cast<uint32_t>((e & kEntryOffsetMask) - first);
-                        const uint32_t b_addr = slot + kDuoAslot + static_cast<uint32_t>(h * half * kStep * 2);
+                        const uint32_t b_addr = slot + static_cast<uint32_t>(p.aslot + h * half * kStep * 2);
                         const bool fresh = pr == 0 && h == 0;
                         if (e & kEntrySparse) {
                             if (e & kEntryMeta)
@@ -519,12 +520,15 @@ double duo_kstep_cycles(int bn) {
     return std::max(2.0 * bn, 256.0 + bn);
 }
 
-DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms) {
+DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms, int max_pair_bytes) {
     DuoPlan best{};
     const int64_t bpairs = (N / kBand) / 2;
     // shared memory per stage: 16 KB of weights + BN/2 tokens x 128 B
-    auto smem_for = [](int bn, int *stages, int *stage_bytes) {
-        *stage_bytes = kDuoAslot + 2 * (bn / 2) * kStep * 2;
+    // a matrix without dense k-pairs needs only an 18 KB weight slot, which
+    // leaves room for one more stage
+    const int aslot = std::min(kDuoAslotMax, (std::max(max_pair_bytes, 2048) + 1023) / 1024 * 1024);
+    auto smem_for = [aslot](int bn, int *stages, int *stage_bytes) {
+        *stage_bytes = aslot + 2 * (bn / 2) * kStep * 2;
         *stages = std::min(kDuoMaxStages, (kDuoSmemLimit - kDuoTailBytes) / *stage_bytes);
         return *stages * *stage_bytes + kDuoTailBytes;
     };
@@ -547,6 +551,7 @@ DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms) {
         }
     }
     best.smem = smem_for(best.bn, &best.stages, &best.stage_bytes);
+    best.aslot = aslot;
     // the same work in per-SM units as the band-pair kernel's estimate: a
     // cluster item covers two SMs, so compare per-SM cycles
     best.cost = best_cost;
@@ -591,6 +596,7 @@ cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream
     p.half = plan.bn / 2;
     p.stages = plan.stages;
     p.stage_bytes = plan.stage_bytes;
+    p.aslot = plan.aslot;
     p.Y = g.Y;
     p.y_fp32 = g.y_fp32;
     p.status = g.status;
