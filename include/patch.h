@@ -144,6 +144,35 @@ patch_status patch_score_mask_noalloc(const void *W_bf16, const void *Xcal_bf16,
 size_t patch_score_mask_noalloc_capacity(void);
 
 /*
+ * Global tile allocation over several matrices of one block (the ablation in
+ * section 4 of "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs": a
+ * single sparsity target for the block, which lets each layer's share vary,
+ * beats the same target in every layer).  The pages learn the allocation by
+ * training; this is its data-free stand-in with Wanda tile losses: of all the
+ * tiles of the `count` matrices, the floor(fraction * total) with the least
+ * pruned-score loss become 2:4.  Ties in loss go to the lower global index,
+ * where the matrices are taken in the order given (tile t of matrix m has
+ * index n_tiles[0] + ... + n_tiles[m-1] + t).
+ *
+ * losses[m]   DEVICE fp64 [n_tiles[m]]: matrix m's tile losses, as written by
+ *             patch_score_mask's tile_loss_out (the caller owns them).
+ * n_tiles[m]  HOST: tile count of matrix m (>= 1).
+ * count       1..64 matrices.  With count = 1 the result equals the map
+ *             patch_score_mask selects for the same fraction.
+ * fraction    0..1 of ALL tiles.
+ * maps_out[m] DEVICE uint32 [ceil(n_tiles[m] / 32)]: matrix m's bitmap (bit
+ *             t % 32 of word t / 32 set for a 2:4 tile), for patch_score_mask's
+ *             map_in and patch_pack.
+ * Stream-ordered on `stream`; scratch comes from the library's pool.
+ * Errors: PATCH_ERR_INVALID_ARG for null pointers, count outside 1..64, a
+ * zero tile count or fraction outside [0, 1]; PATCH_ERR_UNSUPPORTED above
+ * 65535 * 256 tiles in all.
+ */
+patch_status patch_select_maps_global(const double *const *losses, const int64_t *n_tiles,
+                                      int32_t count, double fraction, uint32_t *const *maps_out,
+                                      void *stream);
+
+/*
  * Compressor: lay the dense tiles and the 2:4-compressed tiles (kept values +
  * metadata) out for the hybrid GEMM.  Compressed storage is what turns
  * zeros into speed (SparseGPT-vs-Wanda page, section on structured vs

@@ -51,6 +51,7 @@ def _load():
             "oracle_tile_loss": [p, p, i64, i64, i64, i64, p],
             "oracle_n_sparse": [ctypes.c_double, i64],
             "oracle_select_map": [p, i64, i64, p],
+            "oracle_select_maps_global": [p, p, i64, i64, p, p],
             "oracle_weff": [p, p, p, i64, i64, i64, i64, p],
             "oracle_pack_bytes": [p, i64, i64, i64, i64],
             "oracle_pack": [p, p, p, i64, i64, i64, i64, p, p],
@@ -128,6 +129,20 @@ def select_map(loss: np.ndarray, n_sp: int) -> np.ndarray:
     out = np.zeros((n + 31) // 32, dtype=np.uint32)
     _load().oracle_select_map(_ptr(loss), n, int(n_sp), _ptr(out))
     return out
+
+
+def select_maps_global(losses, fraction: float) -> list:
+    """Per-matrix bitmaps of the floor(fraction * all tiles) tiles of least
+    loss over ALL the matrices (ties: lower matrix, then lower tile)."""
+    losses = [np.ascontiguousarray(l, dtype=np.float64) for l in losses]
+    n = np.array([l.shape[0] for l in losses], dtype=np.int64)
+    words = (n + 31) // 32
+    woff = np.concatenate([[0], np.cumsum(words)[:-1]]).astype(np.int64)
+    cat = np.ascontiguousarray(np.concatenate(losses)) if losses else np.zeros(0)
+    out = np.zeros(int(words.sum()) + 1, dtype=np.uint32)
+    n_sp = n_sparse(fraction, int(n.sum()))
+    _load().oracle_select_maps_global(_ptr(cat), _ptr(n), len(losses), int(n_sp), _ptr(out), _ptr(woff))
+    return [out[woff[m]:woff[m] + words[m]].copy() for m in range(len(losses))]
 
 
 def weff(w_bits, meta, tile_map, tn: int, tk: int) -> np.ndarray:

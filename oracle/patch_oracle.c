@@ -240,6 +240,36 @@ void oracle_select_map(const double *loss, int64_t n_tiles, int64_t n_sparse,
     free(kt);
 }
 
+/*
+ * Global tile allocation over several matrices (the ablation in section 4 of
+ * "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs": one sparsity target
+ * for a whole block, so each layer's share may vary, beats one target per
+ * layer).  The pages learn that allocation; without training, the
+ * n_sparse tiles of least Wanda tile loss over ALL matrices become 2:4.
+ * Matrices are concatenated in the order given: tile t of matrix m has the
+ * global index offset[m] + t, and ties in loss go to the lower global index.
+ * loss: concatenated losses (total tiles); maps: the per-matrix bitmaps,
+ * concatenated, matrix m's words starting at word_offset[m].
+ */
+void oracle_select_maps_global(const double *loss, const int64_t *n_tiles, int64_t count,
+                               int64_t n_sparse, uint32_t *maps, const int64_t *word_offset) {
+    int64_t total = 0;
+    for (int64_t m = 0; m < count; ++m) total += n_tiles[m];
+    uint32_t *global = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)((total + 31) / 32 + 1));
+    oracle_select_map(loss, total, n_sparse, global);
+    int64_t base = 0;
+    for (int64_t m = 0; m < count; ++m) {
+        uint32_t *mm = maps + word_offset[m];
+        for (int64_t w = 0; w < (n_tiles[m] + 31) / 32; ++w) mm[w] = 0;
+        for (int64_t t = 0; t < n_tiles[m]; ++t) {
+            const int64_t g = base + t;
+            if ((global[g / 32] >> (g % 32)) & 1u) mm[t / 32] |= 1u << (t % 32);
+        }
+        base += n_tiles[m];
+    }
+    free(global);
+}
+
 static int tile_is_sparse(const uint32_t *map, int64_t t) {
     return (int)((map[t / 32] >> (t % 32)) & 1u);
 }

@@ -237,6 +237,7 @@ rank_tiles_kernel(const double *__restrict__ loss, int64_t n_tiles, int64_t n_sp
         }
         atomicAdd(rank + t, r);
     }
+    if (!map) return;  // the caller turns ranks into bitmaps itself
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0)
@@ -253,6 +254,54 @@ rank_tiles_kernel(const double *__restrict__ loss, int64_t n_tiles, int64_t n_sp
         }
         map[wd] = bits;
     }
+}
+
+// Global tile allocation: bit t of matrix m's bitmap is set iff the tile's
+// rank over all matrices (concatenated, matrix m starting at offset[m]) is
+// below n_sparse.  One thread per output word.
+struct GlobalMaps {
+    uint32_t *map[kMaxGlobalMatrices];
+    int64_t offset[kMaxGlobalMatrices + 1];  // first global tile of each matrix; [count] = total
+    int64_t word0[kMaxGlobalMatrices + 1];   // first output word of each matrix (prefix)
+    int count;
+};
+
+__global__ void __launch_bounds__(128)
+split_maps_kernel(const int32_t *__restrict__ rank, int64_t n_sparse, const __grid_constant__ GlobalMaps g) {
+    const int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (w >= g.word0[g.count]) return;
+    int m = 0;
+    while (m + 1 < g.count && g.word0[m + 1] <= w) ++m;
+    const int64_t lw = w - g.word0[m];
+    const int64_t n = g.offset[m + 1] - g.offset[m];
+    uint32_t bits = 0;
+    for (int q = 0; q < 32; ++q) {
+        const int64_t t = lw * 32 + q;
+        if (t < n && rank[g.offset[m] + t] < n_sparse) bits |= 1u << q;
+    }
+    g.map[m][lw] = bits;
+}
+
+cudaError_t launch_select_maps_global(const double *loss_cat, const int64_t *n_tiles, int count,
+                                      int64_t n_sparse, int32_t *rank, uint32_t *const *maps,
+                                      cudaStream_t stream) {
+    if (count < 1 || count > kMaxGlobalMatrices) return cudaErrorInvalidValue;
+    GlobalMaps g;
+    g.count = count;
+    g.offset[0] = 0;
+    g.word0[0] = 0;
+    for (int m = 0; m < count; ++m) {
+        g.map[m] = maps[m];
+        g.offset[m + 1] = g.offset[m] + n_tiles[m];
+        g.word0[m + 1] = g.word0[m] + (n_tiles[m] + 31) / 32;
+    }
+    const int64_t total = g.offset[count];
+    dim3 grid(static_cast<unsigned>((total + kRankThreads - 1) / kRankThreads),
+              static_cast<unsigned>((total + kRankSlice - 1) / kRankSlice));
+    rank_tiles_kernel<<<grid, kRankThreads, 0, stream>>>(loss_cat, total, n_sparse, rank, nullptr, nullptr);
+    split_maps_kernel<<<static_cast<unsigned>((g.word0[count] + 127) / 128), 128, 0, stream>>>(rank, n_sparse, g);
+    note_launches(2);
+    return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ launch

@@ -332,6 +332,47 @@ patch_status patch_score_mask_noalloc(const void *W_bf16, const void *Xcal_bf16,
 
 size_t patch_score_mask_noalloc_capacity(void) { return kNoallocScratchBytes; }
 
+patch_status patch_select_maps_global(const double *const *losses, const int64_t *n_tiles,
+                                      int32_t count, double fraction, uint32_t *const *maps_out,
+                                      void *stream_v) {
+    if (!losses || !n_tiles || !maps_out || count < 1 || count > patchk::kMaxGlobalMatrices)
+        return PATCH_ERR_INVALID_ARG;
+    if (!(fraction >= 0.0 && fraction <= 1.0)) return PATCH_ERR_INVALID_ARG;
+    int64_t total = 0;
+    for (int32_t m = 0; m < count; ++m) {
+        if (!losses[m] || !maps_out[m] || n_tiles[m] < 1) return PATCH_ERR_INVALID_ARG;
+        total += n_tiles[m];
+    }
+    if (total > patchk::kMaxGlobalTiles) return PATCH_ERR_UNSUPPORTED;
+    patch_status st = check_device(nullptr);
+    if (st != PATCH_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    // scratch: the losses concatenated | a rank counter per tile
+    const size_t off_rank = round_up(sizeof(double) * static_cast<size_t>(total), 256);
+    const size_t bytes = off_rank + sizeof(int32_t) * static_cast<size_t>(total);
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = patchk::device_pool(&pool);
+    if (e != cudaSuccess) return from_cuda(e);
+    uint8_t *scratch = nullptr;
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&scratch), bytes, pool, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    double *cat = reinterpret_cast<double *>(scratch);
+    int32_t *rank = reinterpret_cast<int32_t *>(scratch + off_rank);
+    int64_t off = 0;
+    for (int32_t m = 0; m < count && e == cudaSuccess; ++m) {
+        e = cudaMemcpyAsync(cat + off, losses[m], sizeof(double) * static_cast<size_t>(n_tiles[m]),
+                            cudaMemcpyDeviceToDevice, stream);
+        off += n_tiles[m];
+    }
+    if (e == cudaSuccess) e = cudaMemsetAsync(rank, 0, sizeof(int32_t) * static_cast<size_t>(total), stream);
+    if (e == cudaSuccess) {
+        const int64_t n_sp = static_cast<int64_t>(floor(fraction * static_cast<double>(total)));
+        e = patchk::launch_select_maps_global(cat, n_tiles, count, n_sp, rank, maps_out, stream);
+    }
+    cudaError_t e2 = cudaFreeAsync(scratch, stream);
+    return from_cuda(e != cudaSuccess ? e : e2);
+}
+
 uint64_t patch_launch_count(void) { return patchk::g_launches.load(std::memory_order_relaxed); }
 
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,

@@ -21,6 +21,16 @@ cudaError_t launch_score_mask(const void *W, const double *norm, int64_t N, int6
 cudaError_t launch_select_map(const double *loss, int64_t n_tiles, int64_t n_sparse, int32_t *rank,
                               uint32_t *done, uint32_t *map, cudaStream_t stream);
 
+// Global tile allocation over up to kMaxGlobalMatrices matrices: `loss_cat`
+// holds their tile losses concatenated, `rank` (zeroed, one per tile) is
+// scratch; writes each matrix's bitmap to maps[m].
+constexpr int kMaxGlobalMatrices = 64;
+// the rank kernel's grid.y counts 256-tile slices of all tiles (<= 65535)
+constexpr int64_t kMaxGlobalTiles = 65535LL * 256;
+cudaError_t launch_select_maps_global(const double *loss_cat, const int64_t *n_tiles, int count,
+                                      int64_t n_sparse, int32_t *rank, uint32_t *const *maps,
+                                      cudaStream_t stream);
+
 // `done` (a zeroed counter) and `ready` (zeroed) live in the handle: the last
 // block to finish publishes ready = 1 with release semantics.
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,

@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "PATCH_OK", 1: "PATCH_ERR_INVALID_ARG", 2: "PATCH_ERR_UNSUPPO
 EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
            "patch_get_status", "patch_packed_info", "patch_packed_export",
            "patch_status_string", "patch_score_mask_noalloc",
-           "patch_score_mask_noalloc_capacity", "patch_launch_count")
+           "patch_score_mask_noalloc_capacity", "patch_launch_count",
+           "patch_select_maps_global")
 
 
 class PatchLibraryError(RuntimeError):
@@ -70,6 +71,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.patch_score_mask_noalloc.restype = ctypes.c_int
     lib.patch_score_mask_noalloc_capacity.argtypes = []
     lib.patch_score_mask_noalloc_capacity.restype = ctypes.c_size_t
+    lib.patch_select_maps_global.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(i64), i32, dbl,
+                                             ctypes.POINTER(vp), vp]
+    lib.patch_select_maps_global.restype = ctypes.c_int
     lib.patch_launch_count.argtypes = []
     lib.patch_launch_count.restype = ctypes.c_uint64
     lib.patch_pack.argtypes = [vp, vp, vp, PatchShape, ctypes.POINTER(vp),
@@ -208,6 +212,21 @@ class PackedWeight:
             self.close()
         except Exception:
             pass
+
+
+def patch_select_maps_global(losses: list, fraction: float, stream=None) -> list:
+    """Tile maps for several matrices at one block-wide target: the
+    floor(fraction * all tiles) tiles of least loss over all matrices become
+    2:4.  `losses` are the fp64 tile losses from patch_score_mask(want_loss=True)."""
+    lib = load_library()
+    count = len(losses)
+    maps = [torch.empty(((l.numel() + 31) // 32,), dtype=torch.int32, device=l.device) for l in losses]
+    lp = (ctypes.c_void_p * count)(*[_dptr(l, torch.float64, "loss").value for l in losses])
+    mp = (ctypes.c_void_p * count)(*[m.data_ptr() for m in maps])
+    nt = (ctypes.c_int64 * count)(*[l.numel() for l in losses])
+    code = lib.patch_select_maps_global(lp, nt, count, float(fraction), mp, _stream(stream))
+    _check("patch_select_maps_global", code)
+    return maps
 
 
 def patch_pack(W: torch.Tensor, meta: torch.Tensor, tile_map: torch.Tensor, *, tile_n: int = 128,

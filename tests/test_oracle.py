@@ -297,6 +297,62 @@ def test_map_all_ties_take_lowest_indices(oracle_mod):
 
 
 # ----------------------------------------------------------------------------
+# global tile allocation over the matrices of a block (PATCH, section 4,
+# ablation on a block-wide target against a per-layer one)
+
+
+def test_global_maps_hand_example(oracle_mod):
+    # two matrices, 3 + 2 tiles; 40 % of 5 tiles = 2 tiles of least loss:
+    # 0.1 (matrix 1, tile 0) and 0.2 (matrix 0, tile 1)
+    maps = oracle_mod.select_maps_global([np.array([0.5, 0.2, 0.9]), np.array([0.1, 0.7])], 0.4)
+    assert [int(m[0]) for m in maps] == [0b010, 0b01]
+    # 60 %: the next is 0.5 (matrix 0, tile 0)
+    maps = oracle_mod.select_maps_global([np.array([0.5, 0.2, 0.9]), np.array([0.1, 0.7])], 0.6)
+    assert [int(m[0]) for m in maps] == [0b011, 0b01]
+
+
+def test_global_maps_single_matrix_is_the_per_matrix_map(oracle_mod):
+    rng = np.random.default_rng(5)
+    loss = rng.standard_normal(777).round(1)
+    for f in [0.0, 0.3, 0.6, 1.0]:
+        (m,) = oracle_mod.select_maps_global([loss], f)
+        ref = oracle_mod.select_map(loss, oracle_mod.n_sparse(f, 777))
+        assert np.array_equal(m, ref[:len(m)])
+
+
+def test_global_maps_invariants(oracle_mod):
+    rng = np.random.default_rng(6)
+    sizes = [33, 1, 100, 64, 7]
+    # different scales per matrix, so the shares differ from the target
+    losses = [rng.standard_normal(n).round(1) * (1 + 2 * i) for i, n in enumerate(sizes)]
+    total = sum(sizes)
+    cat = np.concatenate(losses)
+    for f in [0.0, 0.25, 0.5, 0.99, 1.0]:
+        maps = oracle_mod.select_maps_global(losses, f)
+        bits = np.concatenate([bits_of(m, n) for m, n in zip(maps, sizes)])
+        ns = int(np.floor(f * total))
+        assert bits.sum() == ns
+        for m, n in zip(maps, sizes):
+            assert len(m) == (n + 31) // 32
+            assert popcount(m) == bits_of(m, n).sum()  # no bits past the last tile
+        if 0 < ns < total:
+            assert cat[bits].max() <= cat[~bits].min()
+            v = cat[bits].max()
+            chosen = np.where(bits & (cat == v))[0]
+            left = np.where(~bits & (cat == v))[0]
+            if len(left):
+                assert chosen.max() < left.min()
+
+
+def test_global_maps_ties_go_to_the_earlier_matrix(oracle_mod):
+    maps = oracle_mod.select_maps_global([np.full(40, 1.0), np.full(40, 1.0)], 0.75)
+    # 60 of 80 tied tiles: all of matrix 0, then tiles 0..19 of matrix 1
+    assert bits_of(maps[0], 40).all()
+    b1 = bits_of(maps[1], 40)
+    assert b1[:20].all() and not b1[20:].any()
+
+
+# ----------------------------------------------------------------------------
 # effective weight and product
 # ----------------------------------------------------------------------------
 

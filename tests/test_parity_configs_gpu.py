@@ -190,3 +190,39 @@ def test_block_config(P, block):
                 sampled_check(y, xb, weff, 3000, seed=M + mi, fp32_mode=False)
         assert P.patch_get_status(pk) == 0
         pk.close()
+
+
+def test_block_config_global_allocation(P, block):
+    """One 2:4-tile target for the whole block (30 % sparsity = 60 % of all
+    tiles), spread over the seven matrices by least loss; maps bit-exact."""
+    wl, mats, calib, outl = block
+    frac = wl.fractions[0]
+    colsq_dev = {}
+    colsq_ref = {}
+    losses_dev, losses_ref, sizes = [], [], []
+    for m, w in mats:
+        g = m.input_group
+        wd = w.cuda()
+        if g not in colsq_dev:
+            xc = calib[g].cuda()
+            r = P.patch_score_mask(wd, xc, want_colsq=True, want_loss=True)
+            colsq_dev[g] = r["colsq"]
+            del xc
+            colsq_ref[g] = oracle.colsq(bf16_bits(calib[g]))
+        else:
+            r = P.patch_score_mask(wd, None, colsq_in=colsq_dev[g], want_loss=True)
+        sc = oracle.wanda_scores(bf16_bits(w), colsq_ref[g])
+        loss = oracle.tile_loss(sc, oracle.select_2of4(sc), 128, 128)
+        losses_dev.append(r["loss"])
+        losses_ref.append(loss)
+        sizes.append(loss.shape[0])
+    maps = P.patch_select_maps_global(losses_dev, frac)
+    torch.cuda.synchronize()
+    for ld, lr in zip(losses_dev, losses_ref):
+        assert np.array_equal(ld.cpu().numpy(), lr)
+    ref = oracle.select_maps_global(losses_ref, frac)
+    chosen = 0
+    for (m, _), md, mr in zip(mats, maps, ref):
+        assert np.array_equal(u32(md), mr), m.name
+        chosen += sum(bin(int(v)).count("1") for v in mr)
+    assert chosen == oracle.n_sparse(frac, sum(sizes))

@@ -116,6 +116,74 @@ def test_mask_builder_ties(P, oracle_mod):
     assert np.array_equal(r["loss"].cpu().numpy(), ref["loss"])
 
 
+# ------------------------------------------------- global tile allocation
+
+@pytest.mark.parametrize("frac", [0.0, 0.3, 0.6, 0.999, 1.0])
+def test_global_maps_random_losses(P, oracle_mod, frac):
+    # ragged tile counts (word boundaries, one-tile matrices) and many ties;
+    # enough tiles in all that the rank kernel runs over several slices
+    g = np.random.default_rng(11)
+    sizes = [1, 31, 32, 33, 1000, 4095, 7, 64, 2500]
+    losses = [np.round(g.standard_normal(n) * (1 + i % 3), 1) for i, n in enumerate(sizes)]
+    maps = P.patch_select_maps_global([torch.from_numpy(l).cuda() for l in losses], frac)
+    torch.cuda.synchronize()
+    ref = oracle_mod.select_maps_global(losses, frac)
+    for m, r in zip(maps, ref):
+        assert np.array_equal(u32(m), r)
+
+
+def test_global_maps_64_matrices(P, oracle_mod):
+    g = np.random.default_rng(12)
+    losses = [np.round(g.exponential(1.0 + (i % 5), int(g.integers(1, 300))), 2) for i in range(64)]
+    maps = P.patch_select_maps_global([torch.from_numpy(l).cuda() for l in losses], 0.45)
+    torch.cuda.synchronize()
+    for m, r in zip(maps, oracle_mod.select_maps_global(losses, 0.45)):
+        assert np.array_equal(u32(m), r)
+
+
+def test_global_maps_one_matrix_equals_the_mask_builder_map(P, oracle_mod):
+    w, xc, _ = make_problem(512, 768, 128, 1, seed=21)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), tile_n=64, tile_k=64, fraction=0.4,
+                           want_loss=True)
+    (m,) = P.patch_select_maps_global([r["loss"]], 0.4)
+    torch.cuda.synchronize()
+    assert np.array_equal(u32(m), u32(r["map"]))
+
+
+def test_global_maps_from_mask_builder_losses(P, oracle_mod):
+    # three matrices of one block sharing a calibration set; the block-wide
+    # map then feeds the mask builder's given-map mode and the packer
+    K = 512
+    o = inputs.outlier_channels(K, 31)
+    xc = inputs.activations(256, K, 31, o, role=0)
+    ws = [inputs.weight(n, K, 31 + n) for n in (256, 384, 640)]
+    res = [P.patch_score_mask(w.cuda(), xc.cuda(), want_loss=True, want_colsq=True) for w in ws]
+    maps = P.patch_select_maps_global([r["loss"] for r in res], 0.5)
+    torch.cuda.synchronize()
+    ref_losses = []
+    for w in ws:
+        ref = oracle_mask(oracle_mod, w, xc, 128, 128, frac=0.0)
+        ref_losses.append(ref["loss"])
+    for r, l in zip(res, ref_losses):
+        assert np.array_equal(r["loss"].cpu().numpy(), l)
+    ref_maps = oracle_mod.select_maps_global(ref_losses, 0.5)
+    for w, m, rm in zip(ws, maps, ref_maps):
+        assert np.array_equal(u32(m), rm)
+        r2 = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=m)
+        pk = P.patch_pack(w.cuda(), r2["meta"], r2["map"])
+        torch.cuda.synchronize()
+        assert np.array_equal(u32(r2["map"]), rm)
+        pk.close()
+
+
+def test_global_maps_bad_arguments(P):
+    l = torch.zeros(10, dtype=torch.float64, device="cuda")
+    for losses, f in [([l], -0.1), ([l], 1.5), ([l] * 65, 0.5)]:
+        with pytest.raises(P.PatchError) as e:
+            P.patch_select_maps_global(losses, f)
+        assert e.value.code == 1  # PATCH_ERR_INVALID_ARG
+
+
 # ----------------------------------------------------------------------- pack
 
 @pytest.mark.parametrize("tn,tk", [(64, 64), (128, 128), (64, 128), (128, 64)])
