@@ -17,11 +17,21 @@
 // descriptor (byte offset + the 2:4 flags of its k-steps) is enough to place
 // every k-step, so no table is read: the descriptors of the CTAs' first
 // chunks travel in the kernel parameters and the first copies start at once.
-// One bulk copy per pair (16-32 KB) and one 3-D TMA load of the pair's X
-// tiles (16 rows, rows past M read as zero) complete on the stage mbarrier.
+// A pipeline stage holds two consecutive k-pairs of a chunk (a k-quad, 256
+// input columns): one bulk copy of their packed bytes (36-64 KB) and one 3-D
+// TMA load of their four X tiles (16 rows, rows past M read as zero).  Few,
+// large copies matter: an SM's copy engine spends about as long on a small
+// copy as on a 16 KB one.
+//
+// Issue.  One thread issues every tensor-core instruction of the CTA, and on
+// B200 each tcgen05.mma costs that thread about 75 cycles whatever N is (N =
+// 16 here), a metadata copy about 180 and a commit about 140.  The MMA
+// thread therefore does nothing else: it derives the k-step layout of a stage
+// from the stage's flag word in registers, builds descriptors by adding byte
+// offsets to per-stage base descriptors, and commits once per stage.
 //
 // Launch.  A programmatic dependent of the previous kernel: once the packer's
-// ready flag is seen, the first chunk's weight copies are issued before
+// ready flag is seen, the first stages' weight copies are issued before
 // `griddepcontrol.wait`; X, Y, the partials and the chunk counter are touched
 // only after it.  The fix-up kernel resets the counter for the next call.
 //
@@ -46,25 +56,30 @@ namespace {
 
 constexpr int kDecThreads = 192;
 constexpr int kDecBN = 16;                                // token rows of the MMA (N = 16)
-constexpr int kDecStages = 5;
-constexpr int kDecABytes = 2 * kDenseStepBytes;           // a pair of packed k-steps, at most
-constexpr int kDecBBytes = 2 * kDecBN * kStep * 2;        // the pair's two X tiles
-constexpr int kDecStageBytes = kDecABytes + kDecBBytes;   // 36864
-constexpr int kDecTmemCols = 64;                          // 2 x 16 accumulator + 4 metadata
+constexpr int kDecStages = 3;
+constexpr int kDecChunkPairs = 4;                         // k-pairs per chunk, at most
+constexpr int kDecWBytes = 4 * kDenseStepBytes;           // two packed k-pairs, at most
+constexpr int kDecXStepBytes = kDecBN * kStep * 2;        // one k-step of X: 16 rows x 64
+constexpr int kDecXBytes = 4 * kDecXStepBytes;            // the stage's four X tiles
+constexpr int kDecStageBytes = kDecWBytes + kDecXBytes;   // 73728
+constexpr int kDecTmemCols = 64;                          // 2 x 16 accumulator + 2 x 4 metadata
 constexpr uint32_t kDecEcol = 2 * kDecBN;
 constexpr int kDecSmemBytes = kDecStages * kDecStageBytes + 1024 + 512;
 constexpr uint64_t kDecWaitLimitNs = 2000000000ull;       // 2 s per wait
-
-constexpr uint32_t kTagDone = 1u << 31;   // no more work
-constexpr uint32_t kTagFirst = 1u << 30;  // first pair of its chunk
-constexpr uint32_t kTagLast = 1u << 29;   // last pair of its chunk
-constexpr uint32_t kTagChunk = (1u << 29) - 1;
 
 // chunk descriptor: first byte (40 bits) | 2:4 flag of each k-step (16) | pairs (4)
 constexpr uint64_t kDescOffsetMask = (1ull << 40) - 1;
 constexpr int kDescFlagsShift = 40;
 constexpr int kDescPairsShift = 56;
-constexpr int kDecMaxChunkPairs = 8;
+
+// stage word: chunk (29 bits) | first stage of its chunk | last stage |
+// no more work | pairs in the stage (1 or 2) << 32 | k-step 2:4 flags << 36
+constexpr uint64_t kStageChunk = (1ull << 29) - 1;
+constexpr uint64_t kStageFirst = 1ull << 29;
+constexpr uint64_t kStageLast = 1ull << 30;
+constexpr uint64_t kStageDone = 1ull << 31;
+constexpr int kStagePairsShift = 32;
+constexpr int kStageFlagsShift = 36;
 
 struct DecodeParams {
     const uint8_t *packed;
@@ -83,34 +98,14 @@ struct DecodeParams {
     uint64_t first_desc[kDecMaxCtas];  // chunk_desc[c] for c < gridDim.x
 };
 
-// Place pair i of a chunk: its table-equivalent entries, first byte and size.
-// Mirrors the packer: a 2 KB metadata block precedes the first 2:4 k-step of
-// every k-pair.
-__device__ __forceinline__ void chunk_pair(uint64_t &cur, uint32_t flags, int i, uint64_t &e0,
-                                           uint64_t &e1, uint64_t &first, uint32_t &bytes) {
-    const bool s0 = (flags >> (2 * i)) & 1u, s1 = (flags >> (2 * i + 1)) & 1u;
-    first = cur;
-    if (s0) {
-        cur += kMetaBlockBytes;
-        e0 = kEntrySparse | kEntryMeta | cur;
-        cur += kSparseStepBytes;
-    } else {
-        e0 = cur;
-        cur += kDenseStepBytes;
-    }
-    if (s1) {
-        uint64_t m = 0;
-        if (!s0) {
-            cur += kMetaBlockBytes;
-            m = kEntryMeta;
-        }
-        e1 = kEntrySparse | m | cur;
-        cur += kSparseStepBytes;
-    } else {
-        e1 = cur;
-        cur += kDenseStepBytes;
-    }
-    bytes = static_cast<uint32_t>(cur - first);
+// Bytes of pair i of a chunk whose k-step flags are `flags`, and whether its
+// metadata block is present.  Mirrors the packer: a 2 KB metadata block
+// precedes the first 2:4 k-step of every k-pair.
+__device__ __forceinline__ uint32_t pair_bytes(uint32_t flags, int i) {
+    const uint32_t f = (flags >> (2 * i)) & 3u;
+    return (f == 0u) ? 2u * kDenseStepBytes
+                     : (f == 3u) ? kMetaBlockBytes + 2u * kSparseStepBytes
+                                 : kMetaBlockBytes + kDenseStepBytes + kSparseStepBytes;
 }
 
 __device__ __forceinline__ void store_out(const DecodeParams &p, int64_t idx, float v) {
@@ -133,8 +128,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
     volatile uint32_t *abort_flag = tmem_slot + 1;  // raised by any role that gives up
     volatile uint32_t *never_flag = tmem_slot + 2;  // stays 0: time-only bounded waits
     volatile int32_t *acc_chunk = reinterpret_cast<volatile int32_t *>(tmem_slot + 4);  // [2]
-    uint64_t *stage_info = reinterpret_cast<uint64_t *>(tmem_slot + 8);                 // [STAGES][3]
-    uint32_t *stage_tag = reinterpret_cast<uint32_t *>(stage_info + 3 * kDecStages);    // [STAGES]
+    uint64_t *stage_word = reinterpret_cast<uint64_t *>(tmem_slot + 8);                 // [STAGES]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     bool waited = true;  // thread 0: past griddepcontrol.wait
@@ -171,16 +165,16 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
     if (warp == 0) {
         if (lane == 0 && !skip) {
             // ------------------------------------------------------ producer
-            int it = 0;  // pairs armed so far (stage ring position)
+            int it = 0;  // stages armed so far (ring position)
             bool ok = true;
-            int pend_s[kDecStages], pend_pr[kDecStages];  // X tiles of stages armed before the wait
+            int pend_s[kDecStages], pend_k[kDecStages];  // X loads of stages armed before the wait
             int npend = 0;
             auto flush_x = [&]() {
                 pdl_wait();
                 waited = true;
                 for (int q = 0; q < npend; ++q)
-                    tma_load_3d(smem + pend_s[q] * kDecStageBytes + kDecABytes, &tmap_x, 0, 0,
-                                2 * pend_pr[q], &full[pend_s[q]]);
+                    tma_load_3d(smem + pend_s[q] * kDecStageBytes + kDecWBytes, &tmap_x, 0, 0, pend_k[q],
+                                &full[pend_s[q]]);
                 npend = 0;
             };
             // the next two claimed chunks (claimed only past the wait)
@@ -203,7 +197,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                 const int np = static_cast<int>((d >> kDescPairsShift) & 0xFu);
                 const uint32_t flags = static_cast<uint32_t>((d >> kDescFlagsShift) & 0xFFFFu);
                 uint64_t cur = d & kDescOffsetMask;
-                for (int i = 0; i < np; ++i) {
+                for (int i = 0; i < np; i += 2) {
                     const int s = it % kDecStages;
                     const uint32_t ph = (it / kDecStages) & 1u;
                     if (!waited && it >= kDecStages) flush_x();
@@ -212,24 +206,25 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                         ok = false;
                         break;
                     }
-                    uint64_t e0, e1, first;
-                    uint32_t bytes;
-                    chunk_pair(cur, flags, i, e0, e1, first, bytes);
-                    stage_info[3 * s + 0] = e0;
-                    stage_info[3 * s + 1] = e1;
-                    stage_info[3 * s + 2] = first;
-                    stage_tag[s] = static_cast<uint32_t>(j) | (i == 0 ? kTagFirst : 0u) |
-                                   (i == np - 1 ? kTagLast : 0u);
+                    const int sp = min(2, np - i);
+                    const uint32_t bytes = pair_bytes(flags, i) + (sp == 2 ? pair_bytes(flags, i + 1) : 0u);
+                    const uint32_t sflags = (flags >> (2 * i)) & (sp == 2 ? 0xFu : 0x3u);
+                    stage_word[s] = static_cast<uint64_t>(j) | (i == 0 ? kStageFirst : 0ull) |
+                                    (i + sp >= np ? kStageLast : 0ull) |
+                                    (static_cast<uint64_t>(sp) << kStagePairsShift) |
+                                    (static_cast<uint64_t>(sflags) << kStageFlagsShift);
                     ++it;
+                    const uint64_t src = cur;
+                    cur += bytes;
                     if (p.stall_first_kstep && blockIdx.x == 0 && it == 1) continue;  // never lands
                     uint8_t *st = smem + s * kDecStageBytes;
-                    mbar_arrive_expect_tx(&full[s], bytes + kDecBBytes);
-                    bulk_g2s(st, p.packed + first, bytes, &full[s]);
+                    mbar_arrive_expect_tx(&full[s], bytes + kDecXBytes);
+                    bulk_g2s(st, p.packed + src, bytes, &full[s]);
                     if (waited) {
-                        tma_load_3d(st + kDecABytes, &tmap_x, 0, 0, 2 * (pr0 + i), &full[s]);
+                        tma_load_3d(st + kDecWBytes, &tmap_x, 0, 0, 2 * (pr0 + i), &full[s]);
                     } else {
                         pend_s[npend] = s;
-                        pend_pr[npend] = pr0 + i;
+                        pend_k[npend] = 2 * (pr0 + i);
                         ++npend;
                     }
                 }
@@ -248,14 +243,14 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             }
             if (!waited) flush_x();
             if (ok) {
-                // no more chunks: a stage carrying the done tag (plain arrive)
+                // no more chunks: a stage carrying the done flag (plain arrive)
                 const int s = it % kDecStages;
                 const uint32_t ph = (it / kDecStages) & 1u;
                 if (it >= kDecStages &&
                     !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kDecWaitLimitNs)) {
                     ok = false;
                 } else {
-                    stage_tag[s] = kTagDone;
+                    stage_word[s] = kStageDone;
                     mbar_arrive(&full[s]);
                     ++it;
                 }
@@ -275,8 +270,17 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
     } else if (warp == 1) {
         if (lane == 0 && !skip) {
             // ---------------------------------------------------------- MMA
+            // Descriptors: a template per layout plus the operand's shared
+            // address in 16-byte units (all addresses here are below 256 KB,
+            // so the 14-bit address field never carries into other fields).
+            constexpr uint32_t kIdDense = idesc_bf16(kDecBN, false);
+            constexpr uint32_t kIdSp0 = idesc_bf16(kDecBN, true, 0);
+            constexpr uint32_t kIdSp1 = idesc_bf16(kDecBN, true, 1);
+            const uint64_t t_sw128 = smem_desc(0, 16, 1024, kSwizzle128B);  // dense A, X
+            const uint64_t t_sw64 = smem_desc(0, 16, 512, kSwizzle64B);     // 2:4 A
+            const uint64_t t_meta = smem_desc(0, 16, 128, kSwizzleNone);    // metadata
             const uint32_t e_tmem = tmem_base + kDecEcol;
-            constexpr uint32_t kIdescDense = idesc_bf16(kDecBN, false);
+            const uint32_t smem0 = smem_u32(smem);
             int it = 0, ci = 0;  // stages consumed, chunks finished
             bool ok = true;
             for (;;) {
@@ -287,10 +291,10 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     break;
                 }
                 tc_fence_after();
-                const uint32_t tag = stage_tag[s];
-                if (tag & kTagDone) break;
+                const uint64_t w = stage_word[s];
+                if (w & kStageDone) break;
                 const int buf = ci & 1;
-                if ((tag & kTagFirst) && ci >= 2 &&
+                if ((w & kStageFirst) && ci >= 2 &&
                     !mbar_wait_bounded(&acc_empty[buf], ((ci >> 1) & 1u) ^ 1u, abort_flag,
                                        kDecWaitLimitNs)) {
                     ok = false;
@@ -298,38 +302,44 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * kDecBN;
-                const uint64_t first = stage_info[3 * s + 2];
-                uint8_t *st = smem + s * kDecStageBytes;
+                const uint32_t st16 = (smem0 + s * kDecStageBytes) >> 4;  // stage, 16-byte units
+                const uint64_t x16 = t_sw128 + st16 + (kDecWBytes >> 4);
+                const int sp = static_cast<int>((w >> kStagePairsShift) & 3u);
+                const uint32_t fl = static_cast<uint32_t>(w >> kStageFlagsShift) & 0xFu;
+                uint32_t off16 = 0;  // running offset in the stage, 16-byte units
+                uint32_t acc = (w & kStageFirst) ? 0u : 1u;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint64_t e = stage_info[3 * s + h];
-                    const uint32_t a_addr =
-                        smem_u32(st + static_cast<uint32_t>((e & kEntryOffsetMask) - first));
-                    const uint32_t b_addr = smem_u32(st + kDecABytes + h * (kDecBBytes / 2));
-                    const bool fresh = (tag & kTagFirst) && h == 0;
-                    if (e & kEntrySparse) {
-                        if (e & kEntryMeta)
-                            tmem_cp_128x128b(e_tmem, smem_desc(a_addr - kMetaBlockBytes, 16, 128,
-                                                               kSwizzleNone));
+                for (int t = 0; t < 2; ++t) {
+                    if (t >= sp) break;
+                    const uint32_t f = (fl >> (2 * t)) & 3u;
 #pragma unroll
-                        for (int q = 0; q < 2; ++q) {
-                            const uint64_t ad = smem_desc(a_addr + q * 32, 16, 512, kSwizzle64B);
-                            const uint64_t bd = smem_desc(b_addr + q * 64, 16, 1024, kSwizzle128B);
-                            mma_sparse(d_tmem, ad, bd, e_tmem + 2 * h, idesc_bf16(kDecBN, true, q),
-                                       (fresh && q == 0) ? 0u : 1u);
+                    for (int h = 0; h < 2; ++h) {
+                        const uint64_t bx = x16 + (2 * t + h) * (kDecXStepBytes >> 4);
+                        if ((f >> h) & 1u) {
+                            // the pair's metadata block precedes its first 2:4 k-step
+                            if (h == 0 || !(f & 1u)) {
+                                tmem_cp_128x128b(e_tmem + 4 * t, t_meta + st16 + off16);
+                                off16 += kMetaBlockBytes >> 4;
+                            }
+                            const uint64_t a = t_sw64 + st16 + off16;
+                            const uint32_t e = e_tmem + 4 * t + 2 * h;
+                            mma_sparse(d_tmem, a, bx, e, kIdSp0, acc);
+                            mma_sparse(d_tmem, a + 2, bx + 4, e, kIdSp1, 1u);
+                            off16 += kSparseStepBytes >> 4;
+                        } else {
+                            const uint64_t a = t_sw128 + st16 + off16;
+                            mma_dense(d_tmem, a, bx, kIdDense, acc);
+                            mma_dense(d_tmem, a + 2, bx + 2, kIdDense, 1u);
+                            mma_dense(d_tmem, a + 4, bx + 4, kIdDense, 1u);
+                            mma_dense(d_tmem, a + 6, bx + 6, kIdDense, 1u);
+                            off16 += kDenseStepBytes >> 4;
                         }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint64_t ad = smem_desc(a_addr + q * 32, 16, 1024, kSwizzle128B);
-                            const uint64_t bd = smem_desc(b_addr + q * 32, 16, 1024, kSwizzle128B);
-                            mma_dense(d_tmem, ad, bd, kIdescDense, (fresh && q == 0) ? 0u : 1u);
-                        }
+                        acc = 1u;
                     }
                 }
                 tc_commit(&empty[s]);
-                if (tag & kTagLast) {
-                    acc_chunk[buf] = static_cast<int32_t>(tag & kTagChunk);
+                if (w & kStageLast) {
+                    acc_chunk[buf] = static_cast<int32_t>(w & kStageChunk);
                     tc_commit(&acc_full[buf]);
                     mbar_arrive(&acc_full[buf]);  // publishes acc_chunk
                     ++ci;
@@ -438,7 +448,7 @@ void plan_decode_chunks(int64_t bands, int64_t nsteps, int num_sms, int *cp, int
     // against 1, 2, 6 and 8 for the Llama-7B shapes; smaller chunks cost more
     // partials and claims than they gain in balance, larger ones lose balance
     (void)num_sms;
-    const int64_t c = std::min<int64_t>(std::min<int64_t>(4, kDecMaxChunkPairs), Q);
+    const int64_t c = std::min<int64_t>(kDecChunkPairs, Q);
     *cp = static_cast<int>(c);
     *cpb = static_cast<int>((Q + c - 1) / c);
     *nchunks = static_cast<int>(bands * *cpb);
@@ -469,19 +479,21 @@ cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
     if (attr_err != cudaSuccess) return attr_err;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorInvalidValue;
-    // X [M,K] viewed as (64 columns, M rows, K/64 k-steps); box = one k-pair
-    // of 16 rows, 128-byte swizzle, rows past M read as zero
+    // X [M,K] viewed as (64 columns, M rows, K/64 k-steps); box = the four
+    // k-steps of a stage, 16 rows, 128-byte swizzle, rows past M and k-steps
+    // past K read as zero
     CUtensorMap map;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kStep), static_cast<cuuint64_t>(g.M),
                                 static_cast<cuuint64_t>(g.K / kStep)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.K) * 2, static_cast<cuuint64_t>(kStep) * 2};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kStep), static_cast<cuuint32_t>(kDecBN), 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kStep), static_cast<cuuint32_t>(kDecBN), 4};
     const cuuint32_t estr[3] = {1, 1, 1};
     if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(g.X), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     if (!g.chunk_desc || !g.chunk_desc_host || !g.workspace || !g.counter) return cudaErrorInvalidValue;
+    if (g.dec_cp < 1 || g.dec_cp > kDecChunkPairs) return cudaErrorInvalidValue;
     if (decode_workspace_bytes(g.dec_nchunks) > g.workspace_bytes) return cudaErrorInvalidValue;
 
     DecodeParams p;
