@@ -23,22 +23,25 @@
 // large copies matter: an SM's copy engine spends about as long on a small
 // copy as on a 16 KB one.
 //
-// Issue.  One thread issues every tensor-core instruction of the CTA, and on
-// B200 each tcgen05.mma costs that thread about 75 cycles whatever N is (N =
-// 16 here), a metadata copy about 180 and a commit about 140.  The MMA
-// thread therefore does nothing else: it derives the k-step layout of a stage
-// from the stage's flag word in registers, builds descriptors by adding byte
-// offsets to per-stage base descriptors, and commits once per stage.
+// Issue.  On B200 each tcgen05.mma costs the issuing thread about 75 cycles
+// whatever N is (N = 16 here), a metadata copy about 180 and a commit about
+// 140, while instructions from two threads overlap.  So two issuer warps
+// share the work: ring positions alternate between them, each with its own
+// accumulator per chunk (a chunk's two stages always land on different
+// issuers), and the epilogue adds the two.  An issuer derives the k-step
+// layout of a stage from the stage's word in registers, builds descriptors by
+// adding offsets to per-stage bases, and commits once per stage.
 //
 // Launch.  A programmatic dependent of the previous kernel: once the packer's
 // ready flag is seen, the first stages' weight copies are issued before
 // `griddepcontrol.wait`; X, Y, the partials and the chunk counter are touched
 // only after it.  The fix-up kernel resets the counter for the next call.
 //
-// Roles (192 threads): warp 0 lane 0 producer, warp 1 lane 0 MMA issuer,
-// warps 2..5 epilogue (tcgen05.ld of the 16-column accumulator, fp32 partial
-// stores).  Two accumulators alternate between consecutive chunks.  Every
-// mbarrier wait is bounded by %globaltimer.
+// Roles (224 threads): warp 0 lane 0 producer, lane 0 of warps 1 and 6 MMA
+// issuers (even and odd ring positions), warps 2..5 epilogue (tcgen05.ld of
+// the 16-column accumulators, fp32 partial stores).  Two accumulator sets
+// alternate between consecutive chunks.  Every mbarrier wait is bounded by
+// %globaltimer.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -54,7 +57,7 @@ namespace patchk {
 
 namespace {
 
-constexpr int kDecThreads = 192;
+constexpr int kDecThreads = 224;
 constexpr int kDecBN = 16;                                // token rows of the MMA (N = 16)
 constexpr int kDecStages = 3;
 constexpr int kDecChunkPairs = 4;                         // k-pairs per chunk, at most
@@ -62,8 +65,8 @@ constexpr int kDecWBytes = 4 * kDenseStepBytes;           // two packed k-pairs,
 constexpr int kDecXStepBytes = kDecBN * kStep * 2;        // one k-step of X: 16 rows x 64
 constexpr int kDecXBytes = 4 * kDecXStepBytes;            // the stage's four X tiles
 constexpr int kDecStageBytes = kDecWBytes + kDecXBytes;   // 73728
-constexpr int kDecTmemCols = 64;                          // 2 x 16 accumulator + 2 x 4 metadata
-constexpr uint32_t kDecEcol = 2 * kDecBN;
+constexpr int kDecTmemCols = 128;  // 2 chunks x 2 issuers x 16 accumulator | 2 issuers x 2 x 4 metadata
+constexpr uint32_t kDecEcol = 4 * kDecBN;
 constexpr int kDecSmemBytes = kDecStages * kDecStageBytes + 1024 + 512;
 constexpr uint64_t kDecWaitLimitNs = 2000000000ull;       // 2 s per wait
 
@@ -72,14 +75,18 @@ constexpr uint64_t kDescOffsetMask = (1ull << 40) - 1;
 constexpr int kDescFlagsShift = 40;
 constexpr int kDescPairsShift = 56;
 
-// stage word: chunk (29 bits) | first stage of its chunk | last stage |
-// no more work | pairs in the stage (1 or 2) << 32 | k-step 2:4 flags << 36
+// stage word: chunk (29 bits) | no more work (bit 31) | pairs in the stage (1
+// or 2) << 32 | the chunk has two stages (bit 34) | k-step 2:4 flags << 36 |
+// ordinal of the chunk in this CTA (16 bits; for the done word: chunks in
+// all) << 40 | ring position (low 8 bits) << 56
 constexpr uint64_t kStageChunk = (1ull << 29) - 1;
-constexpr uint64_t kStageFirst = 1ull << 29;
-constexpr uint64_t kStageLast = 1ull << 30;
 constexpr uint64_t kStageDone = 1ull << 31;
 constexpr int kStagePairsShift = 32;
+constexpr uint64_t kStageTwo = 1ull << 34;
 constexpr int kStageFlagsShift = 36;
+constexpr int kStageOrdShift = 40;
+constexpr int kStagePosShift = 56;
+constexpr int kDecMaxChunksPerCta = 65535;
 
 struct DecodeParams {
     const uint8_t *packed;
@@ -108,6 +115,21 @@ __device__ __forceinline__ uint32_t pair_bytes(uint32_t flags, int i) {
                                  : kMetaBlockBytes + kDenseStepBytes + kSparseStepBytes;
 }
 
+// Wait until a shared counter reaches `target` (a counter has no phase
+// aliasing; the issuers may trail or lead one another by a chunk).
+__device__ __forceinline__ bool wait_count_bounded(volatile uint32_t *ctr, uint32_t target,
+                                                   volatile uint32_t *abort_flag, uint64_t limit_ns) {
+    if (*ctr >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (*ctr >= target) return true;
+        if ((i & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > limit_ns) return false;
+        }
+    }
+}
+
 __device__ __forceinline__ void store_out(const DecodeParams &p, int64_t idx, float v) {
     if (p.y_fp32)
         static_cast<float *>(p.Y)[idx] = v;
@@ -122,12 +144,13 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kDecStages * kDecStageBytes);
     uint64_t *empty = full + kDecStages;
-    uint64_t *acc_full = empty + kDecStages;  // [2] MMA commit + the MMA thread's arrive
-    uint64_t *acc_empty = acc_full + 2;       // [2] one arrive per epilogue warp
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *acc_full = empty + kDecStages;  // [2] four arrivals from the issuers per chunk
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 2);
     volatile uint32_t *abort_flag = tmem_slot + 1;  // raised by any role that gives up
     volatile uint32_t *never_flag = tmem_slot + 2;  // stays 0: time-only bounded waits
     volatile int32_t *acc_chunk = reinterpret_cast<volatile int32_t *>(tmem_slot + 4);  // [2]
+    volatile uint32_t *acc_mask = tmem_slot + 6;  // [2] issuers holding a part of the chunk
+    volatile uint32_t *drained = tmem_slot + 3;   // epilogue warps done with a chunk, in all
     uint64_t *stage_word = reinterpret_cast<uint64_t *>(tmem_slot + 8);                 // [STAGES]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -143,11 +166,9 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&acc_full[b], 2);
-            mbar_init(&acc_empty[b], 4);
-        }
+        for (int b = 0; b < 2; ++b) mbar_init(&acc_full[b], 4);
         *never_flag = 0u;
+        *drained = 0u;
         *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
         fence_mbar_init();
     }
@@ -166,6 +187,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         if (lane == 0 && !skip) {
             // ------------------------------------------------------ producer
             int it = 0;  // stages armed so far (ring position)
+            uint64_t cord = 0;  // chunks armed so far
             bool ok = true;
             int pend_s[kDecStages], pend_k[kDecStages];  // X loads of stages armed before the wait
             int npend = 0;
@@ -209,10 +231,11 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     const int sp = min(2, np - i);
                     const uint32_t bytes = pair_bytes(flags, i) + (sp == 2 ? pair_bytes(flags, i + 1) : 0u);
                     const uint32_t sflags = (flags >> (2 * i)) & (sp == 2 ? 0xFu : 0x3u);
-                    stage_word[s] = static_cast<uint64_t>(j) | (i == 0 ? kStageFirst : 0ull) |
-                                    (i + sp >= np ? kStageLast : 0ull) |
+                    stage_word[s] = static_cast<uint64_t>(j) | (np > 2 ? kStageTwo : 0ull) |
                                     (static_cast<uint64_t>(sp) << kStagePairsShift) |
-                                    (static_cast<uint64_t>(sflags) << kStageFlagsShift);
+                                    (static_cast<uint64_t>(sflags) << kStageFlagsShift) |
+                                    (cord << kStageOrdShift) |
+                                    (static_cast<uint64_t>(it & 0xFF) << kStagePosShift);
                     ++it;
                     const uint64_t src = cur;
                     cur += bytes;
@@ -229,6 +252,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     }
                 }
                 if (!ok) break;
+                ++cord;
                 if (!waited) flush_x();
                 if (!claimed) {
                     claim(ja, da);
@@ -242,15 +266,17 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                 if (j < p.nchunks) claim(jb, db);
             }
             if (!waited) flush_x();
-            if (ok) {
-                // no more chunks: a stage carrying the done flag (plain arrive)
+            // no more chunks: a stage carrying the done flag (plain arrive)
+            // for each issuer, with the chunk count
+            for (int q = 0; q < 2 && ok; ++q) {
                 const int s = it % kDecStages;
                 const uint32_t ph = (it / kDecStages) & 1u;
                 if (it >= kDecStages &&
                     !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kDecWaitLimitNs)) {
                     ok = false;
                 } else {
-                    stage_word[s] = kStageDone;
+                    stage_word[s] = kStageDone | (cord << kStageOrdShift) |
+                                    (static_cast<uint64_t>(it & 0xFF) << kStagePosShift);
                     mbar_arrive(&full[s]);
                     ++it;
                 }
@@ -267,9 +293,10 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                                   kDecWaitLimitNs / 4);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 6) {
         if (lane == 0 && !skip) {
             // ---------------------------------------------------------- MMA
+            const int q = warp == 6 ? 1 : 0;  // ring positions q, q + 2, ...
             // Descriptors: a template per layout plus the operand's shared
             // address in 16-byte units (all addresses here are below 256 KB,
             // so the 14-bit address field never carries into other fields).
@@ -279,35 +306,58 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             const uint64_t t_sw128 = smem_desc(0, 16, 1024, kSwizzle128B);  // dense A, X
             const uint64_t t_sw64 = smem_desc(0, 16, 512, kSwizzle64B);     // 2:4 A
             const uint64_t t_meta = smem_desc(0, 16, 128, kSwizzleNone);    // metadata
-            const uint32_t e_tmem = tmem_base + kDecEcol;
+            const uint32_t e_tmem = tmem_base + kDecEcol + 8 * q;
             const uint32_t smem0 = smem_u32(smem);
-            int it = 0, ci = 0;  // stages consumed, chunks finished
+            int it = q;       // ring position
+            int nch = 0;      // chunks of this CTA (from the done word)
             bool ok = true;
-            for (;;) {
+            for (;; it += 2) {
                 const int s = it % kDecStages;
                 const uint32_t ph = (it / kDecStages) & 1u;
-                if (!mbar_wait_bounded(&full[s], ph, abort_flag, kDecWaitLimitNs)) {
+                // The slot's previous phase belongs to the other issuer and may
+                // still be in flight, when a parity wait for ours passes at once:
+                // so the stage is ours only once the wait passes AND the word
+                // carries our position (the producer writes it only after the
+                // previous phase was consumed, and the next phase needs our
+                // commit, so the two together are exact).
+                uint64_t w = 0;
+                {
+                    const uint64_t t0 = globaltimer_ns();
+                    for (uint32_t n = 0;; ++n) {
+                        if (mbar_try_wait(&full[s], ph)) {
+                            w = *reinterpret_cast<volatile uint64_t *>(&stage_word[s]);
+                            if (((w >> kStagePosShift) & 0xFFu) == static_cast<uint64_t>(it & 0xFF)) break;
+                        }
+                        if ((n & 63u) == 63u &&
+                            (*abort_flag || globaltimer_ns() - t0 > kDecWaitLimitNs)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!ok) break;
+                }
+                tc_fence_after();
+                const int c = static_cast<int>((w >> kStageOrdShift) & 0xFFFFu);
+                if (w & kStageDone) {
+                    nch = c;
+                    break;
+                }
+                // this issuer holds at most one stage of chunk c: its accumulator
+                // is free once the epilogue has drained chunks up to c - 2
+                const int buf = c & 1;
+                if (c >= 2 && !wait_count_bounded(drained, 4u * static_cast<uint32_t>(c - 1), abort_flag,
+                                                  kDecWaitLimitNs)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t w = stage_word[s];
-                if (w & kStageDone) break;
-                const int buf = ci & 1;
-                if ((w & kStageFirst) && ci >= 2 &&
-                    !mbar_wait_bounded(&acc_empty[buf], ((ci >> 1) & 1u) ^ 1u, abort_flag,
-                                       kDecWaitLimitNs)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + buf * kDecBN;
+                const uint32_t d_tmem = tmem_base + (2 * buf + q) * kDecBN;
                 const uint32_t st16 = (smem0 + s * kDecStageBytes) >> 4;  // stage, 16-byte units
                 const uint64_t x16 = t_sw128 + st16 + (kDecWBytes >> 4);
                 const int sp = static_cast<int>((w >> kStagePairsShift) & 3u);
                 const uint32_t fl = static_cast<uint32_t>(w >> kStageFlagsShift) & 0xFu;
                 uint32_t off16 = 0;  // running offset in the stage, 16-byte units
-                uint32_t acc = (w & kStageFirst) ? 0u : 1u;
+                uint32_t acc = 0u;  // the stage starts this issuer's part of the chunk
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
                     if (t >= sp) break;
@@ -338,27 +388,31 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     }
                 }
                 tc_commit(&empty[s]);
-                if (w & kStageLast) {
-                    acc_chunk[buf] = static_cast<int32_t>(w & kStageChunk);
-                    tc_commit(&acc_full[buf]);
-                    mbar_arrive(&acc_full[buf]);  // publishes acc_chunk
-                    ++ci;
-                }
-                ++it;
+                // acc_full[buf] takes four arrivals per chunk: a commit and an
+                // arrive from each of two issuers, or a commit and three from one
+                const bool two = (w & kStageTwo) != 0;
+                acc_chunk[buf] = static_cast<int32_t>(w & kStageChunk);
+                acc_mask[buf] = two ? 3u : (1u << q);
+                tc_commit(&acc_full[buf]);
+                mbar_arrive_cnt(&acc_full[buf], two ? 1u : 3u);  // publishes acc_chunk, acc_mask
             }
             if (!ok) {
                 *abort_flag = 1u;
                 atomicOr(p.status, kStatusTimeout);
             }
-            // End of work for the epilogue: a phase whose chunk is -1.  Its
-            // commit fires once every MMA issued has completed, so TMEM is
-            // never freed under a running MMA.
-            const int buf = ci & 1;
-            if (ci >= 2)
-                mbar_wait_bounded(&acc_empty[buf], ((ci >> 1) & 1u) ^ 1u, never_flag, kDecWaitLimitNs);
-            acc_chunk[buf] = -1;
-            tc_commit(&acc_full[buf]);
-            mbar_arrive(&acc_full[buf]);
+            // End of work for the epilogue: a phase whose chunk is -1, one
+            // commit and one arrive from each issuer.  The commits fire once
+            // every MMA issued has completed, so TMEM is never freed under a
+            // running MMA.  (After a timeout the chunk count is unknown and the
+            // epilogue gives up on its own bounded wait.)
+            if (ok) {
+                const int buf = nch & 1;
+                if (nch >= 2)
+                    wait_count_bounded(drained, 4u * static_cast<uint32_t>(nch - 1), never_flag, kDecWaitLimitNs);
+                acc_chunk[buf] = -1;
+                tc_commit(&acc_full[buf]);
+                mbar_arrive(&acc_full[buf]);
+            }
         }
     } else if (!skip) {
         // ------------------------------------------------------- epilogue
@@ -377,19 +431,27 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             }
             const int j = acc_chunk[buf];
             if (j < 0) break;
-            uint32_t r[16];
-            tmem_ld_32x32b_x16(lane_base + buf * kDecBN, r);
+            const uint32_t mask = acc_mask[buf];  // the same for every lane
+            uint32_t r0[16], r1[16];
+            if (mask & 1u) tmem_ld_32x32b_x16(lane_base + (2 * buf) * kDecBN, r0);
+            if (mask & 2u) tmem_ld_32x32b_x16(lane_base + (2 * buf + 1) * kDecBN, r1);
             tmem_ld_wait();
             if (*abort_flag == 0) {
                 float *part = p.partial + static_cast<int64_t>(j) * kDecBN * kBand + row;
 #pragma unroll
-                for (int q = 0; q < 16; ++q)
-                    if (q < p.M) part[q * kBand] = __uint_as_float(r[q]);
+                for (int q = 0; q < 16; ++q) {
+                    const float v = (mask == 3u) ? __fadd_rn(__uint_as_float(r0[q]), __uint_as_float(r1[q]))
+                                                 : __uint_as_float(mask & 1u ? r0[q] : r1[q]);
+                    if (q < p.M) part[q * kBand] = v;
+                }
             }
             // the accumulator may be reused as soon as every lane has read it
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            if (lane == 0) {
+                __threadfence_block();
+                atomicAdd(const_cast<uint32_t *>(drained), 1u);
+            }
         }
     }
     tc_fence_before();
@@ -494,6 +556,10 @@ cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     if (!g.chunk_desc || !g.chunk_desc_host || !g.workspace || !g.counter) return cudaErrorInvalidValue;
     if (g.dec_cp < 1 || g.dec_cp > kDecChunkPairs) return cudaErrorInvalidValue;
+    const int grid_ctas = std::min(std::min(g.num_sms, g.dec_nchunks), kDecMaxCtas);
+    // a CTA's chunk ordinals travel in 16 bits (dynamic claiming could in
+    // principle hand one CTA every chunk)
+    if (g.dec_nchunks > kDecMaxChunksPerCta) return cudaErrorInvalidValue;
     if (decode_workspace_bytes(g.dec_nchunks) > g.workspace_bytes) return cudaErrorInvalidValue;
 
     DecodeParams p;
@@ -512,7 +578,7 @@ cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
     p.status = g.status;
     p.ready = g.ready;
     p.stall_first_kstep = g.stall_first_kstep;
-    const int grid = std::min(std::min(g.num_sms, g.dec_nchunks), kDecMaxCtas);
+    const int grid = grid_ctas;
     for (int c = 0; c < kDecMaxCtas; ++c) p.first_desc[c] = c < grid ? g.chunk_desc_host[c] : 0ull;
 
     cudaLaunchConfig_t cfg = {};

@@ -52,7 +52,7 @@ def check_close(y, yref, fp32_mode):
     else:
         mag = np.maximum(np.abs(y), np.abs(yref))
         ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-30))) - 7)
-        bad = err > 1e-2 * rms + 0.5 * ulp
+        bad = ~(err <= 1e-2 * rms + 0.5 * ulp)  # NaN counts as bad
         assert not bad.any(), (int(bad.sum()), float(err.max()), rms, TOL_NOTE)
 
 

@@ -40,7 +40,7 @@ def rel_rms_check(y, yref_f64, fp32_mode):
     else:
         mag = np.maximum(np.abs(y), np.abs(yref_f64))
         ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-30))) - 7)
-        bad = err > 1e-2 * rms + 0.5 * ulp
+        bad = ~(err <= 1e-2 * rms + 0.5 * ulp)  # NaN counts as bad
         assert not bad.any(), (int(bad.sum()), float(err.max()), rms)
     return float(err.max()), rms
 
