@@ -6,9 +6,11 @@
 // the case where the weights are read once and the run is bound by HBM.
 //
 // Work.  Every 128-row band of W is cut into chunks of `cp` consecutive
-// k-pairs (128 input columns each).  CTA c first runs chunk c, then claims
-// further chunks from an atomic counter, so SMs that stream faster take more
-// chunks and no CTA's static share decides the end of the kernel.  Each
+// k-pairs (128 input columns each).  CTA c first runs chunks c and c + G (G
+// CTAs), then claims further chunks from an atomic counter, so SMs that
+// stream faster take more chunks and no CTA's static share decides the end
+// of the kernel.  A claim is made one chunk ahead, while the current chunk's
+// copies are in flight, so its round trip is off the copy path.  Each
 // chunk leaves its 16 x 128 fp32 partial in its own slot; a fix-up kernel adds
 // the chunks of a band in chunk order, so Y does not depend on which CTA ran
 // which chunk.  No CTA ever waits for another.
@@ -98,11 +100,12 @@ struct DecodeParams {
     void *Y;
     int y_fp32;
     float *partial;     // [nchunks][16][128]
-    uint32_t *counter;  // chunks claimed beyond the first gridDim.x; zero between calls
+    uint32_t *counter;  // chunks claimed beyond the first 2 * gridDim.x; zero between calls
     uint32_t *status;
     const uint32_t *ready;
     int stall_first_kstep;  // failure-detection test hook
-    uint64_t first_desc[kDecMaxCtas];  // chunk_desc[c] for c < gridDim.x
+    uint64_t first_desc[kDecMaxCtas];   // chunk_desc[c] for c < gridDim.x
+    uint64_t second_desc[kDecMaxCtas];  // chunk_desc[c + gridDim.x] where that exists
 };
 
 // Bytes of pair i of a chunk whose k-step flags are `flags`, and whether its
@@ -199,21 +202,16 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                                 &full[pend_s[q]]);
                 npend = 0;
             };
-            // the next two claimed chunks (claimed only past the wait)
-            int ja = 0, jb = 0;
-            uint64_t da = 0, db = 0;
-            auto claim = [&](int &jj, uint64_t &dd) {
-                jj = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(p.counter, 1u));
-                dd = (jj < p.nchunks) ? __ldcg(p.chunk_desc + jj) : 0ull;
-            };
-            bool claimed = false;
-            if (waited) {
-                claim(ja, da);
-                claim(jb, db);
-                claimed = true;
-            }
+            // chunks j (current) and jn (next) are known; the one after jn is
+            // claimed during chunk j, once the counter may be touched (the
+            // previous call's fix-up resets it)
+            const int G = static_cast<int>(gridDim.x);
             int j = blockIdx.x;
             uint64_t d = p.first_desc[blockIdx.x];
+            int jn = blockIdx.x + G;
+            uint64_t dn = (jn < p.nchunks) ? p.second_desc[blockIdx.x] : 0ull;
+            bool have_tk = false;
+            uint32_t tk = 0;
             while (ok && j < p.nchunks) {
                 const int pr0 = (j % p.cpb) * p.cp;
                 const int np = static_cast<int>((d >> kDescPairsShift) & 0xFu);
@@ -239,31 +237,41 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     ++it;
                     const uint64_t src = cur;
                     cur += bytes;
-                    if (p.stall_first_kstep && blockIdx.x == 0 && it == 1) continue;  // never lands
-                    uint8_t *st = smem + s * kDecStageBytes;
-                    mbar_arrive_expect_tx(&full[s], bytes + kDecXBytes);
-                    bulk_g2s(st, p.packed + src, bytes, &full[s]);
-                    if (waited) {
-                        tma_load_3d(st + kDecWBytes, &tmap_x, 0, 0, 2 * (pr0 + i), &full[s]);
-                    } else {
-                        pend_s[npend] = s;
-                        pend_k[npend] = 2 * (pr0 + i);
-                        ++npend;
+                    if (!(p.stall_first_kstep && blockIdx.x == 0 && it == 1)) {  // else never lands
+                        uint8_t *st = smem + s * kDecStageBytes;
+                        mbar_arrive_expect_tx(&full[s], bytes + kDecXBytes);
+                        bulk_g2s(st, p.packed + src, bytes, &full[s]);
+                        if (waited) {
+                            tma_load_3d(st + kDecWBytes, &tmap_x, 0, 0, 2 * (pr0 + i), &full[s]);
+                        } else {
+                            pend_s[npend] = s;
+                            pend_k[npend] = 2 * (pr0 + i);
+                            ++npend;
+                        }
+                    }
+                    // the result is first read at the end of the chunk
+                    if (waited && !have_tk && jn < p.nchunks) {
+                        tk = atomicAdd(p.counter, 1u);
+                        have_tk = true;
                     }
                 }
                 if (!ok) break;
                 ++cord;
-                if (!waited) flush_x();
-                if (!claimed) {
-                    claim(ja, da);
-                    claim(jb, db);
-                    claimed = true;
+                int jnn = p.nchunks;
+                uint64_t dnn = 0;
+                if (jn < p.nchunks) {
+                    if (!have_tk) {
+                        if (!waited) flush_x();
+                        tk = atomicAdd(p.counter, 1u);
+                    }
+                    have_tk = false;
+                    jnn = 2 * G + static_cast<int>(tk);
+                    if (jnn < p.nchunks) dnn = __ldcg(p.chunk_desc + jnn);
                 }
-                j = ja;
-                d = da;
-                ja = jb;
-                da = db;
-                if (j < p.nchunks) claim(jb, db);
+                j = jn;
+                d = dn;
+                jn = jnn;
+                dn = dnn;
             }
             if (!waited) flush_x();
             // no more chunks: a stage carrying the done flag (plain arrive)
@@ -579,7 +587,10 @@ cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
     p.ready = g.ready;
     p.stall_first_kstep = g.stall_first_kstep;
     const int grid = grid_ctas;
-    for (int c = 0; c < kDecMaxCtas; ++c) p.first_desc[c] = c < grid ? g.chunk_desc_host[c] : 0ull;
+    for (int c = 0; c < kDecMaxCtas; ++c) {
+        p.first_desc[c] = c < grid ? g.chunk_desc_host[c] : 0ull;
+        p.second_desc[c] = (c < grid && c + grid < g.dec_nchunks) ? g.chunk_desc_host[c + grid] : 0ull;
+    }
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
