@@ -118,14 +118,19 @@ __device__ __forceinline__ uint32_t pair_bytes(uint32_t flags, int i) {
                                  : kMetaBlockBytes + kDenseStepBytes + kSparseStepBytes;
 }
 
-// Wait until a shared counter reaches `target` (a counter has no phase
-// aliasing; the issuers may trail or lead one another by a chunk).
+// Wait until each of four shared counters (chunks drained by each epilogue
+// warp; the warps run independently, so a sum could hide a lagging one)
+// reaches `target`.  Counters have no phase aliasing; the issuers may trail
+// or lead one another by a chunk.
+__device__ __forceinline__ bool drained_all(volatile uint32_t *ctr, uint32_t target) {
+    return ctr[0] >= target && ctr[1] >= target && ctr[2] >= target && ctr[3] >= target;
+}
 __device__ __forceinline__ bool wait_count_bounded(volatile uint32_t *ctr, uint32_t target,
                                                    volatile uint32_t *abort_flag, uint64_t limit_ns) {
-    if (*ctr >= target) return true;
+    if (drained_all(ctr, target)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (*ctr >= target) return true;
+        if (drained_all(ctr, target)) return true;
         if ((i & 63u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > limit_ns) return false;
@@ -153,7 +158,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
     volatile uint32_t *never_flag = tmem_slot + 2;  // stays 0: time-only bounded waits
     volatile int32_t *acc_chunk = reinterpret_cast<volatile int32_t *>(tmem_slot + 4);  // [2]
     volatile uint32_t *acc_mask = tmem_slot + 6;  // [2] issuers holding a part of the chunk
-    volatile uint32_t *drained = tmem_slot + 3;   // epilogue warps done with a chunk, in all
+    volatile uint32_t *drained = tmem_slot + 16;  // [4] chunks drained by each epilogue quarter
     uint64_t *stage_word = reinterpret_cast<uint64_t *>(tmem_slot + 8);                 // [STAGES]
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -171,7 +176,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         }
         for (int b = 0; b < 2; ++b) mbar_init(&acc_full[b], 4);
         *never_flag = 0u;
-        *drained = 0u;
+        for (int w = 0; w < 4; ++w) drained[w] = 0u;
         *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
         fence_mbar_init();
     }
@@ -353,7 +358,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                 // this issuer holds at most one stage of chunk c: its accumulator
                 // is free once the epilogue has drained chunks up to c - 2
                 const int buf = c & 1;
-                if (c >= 2 && !wait_count_bounded(drained, 4u * static_cast<uint32_t>(c - 1), abort_flag,
+                if (c >= 2 && !wait_count_bounded(drained, static_cast<uint32_t>(c - 1), abort_flag,
                                                   kDecWaitLimitNs)) {
                     ok = false;
                     break;
@@ -416,7 +421,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             if (ok) {
                 const int buf = nch & 1;
                 if (nch >= 2)
-                    wait_count_bounded(drained, 4u * static_cast<uint32_t>(nch - 1), never_flag, kDecWaitLimitNs);
+                    wait_count_bounded(drained, static_cast<uint32_t>(nch - 1), never_flag, kDecWaitLimitNs);
                 acc_chunk[buf] = -1;
                 tc_commit(&acc_full[buf]);
                 mbar_arrive(&acc_full[buf]);
@@ -458,7 +463,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             __syncwarp();
             if (lane == 0) {
                 __threadfence_block();
-                atomicAdd(const_cast<uint32_t *>(drained), 1u);
+                drained[quad] = static_cast<uint32_t>(ci + 1);
             }
         }
     }
