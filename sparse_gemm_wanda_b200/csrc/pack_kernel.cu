@@ -127,6 +127,212 @@ pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
     }
 }
 
+// ------------------------------------------------------------------- plan
+// The layout of every band: per k-step its type (2:4 iff the one or two tiles
+// covering its 128 rows are 2:4) and byte offset, a 2 KB metadata block
+// before the first 2:4 k-step of each k-pair; bands follow one another.  A
+// k-pair's size depends only on its two k-step types (32, 26 or 18 KB), so
+// offsets are prefix sums.  One block of 32 warps: a warp takes a band at a
+// time, gathers its k-step types into bit words in shared memory (one ballot
+// per 32 k-steps), then sizes its k-pairs with a k-pair per lane; the block
+// scans the band sizes; the warps write the entries and the decode chunk
+// descriptors.  All index arithmetic is 32-bit with shifts (tile sides are
+// powers of two).
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanWarps = kPlanThreads / 32;
+constexpr int kPlanMaxWords = 14;  // 448 k-steps (K <= 28672) / 32
+
+// Bit c % 32 of word c / 32 of `bits`: k-step c of band b is 2:4.
+__device__ __forceinline__ void band_types(const uint32_t *__restrict__ map, int b, int nsteps,
+                                           int log_tn, int log_tk, int tiles_k, int lane,
+                                           uint32_t *bits) {
+    const int rows_tiles = kBand >> log_tn;  // 1 or 2
+    const int ti0 = (b * kBand) >> log_tn;
+    for (int c0 = 0; c0 < nsteps; c0 += 32) {
+        const int c = c0 + lane;
+        bool sp = false;
+        if (c < nsteps) {
+            const int tj = (c * kStep) >> log_tk;
+            int t = ti0 * tiles_k + tj;
+            sp = (__ldg(map + (t >> 5)) >> (t & 31)) & 1u;
+            if (rows_tiles == 2) {
+                t += tiles_k;
+                sp = sp && ((__ldg(map + (t >> 5)) >> (t & 31)) & 1u);
+            }
+        }
+        const uint32_t w = __ballot_sync(0xFFFFFFFFu, sp);
+        if (lane == 0) bits[c0 >> 5] = w;
+    }
+    __syncwarp();
+}
+
+__device__ __forceinline__ bool bit_of(const uint32_t *bits, int c) { return (bits[c >> 5] >> (c & 31)) & 1u; }
+
+__device__ __forceinline__ uint32_t kpair_bytes(bool s0, bool s1) {
+    return (s0 ? kMetaBlockBytes + kSparseStepBytes : kDenseStepBytes) +
+           (s1 ? (s0 ? 0 : kMetaBlockBytes) + kSparseStepBytes : kDenseStepBytes);
+}
+
+__global__ void __launch_bounds__(kPlanThreads, 1)
+plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int log_tn, int log_tk, int cp,
+                 int cpb, uint64_t *__restrict__ table, uint64_t *__restrict__ chunk_desc,
+                 int64_t *__restrict__ pair_prefix, uint64_t *__restrict__ band_start,
+                 PackPlan *__restrict__ plan) {
+    __shared__ unsigned long long warp_sum[kPlanWarps];
+    __shared__ uint32_t types[kPlanWarps][2][kPlanMaxWords];
+    __shared__ unsigned long long carry, n_sparse, n_meta;
+    __shared__ unsigned int duo_ok, max_pair;
+    const int tid = threadIdx.x, lane = tid % 32, wid = tid / 32;
+    const int Q = nsteps / 2, tiles_k = (nsteps * kStep) >> log_tk;
+    uint32_t *mine = types[wid][0], *next = types[wid][1];
+    if (tid == 0) {
+        carry = 0;
+        n_sparse = 0;
+        n_meta = 0;
+        duo_ok = (bands % 2 == 0) ? 1u : 0u;
+        max_pair = 0;
+    }
+    __syncthreads();
+    // pass 1: k-pair sizes and their prefix within each band
+    {
+        unsigned long long ns = 0, nm = 0;
+        unsigned int mp = 0;
+        bool agree = true;
+        for (int b = wid; b < bands; b += kPlanWarps) {
+            band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
+            if (b % 2 == 0 && b + 1 < bands) {
+                band_types(map, b + 1, nsteps, log_tn, log_tk, tiles_k, lane, next);
+                for (int w = lane; w < (nsteps + 31) / 32; w += 32)
+                    if (mine[w] != next[w]) agree = false;
+            }
+            int64_t *pre = pair_prefix + static_cast<int64_t>(b) * (Q + 1);
+            if (lane == 0) pre[0] = 0;
+            unsigned long long run = 0;
+            for (int q0 = 0; q0 < Q; q0 += 32) {
+                const int q = q0 + lane;
+                uint32_t bytes = 0;
+                if (q < Q) {
+                    const bool s0 = bit_of(mine, 2 * q), s1 = bit_of(mine, 2 * q + 1);
+                    bytes = kpair_bytes(s0, s1);
+                    ns += s0 + s1;
+                    nm += (s0 || s1) ? 1 : 0;
+                    mp = max(mp, bytes);
+                }
+                unsigned long long incl = bytes;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const unsigned long long v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                if (q < Q) pre[q + 1] = static_cast<int64_t>(run + incl);
+                run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+            }
+            __syncwarp();
+        }
+        atomicAdd(&n_sparse, ns);
+        atomicAdd(&n_meta, nm);
+        atomicMax(&max_pair, mp);
+        if (!agree) atomicAnd(&duo_ok, 0u);
+    }
+    __syncthreads();
+    // pass 2: the first byte of every band (block-wide exclusive scan)
+    for (int base = 0; base < bands; base += kPlanThreads) {
+        const int b = base + tid;
+        const unsigned long long bytes =
+            b < bands ? static_cast<unsigned long long>(pair_prefix[static_cast<int64_t>(b) * (Q + 1) + Q]) : 0ull;
+        unsigned long long incl = bytes;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) warp_sum[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            unsigned long long w = warp_sum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long v = __shfl_up_sync(0xFFFFFFFFu, w, o);
+                if (lane >= o) w += v;
+            }
+            warp_sum[lane] = w;  // inclusive over warps
+        }
+        __syncthreads();
+        if (b < bands) band_start[b] = carry + (wid > 0 ? warp_sum[wid - 1] : 0ull) + (incl - bytes);
+        __syncthreads();
+        if (tid == 0) carry += warp_sum[kPlanWarps - 1];
+        __syncthreads();
+    }
+    // pass 3: k-step entries and decode chunk descriptors
+    for (int b = wid; b < bands; b += kPlanWarps) {
+        band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
+        const uint64_t start = band_start[b];
+        const int64_t *pre = pair_prefix + static_cast<int64_t>(b) * (Q + 1);
+        uint64_t *row = table + static_cast<int64_t>(b) * nsteps;
+        for (int q = lane; q < Q; q += 32) {
+            const bool s0 = bit_of(mine, 2 * q), s1 = bit_of(mine, 2 * q + 1);
+            uint64_t off = start + static_cast<uint64_t>(pre[q]);
+            uint64_t e0, e1;
+            if (s0) {
+                off += kMetaBlockBytes;
+                e0 = kEntrySparse | kEntryMeta | off;
+                off += kSparseStepBytes;
+            } else {
+                e0 = off;
+                off += kDenseStepBytes;
+            }
+            if (s1) {
+                uint64_t m = 0;
+                if (!s0) {
+                    off += kMetaBlockBytes;
+                    m = kEntryMeta;
+                }
+                e1 = kEntrySparse | m | off;
+            } else {
+                e1 = off;
+            }
+            row[2 * q] = e0;
+            row[2 * q + 1] = e1;
+        }
+        for (int q = lane; q < cpb; q += 32) {
+            const int pr0 = q * cp;
+            const int np = min(cp, Q - pr0);
+            uint64_t flags = 0;
+            for (int i = 0; i < 2 * np; ++i)
+                if (bit_of(mine, 2 * pr0 + i)) flags |= 1ull << i;
+            const uint64_t first = start + static_cast<uint64_t>(pre[pr0]);
+            chunk_desc[static_cast<int64_t>(b) * cpb + q] =
+                (first & ((1ull << 40) - 1)) | (flags << 40) | (static_cast<uint64_t>(np) << 56);
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    // the first chunk descriptors, written above by other warps of the block
+    const int64_t nchunks = static_cast<int64_t>(bands) * cpb;
+    for (int64_t j = tid; j < 2 * kDecMaxCtas; j += kPlanThreads)
+        plan->first_desc[j] = j < nchunks ? chunk_desc[j] : 0ull;
+    if (tid == 0) {
+        plan->packed_bytes = carry;
+        plan->sparse_ksteps = n_sparse;
+        plan->meta_blocks = n_meta;
+        plan->duo_ok = duo_ok;
+        plan->max_pair_bytes = max_pair;
+    }
+}
+
+cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, int tk, int cp,
+                             int cpb, uint64_t *table, uint64_t *chunk_desc, int64_t *pair_prefix,
+                             uint64_t *band_start, PackPlan *plan, cudaStream_t stream) {
+    const int64_t nsteps = K / kStep;
+    if (nsteps > 32 * kPlanMaxWords || (N / kBand) > (int64_t(1) << 24)) return cudaErrorInvalidValue;
+    const int log_tn = tn == 64 ? 6 : 7, log_tk = tk == 64 ? 6 : 7;
+    plan_pack_kernel<<<1, kPlanThreads, 0, stream>>>(map, static_cast<int>(N / kBand), static_cast<int>(nsteps),
+                                                     log_tn, log_tk, cp, cpb, table, chunk_desc,
+                                                     pair_prefix, band_start, plan);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                         int64_t K, int tn, int tk, const uint64_t *table, uint8_t *out,
                         uint32_t *done, uint32_t *ready, cudaStream_t stream) {

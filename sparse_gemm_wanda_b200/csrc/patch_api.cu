@@ -20,9 +20,9 @@
 
 struct patch_packed {
     int device;
-    uint8_t *base;             // one pool allocation holding all device arrays below
+    uint8_t *base;             // pool allocation: table, descriptors, prefix, plan, workspace, status
     patch_shape shp;
-    uint8_t *packed;           // packed k-steps
+    uint8_t *packed;           // packed k-steps (a pool allocation of its own, exact size)
     size_t packed_bytes;
     uint64_t *table;           // (N/128) * (K/64) entries
     int64_t sparse_ksteps;
@@ -37,7 +37,10 @@ struct patch_packed {
     uint32_t *status;          // device: status word, pack counter, ready flag
     int num_sms;
     cudaMemPool_t pool;
-    std::vector<int64_t> pair_prefix;  // per band: cumulative packed bytes of its k-pairs
+    int64_t bands;
+    int64_t *pair_prefix_dev;  // device: per band, cumulative packed bytes of its k-pairs
+    // host copy of pair_prefix, fetched by the first call that can use it
+    mutable std::vector<int64_t> pair_prefix;
 };
 
 namespace {
@@ -87,42 +90,26 @@ patch_status check_device(int *num_sms) {
     return PATCH_OK;
 }
 
-// A reusable page-locked staging buffer per device for small host-to-device
-// uploads (the k-step table): the copy is asynchronous, and the next user
-// waits on the event recorded after it before overwriting the buffer.
-struct PinnedStage {
-    void *buf = nullptr;
-    size_t cap = 0;
-    cudaEvent_t done = nullptr;
-};
-
-cudaError_t upload_via_pinned(void *dst, const void *src, size_t bytes, cudaStream_t stream) {
+// The plan summary written by plan_pack_kernel, read back into page-locked
+// memory (one buffer per device, held under the lock until the copy landed).
+cudaError_t read_plan(const patchk::PackPlan *src, patchk::PackPlan *dst, cudaStream_t stream) {
     static std::mutex mu;
-    static std::map<int, PinnedStage> stages;
+    static std::map<int, patchk::PackPlan *> bufs;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
-    PinnedStage &st = stages[dev];
-    if (!st.done) {
-        e = cudaEventCreateWithFlags(&st.done, cudaEventDisableTiming);
-        if (e != cudaSuccess) return e;
-    } else {
-        e = cudaEventSynchronize(st.done);  // the previous upload has left the buffer
-        if (e != cudaSuccess) return e;
+    patchk::PackPlan *&buf = bufs[dev];
+    if (!buf) {
+        e = cudaMallocHost(reinterpret_cast<void **>(&buf), sizeof(patchk::PackPlan));
+        if (e != cudaSuccess) {
+            buf = nullptr;
+            return e;
+        }
     }
-    if (st.cap < bytes) {
-        if (st.buf) cudaFreeHost(st.buf);
-        st.buf = nullptr;
-        st.cap = 0;
-        const size_t cap = std::max<size_t>(bytes, 1 << 20);
-        e = cudaMallocHost(&st.buf, cap);
-        if (e != cudaSuccess) return e;
-        st.cap = cap;
-    }
-    memcpy(st.buf, src, bytes);
-    e = cudaMemcpyAsync(dst, st.buf, bytes, cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess) e = cudaEventRecord(st.done, stream);
+    e = cudaMemcpyAsync(buf, src, sizeof(patchk::PackPlan), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess) *dst = *buf;
     return e;
 }
 
@@ -391,120 +378,68 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
 
     const int64_t N = shp.N, K = shp.K, tn = shp.tile_n, tk = shp.tile_k;
-    const int64_t tiles_k = K / tk, n_tiles = (N / tn) * tiles_k;
-    const int64_t bands = N / kBand, nsteps = K / kStep;
-
-    // the map is read back once to plan the layout
-    std::vector<uint32_t> hmap(static_cast<size_t>((n_tiles + 31) / 32));
-    cudaError_t e = cudaMemcpyAsync(hmap.data(), map, sizeof(uint32_t) * hmap.size(),
-                                    cudaMemcpyDeviceToHost, stream);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-    if (e != cudaSuccess) return from_cuda(e);
-    auto tile_sparse = [&](int64_t t) { return ((hmap[t / 32] >> (t % 32)) & 1u) != 0; };
+    const int64_t bands = N / kBand, nsteps = K / kStep, Q = nsteps / 2;
 
     patch_packed *h = new (std::nothrow) patch_packed();
     if (!h) return PATCH_ERR_OOM;
-    // k-step (b, c) is 2:4 iff the one or two tiles covering its 128 rows (one
-    // tile column, since tk >= 64) are 2:4
-    const int64_t Q = nsteps / 2;
-    std::vector<uint64_t> table(static_cast<size_t>(bands * nsteps));
-    h->pair_prefix.assign(static_cast<size_t>(bands * (Q + 1)), 0);
-    const int64_t rows_tiles = kBand / tn;  // 1 or 2
-    uint64_t offset = 0;
-    int64_t n_sparse = 0, n_meta = 0;
-    for (int64_t b = 0; b < bands; ++b) {
-        const int64_t ti0 = (b * kBand) / tn;
-        const uint64_t band_start = offset;
-        bool prev_sparse = false;
-        for (int64_t c = 0; c < nsteps; ++c) {
-            const int64_t tj = (c * kStep) / tk;
-            bool sp = tile_sparse(ti0 * tiles_k + tj);
-            if (rows_tiles == 2) sp = sp && tile_sparse((ti0 + 1) * tiles_k + tj);
-            uint64_t entry;
-            if (sp) {
-                entry = patchk::kEntrySparse;
-                if (c % 2 == 0 || !prev_sparse) {  // first 2:4 k-step of its pair
-                    offset += patchk::kMetaBlockBytes;
-                    entry |= patchk::kEntryMeta;
-                    ++n_meta;
-                }
-                entry |= offset;
-                offset += patchk::kSparseStepBytes;
-                ++n_sparse;
-            } else {
-                entry = offset;
-                offset += patchk::kDenseStepBytes;
-            }
-            table[static_cast<size_t>(b * nsteps + c)] = entry;
-            prev_sparse = sp;
-            if (c % 2 == 1)  // cumulative bytes of the band's pairs, for stream-K balancing
-                h->pair_prefix[static_cast<size_t>(b * (Q + 1) + c / 2 + 1)] =
-                    static_cast<int64_t>(offset - band_start);
-        }
-    }
-
     cudaGetDevice(&h->device);
     h->shp = shp;
-    h->packed_bytes = static_cast<size_t>(offset);
-    if (offset >= (1ull << 40)) {  // chunk descriptors hold 40-bit offsets
-        delete h;
-        return PATCH_ERR_UNSUPPORTED;
-    }
-    h->sparse_ksteps = n_sparse;
-    h->meta_blocks = n_meta;
     h->num_sms = num_sms;
-    // decode GEMV chunks: descriptors from the table just planned
+    h->bands = bands;
     patchk::plan_decode_chunks(bands, nsteps, num_sms, &h->dec_cp, &h->dec_cpb, &h->dec_nchunks);
-    h->chunk_desc_host.resize(static_cast<size_t>(h->dec_nchunks));
-    for (int64_t b = 0; b < bands; ++b)
-        for (int c = 0; c < h->dec_cpb; ++c) {
-            const int pr0 = c * h->dec_cp;
-            const int np = static_cast<int>(std::min<int64_t>(h->dec_cp, Q - pr0));
-            h->chunk_desc_host[static_cast<size_t>(b * h->dec_cpb + c)] =
-                patchk::decode_chunk_desc(table.data() + b * nsteps, nsteps, pr0, np);
-        }
     h->workspace_bytes = patchk::decode_workspace_bytes(h->dec_nchunks);
-    h->max_pair_bytes = 0;
-    for (int64_t b = 0; b < bands; ++b)
-        for (int64_t q = 0; q < Q; ++q) {
-            const int64_t pb = h->pair_prefix[static_cast<size_t>(b * (Q + 1) + q + 1)] -
-                               h->pair_prefix[static_cast<size_t>(b * (Q + 1) + q)];
-            h->max_pair_bytes = std::max<int>(h->max_pair_bytes, static_cast<int>(pb));
-        }
-    // the two-SM prefill kernel pairs bands 2p and 2p+1 in one instruction
-    h->duo_ok = (bands % 2 == 0) ? 1 : 0;
-    for (int64_t b = 0; h->duo_ok && b < bands; b += 2)
-        for (int64_t c = 0; c < nsteps; ++c)
-            if ((table[static_cast<size_t>(b * nsteps + c)] & patchk::kEntrySparse) !=
-                (table[static_cast<size_t>((b + 1) * nsteps + c)] & patchk::kEntrySparse)) {
-                h->duo_ok = 0;
-                break;
-            }
 
-    // one pool allocation: packed bytes | table | chunk descriptors | workspace | status
-    const size_t off_table = round_up(std::max<size_t>(h->packed_bytes, 16), 256);
-    const size_t off_chunks = off_table + sizeof(uint64_t) * table.size();  // uploaded with the table
-    const size_t off_ws = round_up(off_chunks + sizeof(uint64_t) * h->chunk_desc_host.size(), 256);
+    // The layout is planned on the device from the map (no map read-back, no
+    // table upload); only the plan summary comes back, to size the packed
+    // buffer.  Allocation 1: table | chunk descriptors | k-pair prefix | band
+    // starts | plan | workspace | status.  Allocation 2: the packed bytes.
+    const size_t off_table = 0;
+    const size_t off_chunks = off_table + sizeof(uint64_t) * static_cast<size_t>(bands * nsteps);
+    const size_t off_prefix = round_up(off_chunks + sizeof(uint64_t) * static_cast<size_t>(h->dec_nchunks), 256);
+    const size_t off_bstart = round_up(off_prefix + sizeof(int64_t) * static_cast<size_t>(bands * (Q + 1)), 256);
+    const size_t off_plan = round_up(off_bstart + sizeof(uint64_t) * static_cast<size_t>(bands), 256);
+    const size_t off_ws = round_up(off_plan + sizeof(patchk::PackPlan), 256);
     const size_t off_status = round_up(off_ws + h->workspace_bytes, 256);
     const size_t status_bytes = 256;
     const size_t total = off_status + status_bytes;
-    cudaError_t e2 = patchk::device_pool(&h->pool);
-    if (e2 == cudaSuccess)
-        e2 = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->base), total, h->pool, stream);
-    if (e2 == cudaSuccess) {
-        h->packed = h->base;
-        h->table = reinterpret_cast<uint64_t *>(h->base + off_table);
-        h->chunk_desc = reinterpret_cast<uint64_t *>(h->base + off_chunks);
-        h->workspace = reinterpret_cast<float *>(h->base + off_ws);
-        // status word | pack completion counter | ready flag | decode chunk counter
-        h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
-        e2 = cudaMemsetAsync(h->status, 0, status_bytes, stream);
+    cudaError_t e = patchk::device_pool(&h->pool);
+    if (e == cudaSuccess)
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->base), total, h->pool, stream);
+    if (e != cudaSuccess) {
+        delete h;
+        return from_cuda(e);
     }
-    if (e2 == cudaSuccess) {
-        table.insert(table.end(), h->chunk_desc_host.begin(), h->chunk_desc_host.end());
-        e2 = upload_via_pinned(h->table, table.data(), sizeof(uint64_t) * table.size(), stream);
+    h->table = reinterpret_cast<uint64_t *>(h->base + off_table);
+    h->chunk_desc = reinterpret_cast<uint64_t *>(h->base + off_chunks);
+    h->pair_prefix_dev = reinterpret_cast<int64_t *>(h->base + off_prefix);
+    patchk::PackPlan *plan_dev = reinterpret_cast<patchk::PackPlan *>(h->base + off_plan);
+    h->workspace = reinterpret_cast<float *>(h->base + off_ws);
+    // status word | pack completion counter | ready flag | decode chunk counter
+    h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
+    e = cudaMemsetAsync(h->status, 0, status_bytes, stream);
+    if (e == cudaSuccess)
+        e = patchk::launch_plan_pack(map, N, K, static_cast<int>(tn), static_cast<int>(tk), h->dec_cp,
+                                     h->dec_cpb, h->table, h->chunk_desc, h->pair_prefix_dev,
+                                     reinterpret_cast<uint64_t *>(h->base + off_bstart), plan_dev, stream);
+    patchk::PackPlan plan;
+    if (e == cudaSuccess) e = read_plan(plan_dev, &plan, stream);
+    if (e != cudaSuccess) {
+        patch_free(h, stream_v);
+        return from_cuda(e);
     }
-    e = e2;
+    h->packed_bytes = static_cast<size_t>(plan.packed_bytes);
+    if (plan.packed_bytes >= (1ull << 40)) {  // chunk descriptors hold 40-bit offsets
+        patch_free(h, stream_v);
+        return PATCH_ERR_UNSUPPORTED;
+    }
+    h->sparse_ksteps = static_cast<int64_t>(plan.sparse_ksteps);
+    h->meta_blocks = static_cast<int64_t>(plan.meta_blocks);
+    h->duo_ok = plan.duo_ok ? 1 : 0;
+    h->max_pair_bytes = static_cast<int>(plan.max_pair_bytes);
+    h->chunk_desc_host.assign(plan.first_desc,
+                              plan.first_desc + std::min<int64_t>(h->dec_nchunks, 2 * patchk::kDecMaxCtas));
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->packed),
+                                std::max<size_t>(h->packed_bytes, 16), h->pool, stream);
     if (e == cudaSuccess)
         e = patchk::launch_pack(W_bf16, meta, map, N, K, static_cast<int>(tn), static_cast<int>(tk),
                                 h->table, h->packed, h->status + 1, h->status + 2, stream);
@@ -549,7 +484,20 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.duo_ok = Wp->duo_ok;
     g.max_pair_bytes = Wp->max_pair_bytes;
     g.num_sms = Wp->num_sms;
-    g.pair_prefix = Wp->pair_prefix.data();
+    // the stream-K balance of the prefill kernels uses the k-pair prefix: fetched
+    // once per handle, by the first call that can need it
+    if (M > 16 && Wp->pair_prefix.empty()) {
+        const size_t n = static_cast<size_t>(Wp->bands * (Wp->shp.K / kStep / 2 + 1));
+        Wp->pair_prefix.resize(n);
+        cudaError_t e = cudaMemcpyAsync(Wp->pair_prefix.data(), Wp->pair_prefix_dev, sizeof(int64_t) * n,
+                                        cudaMemcpyDeviceToHost, static_cast<cudaStream_t>(stream_v));
+        if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream_v));
+        if (e != cudaSuccess) {
+            Wp->pair_prefix.clear();
+            return from_cuda(e);
+        }
+    }
+    g.pair_prefix = Wp->pair_prefix.empty() ? nullptr : Wp->pair_prefix.data();
     // Failure-detection test hook: with PATCH_B200_TEST_STALL=1 in the
     // environment, CTA 0 never loads its first k-step, so its bounded wait runs
     // out, the kernel returns early and patch_get_status reports the timeout.
@@ -560,6 +508,7 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
 
 void patch_free(patch_packed *Wp, void *stream_v) {
     if (!Wp) return;
+    if (Wp->packed) cudaFreeAsync(Wp->packed, static_cast<cudaStream_t>(stream_v));
     if (Wp->base) cudaFreeAsync(Wp->base, static_cast<cudaStream_t>(stream_v));
     delete Wp;
 }

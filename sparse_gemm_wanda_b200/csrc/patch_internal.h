@@ -41,6 +41,23 @@ cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map
 // parameters, at most.
 constexpr int kDecMaxCtas = 160;
 
+// Layout plan of a packed matrix, computed on the device from the tile map
+// (plan_pack_kernel) and read back once by patch_pack.
+struct PackPlan {
+    uint64_t packed_bytes;
+    uint64_t sparse_ksteps;
+    uint64_t meta_blocks;
+    uint32_t duo_ok;          // bands 2p, 2p+1 agree in type at every k-step
+    uint32_t max_pair_bytes;  // largest packed k-pair
+    uint64_t first_desc[2 * kDecMaxCtas];  // decode chunk descriptors 0 .. 2*kDecMaxCtas-1
+};
+// Writes the k-step table [bands][nsteps], the decode chunk descriptors
+// [bands][cpb], the per-band cumulative k-pair bytes [bands][nsteps/2 + 1],
+// the first byte of each band (scratch [bands]) and the plan summary; one block.
+cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, int tk, int cp,
+                             int cpb, uint64_t *table, uint64_t *chunk_desc, int64_t *pair_prefix,
+                             uint64_t *band_start, PackPlan *plan, cudaStream_t stream);
+
 struct GemmLaunch {
     const uint8_t *packed;
     const uint64_t *table;
