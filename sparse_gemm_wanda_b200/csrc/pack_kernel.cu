@@ -229,10 +229,21 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
             }
             __syncwarp();
         }
-        atomicAdd(&n_sparse, ns);
-        atomicAdd(&n_meta, nm);
-        atomicMax(&max_pair, mp);
-        if (!agree) atomicAnd(&duo_ok, 0u);
+        // one shared-memory atomic per warp (1024 contending 64-bit atomics on
+        // one address serialise for tens of microseconds)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ns += __shfl_xor_sync(0xFFFFFFFFu, ns, o);
+            nm += __shfl_xor_sync(0xFFFFFFFFu, nm, o);
+            mp = max(mp, __shfl_xor_sync(0xFFFFFFFFu, mp, o));
+        }
+        const bool all_agree = __all_sync(0xFFFFFFFFu, agree);
+        if (lane == 0) {
+            atomicAdd(&n_sparse, ns);
+            atomicAdd(&n_meta, nm);
+            atomicMax(&max_pair, mp);
+            if (!all_agree) atomicAnd(&duo_ok, 0u);
+        }
     }
     __syncthreads();
     // pass 2: the first byte of every band (block-wide exclusive scan)
