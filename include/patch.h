@@ -209,8 +209,10 @@ patch_status patch_select_maps_global(const double *const *losses, const int64_t
  *   - table[b*(K/64)+c] (uint64): bits 0..47 byte offset of the k-step's
  *     data, bit 62 = 2:4, bit 63 = the pair's metadata block precedes it.
  *
- * Synchronises the stream once: the map is read back to plan the layout and
- * size the allocation exactly.
+ * Synchronises the stream once: the layout is planned on the device from the
+ * map (k-step table and decode chunk descriptors written there), and only a
+ * small summary (total bytes, the first chunk descriptors) is read back to
+ * size the packed allocation exactly.
  * Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA.
  */
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
@@ -222,8 +224,9 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
  * memory and one rounding at the end (PATCH page, section 2, inference and
  * deployment: one kernel over mixed dense / 2:4 tiles).  Dense k-steps issue
  * the dense tcgen05 MMA, 2:4 k-steps the sparse tcgen05 MMA, into one
- * accumulator.  M <= 16 (and M <= the handle's max_decode_m) runs the split-K
- * decode configuration; larger M the prefill configuration.
+ * accumulator.  M <= 16 runs the split-K decode configuration; larger M the
+ * prefill configuration (whose first call on a handle reads the per-band
+ * k-pair sizes back once, for stream-K balance).
  *
  *   Wp      handle from patch_pack.
  *   X_bf16  [M,K] bf16, 16-byte aligned.
