@@ -93,6 +93,32 @@ def test_pack_argument_checks(lib):
     assert out.value is None
 
 
+def test_select_maps_global_argument_checks(lib):
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: checks fail first
+    vp3 = (ctypes.c_void_p * 3)(fake, fake, fake)
+    nt3 = (ctypes.c_int64 * 3)(10, 1, 40)
+    # null arrays
+    assert lib.patch_select_maps_global(None, nt3, 3, 0.5, vp3, None) == 1
+    assert lib.patch_select_maps_global(vp3, None, 3, 0.5, vp3, None) == 1
+    assert lib.patch_select_maps_global(vp3, nt3, 3, 0.5, None, None) == 1
+    # count outside 1..64
+    assert lib.patch_select_maps_global(vp3, nt3, 0, 0.5, vp3, None) == 1
+    many = (ctypes.c_void_p * 65)(*([fake] * 65))
+    nt65 = (ctypes.c_int64 * 65)(*([4] * 65))
+    assert lib.patch_select_maps_global(many, nt65, 65, 0.5, many, None) == 1
+    # fraction outside [0, 1], NaN included
+    assert lib.patch_select_maps_global(vp3, nt3, 3, -0.25, vp3, None) == 1
+    assert lib.patch_select_maps_global(vp3, nt3, 3, float("nan"), vp3, None) == 1
+    # a null loss array or a zero tile count among the matrices
+    vp_null = (ctypes.c_void_p * 3)(fake, None, fake)
+    assert lib.patch_select_maps_global(vp_null, nt3, 3, 0.5, vp3, None) == 1
+    nt_zero = (ctypes.c_int64 * 3)(10, 0, 40)
+    assert lib.patch_select_maps_global(vp3, nt_zero, 3, 0.5, vp3, None) == 1
+    # more tiles than one ranking pass covers
+    big = (ctypes.c_int64 * 3)(65535 * 256, 1, 1)
+    assert lib.patch_select_maps_global(vp3, big, 3, 0.5, vp3, None) == 2
+
+
 def test_handle_calls_reject_null(lib):
     assert lib.patch_get_status(None) == 1
     assert lib.patch_packed_info(None, None) == 1
