@@ -29,6 +29,9 @@
  *     caller or taken as the tiles whose 2:4 pruning loses the least Wanda
  *     score (a data-free stand-in for the learned map; PATCH-Tile, section 2
  *     variants, freezes 2:4 patterns from a one-shot method).
+ *   - a block-wide tile budget (one target over several matrices, left free
+ *     to land unevenly): PATCH page, section 4, ablation on a global target
+ *     against a per-layer one; here the least-loss tiles over all matrices.
  *   - compressed storage is required for any speedup: SparseGPT-vs-Wanda
  *     page, section on structured vs unstructured sparsity.  The packed
  *     layout itself is this library's own format (documented in
