@@ -607,7 +607,9 @@ def main():
 
     # --------------------------------------------- isolated GEMM measurements
     extras = {}
-    if not args.no_extras and rank == 0:
+    # one GPU only: under torchrun the other ranks would wait for rank 0 at the
+    # closing barrier for as long as these take
+    if not args.no_extras and rank == 0 and world == 1:
         W0 = mats[-1]["W"]  # the MLP-shaped matrix
         dec = {}
         graph_roof = None
