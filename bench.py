@@ -221,7 +221,7 @@ def run_step(P, wl, mats, calib, timer: CallTimer, keep=None):
 
 
 def algorithmic_bytes(name, wl, mats, packed_bytes):
-    """Bytes each call must move at minimum (roofline section)."""
+    """Bytes each call must move at minimum: W and the codes it reads, what it writes."""
     total = 0.0
     count = 0
     seen_k = set()
