@@ -663,7 +663,9 @@ def main():
             del Wp, Xp
         extras["prefill_gemm_isolated"] = {
             "by_shape": pre_all, "dense_peak_tflops": dense_peak, "peak_source": peak_kind,
-            "note": "effective = 2MNK / t (dense-equivalent); sparse peak = 2 x measured dense peak; "
+            "note": "effective = 2MNK / t (dense-equivalent); sparse peak = 2 x measured dense peak "
+                    "(the sparse MMA itself ran at about 1.6 x the dense rate at N = 256 in a "
+                    "one-SM instruction probe, so about 0.8 of this peak is the ceiling); "
                     "seeded random maps; L2 flushed before every call"}
 
     cpu = None
