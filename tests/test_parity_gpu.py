@@ -247,6 +247,14 @@ def test_gemm_tiles_and_fractions(P, oracle_mod, tn, tk, frac, M):
     run_case(P, oracle_mod, 256, 512, M, tn, tk, frac, seed=tn + tk + M, fp32_mode=True)
 
 
+@pytest.mark.parametrize("N,K", [(128, 128), (128, 384), (256, 640), (384, 896), (128, 1152)])
+@pytest.mark.parametrize("M", [1, 5, 16])
+def test_gemm_decode_ragged_pair_counts(P, oracle_mod, N, K, M):
+    # k-pairs per band of 1, 3, 5, 7, 9: chunks of fewer than four pairs,
+    # stages holding a single k-pair, single-band matrices, fewer chunks than SMs
+    run_case(P, oracle_mod, N, K, M, 128, 128, 0.5, seed=N + K + M, fp32_mode=True)
+
+
 def test_gemm_tiny_config(P, oracle_mod):
     # W 256x256, 64x64 tiles, 8 of 16 tiles 2:4, Xcal 64x256, X 8x256, 3 outlier channels
     wl = inputs.workloads()["tiny"]
