@@ -119,8 +119,8 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
  * values (chunk partials of the column sums, norms, and the loss / rank
  * counters when the caller does not ask for them) live in one fixed array of
  * device memory inside this library, 16 MiB per device
- * (patch_score_mask_noalloc_capacity()), held by every device that loads the
- * library until the process exits.  A call needs
+ * (patch_score_mask_noalloc_capacity()), held on each device from the first
+ * call there (see Set-up) until the process exits.  A call needs
  * 8*K*ceil(T/128) + 8*K + 8*n_tiles + 4*n_tiles bytes of it (plus alignment;
  * the last two terms only when tile_loss_out is NULL / map_in is NULL);
  * larger problems return PATCH_ERR_UNSUPPORTED without launching anything.
@@ -130,9 +130,15 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
  * in it; each call writes every value before reading it.  Calls whose GPU
  * work overlaps (different streams without ordering between them) race on the
  * array and give wrong results: order them on one stream or with events.
- * The first call on each device looks up the array's device address (with
- * that device current) and caches it; make that first call before any stream
- * capture begins.
+ *
+ * Set-up.  The array's device address belongs to a CUDA context; the first
+ * call in each context looks it up (cudaGetSymbolAddress, with the device
+ * current) and caches it under the context's id, so a device reset or a new
+ * primary context is looked up afresh.  Under lazy module loading (the CUDA
+ * default) that first lookup is also what loads this library's module on
+ * the device, i.e. when the 16 MiB are reserved: a caller whose allocator
+ * takes the GPU's memory up front should make one call (any small problem)
+ * at initialisation, before that reservation and before any stream capture.
  */
 patch_status patch_score_mask_noalloc(const void *W_bf16, const void *Xcal_bf16, int64_t T,
                                       const double *colsq_in, patch_shape shp,
@@ -142,6 +148,15 @@ patch_status patch_score_mask_noalloc(const void *W_bf16, const void *Xcal_bf16,
 
 /* Bytes of the fixed scratch array patch_score_mask_noalloc works in. */
 size_t patch_score_mask_noalloc_capacity(void);
+
+/*
+ * Diagnostics: bytes of the library's stream-ordered device pool (current
+ * device) in use now, and the high-water mark of that use.  reset_high != 0
+ * first restarts the mark from the current use, so a later reading above
+ * `used_now` shows that something took pool memory in between.  Host
+ * pointers, either may be NULL.  No device work.  Errors: CUDA.
+ */
+patch_status patch_pool_usage(uint64_t *used_now, uint64_t *used_high, int32_t reset_high);
 
 /*
  * Global tile allocation over several matrices of one block (the ablation in
@@ -211,8 +226,9 @@ patch_status patch_select_maps_global(const double *const *losses, const int64_t
  *
  * Synchronises the stream once: the layout is planned on the device from the
  * map (k-step table and decode chunk descriptors written there), and only a
- * small summary (total bytes, the first chunk descriptors) is read back to
- * size the packed allocation exactly.
+ * small summary (total bytes, the first chunk descriptors) and the per-band
+ * k-pair byte prefix (the prefill kernels' work balance) are read back, in
+ * that one wait, to size the packed allocation exactly.
  * Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA.
  */
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
@@ -225,8 +241,8 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
  * deployment: one kernel over mixed dense / 2:4 tiles).  Dense k-steps issue
  * the dense tcgen05 MMA, 2:4 k-steps the sparse tcgen05 MMA, into one
  * accumulator.  M <= 16 runs the split-K decode configuration; larger M the
- * prefill configuration (whose first call on a handle reads the per-band
- * k-pair sizes back once, for stream-K balance).
+ * prefill configuration.  The call only enqueues work: it never waits for the
+ * device (everything it needs from the device was read back by patch_pack).
  *
  *   Wp      handle from patch_pack.
  *   X_bf16  [M,K] bf16, 16-byte aligned.
@@ -240,12 +256,18 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
  * while the word is set, later calls on the handle skip their work.
  * Errors: INVALID_ARG, CUDA; PATCH_ERR_TIMEOUT is reported by
  * patch_get_status, not here (the call does not synchronise).
- * Test hook: with the environment variable PATCH_B200_TEST_STALL=1 the first
- * CTA never loads its first k-step, which makes that wait run out on purpose
- * (the failure-detection test); leave it unset in normal use.
  */
 patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
                                int32_t y_is_fp32, void *stream);
+
+/*
+ * Failure-detection test hook: while `on` is non-zero, the first CTA of every
+ * later patch_hybrid_gemm never loads its first k-step, so that CTA's bounded
+ * wait runs out on purpose and patch_get_status reports PATCH_ERR_TIMEOUT.
+ * Off by default (the environment variable PATCH_B200_TEST_STALL=1, read once
+ * when the library loads, turns it on from the start).  Tests only.
+ */
+void patch_test_stall_first_kstep(int32_t on);
 
 /* Release a handle's device memory (stream-ordered on `stream`).  NULL ok. */
 void patch_free(patch_packed *Wp, void *stream);

@@ -108,7 +108,9 @@ def select_2of4(score: np.ndarray) -> np.ndarray:
 
 
 def tile_loss(score: np.ndarray, meta: np.ndarray, tn: int, tk: int) -> np.ndarray:
-    """Pruned Wanda score per tile (rows left-to-right, then rows top-to-bottom)."""
+    """Pruned Wanda score per tile: inside each 32-column word of a row left to
+    right, the row's words left to right, then the tile's row sums as a balanced
+    pairwise tree ((0,1), (2,3), ..., then pairs of those)."""
     score = np.ascontiguousarray(score, dtype=np.float64)
     meta = np.ascontiguousarray(meta, dtype=np.uint32)
     N, K = score.shape

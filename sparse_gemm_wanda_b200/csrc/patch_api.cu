@@ -39,8 +39,8 @@ struct patch_packed {
     cudaMemPool_t pool;
     int64_t bands;
     int64_t *pair_prefix_dev;  // device: per band, cumulative packed bytes of its k-pairs
-    // host copy of pair_prefix, fetched by the first call that can use it
-    mutable std::vector<int64_t> pair_prefix;
+    // host copy of pair_prefix, read back by patch_pack
+    std::vector<int64_t> pair_prefix;
 };
 
 namespace {
@@ -91,8 +91,12 @@ patch_status check_device(int *num_sms) {
 }
 
 // The plan summary written by plan_pack_kernel, read back into page-locked
-// memory (one buffer per device, held under the lock until the copy landed).
-cudaError_t read_plan(const patchk::PackPlan *src, patchk::PackPlan *dst, cudaStream_t stream) {
+// memory (one buffer per device, held under the lock until the copy landed),
+// and the per-band k-pair prefix the prefill kernels balance their work with
+// (into `prefix`, pageable: that copy returns once it has landed).  The
+// stream is waited for once, here; no later call on the handle waits.
+cudaError_t read_plan(const patchk::PackPlan *src, patchk::PackPlan *dst, const int64_t *prefix_src,
+                      std::vector<int64_t> *prefix, cudaStream_t stream) {
     static std::mutex mu;
     static std::map<int, patchk::PackPlan *> bufs;
     int dev = 0;
@@ -108,10 +112,21 @@ cudaError_t read_plan(const patchk::PackPlan *src, patchk::PackPlan *dst, cudaSt
         }
     }
     e = cudaMemcpyAsync(buf, src, sizeof(patchk::PackPlan), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess && !prefix->empty())
+        e = cudaMemcpyAsync(prefix->data(), prefix_src, sizeof(int64_t) * prefix->size(),
+                            cudaMemcpyDeviceToHost, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
     if (e == cudaSuccess) *dst = *buf;
     return e;
 }
+
+// Failure-detection test hook (see patch_test_stall_first_kstep): read from
+// the environment once, when the library is loaded; changed only by the
+// exported setter.
+std::atomic<int> g_test_stall{[] {
+    const char *v = getenv("PATCH_B200_TEST_STALL");
+    return (v && v[0] == '1') ? 1 : 0;
+}()};
 
 patch_status from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return PATCH_OK;
@@ -242,22 +257,54 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
 constexpr size_t kNoallocScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
 
+// Driver entry points for the current context and its process-unique id,
+// fetched through the runtime (the library links no driver stub).
+using CtxGetCurrentFn = int (*)(void **);
+using CtxGetIdFn = int (*)(void *, unsigned long long *);
+
+static bool current_context_id(unsigned long long *id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    void *ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != 0 || !ctx) return false;
+    return get_id(ctx, id) == 0;
+}
+
+// Device address of the scratch array in the current context.  The address
+// belongs to a context (a device reset or a new primary context maps the
+// module again, elsewhere), so it is cached per context id, never per device
+// ordinal.  A miss, or a context the driver cannot name, looks it up with
+// cudaGetSymbolAddress; under lazy module loading that first lookup loads
+// this library's module on the device, which is when the array is reserved.
 static cudaError_t noalloc_scratch_address(uint8_t **ptr) {
     static std::mutex mu;
-    static std::map<int, uint8_t *> addr;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
+    static std::map<unsigned long long, uint8_t *> addr;
     std::lock_guard<std::mutex> lock(mu);
-    auto it = addr.find(dev);
-    if (it != addr.end()) {
-        *ptr = it->second;
-        return cudaSuccess;
+    unsigned long long id = 0;
+    const bool named = current_context_id(&id);
+    if (named) {
+        auto it = addr.find(id);
+        if (it != addr.end()) {
+            *ptr = it->second;
+            return cudaSuccess;
+        }
     }
     void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // with `dev` current
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // with the device current
     if (e != cudaSuccess) return e;
-    addr[dev] = static_cast<uint8_t *>(p);
+    // the lookup made the runtime's context current if none was: cache under it
+    if (current_context_id(&id)) addr[id] = static_cast<uint8_t *>(p);
     *ptr = static_cast<uint8_t *>(p);
     return cudaSuccess;
 }
@@ -319,6 +366,24 @@ patch_status patch_score_mask_noalloc(const void *W_bf16, const void *Xcal_bf16,
 
 size_t patch_score_mask_noalloc_capacity(void) { return kNoallocScratchBytes; }
 
+patch_status patch_pool_usage(uint64_t *used_now, uint64_t *used_high, int32_t reset_high) {
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = patchk::device_pool(&pool);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (reset_high) {
+        uint64_t zero = 0;
+        e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &zero);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
+    uint64_t now = 0, high = 0;
+    e = cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemCurrent, &now);
+    if (e == cudaSuccess) e = cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &high);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (used_now) *used_now = now;
+    if (used_high) *used_high = high;
+    return PATCH_OK;
+}
+
 patch_status patch_select_maps_global(const double *const *losses, const int64_t *n_tiles,
                                       int32_t count, double fraction, uint32_t *const *maps_out,
                                       void *stream_v) {
@@ -361,6 +426,8 @@ patch_status patch_select_maps_global(const double *const *losses, const int64_t
 }
 
 uint64_t patch_launch_count(void) { return patchk::g_launches.load(std::memory_order_relaxed); }
+
+void patch_test_stall_first_kstep(int32_t on) { g_test_stall.store(on ? 1 : 0, std::memory_order_relaxed); }
 
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
                         patch_shape shp, patch_packed **out,
@@ -422,7 +489,8 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
                                      h->dec_cpb, h->table, h->chunk_desc, h->pair_prefix_dev,
                                      reinterpret_cast<uint64_t *>(h->base + off_bstart), plan_dev, stream);
     patchk::PackPlan plan;
-    if (e == cudaSuccess) e = read_plan(plan_dev, &plan, stream);
+    h->pair_prefix.assign(static_cast<size_t>(bands * (Q + 1)), 0);
+    if (e == cudaSuccess) e = read_plan(plan_dev, &plan, h->pair_prefix_dev, &h->pair_prefix, stream);
     if (e != cudaSuccess) {
         patch_free(h, stream_v);
         return from_cuda(e);
@@ -484,25 +552,10 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.duo_ok = Wp->duo_ok;
     g.max_pair_bytes = Wp->max_pair_bytes;
     g.num_sms = Wp->num_sms;
-    // the stream-K balance of the prefill kernels uses the k-pair prefix: fetched
-    // once per handle, by the first call that can need it
-    if (M > 16 && Wp->pair_prefix.empty()) {
-        const size_t n = static_cast<size_t>(Wp->bands * (Wp->shp.K / kStep / 2 + 1));
-        Wp->pair_prefix.resize(n);
-        cudaError_t e = cudaMemcpyAsync(Wp->pair_prefix.data(), Wp->pair_prefix_dev, sizeof(int64_t) * n,
-                                        cudaMemcpyDeviceToHost, static_cast<cudaStream_t>(stream_v));
-        if (e == cudaSuccess) e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream_v));
-        if (e != cudaSuccess) {
-            Wp->pair_prefix.clear();
-            return from_cuda(e);
-        }
-    }
+    // the stream-K balance of the prefill kernels uses the k-pair prefix,
+    // read back once by patch_pack: nothing here waits for the device
     g.pair_prefix = Wp->pair_prefix.empty() ? nullptr : Wp->pair_prefix.data();
-    // Failure-detection test hook: with PATCH_B200_TEST_STALL=1 in the
-    // environment, CTA 0 never loads its first k-step, so its bounded wait runs
-    // out, the kernel returns early and patch_get_status reports the timeout.
-    const char *stall = getenv("PATCH_B200_TEST_STALL");
-    g.stall_first_kstep = (stall && stall[0] == '1') ? 1 : 0;
+    g.stall_first_kstep = g_test_stall.load(std::memory_order_relaxed);
     return from_cuda(patchk::launch_hybrid_gemm(g, static_cast<cudaStream_t>(stream_v)));
 }
 

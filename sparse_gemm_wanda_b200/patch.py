@@ -24,7 +24,7 @@ EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
            "patch_get_status", "patch_packed_info", "patch_packed_export",
            "patch_status_string", "patch_score_mask_noalloc",
            "patch_score_mask_noalloc_capacity", "patch_launch_count",
-           "patch_select_maps_global")
+           "patch_select_maps_global", "patch_test_stall_first_kstep", "patch_pool_usage")
 
 
 class PatchLibraryError(RuntimeError):
@@ -76,6 +76,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.patch_select_maps_global.restype = ctypes.c_int
     lib.patch_launch_count.argtypes = []
     lib.patch_launch_count.restype = ctypes.c_uint64
+    lib.patch_test_stall_first_kstep.argtypes = [i32]
+    lib.patch_test_stall_first_kstep.restype = None
+    lib.patch_pool_usage.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
+                                     i32]
+    lib.patch_pool_usage.restype = ctypes.c_int
     lib.patch_pack.argtypes = [vp, vp, vp, PatchShape, ctypes.POINTER(vp),
                                ctypes.POINTER(ctypes.c_size_t), vp]
     lib.patch_hybrid_gemm.argtypes = [vp, vp, i64, vp, i32, vp]
@@ -96,6 +101,21 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 def launch_count() -> int:
     """Kernels the library has enqueued so far in this process."""
     return int(load_library().patch_launch_count())
+
+
+def test_stall_first_kstep(on: bool) -> None:
+    """Failure-detection hook: while on, the first CTA of every GEMM never
+    receives its first k-step, so its bounded wait runs out (tests only)."""
+    load_library().patch_test_stall_first_kstep(1 if on else 0)
+
+
+def pool_usage(reset_high: bool = False) -> tuple:
+    """(bytes in use, high-water mark) of the library's device memory pool on
+    the current device; reset_high restarts the mark from the current use."""
+    now, high = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    _check("patch_pool_usage", load_library().patch_pool_usage(
+        ctypes.byref(now), ctypes.byref(high), 1 if reset_high else 0))
+    return int(now.value), int(high.value)
 
 
 def _check(fn: str, code: int):

@@ -1,7 +1,15 @@
-"""Full-size parity for the 13B-shaped prefill and the whole 7B-shaped block.
+"""Full-size parity for the 7B prefill sweep, the 13B-shaped prefill and the
+whole 7B-shaped block.
 
-Both run at the sizes the benchmark uses, through the C ABI, against the
-oracle on the same seeded inputs:
+All run at the workloads' own sizes, through the C ABI, against the oracle on
+the same seeded inputs; every expected value comes from the oracle alone (the
+GPU's codes and maps are asserted equal to the oracle's, never reused):
+
+* 7B prefill sweep: W 11008x4096 and 4096x11008, 128x128 tiles, M = 2048,
+  seeded random maps with 0, 25, 50, 75 and 100 % of the tiles 2:4; 2:4
+  patterns from Wanda with the input X itself as calibration set.  Codes, map,
+  losses, packed bytes and k-step table bit-exact; GEMM on two whole 128-row
+  bands x all 2048 tokens (bf16 and fp32 output) and on sampled outputs.
 
 * 13B prefill: W 13824x5120 and 5120x13824, 128x128 tiles, every tile 2:4
   (50 % sparsity) and a seeded random map with 75 % of the tiles 2:4 (37.5 %);
@@ -69,6 +77,24 @@ def sampled_check(y, x_bits, weff, n_samples, seed, fp32_mode):
     check_close(ys, yref, fp32_mode)
 
 
+def band_check(y, x_bits, weff, bands, fp32_mode):
+    """Whole 128-row output bands, every token: y[:, 128b:128b+128] against the
+    oracle's full sums for those rows."""
+    for b in bands:
+        rows = slice(128 * b, 128 * b + 128)
+        yref = oracle.gemm(x_bits, np.ascontiguousarray(weff[rows]))
+        check_close(y[:, rows], yref, fp32_mode)
+
+
+def mixed_band(tmap_bits, n_bands, tiles_k):
+    """The first band whose tiles hold both kinds (else band 0)."""
+    for b in range(n_bands):
+        kinds = {(int(tmap_bits[t // 32]) >> (t % 32)) & 1 for t in range(b * tiles_k, (b + 1) * tiles_k)}
+        if len(kinds) == 2:
+            return b
+    return 0
+
+
 def check_pack(pk, w_bits, meta, tmap, tn, tk):
     packed, table = pk.export()
     torch.cuda.synchronize()
@@ -76,6 +102,46 @@ def check_pack(pk, w_bits, meta, tmap, tn, tk):
     assert pk.packed_bytes == ref_packed.size
     assert np.array_equal(table.cpu().numpy().view(np.uint64), ref_table)
     assert np.array_equal(packed.cpu().numpy(), ref_packed)
+
+
+# --------------------------------------------------------- 7B prefill sweep
+
+@pytest.mark.parametrize("N,K", [(11008, 4096), (4096, 11008)])
+@pytest.mark.parametrize("frac", [0.0, 0.25, 0.5, 0.75, 1.0])
+def test_7b_prefill_sweep_config(P, N, K, frac):
+    wl = inputs.workloads()["llama7b-prefill"]
+    seed = wl.seed + N + int(frac * 100)
+    M = 2048
+    w = inputs.weight(N, K, seed)
+    o = inputs.outlier_channels(K, wl.seed)
+    x = inputs.activations(M, K, wl.seed, o, role=1)
+    nt = (N // 128) * (K // 128)
+    tmap = inputs.random_map(nt, inputs.n_sparse_tiles(frac, nt), seed)
+    wd, xd = w.cuda(), x.cuda()
+    # the workload's 2:4 patterns: Wanda with its own input X as calibration
+    r = P.patch_score_mask(wd, xd, map_in=tmap.cuda(), want_colsq=True, want_loss=True)
+    pk = P.patch_pack(wd, r["meta"], r["map"])
+    y = P.patch_hybrid_gemm(pk, xd)
+    y32 = P.patch_hybrid_gemm(pk, xd, out_fp32=True)
+    torch.cuda.synchronize()
+    assert P.patch_get_status(pk) == 0
+
+    wb, xb = bf16_bits(w), bf16_bits(x)
+    tm = tmap.numpy().view(np.uint32)
+    ref = oracle.score_mask(wb, xb, 128, 128, tile_map=tm)
+    assert np.array_equal(r["colsq"].cpu().numpy(), ref["colsq"])
+    assert np.array_equal(u32(r["meta"]), ref["meta"])
+    assert np.array_equal(r["loss"].cpu().numpy(), ref["loss"])
+    assert np.array_equal(u32(r["map"]), ref["map"])
+    check_pack(pk, wb, ref["meta"], tm, 128, 128)
+    weff = oracle.weff(wb, ref["meta"], tm, 128, 128)
+    zero = float(np.mean(weff == 0))
+    assert abs(zero - frac / 2) < 2e-3, zero
+    bands = sorted({mixed_band(tm, N // 128, K // 128), N // 128 - 1})
+    band_check(y, xb, weff, bands, fp32_mode=False)
+    band_check(y32, xb, weff, bands, fp32_mode=True)
+    sampled_check(y, xb, weff, 6000, seed, fp32_mode=False)
+    pk.close()
 
 
 # ------------------------------------------------------------- 13B prefill
@@ -110,6 +176,7 @@ def test_13b_prefill_config(P, N, K, frac):
     weff = oracle.weff(wb, ref["meta"], tm, 128, 128)
     zero = float(np.mean(weff == 0))
     assert abs(zero - frac / 2) < 2e-3, zero
+    band_check(y, xb, weff, [mixed_band(tm, N // 128, K // 128)], fp32_mode=False)
     sampled_check(y, xb, weff, 6000, seed, fp32_mode=False)
     pk.close()
 
@@ -187,6 +254,7 @@ def test_block_config(P, block):
                 torch.cuda.synchronize()
                 check_close(y32, oracle.gemm(xb, weff), fp32_mode=True)
             else:
+                band_check(y, xb, weff, [mixed_band(tmap, m.N // 128, m.K // 128)], fp32_mode=False)
                 sampled_check(y, xb, weff, 3000, seed=M + mi, fp32_mode=False)
         assert P.patch_get_status(pk) == 0
         pk.close()

@@ -59,6 +59,18 @@ def oracle_mask(oracle_mod, w, xc, tn, tk, frac=None, tmap=None):
                                  tile_map=tmap)
 
 
+def oracle_weff_checked(oracle_mod, r, w, xc, tn, tk, tmap=None, frac=None):
+    """W_eff from the oracle alone: its 2:4 codes and tile map for (w, xc),
+    after asserting that the GPU's codes and map (in `r`) equal them.  With
+    `tmap` (a caller map) the map is given; otherwise it is the oracle's
+    least-loss map at `frac`."""
+    tm = None if tmap is None else tmap.numpy().view(np.uint32)
+    ref = oracle_mask(oracle_mod, w, xc, tn, tk, frac=frac, tmap=tm)
+    assert np.array_equal(u32(r["meta"]), ref["meta"]), "2:4 codes differ from the oracle's"
+    assert np.array_equal(u32(r["map"]), ref["map"]), "tile map differs from the oracle's"
+    return oracle_mod.weff(bf16_bits(w), ref["meta"], ref["map"], tn, tk)
+
+
 # ---------------------------------------------------------------- mask builder
 
 @pytest.mark.parametrize("N,K,T,tn,tk,frac", [
@@ -217,8 +229,7 @@ def run_case(P, oracle_mod, N, K, M, tn, tk, frac, seed, fp32_mode, sample=None)
     y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=fp32_mode)
     torch.cuda.synchronize()
     assert P.patch_get_status(pk) == 0
-    meta = u32(r["meta"])
-    weff = oracle_mod.weff(bf16_bits(w), meta, tmap.numpy().view(np.uint32), tn, tk)
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, tn, tk, tmap=tmap)
     if sample is None:
         yref = oracle_mod.gemm(bf16_bits(x), weff)
         out = rel_rms_check(y, yref, fp32_mode)
@@ -324,7 +335,8 @@ def test_gemm_decode_config_full(P, oracle_mod, N, M):
     y16 = P.patch_hybrid_gemm(pk, x.cuda())
     y32 = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
     torch.cuda.synchronize()
-    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), u32(r["map"]), 128, 128)
+    # codes AND least-loss map from the oracle (the GPU's asserted equal)
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, frac=0.5)
     yref = oracle_mod.gemm(bf16_bits(x), weff)
     rel_rms_check(y32, yref, True)
     rel_rms_check(y16, yref, False)
@@ -339,6 +351,42 @@ def test_gemm_prefill_config_sampled(P, oracle_mod, N, K, frac):
              fp32_mode=False, sample=4000)
 
 
+@pytest.mark.parametrize("M", [8, 300, 2048])
+def test_gemm_first_call_does_not_block_the_host(P, oracle_mod, M):
+    # The first GEMM on a fresh handle (decode and prefill token counts) must
+    # only enqueue: queued behind a ~1 s spin kernel, the call returns while
+    # the stream is still busy.  The result is then checked as usual.
+    import time
+    N, K = 1024, 1024
+    w, xc, x = make_problem(N, K, 64, M, seed=61 + M)
+    nt = (N // 128) * (K // 128)
+    tmap = inputs.random_map(nt, nt // 2, seed=61)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    xd = x.cuda()
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    torch.cuda._sleep(2_000_000_000)  # about a second of GPU cycles
+    t0 = time.perf_counter()
+    P.patch_hybrid_gemm(pk, xd, out=y, out_fp32=True)
+    dt = time.perf_counter() - t0
+    busy = not stream.query()
+    torch.cuda.synchronize()
+    assert busy, "the stream finished before the call returned: the call waited for it"
+    assert dt < 0.25, dt
+    assert P.patch_get_status(pk) == 0
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap)
+    if M <= 300:
+        rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), weff), True)
+    else:
+        g = np.random.default_rng(M)
+        ms, ns = g.integers(0, M, 3000), g.integers(0, N, 3000)
+        yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
+        rel_rms_check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, True)
+    pk.close()
+
+
 def test_gemm_repeated_calls_reset_tickets(P, oracle_mod):
     # stream-K tiles shared by several CTAs: every call must find its tickets at zero
     N, K, M = 1024, 2048, 5
@@ -347,7 +395,7 @@ def test_gemm_repeated_calls_reset_tickets(P, oracle_mod):
     tmap = inputs.random_map(nt, nt // 2, seed=31)
     r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
     pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
-    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap)
     for rep in range(3):
         x = inputs.activations(M, K, 100 + rep, None)
         y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
@@ -357,7 +405,7 @@ def test_gemm_repeated_calls_reset_tickets(P, oracle_mod):
     pk.close()
 
 
-def test_gemm_bounded_wait_reports_timeout(P, oracle_mod, monkeypatch):
+def test_gemm_bounded_wait_reports_timeout(P, oracle_mod):
     # Failure detection without a GPU fault: the first CTA never receives its
     # first k-step; its bounded wait runs out, the kernel returns, the status
     # word reports the timeout, and the handle works again once cleared.
@@ -366,14 +414,16 @@ def test_gemm_bounded_wait_reports_timeout(P, oracle_mod, monkeypatch):
     tmap = inputs.random_map(4, 2, seed=41)
     r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
     pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
-    monkeypatch.setenv("PATCH_B200_TEST_STALL", "1")
-    P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
-    monkeypatch.delenv("PATCH_B200_TEST_STALL")
+    P.test_stall_first_kstep(True)
+    try:
+        P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    finally:
+        P.test_stall_first_kstep(False)
     assert P.patch_get_status(pk) == 5  # PATCH_ERR_TIMEOUT, read and cleared
     assert P.patch_get_status(pk) == 0
     y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
     torch.cuda.synchronize()
-    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap)
     rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), weff), True)
     pk.close()
 
@@ -393,8 +443,7 @@ def test_gemm_chain_overlapped_matches_serialised(P, oracle_mod):
         tmap = inputs.random_map(nt, nt // 2, seed=700 + i)
         r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
         pks.append(P.patch_pack(w.cuda(), r["meta"], r["map"]))
-        weffs.append(oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32),
-                                     128, 128))
+        weffs.append(oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap))
     for M in (3, 16, 200):
         x0 = inputs.activations(M, shapes[0][1], 800 + M, None)
         xs = x0.cuda()
@@ -428,7 +477,7 @@ def test_gemm_band_pair_kernel(P, oracle_mod, N, K, M, tn, tk, frac, fp32_mode):
              sample=6000)
 
 
-def test_gemm_band_pair_kernel_bounded_wait(P, oracle_mod, monkeypatch):
+def test_gemm_band_pair_kernel_bounded_wait(P, oracle_mod):
     # the failure-detection hook on the band-pair kernel: CTA 0's first stage
     # never lands, its waits run out, the status reports the timeout and the
     # handle computes correctly once the status is read
@@ -438,14 +487,16 @@ def test_gemm_band_pair_kernel_bounded_wait(P, oracle_mod, monkeypatch):
     tmap = inputs.random_map(nt, nt // 2, seed=43)
     r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
     pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
-    monkeypatch.setenv("PATCH_B200_TEST_STALL", "1")
-    P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
-    monkeypatch.delenv("PATCH_B200_TEST_STALL")
+    P.test_stall_first_kstep(True)
+    try:
+        P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    finally:
+        P.test_stall_first_kstep(False)
     assert P.patch_get_status(pk) == 5
     assert P.patch_get_status(pk) == 0
     y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
     torch.cuda.synchronize()
-    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap)
     g = np.random.default_rng(43)
     ms, ns = g.integers(0, M, 3000), g.integers(0, N, 3000)
     yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
@@ -493,7 +544,7 @@ def test_gemm_two_sm_kernel_band_aligned_mixed_map(P, oracle_mod, fp32_mode):
     y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=fp32_mode)
     torch.cuda.synchronize()
     assert P.patch_get_status(pk) == 0
-    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap)
     g = np.random.default_rng(91)
     ms, ns = g.integers(0, M, 6000), g.integers(0, N, 6000)
     yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
@@ -501,7 +552,7 @@ def test_gemm_two_sm_kernel_band_aligned_mixed_map(P, oracle_mod, fp32_mode):
     pk.close()
 
 
-def test_gemm_two_sm_kernel_bounded_wait(P, oracle_mod, monkeypatch):
+def test_gemm_two_sm_kernel_bounded_wait(P, oracle_mod):
     # the failure-detection hook on the two-SM kernel: the first CTA never
     # arms its first stage; both CTAs of its pair give up within their bounds,
     # meet at the final cluster barrier, and the handle works afterwards
@@ -511,14 +562,16 @@ def test_gemm_two_sm_kernel_bounded_wait(P, oracle_mod, monkeypatch):
     tmap = inputs.random_map(nt, nt, seed=47)
     r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
     pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
-    monkeypatch.setenv("PATCH_B200_TEST_STALL", "1")
-    P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
-    monkeypatch.delenv("PATCH_B200_TEST_STALL")
+    P.test_stall_first_kstep(True)
+    try:
+        P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    finally:
+        P.test_stall_first_kstep(False)
     assert P.patch_get_status(pk) == 5
     assert P.patch_get_status(pk) == 0
     y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
     torch.cuda.synchronize()
-    weff = oracle_mod.weff(bf16_bits(w), u32(r["meta"]), tmap.numpy().view(np.uint32), 128, 128)
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap)
     g = np.random.default_rng(47)
     ms, ns = g.integers(0, M, 3000), g.integers(0, N, 3000)
     yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
