@@ -1,22 +1,28 @@
 """Benchmark of the tile-hybrid (dense / 2:4) Wanda-masked linear layer on B200.
 
 One step = one pass of the whole hot path over one batch of synthetic input,
-for every weight matrix of the workload:
-  column norms of the calibration set -> Wanda scores / 2:4 codes / tile loss
-  -> tile map (least-loss tiles become 2:4) -> pack -> hybrid GEMM for every
-  token count of the workload.
-Default workload: Llama-7B-shaped decode (W 4096x4096 and 11008x4096, 128x128
-tiles, half the tiles 2:4 chosen by least Wanda tile loss, calibration
-2048x4096 with 1% outlier channels x20, M in {1, 4, 16}).
+for every weight matrix of the workload, in four phases:
+  1. column sums of squares of each distinct calibration set (patch_colsq);
+  2. Wanda scores / 2:4 codes / tile loss / tile map per matrix
+     (patch_score_mask, reusing the column sums of the matrix's input);
+  3. pack per matrix (patch_pack);
+  4. hybrid GEMM for every matrix and every token count, largest M first
+     (patch_hybrid_gemm).
+Default workload: the full Llama-7B-shaped decoder block (q, k, v, o
+4096x4096; gate, up 11008x4096; down 4096x11008), 128x128 tiles, Wanda masks
+from 128 x 2048 = 262144 calibration tokens per distinct layer input, the 60 %
+of tiles with the least pruned-score loss 2:4 (30 % target sparsity), GEMMs at
+M in {4096, 512, 64, 8, 1}.
 
-Metric: dense-equivalent GEMM TFLOP/s = sum over the step's GEMMs of 2*M*N*K,
-divided by the step's device time (mask build and pack included).  Also
-reported: tokens/s, per-call times, the roofline of the kernel with the
-largest share of device time (the decode GEMM: its calls timed back to back in
-a CUDA graph over weight copies larger than L2, as a decode loop runs them),
-isolated decode-GEMM and prefill-GEMM measurements (speedup over the same
-kernel with an all-dense map), end-to-end time with host buffers, and the CPU
-oracle timed on the host cores.
+Metric: effective TFLOP/s of the step's hybrid GEMMs = sum over the GEMMs of
+2*M*N*K (dense-equivalent) / the device time of the GEMM phase.  Tokens/s per
+token count M = M / the time of that M's GEMMs over all the matrices.  The
+column-norm, mask and pack phases are timed and reported beside it
+(`phases_ms`); `ms_per_step` is the whole step.  Also reported: the roofline
+of the kernel with the largest share of device time, isolated GEMM timings
+over the 2:4-tile fraction (speedup over the same kernel with an all-dense
+map), the decode GEMV in a CUDA graph, the end-to-end time through host
+buffers, and the CPU oracle on a bounded sample.
 
 Launch: ``python bench.py [--gpus N --steps K --warmup W]``; for N > 1 under
 ``torch.distributed.run`` one rank per GPU, each rank running the step on its
@@ -28,7 +34,6 @@ import argparse
 import datetime
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -44,6 +49,12 @@ sys.path.insert(0, ROOT)
 from sparse_gemm_wanda_b200 import inputs  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# The oracle's bounded sample (CPU baseline and reference arm alike): the
+# first 128 rows (one band) of every matrix, the first 16384 tokens of every
+# calibration set, every token count.
+ORACLE_ROWS = 128
+ORACLE_CALIB_TOKENS = 16384
 
 
 # ----------------------------------------------------------------- utilities
@@ -126,34 +137,6 @@ class L2Flusher:
         self.buf.fill_(1)
 
 
-class CallTimer:
-    """CUDA events around each ABI call on the launching stream."""
-
-    def __init__(self):
-        self.open = []
-        self.enabled = False
-
-    def wrap(self, name, fn, *a, **kw):
-        if not self.enabled:
-            return fn(*a, **kw)
-        s = torch.cuda.current_stream()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(s)
-        out = fn(*a, **kw)
-        e1.record(s)
-        self.open.append((name, e0, e1))
-        return out
-
-    def summary(self):
-        torch.cuda.synchronize()
-        agg = {}
-        for name, e0, e1 in self.open:
-            agg.setdefault(name, []).append(e0.elapsed_time(e1))
-        return {k: {"launches": len(v), "mean_ms": sum(v) / len(v), "total_ms": sum(v)}
-                for k, v in agg.items()}
-
-
 def max_over_ranks(value: float, device) -> float:
     """The largest value over all ranks (the job's time is its slowest rank's)."""
     import torch.distributed as dist
@@ -164,12 +147,22 @@ def max_over_ranks(value: float, device) -> float:
     return float(t.item())
 
 
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
 # ----------------------------------------------------------------- workload
-def make_tensors(wl, rank: int, device="cpu"):
-    """Synthetic weights, calibration and inputs of a workload (per-rank seed).
+def make_tensors(wl, rank: int, device="cpu", rows=None, calib_tokens=None):
+    """Synthetic weights, calibration sets and inputs of a workload (per-rank seed).
 
     Calibration sets are keyed by input group: layers that read the same
-    activations (q/k/v; gate/up) share one set and hence one column norm."""
+    activations (q/k/v; gate/up) share one set and hence one column norm.
+    `rows` / `calib_tokens` cut a bounded sample (the first rows of every
+    matrix, the first tokens of every calibration set: the same values as the
+    full draw's)."""
     seed = wl.seed + 1009 * rank
     mats = []
     outl = {}
@@ -179,75 +172,120 @@ def make_tensors(wl, rank: int, device="cpu"):
             outl[m.K] = inputs.outlier_channels(m.K, seed, wl.outlier_count)
         g = m.input_group
         if wl.calib_tokens and g not in calib:
-            buf = torch.empty((wl.calib_tokens, m.K), dtype=torch.bfloat16,
+            T = min(wl.calib_tokens, calib_tokens or wl.calib_tokens)
+            buf = torch.empty((T, m.K), dtype=torch.bfloat16,
                               pin_memory=device != "cpu" and torch.cuda.is_available())
-            inputs.activations_chunked(wl.calib_tokens, m.K, seed, outl[m.K],
-                                       role=10 * len(calib), out=buf)
+            inputs.activations_chunked(T, m.K, seed, outl[m.K], role=10 * len(calib), out=buf)
             calib[g] = buf.to(device)
         w = inputs.weight(m.N, m.K, seed + 17 * (mi + 1))
+        if rows is not None:
+            w = w[:rows].contiguous()
         xs = {M: inputs.activations(M, m.K, seed, outl[m.K], role=1 + mi * 100 + M)
               for M in wl.tokens}
-        mats.append({"name": m.name, "N": m.N, "K": m.K, "group": g, "W": w.to(device),
+        mats.append({"name": m.name, "N": w.shape[0], "K": m.K, "group": g, "W": w.to(device),
                      "X": {M: x.to(device) for M, x in xs.items()}})
     return mats, calib
 
 
-def gemm_flops(mats, tokens):
-    return sum(2.0 * M * m["N"] * m["K"] for m in mats for M in tokens)
+def units_of(wl, mats):
+    """(matrix index, 2:4-tile fraction) pairs of one step: every matrix at the
+    workload's fraction; a random-map sweep runs every matrix at every fraction."""
+    if wl.map_rule == "random":
+        return [(mi, f) for mi in range(len(mats)) for f in wl.fractions]
+    return [(mi, wl.fractions[0]) for mi in range(len(mats))]
 
 
-def run_step(P, wl, mats, calib, timer: CallTimer, keep=None):
-    """The hot path once for every matrix; returns the GEMM outputs."""
-    outs = []
-    colsq_cache = {}
-    for m in mats:
-        g = m["group"]
-        cin = colsq_cache.get(g)
-        r = timer.wrap("score_mask", P.patch_score_mask, m["W"], calib[g] if cin is None else None,
-                       tile_n=wl.tile_n, tile_k=wl.tile_k, fraction=wl.fractions[0],
-                       colsq_in=cin, want_colsq=cin is None)
-        if cin is None:
-            colsq_cache[g] = r["colsq"]
-        pk = timer.wrap("pack", P.patch_pack, m["W"], r["meta"], r["map"], tile_n=wl.tile_n,
-                        tile_k=wl.tile_k)
-        for M in wl.tokens:
-            outs.append(timer.wrap(f"gemm_m{M}" if M <= 16 else "gemm_prefill",
-                                   P.patch_hybrid_gemm, pk, m["X"][M]))
-        if keep is not None:
-            keep.append((m, r, pk))
+def random_maps(wl, mats, rank, device):
+    """Seeded random tile maps of the random-map workloads, one per unit."""
+    maps = {}
+    if wl.map_rule != "random":
+        return maps
+    for mi, f in units_of(wl, mats):
+        m = wl.matrices[mi]  # the full matrix's tiles, also for a row sample
+        nt = (m.N // wl.tile_n) * (m.K // wl.tile_k)
+        maps[(mi, f)] = inputs.random_map(nt, inputs.n_sparse_tiles(f, nt),
+                                          wl.seed + 1009 * rank + 31 * mi + int(f * 100)).to(device)
+    return maps
+
+
+def gemm_flops(wl, mats):
+    return sum(2.0 * M * mats[mi]["N"] * mats[mi]["K"] for mi, _ in units_of(wl, mats) for M in wl.tokens)
+
+
+class StepEvents:
+    """CUDA events at the phase boundaries of one step (on the launching stream)."""
+
+    def __init__(self):
+        self.marks = []
+
+    def mark(self, name):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(torch.cuda.current_stream())
+        self.marks.append((name, e))
+
+    def spans(self):
+        """{name: ms} between consecutive marks (a mark's span runs to the next)."""
+        out = {}
+        for (name, e0), (_, e1) in zip(self.marks, self.marks[1:]):
+            out[name] = out.get(name, 0.0) + e0.elapsed_time(e1)
+        return out
+
+
+def run_step(P, wl, mats, calib, maps, ys, ev: StepEvents | None = None, colsq_calls=None):
+    """The hot path once for every unit of the workload.
+
+    Phases in order: column sums of squares per calibration set, masks, packs,
+    GEMMs (largest token count first, so that the host has queued the short
+    decode calls long before the device reaches them).  `ev` gets a mark at
+    every phase boundary and before each token count's GEMMs; `colsq_calls`
+    collects (event, event, T, K) around each column-norm call."""
+    mark = ev.mark if ev is not None else (lambda name: None)
+    units = units_of(wl, mats)
+    mark("colsq")
+    colsq = {}
+    if wl.calib_tokens:
+        for g, xc in calib.items():
+            if colsq_calls is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(torch.cuda.current_stream())
+                colsq[g] = P.patch_colsq(xc)
+                e1.record(torch.cuda.current_stream())
+                colsq_calls.append((e0, e1, xc.shape[0], xc.shape[1]))
+            else:
+                colsq[g] = P.patch_colsq(xc)
+    mark("mask")
+    masks = []
+    Mmax = max(wl.tokens)
+    for mi, f in units:
+        m = mats[mi]
+        if wl.calib_tokens:
+            r = P.patch_score_mask(m["W"], None, tile_n=wl.tile_n, tile_k=wl.tile_k, fraction=f,
+                                   colsq_in=colsq[m["group"]])
         else:
-            pk.close()
-    return outs
+            # random-map workloads: 2:4 patterns from Wanda with the input X as calibration
+            r = P.patch_score_mask(m["W"], m["X"][Mmax], tile_n=wl.tile_n, tile_k=wl.tile_k,
+                                   map_in=maps[(mi, f)])
+        masks.append(r)
+    mark("pack")
+    pks = [P.patch_pack(mats[mi]["W"], r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k)
+           for (mi, _), r in zip(units, masks)]
+    for M in sorted(wl.tokens, reverse=True):
+        mark(f"gemm_m{M}")
+        for (mi, f), pk in zip(units, pks):
+            P.patch_hybrid_gemm(pk, mats[mi]["X"][M], out=ys[(mi, f, M)])
+    mark("end")
+    return pks
 
 
-def algorithmic_bytes(name, wl, mats, packed_bytes):
-    """Bytes each call must move at minimum: W and the codes it reads, what it writes."""
-    total = 0.0
-    count = 0
-    seen_k = set()
-    for m, pb in zip(mats, packed_bytes):
-        N, K = m["N"], m["K"]
-        nt = (N // wl.tile_n) * (K // wl.tile_k)
-        if name == "score_mask":
-            b = 2 * N * K + N * K / 8 + 8 * nt + (nt + 31) // 32 * 4
-            if K not in seen_k and wl.calib_tokens:
-                b += 2 * wl.calib_tokens * K + 8 * K
-                seen_k.add(K)
-            total += b
-            count += 1
-        elif name == "pack":
-            total += 2 * N * K + N * K / 8 + pb + 8 * (N // 128) * (K // 64)
-            count += 1
-        elif name.startswith("gemm_m"):
-            M = int(name[6:])
-            total += pb + 8 * (N // 128) * (K // 64) + 2 * M * K + 2 * M * N
-            count += 1
-    return total / max(count, 1)
+def close_all(pks):
+    for pk in pks:
+        pk.close()
 
 
 def traffic_for(kernel_key: str):
     """dram read+write bytes per launch from the committed ncu summary, if the
-    kernel source is unchanged since the capture; else None."""
+    kernel's source is unchanged since the capture; else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
@@ -262,15 +300,23 @@ def traffic_for(kernel_key: str):
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     if h != ent.get("source_sha256_16"):
         return None
-    return ent.get("bytes_per_launch")
+    return ent
+
+
+def colsq_bytes(T, K):
+    """Algorithmic bytes of one column-norm call: the calibration set read once,
+    the 128-token chunk partials written and read back, the sums written."""
+    chunks = (T + 127) // 128
+    return 2.0 * T * K + 2 * 8.0 * chunks * K + 8.0 * K
 
 
 # ----------------------------------------------------------- isolated GEMMs
 def isolated_gemm(P, wl, W, M, frac_map, X, flush, reps=20, seed=0):
-    """Time one GEMM configuration with L2 flushed before every call."""
+    """Time one GEMM configuration with L2 flushed before every call.  The
+    2:4 patterns are Wanda's with X as calibration; the map is seeded random."""
     N, K = W.shape
     nt = (N // wl.tile_n) * (K // wl.tile_k)
-    tmap = inputs.random_map(nt, int(round(frac_map * nt)), seed).cuda()
+    tmap = inputs.random_map(nt, inputs.n_sparse_tiles(frac_map, nt), seed).cuda()
     r = P.patch_score_mask(W, X, tile_n=wl.tile_n, tile_k=wl.tile_k, map_in=tmap)
     pk = P.patch_pack(W, r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
@@ -287,8 +333,11 @@ def isolated_gemm(P, wl, W, M, frac_map, X, flush, reps=20, seed=0):
         e1.record(s)
         e1.synchronize()
         ts.append(e0.elapsed_time(e1))
+    status = P.patch_get_status(pk)
     nbytes = pk.packed_bytes
     pk.close()
+    if status:
+        raise RuntimeError(f"GEMM status {status}")
     return statistics.median(ts), nbytes
 
 
@@ -301,7 +350,7 @@ def graph_gemm(P, wl, W, M, frac_map, X, calls_per_copy=8, replays=5, seed=0):
     Returns (ms per call, packed bytes of one copy, copies)."""
     N, K = W.shape
     nt = (N // wl.tile_n) * (K // wl.tile_k)
-    tmap = inputs.random_map(nt, int(round(frac_map * nt)), seed).cuda()
+    tmap = inputs.random_map(nt, inputs.n_sparse_tiles(frac_map, nt), seed).cuda()
     r = P.patch_score_mask(W, X, tile_n=wl.tile_n, tile_k=wl.tile_k, map_in=tmap)
     first = P.patch_pack(W, r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k)
     l2 = torch.cuda.get_device_properties(0).L2_cache_size
@@ -344,101 +393,141 @@ def graph_gemm(P, wl, W, M, frac_map, X, calls_per_copy=8, replays=5, seed=0):
     return statistics.median(ts), nbytes, copies
 
 
-def step_gemm_graph(P, wl, kept, replays=5):
-    """The step's decode GEMMs (every matrix, every M <= 16) back to back in a
-    CUDA graph, each matrix packed into enough copies that consecutive calls
-    never find their weights in L2.  Returns (ms per call, algorithmic bytes
-    per call, launches of the library per call)."""
-    l2 = torch.cuda.get_device_properties(0).L2_cache_size
-    per_set = sum(pk.packed_bytes for _, _, pk in kept)
-    copies = max(2, -(-3 * l2 // per_set))
-    sets = [[pk for _, _, pk in kept]]
-    for _ in range(copies - 1):
-        sets.append([P.patch_pack(m["W"], r["meta"], r["map"], tile_n=wl.tile_n,
-                                  tile_k=wl.tile_k) for m, r, _ in kept])
-    toks = [M for M in wl.tokens if M <= 16]
-    outs = {(mi, M): torch.empty((M, m["N"]), dtype=torch.bfloat16, device="cuda")
-            for mi, (m, _, _) in enumerate(kept) for M in toks}
-    order = [(M, c, mi) for M in toks for c in range(copies) for mi in range(len(kept))]
+def prefill_sweep(P, wl_name, flush, peaks):
+    """Isolated prefill GEMMs over the 2:4-tile fraction: the Llama-7B MLP shapes
+    at M = 2048 (f in {0, .25, .5, .75, 1}) and the 13B MLP shapes at M = 4096
+    (f in {0, .75, 1}), each with its speedup over the all-dense map."""
+    wls = inputs.workloads()
+    dense_peak = float(peaks["bf16_tflops"])
+    out = {}
+    for name, fracs in (("llama7b-prefill", (0.0, 0.25, 0.5, 0.75, 1.0)),
+                        ("llama13b-prefill", (0.0, 0.75, 1.0))):
+        w = wls[name]
+        M = w.tokens[0]
+        for mi, m in enumerate(w.matrices):
+            o = inputs.outlier_channels(m.K, w.seed)
+            Wd = inputs.weight(m.N, m.K, w.seed + m.N).cuda()
+            Xd = inputs.activations(M, m.K, w.seed, o, role=1).cuda()
+            ent = {}
+            base = None
+            for f in fracs:
+                t_ms, _ = isolated_gemm(P, w, Wd, M, f, Xd, flush, seed=w.seed + m.N + int(f * 100))
+                fl = 2.0 * M * m.N * m.K
+                nt = (m.N // 128) * (m.K // 128)
+                s_ach = inputs.n_sparse_tiles(f, nt) / nt / 2.0
+                eff = fl / (t_ms * 1e-3) / 1e12
+                useful = fl * (1 - s_ach) / (t_ms * 1e-3) / 1e12
+                if f == 0.0:
+                    base = t_ms
+                e = {"us": t_ms * 1e3, "sparsity": s_ach, "effective_tflops": eff,
+                     "useful_tflops": useful, "speedup_vs_all_dense": base / t_ms,
+                     "useful_frac_of_dense_peak": useful / dense_peak}
+                if f == 1.0:
+                    e["frac_of_sparse_peak"] = eff / (2.0 * dense_peak)
+                ent[f"f{f}"] = e
+            out[f"{name} M={M} N={m.N} K={m.K}"] = ent
+            del Wd, Xd
+    return {"by_shape": out, "dense_peak_tflops": dense_peak,
+            "note": "effective = 2MNK / t (dense-equivalent); useful = 2MNK(1-s) / t against the "
+                    "burst dense peak (a kernel timed alone); sparse peak = 2 x the dense peak; "
+                    "seeded random maps, 2:4 patterns from Wanda with X as calibration; L2 "
+                    "flushed before every call"}
 
-    def body():
-        for M, c, mi in order:
-            P.patch_hybrid_gemm(sets[c][mi], kept[mi][0]["X"][M], out=outs[(mi, M)])
 
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        body()
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    n0 = P.launch_count()
-    with torch.cuda.graph(graph):
-        body()
-    launches = P.launch_count() - n0
-    graph.replay()
-    torch.cuda.synchronize()
-    s = torch.cuda.current_stream()
-    ts = []
-    for _ in range(replays):
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(s)
-        graph.replay()
-        e1.record(s)
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1))
-    byts = sum(sets[c][mi].packed_bytes + 2 * M * (kept[mi][0]["K"] + kept[mi][0]["N"])
-               for M, c, mi in order)
-    status = [P.patch_get_status(pk) for st in sets for pk in st]
-    del graph
-    for st in sets[1:]:
-        for pk in st:
-            pk.close()
-    torch.cuda.synchronize()
-    if any(status):
-        raise RuntimeError(f"GEMM status {status}")
-    n = len(order)
-    return statistics.median(ts) / n, byts / n, launches / n, copies
+def decode_isolated(P, flush, peaks):
+    """The decode GEMV on the Llama-7B decode shapes at M in {1, 4, 16}: one
+    CUDA graph of back-to-back calls over copies larger than 3x L2, per call."""
+    w = inputs.workloads()["llama7b-decode"]
+    hbm = float(peaks["hbm_gbs"])
+    out = {}
+    for mi, m in enumerate(w.matrices):
+        o = inputs.outlier_channels(m.K, w.seed)
+        Wd = inputs.weight(m.N, m.K, w.seed + m.N).cuda()
+        for M in w.tokens:
+            X = inputs.activations(M, m.K, w.seed, o, role=1 + M).cuda()
+            tg_ms, nbytes, copies = graph_gemm(P, w, Wd, M, w.fractions[0], X, seed=M)
+            b = nbytes + 2 * M * m.K + 2 * M * m.N
+            out[f"{m.N}x{m.K} m{M}"] = {"us_graph": tg_ms * 1e3, "compressed_bytes": b,
+                                        "achieved_gbs": b / (tg_ms * 1e-3) / 1e9,
+                                        "frac_of_hbm": b / (tg_ms * 1e-3) / 1e9 / hbm}
+        del Wd
+    return {"by_shape": out, "map": "seeded random, half the tiles 2:4 (2:4 patterns from Wanda "
+                                     "with X as calibration)",
+            "timing": "one CUDA graph of back-to-back calls cycling through packed copies larger "
+                      "than 3x L2, per call",
+            "bytes": "packed weight bytes (values + metadata) + X + Y"}
 
 
 # -------------------------------------------------------------- CPU oracle
-def cpu_oracle_sample(wl, rows=512, reps=1):
-    """The oracle as it stands on a bounded sample: the first `rows` rows of every
-    matrix through every step (full calibration set).  Returns (seconds, flops)."""
+def oracle_sample(wl, reps=1):
+    """The oracle as it stands on the bounded sample (ORACLE_ROWS rows of every
+    matrix, ORACLE_CALIB_TOKENS tokens of every calibration set, every token
+    count), every step of the path.  Returns (seconds of the GEMMs, GEMM flops,
+    seconds of everything, description)."""
     import numpy as np
     import oracle
-    mats, calib = make_tensors(wl, 0)
+    mats, calib = make_tensors(wl, 0, rows=ORACLE_ROWS, calib_tokens=ORACLE_CALIB_TOKENS)
+    maps = random_maps(wl, mats, 0, "cpu")
 
     def bits(t):
         return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
-    t0 = time.perf_counter()
+    t_all = time.perf_counter()
+    t_gemm = 0.0
     flops = 0.0
+    Mmax = max(wl.tokens)
     for _ in range(reps):
-        colsq = {}
-        for m in mats:
-            K, g = m["K"], m["group"]
-            if g not in colsq:
-                colsq[g] = oracle.colsq(bits(calib[g]))
-            w = bits(m["W"][:rows])
-            sc = oracle.wanda_scores(w, colsq[g])
+        colsq = {g: oracle.colsq(bits(x)) for g, x in calib.items()}
+        for mi, f in units_of(wl, mats):
+            m = mats[mi]
+            w = bits(m["W"])
+            if wl.calib_tokens:
+                s = colsq[m["group"]]
+            else:
+                s = oracle.colsq(bits(m["X"][Mmax]))
+            sc = oracle.wanda_scores(w, s)
             meta = oracle.select_2of4(sc)
             loss = oracle.tile_loss(sc, meta, wl.tile_n, wl.tile_k)
-            tmap = oracle.select_map(loss, oracle.n_sparse(wl.fractions[0], loss.shape[0]))
+            if wl.map_rule == "random":
+                # the sample's rows are the first tile row: its tiles keep
+                # their types from the full matrix's map (tiles 0 .. K/tk - 1)
+                full = maps[(mi, f)].numpy().view(np.uint32)
+                nt = loss.shape[0]
+                tmap = np.zeros((nt + 31) // 32, dtype=np.uint32)
+                for t in range(nt):
+                    if (int(full[t // 32]) >> (t % 32)) & 1:
+                        tmap[t // 32] |= np.uint32(1 << (t % 32))
+            else:
+                tmap = oracle.select_map(loss, oracle.n_sparse(f, loss.shape[0]))
             oracle.pack(w, meta, tmap, wl.tile_n, wl.tile_k)
             weff = oracle.weff(w, meta, tmap, wl.tile_n, wl.tile_k)
             for M in wl.tokens:
+                t0 = time.perf_counter()
                 oracle.gemm(bits(m["X"][M]), weff)
-                flops += 2.0 * M * rows * K
-    return time.perf_counter() - t0, flops
+                t_gemm += time.perf_counter() - t0
+                flops += 2.0 * M * m["N"] * m["K"]
+    secs = time.perf_counter() - t_all
+    desc = (f"first {ORACLE_ROWS} rows of every matrix"
+            + (f", first {ORACLE_CALIB_TOKENS} tokens of every calibration set" if wl.calib_tokens
+               else "") + f", M in {wl.tokens}, every step (column norms, scores, codes, tile "
+            f"loss, map, pack, W_eff, GEMM); value = sample GEMM flops / GEMM seconds")
+    return t_gemm, flops, secs, desc
 
 
-def cpu_cores():
-    try:
-        return len(os.sched_getaffinity(0))
-    except AttributeError:
-        return os.cpu_count()
+def config_of(wl, world):
+    return {"workload": wl.name,
+            "matrices": [f"{m.name} {m.N}x{m.K}" for m in wl.matrices],
+            "tiles": f"{wl.tile_n}x{wl.tile_k}",
+            "fractions_2to4_tiles": wl.fractions,
+            "map": "least Wanda tile loss" if wl.map_rule == "loss" else "seeded random",
+            "calibration_tokens_per_input": wl.calib_tokens, "tokens": wl.tokens,
+            "l2": "flushed (512 MB write) before every timed step, outside its events; the "
+                  "calibration sets (2.1-5.8 GB) exceed L2",
+            "parallelism": f"independent matrices per rank x{world}"}
+
+
+METRIC = ("hybrid-sparse GEMM effective TFLOP/s (dense-equivalent 2*M*N*K over the device time "
+          "of the step's hybrid GEMMs) & tokens/s, vs sparsity; %roofline")
 
 
 # --------------------------------------------------------------------- main
@@ -448,13 +537,14 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama7b-decode")
+    ap.add_argument("--workload", default="llama7b-block")
     ap.add_argument("--no-extras", action="store_true", help="skip isolated GEMM / oracle legs")
-    ap.add_argument("--case", choices=["gemm", "mask", "pack"], default=None,
+    ap.add_argument("--case", choices=["gemm", "mask", "pack", "colsq"], default=None,
                     help="run one operation a few times and exit (profiling aid, no JSON)")
     ap.add_argument("--N", type=int, default=11008)
     ap.add_argument("--K", type=int, default=4096)
     ap.add_argument("--M", type=int, default=2048)
+    ap.add_argument("--T", type=int, default=2048)
     ap.add_argument("--frac", type=float, default=0.5)
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
@@ -480,13 +570,16 @@ def main():
     P.load_library()
 
     mats, calib = make_tensors(wl, rank, device="cuda")
-    flops = gemm_flops(mats, wl.tokens)
-    tokens = sum(wl.tokens) * len(mats)
+    maps = random_maps(wl, mats, rank, "cuda")
+    units = units_of(wl, mats)
+    ys = {(mi, f, M): torch.empty((M, mats[mi]["N"]), dtype=torch.bfloat16, device="cuda")
+          for mi, f in units for M in wl.tokens}
+    flops = gemm_flops(wl, mats)
     flush = L2Flusher()
-    timer = CallTimer()
+    s = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
-        run_step(P, wl, mats, calib, timer)
+        close_all(run_step(P, wl, mats, calib, maps, ys))
     torch.cuda.synchronize()
 
     # ------------------------------------------------------------ timed steps
@@ -495,192 +588,140 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
-    s = torch.cuda.current_stream()
-    step_ms = []
-    events = []
+    steps = []
+    colsq_calls = []
     launches0 = P.launch_count()
     for _ in range(args.steps):
         flush()  # between timed steps, outside the events
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(s)
-        run_step(P, wl, mats, calib, timer)
-        e1.record(s)
-        events.append((e0, e1))
+        ev = StepEvents()
+        close_all(run_step(P, wl, mats, calib, maps, ys, ev=ev, colsq_calls=colsq_calls))
+        steps.append(ev)
     launches = P.launch_count() - launches0
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    timer.enabled = False
     clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in events]
+
+    spans = [ev.spans() for ev in steps]
+    step_ms = [sum(sp.values()) for sp in spans]
     total_ms = max_over_ranks(sum(step_ms), "cuda")
     ms_per_step = total_ms / args.steps
-
-    # per-call breakdown: the same steps again with CUDA events around every
-    # call (kept out of the timed steps: recording events costs host time,
-    # and the step is host-bound)
-    timer.enabled = True
-    for _ in range(args.steps):
-        flush()
-        run_step(P, wl, mats, calib, timer)
-    timer.enabled = False
-    calls = timer.summary()
-
-    # packed sizes, for algorithmic bytes
-    keep = []
-    run_step(P, wl, mats, calib, CallTimer(), keep=keep)
-    packed_bytes = [pk.packed_bytes for _, _, pk in keep]
-    torch.cuda.synchronize()
+    phase = {k: statistics.fmean(sp[k] for sp in spans) for k in spans[0]}
+    gemm_keys = [k for k in phase if k.startswith("gemm_m")]
+    gemm_ms = max_over_ranks(sum(phase[k] for k in gemm_keys), "cuda")
+    value = flops * world / (gemm_ms * 1e-3) / 1e12
+    n_mats = len(units)
+    by_m = {}
+    for M in wl.tokens:
+        t = max_over_ranks(phase[f"gemm_m{M}"], "cuda")
+        fl = sum(2.0 * M * mats[mi]["N"] * mats[mi]["K"] for mi, _ in units)
+        by_m[f"m{M}"] = {"ms": t, "tokens_per_s": M * world / (t * 1e-3),
+                         "effective_tflops": fl * world / (t * 1e-3) / 1e12,
+                         "gemms": n_mats}
+    tokens_per_s = sum(wl.tokens) * world / (gemm_ms * 1e-3)
+    phases_max = {k: max_over_ranks(v, "cuda") for k, v in phase.items()}  # every rank takes part
 
     peaks, peak_kind = load_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
-    roof = None
-    if all(M <= 16 for M in wl.tokens):
-        # the decode GEMM is the kernel with the largest share of device time
-        # (launch list under profiles/); its launches, back to back in a graph
-        ms_call, b_call, l_call, copies = step_gemm_graph(P, wl, keep)
-        ach = b_call / (ms_call * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
-                "frac": ach / hbm_peak, "traffic": traffic_for("hybrid_gemm_decode"),
-                "kernel": "decode_gemm_kernel (+ decode_reduce_kernel)",
-                "algorithmic_bytes_per_launch": b_call, "launch_us": ms_call * 1e3,
-                "launches_per_call": l_call,
-                "timing": f"CUDA events around a graph of the step's decode GEMMs cycling "
-                          f"{copies} packed copies of each matrix (> 3x L2)",
-                "peak_source": peak_kind}
-    else:
-        dominant = max((k for k in calls if k.startswith("gemm_prefill")),
-                       key=lambda k: calls[k]["total_ms"])
-        fl = sum(2.0 * M * m["N"] * m["K"] for m in mats for M in wl.tokens if M > 16) / \
-            max(1, calls[dominant]["launches"] // args.steps)
-        ach = fl / (calls[dominant]["mean_ms"] * 1e-3) / 1e12
-        pk_ = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
-        roof = {"bound": "tensor", "achieved": ach, "peak": pk_, "unit": "TFLOP/s",
-                "frac": ach / pk_, "traffic": None, "kernel": "hybrid_gemm_kernel (prefill)",
-                "peak_source": peak_kind}
-    for _, _, pk in keep:
-        pk.close()
-    torch.cuda.synchronize()
-    per_call = {}
-    for k, v in calls.items():
-        ent = {"launches_per_step": v["launches"] / args.steps, "mean_us": v["mean_ms"] * 1e3,
-               "share": v["total_ms"] / max(sum(c["total_ms"] for c in calls.values()), 1e-9)}
-        if not k.startswith("gemm_prefill"):
-            b = algorithmic_bytes(k, wl, mats, packed_bytes)
-            ent["algorithmic_bytes"] = b
-            ent["achieved_gbs"] = b / (v["mean_ms"] * 1e-3) / 1e9
-        per_call[k] = ent
+    dense_burst = float(peaks["bf16_tflops"])
+
+    # ---------------------------------------------------- rooflines
+    rooflines = {}
+    if colsq_calls:
+        tot_ms = sum(e0.elapsed_time(e1) for e0, e1, _, _ in colsq_calls)
+        tot_b = sum(colsq_bytes(T, K) for _, _, T, K in colsq_calls)
+        n = len(colsq_calls)
+        ach = tot_b / (tot_ms * 1e-3) / 1e9
+        tr = traffic_for("colsq")
+        traffic = None
+        if tr:
+            # captured on a smaller calibration set: scaled by the tokens per call
+            tok = statistics.fmean(T for _, _, T, _ in colsq_calls)
+            kk = statistics.fmean(T * K for _, _, T, K in colsq_calls) / tok
+            traffic = tr["bytes_per_token_column"] * tok * kk
+        rooflines["colsq"] = {
+            "bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+            "frac": ach / hbm_peak, "traffic": traffic,
+            "kernel": "colsq_partial_kernel (+ colsq_final_kernel, the in-order fold)",
+            "algorithmic_bytes_per_launch": tot_b / n, "launch_us": tot_ms / n * 1e3,
+            "share_of_step": phase["colsq"] / ms_per_step,
+            "timing": "CUDA events around every patch_colsq call of the timed steps",
+            "bytes": "2*T*K calibration read + 16*K*ceil(T/128) chunk partials written and "
+                     "re-read + 8*K sums",
+            "peak_source": peak_kind}
+    big = max(M for M in wl.tokens)
+    if big > 16:
+        units_fl = sum(2.0 * big * mats[mi]["N"] * mats[mi]["K"] * (1 - f / 2) for mi, f in units)
+        t = phase[f"gemm_m{big}"]
+        ach = units_fl / (t * 1e-3) / 1e12
+        rooflines["gemm_prefill"] = {
+            "bound": "tensor", "achieved": ach, "peak": dense_burst, "unit": "TFLOP/s",
+            "frac": ach / dense_burst, "traffic": None,
+            "kernel": f"hybrid GEMM at M = {big} (two-SM / band-pair kernels)",
+            "share_of_step": t / ms_per_step,
+            "flops": "useful 2*M*N*K*(1 - f/2) over the step's GEMMs at this M",
+            "peak_note": "burst bf16 dense peak (tcgen05 dense and sparse MMAs together)",
+            "peak_source": peak_kind}
+    dominant = max(rooflines, key=lambda k: rooflines[k]["share_of_step"]) if rooflines else None
+    roof = rooflines.get(dominant)
 
     # ------------------------------------------------------- end to end
     e2e = None
-    if rank == 0 or world > 1:
+    if not args.no_extras or world > 1:
         host = {"W": [m["W"].cpu().pin_memory() for m in mats],
                 "X": [{M: x.cpu().pin_memory() for M, x in m["X"].items()} for m in mats],
-                "C": {K: c.cpu().pin_memory() for K, c in calib.items()}}
+                "C": {g: c.cpu().pin_memory() for g, c in calib.items()}}
         h2d = sum(t.numel() * 2 for t in host["W"]) + sum(c.numel() * 2 for c in host["C"].values()) \
             + sum(x.numel() * 2 for d in host["X"] for x in d.values())
-        d2h = sum(m["N"] * M * 2 for m in mats for M in wl.tokens)
-        e2e_events = []
-        for it in range(args.warmup + args.steps):
+        hy = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in ys.items()}
+        d2h = sum(v.numel() * 2 for v in ys.values())
+        e2e_ms = []
+        n_e2e = min(args.steps, 5)
+        for it in range(args.warmup + n_e2e):
             flush()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(s)
-            dm = []
-            for mi, m in enumerate(mats):
-                dm.append({"name": m["name"], "N": m["N"], "K": m["K"], "group": m["group"],
-                           "W": host["W"][mi].to("cuda", non_blocking=True),
-                           "X": {M: x.to("cuda", non_blocking=True) for M, x in host["X"][mi].items()}})
-            dc = {K: c.to("cuda", non_blocking=True) for K, c in host["C"].items()}
-            outs = run_step(P, wl, dm, dc, CallTimer())
-            hy = [o.to("cpu", non_blocking=True) for o in outs]
+            dm = [{"name": m["name"], "N": m["N"], "K": m["K"], "group": m["group"],
+                   "W": host["W"][mi].to("cuda", non_blocking=True),
+                   "X": {M: x.to("cuda", non_blocking=True) for M, x in host["X"][mi].items()}}
+                  for mi, m in enumerate(mats)]
+            dc = {g: c.to("cuda", non_blocking=True) for g, c in host["C"].items()}
+            close_all(run_step(P, wl, dm, dc, maps, ys))
+            for k, v in ys.items():
+                hy[k].copy_(v, non_blocking=True)
             e1.record(s)
             e1.synchronize()
-            del hy
+            del dm, dc
             if it >= args.warmup:
-                e2e_events.append(e0.elapsed_time(e1))
-        e2e_ms = max_over_ranks(sum(e2e_events) / len(e2e_events), "cuda")
-        e2e = {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+                e2e_ms.append(e0.elapsed_time(e1))
+        e_ms = max_over_ranks(statistics.fmean(e2e_ms), "cuda")
+        e2e = {"value": flops * world / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "note": "the step's GEMM flops over the whole end-to-end step: host->device copies "
+                       "of W, calibration sets and X from pinned memory, every phase, and the "
+                       "device->host copy of every Y, through the binding's public calls"}
+        del host, hy
 
-    # --------------------------------------------- isolated GEMM measurements
+    # --------------------------------------------- isolated measurements
     extras = {}
     # one GPU only: under torchrun the other ranks would wait for rank 0 at the
     # closing barrier for as long as these take
     if not args.no_extras and rank == 0 and world == 1:
-        W0 = mats[-1]["W"]  # the MLP-shaped matrix
-        dec = {}
-        graph_roof = None
-        for M in wl.tokens:
-            if M > 16:
-                continue
-            X = mats[-1]["X"][M]
-            t_ms, nb = isolated_gemm(P, wl, W0, M, wl.fractions[0], X, flush, seed=M)
-            tg_ms, _, copies = graph_gemm(P, wl, W0, M, wl.fractions[0], X, seed=M)
-            b = nb + 2 * M * W0.shape[1] + 2 * M * W0.shape[0]
-            dec[f"m{M}"] = {"us_graph": tg_ms * 1e3, "us_single_flushed": t_ms * 1e3,
-                            "compressed_bytes": b,
-                            "achieved_gbs": b / (tg_ms * 1e-3) / 1e9,
-                            "frac_of_hbm": b / (tg_ms * 1e-3) / 1e9 / hbm_peak,
-                            "achieved_gbs_single": b / (t_ms * 1e-3) / 1e9}
-        extras["decode_gemm_isolated"] = {
-            "matrix": f"{W0.shape[0]}x{W0.shape[1]}", "fraction_2to4_tiles": wl.fractions[0],
-            "by_m": dec,
-            "timing": f"us_graph: one CUDA graph of back-to-back calls cycling through {copies} "
-                      "packed copies (> 3x L2), per call; us_single_flushed: one call after an "
-                      "L2 flush, host launch latency included",
-            "bytes": "packed weight bytes (values + metadata) + X + Y"}
-        # prefill GEMMs: the Llama-7B MLP shapes at M = 2048 (f in {0, .5, 1})
-        # and the 13B MLP shapes at M = 4096 (f in {0, 1}); the 2:4 target is
-        # 60 % of the sparse bf16 peak, counted as 2x the measured dense peak
-        g = torch.Generator().manual_seed(4242)
-        dense_peak = float(peaks["bf16_tflops"])
-        shapes = [(11008, 4096, 2048, (0.0, 0.5, 1.0)), (4096, 11008, 2048, (0.0, 0.5, 1.0)),
-                  (13824, 5120, 4096, (0.0, 1.0)), (5120, 13824, 4096, (0.0, 1.0))]
-        pre_all = {}
-        for N_, K_, M_, fracs in shapes:
-            Wp = (torch.randn(N_, K_, generator=g) * 0.02).to(torch.bfloat16).cuda()
-            Xp = torch.randn(M_, K_, generator=g).to(torch.bfloat16).cuda()
-            pre = {}
-            base = None
-            for f in fracs:
-                t_ms, _ = isolated_gemm(P, wl, Wp, M_, f, Xp, flush, seed=7)
-                fl = 2.0 * M_ * N_ * K_
-                eff = fl / (t_ms * 1e-3) / 1e12
-                useful = fl * (1 - f / 2) / (t_ms * 1e-3) / 1e12
-                if f == 0.0:
-                    base = t_ms
-                ent = {"us": t_ms * 1e3, "effective_tflops": eff, "useful_tflops": useful,
-                       "speedup_vs_all_dense": base / t_ms}
-                if f == 0.0:
-                    ent["frac_of_dense_peak"] = eff / dense_peak
-                if f == 1.0:
-                    ent["frac_of_sparse_peak"] = eff / (2.0 * dense_peak)
-                pre[f"f{f}"] = ent
-            pre_all[f"M={M_} N={N_} K={K_}"] = pre
-            del Wp, Xp
-        extras["prefill_gemm_isolated"] = {
-            "by_shape": pre_all, "dense_peak_tflops": dense_peak, "peak_source": peak_kind,
-            "note": "effective = 2MNK / t (dense-equivalent); sparse peak = 2 x measured dense peak "
-                    "(the sparse MMA itself ran at about 1.6 x the dense rate at N = 256 in a "
-                    "one-SM instruction probe, so about 0.8 of this peak is the ceiling); "
-                    "seeded random maps; L2 flushed before every call"}
+        extras["prefill_gemm_isolated"] = prefill_sweep(P, wl.name, flush, peaks)
+        extras["decode_gemm_isolated"] = decode_isolated(P, flush, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
-        secs, fl = cpu_oracle_sample(wl)
-        cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
-               "kind": "oracle",
-               "sample": "first 512 rows of each matrix through every step, full calibration "
-                         f"set, M in {wl.tokens}; {secs:.1f} s"}
+        t_gemm, fl, secs, desc = oracle_sample(wl)
+        cpu = {"value": fl / t_gemm / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
+               "kind": "oracle", "sample": f"{desc}; {secs:.1f} s in all, {t_gemm:.1f} s GEMMs"}
 
     if rank == 0:
         line = {
-            "metric": "hybrid-sparse GEMM effective TFLOP/s (dense-equivalent 2*M*N*K over the "
-                      "whole step: mask build + pack + GEMMs)",
-            "value": flops * world / (ms_per_step * 1e-3) / 1e12,
+            "metric": METRIC,
+            "value": value,
             "unit": "TFLOP/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -692,17 +733,15 @@ def main():
             "dtype": "bf16",
             "data": "synthetic (seeded Llama-shaped weights N(0,0.02); activations N(0,1) with "
                     "1% outlier channels x20)",
-            "config": {"workload": wl.name, "matrices": [f"{m['N']}x{m['K']}" for m in mats],
-                       "tiles": f"{wl.tile_n}x{wl.tile_k}", "fraction_2to4_tiles": wl.fractions[0],
-                       "map": "least Wanda tile loss" if wl.map_rule == "loss" else "seeded random",
-                       "calibration_tokens": wl.calib_tokens, "tokens": wl.tokens,
-                       "l2": "flushed (512 MB write) between timed steps",
-                       "parallelism": f"independent matrices per rank x{world}"},
-            "tokens_per_s": tokens * world / (ms_per_step * 1e-3),
+            "config": config_of(wl, world),
+            "gemm_ms_per_step": gemm_ms,
+            "phases_ms": phases_max,
+            "tokens_per_s": tokens_per_s,
+            "by_m": by_m,
             "e2e": e2e,
             "gpu_launches": launches,
             "roofline": roof,
-            "calls": per_call,
+            "rooflines": rooflines,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -719,9 +758,16 @@ def run_case(args):
     torch.cuda.set_device(0)
     P.load_library()
     g = torch.Generator().manual_seed(4242)
+    if args.case == "colsq":
+        Xcal = torch.randn(args.T, args.K, generator=g).to(torch.bfloat16).cuda()
+        for _ in range(args.reps):
+            P.patch_colsq(Xcal)
+        torch.cuda.synchronize()
+        print(f"case colsq T={args.T} K={args.K} ok")
+        return
     W = (torch.randn(args.N, args.K, generator=g) * 0.02).to(torch.bfloat16).cuda()
     X = torch.randn(args.M, args.K, generator=g).to(torch.bfloat16).cuda()
-    Xcal = torch.randn(2048, args.K, generator=g).to(torch.bfloat16).cuda()
+    Xcal = torch.randn(args.T, args.K, generator=g).to(torch.bfloat16).cuda()
     nt = (args.N // 128) * (args.K // 128)
     tmap = inputs.random_map(nt, int(round(args.frac * nt)), 7).cuda()
     if args.case == "mask":
@@ -744,30 +790,30 @@ def run_case(args):
 
 
 def main_reference(args, wl, world, rank):
-    """The oracle as it stands on the host cores, on a bounded sample per step."""
+    """The oracle as it stands on the host cores, on the bounded sample, per step."""
     if rank != 0:
         return
-    rows = 256
     for _ in range(args.warmup):
-        cpu_oracle_sample(wl, rows=rows)
-    tot_s, tot_f = 0.0, 0.0
+        oracle_sample(wl)
+    tot_g, tot_f, tot_s = 0.0, 0.0, 0.0
+    desc = ""
     for _ in range(args.steps):
-        sec, fl = cpu_oracle_sample(wl, rows=rows)
-        tot_s += sec
+        t_gemm, fl, secs, desc = oracle_sample(wl)
+        tot_g += t_gemm
         tot_f += fl
-    v = tot_f / tot_s / 1e12
+        tot_s += secs
+    v = tot_f / tot_g / 1e12
     line = {
         "impl": "reference",
-        "metric": "hybrid-sparse GEMM effective TFLOP/s (dense-equivalent 2*M*N*K over the whole "
-                  "step: mask build + pack + GEMMs)",
+        "metric": METRIC,
         "value": v, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": wl.name,
-                                        "sample": f"first {rows} rows of each matrix"},
+        "data": "synthetic (seeded Llama-shaped weights N(0,0.02); activations N(0,1) with "
+                "1% outlier channels x20)",
+        "config": config_of(wl, world),
         "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-                         "sample": f"first {rows} rows of each matrix, full calibration set, "
-                                   f"M in {wl.tokens}"},
+                         "sample": desc},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -107,6 +107,40 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
                               double *tile_loss_out, void *stream);
 
 /*
+ * Column sums of squares of calibration activations alone: the activation
+ * term of the Wanda score (SparseGPT-vs-Wanda page, section on Wanda: the
+ * weight magnitude is weighed by the input activation of its channel; here
+ * ||X_:,j||_2^2 over the calibration tokens).  colsq_out [K] fp64 receives
+ * exactly what patch_score_mask writes to colsq_out for the same Xcal (the
+ * fixed order above), ready for its colsq_in: one call per distinct layer
+ * input, shared by the matrices that read it.
+ *   Xcal_bf16 [T,K] bf16, 16-byte aligned; T >= 1; K a multiple of 64.
+ * Scratch (8*K*ceil(T/128) bytes of chunk partials) comes from the library's
+ * pool, released on the stream.  Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA.
+ */
+patch_status patch_colsq(const void *Xcal_bf16, int64_t T, int64_t K, double *colsq_out,
+                         void *stream);
+
+/*
+ * The two halves of patch_colsq, for callers that hold the calibration tokens
+ * in pieces (e.g. one piece per GPU, each a multiple of 128 tokens except the
+ * last).
+ *   patch_colsq_partials: partials_out [ceil(T/128), K] fp64 (16-byte
+ *     aligned, written): row c is the sum of x_tj^2 over tokens 128c ..
+ *     128c+127 of this Xcal, added token by token from 0.0.
+ *   patch_colsq_fold: colsq_out[j] = the rows of partials [chunks, K] added
+ *     row by row from 0.0.
+ * The partials of consecutive pieces, stacked in token order and folded, give
+ * bit for bit patch_colsq's result for the whole set.  No scratch.  Errors:
+ * INVALID_ARG (null pointers, T or chunks < 1, K not a multiple of 64,
+ * misalignment), UNSUPPORTED, CUDA.
+ */
+patch_status patch_colsq_partials(const void *Xcal_bf16, int64_t T, int64_t K,
+                                  double *partials_out, void *stream);
+patch_status patch_colsq_fold(const double *partials, int64_t chunks, int64_t K, double *colsq_out,
+                              void *stream);
+
+/*
  * Allocation-free variant of patch_score_mask.  The pages have no
  * counterpart: this entry point exists for callers that may not allocate
  * device memory at all, e.g. code running inside a framework whose caching

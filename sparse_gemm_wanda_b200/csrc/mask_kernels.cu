@@ -1,10 +1,8 @@
 // Wanda 2:4 mask builder for the tile-hybrid sparse linear layer (sm_100a).
 //
 // Steps (each a kernel, all HBM-streaming):
-//   1. colsq_partial / colsq_final: s_j = sum_t x_tj^2 over calibration tokens
-//      in a fixed order (128-token chunks summed token by token, chunk sums
-//      added chunk by chunk), so s is bit-reproducible for any launch shape;
-//      n_j = sqrt(s_j) (IEEE round-to-nearest).
+//   1. column sums of squares of the calibration set: csrc/colsq_kernels.cu;
+//      here only n_j = sqrt(s_j) from caller-given sums.
 //   2. score_mask: per tile, Wanda scores |W_ij| * n_j (one fp64 multiply),
 //      top-2-of-4 per group (score descending, lower index on ties), the 4-bit
 //      code idx0 | idx1 << 2, and the tile's pruned-score loss (32-column words
@@ -25,99 +23,6 @@
 #include "patch_internal.h"
 
 namespace patchk {
-
-constexpr int kColsqChunk = 128;   // tokens per fixed-order chunk
-constexpr int kColsqThreads = 128;  // a block: 128 threads x 8 columns = 1024 columns
-constexpr int kColsqUnroll = 8;     // token rows in flight per thread
-constexpr int kFoldCols = 32;       // columns per fold block (one warp folds them)
-constexpr int kFoldRows = 64;       // chunk partials staged per fold step
-constexpr int kFoldThreads = 256;
-
-// One thread = 8 consecutive columns x one 128-token chunk, the chunk's tokens
-// in order.  Every token row is read with one 16-byte load per thread, so a
-// warp reads 512 contiguous bytes of each row; kColsqUnroll rows are in flight
-// before the first is used.  Per column the sum is the same chain of fp64
-// additions as a one-column loop: a = 0; a = a + x_t^2 for t in the chunk.
-__global__ void __launch_bounds__(kColsqThreads)
-colsq_partial_kernel(const uint16_t *__restrict__ X, int64_t T, int64_t K,
-                     double *__restrict__ partial) {
-    // grid.x: chunks (no limit that matters for T), grid.y: 1024-column blocks
-    const int64_t cg = static_cast<int64_t>(blockIdx.y) * kColsqThreads + threadIdx.x;
-    if (cg * 8 >= K) return;
-    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kColsqChunk;
-    const int64_t t1 = min(T, t0 + kColsqChunk);
-    const uint4 *src = reinterpret_cast<const uint4 *>(X + t0 * K) + cg;
-    const int64_t row16 = K / 8;  // 16-byte words per token row
-    double a[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) a[q] = 0.0;
-    auto add_row = [&](const uint4 v) {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const double lo = static_cast<double>(__uint_as_float(w[h] << 16));
-            const double hi = static_cast<double>(__uint_as_float(w[h] & 0xFFFF0000u));
-            a[2 * h] = __dadd_rn(a[2 * h], __dmul_rn(lo, lo));
-            a[2 * h + 1] = __dadd_rn(a[2 * h + 1], __dmul_rn(hi, hi));
-        }
-    };
-    int64_t t = t0;
-    for (; t + kColsqUnroll <= t1; t += kColsqUnroll) {
-        uint4 v[kColsqUnroll];
-#pragma unroll
-        for (int u = 0; u < kColsqUnroll; ++u) v[u] = __ldcs(src + u * row16);
-#pragma unroll
-        for (int u = 0; u < kColsqUnroll; ++u) add_row(v[u]);
-        src += kColsqUnroll * row16;
-    }
-    for (; t < t1; ++t) {
-        add_row(__ldcs(src));
-        src += row16;
-    }
-    double2 *dst = reinterpret_cast<double2 *>(partial + static_cast<int64_t>(blockIdx.x) * K + cg * 8);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_double2(a[2 * q], a[2 * q + 1]);
-}
-
-// s_j = chunk sums added in chunk order; n_j = sqrt(s_j).  A block owns 32
-// columns: all its warps stage kFoldRows chunk rows of them in shared memory
-// (one 256-byte row per warp load), then warp 0 adds them, lane j to column j,
-// in chunk order.  The next rows are loaded into registers before the fold.
-__global__ void __launch_bounds__(kFoldThreads)
-colsq_final_kernel(const double *__restrict__ partial, int64_t chunks, int64_t K,
-                   double *__restrict__ colsq_out, double *__restrict__ norm_out) {
-    constexpr int kWarps = kFoldThreads / 32;
-    constexpr int kPer = kFoldRows / kWarps;  // rows each warp stages per step
-    __shared__ double tile[kFoldRows][kFoldCols];
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t j = static_cast<int64_t>(blockIdx.x) * kFoldCols + lane;
-    const bool col_ok = j < K;
-    double reg[kPer];
-    auto load = [&](int64_t c0) {
-#pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            const int64_t c = c0 + warp + q * kWarps;
-            reg[q] = (col_ok && c < chunks) ? __ldcs(partial + c * K + j) : 0.0;
-        }
-    };
-    double s = 0.0;
-    load(0);
-    for (int64_t c0 = 0; c0 < chunks; c0 += kFoldRows) {
-#pragma unroll
-        for (int q = 0; q < kPer; ++q) tile[warp + q * kWarps][lane] = reg[q];
-        __syncthreads();
-        if (c0 + kFoldRows < chunks) load(c0 + kFoldRows);
-        if (warp == 0) {
-            const int n = static_cast<int>(min(static_cast<int64_t>(kFoldRows), chunks - c0));
-            for (int r = 0; r < n; ++r) s = __dadd_rn(s, tile[r][lane]);
-        }
-        __syncthreads();
-    }
-    if (warp == 0 && col_ok) {
-        if (colsq_out) colsq_out[j] = s;
-        norm_out[j] = __dsqrt_rn(s);
-    }
-}
 
 // Norms from caller-provided sums of squares (shared-input matrices).
 __global__ void norms_from_colsq_kernel(const double *__restrict__ colsq_in, int64_t K,
@@ -338,20 +243,6 @@ cudaError_t launch_select_maps_global(const double *loss_cat, const int64_t *n_t
 }
 
 // ------------------------------------------------------------------ launch
-cudaError_t launch_colsq(const void *Xcal, int64_t T, int64_t K, double *partial,
-                         double *colsq_out, double *norm_out, cudaStream_t stream) {
-    const int64_t chunks = (T + kColsqChunk - 1) / kColsqChunk;
-    const int64_t col_blocks = (K / 8 + kColsqThreads - 1) / kColsqThreads;
-    if (K % 8 != 0 || col_blocks > 65535 || chunks > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    dim3 grid(static_cast<unsigned>(chunks), static_cast<unsigned>(col_blocks));
-    colsq_partial_kernel<<<grid, kColsqThreads, 0, stream>>>(static_cast<const uint16_t *>(Xcal), T,
-                                                             K, partial);
-    colsq_final_kernel<<<static_cast<unsigned>((K + kFoldCols - 1) / kFoldCols), kFoldThreads, 0, stream>>>(
-        partial, chunks, K, colsq_out, norm_out);
-    note_launches(2);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_norms_from_colsq(const double *colsq_in, int64_t K, double *colsq_out,
                                     double *norm_out, cudaStream_t stream) {
     norms_from_colsq_kernel<<<static_cast<unsigned>((K + 255) / 256), 256, 0, stream>>>(

@@ -249,6 +249,46 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
     return from_cuda(e != cudaSuccess ? e : e2);
 }
 
+patch_status patch_colsq(const void *Xcal_bf16, int64_t T, int64_t K, double *colsq_out,
+                         void *stream_v) {
+    if (!Xcal_bf16 || !colsq_out || T < 1 || K < 64 || K % 64 != 0 || !aligned16(Xcal_bf16))
+        return PATCH_ERR_INVALID_ARG;
+    patch_status st = check_device(nullptr);
+    if (st != PATCH_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    const int64_t chunks = (T + 127) / 128;
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = patchk::device_pool(&pool);
+    if (e != cudaSuccess) return from_cuda(e);
+    double *partial = nullptr;
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&partial),
+                                sizeof(double) * static_cast<size_t>(chunks * K), pool, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    e = patchk::launch_colsq(Xcal_bf16, T, K, partial, colsq_out, nullptr, stream);
+    cudaError_t e2 = cudaFreeAsync(partial, stream);
+    return from_cuda(e != cudaSuccess ? e : e2);
+}
+
+patch_status patch_colsq_partials(const void *Xcal_bf16, int64_t T, int64_t K,
+                                  double *partials_out, void *stream_v) {
+    if (!Xcal_bf16 || !partials_out || T < 1 || K < 64 || K % 64 != 0 || !aligned16(Xcal_bf16) ||
+        !aligned16(partials_out))
+        return PATCH_ERR_INVALID_ARG;
+    patch_status st = check_device(nullptr);
+    if (st != PATCH_OK) return st;
+    return from_cuda(patchk::launch_colsq_partials(Xcal_bf16, T, K, partials_out,
+                                                   static_cast<cudaStream_t>(stream_v)));
+}
+
+patch_status patch_colsq_fold(const double *partials, int64_t chunks, int64_t K, double *colsq_out,
+                              void *stream_v) {
+    if (!partials || !colsq_out || chunks < 1 || K < 64 || K % 64 != 0) return PATCH_ERR_INVALID_ARG;
+    patch_status st = check_device(nullptr);
+    if (st != PATCH_OK) return st;
+    return from_cuda(patchk::launch_colsq_fold(partials, chunks, K, colsq_out, nullptr,
+                                               static_cast<cudaStream_t>(stream_v)));
+}
+
 // ------------------------------------------------------ allocation-free mask
 // Scratch of patch_score_mask_noalloc: a fixed array in device memory that
 // every device loading this library holds until the process exits.  Host code

@@ -9,6 +9,13 @@ namespace patchk {
 // Counts kernels enqueued by the library (exported as patch_launch_count).
 void note_launches(int n);
 
+// Column sums of squares: chunk partials [ceil(T/128), K] (chunk c = tokens
+// 128c .. 128c+127 added in token order from 0.0), the in-order fold of the
+// partials (colsq_out and / or norm_out = sqrt, either may be null), or both.
+cudaError_t launch_colsq_partials(const void *Xcal, int64_t T, int64_t K, double *partial,
+                                  cudaStream_t stream);
+cudaError_t launch_colsq_fold(const double *partial, int64_t chunks, int64_t K, double *colsq_out,
+                              double *norm_out, cudaStream_t stream);
 cudaError_t launch_colsq(const void *Xcal, int64_t T, int64_t K, double *partial,
                          double *colsq_out, double *norm_out, cudaStream_t stream);
 cudaError_t launch_norms_from_colsq(const double *colsq_in, int64_t K, double *colsq_out,

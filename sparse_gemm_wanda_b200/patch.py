@@ -24,7 +24,8 @@ EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
            "patch_get_status", "patch_packed_info", "patch_packed_export",
            "patch_status_string", "patch_score_mask_noalloc",
            "patch_score_mask_noalloc_capacity", "patch_launch_count",
-           "patch_select_maps_global", "patch_test_stall_first_kstep", "patch_pool_usage")
+           "patch_select_maps_global", "patch_test_stall_first_kstep", "patch_pool_usage",
+           "patch_colsq", "patch_colsq_partials", "patch_colsq_fold")
 
 
 class PatchLibraryError(RuntimeError):
@@ -76,6 +77,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.patch_select_maps_global.restype = ctypes.c_int
     lib.patch_launch_count.argtypes = []
     lib.patch_launch_count.restype = ctypes.c_uint64
+    lib.patch_colsq.argtypes = [vp, i64, i64, vp, vp]
+    lib.patch_colsq_partials.argtypes = [vp, i64, i64, vp, vp]
+    lib.patch_colsq_fold.argtypes = [vp, i64, i64, vp, vp]
+    for name in ("patch_colsq", "patch_colsq_partials", "patch_colsq_fold"):
+        getattr(lib, name).restype = ctypes.c_int
     lib.patch_test_stall_first_kstep.argtypes = [i32]
     lib.patch_test_stall_first_kstep.restype = None
     lib.patch_pool_usage.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
@@ -166,6 +172,44 @@ def patch_score_mask(W: torch.Tensor, Xcal: torch.Tensor | None = None, *, tile_
         _dptr(tmap), _dptr(colsq), _dptr(loss), _stream(stream))
     _check("patch_score_mask", code)
     return {"meta": meta, "map": tmap, "colsq": colsq, "loss": loss}
+
+
+COLSQ_CHUNK = 128  # calibration tokens per chunk partial of the column sums
+
+
+def patch_colsq(Xcal: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """colsq[j] = sum_t Xcal[t, j]^2 (fp64, the fixed chunked order) for Xcal[T,K] bf16."""
+    T, K = Xcal.shape
+    if out is None:
+        out = torch.empty((K,), dtype=torch.float64, device=Xcal.device)
+    _check("patch_colsq", load_library().patch_colsq(
+        _dptr(Xcal, torch.bfloat16, "Xcal"), T, K, _dptr(out, torch.float64, "colsq"), _stream(stream)))
+    return out
+
+
+def patch_colsq_partials(Xcal: torch.Tensor, out: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """Chunk partials [ceil(T/128), K] fp64 of the column sums of squares."""
+    T, K = Xcal.shape
+    if out is None:
+        out = torch.empty(((T + COLSQ_CHUNK - 1) // COLSQ_CHUNK, K), dtype=torch.float64,
+                          device=Xcal.device)
+    _check("patch_colsq_partials", load_library().patch_colsq_partials(
+        _dptr(Xcal, torch.bfloat16, "Xcal"), T, K, _dptr(out, torch.float64, "partials"),
+        _stream(stream)))
+    return out
+
+
+def patch_colsq_fold(partials: torch.Tensor, out: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Column sums of squares from chunk partials [chunks, K], added in chunk order."""
+    chunks, K = partials.shape
+    if out is None:
+        out = torch.empty((K,), dtype=torch.float64, device=partials.device)
+    _check("patch_colsq_fold", load_library().patch_colsq_fold(
+        _dptr(partials, torch.float64, "partials"), chunks, K, _dptr(out, torch.float64, "colsq"),
+        _stream(stream)))
+    return out
 
 
 def patch_score_mask_noalloc(W: torch.Tensor, Xcal: torch.Tensor | None = None, *,

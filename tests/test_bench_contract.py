@@ -23,7 +23,7 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference"
     assert d["value"] > 0 and d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
     assert d["warmup"] >= 3  # the contract's minimum, whatever was asked
-    assert d["config"]["workload"] == "llama7b-decode"
+    assert d["config"]["workload"] == "llama7b-block"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["e2e"]["value"] == d["value"]

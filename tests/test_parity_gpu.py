@@ -94,6 +94,28 @@ def test_mask_builder_bit_exact(P, oracle_mod, N, K, T, tn, tk, frac):
     assert np.array_equal(u32(r["map"]), ref["map"])
 
 
+@pytest.mark.parametrize("T,K,cut", [(300, 512, 128), (2048, 4096, 1024), (129, 256, 0),
+                                     (5000, 1024, 2560)])
+def test_colsq_calls_bit_exact(P, oracle_mod, T, K, cut):
+    # patch_colsq alone, and its halves over two pieces of the calibration set
+    # cut at a multiple of 128 tokens (partials stacked in token order, then
+    # folded): both bit-identical to the oracle's fixed-order sums
+    o = inputs.outlier_channels(K, T + K)
+    xc = inputs.activations(T, K, T + K, o, role=0)
+    ref = oracle_mod.colsq(bf16_bits(xc))
+    xd = xc.cuda()
+    s = P.patch_colsq(xd)
+    if cut:
+        parts = torch.cat([P.patch_colsq_partials(xd[:cut]), P.patch_colsq_partials(xd[cut:])])
+    else:
+        parts = P.patch_colsq_partials(xd)
+    assert parts.shape == ((T + 127) // 128, K)
+    s2 = P.patch_colsq_fold(parts)
+    torch.cuda.synchronize()
+    assert np.array_equal(s.cpu().numpy(), ref)
+    assert np.array_equal(s2.cpu().numpy(), ref)
+
+
 def test_mask_builder_given_map_and_colsq(P, oracle_mod):
     N, K, tn, tk = 512, 512, 128, 64
     w, xc, _ = make_problem(N, K, 200, 1, seed=7)
