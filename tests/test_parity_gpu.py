@@ -599,3 +599,46 @@ def test_gemm_two_sm_kernel_bounded_wait(P, oracle_mod):
     yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
     rel_rms_check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, True)
     pk.close()
+
+
+# ------------------------------------------------- multi-GPU split, one GPU
+
+@pytest.mark.parametrize("world,N,K,T,M,frac", [
+    (2, 1024, 1024, 1000, 200, 0.5),
+    (3, 4096, 4096, 2048, 16, 0.5),
+])
+def test_sharded_pieces_match_whole(P, oracle_mod, world, N, K, T, M, frac):
+    # The pieces the multi-GPU split gives each rank (sparse_gemm_wanda_b200/
+    # sharded.py), computed one after another on this GPU: the token pieces'
+    # chunk partials folded in order equal the whole set's sums; each row
+    # piece's codes and losses equal those rows of the whole matrix; the
+    # least-loss selection over the pieces' losses (rank order) gives each
+    # piece its slice of the whole map; each piece's GEMM matches the oracle.
+    from sparse_gemm_wanda_b200 import sharded
+    w, xc, x = make_problem(N, K, T, M, seed=900 + world)
+    ref = oracle_mask(oracle_mod, w, xc, 128, 128, frac=frac)
+    wd, xcd, xd = w.cuda(), xc.cuda(), x.cuda()
+    parts = [P.patch_colsq_partials(xcd[t0:t1]) for t0, t1 in sharded.token_ranges(T, world) if t1 > t0]
+    s = P.patch_colsq_fold(torch.cat(parts))
+    torch.cuda.synchronize()
+    assert np.array_equal(s.cpu().numpy(), ref["colsq"])
+    rows = sharded.row_ranges(N, world)
+    res = [P.patch_score_mask(wd[n0:n1], None, fraction=frac, colsq_in=s, want_loss=True)
+           for n0, n1 in rows]
+    maps = P.patch_select_maps_global([r["loss"] for r in res], frac)
+    torch.cuda.synchronize()
+    tiles_k = K // 128
+    full_bits = np.unpackbits(ref["map"].view(np.uint8), bitorder="little")
+    weff = oracle_mod.weff(bf16_bits(w), ref["meta"], ref["map"], 128, 128)
+    for (n0, n1), r, m in zip(rows, res, maps):
+        assert np.array_equal(u32(r["meta"]), ref["meta"][n0:n1])
+        nt = (n1 - n0) // 128 * tiles_k
+        g0 = n0 // 128 * tiles_k
+        mine = np.unpackbits(u32(m).view(np.uint8), bitorder="little")[:nt]
+        assert np.array_equal(mine, full_bits[g0:g0 + nt])
+        pk = P.patch_pack(wd[n0:n1], r["meta"], m)
+        y = P.patch_hybrid_gemm(pk, xd, out_fp32=True)
+        torch.cuda.synchronize()
+        assert P.patch_get_status(pk) == 0
+        rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), np.ascontiguousarray(weff[n0:n1])), True)
+        pk.close()
