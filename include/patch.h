@@ -303,6 +303,15 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
  */
 void patch_test_stall_first_kstep(int32_t on);
 
+/*
+ * Test hook: the prefill kernel every later patch_hybrid_gemm with M > 16
+ * uses.  0 = chosen by the library (the default), 1 = one band per CTA,
+ * 2 = two bands per CTA sharing each token tile, 3 = two-SM (CTA pair)
+ * kernel, used only where the band count is even (else as 0).  Results are
+ * the same up to fp32 rounding order; this only lets tests reach each kernel.
+ */
+void patch_test_prefill_kernel(int32_t which);
+
 /* Release a handle's device memory (stream-ordered on `stream`).  NULL ok. */
 void patch_free(patch_packed *Wp, void *stream);
 

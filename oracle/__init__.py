@@ -58,6 +58,12 @@ def _load():
             "oracle_unpack": [p, p, i64, i64, p],
             "oracle_gemm": [p, p, i64, i64, i64, p],
             "oracle_gemm_at": [p, p, i64, p, p, i64, p],
+            "oracle_select_4of8": [p, i64, i64, p],
+            "oracle_tile_loss_4of8": [p, p, i64, i64, i64, i64, p],
+            "oracle_weff_4of8": [p, p, p, i64, i64, i64, i64, p],
+            "oracle_pack_bytes_4of8": [p, i64, i64, i64, i64],
+            "oracle_pack_4of8": [p, p, p, i64, i64, i64, i64, p, p],
+            "oracle_unpack_4of8": [p, p, i64, i64, p],
         }
         for name, args in sig.items():
             fn = getattr(_lib, name)
@@ -65,6 +71,7 @@ def _load():
             fn.restype = None
         _lib.oracle_n_sparse.restype = i64
         _lib.oracle_pack_bytes.restype = i64
+        _lib.oracle_pack_bytes_4of8.restype = i64
     return _lib
 
 
@@ -213,6 +220,75 @@ def score_mask(w_bits, xcal_bits=None, tn: int = 128, tk: int = 128, fraction: f
     sc = wanda_scores(w_bits, s)
     meta = select_2of4(sc)
     loss = tile_loss(sc, meta, tn, tk)
+    if tile_map is None:
+        tile_map = select_map(loss, n_sparse(fraction, loss.shape[0]))
+    return {"colsq": s, "score": sc, "meta": meta, "loss": loss,
+            "map": np.ascontiguousarray(tile_map, dtype=np.uint32)}
+
+
+# ---------------------------------------------------------------- 4:8 pattern
+
+def select_4of8(score: np.ndarray) -> np.ndarray:
+    """Top-4-of-8 keep masks (bit q = position q kept), 4 groups per uint32 word."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    N, K = score.shape
+    meta = np.empty((N, K // 32), dtype=np.uint32)
+    _load().oracle_select_4of8(_ptr(score), N, K, _ptr(meta))
+    return meta
+
+
+def tile_loss_4of8(score: np.ndarray, meta: np.ndarray, tn: int, tk: int) -> np.ndarray:
+    """Pruned Wanda score per tile with the 4:8 kept set (same order as tile_loss)."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    N, K = score.shape
+    out = np.empty((N // tn) * (K // tk), dtype=np.float64)
+    _load().oracle_tile_loss_4of8(_ptr(score), _ptr(meta), N, K, tn, tk, _ptr(out))
+    return out
+
+
+def weff_4of8(w_bits, meta, tile_map, tn: int, tk: int) -> np.ndarray:
+    w = _u16(w_bits)
+    N, K = w.shape
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    tile_map = np.ascontiguousarray(tile_map, dtype=np.uint32)
+    out = np.empty_like(w)
+    _load().oracle_weff_4of8(_ptr(w), _ptr(meta), _ptr(tile_map), N, K, tn, tk, _ptr(out))
+    return out
+
+
+def pack_bytes_4of8(tile_map, N: int, K: int, tn: int, tk: int) -> int:
+    tile_map = np.ascontiguousarray(tile_map, dtype=np.uint32)
+    return int(_load().oracle_pack_bytes_4of8(_ptr(tile_map), N, K, tn, tk))
+
+
+def pack_4of8(w_bits, meta, tile_map, tn: int, tk: int):
+    """Packed bytes (uint8) and k-step table (uint64) of a 4:8 handle."""
+    w = _u16(w_bits)
+    N, K = w.shape
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    tile_map = np.ascontiguousarray(tile_map, dtype=np.uint32)
+    out = np.zeros(pack_bytes_4of8(tile_map, N, K, tn, tk), dtype=np.uint8)
+    table = np.zeros((N // 128) * (K // 64), dtype=np.uint64)
+    _load().oracle_pack_4of8(_ptr(w), _ptr(meta), _ptr(tile_map), N, K, tn, tk, _ptr(out), _ptr(table))
+    return out, table
+
+
+def unpack_4of8(packed: np.ndarray, table: np.ndarray, N: int, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    table = np.ascontiguousarray(table, dtype=np.uint64)
+    out = np.zeros((N, K), dtype=np.uint16)
+    _load().oracle_unpack_4of8(_ptr(packed), _ptr(table), N, K, _ptr(out))
+    return out
+
+
+def score_mask_4of8(w_bits, xcal_bits=None, tn: int = 128, tk: int = 128, fraction: float = 0.0,
+                    tile_map=None, colsq_in=None):
+    """Steps 1-5 with 4:8 groups: dict(colsq, score, meta, loss, map)."""
+    s = colsq(xcal_bits) if colsq_in is None else np.ascontiguousarray(colsq_in, dtype=np.float64)
+    sc = wanda_scores(w_bits, s)
+    meta = select_4of8(sc)
+    loss = tile_loss_4of8(sc, meta, tn, tk)
     if tile_map is None:
         tile_map = select_map(loss, n_sparse(fraction, loss.shape[0]))
     return {"colsq": s, "score": sc, "meta": meta, "loss": loss,

@@ -515,3 +515,188 @@ void oracle_gemm_at(const uint16_t *X, const uint16_t *Weff, int64_t K,
         y[q] = acc;
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* Another N:M pattern: 4 of every 8 (4:8)                             */
+/* ------------------------------------------------------------------ */
+
+/*
+ * PATCH's closing section ("PATCH: Learnable Tile-level Hybrid Sparsity for
+ * LLMs", section 5, significance) says the tile-level scheme does not depend
+ * on 2:4 and extends to other N:M patterns such as 4:8.  Here: inside a 4:8
+ * tile every group of 8 consecutive input channels keeps the 4 weights with
+ * the highest Wanda score, ties to the lower index (the same rule as 2:4,
+ * with groups of 8).  Everything else (tile loss, map, W_eff) is the 2:4
+ * definition with this kept set.
+ *
+ * Codes: group g of row i (columns 8g..8g+7) is an 8-bit mask with bit q set
+ * for a kept position q (exactly four bits), at bits 8*(g%4) of meta[i, g/4]
+ * (K/32 words per row, like the 2:4 codes).
+ */
+static unsigned select_group_4of8(const double *sc) {
+    /* four picks, each the largest remaining score, lowest index on ties */
+    unsigned mask = 0;
+    for (int pick = 0; pick < 4; ++pick) {
+        int best = -1;
+        for (int q = 0; q < 8; ++q) {
+            if ((mask >> q) & 1u) continue;
+            if (best < 0 || sc[q] > sc[best]) best = q;
+        }
+        mask |= 1u << best;
+    }
+    return mask;
+}
+
+void oracle_select_4of8(const double *score, int64_t N, int64_t K, uint32_t *meta) {
+    int64_t words = K / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i)
+        for (int64_t w = 0; w < words; ++w) {
+            uint32_t word = 0;
+            for (int g4 = 0; g4 < 4; ++g4)
+                word |= (uint32_t)select_group_4of8(score + i * K + w * 32 + g4 * 8) << (8 * g4);
+            meta[i * words + w] = word;
+        }
+}
+
+static int kept_4of8(const uint32_t *meta, int64_t K, int64_t i, int64_t j) {
+    uint32_t word = meta[i * (K / 32) + j / 32];
+    unsigned mask = (word >> (8 * ((j % 32) / 8))) & 0xFFu;
+    return (int)((mask >> (j % 8)) & 1u);
+}
+
+/* Tile loss with the 4:8 kept set, in the order of oracle_tile_loss. */
+void oracle_tile_loss_4of8(const double *score, const uint32_t *meta, int64_t N,
+                           int64_t K, int64_t tn, int64_t tk, double *loss) {
+    int64_t tiles_k = K / tk, tiles_n = N / tn;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < tiles_n * tiles_k; ++t) {
+        int64_t i0 = (t / tiles_k) * tn, j0 = (t % tiles_k) * tk;
+        double *rows = (double *)malloc(sizeof(double) * (size_t)tn);
+        for (int64_t r = 0; r < tn; ++r) {
+            double row = 0.0;
+            for (int64_t w0 = j0; w0 < j0 + tk; w0 += 32) {
+                double wsum = 0.0;
+                for (int64_t j = w0; j < w0 + 32; ++j)
+                    if (!kept_4of8(meta, K, i0 + r, j)) wsum = wsum + score[(i0 + r) * K + j];
+                row = row + wsum;
+            }
+            rows[r] = row;
+        }
+        for (int64_t n = tn; n > 1; n /= 2)
+            for (int64_t q = 0; q < n / 2; ++q) rows[q] = rows[2 * q] + rows[2 * q + 1];
+        loss[t] = rows[0];
+        free(rows);
+    }
+}
+
+/* W_eff with 4:8 tiles: kept entries of W there, +0 elsewhere. */
+void oracle_weff_4of8(const uint16_t *W, const uint32_t *meta, const uint32_t *map,
+                      int64_t N, int64_t K, int64_t tn, int64_t tk, uint16_t *weff) {
+    int64_t tiles_k = K / tk;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i)
+        for (int64_t j = 0; j < K; ++j) {
+            int64_t t = (i / tn) * tiles_k + j / tk;
+            uint16_t w = W[i * K + j];
+            if (tile_is_sparse(map, t) && !kept_4of8(meta, K, i, j)) w = 0;
+            weff[i * K + j] = w;
+        }
+}
+
+/*
+ * Packed layout of a 4:8 handle (this library's own format, stated in
+ * include/patch.h).  Bands of 128 rows and k-steps of 64 columns as for 2:4;
+ * a k-step is 4:8-compressed iff every map tile overlapping it is a 4:8
+ * tile, otherwise dense (the 2:4 handles' dense layout, holding W_eff).
+ *   - 4:8 k-step: 9216 bytes.  Kept value v (v < 32, column order, four per
+ *     group) of row r at byte r*64 + v*2; the keep mask of group g (g < 8)
+ *     of row r at byte 8192 + r*8 + g (bit q: position q kept).
+ *   - table[b*(K/64) + c] (uint64): bits 0..47 byte offset; bit 60 set for a
+ *     4:8 k-step.
+ */
+#define STEP48_BYTES 9216
+
+int64_t oracle_pack_bytes_4of8(const uint32_t *map, int64_t N, int64_t K, int64_t tn,
+                               int64_t tk) {
+    int64_t total = 0;
+    for (int64_t b = 0; b < N / BAND; ++b)
+        for (int64_t c = 0; c < K / KSTEP; ++c)
+            total += kstep_sparse(map, K, tn, tk, b, c) ? STEP48_BYTES : 16384;
+    return total;
+}
+
+void oracle_pack_4of8(const uint16_t *W, const uint32_t *meta, const uint32_t *map,
+                      int64_t N, int64_t K, int64_t tn, int64_t tk, uint8_t *out,
+                      uint64_t *table) {
+    int64_t steps = K / KSTEP, off = 0;
+    for (int64_t b = 0; b < N / BAND; ++b)
+        for (int64_t c = 0; c < steps; ++c) {
+            if (!kstep_sparse(map, K, tn, tk, b, c)) {
+                for (int64_t r = 0; r < BAND; ++r)
+                    for (int64_t k = 0; k < KSTEP; ++k) {
+                        int64_t i = b * BAND + r, j = c * KSTEP + k;
+                        int64_t t = (i / tn) * (K / tk) + j / tk;
+                        uint16_t w = W[i * K + j];
+                        if (tile_is_sparse(map, t) && !kept_4of8(meta, K, i, j)) w = 0;
+                        int64_t byte = (r / 8) * 1024 + (r % 8) * 128 +
+                                       (((k / 8) ^ (r % 8)) * 16) + (k % 8) * 2;
+                        memcpy(out + off + byte, &w, 2);
+                    }
+                table[b * steps + c] = (uint64_t)off;
+                off += 16384;
+            } else {
+                for (int64_t r = 0; r < BAND; ++r) {
+                    int64_t i = b * BAND + r;
+                    int v = 0;
+                    for (int64_t g = 0; g < KSTEP / 8; ++g) {
+                        unsigned mask = 0;
+                        for (int64_t q = 0; q < 8; ++q) {
+                            int64_t j = c * KSTEP + g * 8 + q;
+                            if (!kept_4of8(meta, K, i, j)) continue;
+                            mask |= 1u << q;
+                            memcpy(out + off + r * 64 + v * 2, &W[i * K + j], 2);
+                            ++v;
+                        }
+                        out[off + 8192 + r * 8 + g] = (uint8_t)mask;
+                    }
+                }
+                table[b * steps + c] = (uint64_t)off | (1ull << 60);
+                off += STEP48_BYTES;
+            }
+        }
+}
+
+/* Inverse of oracle_pack_4of8: W_eff from the packed bytes and table alone. */
+void oracle_unpack_4of8(const uint8_t *packed, const uint64_t *table, int64_t N, int64_t K,
+                        uint16_t *weff) {
+    int64_t steps = K / KSTEP;
+    for (int64_t b = 0; b < N / BAND; ++b)
+        for (int64_t c = 0; c < steps; ++c) {
+            uint64_t e = table[b * steps + c];
+            int64_t off = (int64_t)(e & ((1ull << 48) - 1));
+            for (int64_t r = 0; r < BAND; ++r) {
+                uint16_t *dst = weff + (b * BAND + r) * K + c * KSTEP;
+                if (!((e >> 60) & 1u)) {
+                    for (int64_t k = 0; k < KSTEP; ++k) {
+                        int64_t byte = (r / 8) * 1024 + (r % 8) * 128 +
+                                       (((k / 8) ^ (r % 8)) * 16) + (k % 8) * 2;
+                        memcpy(&dst[k], packed + off + byte, 2);
+                    }
+                    continue;
+                }
+                int v = 0;
+                for (int64_t g = 0; g < KSTEP / 8; ++g) {
+                    unsigned mask = packed[off + 8192 + r * 8 + g];
+                    for (int64_t q = 0; q < 8; ++q) {
+                        uint16_t w = 0;
+                        if ((mask >> q) & 1u) {
+                            memcpy(&w, packed + off + r * 64 + v * 2, 2);
+                            ++v;
+                        }
+                        dst[g * 8 + q] = w;
+                    }
+                }
+            }
+        }
+}

@@ -651,6 +651,13 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
 
 cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     if (g.M <= 16) return launch_decode_gemm(g, stream);  // split-K GEMV, csrc/decode_gemm.cu
+    // test hook: one prefill kernel for every M > 16 (parity of each kernel)
+    if (g.force_kernel == 1) return run<160, 3>(g, 1, stream);
+    if (g.force_kernel == 2 && g.K / kStep <= 448) return launch_pair_gemm(g, plan_pair_gemm(g.N, g.M, g.num_sms), stream);
+    if (g.force_kernel == 3 && g.duo_ok && g.K / kStep <= 448) {
+        const DuoPlan dp = plan_duo_gemm(g.N, g.M, g.num_sms, g.max_pair_bytes);
+        if (dp.bn > 0) return launch_duo_gemm(g, dp, stream);
+    }
     if (g.M <= 64) return run<64, 4>(g, 1, stream);   // 48 KB stages
     if (g.M <= 128) return run<128, 3>(g, 1, stream); // 64 KB stages
     // larger token counts: the band-pair kernel (two bands share each X tile)
@@ -663,7 +670,8 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     const int64_t waves1 = (items1 + g.num_sms - 1) / g.num_sms;
     const double t_one = static_cast<double>(waves1) * 576.0;
     if (g.duo_ok && g.K / kStep <= 448) {
-        // two-SM MMA when the matrix allows it and its estimate is lowest
+        // two-SM MMA (through the prefill table, whose band pairs agree in
+        // type) when its estimate is lowest
         const DuoPlan dp = plan_duo_gemm(g.N, g.M, g.num_sms, g.max_pair_bytes);
         if (dp.bn > 0 && dp.cost <= pp.cost && dp.cost <= t_one) return launch_duo_gemm(g, dp, stream);
     }

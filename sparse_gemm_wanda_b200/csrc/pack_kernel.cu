@@ -51,17 +51,24 @@ __device__ __forceinline__ uint32_t kept_pair(uint32_t a, uint32_t b, uint32_t c
 __global__ void __launch_bounds__(kPackThreads)
 pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
             const uint32_t *__restrict__ map, int64_t N, int64_t K, int tn, int tk,
-            const uint64_t *__restrict__ table, uint8_t *__restrict__ out,
-            uint32_t *__restrict__ done, uint32_t *__restrict__ ready) {
+            const uint64_t *__restrict__ table, const uint64_t *__restrict__ ptable,
+            uint8_t *__restrict__ out, uint32_t *__restrict__ done, uint32_t *__restrict__ ready) {
     const int64_t nsteps = K / kStep;
-    const int64_t b = blockIdx.x / nsteps, c = blockIdx.x % nsteps;
-    const uint64_t entry = table[blockIdx.x];
+    const int64_t steps_all = (N / kBand) * nsteps;
+    // blocks [0, steps_all): the packed k-steps; blocks [steps_all, 2 steps_all)
+    // (launched only with a prefill table): the dense side copies it points to
+    const bool side = static_cast<int64_t>(blockIdx.x) >= steps_all;
+    const int64_t idx = side ? blockIdx.x - steps_all : blockIdx.x;
+    const int64_t b = idx / nsteps, c = idx % nsteps;
+    const uint64_t entry = side ? ptable[idx] : table[idx];
     const int64_t off = static_cast<int64_t>(entry & kEntryOffsetMask);
     const int tid = threadIdx.x;
     const int64_t row0 = b * kBand, col0 = c * kStep;
     const int64_t words_k = K / 32;
 
-    if (!(entry & kEntrySparse)) {
+    if (side && !(entry & kEntrySide)) {
+        // the prefill table reuses the packed k-step here: nothing to write
+    } else if (!(entry & kEntrySparse)) {
         // dense: chunk u = r*8 + ((k/8) ^ (r%8)); W_eff, i.e. pruned entries of
         // a 2:4 tile (64-row tiles sharing a band with a dense tile) are zeroed
 #pragma unroll 4
@@ -177,11 +184,12 @@ __global__ void __launch_bounds__(kPlanThreads, 1)
 plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int log_tn, int log_tk, int cp,
                  int cpb, uint64_t *__restrict__ table, uint64_t *__restrict__ chunk_desc,
                  int64_t *__restrict__ pair_prefix, uint64_t *__restrict__ band_start,
+                 uint64_t *__restrict__ ptable, uint64_t *__restrict__ side_start,
                  PackPlan *__restrict__ plan) {
     __shared__ unsigned long long warp_sum[kPlanWarps];
     __shared__ uint32_t types[kPlanWarps][2][kPlanMaxWords];
-    __shared__ unsigned long long carry, n_sparse, n_meta;
-    __shared__ unsigned int duo_ok, max_pair;
+    __shared__ unsigned long long carry, n_sparse, n_meta, side_carry;
+    __shared__ unsigned int duo_ok, max_pair, pmax_pair;
     const int tid = threadIdx.x, lane = tid % 32, wid = tid / 32;
     const int Q = nsteps / 2, tiles_k = (nsteps * kStep) >> log_tk;
     uint32_t *mine = types[wid][0], *next = types[wid][1];
@@ -191,20 +199,16 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
         n_meta = 0;
         duo_ok = (bands % 2 == 0) ? 1u : 0u;
         max_pair = 0;
+        pmax_pair = 0;
+        side_carry = 0;
     }
     __syncthreads();
     // pass 1: k-pair sizes and their prefix within each band
     {
         unsigned long long ns = 0, nm = 0;
         unsigned int mp = 0;
-        bool agree = true;
         for (int b = wid; b < bands; b += kPlanWarps) {
             band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
-            if (b % 2 == 0 && b + 1 < bands) {
-                band_types(map, b + 1, nsteps, log_tn, log_tk, tiles_k, lane, next);
-                for (int w = lane; w < (nsteps + 31) / 32; w += 32)
-                    if (mine[w] != next[w]) agree = false;
-            }
             int64_t *pre = pair_prefix + static_cast<int64_t>(b) * (Q + 1);
             if (lane == 0) pre[0] = 0;
             unsigned long long run = 0;
@@ -237,12 +241,10 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
             nm += __shfl_xor_sync(0xFFFFFFFFu, nm, o);
             mp = max(mp, __shfl_xor_sync(0xFFFFFFFFu, mp, o));
         }
-        const bool all_agree = __all_sync(0xFFFFFFFFu, agree);
         if (lane == 0) {
             atomicAdd(&n_sparse, ns);
             atomicAdd(&n_meta, nm);
             atomicMax(&max_pair, mp);
-            if (!all_agree) atomicAnd(&duo_ok, 0u);
         }
     }
     __syncthreads();
@@ -318,6 +320,104 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
         __syncwarp();
     }
     __syncthreads();
+    // pass 4: the prefill table.  The two-SM prefill kernel runs bands 2p and
+    // 2p+1 through one M = 256 instruction, which must be of one kind.  Where
+    // the pair's k-pair types differ, each band of it holding a 2:4 k-step
+    // gets a dense copy of that k-pair (W_eff, 32 KB) in a side region after
+    // the packed bytes; elsewhere the prefill table repeats the packed entry.
+    // 4a: densified k-pairs per band (counted into side_start)
+    for (int pb = wid; 2 * pb < bands; pb += kPlanWarps) {
+        const int b = 2 * pb;
+        const bool paired = b + 1 < bands;
+        band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
+        if (paired) band_types(map, b + 1, nsteps, log_tn, log_tk, tiles_k, lane, next);
+        unsigned int n0 = 0, n1 = 0, mp = 0;
+        for (int q0 = 0; q0 < Q; q0 += 32) {
+            const int q = q0 + lane;
+            bool d0 = false, d1 = false;
+            if (q < Q) {
+                const bool s0 = bit_of(mine, 2 * q), s1 = bit_of(mine, 2 * q + 1);
+                const bool t0 = paired && bit_of(next, 2 * q), t1 = paired && bit_of(next, 2 * q + 1);
+                const bool mis = paired && (s0 != t0 || s1 != t1);
+                d0 = mis && (s0 || s1);
+                d1 = mis && (t0 || t1);
+                mp = max(mp, d0 || d1 ? static_cast<unsigned int>(kSidePairBytes)
+                                      : max(kpair_bytes(s0, s1), paired ? kpair_bytes(t0, t1) : 0u));
+            }
+            n0 += __popc(__ballot_sync(0xFFFFFFFFu, d0));
+            n1 += __popc(__ballot_sync(0xFFFFFFFFu, d1));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mp = max(mp, __shfl_xor_sync(0xFFFFFFFFu, mp, o));
+        if (lane == 0) {
+            side_start[b] = n0;
+            if (paired) side_start[b + 1] = n1;
+            atomicMax(&pmax_pair, mp);
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    // 4b: side offsets, an exclusive scan of 32 KB per densified k-pair
+    for (int base = 0; base < bands; base += kPlanThreads) {
+        const int b = base + tid;
+        const unsigned long long bytes = b < bands ? side_start[b] * static_cast<unsigned long long>(kSidePairBytes) : 0ull;
+        unsigned long long incl = bytes;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) warp_sum[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            unsigned long long w = warp_sum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long v = __shfl_up_sync(0xFFFFFFFFu, w, o);
+                if (lane >= o) w += v;
+            }
+            warp_sum[lane] = w;
+        }
+        __syncthreads();
+        if (b < bands) side_start[b] = carry + side_carry + (wid > 0 ? warp_sum[wid - 1] : 0ull) + (incl - bytes);
+        __syncthreads();
+        if (tid == 0) side_carry += warp_sum[kPlanWarps - 1];
+        __syncthreads();
+    }
+    // 4c: the entries; densified k-pairs are numbered in order within a band
+    for (int b = wid; b < bands; b += kPlanWarps) {
+        const int partner = b ^ 1;
+        const bool paired = partner < bands;
+        band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
+        if (paired) band_types(map, partner, nsteps, log_tn, log_tk, tiles_k, lane, next);
+        const uint64_t *row = table + static_cast<int64_t>(b) * nsteps;
+        uint64_t *prow = ptable + static_cast<int64_t>(b) * nsteps;
+        unsigned int run = 0;
+        for (int q0 = 0; q0 < Q; q0 += 32) {
+            const int q = q0 + lane;
+            bool d = false;
+            if (q < Q) {
+                const bool s0 = bit_of(mine, 2 * q), s1 = bit_of(mine, 2 * q + 1);
+                const bool t0 = paired && bit_of(next, 2 * q), t1 = paired && bit_of(next, 2 * q + 1);
+                d = paired && (s0 != t0 || s1 != t1) && (s0 || s1);
+            }
+            const uint32_t ball = __ballot_sync(0xFFFFFFFFu, d);
+            if (q < Q) {
+                if (d) {
+                    const unsigned int k = run + __popc(ball & ((1u << lane) - 1u));
+                    const uint64_t off = side_start[b] + static_cast<uint64_t>(k) * kSidePairBytes;
+                    prow[2 * q] = kEntrySide | off;
+                    prow[2 * q + 1] = kEntrySide | (off + kDenseStepBytes);
+                } else {
+                    prow[2 * q] = row[2 * q];
+                    prow[2 * q + 1] = row[2 * q + 1];
+                }
+            }
+            run += __popc(ball);
+        }
+        __syncwarp();
+    }
+    __syncthreads();
     // the first chunk descriptors, written above by other warps of the block
     const int64_t nchunks = static_cast<int64_t>(bands) * cpb;
     for (int64_t j = tid; j < 2 * kDecMaxCtas; j += kPlanThreads)
@@ -328,28 +428,32 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
         plan->meta_blocks = n_meta;
         plan->duo_ok = duo_ok;
         plan->max_pair_bytes = max_pair;
+        plan->side_bytes = side_carry;
+        plan->pair_max_bytes = pmax_pair;
     }
 }
 
 cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, int tk, int cp,
                              int cpb, uint64_t *table, uint64_t *chunk_desc, int64_t *pair_prefix,
-                             uint64_t *band_start, PackPlan *plan, cudaStream_t stream) {
+                             uint64_t *band_start, uint64_t *ptable, uint64_t *side_start,
+                             PackPlan *plan, cudaStream_t stream) {
     const int64_t nsteps = K / kStep;
     if (nsteps > 32 * kPlanMaxWords || (N / kBand) > (int64_t(1) << 24)) return cudaErrorInvalidValue;
     const int log_tn = tn == 64 ? 6 : 7, log_tk = tk == 64 ? 6 : 7;
     plan_pack_kernel<<<1, kPlanThreads, 0, stream>>>(map, static_cast<int>(N / kBand), static_cast<int>(nsteps),
                                                      log_tn, log_tk, cp, cpb, table, chunk_desc,
-                                                     pair_prefix, band_start, plan);
+                                                     pair_prefix, band_start, ptable, side_start, plan);
     note_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
-                        int64_t K, int tn, int tk, const uint64_t *table, uint8_t *out,
-                        uint32_t *done, uint32_t *ready, cudaStream_t stream) {
-    const int64_t blocks = (N / kBand) * (K / kStep);
+                        int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
+                        uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream) {
+    const int64_t blocks = (N / kBand) * (K / kStep) * (ptable ? 2 : 1);
+    if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
     pack_kernel<<<static_cast<unsigned>(blocks), kPackThreads, 0, stream>>>(
-        static_cast<const uint16_t *>(W), meta, map, N, K, tn, tk, table, out, done, ready);
+        static_cast<const uint16_t *>(W), meta, map, N, K, tn, tk, table, ptable, out, done, ready);
     note_launches(1);
     return cudaGetLastError();
 }

@@ -22,9 +22,11 @@ struct patch_packed {
     int device;
     uint8_t *base;             // pool allocation: table, descriptors, prefix, plan, workspace, status
     patch_shape shp;
-    uint8_t *packed;           // packed k-steps (a pool allocation of its own, exact size)
-    size_t packed_bytes;
+    uint8_t *packed;           // packed k-steps, then the side copies (a pool allocation of its own, exact size)
+    size_t packed_bytes;       // the packed k-steps (the normative format)
+    size_t side_bytes;         // dense k-pair copies after them, for the prefill table
     uint64_t *table;           // (N/128) * (K/64) entries
+    uint64_t *ptable;          // prefill table: (N/128) * (K/64) entries
     int64_t sparse_ksteps;
     int64_t meta_blocks;
     float *workspace;          // decode partials (one slot per chunk); reused by stream-K
@@ -32,8 +34,8 @@ struct patch_packed {
     uint64_t *chunk_desc;      // device: decode chunk descriptors
     std::vector<uint64_t> chunk_desc_host;
     int dec_cp, dec_cpb, dec_nchunks;
-    int duo_ok;                // bands 2p, 2p+1 agree in type at every k-step
-    int max_pair_bytes;        // largest packed k-pair
+    int duo_ok;                // even band count: the prefill table pairs bands 2p, 2p+1
+    int max_pair_bytes;        // largest k-pair the prefill table points to
     uint32_t *status;          // device: status word, pack counter, ready flag
     int num_sms;
     cudaMemPool_t pool;
@@ -123,6 +125,8 @@ cudaError_t read_plan(const patchk::PackPlan *src, patchk::PackPlan *dst, const 
 // Failure-detection test hook (see patch_test_stall_first_kstep): read from
 // the environment once, when the library is loaded; changed only by the
 // exported setter.
+std::atomic<int> g_test_kernel{0};  // patch_test_prefill_kernel
+
 std::atomic<int> g_test_stall{[] {
     const char *v = getenv("PATCH_B200_TEST_STALL");
     return (v && v[0] == '1') ? 1 : 0;
@@ -469,6 +473,10 @@ uint64_t patch_launch_count(void) { return patchk::g_launches.load(std::memory_o
 
 void patch_test_stall_first_kstep(int32_t on) { g_test_stall.store(on ? 1 : 0, std::memory_order_relaxed); }
 
+void patch_test_prefill_kernel(int32_t which) {
+    g_test_kernel.store((which >= 0 && which <= 3) ? which : 0, std::memory_order_relaxed);
+}
+
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
                         patch_shape shp, patch_packed **out,
                         size_t *packed_bytes, void *stream_v) {
@@ -504,7 +512,9 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     const size_t off_chunks = off_table + sizeof(uint64_t) * static_cast<size_t>(bands * nsteps);
     const size_t off_prefix = round_up(off_chunks + sizeof(uint64_t) * static_cast<size_t>(h->dec_nchunks), 256);
     const size_t off_bstart = round_up(off_prefix + sizeof(int64_t) * static_cast<size_t>(bands * (Q + 1)), 256);
-    const size_t off_plan = round_up(off_bstart + sizeof(uint64_t) * static_cast<size_t>(bands), 256);
+    const size_t off_ptable = round_up(off_bstart + sizeof(uint64_t) * static_cast<size_t>(bands), 256);
+    const size_t off_sstart = round_up(off_ptable + sizeof(uint64_t) * static_cast<size_t>(bands * nsteps), 256);
+    const size_t off_plan = round_up(off_sstart + sizeof(uint64_t) * static_cast<size_t>(bands), 256);
     const size_t off_ws = round_up(off_plan + sizeof(patchk::PackPlan), 256);
     const size_t off_status = round_up(off_ws + h->workspace_bytes, 256);
     const size_t status_bytes = 256;
@@ -519,6 +529,7 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     h->table = reinterpret_cast<uint64_t *>(h->base + off_table);
     h->chunk_desc = reinterpret_cast<uint64_t *>(h->base + off_chunks);
     h->pair_prefix_dev = reinterpret_cast<int64_t *>(h->base + off_prefix);
+    h->ptable = reinterpret_cast<uint64_t *>(h->base + off_ptable);
     patchk::PackPlan *plan_dev = reinterpret_cast<patchk::PackPlan *>(h->base + off_plan);
     h->workspace = reinterpret_cast<float *>(h->base + off_ws);
     // status word | pack completion counter | ready flag | decode chunk counter
@@ -527,7 +538,8 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     if (e == cudaSuccess)
         e = patchk::launch_plan_pack(map, N, K, static_cast<int>(tn), static_cast<int>(tk), h->dec_cp,
                                      h->dec_cpb, h->table, h->chunk_desc, h->pair_prefix_dev,
-                                     reinterpret_cast<uint64_t *>(h->base + off_bstart), plan_dev, stream);
+                                     reinterpret_cast<uint64_t *>(h->base + off_bstart), h->ptable,
+                                     reinterpret_cast<uint64_t *>(h->base + off_sstart), plan_dev, stream);
     patchk::PackPlan plan;
     h->pair_prefix.assign(static_cast<size_t>(bands * (Q + 1)), 0);
     if (e == cudaSuccess) e = read_plan(plan_dev, &plan, h->pair_prefix_dev, &h->pair_prefix, stream);
@@ -536,21 +548,24 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
         return from_cuda(e);
     }
     h->packed_bytes = static_cast<size_t>(plan.packed_bytes);
-    if (plan.packed_bytes >= (1ull << 40)) {  // chunk descriptors hold 40-bit offsets
+    h->side_bytes = static_cast<size_t>(plan.side_bytes);
+    if (plan.packed_bytes >= (1ull << 40) || plan.packed_bytes + plan.side_bytes >= (1ull << 47)) {
+        // chunk descriptors hold 40-bit offsets, table entries 48-bit ones
         patch_free(h, stream_v);
         return PATCH_ERR_UNSUPPORTED;
     }
     h->sparse_ksteps = static_cast<int64_t>(plan.sparse_ksteps);
     h->meta_blocks = static_cast<int64_t>(plan.meta_blocks);
     h->duo_ok = plan.duo_ok ? 1 : 0;
-    h->max_pair_bytes = static_cast<int>(plan.max_pair_bytes);
+    h->max_pair_bytes = static_cast<int>(plan.pair_max_bytes);
     h->chunk_desc_host.assign(plan.first_desc,
                               plan.first_desc + std::min<int64_t>(h->dec_nchunks, 2 * patchk::kDecMaxCtas));
     e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->packed),
-                                std::max<size_t>(h->packed_bytes, 16), h->pool, stream);
+                                std::max<size_t>(h->packed_bytes + h->side_bytes, 16), h->pool, stream);
     if (e == cudaSuccess)
         e = patchk::launch_pack(W_bf16, meta, map, N, K, static_cast<int>(tn), static_cast<int>(tk),
-                                h->table, h->packed, h->status + 1, h->status + 2, stream);
+                                h->table, h->side_bytes ? h->ptable : nullptr, h->packed,
+                                h->status + 1, h->status + 2, stream);
     if (e != cudaSuccess) {
         patch_free(h, stream_v);
         return from_cuda(e);
@@ -588,7 +603,8 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.dec_cp = Wp->dec_cp;
     g.dec_cpb = Wp->dec_cpb;
     g.dec_nchunks = Wp->dec_nchunks;
-    g.packed_rows = Wp->packed_bytes / 128;
+    g.packed_rows = (Wp->packed_bytes + Wp->side_bytes) / 128;
+    g.ptable = Wp->ptable;
     g.duo_ok = Wp->duo_ok;
     g.max_pair_bytes = Wp->max_pair_bytes;
     g.num_sms = Wp->num_sms;
@@ -596,6 +612,7 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     // read back once by patch_pack: nothing here waits for the device
     g.pair_prefix = Wp->pair_prefix.empty() ? nullptr : Wp->pair_prefix.data();
     g.stall_first_kstep = g_test_stall.load(std::memory_order_relaxed);
+    g.force_kernel = g_test_kernel.load(std::memory_order_relaxed);
     return from_cuda(patchk::launch_hybrid_gemm(g, static_cast<cudaStream_t>(stream_v)));
 }
 

@@ -18,6 +18,10 @@ constexpr int kMetaBlockBytes = kBand * 16;              // 2048 (one 16-B line 
 constexpr uint64_t kEntryOffsetMask = (1ull << 48) - 1;
 constexpr uint64_t kEntrySparse = 1ull << 62;
 constexpr uint64_t kEntryMeta = 1ull << 63;
+// Prefill table only: the k-step is a dense copy of W_eff in the side region
+// that follows the packed bytes (see plan_pack_kernel).
+constexpr uint64_t kEntrySide = 1ull << 61;
+constexpr int kSidePairBytes = 2 * kDenseStepBytes;
 
 // Bit of the device status word set when a bounded wait runs out.
 constexpr uint32_t kStatusTimeout = 1u;

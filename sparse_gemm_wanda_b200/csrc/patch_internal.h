@@ -40,9 +40,11 @@ cudaError_t launch_select_maps_global(const double *loss_cat, const int64_t *n_t
 
 // `done` (a zeroed counter) and `ready` (zeroed) live in the handle: the last
 // block to finish publishes ready = 1 with release semantics.
+// `ptable` (may be null) adds the dense copies of the prefill table's side
+// entries, written after the packed bytes.
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
-                        int64_t K, int tn, int tk, const uint64_t *table, uint8_t *out,
-                        uint32_t *done, uint32_t *ready, cudaStream_t stream);
+                        int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
+                        uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream);
 
 // Decode (M <= 16) GEMV: CTAs whose first chunk travels in the kernel
 // parameters, at most.
@@ -54,16 +56,22 @@ struct PackPlan {
     uint64_t packed_bytes;
     uint64_t sparse_ksteps;
     uint64_t meta_blocks;
-    uint32_t duo_ok;          // bands 2p, 2p+1 agree in type at every k-step
+    uint32_t duo_ok;          // the band count is even: the prefill table pairs bands 2p, 2p+1
     uint32_t max_pair_bytes;  // largest packed k-pair
+    uint64_t side_bytes;      // dense copies after the packed bytes (prefill table)
+    uint32_t pair_max_bytes;  // largest k-pair the prefill table points to
+    uint32_t pad_;
     uint64_t first_desc[2 * kDecMaxCtas];  // decode chunk descriptors 0 .. 2*kDecMaxCtas-1
 };
 // Writes the k-step table [bands][nsteps], the decode chunk descriptors
 // [bands][cpb], the per-band cumulative k-pair bytes [bands][nsteps/2 + 1],
-// the first byte of each band (scratch [bands]) and the plan summary; one block.
+// the first byte of each band (scratch [bands]), the prefill table
+// [bands][nsteps] with the side-region offsets of its dense copies (scratch
+// side_start [bands]) and the plan summary; one block.
 cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, int tk, int cp,
                              int cpb, uint64_t *table, uint64_t *chunk_desc, int64_t *pair_prefix,
-                             uint64_t *band_start, PackPlan *plan, cudaStream_t stream);
+                             uint64_t *band_start, uint64_t *ptable, uint64_t *side_start,
+                             PackPlan *plan, cudaStream_t stream);
 
 struct GemmLaunch {
     const uint8_t *packed;
@@ -83,11 +91,13 @@ struct GemmLaunch {
     const uint64_t *chunk_desc_host;  // host copy
     int dec_cp, dec_cpb, dec_nchunks;
     uint32_t *counter;                // device: chunks claimed, zero between calls
-    uint64_t packed_rows;             // packed bytes / 128
-    int duo_ok;                       // bands 2p, 2p+1 agree in type at every k-step
-    int max_pair_bytes;               // largest packed k-pair of the matrix
+    uint64_t packed_rows;             // (packed bytes + side copies) / 128
+    const uint64_t *ptable;           // prefill table: bands 2p, 2p+1 agree in type at every k-step
+    int duo_ok;                       // the prefill table pairs every band (even band count)
+    int max_pair_bytes;               // largest k-pair the prefill table points to
     int num_sms;
     int stall_first_kstep;   // failure-detection test hook (see patch_hybrid_gemm)
+    int force_kernel;        // test hook: 0 auto, 1 one-band, 2 band-pair, 3 two-SM (M > 16)
     const int64_t *pair_prefix;  // host: per band, cumulative packed bytes of its k-pairs
 };
 

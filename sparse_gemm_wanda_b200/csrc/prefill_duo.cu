@@ -584,7 +584,7 @@ cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream
         !encode_rows(enc, &maps.a_ss, g.packed, rows, (kMetaBlockBytes + 2 * kSparseStepBytes) / 2048))
         return cudaErrorInvalidValue;
     DuoParams p;
-    p.table = g.table;
+    p.table = g.ptable;  // the prefill table: the bands of every pair agree in type
     p.N = g.N;
     p.K = g.K;
     p.M = g.M;

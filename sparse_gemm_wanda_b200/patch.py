@@ -25,7 +25,7 @@ EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
            "patch_status_string", "patch_score_mask_noalloc",
            "patch_score_mask_noalloc_capacity", "patch_launch_count",
            "patch_select_maps_global", "patch_test_stall_first_kstep", "patch_pool_usage",
-           "patch_colsq", "patch_colsq_partials", "patch_colsq_fold")
+           "patch_colsq", "patch_colsq_partials", "patch_colsq_fold", "patch_test_prefill_kernel")
 
 
 class PatchLibraryError(RuntimeError):
@@ -82,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.patch_colsq_fold.argtypes = [vp, i64, i64, vp, vp]
     for name in ("patch_colsq", "patch_colsq_partials", "patch_colsq_fold"):
         getattr(lib, name).restype = ctypes.c_int
+    lib.patch_test_prefill_kernel.argtypes = [i32]
+    lib.patch_test_prefill_kernel.restype = None
     lib.patch_test_stall_first_kstep.argtypes = [i32]
     lib.patch_test_stall_first_kstep.restype = None
     lib.patch_pool_usage.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
@@ -113,6 +115,11 @@ def test_stall_first_kstep(on: bool) -> None:
     """Failure-detection hook: while on, the first CTA of every GEMM never
     receives its first k-step, so its bounded wait runs out (tests only)."""
     load_library().patch_test_stall_first_kstep(1 if on else 0)
+
+
+def test_prefill_kernel(which: int) -> None:
+    """Test hook: 0 auto, 1 one-band, 2 band-pair, 3 two-SM prefill kernel (M > 16)."""
+    load_library().patch_test_prefill_kernel(int(which))
 
 
 def pool_usage(reset_high: bool = False) -> tuple:

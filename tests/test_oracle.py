@@ -476,3 +476,149 @@ def test_pack_bytes_closed_form(oracle_mod, frac):
     sparse_steps = int(((table >> np.uint64(62)) & np.uint64(1)).sum())
     e_blocks = int((table >> np.uint64(63)).sum())
     assert sparse_steps == 2 * ns and e_blocks == ns
+
+
+# ----------------------------------------------------------------------------
+# 4:8 groups ("PATCH: Learnable Tile-level Hybrid Sparsity for LLMs", section 5:
+# the tile scheme extends to other N:M patterns such as 4:8)
+# ----------------------------------------------------------------------------
+
+def masks_of(meta):
+    """Unpack uint32 meta words into per-group 8-bit keep masks [N, K/8]."""
+    meta = np.asarray(meta, dtype=np.uint32)
+    shifts = (np.arange(4, dtype=np.uint32) * 8)
+    m = (meta[..., None] >> shifts) & 0xFF
+    return m.reshape(meta.shape[0], -1)
+
+
+def brute_4of8(group):
+    """Among the 70 keep sets of size 4, the largest exact (rational) score sum;
+    ties between sets go to the lexicographically smallest sorted index tuple.
+    Returns the 8-bit mask."""
+    best, best_key = None, None
+    for subset in combinations(range(8), 4):
+        s = sum(Fraction(float(group[q])) for q in subset)
+        key = (-s, subset)
+        if best_key is None or key < best_key:
+            best_key, best = key, subset
+    return sum(1 << q for q in best)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_select_4of8_equals_bruteforce_with_ties(oracle_mod, seed):
+    g = np.random.default_rng(seed)
+    # few distinct values: ties inside most groups
+    score = g.choice(np.array([0.0, 0.25, 0.5, 1.0, 3.0]), size=(16, 64))
+    masks = masks_of(oracle_mod.select_4of8(score))
+    for i in range(score.shape[0]):
+        for gi in range(score.shape[1] // 8):
+            assert masks[i, gi] == brute_4of8(score[i, 8 * gi:8 * gi + 8]), (i, gi)
+
+
+def test_select_4of8_equals_bruteforce_random(oracle_mod):
+    g = np.random.default_rng(5)
+    score = np.abs(g.standard_normal((8, 128))) * np.exp(g.standard_normal((1, 128)))
+    masks = masks_of(oracle_mod.select_4of8(score))
+    for i in range(score.shape[0]):
+        for gi in range(score.shape[1] // 8):
+            assert masks[i, gi] == brute_4of8(score[i, 8 * gi:8 * gi + 8])
+
+
+@pytest.mark.parametrize("group,mask", [
+    ([1.0] * 8, 0x0F),                                    # all equal: the four lowest indices
+    ([8, 7, 6, 5, 4, 3, 2, 1], 0x0F),
+    ([1, 2, 3, 4, 5, 6, 7, 8], 0xF0),
+    ([0, 5, 0, 5, 0, 5, 0, 5], 0xAA),
+    ([2, 2, 9, 2, 2, 2, 9, 2], 0x47),                      # 9s, then the two lowest 2s
+])
+def test_select_4of8_special_cases(oracle_mod, group, mask):
+    score = np.zeros((1, 32))
+    score[0, :8] = group
+    assert masks_of(oracle_mod.select_4of8(score))[0, 0] == mask
+
+
+def test_select_4of8_dominance_and_count(oracle_mod):
+    g = np.random.default_rng(9)
+    score = np.round(np.abs(g.standard_normal((32, 256))) * 4) / 4
+    masks = masks_of(oracle_mod.select_4of8(score))
+    for i in range(32):
+        for gi in range(32):
+            m = int(masks[i, gi])
+            assert bin(m).count("1") == 4
+            grp = score[i, 8 * gi:8 * gi + 8]
+            kept = [q for q in range(8) if m >> q & 1]
+            drop = [q for q in range(8) if not m >> q & 1]
+            for a in kept:
+                for b in drop:
+                    assert grp[a] > grp[b] or (grp[a] == grp[b] and a < b)
+
+
+def test_tile_loss_4of8_plus_kept_is_total(oracle_mod):
+    # dyadic scores: every sum is exact, so pruned + kept = all, tile by tile
+    g = np.random.default_rng(4)
+    N, K, tn, tk = 128, 256, 64, 128
+    score = g.integers(0, 64, size=(N, K)).astype(np.float64) / 8
+    meta = oracle_mod.select_4of8(score)
+    loss = oracle_mod.tile_loss_4of8(score, meta, tn, tk)
+    bits = np.unpackbits(masks_of(meta).astype(np.uint8)[..., None], axis=-1, bitorder="little")
+    keep = bits.reshape(N, K).astype(bool)
+    for t in range(loss.shape[0]):
+        i0, j0 = (t // (K // tk)) * tn, (t % (K // tk)) * tk
+        sub, kp = score[i0:i0 + tn, j0:j0 + tk], keep[i0:i0 + tn, j0:j0 + tk]
+        assert loss[t] == sub[~kp].sum()
+        assert loss[t] + sub[kp].sum() == sub.sum()
+
+
+def test_weff_4of8_all_sparse_is_masked_gemm(oracle_mod):
+    g = torch.Generator().manual_seed(11)
+    N, K, M = 256, 128, 5
+    w = (torch.randn(N, K, generator=g) * 0.1).to(torch.bfloat16)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    wb, xb = bf16_bits(w), bf16_bits(x)
+    score = np.abs(oracle_mod.bf16_bits_to_f64(wb)) * np.exp(np.linspace(0, 1, K))
+    meta = oracle_mod.select_4of8(score)
+    nt = (N // 64) * (K // 64)
+    allmap = np.full((nt + 31) // 32, 0xFFFFFFFF, dtype=np.uint32)
+    weff = oracle_mod.weff_4of8(wb, meta, allmap, 64, 64)
+    wf = oracle_mod.bf16_bits_to_f64(wb)
+    # the masks from brute force, not from the oracle's own codes
+    keep = np.zeros((N, K), dtype=bool)
+    for i in range(N):
+        for gi in range(K // 8):
+            m = brute_4of8(score[i, 8 * gi:8 * gi + 8])
+            for q in range(8):
+                keep[i, 8 * gi + q] = bool(m >> q & 1)
+    assert np.array_equal(oracle_mod.bf16_bits_to_f64(weff), np.where(keep, wf, 0.0))
+    y = oracle_mod.gemm(xb, weff)
+    yref = oracle_mod.bf16_bits_to_f64(xb) @ np.where(keep, wf, 0.0).T
+    assert np.allclose(y, yref, rtol=1e-12, atol=1e-12)
+    # achieved sparsity of an all-4:8 map is exactly half (no zero weights drawn)
+    assert np.mean(weff == 0) == 0.5
+
+
+@pytest.mark.parametrize("tn,tk", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("frac", [0.0, 0.4, 1.0])
+def test_pack_4of8_round_trip_and_bytes(oracle_mod, tn, tk, frac):
+    from sparse_gemm_wanda_b200 import inputs
+    N, K = 256, 384
+    w = inputs.weight(N, K, 3)
+    wb = bf16_bits(w)
+    score = np.abs(oracle_mod.bf16_bits_to_f64(wb))
+    meta = oracle_mod.select_4of8(score)
+    nt = (N // tn) * (K // tk)
+    tmap = inputs.random_map(nt, int(frac * nt), 5).numpy().view(np.uint32)
+    packed, table = oracle_mod.pack_4of8(wb, meta, tmap, tn, tk)
+    assert np.array_equal(oracle_mod.unpack_4of8(packed, table, N, K),
+                          oracle_mod.weff_4of8(wb, meta, tmap, tn, tk))
+    # closed form: a k-step is 4:8 iff every tile it overlaps is; 16384 or 9216 bytes
+    sparse_steps = 0
+    for b in range(N // 128):
+        for c in range(K // 64):
+            rows = range((128 * b) // tn, (128 * b + 127) // tn + 1)
+            cols = range((64 * c) // tk, (64 * c + 63) // tk + 1)
+            if all((tmap[(r * (K // tk) + q) // 32] >> ((r * (K // tk) + q) % 32)) & 1
+                   for r in rows for q in cols):
+                sparse_steps += 1
+    total = (N // 128) * (K // 64)
+    assert packed.size == 9216 * sparse_steps + 16384 * (total - sparse_steps)
+    assert int(((table >> np.uint64(60)) & np.uint64(1)).sum()) == sparse_steps

@@ -31,6 +31,20 @@ def u32(t):
     return t.cpu().numpy().view(np.uint32)
 
 
+class forced_kernel:
+    """Run the block's GEMMs (M > 16) on one prefill kernel: 1 one-band,
+    2 band-pair, 3 two-SM (test hook of the library; 0 restores the choice)."""
+
+    def __init__(self, P, which):
+        self.P, self.which = P, which
+
+    def __enter__(self):
+        self.P.test_prefill_kernel(self.which)
+
+    def __exit__(self, *exc):
+        self.P.test_prefill_kernel(0)
+
+
 def rel_rms_check(y, yref_f64, fp32_mode):
     y = y.double().cpu().numpy()
     rms = float(np.sqrt(np.mean(yref_f64 ** 2))) if yref_f64.size else 0.0
@@ -493,10 +507,18 @@ def test_gemm_chain_overlapped_matches_serialised(P, oracle_mod):
 ])
 @pytest.mark.parametrize("fp32_mode", [True, False])
 def test_gemm_band_pair_kernel(P, oracle_mod, N, K, M, tn, tk, frac, fp32_mode):
-    # token counts whose one-band tiling takes two or more waves of SMs take
-    # the band-pair kernel (two bands per CTA sharing each X tile)
-    run_case(P, oracle_mod, N, K, M, tn, tk, frac, seed=N + M + tn, fp32_mode=fp32_mode,
-             sample=6000)
+    # the band-pair kernel (two bands per CTA sharing each X tile), forced
+    with forced_kernel(P, 2):
+        run_case(P, oracle_mod, N, K, M, tn, tk, frac, seed=N + M + tn, fp32_mode=fp32_mode,
+                 sample=6000)
+
+
+@pytest.mark.parametrize("M", [200, 1300])
+def test_gemm_one_band_kernel_forced(P, oracle_mod, M):
+    # the one-band kernel (stream-K below two waves of tiles) at prefill sizes
+    with forced_kernel(P, 1):
+        run_case(P, oracle_mod, 2048, 1024, M, 128, 128, 0.5, seed=M + 5, fp32_mode=True,
+                 sample=6000)
 
 
 def test_gemm_band_pair_kernel_bounded_wait(P, oracle_mod):
@@ -511,12 +533,14 @@ def test_gemm_band_pair_kernel_bounded_wait(P, oracle_mod):
     pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
     P.test_stall_first_kstep(True)
     try:
-        P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+        with forced_kernel(P, 2):
+            P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
     finally:
         P.test_stall_first_kstep(False)
     assert P.patch_get_status(pk) == 5
     assert P.patch_get_status(pk) == 0
-    y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    with forced_kernel(P, 2):
+        y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
     torch.cuda.synchronize()
     weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap)
     g = np.random.default_rng(43)
@@ -548,10 +572,29 @@ def band_aligned_map(n_rows_tiles, n_col_tiles, seed):
 ])
 @pytest.mark.parametrize("fp32_mode", [True, False])
 def test_gemm_two_sm_kernel(P, oracle_mod, N, K, M, tn, frac, fp32_mode):
-    # maps whose bands 2p and 2p+1 agree in type at every k-step take the
-    # cta_group::2 kernel (one band per SM of a CTA pair, M = 256 MMAs)
-    run_case(P, oracle_mod, N, K, M, tn, tn, frac, seed=N + M + 7 * tn, fp32_mode=fp32_mode,
-             sample=6000)
+    # maps whose bands 2p and 2p+1 agree in type at every k-step run the
+    # cta_group::2 kernel on the packed k-steps alone (one band per SM of a
+    # CTA pair, M = 256 MMAs)
+    with forced_kernel(P, 3):
+        run_case(P, oracle_mod, N, K, M, tn, tn, frac, seed=N + M + 7 * tn, fp32_mode=fp32_mode,
+                 sample=6000)
+
+
+@pytest.mark.parametrize("N,K,M,tn,tk,frac", [
+    (4096, 1024, 1300, 128, 128, 0.5),   # random map: half the k-pairs of a band pair differ
+    (4096, 1024, 1300, 128, 128, 0.25),
+    (4096, 1024, 1300, 64, 64, 0.5),     # 64-row tiles: mixed halves inside a band
+    (4096, 1024, 1300, 128, 64, 0.5),    # 64-column tiles: k-pairs of mixed type
+    (2048, 768, 700, 64, 128, 0.75),
+])
+@pytest.mark.parametrize("fp32_mode", [True, False])
+def test_gemm_two_sm_kernel_mixed_maps(P, oracle_mod, N, K, M, tn, tk, frac, fp32_mode):
+    # any map runs the two-SM kernel through the prefill table: where the two
+    # bands of an instruction differ in type, their k-pairs come from dense
+    # copies of W_eff written by the packer after the packed bytes
+    with forced_kernel(P, 3):
+        run_case(P, oracle_mod, N, K, M, tn, tk, frac, seed=N + M + tn + tk, fp32_mode=fp32_mode,
+                 sample=6000)
 
 
 @pytest.mark.parametrize("fp32_mode", [True, False])
