@@ -547,6 +547,8 @@ def main():
     ap.add_argument("--T", type=int, default=2048)
     ap.add_argument("--frac", type=float, default=0.5)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--force-kernel", type=int, default=0,
+                    help="--case gemm: prefill kernel (library test hook; 0 = the library's choice)")
     args = ap.parse_args()
     if args.case:
         return run_case(args)
@@ -780,6 +782,7 @@ def run_case(args):
                 P.patch_pack(W, r["meta"], r["map"]).close()
         else:
             pk = P.patch_pack(W, r["meta"], r["map"])
+            P.test_prefill_kernel(args.force_kernel)
             for _ in range(args.reps):
                 P.patch_hybrid_gemm(pk, X)
             torch.cuda.synchronize()

@@ -307,7 +307,8 @@ void patch_test_stall_first_kstep(int32_t on);
  * Test hook: the prefill kernel every later patch_hybrid_gemm with M > 16
  * uses.  0 = chosen by the library (the default), 1 = one band per CTA,
  * 2 = two bands per CTA sharing each token tile, 3 = two-SM (CTA pair)
- * kernel, used only where the band count is even (else as 0).  Results are
+ * kernel, 4 = two-SM kernel with two bands per SM; 3 and 4 only where the
+ * band count is even (else as 0).  Results are
  * the same up to fp32 rounding order; this only lets tests reach each kernel.
  */
 void patch_test_prefill_kernel(int32_t which);

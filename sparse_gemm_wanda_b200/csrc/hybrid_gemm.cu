@@ -658,6 +658,10 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
         const DuoPlan dp = plan_duo_gemm(g.N, g.M, g.num_sms, g.max_pair_bytes);
         if (dp.bn > 0) return launch_duo_gemm(g, dp, stream);
     }
+    if (g.force_kernel == 4 && g.duo_ok && g.K / kStep <= 448) {
+        const QuadPlan qp = plan_quad_gemm(g.N, g.M, g.num_sms);
+        if (qp.bn > 0) return launch_quad_gemm(g, qp, stream);
+    }
     if (g.M <= 64) return run<64, 4>(g, 1, stream);   // 48 KB stages
     if (g.M <= 128) return run<128, 3>(g, 1, stream); // 64 KB stages
     // larger token counts: the band-pair kernel (two bands share each X tile)
@@ -670,9 +674,13 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     const int64_t waves1 = (items1 + g.num_sms - 1) / g.num_sms;
     const double t_one = static_cast<double>(waves1) * 576.0;
     if (g.duo_ok && g.K / kStep <= 448) {
-        // two-SM MMA (through the prefill table, whose band pairs agree in
-        // type) when its estimate is lowest
+        // two-SM MMAs (through the prefill table, whose band pairs agree in
+        // type) when their estimate is lowest: four bands per CTA pair, else two
         const DuoPlan dp = plan_duo_gemm(g.N, g.M, g.num_sms, g.max_pair_bytes);
+        const QuadPlan qp = plan_quad_gemm(g.N, g.M, g.num_sms);
+        const double best_duo = dp.bn > 0 ? dp.cost : 1e30;
+        if (qp.bn > 0 && qp.cost <= best_duo && qp.cost <= pp.cost && qp.cost <= t_one)
+            return launch_quad_gemm(g, qp, stream);
         if (dp.bn > 0 && dp.cost <= pp.cost && dp.cost <= t_one) return launch_duo_gemm(g, dp, stream);
     }
     if (pp.cost <= t_one && g.K / kStep <= 448)

@@ -474,7 +474,7 @@ uint64_t patch_launch_count(void) { return patchk::g_launches.load(std::memory_o
 void patch_test_stall_first_kstep(int32_t on) { g_test_stall.store(on ? 1 : 0, std::memory_order_relaxed); }
 
 void patch_test_prefill_kernel(int32_t which) {
-    g_test_kernel.store((which >= 0 && which <= 3) ? which : 0, std::memory_order_relaxed);
+    g_test_kernel.store((which >= 0 && which <= 4) ? which : 0, std::memory_order_relaxed);
 }
 
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,

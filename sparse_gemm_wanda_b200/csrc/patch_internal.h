@@ -97,7 +97,7 @@ struct GemmLaunch {
     int max_pair_bytes;               // largest k-pair the prefill table points to
     int num_sms;
     int stall_first_kstep;   // failure-detection test hook (see patch_hybrid_gemm)
-    int force_kernel;        // test hook: 0 auto, 1 one-band, 2 band-pair, 3 two-SM (M > 16)
+    int force_kernel;        // test hook: 0 auto, 1 one-band, 2 band-pair, 3 two-SM, 4 two-SM four-band (M > 16)
     const int64_t *pair_prefix;  // host: per band, cumulative packed bytes of its k-pairs
 };
 
@@ -134,6 +134,20 @@ struct DuoPlan {
 DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms, int max_pair_bytes);
 cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream_t stream);
 double duo_kstep_cycles(int bn);
+
+// Two-SM, four-band prefill GEMM (csrc/prefill_quad.cu): each SM of a CTA
+// pair holds two bands (pairs 2p, 2p+1 of the prefill table) sharing its half
+// of the token tile.
+struct QuadPlan {
+    int bn;           // tokens per tile (each CTA of the pair holds bn / 2)
+    int ttiles, items;
+    int clusters;     // CTA pairs launched
+    int stages, stage_bytes, smem;
+    double cost;      // waves x estimated cycles per k-step of an item
+};
+QuadPlan plan_quad_gemm(int64_t N, int64_t M, int num_sms);
+cudaError_t launch_quad_gemm(const GemmLaunch &g, const QuadPlan &plan, cudaStream_t stream);
+double quad_kstep_cycles(int bn);
 
 // Decode GEMV for M <= 16 (csrc/decode_gemm.cu).
 cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream);

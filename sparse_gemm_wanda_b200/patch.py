@@ -118,7 +118,8 @@ def test_stall_first_kstep(on: bool) -> None:
 
 
 def test_prefill_kernel(which: int) -> None:
-    """Test hook: 0 auto, 1 one-band, 2 band-pair, 3 two-SM prefill kernel (M > 16)."""
+    """Test hook: 0 auto, 1 one-band, 2 band-pair, 3 two-SM, 4 two-SM four-band
+    prefill kernel (M > 16)."""
     load_library().patch_test_prefill_kernel(int(which))
 
 

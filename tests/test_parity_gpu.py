@@ -685,3 +685,51 @@ def test_sharded_pieces_match_whole(P, oracle_mod, world, N, K, T, M, frac):
         assert P.patch_get_status(pk) == 0
         rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), np.ascontiguousarray(weff[n0:n1])), True)
         pk.close()
+
+
+# ------------------------------------------- two-SM kernel, two bands per SM
+
+@pytest.mark.parametrize("N,K,M,tn,tk,frac", [
+    (4096, 1024, 1300, 128, 128, 0.0),   # every tile dense
+    (4096, 1024, 1300, 128, 128, 1.0),   # every tile 2:4
+    (4096, 1024, 1300, 128, 128, 0.5),   # random map through the prefill table
+    (4352, 512, 700, 64, 64, 0.5),       # 34 bands: the last quad holds one band pair
+    (768, 1024, 333, 128, 64, 0.75),     # 6 bands, 64-column tiles, ragged token tile
+    (2048, 768, 2000, 64, 128, 1.0),
+])
+@pytest.mark.parametrize("fp32_mode", [True, False])
+def test_gemm_quad_kernel(P, oracle_mod, N, K, M, tn, tk, frac, fp32_mode):
+    # four bands per CTA pair: bands 4q+2j (leader) and 4q+2j+1 (peer) in one
+    # M = 256 instruction per pair j, both pairs sharing each SM's X half
+    with forced_kernel(P, 4):
+        run_case(P, oracle_mod, N, K, M, tn, tk, frac, seed=N + M + 3 * tn + tk,
+                 fp32_mode=fp32_mode, sample=6000)
+
+
+def test_gemm_quad_kernel_bounded_wait(P, oracle_mod):
+    # the failure-detection hook on the four-band kernel: the first CTA never
+    # arms its first stage; both CTAs of its pair give up within their bounds,
+    # meet at the final cluster barrier, and the handle works afterwards
+    N, K, M = 4096, 512, 1300
+    w, xc, x = make_problem(N, K, 64, M, seed=53)
+    nt = (N // 128) * (K // 128)
+    tmap = inputs.random_map(nt, nt // 2, seed=53)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    P.test_stall_first_kstep(True)
+    try:
+        with forced_kernel(P, 4):
+            P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    finally:
+        P.test_stall_first_kstep(False)
+    assert P.patch_get_status(pk) == 5
+    assert P.patch_get_status(pk) == 0
+    with forced_kernel(P, 4):
+        y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap)
+    g = np.random.default_rng(53)
+    ms, ns = g.integers(0, M, 3000), g.integers(0, N, 3000)
+    yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
+    rel_rms_check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, True)
+    pk.close()
