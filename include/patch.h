@@ -107,6 +107,25 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
                               double *tile_loss_out, void *stream);
 
 /*
+ * The mask builder for another N:M pattern ("PATCH: Learnable Tile-level
+ * Hybrid Sparsity for LLMs", section 5, significance: the tile scheme is not
+ * tied to 2:4 and extends to patterns such as 4:8).  (n_keep, m_group) =
+ * (2, 4) is exactly patch_score_mask; (4, 8): inside a sparse tile every
+ * group of 8 consecutive input channels keeps the 4 weights with the highest
+ * Wanda score (ties to the lower index).  Arguments, outputs, tile loss order
+ * and map rule as patch_score_mask, except the codes:
+ *   meta [N, K/32] uint32: group g of row i (columns 8g..8g+7) is an 8-bit
+ *        keep mask (bit q set for a kept position q; four bits set) at bits
+ *        8*(g%4) of word [i, g/4].
+ * Errors as patch_score_mask; PATCH_ERR_UNSUPPORTED for other (n, m).
+ */
+patch_status patch_score_mask_nm(const void *W_bf16, const void *Xcal_bf16, int64_t T,
+                                 const double *colsq_in, patch_shape shp, int32_t n_keep,
+                                 int32_t m_group, double sparse_tile_fraction, const uint32_t *map_in,
+                                 uint32_t *meta_out, uint32_t *map_out, double *colsq_out,
+                                 double *tile_loss_out, void *stream);
+
+/*
  * Column sums of squares of calibration activations alone: the activation
  * term of the Wanda score (SparseGPT-vs-Wanda page, section on Wanda: the
  * weight magnitude is weighed by the input activation of its channel; here
@@ -268,6 +287,25 @@ patch_status patch_select_maps_global(const double *const *losses, const int64_t
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
                         patch_shape shp, patch_packed **out, size_t *packed_bytes,
                         void *stream);
+
+/*
+ * Compressor for another N:M pattern (see patch_score_mask_nm).  (2, 4) is
+ * exactly patch_pack.  (4, 8): the 4:8 handle's packed format (normative):
+ *   - bands of 128 rows, k-steps of 64 columns; a k-step is 4:8-compressed
+ *     iff every map tile overlapping it is 4:8, otherwise dense (the dense
+ *     layout above, holding W_eff: pruned entries of 4:8 tiles +0);
+ *   - 4:8 k-step: 9216 bytes: kept value v (v < 32, column order, four per
+ *     group of 8) of row r at byte r*64 + v*2; the keep mask of group g
+ *     (g < 8) of row r at byte 8192 + r*8 + g;
+ *   - table[b*(K/64)+c] (uint64): bits 0..47 byte offset; bit 60 = 4:8.
+ * The tensor cores have no 4:8 mode for 16-bit inputs: patch_hybrid_gemm on
+ * a 4:8 handle expands each 4:8 k-step in shared memory into the dense tile
+ * and issues dense MMAs (the compressed bytes are what it reads from memory).
+ * Errors as patch_pack; PATCH_ERR_UNSUPPORTED for other (n, m).
+ */
+patch_status patch_pack_nm(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
+                           patch_shape shp, int32_t n_keep, int32_t m_group, patch_packed **out,
+                           size_t *packed_bytes, void *stream);
 
 /*
  * Hybrid product Y[M,N] = X[M,K] * W_eff^T with fp32 accumulation in tensor

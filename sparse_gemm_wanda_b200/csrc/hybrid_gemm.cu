@@ -38,6 +38,13 @@
 //     main loop of the next.
 //   * warps 2..5: epilogue.  tcgen05.ld (each warp its 32-lane quarter), one
 //     rounding to bf16 (or fp32 out), stores to Y, or partials.
+//   * 4:8 handles only (NM = true, 320 threads): warps 6..9, converters.  The
+//     tensor core has no 4:8 sparse mode for 16-bit inputs, so a 4:8 k-step
+//     (kept values + 8-bit keep masks, 9 KB) lands in its stage's 16 KB region
+//     and the converters rewrite it in place as the dense 128-byte-swizzled
+//     tile (thread = row: read its 32 values and 8 masks, all four warps meet
+//     on an mbarrier, write its 8 chunks of 16 B), then fence to the async
+//     proxy and release the stage to the MMA thread, which issues dense MMAs.
 //
 // Every mbarrier wait is bounded by %globaltimer; when one runs out the CTA
 // raises the status word, drains its copies in flight and returns.
@@ -56,6 +63,7 @@
 namespace patchk {
 
 constexpr int kGemmThreads = 192;
+constexpr int kGemmThreadsNM = 320;  // + 4 converter warps for 4:8 handles
 // k-steps of one segment whose table entries are staged in shared memory
 // (K <= 28672)
 constexpr int kMaxTableSteps = 448;
@@ -76,7 +84,7 @@ struct GemmCfg {
     static constexpr int kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128
                                      : kCols <= 256 ? 256 : 512;
     static constexpr int kEcol = 2 * BN;
-    static constexpr int kBarBytes = 8 * (2 * STAGES + 6) + 32 + 24 * STAGES;
+    static constexpr int kBarBytes = 8 * (4 * STAGES + 6) + 32 + 24 * STAGES;
     static constexpr int kTabBytes = 2 * kMaxTableSteps * 8;  // two segments of table entries
     static constexpr int kSmemBytes = STAGES * kStageBytes + kTabBytes + 1024 + kBarBytes;
     static_assert(kBTileBytes % 1024 == 0, "stage regions must stay 1024-B aligned");
@@ -158,8 +166,57 @@ __device__ __forceinline__ void store_y(const GemmParams &p, int64_t idx, float 
         static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
 }
 
-template <int BN, int STAGES>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// One 4:8 k-step of a stage region, in place: 128 rows x (32 kept bf16 at
+// r*64, 8 keep masks at 8192 + r*8) -> 128 x 64 bf16 in the K-major
+// 128-byte-swizzled layout (row r, 16-byte chunk g at r*128 + (g ^ (r%8))*16).
+// Thread `row` holds its row's inputs in `v` (16 words) and `m` (2 words).
+__device__ __forceinline__ void nm48_read(const uint8_t *region, int row, uint32_t (&v)[16],
+                                          uint32_t (&m)[2]) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(region + row * 64);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 x = src[q];
+        v[4 * q] = x.x;
+        v[4 * q + 1] = x.y;
+        v[4 * q + 2] = x.z;
+        v[4 * q + 3] = x.w;
+    }
+    const uint2 mm = *reinterpret_cast<const uint2 *>(region + 8192 + row * 8);
+    m[0] = mm.x;
+    m[1] = mm.y;
+}
+__device__ __forceinline__ void nm48_write(uint8_t *region, int row, const uint32_t (&v)[16],
+                                           const uint32_t (&m)[2]) {
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        const uint32_t mask = (m[g / 4] >> (8 * (g % 4))) & 0xFFu;
+        // the group's four kept values, in column order
+        const uint32_t k[4] = {v[2 * g] & 0xFFFFu, v[2 * g] >> 16, v[2 * g + 1] & 0xFFFFu,
+                               v[2 * g + 1] >> 16};
+        uint32_t o[4];
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2) {
+            uint32_t h[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int q = 2 * q2 + t;
+                const uint32_t idx = __popc(mask & ((1u << q) - 1u));
+                const uint32_t val = idx == 0 ? k[0] : (idx == 1 ? k[1] : (idx == 2 ? k[2] : k[3]));
+                h[t] = ((mask >> q) & 1u) ? val : 0u;
+            }
+            o[q2] = h[0] | (h[1] << 16);
+        }
+        *reinterpret_cast<uint4 *>(region + row * 128 + ((g ^ (row % 8)) * 16)) =
+            make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+__device__ __forceinline__ void fence_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int BN, int STAGES, bool NM>
+__global__ void __launch_bounds__(NM ? kGemmThreadsNM : kGemmThreads, 1)
 hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmParams p) {
     using C = GemmCfg<BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
@@ -171,7 +228,9 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
     uint64_t *acc_full = empty + STAGES;   // [2]
     uint64_t *acc_empty = acc_full + 2;    // [2]
     uint64_t *tab_full = acc_empty + 2;    // [2]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tab_full + 2);
+    uint64_t *conv = tab_full + 2;         // [STAGES] 4:8: stage converted (4 warps)
+    uint64_t *cread = conv + STAGES;       // [STAGES] 4:8: inputs read (4 warps)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cread + STAGES);
     volatile uint32_t *abort_flag = tmem_slot + 1;  // raised by any role that gives up
     volatile uint32_t *never_flag = tmem_slot + 2;  // stays 0: time-only bounded waits
     // per stage, written by the producer before it arms the stage: the pair's two
@@ -192,6 +251,8 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&conv[s], 4);
+            mbar_init(&cread[s], 4);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -278,8 +339,18 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     ++it;
                     if (p.stall_first_kstep && cta == 0 && it == 1) continue;  // never lands
                     uint8_t *st = smem + s * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], bytes + C::kBBytes);
-                    bulk_g2s(st, p.packed + first, bytes, &full[s]);
+                    if constexpr (NM) {
+                        // 4:8 handle: each k-step into its own 16 KB region,
+                        // where the converters expand a 4:8 one in place
+                        const uint32_t b0 = (c0 & kEntryNM48) ? kNM48StepBytes : kDenseStepBytes;
+                        const uint32_t b1 = (c1 & kEntryNM48) ? kNM48StepBytes : kDenseStepBytes;
+                        mbar_arrive_expect_tx(&full[s], b0 + b1 + C::kBBytes);
+                        bulk_g2s(st, p.packed + (c0 & kEntryOffsetMask), b0, &full[s]);
+                        bulk_g2s(st + kDenseStepBytes, p.packed + (c1 & kEntryOffsetMask), b1, &full[s]);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], bytes + C::kBBytes);
+                        bulk_g2s(st, p.packed + first, bytes, &full[s]);
+                    }
                     if (waited) {
                         tma_load_3d(st + C::kABytes, &tmap_x, 0, sg.ttile * BN, 2 * pr, &full[s]);
                     } else {
@@ -342,14 +413,20 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                         ok = false;
                         break;
                     }
+                    // 4:8 handle: the converters have rewritten the stage as dense tiles
+                    if (NM && !mbar_wait_bounded(&conv[s], ph, abort_flag, kWaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint64_t first = stage_info[3 * s + 2];
                     uint8_t *st = smem + s * C::kStageBytes;
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const uint64_t e = stage_info[3 * s + h];
+                        const uint64_t e = NM ? 0ull : stage_info[3 * s + h];  // 4:8: all dense now
                         const uint32_t a_addr =
-                            smem_u32(st + static_cast<uint32_t>((e & kEntryOffsetMask) - first));
+                            NM ? smem_u32(st + h * kDenseStepBytes)
+                               : smem_u32(st + static_cast<uint32_t>((e & kEntryOffsetMask) - first));
                         const uint32_t b_addr = smem_u32(st + C::kABytes + h * C::kBTileBytes);
                         const bool first_step = (pr == sg.ks0 / 2) && h == 0;
                         if (e & kEntrySparse) {
@@ -381,6 +458,50 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             if (!ok) {
                 *abort_flag = 1u;
                 atomicOr(p.status, kStatusTimeout);
+            }
+        }
+    } else if (warp >= 6) {
+        if constexpr (NM) {
+            if (!skip) {
+                // -------------------------------------------- 4:8 converters
+                // every stage in the MMA's order; a 4:8 k-step is rewritten in
+                // place, so all rows are read (all four warps meet on `cread`)
+                // before any row is written
+                const int row = (warp - 6) * 32 + lane;
+                int it = 0;
+                bool ok = true;
+                Segment sg;
+                for (int i = 0; ok && get_segment(p, cta, i, sg); ++i) {
+                    for (int pr = sg.ks0 / 2; pr < sg.ks1 / 2; ++pr, ++it) {
+                        const int s = it % STAGES;
+                        const uint32_t ph = (it / STAGES) & 1u;
+                        if (!mbar_wait_bounded(&full[s], ph, abort_flag, kWaitLimitNs)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *st = smem + s * C::kStageBytes;
+                        const bool c0 = (stage_info[3 * s + 0] & kEntryNM48) != 0;
+                        const bool c1 = (stage_info[3 * s + 1] & kEntryNM48) != 0;
+                        uint32_t v0[16], m0[2], v1[16], m1[2];
+                        if (c0) nm48_read(st, row, v0, m0);
+                        if (c1) nm48_read(st + kDenseStepBytes, row, v1, m1);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&cread[s]);
+                        if (!mbar_wait_bounded(&cread[s], ph, abort_flag, kWaitLimitNs)) {
+                            ok = false;
+                            break;
+                        }
+                        if (c0) nm48_write(st, row, v0, m0);
+                        if (c1) nm48_write(st + kDenseStepBytes, row, v1, m1);
+                        fence_async_shared();  // the generic-proxy writes, visible to the MMA
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&conv[s]);
+                    }
+                }
+                if (!ok) {
+                    *abort_flag = 1u;
+                    atomicOr(p.status, kStatusTimeout);
+                }
             }
         }
     } else if (!skip) {
@@ -568,13 +689,13 @@ void streamk_bounds(const GemmLaunch &g, GemmParams &p, int bn, int P) {
         if (p.u0[c] >= p.u0[c + 1]) p.u0[c] = p.u0[c + 1] - 1;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool NM = false>
 cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     using C = GemmCfg<BN, STAGES>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(hybrid_gemm_kernel<BN, STAGES>,
+        attr_err = cudaFuncSetAttribute(hybrid_gemm_kernel<BN, STAGES, NM>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
@@ -622,7 +743,7 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     // before griddepcontrol.wait)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(NM ? kGemmThreadsNM : kGemmThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -630,7 +751,7 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t err = cudaLaunchKernelEx(&cfg, hybrid_gemm_kernel<BN, STAGES>, map, p);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, hybrid_gemm_kernel<BN, STAGES, NM>, map, p);
     if (err == cudaSuccess) note_launches(1);
     if (err == cudaSuccess && sk) {
         cfg.gridDim = dim3(static_cast<unsigned>((BN * kBand + 255) / 256), static_cast<unsigned>(tiles));
@@ -650,6 +771,12 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
+    if (g.pattern == 4) {
+        // 4:8 handles: the one-band kernel with converter warps, every M
+        // (stream-K over (tile, k-pair) units when tiles are few)
+        if (g.M <= 64) return run<64, 4, true>(g, 1, stream);
+        return run<160, 3, true>(g, 1, stream);
+    }
     if (g.M <= 16) return launch_decode_gemm(g, stream);  // split-K GEMV, csrc/decode_gemm.cu
     // test hook: one prefill kernel for every M > 16 (parity of each kernel)
     if (g.force_kernel == 1) return run<160, 3>(g, 1, stream);

@@ -53,6 +53,27 @@ __device__ __forceinline__ uint32_t top2_code(const double s[4]) {
     return lo | (hi << 2);
 }
 
+// 4:8 groups: q is kept iff fewer than four other candidates come before it
+// in the order (score desc, index asc); returns the 8-bit keep mask.
+__device__ __forceinline__ uint32_t top4_mask(const double s[8]) {
+    int r[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) r[q] = 0;
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = a + 1; b < 8; ++b) {
+            // a < b: a precedes b iff s_a >= s_b (a tie goes to the lower index)
+            const int ab = s[a] >= s[b];
+            r[b] += ab;
+            r[a] += 1 - ab;
+        }
+    uint32_t m = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) m |= static_cast<uint32_t>(r[q] < 4) << q;
+    return m;
+}
+
 // |w| of a bf16 bit pattern, exactly, as a double (sign cleared: -0 -> +0).
 // Normal values are rebuilt with integer operations (exponent rebias 127 ->
 // 1023, mantissa moved up); zero and subnormals take the conversion path.
@@ -64,10 +85,11 @@ __device__ __forceinline__ double bf16_abs_f64(uint32_t bits16) {
 
 // One CTA per tile, one thread per (row, 32-column word) of the tile.  A
 // thread reads its 64 bytes of W with coalesced 16-byte loads (a warp covers
-// whole rows), scores its 8 groups, writes the meta word and the word's
-// pruned-score sum (left to right).  The CTA then adds each row's words left
-// to right and the rows as a balanced pairwise tree.
-template <int TN, int TK>
+// whole rows), scores its groups (PAT = 2: eight 2:4 groups, 4-bit codes;
+// PAT = 4: four 4:8 groups, 8-bit keep masks), writes the meta word and the
+// word's pruned-score sum (left to right).  The CTA then adds each row's
+// words left to right and the rows as a balanced pairwise tree.
+template <int TN, int TK, int PAT>
 __global__ void __launch_bounds__(TN *(TK / 32))
 score_mask_kernel(const uint16_t *__restrict__ W, const double *__restrict__ norm, int64_t N,
                   int64_t K, uint32_t *__restrict__ meta, double *__restrict__ loss,
@@ -94,6 +116,23 @@ score_mask_kernel(const uint16_t *__restrict__ W, const double *__restrict__ nor
     const double *nw = ns + w * kNormStride;
     double acc = 0.0;
     uint32_t word = 0;
+    if constexpr (PAT == 4) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {  // group h: columns 8h .. 8h+7 of the word
+            const uint32_t e[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+            double sc[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t bits = (q & 1) ? (e[q / 2] >> 16) : (e[q / 2] & 0xFFFFu);
+                sc[q] = __dmul_rn(bf16_abs_f64(bits), nw[8 * h + q]);
+            }
+            const uint32_t m = top4_mask(sc);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (!((m >> q) & 1u)) acc = __dadd_rn(acc, sc[q]);
+            word |= m << (8 * h);
+        }
+    } else
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
         const uint32_t e[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
@@ -253,22 +292,28 @@ cudaError_t launch_norms_from_colsq(const double *colsq_in, int64_t K, double *c
 
 cudaError_t launch_score_mask(const void *W, const double *norm, int64_t N, int64_t K, int tn,
                               int tk, uint32_t *meta, double *loss, int32_t *rank, uint32_t *done,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, int pattern) {
     const int64_t n_tiles = (N / tn) * (K / tk);
     const uint16_t *w = static_cast<const uint16_t *>(W);
     const unsigned g = static_cast<unsigned>(n_tiles);
-    if (tn == 128 && tk == 128)
-        score_mask_kernel<128, 128><<<g, 512, 0, stream>>>(w, norm, N, K, meta, loss, rank, done);
-    else if (tn == 128 && tk == 64)
-        score_mask_kernel<128, 64><<<g, 256, 0, stream>>>(w, norm, N, K, meta, loss, rank, done);
-    else if (tn == 64 && tk == 128)
-        score_mask_kernel<64, 128><<<g, 256, 0, stream>>>(w, norm, N, K, meta, loss, rank, done);
-    else if (tn == 64 && tk == 64)
-        score_mask_kernel<64, 64><<<g, 128, 0, stream>>>(w, norm, N, K, meta, loss, rank, done);
-    else
-        return cudaErrorInvalidValue;
-    note_launches(1);
-    return cudaGetLastError();
+#define PATCH_SCORE_LAUNCH(TN, TK)                                                                  \
+    if (tn == TN && tk == TK) {                                                                     \
+        if (pattern == 4)                                                                           \
+            score_mask_kernel<TN, TK, 4><<<g, TN *(TK / 32), 0, stream>>>(w, norm, N, K, meta, loss, \
+                                                                        rank, done);               \
+        else                                                                                        \
+            score_mask_kernel<TN, TK, 2><<<g, TN *(TK / 32), 0, stream>>>(w, norm, N, K, meta, loss, \
+                                                                        rank, done);               \
+        note_launches(1);                                                                           \
+        return cudaGetLastError();                                                                  \
+    }
+    if (pattern != 2 && pattern != 4) return cudaErrorInvalidValue;
+    PATCH_SCORE_LAUNCH(128, 128)
+    PATCH_SCORE_LAUNCH(128, 64)
+    PATCH_SCORE_LAUNCH(64, 128)
+    PATCH_SCORE_LAUNCH(64, 64)
+#undef PATCH_SCORE_LAUNCH
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_select_map(const double *loss, int64_t n_tiles, int64_t n_sparse, int32_t *rank,

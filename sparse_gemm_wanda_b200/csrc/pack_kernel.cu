@@ -36,6 +36,15 @@ __device__ __forceinline__ uint4 mask_two_groups(uint4 v, uint32_t codes8) {
     return make_uint4(e[0], e[1], e[2], e[3]);
 }
 
+// Keep the entries of one 4:8 group (8 bf16 in a uint4) whose mask bits are set.
+__device__ __forceinline__ uint4 mask_eight(uint4 v, uint32_t m) {
+    uint32_t e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+        if (!((m >> q) & 1u)) e[q / 2] &= (q & 1) ? 0x0000FFFFu : 0xFFFF0000u;
+    return make_uint4(e[0], e[1], e[2], e[3]);
+}
+
 // The two kept values of one group (4 bf16 in the 32-bit words a, b) as one
 // 32-bit word, lower position first.
 __device__ __forceinline__ uint32_t kept_pair(uint32_t a, uint32_t b, uint32_t code) {
@@ -52,7 +61,8 @@ __global__ void __launch_bounds__(kPackThreads)
 pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
             const uint32_t *__restrict__ map, int64_t N, int64_t K, int tn, int tk,
             const uint64_t *__restrict__ table, const uint64_t *__restrict__ ptable,
-            uint8_t *__restrict__ out, uint32_t *__restrict__ done, uint32_t *__restrict__ ready) {
+            uint8_t *__restrict__ out, uint32_t *__restrict__ done, uint32_t *__restrict__ ready,
+            int pattern) {
     const int64_t nsteps = K / kStep;
     const int64_t steps_all = (N / kBand) * nsteps;
     // blocks [0, steps_all): the packed k-steps; blocks [steps_all, 2 steps_all)
@@ -68,6 +78,39 @@ pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
 
     if (side && !(entry & kEntrySide)) {
         // the prefill table reuses the packed k-step here: nothing to write
+    } else if (entry & kEntryNM48) {
+        // 4:8: thread = row; its 32 kept values (in column order, four per
+        // group of 8) at r*64, its 8 keep masks at 8192 + r*8
+        const int r = tid;
+        const int64_t i = row0 + r;
+        const uint4 *src = reinterpret_cast<const uint4 *>(W + i * K + col0);
+        const uint32_t m0 = __ldg(meta + i * words_k + col0 / 32), m1 = __ldg(meta + i * words_k + col0 / 32 + 1);
+        uint32_t vals[16];
+        uint32_t masks[2] = {0u, 0u};
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            const uint4 q4 = __ldg(src + g);
+            const uint32_t e[4] = {q4.x, q4.y, q4.z, q4.w};
+            const uint32_t m = ((g < 4 ? m0 : m1) >> (8 * (g % 4))) & 0xFFu;
+            masks[g / 4] |= m << (8 * (g % 4));
+            // exactly four kept per group: slots k[0..3] in column order
+            uint32_t k[4] = {0u, 0u, 0u, 0u};
+            int c = 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t h = (q & 1) ? (e[q / 2] >> 16) : (e[q / 2] & 0xFFFFu);
+                const bool keep = (m >> q) & 1u;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) k[t] = (keep && c == t) ? h : k[t];
+                c += keep ? 1 : 0;
+            }
+            vals[2 * g] = k[0] | (k[1] << 16);
+            vals[2 * g + 1] = k[2] | (k[3] << 16);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(out + off + r * 64);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(vals[4 * q], vals[4 * q + 1], vals[4 * q + 2], vals[4 * q + 3]);
+        *reinterpret_cast<uint2 *>(out + off + 8192 + r * 8) = make_uint2(masks[0], masks[1]);
     } else if (!(entry & kEntrySparse)) {
         // dense: chunk u = r*8 + ((k/8) ^ (r%8)); W_eff, i.e. pruned entries of
         // a 2:4 tile (64-row tiles sharing a band with a dense tile) are zeroed
@@ -79,7 +122,10 @@ pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
             const int64_t tile = (i / tn) * (K / tk) + j / tk;
             if ((__ldg(map + tile / 32) >> (tile % 32)) & 1u) {
                 const uint32_t mw = __ldg(meta + i * words_k + j / 32);
-                v = mask_two_groups(v, mw >> (4 * ((j % 32) / 4)));
+                if (pattern == 4)
+                    v = mask_eight(v, (mw >> (8 * ((j % 32) / 8))) & 0xFFu);
+                else
+                    v = mask_two_groups(v, mw >> (4 * ((j % 32) / 4)));
             }
             reinterpret_cast<uint4 *>(out + off)[u] = v;
         }
@@ -175,7 +221,9 @@ __device__ __forceinline__ void band_types(const uint32_t *__restrict__ map, int
 
 __device__ __forceinline__ bool bit_of(const uint32_t *bits, int c) { return (bits[c >> 5] >> (c & 31)) & 1u; }
 
-__device__ __forceinline__ uint32_t kpair_bytes(bool s0, bool s1) {
+__device__ __forceinline__ uint32_t kpair_bytes(bool s0, bool s1, int pattern = 2) {
+    if (pattern == 4)
+        return (s0 ? kNM48StepBytes : kDenseStepBytes) + (s1 ? kNM48StepBytes : kDenseStepBytes);
     return (s0 ? kMetaBlockBytes + kSparseStepBytes : kDenseStepBytes) +
            (s1 ? (s0 ? 0 : kMetaBlockBytes) + kSparseStepBytes : kDenseStepBytes);
 }
@@ -185,7 +233,7 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
                  int cpb, uint64_t *__restrict__ table, uint64_t *__restrict__ chunk_desc,
                  int64_t *__restrict__ pair_prefix, uint64_t *__restrict__ band_start,
                  uint64_t *__restrict__ ptable, uint64_t *__restrict__ side_start,
-                 PackPlan *__restrict__ plan) {
+                 PackPlan *__restrict__ plan, int pattern) {
     __shared__ unsigned long long warp_sum[kPlanWarps];
     __shared__ uint32_t types[kPlanWarps][2][kPlanMaxWords];
     __shared__ unsigned long long carry, n_sparse, n_meta, side_carry;
@@ -197,7 +245,7 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
         carry = 0;
         n_sparse = 0;
         n_meta = 0;
-        duo_ok = (bands % 2 == 0) ? 1u : 0u;
+        duo_ok = (bands % 2 == 0 && pattern == 2) ? 1u : 0u;
         max_pair = 0;
         pmax_pair = 0;
         side_carry = 0;
@@ -217,9 +265,9 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
                 uint32_t bytes = 0;
                 if (q < Q) {
                     const bool s0 = bit_of(mine, 2 * q), s1 = bit_of(mine, 2 * q + 1);
-                    bytes = kpair_bytes(s0, s1);
+                    bytes = kpair_bytes(s0, s1, pattern);
                     ns += s0 + s1;
-                    nm += (s0 || s1) ? 1 : 0;
+                    nm += (pattern == 2 && (s0 || s1)) ? 1 : 0;
                     mp = max(mp, bytes);
                 }
                 unsigned long long incl = bytes;
@@ -286,6 +334,13 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
             const bool s0 = bit_of(mine, 2 * q), s1 = bit_of(mine, 2 * q + 1);
             uint64_t off = start + static_cast<uint64_t>(pre[q]);
             uint64_t e0, e1;
+            if (pattern == 4) {
+                e0 = off | (s0 ? kEntryNM48 : 0ull);
+                off += s0 ? kNM48StepBytes : kDenseStepBytes;
+                row[2 * q] = e0;
+                row[2 * q + 1] = off | (s1 ? kEntryNM48 : 0ull);
+                continue;
+            }
             if (s0) {
                 off += kMetaBlockBytes;
                 e0 = kEntrySparse | kEntryMeta | off;
@@ -328,7 +383,7 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
     // 4a: densified k-pairs per band (counted into side_start)
     for (int pb = wid; 2 * pb < bands; pb += kPlanWarps) {
         const int b = 2 * pb;
-        const bool paired = b + 1 < bands;
+        const bool paired = b + 1 < bands && pattern == 2;
         band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
         if (paired) band_types(map, b + 1, nsteps, log_tn, log_tk, tiles_k, lane, next);
         unsigned int n0 = 0, n1 = 0, mp = 0;
@@ -387,7 +442,7 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
     // 4c: the entries; densified k-pairs are numbered in order within a band
     for (int b = wid; b < bands; b += kPlanWarps) {
         const int partner = b ^ 1;
-        const bool paired = partner < bands;
+        const bool paired = partner < bands && pattern == 2;
         band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
         if (paired) band_types(map, partner, nsteps, log_tn, log_tk, tiles_k, lane, next);
         const uint64_t *row = table + static_cast<int64_t>(b) * nsteps;
@@ -436,24 +491,27 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
 cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, int tk, int cp,
                              int cpb, uint64_t *table, uint64_t *chunk_desc, int64_t *pair_prefix,
                              uint64_t *band_start, uint64_t *ptable, uint64_t *side_start,
-                             PackPlan *plan, cudaStream_t stream) {
+                             PackPlan *plan, cudaStream_t stream, int pattern) {
     const int64_t nsteps = K / kStep;
     if (nsteps > 32 * kPlanMaxWords || (N / kBand) > (int64_t(1) << 24)) return cudaErrorInvalidValue;
+    if (pattern != 2 && pattern != 4) return cudaErrorInvalidValue;
     const int log_tn = tn == 64 ? 6 : 7, log_tk = tk == 64 ? 6 : 7;
     plan_pack_kernel<<<1, kPlanThreads, 0, stream>>>(map, static_cast<int>(N / kBand), static_cast<int>(nsteps),
                                                      log_tn, log_tk, cp, cpb, table, chunk_desc,
-                                                     pair_prefix, band_start, ptable, side_start, plan);
+                                                     pair_prefix, band_start, ptable, side_start, plan,
+                                                     pattern);
     note_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                         int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
-                        uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream) {
+                        uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream, int pattern) {
     const int64_t blocks = (N / kBand) * (K / kStep) * (ptable ? 2 : 1);
-    if (blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    if (blocks > 0x7FFFFFFF || (pattern != 2 && pattern != 4)) return cudaErrorInvalidValue;
     pack_kernel<<<static_cast<unsigned>(blocks), kPackThreads, 0, stream>>>(
-        static_cast<const uint16_t *>(W), meta, map, N, K, tn, tk, table, ptable, out, done, ready);
+        static_cast<const uint16_t *>(W), meta, map, N, K, tn, tk, table, ptable, out, done, ready,
+        pattern);
     note_launches(1);
     return cudaGetLastError();
 }

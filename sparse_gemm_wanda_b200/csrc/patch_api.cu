@@ -20,6 +20,7 @@
 
 struct patch_packed {
     int device;
+    int pattern;               // 2: dense / 2:4 tiles; 4: dense / 4:8 tiles
     uint8_t *base;             // pool allocation: table, descriptors, prefix, plan, workspace, status
     patch_shape shp;
     uint8_t *packed;           // packed k-steps, then the side copies (a pool allocation of its own, exact size)
@@ -194,11 +195,11 @@ const char *patch_status_string(patch_status s) {
     return "unknown status";
 }
 
-patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t T,
-                              const double *colsq_in, patch_shape shp,
-                              double sparse_tile_fraction, const uint32_t *map_in,
-                              uint32_t *meta_out, uint32_t *map_out, double *colsq_out,
-                              double *tile_loss_out, void *stream_v) {
+static patch_status score_mask_impl(const void *W_bf16, const void *Xcal_bf16, int64_t T,
+                                    const double *colsq_in, patch_shape shp,
+                                    double sparse_tile_fraction, const uint32_t *map_in,
+                                    uint32_t *meta_out, uint32_t *map_out, double *colsq_out,
+                                    double *tile_loss_out, void *stream_v, int pattern) {
     patch_status st = check_shape(shp);
     if (st != PATCH_OK) return st;
     if (!W_bf16 || !meta_out || !map_out || !aligned16(W_bf16)) return PATCH_ERR_INVALID_ARG;
@@ -238,7 +239,7 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
         e = patchk::launch_colsq(Xcal_bf16, T, K, partial, colsq_out, norm, stream);
     if (e == cudaSuccess)
         e = patchk::launch_score_mask(W_bf16, norm, N, K, shp.tile_n, shp.tile_k, meta_out, loss,
-                                      rank, done, stream);
+                                      rank, done, stream, pattern);
     if (e == cudaSuccess) {
         if (map_in) {
             e = cudaMemcpyAsync(map_out, map_in, sizeof(uint32_t) * ((n_tiles + 31) / 32),
@@ -251,6 +252,33 @@ patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t
     }
     cudaError_t e2 = cudaFreeAsync(scratch, stream);
     return from_cuda(e != cudaSuccess ? e : e2);
+}
+
+// (n_keep, m_group) -> pattern code: 2 for 2:4, 4 for 4:8, 0 otherwise
+static int pattern_of(int32_t n_keep, int32_t m_group) {
+    if (n_keep == 2 && m_group == 4) return 2;
+    if (n_keep == 4 && m_group == 8) return 4;
+    return 0;
+}
+
+patch_status patch_score_mask(const void *W_bf16, const void *Xcal_bf16, int64_t T,
+                              const double *colsq_in, patch_shape shp,
+                              double sparse_tile_fraction, const uint32_t *map_in,
+                              uint32_t *meta_out, uint32_t *map_out, double *colsq_out,
+                              double *tile_loss_out, void *stream_v) {
+    return score_mask_impl(W_bf16, Xcal_bf16, T, colsq_in, shp, sparse_tile_fraction, map_in, meta_out,
+                           map_out, colsq_out, tile_loss_out, stream_v, 2);
+}
+
+patch_status patch_score_mask_nm(const void *W_bf16, const void *Xcal_bf16, int64_t T,
+                                 const double *colsq_in, patch_shape shp, int32_t n_keep,
+                                 int32_t m_group, double sparse_tile_fraction, const uint32_t *map_in,
+                                 uint32_t *meta_out, uint32_t *map_out, double *colsq_out,
+                                 double *tile_loss_out, void *stream_v) {
+    const int pattern = pattern_of(n_keep, m_group);
+    if (!pattern) return PATCH_ERR_UNSUPPORTED;
+    return score_mask_impl(W_bf16, Xcal_bf16, T, colsq_in, shp, sparse_tile_fraction, map_in, meta_out,
+                           map_out, colsq_out, tile_loss_out, stream_v, pattern);
 }
 
 patch_status patch_colsq(const void *Xcal_bf16, int64_t T, int64_t K, double *colsq_out,
@@ -477,9 +505,9 @@ void patch_test_prefill_kernel(int32_t which) {
     g_test_kernel.store((which >= 0 && which <= 4) ? which : 0, std::memory_order_relaxed);
 }
 
-patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
-                        patch_shape shp, patch_packed **out,
-                        size_t *packed_bytes, void *stream_v) {
+static patch_status pack_impl(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
+                              patch_shape shp, patch_packed **out, size_t *packed_bytes,
+                              void *stream_v, int pattern) {
     if (!out) return PATCH_ERR_INVALID_ARG;
     *out = nullptr;
     patch_status st = check_shape(shp);
@@ -498,6 +526,7 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     patch_packed *h = new (std::nothrow) patch_packed();
     if (!h) return PATCH_ERR_OOM;
     cudaGetDevice(&h->device);
+    h->pattern = pattern;
     h->shp = shp;
     h->num_sms = num_sms;
     h->bands = bands;
@@ -539,7 +568,8 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
         e = patchk::launch_plan_pack(map, N, K, static_cast<int>(tn), static_cast<int>(tk), h->dec_cp,
                                      h->dec_cpb, h->table, h->chunk_desc, h->pair_prefix_dev,
                                      reinterpret_cast<uint64_t *>(h->base + off_bstart), h->ptable,
-                                     reinterpret_cast<uint64_t *>(h->base + off_sstart), plan_dev, stream);
+                                     reinterpret_cast<uint64_t *>(h->base + off_sstart), plan_dev, stream,
+                                     pattern);
     patchk::PackPlan plan;
     h->pair_prefix.assign(static_cast<size_t>(bands * (Q + 1)), 0);
     if (e == cudaSuccess) e = read_plan(plan_dev, &plan, h->pair_prefix_dev, &h->pair_prefix, stream);
@@ -565,7 +595,7 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     if (e == cudaSuccess)
         e = patchk::launch_pack(W_bf16, meta, map, N, K, static_cast<int>(tn), static_cast<int>(tk),
                                 h->table, h->side_bytes ? h->ptable : nullptr, h->packed,
-                                h->status + 1, h->status + 2, stream);
+                                h->status + 1, h->status + 2, stream, pattern);
     if (e != cudaSuccess) {
         patch_free(h, stream_v);
         return from_cuda(e);
@@ -573,6 +603,20 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
     if (packed_bytes) *packed_bytes = h->packed_bytes;
     *out = h;
     return PATCH_OK;
+}
+
+patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
+                        patch_shape shp, patch_packed **out, size_t *packed_bytes, void *stream_v) {
+    return pack_impl(W_bf16, meta, map, shp, out, packed_bytes, stream_v, 2);
+}
+
+patch_status patch_pack_nm(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
+                           patch_shape shp, int32_t n_keep, int32_t m_group, patch_packed **out,
+                           size_t *packed_bytes, void *stream_v) {
+    if (out) *out = nullptr;
+    const int pattern = pattern_of(n_keep, m_group);
+    if (!pattern) return PATCH_ERR_UNSUPPORTED;
+    return pack_impl(W_bf16, meta, map, shp, out, packed_bytes, stream_v, pattern);
 }
 
 patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
@@ -613,6 +657,7 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.pair_prefix = Wp->pair_prefix.empty() ? nullptr : Wp->pair_prefix.data();
     g.stall_first_kstep = g_test_stall.load(std::memory_order_relaxed);
     g.force_kernel = g_test_kernel.load(std::memory_order_relaxed);
+    g.pattern = Wp->pattern;
     return from_cuda(patchk::launch_hybrid_gemm(g, static_cast<cudaStream_t>(stream_v)));
 }
 

@@ -22,6 +22,10 @@ constexpr uint64_t kEntryMeta = 1ull << 63;
 // that follows the packed bytes (see plan_pack_kernel).
 constexpr uint64_t kEntrySide = 1ull << 61;
 constexpr int kSidePairBytes = 2 * kDenseStepBytes;
+// 4:8 handles: a 4:8-compressed k-step (kept values 128 x 32 bf16, row-major,
+// then the 8-bit keep masks 128 x 8); no metadata blocks, no 2:4 k-steps.
+constexpr uint64_t kEntryNM48 = 1ull << 60;
+constexpr int kNM48StepBytes = kBand * 32 * 2 + kBand * 8;  // 9216
 
 // Bit of the device status word set when a bounded wait runs out.
 constexpr uint32_t kStatusTimeout = 1u;

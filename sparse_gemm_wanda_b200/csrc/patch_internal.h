@@ -21,10 +21,11 @@ cudaError_t launch_colsq(const void *Xcal, int64_t T, int64_t K, double *partial
 cudaError_t launch_norms_from_colsq(const double *colsq_in, int64_t K, double *colsq_out,
                                     double *norm_out, cudaStream_t stream);
 // `rank` / `done` (may be null when no map is selected) are zeroed here for
-// launch_select_map, which must follow on the same stream.
+// launch_select_map, which must follow on the same stream.  pattern 2: 2:4
+// groups (4-bit codes); 4: 4:8 groups (8-bit keep masks).
 cudaError_t launch_score_mask(const void *W, const double *norm, int64_t N, int64_t K, int tn,
                               int tk, uint32_t *meta, double *loss, int32_t *rank, uint32_t *done,
-                              cudaStream_t stream);
+                              cudaStream_t stream, int pattern = 2);
 cudaError_t launch_select_map(const double *loss, int64_t n_tiles, int64_t n_sparse, int32_t *rank,
                               uint32_t *done, uint32_t *map, cudaStream_t stream);
 
@@ -44,7 +45,8 @@ cudaError_t launch_select_maps_global(const double *loss_cat, const int64_t *n_t
 // entries, written after the packed bytes.
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                         int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
-                        uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream);
+                        uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream,
+                        int pattern = 2);
 
 // Decode (M <= 16) GEMV: CTAs whose first chunk travels in the kernel
 // parameters, at most.
@@ -71,7 +73,7 @@ struct PackPlan {
 cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, int tk, int cp,
                              int cpb, uint64_t *table, uint64_t *chunk_desc, int64_t *pair_prefix,
                              uint64_t *band_start, uint64_t *ptable, uint64_t *side_start,
-                             PackPlan *plan, cudaStream_t stream);
+                             PackPlan *plan, cudaStream_t stream, int pattern = 2);
 
 struct GemmLaunch {
     const uint8_t *packed;
@@ -98,6 +100,7 @@ struct GemmLaunch {
     int num_sms;
     int stall_first_kstep;   // failure-detection test hook (see patch_hybrid_gemm)
     int force_kernel;        // test hook: 0 auto, 1 one-band, 2 band-pair, 3 two-SM, 4 two-SM four-band (M > 16)
+    int pattern;             // 2: dense / 2:4 tiles; 4: dense / 4:8 tiles
     const int64_t *pair_prefix;  // host: per band, cumulative packed bytes of its k-pairs
 };
 

@@ -25,7 +25,8 @@ EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
            "patch_status_string", "patch_score_mask_noalloc",
            "patch_score_mask_noalloc_capacity", "patch_launch_count",
            "patch_select_maps_global", "patch_test_stall_first_kstep", "patch_pool_usage",
-           "patch_colsq", "patch_colsq_partials", "patch_colsq_fold", "patch_test_prefill_kernel")
+           "patch_colsq", "patch_colsq_partials", "patch_colsq_fold", "patch_test_prefill_kernel",
+           "patch_score_mask_nm", "patch_pack_nm")
 
 
 class PatchLibraryError(RuntimeError):
@@ -77,6 +78,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.patch_select_maps_global.restype = ctypes.c_int
     lib.patch_launch_count.argtypes = []
     lib.patch_launch_count.restype = ctypes.c_uint64
+    lib.patch_score_mask_nm.argtypes = [vp, vp, i64, vp, PatchShape, i32, i32, dbl, vp, vp, vp, vp,
+                                        vp, vp]
+    lib.patch_score_mask_nm.restype = ctypes.c_int
+    lib.patch_pack_nm.argtypes = [vp, vp, vp, PatchShape, i32, i32, ctypes.POINTER(vp),
+                                  ctypes.POINTER(ctypes.c_size_t), vp]
+    lib.patch_pack_nm.restype = ctypes.c_int
     lib.patch_colsq.argtypes = [vp, i64, i64, vp, vp]
     lib.patch_colsq_partials.argtypes = [vp, i64, i64, vp, vp]
     lib.patch_colsq_fold.argtypes = [vp, i64, i64, vp, vp]
@@ -162,8 +169,9 @@ def n_tiles(N: int, K: int, tile_n: int, tile_k: int) -> int:
 def patch_score_mask(W: torch.Tensor, Xcal: torch.Tensor | None = None, *, tile_n: int = 128,
                      tile_k: int = 128, fraction: float = 0.0, map_in: torch.Tensor | None = None,
                      colsq_in: torch.Tensor | None = None, want_colsq: bool = False,
-                     want_loss: bool = False, stream=None) -> dict:
-    """Wanda 2:4 codes, tile map (and optionally colsq, tile loss) for W[N,K] bf16."""
+                     want_loss: bool = False, nm: tuple = (2, 4), stream=None) -> dict:
+    """Wanda N:M codes (2:4 by default, or nm=(4, 8)), tile map (and optionally
+    colsq, tile loss) for W[N,K] bf16."""
     lib = load_library()
     N, K = W.shape
     nt = n_tiles(N, K, tile_n, tile_k)
@@ -173,12 +181,21 @@ def patch_score_mask(W: torch.Tensor, Xcal: torch.Tensor | None = None, *, tile_
     colsq = torch.empty((K,), dtype=torch.float64, device=dev) if want_colsq else None
     loss = torch.empty((nt,), dtype=torch.float64, device=dev) if want_loss else None
     T = Xcal.shape[0] if Xcal is not None else 0
-    code = lib.patch_score_mask(
-        _dptr(W, torch.bfloat16, "W"), _dptr(Xcal, torch.bfloat16, "Xcal"), T,
-        _dptr(colsq_in, torch.float64, "colsq_in"), PatchShape(N, K, tile_n, tile_k),
-        float(fraction), _dptr(map_in, (torch.int32, torch.uint32), "map_in"), _dptr(meta),
-        _dptr(tmap), _dptr(colsq), _dptr(loss), _stream(stream))
-    _check("patch_score_mask", code)
+    if tuple(nm) == (2, 4):
+        code = lib.patch_score_mask(
+            _dptr(W, torch.bfloat16, "W"), _dptr(Xcal, torch.bfloat16, "Xcal"), T,
+            _dptr(colsq_in, torch.float64, "colsq_in"), PatchShape(N, K, tile_n, tile_k),
+            float(fraction), _dptr(map_in, (torch.int32, torch.uint32), "map_in"), _dptr(meta),
+            _dptr(tmap), _dptr(colsq), _dptr(loss), _stream(stream))
+        _check("patch_score_mask", code)
+    else:
+        code = lib.patch_score_mask_nm(
+            _dptr(W, torch.bfloat16, "W"), _dptr(Xcal, torch.bfloat16, "Xcal"), T,
+            _dptr(colsq_in, torch.float64, "colsq_in"), PatchShape(N, K, tile_n, tile_k),
+            int(nm[0]), int(nm[1]), float(fraction),
+            _dptr(map_in, (torch.int32, torch.uint32), "map_in"), _dptr(meta), _dptr(tmap),
+            _dptr(colsq), _dptr(loss), _stream(stream))
+        _check("patch_score_mask_nm", code)
     return {"meta": meta, "map": tmap, "colsq": colsq, "loss": loss}
 
 
@@ -302,17 +319,27 @@ def patch_select_maps_global(losses: list, fraction: float, stream=None) -> list
 
 
 def patch_pack(W: torch.Tensor, meta: torch.Tensor, tile_map: torch.Tensor, *, tile_n: int = 128,
-               tile_k: int = 128, stream=None) -> PackedWeight:
-    """Compress W (dense tiles + 2:4 tiles) into a library-owned handle."""
+               tile_k: int = 128, nm: tuple = (2, 4), stream=None) -> PackedWeight:
+    """Compress W (dense tiles + 2:4 tiles, or 4:8 tiles with nm=(4, 8)) into a
+    library-owned handle."""
     lib = load_library()
     N, K = W.shape
     out = ctypes.c_void_p(0)
     nbytes = ctypes.c_size_t(0)
-    code = lib.patch_pack(_dptr(W, torch.bfloat16, "W"), _dptr(meta, (torch.int32, torch.uint32), "meta"),
-                          _dptr(tile_map, (torch.int32, torch.uint32), "map"),
-                          PatchShape(N, K, tile_n, tile_k), ctypes.byref(out),
-                          ctypes.byref(nbytes), _stream(stream))
-    _check("patch_pack", code)
+    if tuple(nm) == (2, 4):
+        code = lib.patch_pack(_dptr(W, torch.bfloat16, "W"),
+                              _dptr(meta, (torch.int32, torch.uint32), "meta"),
+                              _dptr(tile_map, (torch.int32, torch.uint32), "map"),
+                              PatchShape(N, K, tile_n, tile_k), ctypes.byref(out),
+                              ctypes.byref(nbytes), _stream(stream))
+        _check("patch_pack", code)
+    else:
+        code = lib.patch_pack_nm(_dptr(W, torch.bfloat16, "W"),
+                                 _dptr(meta, (torch.int32, torch.uint32), "meta"),
+                                 _dptr(tile_map, (torch.int32, torch.uint32), "map"),
+                                 PatchShape(N, K, tile_n, tile_k), int(nm[0]), int(nm[1]),
+                                 ctypes.byref(out), ctypes.byref(nbytes), _stream(stream))
+        _check("patch_pack_nm", code)
     return PackedWeight(out.value, (N, K, tile_n, tile_k), nbytes.value)
 
 
