@@ -311,14 +311,15 @@ def colsq_bytes(T, K):
 
 
 # ----------------------------------------------------------- isolated GEMMs
-def isolated_gemm(P, wl, W, M, frac_map, X, flush, reps=20, seed=0):
+def isolated_gemm(P, wl, W, M, frac_map, X, flush, reps=20, seed=0, nm=(2, 4)):
     """Time one GEMM configuration with L2 flushed before every call.  The
-    2:4 patterns are Wanda's with X as calibration; the map is seeded random."""
+    N:M patterns (2:4, or 4:8) are Wanda's with X as calibration; the map is
+    seeded random."""
     N, K = W.shape
     nt = (N // wl.tile_n) * (K // wl.tile_k)
     tmap = inputs.random_map(nt, inputs.n_sparse_tiles(frac_map, nt), seed).cuda()
-    r = P.patch_score_mask(W, X, tile_n=wl.tile_n, tile_k=wl.tile_k, map_in=tmap)
-    pk = P.patch_pack(W, r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k)
+    r = P.patch_score_mask(W, X, tile_n=wl.tile_n, tile_k=wl.tile_k, map_in=tmap, nm=nm)
+    pk = P.patch_pack(W, r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k, nm=nm)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     for _ in range(3):
         P.patch_hybrid_gemm(pk, X, out=Y)
@@ -432,6 +433,38 @@ def prefill_sweep(P, wl_name, flush, peaks):
                     "burst dense peak (a kernel timed alone); sparse peak = 2 x the dense peak; "
                     "seeded random maps, 2:4 patterns from Wanda with X as calibration; L2 "
                     "flushed before every call"}
+
+
+def nm48_isolated(P, flush, peaks):
+    """4:8 tiles (expanded in shared memory for dense MMAs) against 2:4 and the
+    all-dense map on the Llama-7B MLP shape, half the tiles sparse, one call
+    after an L2 flush: M = 16 (bound by the compressed weight bytes) and
+    M = 2048."""
+    w = inputs.workloads()["llama7b-prefill"]
+    m = w.matrices[0]
+    o = inputs.outlier_channels(m.K, w.seed)
+    Wd = inputs.weight(m.N, m.K, w.seed + m.N).cuda()
+    hbm = float(peaks["hbm_gbs"])
+    out = {}
+    for M in (16, 2048):
+        Xd = inputs.activations(M, m.K, w.seed, o, role=1).cuda()
+        ent = {}
+        for name, f, nm in (("dense", 0.0, (2, 4)), ("2:4 f=0.5", 0.5, (2, 4)), ("4:8 f=0.5", 0.5, (4, 8))):
+            # the same map, the same Wanda ranking; only the pattern differs
+            t_ms, nb = isolated_gemm(P, w, Wd, M, f, Xd, flush, seed=w.seed + 5, nm=nm)
+            e = {"us": t_ms * 1e3, "packed_bytes": nb,
+                 "effective_tflops": 2.0 * M * m.N * m.K / (t_ms * 1e-3) / 1e12}
+            if M <= 16:
+                b = nb + 2 * M * (m.N + m.K)
+                e["achieved_gbs"] = b / (t_ms * 1e-3) / 1e9
+                e["frac_of_hbm"] = e["achieved_gbs"] / hbm
+            ent[name] = e
+        out[f"M={M} N={m.N} K={m.K}"] = ent
+        del Xd
+    return {"by_shape": out,
+            "note": "4:8 handles run the one-band kernel whose converter warps expand 4:8 k-steps "
+                    "into dense tiles in shared memory (no 4:8 tensor-core mode for 16-bit "
+                    "inputs); L2 flushed before every call"}
 
 
 def decode_isolated(P, flush, peaks):
@@ -713,6 +746,7 @@ def main():
     if not args.no_extras and rank == 0 and world == 1:
         extras["prefill_gemm_isolated"] = prefill_sweep(P, wl.name, flush, peaks)
         extras["decode_gemm_isolated"] = decode_isolated(P, flush, peaks)
+        extras["nm48_gemm_isolated"] = nm48_isolated(P, flush, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:

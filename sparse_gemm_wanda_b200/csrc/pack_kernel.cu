@@ -397,7 +397,8 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
                 d0 = mis && (s0 || s1);
                 d1 = mis && (t0 || t1);
                 mp = max(mp, d0 || d1 ? static_cast<unsigned int>(kSidePairBytes)
-                                      : max(kpair_bytes(s0, s1), paired ? kpair_bytes(t0, t1) : 0u));
+                                      : max(kpair_bytes(s0, s1, pattern),
+                                            paired ? kpair_bytes(t0, t1, pattern) : 0u));
             }
             n0 += __popc(__ballot_sync(0xFFFFFFFFu, d0));
             n1 += __popc(__ballot_sync(0xFFFFFFFFu, d1));
@@ -405,8 +406,10 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mp = max(mp, __shfl_xor_sync(0xFFFFFFFFu, mp, o));
         if (lane == 0) {
+            // every band's count is written (a band without a partner, or of a
+            // handle without a prefill table, densifies nothing)
             side_start[b] = n0;
-            if (paired) side_start[b + 1] = n1;
+            if (b + 1 < bands) side_start[b + 1] = paired ? n1 : 0u;
             atomicMax(&pmax_pair, mp);
         }
         __syncwarp();
