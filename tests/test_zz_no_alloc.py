@@ -55,7 +55,9 @@ def call_noalloc(P, w, xc, tn, tk, frac, map_in=None, colsq_in=None, want_loss=T
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     used0, _ = P.pool_usage(reset_high=True)
-    torch_bytes = torch.cuda.memory_allocated()
+    # PyTorch's cumulative count of allocation requests (freeing garbage left
+    # by earlier tests can change the bytes in use, never this count)
+    torch_allocs = torch.cuda.memory_stats()["allocation.all.allocated"]
     code = lib.patch_score_mask_noalloc(
         ctypes.c_void_p(w.data_ptr()), ctypes.c_void_p(xc.data_ptr()) if xc is not None else None,
         xc.shape[0] if xc is not None else 0,
@@ -72,7 +74,7 @@ def call_noalloc(P, w, xc, tn, tk, frac, map_in=None, colsq_in=None, want_loss=T
     # have lifted the mark above the use before the call (the reset may leave
     # the mark below that use, never above it)
     assert used1 == used0 and high <= used0, "the call took memory from the library's pool"
-    assert torch.cuda.memory_allocated() == torch_bytes
+    assert torch.cuda.memory_stats()["allocation.all.allocated"] == torch_allocs
     return {"meta": meta, "map": tmap, "colsq": colsq, "loss": loss}
 
 
