@@ -38,13 +38,16 @@
 //     main loop of the next.
 //   * warps 2..5: epilogue.  tcgen05.ld (each warp its 32-lane quarter), one
 //     rounding to bf16 (or fp32 out), stores to Y, or partials.
-//   * 4:8 handles only (NM = true, 320 threads): warps 6..9, converters.  The
+//   * 4:8 handles only (NM = true, 448 threads): warps 6..13, converters.  The
 //     tensor core has no 4:8 sparse mode for 16-bit inputs, so a 4:8 k-step
 //     (kept values + 8-bit keep masks, 9 KB) lands in its stage's 16 KB region
 //     and the converters rewrite it in place as the dense 128-byte-swizzled
-//     tile (thread = row: read its 32 values and 8 masks, all four warps meet
-//     on an mbarrier, write its 8 chunks of 16 B), then fence to the async
-//     proxy and release the stage to the MMA thread, which issues dense MMAs.
+//     tile: two threads per row, each reads its 4 groups' 16 values and 4
+//     masks, all eight warps meet on an mbarrier (reads before writes), then
+//     each writes its 4 chunks of 16 B, built with two byte permutes per
+//     32-bit word from a 256-entry table (selectors and zero masks per keep
+//     mask) in shared memory; a fence to the async proxy, and the stage goes
+//     to the MMA thread, which issues dense MMAs.
 //
 // Every mbarrier wait is bounded by %globaltimer; when one runs out the CTA
 // raises the status word, drains its copies in flight and returns.
@@ -63,7 +66,9 @@
 namespace patchk {
 
 constexpr int kGemmThreads = 192;
-constexpr int kGemmThreadsNM = 320;  // + 4 converter warps for 4:8 handles
+constexpr int kGemmThreadsNM = 448;  // + 8 converter warps for 4:8 handles
+constexpr int kConvWarps = 8;
+constexpr int kLutBytes = 256 * 32;  // per keep mask: 4 byte-permute selectors, 4 zero masks
 // k-steps of one segment whose table entries are staged in shared memory
 // (K <= 28672)
 constexpr int kMaxTableSteps = 448;
@@ -166,48 +171,48 @@ __device__ __forceinline__ void store_y(const GemmParams &p, int64_t idx, float 
         static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
 }
 
-// One 4:8 k-step of a stage region, in place: 128 rows x (32 kept bf16 at
-// r*64, 8 keep masks at 8192 + r*8) -> 128 x 64 bf16 in the K-major
-// 128-byte-swizzled layout (row r, 16-byte chunk g at r*128 + (g ^ (r%8))*16).
-// Thread `row` holds its row's inputs in `v` (16 words) and `m` (2 words).
-__device__ __forceinline__ void nm48_read(const uint8_t *region, int row, uint32_t (&v)[16],
-                                          uint32_t (&m)[2]) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(region + row * 64);
+// 4:8 expansion.  A stage region holds a 4:8 k-step as 128 rows x (32 kept
+// bf16 at r*64, 8 keep masks at 8192 + r*8); in place it becomes 128 x 64 bf16
+// in the K-major 128-byte-swizzled layout (row r, 16-byte chunk g at
+// r*128 + (g ^ (r%8))*16).  Thread (row, hv) handles groups 4hv .. 4hv+3.
+//
+// The table entry of keep mask m (two uint4): for each 32-bit output word w
+// (positions 2w, 2w+1 of the group) the byte-permute selector that picks the
+// kept values' bytes out of {k01, k23} (the group's four kept values), and the
+// mask that zeroes the pruned half-words.
+__device__ __forceinline__ void nm48_lut_entry(uint32_t m, uint4 *lut) {
+    uint32_t sel[4], zm[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint4 x = src[q];
-        v[4 * q] = x.x;
-        v[4 * q + 1] = x.y;
-        v[4 * q + 2] = x.z;
-        v[4 * q + 3] = x.w;
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t i0 = __popc(m & ((1u << (2 * w)) - 1u)) & 3u;
+        const uint32_t i1 = __popc(m & ((1u << (2 * w + 1)) - 1u)) & 3u;
+        sel[w] = (2 * i0) | ((2 * i0 + 1) << 4) | ((2 * i1) << 8) | ((2 * i1 + 1) << 12);
+        zm[w] = (((m >> (2 * w)) & 1u) ? 0x0000FFFFu : 0u) | (((m >> (2 * w + 1)) & 1u) ? 0xFFFF0000u : 0u);
     }
-    const uint2 mm = *reinterpret_cast<const uint2 *>(region + 8192 + row * 8);
-    m[0] = mm.x;
-    m[1] = mm.y;
+    lut[2 * m] = make_uint4(sel[0] | (sel[1] << 16), sel[2] | (sel[3] << 16), zm[0], zm[1]);
+    lut[2 * m + 1] = make_uint4(zm[2], zm[3], 0u, 0u);
 }
-__device__ __forceinline__ void nm48_write(uint8_t *region, int row, const uint32_t (&v)[16],
-                                           const uint32_t (&m)[2]) {
+__device__ __forceinline__ void nm48_read(const uint8_t *region, int row, int hv, uint32_t (&v)[8],
+                                          uint32_t &m) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(region + row * 64 + hv * 32);
+    const uint4 a = src[0], b = src[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    m = *reinterpret_cast<const uint32_t *>(region + 8192 + row * 8 + hv * 4);
+}
+__device__ __forceinline__ void nm48_write(uint8_t *region, int row, int hv, const uint32_t (&v)[8],
+                                           uint32_t m, const uint4 *lut) {
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        const uint32_t mask = (m[g / 4] >> (8 * (g % 4))) & 0xFFu;
-        // the group's four kept values, in column order
-        const uint32_t k[4] = {v[2 * g] & 0xFFFFu, v[2 * g] >> 16, v[2 * g + 1] & 0xFFFFu,
-                               v[2 * g + 1] >> 16};
-        uint32_t o[4];
-#pragma unroll
-        for (int q2 = 0; q2 < 4; ++q2) {
-            uint32_t h[2];
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                const int q = 2 * q2 + t;
-                const uint32_t idx = __popc(mask & ((1u << q) - 1u));
-                const uint32_t val = idx == 0 ? k[0] : (idx == 1 ? k[1] : (idx == 2 ? k[2] : k[3]));
-                h[t] = ((mask >> q) & 1u) ? val : 0u;
-            }
-            o[q2] = h[0] | (h[1] << 16);
-        }
-        *reinterpret_cast<uint4 *>(region + row * 128 + ((g ^ (row % 8)) * 16)) =
-            make_uint4(o[0], o[1], o[2], o[3]);
+    for (int gg = 0; gg < 4; ++gg) {
+        const uint32_t mask = (m >> (8 * gg)) & 0xFFu;
+        const uint4 e0 = lut[2 * mask], e1 = lut[2 * mask + 1];
+        const uint32_t k01 = v[2 * gg], k23 = v[2 * gg + 1];
+        const uint4 o = make_uint4(__byte_perm(k01, k23, e0.x & 0xFFFFu) & e0.z,
+                                   __byte_perm(k01, k23, e0.x >> 16) & e0.w,
+                                   __byte_perm(k01, k23, e0.y & 0xFFFFu) & e1.x,
+                                   __byte_perm(k01, k23, e0.y >> 16) & e1.y);
+        const int g = 4 * hv + gg;
+        *reinterpret_cast<uint4 *>(region + row * 128 + ((g ^ (row % 8)) * 16)) = o;
     }
 }
 
@@ -223,13 +228,16 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t *tab_buf = reinterpret_cast<uint64_t *>(smem + STAGES * C::kStageBytes);  // [2][kMaxTableSteps]
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::kStageBytes + C::kTabBytes);
+    // 4:8: the expansion table, between the table entries and the barriers
+    uint4 *lut = reinterpret_cast<uint4 *>(smem + STAGES * C::kStageBytes + C::kTabBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * C::kStageBytes + C::kTabBytes +
+                                                  (NM ? kLutBytes : 0));
     uint64_t *empty = full + STAGES;
     uint64_t *acc_full = empty + STAGES;   // [2]
     uint64_t *acc_empty = acc_full + 2;    // [2]
     uint64_t *tab_full = acc_empty + 2;    // [2]
-    uint64_t *conv = tab_full + 2;         // [STAGES] 4:8: stage converted (4 warps)
-    uint64_t *cread = conv + STAGES;       // [STAGES] 4:8: inputs read (4 warps)
+    uint64_t *conv = tab_full + 2;         // [STAGES] 4:8: stage converted (8 warps)
+    uint64_t *cread = conv + STAGES;       // [STAGES] 4:8: inputs read (8 warps)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cread + STAGES);
     volatile uint32_t *abort_flag = tmem_slot + 1;  // raised by any role that gives up
     volatile uint32_t *never_flag = tmem_slot + 2;  // stays 0: time-only bounded waits
@@ -251,8 +259,8 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&conv[s], 4);
-            mbar_init(&cread[s], 4);
+            mbar_init(&conv[s], kConvWarps);
+            mbar_init(&cread[s], kConvWarps);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -278,6 +286,10 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) prefetch_tmap(&tmap_x);
+    if constexpr (NM) {
+        for (int m = static_cast<int>(threadIdx.x) - 192; m >= 0 && m < 256; m += kConvWarps * 32)
+            nm48_lut_entry(static_cast<uint32_t>(m), lut);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -465,9 +477,10 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             if (!skip) {
                 // -------------------------------------------- 4:8 converters
                 // every stage in the MMA's order; a 4:8 k-step is rewritten in
-                // place, so all rows are read (all four warps meet on `cread`)
+                // place, so all rows are read (all eight warps meet on `cread`)
                 // before any row is written
-                const int row = (warp - 6) * 32 + lane;
+                const int t = (warp - 6) * 32 + lane;
+                const int row = t >> 1, hv = t & 1;
                 int it = 0;
                 bool ok = true;
                 Segment sg;
@@ -482,17 +495,17 @@ hybrid_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                         uint8_t *st = smem + s * C::kStageBytes;
                         const bool c0 = (stage_info[3 * s + 0] & kEntryNM48) != 0;
                         const bool c1 = (stage_info[3 * s + 1] & kEntryNM48) != 0;
-                        uint32_t v0[16], m0[2], v1[16], m1[2];
-                        if (c0) nm48_read(st, row, v0, m0);
-                        if (c1) nm48_read(st + kDenseStepBytes, row, v1, m1);
+                        uint32_t v0[8], v1[8], m0 = 0, m1 = 0;
+                        if (c0) nm48_read(st, row, hv, v0, m0);
+                        if (c1) nm48_read(st + kDenseStepBytes, row, hv, v1, m1);
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&cread[s]);
                         if (!mbar_wait_bounded(&cread[s], ph, abort_flag, kWaitLimitNs)) {
                             ok = false;
                             break;
                         }
-                        if (c0) nm48_write(st, row, v0, m0);
-                        if (c1) nm48_write(st + kDenseStepBytes, row, v1, m1);
+                        if (c0) nm48_write(st, row, hv, v0, m0, lut);
+                        if (c1) nm48_write(st + kDenseStepBytes, row, hv, v1, m1, lut);
                         fence_async_shared();  // the generic-proxy writes, visible to the MMA
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&conv[s]);
@@ -694,9 +707,11 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     using C = GemmCfg<BN, STAGES>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
+    constexpr int kSmem = C::kSmemBytes + (NM ? kLutBytes : 0);
+    static_assert(kSmem <= 232448, "shared memory per CTA");
     std::call_once(once, [] {
         attr_err = cudaFuncSetAttribute(hybrid_gemm_kernel<BN, STAGES, NM>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap map;
@@ -744,7 +759,7 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(NM ? kGemmThreadsNM : kGemmThreads);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.dynamicSmemBytes = kSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -775,7 +790,7 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
         // 4:8 handles: the one-band kernel with converter warps, every M
         // (stream-K over (tile, k-pair) units when tiles are few)
         if (g.M <= 64) return run<64, 4, true>(g, 1, stream);
-        return run<160, 3, true>(g, 1, stream);
+        return run<128, 3, true>(g, 1, stream);
     }
     if (g.M <= 16) return launch_decode_gemm(g, stream);  // split-K GEMV, csrc/decode_gemm.cu
     // test hook: one prefill kernel for every M > 16 (parity of each kernel)

@@ -27,7 +27,10 @@
 // 2 KB rows: 16 KB dense, 2 KB metadata + 8 KB kept values, or 8 KB) and its
 // half of the X tile (TMA, 128-byte swizzle, rows past M zero); every load of
 // both CTAs completes on the leader's stage mbarrier (TMA .cta_group::2).
-// Weights and X are issued by two threads in different warps.  The leader's
+// Each band slot and X have an issuing thread of their own (warps 0, 3, 2):
+// the copies one thread issues are processed largely one after another, at
+// about 0.16 us each, which for two weight copies per k-step from one thread
+// would exceed a 2:4 k-step's MMA time.  The leader's
 // MMA thread issues, per pair, 4 dense M256 x BN x K16 or 2 sparse
 // M256 x BN x K32 (after one tcgen05.cp of the pair's metadata block into 4
 // TMEM columns when the k-pair starts); tcgen05.commit with a CTA mask frees
@@ -54,7 +57,7 @@ namespace patchk {
 
 namespace {
 
-constexpr int kQdThreads = 384;     // 12 warps: producers 0 and 2, MMA 1, epilogue 4..11
+constexpr int kQdThreads = 384;     // 12 warps: producers 0, 3 (weights) and 2 (X), MMA 1, epilogue 4..11
 constexpr int kQdMaxStages = 6;
 constexpr int kQdTabSteps = 448;                           // k-steps per band (K <= 28672)
 constexpr int kQdTabBytes = 2 * 2 * kQdTabSteps * 8;       // two items x two bands
@@ -110,8 +113,8 @@ quad_gemm_kernel(const __grid_constant__ QuadMaps maps, const __grid_constant__ 
     uint64_t *empty = full + kQdMaxStages;            // both: freed by the leader's commit
     uint64_t *acc_full = empty + kQdMaxStages;        // both
     uint64_t *acc_empty = acc_full + 1;               // leader: 8 warps x 2 CTAs
-    uint64_t *tab_full = acc_empty + 1;               // [2] own table copies
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tab_full + 2);
+    uint64_t *tab_full = acc_empty + 1;               // [2 buffers][2 slots] own table copies
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tab_full + 4);
     volatile uint32_t *abort_flag = tmem_slot + 1;
     volatile uint32_t *never_flag = tmem_slot + 2;
     uint64_t *stage_info = reinterpret_cast<uint64_t *>(tmem_slot + 4);  // [S][2]: the leader's entries
@@ -124,13 +127,17 @@ quad_gemm_kernel(const __grid_constant__ QuadMaps maps, const __grid_constant__ 
     // pairs of an item: pair 1 is absent in a last quad of only two bands
     auto pairs_of = [&](int item) { return (4 * (item / p.ttiles) + 3 < p.bands) ? 2 : 1; };
     auto band_of = [&](int item, int j) { return 4 * (item / p.ttiles) + 2 * j + static_cast<int>(rank); };
-    auto fetch_table = [&](int item, int buf) {
-        const int np = pairs_of(item);
+    // slot j's table of an item (nothing for an absent pair: a plain arrival)
+    auto fetch_table = [&](int item, int buf, int j) {
+        uint64_t *bar = &tab_full[buf * 2 + j];
+        if (j >= pairs_of(item)) {
+            mbar_arrive(bar);
+            return;
+        }
         const uint32_t nb = static_cast<uint32_t>(p.nsteps) * 8u;
-        mbar_arrive_expect_tx(&tab_full[buf], static_cast<uint32_t>(np) * nb);
-        for (int j = 0; j < np; ++j)
-            bulk_g2s(tab_buf + (buf * 2 + j) * kQdTabSteps,
-                     p.ptable + static_cast<int64_t>(band_of(item, j)) * p.nsteps, nb, &tab_full[buf]);
+        mbar_arrive_expect_tx(bar, nb);
+        bulk_g2s(tab_buf + (buf * 2 + j) * kQdTabSteps,
+                 p.ptable + static_cast<int64_t>(band_of(item, j)) * p.nsteps, nb, bar);
     };
     auto give_up = [&]() {
         *abort_flag = 1u;
@@ -144,13 +151,12 @@ quad_gemm_kernel(const __grid_constant__ QuadMaps maps, const __grid_constant__ 
         // (the packer may be the kernel just before) wait first
         if (ld_acquire_gpu(p.ready) == 0u) pdl_wait();
         for (int s = 0; s < kQdMaxStages; ++s) {
-            mbar_init(&full[s], 2);  // the leader's weight and X producers
+            mbar_init(&full[s], 3);  // the leader's two weight producers and its X producer
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * kQdEpiWarps);
-        mbar_init(&tab_full[0], 1);
-        mbar_init(&tab_full[1], 1);
+        for (int b = 0; b < 4; ++b) mbar_init(&tab_full[b], 1);
         *never_flag = 0u;
         *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
         fence_mbar_init_cluster();
@@ -173,28 +179,29 @@ quad_gemm_kernel(const __grid_constant__ QuadMaps maps, const __grid_constant__ 
     // a CTA that starts with its status raised skips all work but still meets
     // its peer at the end; the peer's waits then run out and it does the same
     const bool skip = *abort_flag != 0;
-    if (threadIdx.x == 0 && !skip) {
-        for (int i = 0; i < 2 && cl + i * C < p.items; ++i) fetch_table(cl + i * C, i);
-    }
 
-    if (warp == 0) {
+    if (warp == 0 || warp == 3) {
         if (lane == 0 && !skip) {
-            // ------------------------------------------------ weight producer
+            // ---------------------------------------- weight producer, slot j
             // (both CTAs; every load completes on the LEADER's stage barrier)
+            const int j = warp == 0 ? 0 : 1;
             int it = 0;
             bool ok = true;
             int tabs = 0;
-            for (int i = 0; i < 2 && cl + i * C < p.items; ++i) ++tabs;
+            for (int i = 0; i < 2 && cl + i * C < p.items; ++i) {
+                fetch_table(cl + i * C, i, j);
+                ++tabs;
+            }
             for (int i = 0; ok; ++i) {
                 const int item = cl + i * C;
                 if (item >= p.items) break;
-                const int buf = i & 1, np = pairs_of(item);
-                if (!mbar_wait_bounded(&tab_full[buf], (i >> 1) & 1u, abort_flag, kQdWaitLimitNs)) {
+                const int buf = i & 1;
+                const bool live = j < pairs_of(item);
+                if (!mbar_wait_bounded(&tab_full[buf * 2 + j], (i >> 1) & 1u, abort_flag, kQdWaitLimitNs)) {
                     ok = false;
                     break;
                 }
-                const uint64_t *tab0 = tab_buf + (buf * 2 + 0) * kQdTabSteps;
-                const uint64_t *tab1 = tab_buf + (buf * 2 + 1) * kQdTabSteps;
+                const uint64_t *tab = tab_buf + (buf * 2 + j) * kQdTabSteps;
                 for (int c = 0; c < p.nsteps; ++c) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
@@ -202,34 +209,28 @@ quad_gemm_kernel(const __grid_constant__ QuadMaps maps, const __grid_constant__ 
                         ok = false;
                         break;
                     }
-                    const uint64_t e0 = tab0[c], e1 = np > 1 ? tab1[c] : 0ull;
-                    stage_info[2 * s + 0] = e0;
-                    stage_info[2 * s + 1] = e1;
+                    const uint64_t e = live ? tab[c] : 0ull;
+                    stage_info[2 * s + j] = e;
                     ++it;
                     if (p.stall_first_kstep && blockIdx.x == 0 && it == 1) continue;  // never lands
-                    const uint32_t b0 = kstep_bytes(e0), b1 = np > 1 ? kstep_bytes(e1) : 0u;
+                    const uint32_t bytes = live ? kstep_bytes(e) : 0u;
                     // the bands of a pair agree in kind and metadata placement,
-                    // so the leader arms the barrier for both CTAs' weight bytes
-                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (b0 + b1));
-                    uint8_t *st = smem + s * p.stage_bytes;
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        if (j >= np) break;
-                        const uint64_t e = j ? e1 : e0;
-                        const uint32_t bytes = j ? b1 : b0;
+                    // so the leader arms the barrier for both CTAs' bytes
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * bytes);
+                    if (live) {
                         const CUtensorMap *am = bytes == kDenseStepBytes ? &maps.a_dense
                                               : (bytes == kSparseStepBytes ? &maps.a_sparse : &maps.a_meta);
-                        tma2d_pair(st + j * kQdAslot, am, 0, static_cast<int32_t>(kstep_first(e) / 2048),
-                                   map_to_rank(&full[s], 0));
+                        tma2d_pair(smem + s * p.stage_bytes + j * kQdAslot, am, 0,
+                                   static_cast<int32_t>(kstep_first(e) / 2048), map_to_rank(&full[s], 0));
                     }
                 }
                 if (ok && cl + (i + 2) * C < p.items) {
-                    fetch_table(cl + (i + 2) * C, buf);
+                    fetch_table(cl + (i + 2) * C, buf, j);
                     ++tabs;
                 }
             }
             for (int q = (tabs > 2 ? tabs - 2 : 0); q < tabs; ++q)
-                mbar_wait_bounded(&tab_full[q & 1], (q >> 1) & 1u, never_flag, kQdWaitLimitNs / 4);
+                mbar_wait_bounded(&tab_full[(q & 1) * 2 + j], (q >> 1) & 1u, never_flag, kQdWaitLimitNs / 4);
             if (!ok) give_up();
             // Drain.  The leader waits for the last phase of every stage (its
             // barrier counts both CTAs' loads); the peer waits until the
