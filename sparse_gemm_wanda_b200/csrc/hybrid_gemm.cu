@@ -817,12 +817,11 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     const double t_one = static_cast<double>(waves1) * 576.0;
     if (g.duo_ok && g.K / kStep <= 448) {
         // two-SM MMAs (through the prefill table, whose band pairs agree in
-        // type) when their estimate is lowest: four bands per CTA pair, else two
+        // type) when their estimate is lowest.  The four-band variant
+        // (prefill_quad.cu) measured slower than this one on the 7B and 13B
+        // MLP shapes (latency-bound at about a third of the tensor pipe), so
+        // it is reached only through the test hook.
         const DuoPlan dp = plan_duo_gemm(g.N, g.M, g.num_sms, g.max_pair_bytes);
-        const QuadPlan qp = plan_quad_gemm(g.N, g.M, g.num_sms);
-        const double best_duo = dp.bn > 0 ? dp.cost : 1e30;
-        if (qp.bn > 0 && qp.cost <= best_duo && qp.cost <= pp.cost && qp.cost <= t_one)
-            return launch_quad_gemm(g, qp, stream);
         if (dp.bn > 0 && dp.cost <= pp.cost && dp.cost <= t_one) return launch_duo_gemm(g, dp, stream);
     }
     if (pp.cost <= t_one && g.K / kStep <= 448)
