@@ -64,6 +64,14 @@ def _load():
             "oracle_pack_bytes_4of8": [p, i64, i64, i64, i64],
             "oracle_pack_4of8": [p, p, p, i64, i64, i64, i64, p, p],
             "oracle_unpack_4of8": [p, p, i64, i64, p],
+            "oracle_e4m3_encode_array": [p, i64, p],
+            "oracle_fp8_row_scales": [p, i64, i64, p],
+            "oracle_fp8_quantize": [p, p, i64, i64, p],
+            "oracle_gemm_fp8": [p, p, p, p, i64, i64, i64, p],
+            "oracle_gemm_fp8_at": [p, p, p, p, i64, p, p, i64, p],
+            "oracle_pack_bytes_fp8": [p, i64, i64, i64, i64],
+            "oracle_pack_fp8": [p, p, p, i64, i64, i64, i64, p, p],
+            "oracle_unpack_fp8": [p, p, i64, i64, p],
         }
         for name, args in sig.items():
             fn = getattr(_lib, name)
@@ -72,6 +80,9 @@ def _load():
         _lib.oracle_n_sparse.restype = i64
         _lib.oracle_pack_bytes.restype = i64
         _lib.oracle_pack_bytes_4of8.restype = i64
+        _lib.oracle_pack_bytes_fp8.restype = i64
+        _lib.oracle_e4m3_decode.argtypes = [ctypes.c_ubyte]
+        _lib.oracle_e4m3_decode.restype = ctypes.c_float
     return _lib
 
 
@@ -293,6 +304,90 @@ def score_mask_4of8(w_bits, xcal_bits=None, tn: int = 128, tk: int = 128, fracti
         tile_map = select_map(loss, n_sparse(fraction, loss.shape[0]))
     return {"colsq": s, "score": sc, "meta": meta, "loss": loss,
             "map": np.ascontiguousarray(tile_map, dtype=np.uint32)}
+
+
+# ------------------------------------------------------ FP8 (e4m3) values
+
+def e4m3_encode(v) -> np.ndarray:
+    """e4m3 codes (uint8) of fp32 values: nearest, ties to the even code, saturating at 448."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _load().oracle_e4m3_encode_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """fp32 values of e4m3 codes."""
+    lib = _load()
+    codes = np.asarray(codes, dtype=np.uint8)
+    table = np.array([lib.oracle_e4m3_decode(c) for c in range(256)], dtype=np.float32)
+    return table[codes]
+
+
+def fp8_row_scales(x_bits) -> np.ndarray:
+    """fp32 scale per row of a bf16 matrix: amax / 448 (1 for a zero row)."""
+    x = _u16(x_bits)
+    R, C = x.shape
+    out = np.empty(R, dtype=np.float32)
+    _load().oracle_fp8_row_scales(_ptr(x), R, C, _ptr(out))
+    return out
+
+
+def fp8_quantize(x_bits, scale) -> np.ndarray:
+    """e4m3 codes of x / scale[row] (the quotient in fp32)."""
+    x = _u16(x_bits)
+    R, C = x.shape
+    scale = np.ascontiguousarray(scale, dtype=np.float32)
+    out = np.empty((R, C), dtype=np.uint8)
+    _load().oracle_fp8_quantize(_ptr(x), _ptr(scale), R, C, _ptr(out))
+    return out
+
+
+def gemm_fp8(qx, sx, qw, sw) -> np.ndarray:
+    """y = sx[m] sw[n] sum_k dec(qx) dec(qw), fp64, k in order."""
+    qx = np.ascontiguousarray(qx, dtype=np.uint8)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    M, K = qx.shape
+    N = qw.shape[0]
+    y = np.empty((M, N), dtype=np.float64)
+    _load().oracle_gemm_fp8(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), M, N, K, _ptr(y))
+    return y
+
+
+def gemm_fp8_at(qx, sx, qw, sw, ms, ns) -> np.ndarray:
+    qx = np.ascontiguousarray(qx, dtype=np.uint8)
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    y = np.empty(ms.shape[0], dtype=np.float64)
+    _load().oracle_gemm_fp8_at(_ptr(qx), _ptr(sx), _ptr(qw), _ptr(sw), qx.shape[1], _ptr(ms), _ptr(ns),
+                               ms.shape[0], _ptr(y))
+    return y
+
+
+def pack_fp8(qw, meta, tile_map, tn: int, tk: int):
+    """Packed bytes and k-step table of an FP8 handle from the codes of W_eff."""
+    qw = np.ascontiguousarray(qw, dtype=np.uint8)
+    N, K = qw.shape
+    meta = np.ascontiguousarray(meta, dtype=np.uint32)
+    tile_map = np.ascontiguousarray(tile_map, dtype=np.uint32)
+    nbytes = int(_load().oracle_pack_bytes_fp8(_ptr(tile_map), N, K, tn, tk))
+    out = np.zeros(nbytes, dtype=np.uint8)
+    table = np.zeros((N // 128) * (K // 128), dtype=np.uint64)
+    _load().oracle_pack_fp8(_ptr(qw), _ptr(meta), _ptr(tile_map), N, K, tn, tk, _ptr(out), _ptr(table))
+    return out, table
+
+
+def unpack_fp8(packed, table, N: int, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    table = np.ascontiguousarray(table, dtype=np.uint64)
+    out = np.zeros((N, K), dtype=np.uint8)
+    _load().oracle_unpack_fp8(_ptr(packed), _ptr(table), N, K, _ptr(out))
+    return out
 
 
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:

@@ -700,3 +700,250 @@ void oracle_unpack_4of8(const uint8_t *packed, const uint64_t *table, int64_t N,
             }
         }
 }
+
+/* ------------------------------------------------------------------ */
+/* FP8 (e4m3) values inside dense and 2:4 tiles                         */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Prune first, then quantise ("SparseGPT vs Wanda: one-shot LLM pruning
+ * without retraining", FAQ on combining pruning with quantisation: prune,
+ * then quantise the surviving weights).  Here the Wanda 2:4 codes and the
+ * tile map are decided on the bf16 weights exactly as above; W_eff (kept
+ * entries, zeros elsewhere) is then quantised to FP8 e4m3 with one fp32
+ * scale per output row, and the activations X with one fp32 scale per
+ * token.  The product is
+ *     y[m,n] = sx[m] * sw[n] * sum_k dec(qx[m,k]) * dec(qw[n,k]).
+ *
+ * e4m3 (the OCP 8-bit floating-point format, "fn" variant): sign, 4 exponent
+ * bits (bias 7), 3 mantissa bits, no infinities; code 0x7F/0xFF is NaN; the
+ * largest finite value is 448, the smallest subnormal 2^-9.  Encoding rounds
+ * to nearest, ties to the even code, and saturates at +-448.
+ *
+ * Scales and the quotient x / s are fp32 (IEEE single, round to nearest):
+ *     s = amax / 448 (amax = largest |value| of the row; s = 1 when amax = 0)
+ *     q = enc(x / s).
+ * Where floating point decides an integer code, both this oracle and the GPU
+ * take that decision in fp32 with these exact operations.
+ */
+static float e4m3_decode_value(unsigned c) {
+    unsigned e = (c >> 3) & 0xFu, m = c & 7u;
+    float v = (e == 0) ? (float)m * 0.001953125f /* 2^-9 */
+                       : ldexpf((float)(8u + m), (int)e - 10);
+    return (c & 0x80u) ? -v : v;
+}
+
+/* The 127 non-negative finite values in increasing order: code i has value
+ * table[i] for i = 0 .. 126 (0x7F is NaN). */
+static float g_e4m3_table[127];
+static int g_e4m3_ready = 0;
+
+static void e4m3_init(void) {
+    if (g_e4m3_ready) return;
+    for (unsigned c = 0; c < 127; ++c) g_e4m3_table[c] = e4m3_decode_value(c);
+    g_e4m3_ready = 1;
+}
+
+unsigned char oracle_e4m3_encode(float v) {
+    e4m3_init();
+    unsigned sign = (v < 0.0f || (v == 0.0f && signbit(v))) ? 0x80u : 0u;
+    float a = fabsf(v);
+    if (!(a == a)) return 0x7F; /* NaN in, NaN out (not used by the path) */
+    if (a >= 448.0f) return (unsigned char)(sign | 0x7Eu);
+    /* largest code with value <= a (binary search), then the nearer of it and
+     * the next one; a tie goes to the even code */
+    int lo = 0, hi = 126;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if (g_e4m3_table[mid] <= a) lo = mid; else hi = mid - 1;
+    }
+    unsigned c = (unsigned)lo;
+    if (g_e4m3_table[c] != a) {
+        double below = (double)a - (double)g_e4m3_table[c];
+        double above = (double)g_e4m3_table[c + 1] - (double)a;
+        if (above < below || (above == below && ((c + 1) & 1u) == 0)) c = c + 1;
+    }
+    return (unsigned char)(sign | c);
+}
+
+float oracle_e4m3_decode(unsigned char c) { return e4m3_decode_value(c); }
+
+void oracle_e4m3_encode_array(const float *v, int64_t n, uint8_t *out) {
+    e4m3_init();
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(v[i]);
+}
+
+/* Row scales of a bf16 matrix [R, C]: s = amax / 448 in fp32 (1 for a zero row). */
+void oracle_fp8_row_scales(const uint16_t *x, int64_t R, int64_t C, float *scale) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        float amax = 0.0f;
+        for (int64_t c = 0; c < C; ++c) {
+            float a = fabsf((float)bf16_bits_to_f64(x[r * C + c]));
+            if (a > amax) amax = a;
+        }
+        scale[r] = amax > 0.0f ? amax / 448.0f : 1.0f;
+    }
+}
+
+/* q[r,c] = enc(x[r,c] / scale[r]), the quotient in fp32. */
+void oracle_fp8_quantize(const uint16_t *x, const float *scale, int64_t R, int64_t C, uint8_t *q) {
+    e4m3_init();
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t c = 0; c < C; ++c) {
+            float v = (float)bf16_bits_to_f64(x[r * C + c]);
+            float quot = v / scale[r];
+            q[r * C + c] = oracle_e4m3_encode(quot);
+        }
+}
+
+/* y[m,n] = sx[m] * sw[n] * sum_k dec(qx[m,k]) * dec(qw[n,k]); fp64, k in order. */
+void oracle_gemm_fp8(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw,
+                     int64_t M, int64_t N, int64_t K, double *y) {
+    e4m3_init();
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc = acc + (double)e4m3_decode_value(qx[m * K + k]) *
+                                (double)e4m3_decode_value(qw[n * K + k]);
+            y[m * N + n] = (double)sx[m] * (double)sw[n] * acc;
+        }
+}
+
+/* The same sums at listed (m, n) positions only. */
+void oracle_gemm_fp8_at(const uint8_t *qx, const float *sx, const uint8_t *qw, const float *sw,
+                        int64_t K, const int64_t *ms, const int64_t *ns, int64_t count, double *y) {
+    e4m3_init();
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i) {
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k)
+            acc = acc + (double)e4m3_decode_value(qx[ms[i] * K + k]) *
+                            (double)e4m3_decode_value(qw[ns[i] * K + k]);
+        y[i] = (double)sx[ms[i]] * (double)sw[ns[i]] * acc;
+    }
+}
+
+/*
+ * Packed layout of an FP8 handle (this library's own format, stated in
+ * include/patch.h).  Bands of 128 rows; k-steps of 128 columns (128 bytes of
+ * e4m3 per row).  A k-step is 2:4-compressed iff every map tile overlapping
+ * it is a 2:4 tile; otherwise dense (the codes of W_eff).
+ *   - dense k-step: 16384 bytes, code (r, k) at
+ *       (r/8)*1024 + (r%8)*128 + ((k/16) ^ (r%8))*16 + k%16.
+ *   - 2:4 k-step: a 2048-byte metadata block, then 8192 bytes of kept codes:
+ *     kept code v (v < 64, column order, two per group) of row r at
+ *       (r/8)*512 + (r%8)*64 + ((v/16) ^ ((r%8)/2))*16 + v%16;
+ *     metadata: for row m = m0 + 8*m1 + 16*m2 (m0<8, m1<2, m2<8) and column
+ *     k = k0 + 16*k1 + 32*k2 (k0<16, k1<2, k2<4) of the k-step, the code bit
+ *     of column k is in 16-byte line m0 + 8*k1 + 16*m2 at bit 32*k2 + 16*m1 + k0
+ *     (the 16-bit handles' placement over the k-step's 128 columns).
+ *   - table[b*(K/128) + c] (uint64): bits 0..47 offset of the k-step's codes
+ *     (after its metadata block for 2:4), bit 62 = 2:4.
+ */
+#define KSTEP8 128
+
+static int kstep8_sparse(const uint32_t *map, int64_t K, int64_t tn, int64_t tk, int64_t b,
+                         int64_t c) {
+    int64_t tiles_k = K / tk;
+    for (int64_t ti = (b * BAND) / tn; ti <= (b * BAND + BAND - 1) / tn; ++ti)
+        for (int64_t tj = (c * KSTEP8) / tk; tj <= (c * KSTEP8 + KSTEP8 - 1) / tk; ++tj)
+            if (!tile_is_sparse(map, ti * tiles_k + tj)) return 0;
+    return 1;
+}
+
+int64_t oracle_pack_bytes_fp8(const uint32_t *map, int64_t N, int64_t K, int64_t tn, int64_t tk) {
+    int64_t total = 0;
+    for (int64_t b = 0; b < N / BAND; ++b)
+        for (int64_t c = 0; c < K / KSTEP8; ++c)
+            total += kstep8_sparse(map, K, tn, tk, b, c) ? 2048 + 8192 : 16384;
+    return total;
+}
+
+/* qw: the e4m3 codes of W_eff [N, K] (pruned entries encode +0 = 0x00). */
+void oracle_pack_fp8(const uint8_t *qw, const uint32_t *meta, const uint32_t *map, int64_t N,
+                     int64_t K, int64_t tn, int64_t tk, uint8_t *out, uint64_t *table) {
+    int64_t steps = K / KSTEP8, off = 0;
+    for (int64_t b = 0; b < N / BAND; ++b)
+        for (int64_t c = 0; c < steps; ++c) {
+            if (!kstep8_sparse(map, K, tn, tk, b, c)) {
+                for (int64_t r = 0; r < BAND; ++r)
+                    for (int64_t k = 0; k < KSTEP8; ++k)
+                        out[off + (r / 8) * 1024 + (r % 8) * 128 + (((k / 16) ^ (r % 8)) * 16) + k % 16] =
+                            qw[(b * BAND + r) * K + c * KSTEP8 + k];
+                table[b * steps + c] = (uint64_t)off;
+                off += 16384;
+                continue;
+            }
+            uint8_t *eb = out + off;
+            memset(eb, 0, 2048);
+            for (int64_t m = 0; m < BAND; ++m)
+                for (int64_t k = 0; k < KSTEP8; ++k) {
+                    int64_t i = b * BAND + m, j = c * KSTEP8 + k;
+                    uint32_t word = meta[i * (K / 32) + j / 32];
+                    unsigned code = (word >> (4 * ((j % 32) / 4))) & 0xFu;
+                    unsigned bit = (code >> (j % 4)) & 1u;
+                    int64_t m0 = m % 8, m1 = (m / 8) % 2, m2 = m / 16;
+                    int64_t k0 = k % 16, k1 = (k / 16) % 2, k2 = k / 32;
+                    int64_t line = m0 + 8 * k1 + 16 * m2, pos = 32 * k2 + 16 * m1 + k0;
+                    if (bit) eb[line * 16 + pos / 8] |= (uint8_t)(1u << (pos % 8));
+                }
+            off += 2048;
+            for (int64_t r = 0; r < BAND; ++r) {
+                int64_t i = b * BAND + r;
+                int v = 0;
+                for (int64_t k = 0; k < KSTEP8; ++k) {
+                    int64_t j = c * KSTEP8 + k;
+                    if (!kept(meta, K, i, j)) continue;
+                    out[off + (r / 8) * 512 + (r % 8) * 64 + (((v / 16) ^ ((r % 8) / 2)) * 16) + v % 16] =
+                        qw[i * K + j];
+                    ++v;
+                }
+            }
+            table[b * steps + c] = (uint64_t)off | (1ull << 62);
+            off += 8192;
+        }
+}
+
+/* Inverse of oracle_pack_fp8: the codes of W_eff from the packed bytes and table. */
+void oracle_unpack_fp8(const uint8_t *packed, const uint64_t *table, int64_t N, int64_t K,
+                       uint8_t *qw) {
+    int64_t steps = K / KSTEP8;
+    for (int64_t b = 0; b < N / BAND; ++b)
+        for (int64_t c = 0; c < steps; ++c) {
+            uint64_t e = table[b * steps + c];
+            int64_t off = (int64_t)(e & ((1ull << 48) - 1));
+            for (int64_t r = 0; r < BAND; ++r) {
+                uint8_t *dst = qw + (b * BAND + r) * K + c * KSTEP8;
+                if (!((e >> 62) & 1u)) {
+                    for (int64_t k = 0; k < KSTEP8; ++k)
+                        dst[k] = packed[off + (r / 8) * 1024 + (r % 8) * 128 + (((k / 16) ^ (r % 8)) * 16) + k % 16];
+                    continue;
+                }
+                const uint8_t *eb = packed + off - 2048;
+                int v = 0;
+                for (int64_t k = 0; k < KSTEP8; ++k) {
+                    int64_t m0 = r % 8, m1 = (r / 8) % 2, m2 = r / 16;
+                    int64_t k0 = k % 16, k1 = (k / 16) % 2, k2 = k / 32;
+                    int64_t line = m0 + 8 * k1 + 16 * m2, pos = 32 * k2 + 16 * m1 + k0;
+                    int64_t gpos = pos - (k0 % 4);
+                    unsigned code = 0;
+                    for (int q = 0; q < 4; ++q) {
+                        int64_t p = gpos + q;
+                        code |= ((eb[line * 16 + p / 8] >> (p % 8)) & 1u) << q;
+                    }
+                    unsigned here = (unsigned)(k % 4);
+                    uint8_t w = 0;
+                    if (here == (code & 3u) || here == (code >> 2)) {
+                        w = packed[off + (r / 8) * 512 + (r % 8) * 64 + (((v / 16) ^ ((r % 8) / 2)) * 16) + v % 16];
+                        ++v;
+                    }
+                    dst[k] = w;
+                }
+            }
+        }
+}

@@ -622,3 +622,123 @@ def test_pack_4of8_round_trip_and_bytes(oracle_mod, tn, tk, frac):
     total = (N // 128) * (K // 64)
     assert packed.size == 9216 * sparse_steps + 16384 * (total - sparse_steps)
     assert int(((table >> np.uint64(60)) & np.uint64(1)).sum()) == sparse_steps
+
+
+# ----------------------------------------------------------------------------
+# FP8 (e4m3) values ("SparseGPT vs Wanda", FAQ: prune first, then quantise)
+# ----------------------------------------------------------------------------
+
+def torch_e4m3(v):
+    """PyTorch's float8_e4m3fn cast (nearest, ties to even), clamped to +-448
+    first so that the library's overflow-to-NaN becomes the saturation the
+    oracle defines."""
+    t = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32)).clamp(-448.0, 448.0)
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_encode_every_bf16_value(oracle_mod):
+    bits = np.arange(65536, dtype=np.uint32)
+    v = (bits << 16).view(np.float32)
+    v = v[~np.isnan(v)]
+    got = oracle_mod.e4m3_encode(v)
+    ref = torch_e4m3(v)
+    # +-0 and values rounding to zero: the library keeps the sign of zero too
+    assert np.array_equal(got, ref)
+
+
+def test_e4m3_encode_random_quotients(oracle_mod):
+    g = np.random.default_rng(8)
+    x = np.concatenate([g.uniform(-460, 460, 200000), g.uniform(-0.02, 0.02, 100000),
+                        g.standard_normal(100000) * 30]).astype(np.float32)
+    assert np.array_equal(oracle_mod.e4m3_encode(x), torch_e4m3(x))
+
+
+def test_e4m3_decode_every_code(oracle_mod):
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+    assert np.array_equal(oracle_mod.e4m3_decode(codes), ref)
+    assert oracle_mod.e4m3_decode(np.array([0x7E], dtype=np.uint8))[0] == 448.0
+    assert oracle_mod.e4m3_decode(np.array([0x01], dtype=np.uint8))[0] == 2.0 ** -9
+
+
+def test_fp8_row_scales_closed_form(oracle_mod):
+    x = np.zeros((3, 64), dtype=np.float32)
+    x[0, 5] = -7.0
+    x[0, 9] = 3.0
+    x[2, :] = 448.0
+    s = oracle_mod.fp8_row_scales(to_bits(x))
+    assert s[0] == np.float32(7.0) / np.float32(448.0)
+    assert s[1] == 1.0          # a zero row: scale 1, every code 0
+    assert s[2] == 1.0          # amax 448: scale exactly 1
+    q = oracle_mod.fp8_quantize(to_bits(x), s)
+    assert np.all(q[1] == 0) and np.all(q[2] == 0x7E)
+    assert oracle_mod.e4m3_decode(q[0, 5:6])[0] * s[0] == -7.0
+
+
+def test_fp8_quantize_representable_values_exactly(oracle_mod):
+    # rows whose largest magnitude is 448 have scale 1; values that e4m3 holds
+    # exactly come back unchanged
+    g = np.random.default_rng(2)
+    codes = g.integers(0, 0x7F, size=(16, 128)).astype(np.uint8)
+    codes[:, 0] = 0x7E  # 448 in every row
+    vals = oracle_mod.e4m3_decode(codes) * np.where(g.random((16, 128)) < 0.5, -1, 1)
+    q = oracle_mod.fp8_quantize(to_bits(vals), oracle_mod.fp8_row_scales(to_bits(vals)))
+    assert np.array_equal(oracle_mod.e4m3_decode(q), vals.astype(np.float32))
+
+
+def test_fp8_quantize_error_bound(oracle_mod):
+    # |dec(q) s - x| <= s * (half the e4m3 spacing at |x/s|) + fp32 rounding
+    g = torch.Generator().manual_seed(4)
+    x = (torch.randn(64, 256, generator=g) * 0.05).to(torch.bfloat16)
+    xb = bf16_bits(x)
+    s = oracle_mod.fp8_row_scales(xb)
+    q = oracle_mod.fp8_quantize(xb, s)
+    xv = oracle_mod.bf16_bits_to_f64(xb)
+    a = np.abs(xv / s[:, None])
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))
+    spacing = np.exp2(e - 3)  # normal spacing; the subnormal spacing is 2^-9 = 2^(-6-3)
+    err = np.abs(oracle_mod.e4m3_decode(q).astype(np.float64) * s[:, None] - xv)
+    assert np.all(err <= s[:, None] * (0.5 * spacing * (1 + 1e-6)) + 1e-12)
+
+
+def test_gemm_fp8_equals_numpy_on_decoded_codes(oracle_mod):
+    g = np.random.default_rng(6)
+    qx = g.integers(0, 0x7F, size=(5, 96)).astype(np.uint8) | (g.integers(0, 2, size=(5, 96)) << 7).astype(np.uint8)
+    qw = g.integers(0, 0x7F, size=(7, 96)).astype(np.uint8)
+    sx = g.uniform(0.01, 2, 5).astype(np.float32)
+    sw = g.uniform(0.01, 2, 7).astype(np.float32)
+    y = oracle_mod.gemm_fp8(qx, sx, qw, sw)
+    ref = (sx[:, None].astype(np.float64) * sw[None, :].astype(np.float64)) * (
+        oracle_mod.e4m3_decode(qx).astype(np.float64) @ oracle_mod.e4m3_decode(qw).astype(np.float64).T)
+    assert np.allclose(y, ref, rtol=1e-12, atol=0)
+    ms, ns = np.array([0, 4, 2]), np.array([6, 0, 3])
+    assert np.array_equal(oracle_mod.gemm_fp8_at(qx, sx, qw, sw, ms, ns), y[ms, ns])
+
+
+@pytest.mark.parametrize("tn,tk", [(128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
+def test_pack_fp8_round_trip_and_bytes(oracle_mod, tn, tk, frac):
+    from sparse_gemm_wanda_b200 import inputs
+    N, K = 256, 512
+    w = inputs.weight(N, K, 4)
+    wb = bf16_bits(w)
+    sc = np.abs(oracle_mod.bf16_bits_to_f64(wb))
+    meta = oracle_mod.select_2of4(sc)
+    nt = (N // tn) * (K // tk)
+    tmap = inputs.random_map(nt, int(frac * nt), 6).numpy().view(np.uint32)
+    weff = oracle_mod.weff(wb, meta, tmap, tn, tk)
+    qw = oracle_mod.fp8_quantize(weff, oracle_mod.fp8_row_scales(weff))
+    packed, table = oracle_mod.pack_fp8(qw, meta, tmap, tn, tk)
+    back = oracle_mod.unpack_fp8(packed, table, N, K)
+    # pruned entries quantise to code 0 and come back as 0
+    assert np.array_equal(back, qw)
+    sparse = 0
+    for b in range(N // 128):
+        for c in range(K // 128):
+            rows = range((128 * b) // tn, (128 * b + 127) // tn + 1)
+            cols = range((128 * c) // tk, (128 * c + 127) // tk + 1)
+            if all((tmap[(r * (K // tk) + q) // 32] >> ((r * (K // tk) + q) % 32)) & 1
+                   for r in rows for q in cols):
+                sparse += 1
+    total = (N // 128) * (K // 128)
+    assert packed.size == 10240 * sparse + 16384 * (total - sparse)
