@@ -838,10 +838,11 @@ void oracle_gemm_fp8_at(const uint8_t *qx, const float *sx, const uint8_t *qw, c
  *   - 2:4 k-step: a 2048-byte metadata block, then 8192 bytes of kept codes:
  *     kept code v (v < 64, column order, two per group) of row r at
  *       (r/8)*512 + (r%8)*64 + ((v/16) ^ ((r%8)/2))*16 + v%16;
- *     metadata: for row m = m0 + 8*m1 + 16*m2 (m0<8, m1<2, m2<8) and column
- *     k = k0 + 16*k1 + 32*k2 (k0<16, k1<2, k2<4) of the k-step, the code bit
- *     of column k is in 16-byte line m0 + 8*k1 + 16*m2 at bit 32*k2 + 16*m1 + k0
- *     (the 16-bit handles' placement over the k-step's 128 columns).
+ *     metadata: 16-byte line m holds row m; bit k (k < 128, LSB first) is the
+ *     code bit of column k of the k-step (a group's 4-bit code over its four
+ *     columns, LSB first).  This is the tensor-memory layout the sparse MMA
+ *     for 8-bit inputs reads (one lane per row, one bit per K column), not
+ *     the interleaved one of the 16-bit handles.
  *   - table[b*(K/128) + c] (uint64): bits 0..47 offset of the k-step's codes
  *     (after its metadata block for 2:4), bit 62 = 2:4.
  */
@@ -887,10 +888,7 @@ void oracle_pack_fp8(const uint8_t *qw, const uint32_t *meta, const uint32_t *ma
                     uint32_t word = meta[i * (K / 32) + j / 32];
                     unsigned code = (word >> (4 * ((j % 32) / 4))) & 0xFu;
                     unsigned bit = (code >> (j % 4)) & 1u;
-                    int64_t m0 = m % 8, m1 = (m / 8) % 2, m2 = m / 16;
-                    int64_t k0 = k % 16, k1 = (k / 16) % 2, k2 = k / 32;
-                    int64_t line = m0 + 8 * k1 + 16 * m2, pos = 32 * k2 + 16 * m1 + k0;
-                    if (bit) eb[line * 16 + pos / 8] |= (uint8_t)(1u << (pos % 8));
+                    if (bit) eb[m * 16 + k / 8] |= (uint8_t)(1u << (k % 8));
                 }
             off += 2048;
             for (int64_t r = 0; r < BAND; ++r) {
@@ -927,14 +925,11 @@ void oracle_unpack_fp8(const uint8_t *packed, const uint64_t *table, int64_t N, 
                 const uint8_t *eb = packed + off - 2048;
                 int v = 0;
                 for (int64_t k = 0; k < KSTEP8; ++k) {
-                    int64_t m0 = r % 8, m1 = (r / 8) % 2, m2 = r / 16;
-                    int64_t k0 = k % 16, k1 = (k / 16) % 2, k2 = k / 32;
-                    int64_t line = m0 + 8 * k1 + 16 * m2, pos = 32 * k2 + 16 * m1 + k0;
-                    int64_t gpos = pos - (k0 % 4);
+                    int64_t gpos = k - (k % 4);
                     unsigned code = 0;
                     for (int q = 0; q < 4; ++q) {
                         int64_t p = gpos + q;
-                        code |= ((eb[line * 16 + p / 8] >> (p % 8)) & 1u) << q;
+                        code |= ((eb[r * 16 + p / 8] >> (p % 8)) & 1u) << q;
                     }
                     unsigned here = (unsigned)(k % 4);
                     uint8_t w = 0;

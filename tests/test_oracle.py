@@ -732,6 +732,16 @@ def test_pack_fp8_round_trip_and_bytes(oracle_mod, tn, tk, frac):
     back = oracle_mod.unpack_fp8(packed, table, N, K)
     # pruned entries quantise to code 0 and come back as 0
     assert np.array_equal(back, qw)
+    # a 2:4 k-step's metadata block: line m, bit k is bit k%4 of the 4-bit code
+    # of row m's group k//4 (so the line's 32-bit words are the row's meta words)
+    for b in range(N // 128):
+        for c in range(K // 128):
+            e = int(table[b * (K // 128) + c])
+            if not (e >> 62) & 1:
+                continue
+            off = e & ((1 << 48) - 1)
+            block = packed[off - 2048:off].view(np.uint32).reshape(128, 4)
+            assert np.array_equal(block, meta[128 * b:128 * b + 128, 4 * c:4 * c + 4])
     sparse = 0
     for b in range(N // 128):
         for c in range(K // 128):
