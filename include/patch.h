@@ -308,6 +308,54 @@ patch_status patch_pack_nm(const void *W_bf16, const uint32_t *meta, const uint3
                            size_t *packed_bytes, void *stream);
 
 /*
+ * FP8 values inside dense and 2:4 tiles ("SparseGPT vs Wanda: one-shot LLM
+ * pruning without retraining", FAQ: pruning combines with quantisation,
+ * prune first, then quantise).  The Wanda 2:4 codes and the tile map come
+ * from patch_score_mask as for bf16; W_eff is then quantised to e4m3 with one
+ * fp32 scale per output row, and patch_hybrid_gemm on the handle quantises X
+ * with one fp32 scale per token (each call, into pool scratch of M*K + 4*M
+ * bytes) and computes
+ *     Y[m,n] = sx[m] * sw[n] * sum_k dec(qx[m,k]) * dec(qw[n,k])
+ * on the tensor cores (tcgen05 kind::f8f6f4: dense MMAs for dense k-steps,
+ * the sparse MMA for 2:4 k-steps), fp32 accumulation, one rounding.
+ * Quantisation of a row: s = amax / 448 in fp32 (1 for an all-zero row);
+ * q = e4m3(x / s) with the quotient in fp32, rounded to nearest with ties to
+ * the even code, saturating at +-448.
+ *
+ * patch_pack_fp8: W_bf16, meta, map, shp as patch_pack (K a multiple of 128).
+ * Synchronises once (it reads the map back to plan the layout).  Packed
+ * format (normative): bands of 128 rows, k-steps of 128 columns; a k-step is
+ * 2:4 iff every map tile overlapping it is 2:4, otherwise dense (codes of
+ * W_eff);
+ *   - dense k-step: 16384 bytes, code (r,k) at
+ *     (r/8)*1024 + (r%8)*128 + ((k/16) ^ (r%8))*16 + k%16;
+ *   - 2:4 k-step: a 2048-byte metadata block (16-byte line m holds row m's
+ *     code bits, bit k = bit k%4 of the 4-bit code of column group k/4: the
+ *     row's four meta words for these columns), then 8192 bytes of kept
+ *     codes, kept code v (v < 64, column order) of row r at
+ *     (r/8)*512 + (r%8)*64 + ((v/16) ^ ((r%8)/2))*16 + v%16;
+ *   - table[b*(K/128)+c] (uint64): bits 0..47 offset of the k-step's codes,
+ *     bit 62 = 2:4.
+ * Errors as patch_pack.
+ */
+patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
+                            patch_shape shp, patch_packed **out, size_t *packed_bytes,
+                            void *stream);
+
+/*
+ * The per-row e4m3 quantisation above, on its own: X_bf16 [R,C] (16-byte
+ * aligned, C a multiple of 8) -> codes_out [R,C] uint8 (8-byte aligned) and
+ * scales_out [R] fp32.  Stream-ordered, no scratch.  Errors: INVALID_ARG,
+ * UNSUPPORTED, CUDA.
+ */
+patch_status patch_quantize_fp8(const void *X_bf16, int64_t R, int64_t C, uint8_t *codes_out,
+                                float *scales_out, void *stream);
+
+/* Copy an FP8 handle's W_eff row scales ([N] fp32) to scales_dst (device),
+ * stream-ordered.  INVALID_ARG for other handles. */
+patch_status patch_packed_fp8_scales(const patch_packed *Wp, float *scales_dst, void *stream);
+
+/*
  * Hybrid product Y[M,N] = X[M,K] * W_eff^T with fp32 accumulation in tensor
  * memory and one rounding at the end (PATCH page, section 2, inference and
  * deployment: one kernel over mixed dense / 2:4 tiles).  Dense k-steps issue
@@ -376,7 +424,8 @@ patch_status patch_packed_info(const patch_packed *Wp, patch_packed_view *view);
 
 /*
  * Copy a handle's packed bytes (view.packed_bytes) and k-step table
- * ((N/128)*(K/64) uint64) into caller-owned DEVICE buffers, stream-ordered.
+ * ((N/128)*(K/64) uint64; (N/128)*(K/128) for FP8 handles) into caller-owned
+ * DEVICE buffers, stream-ordered.
  * Either destination may be NULL to skip it.  For inspection and tests.
  */
 patch_status patch_packed_export(const patch_packed *Wp, void *packed_dst, uint64_t *table_dst,

@@ -1,0 +1,357 @@
+// FP8 hybrid GEMM on the sm_100a tensor cores: Y = diag(sx) (QX QW^T) diag(sw).
+//
+// FP8 values inside dense and 2:4 tiles ("SparseGPT vs Wanda: one-shot LLM
+// pruning without retraining", FAQ: prune first, then quantise; the tile
+// scheme of "PATCH: Learnable Tile-level Hybrid Sparsity for LLMs", section
+// 2): dense k-steps issue tcgen05.mma kind::f8f6f4 (4 x M128 N=BN K32 per
+// 128-column k-step), 2:4 k-steps tcgen05.mma.sp kind::f8f6f4 (2 x M128 N=BN
+// K64, after one tcgen05.cp of the k-step's metadata block into 4 TMEM
+// columns; the metadata of sparse MMA q sits at TMEM column 2q with selector
+// 0).  Both e4m3, fp32 accumulation in tensor memory; the epilogue multiplies
+// by the token's and the output row's fp32 scales and rounds once.
+//
+// Work: an output tile is one 128-row band x BN tokens; persistent CTAs take
+// tiles c, c + P, ...; two accumulators alternate so one tile's epilogue
+// overlaps the next tile's main loop.  A stage is one k-step: one bulk copy of
+// its packed bytes (16 KB dense, or 2 KB metadata + 8 KB kept codes) and one
+// TMA load of the BN x 128-byte X tile (128-byte swizzle, rows past M zero).
+// Roles (192 threads): warp 0 lane 0 producer, warp 1 lane 0 MMA (warp 1 also
+// allocates tensor memory), warps 2..5 epilogue.  Every mbarrier wait is
+// bounded by %globaltimer; a wait that runs out raises the handle's status.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "patch_common.cuh"
+#include "patch_internal.h"
+
+namespace patchk {
+
+namespace {
+
+constexpr int kF8Threads = 192;
+constexpr int kF8Step = 128;                 // columns (bytes of codes) per k-step
+constexpr int kF8Aslot = kDenseStepBytes;    // 16 KB: a dense k-step, or metadata + kept codes
+constexpr int kF8SmemLimit = 232448;
+constexpr int kF8MaxStages = 8;
+constexpr uint64_t kF8WaitLimitNs = 2000000000ull;
+
+struct F8Params {
+    const uint8_t *packed;
+    const uint64_t *table;   // [bands][K/128]
+    const float *sw;         // [N] weight row scales
+    const float *sx;         // [M] token scales
+    int64_t N, K, M;
+    int steps, bands, ttiles, tiles;
+    void *Y;
+    int y_fp32;
+    uint32_t *status;
+};
+
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_f8_sparse(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// kind::f8f6f4 instruction descriptor: A and B e4m3 (format 0), K-major, fp32
+// D, M = 128, the given N; `sparse` sets the 2:4 flag (selector 0).
+__host__ __device__ constexpr uint32_t idesc_e4m3(int n, bool sparse) {
+    return (sparse ? (1u << 2) : 0u) | (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void store_y(const F8Params &p, int64_t idx, float v) {
+    if (p.y_fp32)
+        static_cast<float *>(p.Y)[idx] = v;
+    else
+        static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
+}
+
+template <int BN>
+struct F8Cfg {
+    static constexpr int kXBytes = BN * kF8Step;
+    static constexpr int kStageBytes = kF8Aslot + kXBytes;
+    static constexpr int kTail = 1024 + 512;
+    static constexpr int kStages = std::min(kF8MaxStages, (kF8SmemLimit - kTail) / kStageBytes);
+    static constexpr int kSmem = kStages * kStageBytes + kTail;
+    static constexpr int kCols = 2 * BN + 4;
+    static constexpr int kTmemCols = kCols <= 128 ? 128 : (kCols <= 256 ? 256 : 512);
+    static_assert(kStages >= 2, "at least two stages");
+    static_assert(kXBytes % 1024 == 0, "stage regions stay 1024-B aligned");
+    static_assert(kCols <= 512, "tensor memory holds 512 columns");
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kF8Threads, 1)
+fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ F8Params p) {
+    using C = F8Cfg<BN>;
+    constexpr int S = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * C::kStageBytes);
+    uint64_t *empty = full + S;
+    uint64_t *acc_full = empty + S;   // [2]
+    uint64_t *acc_empty = acc_full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+    volatile uint32_t *never_flag = tmem_slot + 2;
+    uint64_t *stage_info = reinterpret_cast<uint64_t *>(tmem_slot + 4);  // [S]
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int cta = blockIdx.x, P = gridDim.x;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        *never_flag = 0u;
+        *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) prefetch_tmap(&tmap_x);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+
+    if (warp == 0) {
+        if (lane == 0 && !skip) {
+            // ------------------------------------------------------ producer
+            int it = 0;
+            bool ok = true;
+            for (int i = 0; ok; ++i) {
+                const int tile = cta + i * P;
+                if (tile >= p.tiles) break;
+                const int band = tile / p.ttiles, tt = tile % p.ttiles;
+                const uint64_t *tab = p.table + static_cast<int64_t>(band) * p.steps;
+                for (int c = 0; c < p.steps; ++c) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (it >= S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kF8WaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint64_t e = __ldg(tab + c);
+                    const bool sp = (e & kEntrySparse) != 0;
+                    const uint64_t first = (e & kEntryOffsetMask) - (sp ? kMetaBlockBytes : 0);
+                    const uint32_t bytes = sp ? kMetaBlockBytes + kSparseStepBytes : kDenseStepBytes;
+                    stage_info[s] = e;
+                    ++it;
+                    uint8_t *st = smem + s * C::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], bytes + C::kXBytes);
+                    bulk_g2s(st, p.packed + first, bytes, &full[s]);
+                    tma_load_2d(st + kF8Aslot, &tmap_x, c * kF8Step, tt * BN, &full[s]);
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1u;
+                atomicOr(p.status, kStatusTimeout);
+            }
+            // the last phase issued on every stage lands before the CTA exits
+            for (int q = (it > S ? it - S : 0); q < it; ++q)
+                mbar_wait_bounded(&full[q % S], (q / S) & 1u, never_flag, kF8WaitLimitNs / 4);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && !skip) {
+            // ---------------------------------------------------------- MMA
+            const uint32_t e_tmem = tmem_base + static_cast<uint32_t>(2 * BN);
+            constexpr uint32_t kIdDense = idesc_e4m3(BN, false);
+            constexpr uint32_t kIdSparse = idesc_e4m3(BN, true);
+            int it = 0;
+            bool ok = true;
+            for (int i = 0; ok; ++i) {
+                const int tile = cta + i * P;
+                if (tile >= p.tiles) break;
+                const int buf = i & 1;
+                if (i >= 2 &&
+                    !mbar_wait_bounded(&acc_empty[buf], ((i >> 1) & 1u) ^ 1u, abort_flag, kF8WaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                for (int c = 0; c < p.steps; ++c, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait_bounded(&full[s], ph, abort_flag, kF8WaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t slot = smem_u32(smem + s * C::kStageBytes);
+                    const uint32_t b_addr = slot + kF8Aslot;
+                    if (stage_info[s] & kEntrySparse) {
+                        tmem_cp_128x128b(e_tmem, smem_desc(slot, 16, 128, kSwizzleNone));
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            const uint64_t ad = smem_desc(slot + kMetaBlockBytes + q * 32, 16, 512, kSwizzle64B);
+                            const uint64_t bd = smem_desc(b_addr + q * 64, 16, 1024, kSwizzle128B);
+                            mma_f8_sparse(d_tmem, ad, bd, e_tmem + 2 * q, kIdSparse, (c == 0 && q == 0) ? 0u : 1u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const uint64_t ad = smem_desc(slot + q * 32, 16, 1024, kSwizzle128B);
+                            const uint64_t bd = smem_desc(b_addr + q * 32, 16, 1024, kSwizzle128B);
+                            mma_f8(d_tmem, ad, bd, kIdDense, (c == 0 && q == 0) ? 0u : 1u);
+                        }
+                    }
+                    tc_commit(&empty[s]);
+                }
+                // fires once every MMA of the tile has completed (also after a
+                // failure, so the epilogue never frees TMEM under a running MMA)
+                tc_commit(&acc_full[buf]);
+            }
+            if (!ok) {
+                *abort_flag = 1u;
+                atomicOr(p.status, kStatusTimeout);
+            }
+        }
+    } else if (!skip) {
+        // ------------------------------------------------------- epilogue
+        const int quad = warp % 4;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+        for (int i = 0;; ++i) {
+            const int tile = cta + i * P;
+            if (tile >= p.tiles) break;
+            const int buf = i & 1;
+            const bool ok = mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1u, never_flag, kF8WaitLimitNs);
+            tc_fence_after();
+            if (!ok) {
+                *abort_flag = 1u;
+                atomicOr(p.status, kStatusTimeout);
+                break;
+            }
+            const int band = tile / p.ttiles, tt = tile % p.ttiles;
+            const int64_t n = static_cast<int64_t>(band) * kBand + row;
+            const int64_t m_base = static_cast<int64_t>(tt) * BN;
+            const int m_valid = static_cast<int>(min(static_cast<int64_t>(BN), p.M - m_base));
+            const float swn = __ldg(p.sw + n);
+            if (*abort_flag == 0) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < m_valid; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(buf * BN + c0), r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        if (c0 + q < m_valid) {
+                            const int64_t m = m_base + c0 + q;
+                            store_y(p, m * p.N + n, __uint_as_float(r[q]) * swn * __ldg(p.sx + m));
+                        }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+template <int BN>
+cudaError_t run_fp8(const Fp8Launch &g, cudaStream_t stream) {
+    using C = F8Cfg<BN>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(fp8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::kSmem);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorInvalidValue;
+    // X codes [M, K] uint8 row-major: box = 128 bytes x BN rows, 128-byte
+    // swizzle, rows past M read as zero
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(g.K), static_cast<cuuint64_t>(g.M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(g.K)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kF8Step), static_cast<cuuint32_t>(BN)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(g.xq), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    F8Params p;
+    p.packed = g.packed;
+    p.table = g.table;
+    p.sw = g.sw;
+    p.sx = g.sx;
+    p.N = g.N;
+    p.K = g.K;
+    p.M = g.M;
+    p.steps = static_cast<int>(g.K / kF8Step);
+    p.bands = static_cast<int>(g.N / kBand);
+    p.ttiles = static_cast<int>((g.M + BN - 1) / BN);
+    p.tiles = p.bands * p.ttiles;
+    p.Y = g.Y;
+    p.y_fp32 = g.y_fp32;
+    p.status = g.status;
+    const int grid = std::min(g.num_sms, p.tiles);
+    fp8_gemm_kernel<BN><<<grid, kF8Threads, C::kSmem, stream>>>(map, p);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fp8_gemm(const Fp8Launch &g, cudaStream_t stream) {
+    if (g.K % kF8Step != 0 || g.N % kBand != 0 || g.M < 1) return cudaErrorInvalidValue;
+    if (g.M <= 64) return run_fp8<64>(g, stream);
+    if (g.M <= 128) return run_fp8<128>(g, stream);
+    return run_fp8<240>(g, stream);
+}
+
+}  // namespace patchk

@@ -20,7 +20,8 @@
 
 struct patch_packed {
     int device;
-    int pattern;               // 2: dense / 2:4 tiles; 4: dense / 4:8 tiles
+    int pattern;               // 2: dense / 2:4 tiles; 4: dense / 4:8 tiles; 8: FP8 dense / 2:4
+    float *fp8_scale;          // FP8 handles: W_eff row scales [N]
     uint8_t *base;             // pool allocation: table, descriptors, prefix, plan, workspace, status
     patch_shape shp;
     uint8_t *packed;           // packed k-steps, then the side copies (a pool allocation of its own, exact size)
@@ -619,6 +620,139 @@ patch_status patch_pack_nm(const void *W_bf16, const uint32_t *meta, const uint3
     return pack_impl(W_bf16, meta, map, shp, out, packed_bytes, stream_v, pattern);
 }
 
+patch_status patch_quantize_fp8(const void *X_bf16, int64_t R, int64_t C, uint8_t *codes_out,
+                                float *scales_out, void *stream_v) {
+    if (!X_bf16 || !codes_out || !scales_out || R < 1 || C < 8 || C % 8 != 0 || !aligned16(X_bf16) ||
+        (reinterpret_cast<uintptr_t>(codes_out) & 7u) != 0 || R > 0x7FFFFFFF)
+        return PATCH_ERR_INVALID_ARG;
+    patch_status st = check_device(nullptr);
+    if (st != PATCH_OK) return st;
+    return from_cuda(patchk::launch_fp8_quantize_rows(X_bf16, R, C, codes_out, scales_out,
+                                                      static_cast<cudaStream_t>(stream_v)));
+}
+
+patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
+                            patch_shape shp, patch_packed **out, size_t *packed_bytes,
+                            void *stream_v) {
+    if (!out) return PATCH_ERR_INVALID_ARG;
+    *out = nullptr;
+    patch_status st = check_shape(shp);
+    if (st != PATCH_OK) return st;
+    if (shp.N % kBand != 0 || shp.K % 128 != 0 || shp.K > 28672) return PATCH_ERR_INVALID_ARG;
+    if (!W_bf16 || !meta || !map || !aligned16(W_bf16) || !aligned16(meta)) return PATCH_ERR_INVALID_ARG;
+    int num_sms = 0;
+    st = check_device(&num_sms);
+    if (st != PATCH_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    const int64_t N = shp.N, K = shp.K, tn = shp.tile_n, tk = shp.tile_k;
+    const int64_t bands = N / kBand, steps = K / 128, tiles_k = K / tk;
+    const int64_t n_tiles = (N / tn) * tiles_k;
+    // the layout is planned on the host from the map (read back in the one
+    // wait of this call): a k-step is 2:4 iff every tile it overlaps is
+    std::vector<uint32_t> hmap(static_cast<size_t>((n_tiles + 31) / 32));
+    cudaError_t e = cudaMemcpyAsync(hmap.data(), map, sizeof(uint32_t) * hmap.size(), cudaMemcpyDeviceToHost,
+                                    stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    auto sparse_tile = [&](int64_t t) { return (hmap[static_cast<size_t>(t / 32)] >> (t % 32)) & 1u; };
+    std::vector<uint64_t> table(static_cast<size_t>(bands * steps));
+    uint64_t off = 0, n_sparse = 0;
+    for (int64_t b = 0; b < bands; ++b)
+        for (int64_t c = 0; c < steps; ++c) {
+            bool sp = true;
+            for (int64_t ti = (b * kBand) / tn; ti <= (b * kBand + kBand - 1) / tn; ++ti)
+                for (int64_t tj = (c * 128) / tk; tj <= (c * 128 + 127) / tk; ++tj)
+                    if (!sparse_tile(ti * tiles_k + tj)) sp = false;
+            if (sp) {
+                table[static_cast<size_t>(b * steps + c)] = (off + patchk::kMetaBlockBytes) | patchk::kEntrySparse;
+                off += patchk::kMetaBlockBytes + patchk::kSparseStepBytes;
+                ++n_sparse;
+            } else {
+                table[static_cast<size_t>(b * steps + c)] = off;
+                off += patchk::kDenseStepBytes;
+            }
+        }
+    patch_packed *h = new (std::nothrow) patch_packed();
+    if (!h) return PATCH_ERR_OOM;
+    cudaGetDevice(&h->device);
+    h->pattern = 8;
+    h->shp = shp;
+    h->num_sms = num_sms;
+    h->bands = bands;
+    h->packed_bytes = off;
+    h->sparse_ksteps = static_cast<int64_t>(n_sparse);
+    h->meta_blocks = static_cast<int64_t>(n_sparse);
+    // allocation 1: table | row scales | status; allocation 2: the packed bytes
+    const size_t off_scale = round_up(sizeof(uint64_t) * table.size(), 256);
+    const size_t off_status = round_up(off_scale + sizeof(float) * static_cast<size_t>(N), 256);
+    const size_t total = off_status + 256;
+    e = patchk::device_pool(&h->pool);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->base), total, h->pool, stream);
+    if (e != cudaSuccess) {
+        delete h;
+        return from_cuda(e);
+    }
+    h->table = reinterpret_cast<uint64_t *>(h->base);
+    h->ptable = h->table;
+    h->fp8_scale = reinterpret_cast<float *>(h->base + off_scale);
+    h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
+    e = cudaMemsetAsync(h->status, 0, 256, stream);
+    if (e == cudaSuccess)
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->packed), std::max<size_t>(off, 16), h->pool,
+                                    stream);
+    // pageable source: the call returns once the table has been staged
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(h->table, table.data(), sizeof(uint64_t) * table.size(), cudaMemcpyHostToDevice,
+                            stream);
+    if (e == cudaSuccess)
+        e = patchk::launch_pack_fp8(W_bf16, meta, map, N, K, static_cast<int>(tn), static_cast<int>(tk),
+                                    h->table, h->fp8_scale, h->packed, stream);
+    if (e != cudaSuccess) {
+        patch_free(h, stream_v);
+        return from_cuda(e);
+    }
+    if (packed_bytes) *packed_bytes = h->packed_bytes;
+    *out = h;
+    return PATCH_OK;
+}
+
+patch_status patch_packed_fp8_scales(const patch_packed *Wp, float *scales_dst, void *stream_v) {
+    if (!Wp || !scales_dst || Wp->pattern != 8) return PATCH_ERR_INVALID_ARG;
+    return from_cuda(cudaMemcpyAsync(scales_dst, Wp->fp8_scale, sizeof(float) * static_cast<size_t>(Wp->shp.N),
+                                     cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream_v)));
+}
+
+static patch_status fp8_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
+                             int32_t y_is_fp32, cudaStream_t stream) {
+    const int64_t K = Wp->shp.K;
+    // the activations' codes and token scales, for this call only
+    const size_t off_sx = round_up(static_cast<size_t>(M * K), 256);
+    const size_t bytes = off_sx + sizeof(float) * static_cast<size_t>(M);
+    uint8_t *ws = nullptr;
+    cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), bytes, Wp->pool, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    float *sx = reinterpret_cast<float *>(ws + off_sx);
+    e = patchk::launch_fp8_quantize_rows(X_bf16, M, K, ws, sx, stream);
+    if (e == cudaSuccess) {
+        patchk::Fp8Launch g;
+        g.packed = Wp->packed;
+        g.table = Wp->table;
+        g.sw = Wp->fp8_scale;
+        g.xq = ws;
+        g.sx = sx;
+        g.N = Wp->shp.N;
+        g.K = K;
+        g.M = M;
+        g.Y = Y;
+        g.y_fp32 = y_is_fp32;
+        g.status = Wp->status;
+        g.num_sms = Wp->num_sms;
+        e = patchk::launch_fp8_gemm(g, stream);
+    }
+    cudaError_t e2 = cudaFreeAsync(ws, stream);
+    return from_cuda(e != cudaSuccess ? e : e2);
+}
+
 patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
                                int32_t y_is_fp32, void *stream_v) {
     if (!Wp || M < 0) return PATCH_ERR_INVALID_ARG;
@@ -627,6 +761,7 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     if (!aligned16(X_bf16) || !aligned16(Y)) return PATCH_ERR_INVALID_ARG;
     if (y_is_fp32 != 0 && y_is_fp32 != 1) return PATCH_ERR_INVALID_ARG;
     if (M > (int64_t(1) << 31)) return PATCH_ERR_INVALID_ARG;
+    if (Wp->pattern == 8) return fp8_gemm(Wp, X_bf16, M, Y, y_is_fp32, static_cast<cudaStream_t>(stream_v));
     patchk::GemmLaunch g;
     g.packed = Wp->packed;
     g.table = Wp->table;
@@ -704,7 +839,8 @@ patch_status patch_packed_export(const patch_packed *Wp, void *packed_dst, uint6
                             stream);
     if (e == cudaSuccess && table_dst)
         e = cudaMemcpyAsync(table_dst, Wp->table,
-                            sizeof(uint64_t) * (Wp->shp.N / kBand) * (Wp->shp.K / kStep),
+                            sizeof(uint64_t) * (Wp->shp.N / kBand) *
+                                (Wp->shp.K / (Wp->pattern == 8 ? 128 : kStep)),
                             cudaMemcpyDeviceToDevice, stream);
     return from_cuda(e);
 }

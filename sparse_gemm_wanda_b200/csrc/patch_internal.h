@@ -163,6 +163,30 @@ uint64_t decode_chunk_desc(const uint64_t *band_table, int64_t nsteps, int pr0, 
 // fp32 partial bytes of the decode GEMV (one 16 x 128 slot per chunk).
 size_t decode_workspace_bytes(int nchunks);
 
+// FP8 handles (csrc/fp8_kernels.cu, csrc/fp8_gemm.cu).
+// Per-row e4m3 quantisation of a bf16 matrix [R, C]: scale[r] = amax / 448
+// (1 for a zero row), q = e4m3(x / scale) (fp32 quotient, round to nearest,
+// saturating).
+cudaError_t launch_fp8_quantize_rows(const void *x, int64_t R, int64_t C, uint8_t *q, float *scale,
+                                     cudaStream_t stream);
+// W_eff row scales into `scale` [N] and the packed k-steps at the table's offsets.
+cudaError_t launch_pack_fp8(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
+                            int64_t K, int tn, int tk, const uint64_t *table, float *scale,
+                            uint8_t *out, cudaStream_t stream);
+struct Fp8Launch {
+    const uint8_t *packed;
+    const uint64_t *table;  // [N/128][K/128]
+    const float *sw;        // [N]
+    const uint8_t *xq;      // [M, K] e4m3 codes of X
+    const float *sx;        // [M]
+    int64_t N, K, M;
+    void *Y;
+    int y_fp32;
+    uint32_t *status;
+    int num_sms;
+};
+cudaError_t launch_fp8_gemm(const Fp8Launch &g, cudaStream_t stream);
+
 // The library's stream-ordered memory pool for the current device (cached
 // memory is kept, not returned to the system between calls).
 cudaError_t device_pool(cudaMemPool_t *pool);

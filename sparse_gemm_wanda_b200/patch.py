@@ -26,7 +26,8 @@ EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
            "patch_score_mask_noalloc_capacity", "patch_launch_count",
            "patch_select_maps_global", "patch_test_stall_first_kstep", "patch_pool_usage",
            "patch_colsq", "patch_colsq_partials", "patch_colsq_fold", "patch_test_prefill_kernel",
-           "patch_score_mask_nm", "patch_pack_nm")
+           "patch_score_mask_nm", "patch_pack_nm", "patch_pack_fp8", "patch_quantize_fp8",
+           "patch_packed_fp8_scales")
 
 
 class PatchLibraryError(RuntimeError):
@@ -84,6 +85,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.patch_pack_nm.argtypes = [vp, vp, vp, PatchShape, i32, i32, ctypes.POINTER(vp),
                                   ctypes.POINTER(ctypes.c_size_t), vp]
     lib.patch_pack_nm.restype = ctypes.c_int
+    lib.patch_pack_fp8.argtypes = [vp, vp, vp, PatchShape, ctypes.POINTER(vp),
+                                   ctypes.POINTER(ctypes.c_size_t), vp]
+    lib.patch_pack_fp8.restype = ctypes.c_int
+    lib.patch_quantize_fp8.argtypes = [vp, i64, i64, vp, vp, vp]
+    lib.patch_quantize_fp8.restype = ctypes.c_int
+    lib.patch_packed_fp8_scales.argtypes = [vp, vp, vp]
+    lib.patch_packed_fp8_scales.restype = ctypes.c_int
     lib.patch_colsq.argtypes = [vp, i64, i64, vp, vp]
     lib.patch_colsq_partials.argtypes = [vp, i64, i64, vp, vp]
     lib.patch_colsq_fold.argtypes = [vp, i64, i64, vp, vp]
@@ -272,10 +280,11 @@ def patch_score_mask_noalloc(W: torch.Tensor, Xcal: torch.Tensor | None = None, 
 class PackedWeight:
     """Owns a patch_packed handle; released by patch_free on close / deletion."""
 
-    def __init__(self, handle: int, shape: tuple, packed_bytes: int):
+    def __init__(self, handle: int, shape: tuple, packed_bytes: int, fp8: bool = False):
         self.handle = ctypes.c_void_p(handle)
         self.N, self.K, self.tile_n, self.tile_k = shape
         self.packed_bytes = packed_bytes
+        self.fp8 = fp8
 
     def view(self) -> PatchPackedView:
         v = PatchPackedView()
@@ -286,10 +295,18 @@ class PackedWeight:
         """Copies of the packed bytes (uint8) and the k-step table (int64) as CUDA tensors."""
         v = self.view()
         packed = torch.empty((v.packed_bytes,), dtype=torch.uint8, device="cuda")
-        table = torch.empty(((self.N // 128) * (self.K // 64),), dtype=torch.int64, device="cuda")
+        steps = self.K // (128 if self.fp8 else 64)
+        table = torch.empty(((self.N // 128) * steps,), dtype=torch.int64, device="cuda")
         _check("patch_packed_export", load_library().patch_packed_export(
             self.handle, _dptr(packed), _dptr(table), _stream(stream)))
         return packed, table
+
+    def fp8_scales(self, stream=None) -> torch.Tensor:
+        """The W_eff row scales of an FP8 handle ([N] fp32)."""
+        out = torch.empty((self.N,), dtype=torch.float32, device="cuda")
+        _check("patch_packed_fp8_scales", load_library().patch_packed_fp8_scales(
+            self.handle, _dptr(out), _stream(stream)))
+        return out
 
     def close(self, stream=None):
         if self.handle and self.handle.value:
@@ -341,6 +358,31 @@ def patch_pack(W: torch.Tensor, meta: torch.Tensor, tile_map: torch.Tensor, *, t
                                  ctypes.byref(out), ctypes.byref(nbytes), _stream(stream))
         _check("patch_pack_nm", code)
     return PackedWeight(out.value, (N, K, tile_n, tile_k), nbytes.value)
+
+
+def patch_pack_fp8(W: torch.Tensor, meta: torch.Tensor, tile_map: torch.Tensor, *, tile_n: int = 128,
+                   tile_k: int = 128, stream=None) -> PackedWeight:
+    """FP8 handle: W_eff quantised to e4m3 per output row, dense and 2:4 tiles."""
+    lib = load_library()
+    N, K = W.shape
+    out = ctypes.c_void_p(0)
+    nbytes = ctypes.c_size_t(0)
+    code = lib.patch_pack_fp8(_dptr(W, torch.bfloat16, "W"), _dptr(meta, (torch.int32, torch.uint32), "meta"),
+                              _dptr(tile_map, (torch.int32, torch.uint32), "map"),
+                              PatchShape(N, K, tile_n, tile_k), ctypes.byref(out), ctypes.byref(nbytes),
+                              _stream(stream))
+    _check("patch_pack_fp8", code)
+    return PackedWeight(out.value, (N, K, tile_n, tile_k), nbytes.value, fp8=True)
+
+
+def patch_quantize_fp8(X: torch.Tensor, stream=None) -> tuple:
+    """(codes uint8 [R, C], scales fp32 [R]) of the per-row e4m3 quantisation of X bf16."""
+    R, C = X.shape
+    codes = torch.empty((R, C), dtype=torch.uint8, device=X.device)
+    scales = torch.empty((R,), dtype=torch.float32, device=X.device)
+    _check("patch_quantize_fp8", load_library().patch_quantize_fp8(
+        _dptr(X, torch.bfloat16, "X"), R, C, _dptr(codes), _dptr(scales), _stream(stream)))
+    return codes, scales
 
 
 def patch_hybrid_gemm(packed: PackedWeight, X: torch.Tensor, out: torch.Tensor | None = None,

@@ -1,0 +1,137 @@
+"""FP8 (e4m3) values inside dense and 2:4 tiles on the GPU against the oracle,
+through the C ABI ("SparseGPT vs Wanda", FAQ: prune first, then quantise).
+
+Bit-exact: the e4m3 codes and fp32 scales of the per-row quantisation (X per
+token, W_eff per output row), the packed bytes and the k-step table.  GEMM
+(tcgen05 kind::f8f6f4, dense and sparse MMAs): against the oracle's fp64 sums
+of the oracle's own codes, within the tolerance reading of the bf16 tests
+(fp32 output: max err <= 1e-2 RMS; bf16 output: + half a bf16 ulp).
+"""
+import numpy as np
+import pytest
+import torch
+
+from sparse_gemm_wanda_b200 import inputs
+from tests.conftest import bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU machines, skipped there
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+
+@pytest.fixture(scope="module")
+def P():
+    from sparse_gemm_wanda_b200 import build, patch
+    build.build()
+    patch.load_library()
+    return patch
+
+
+def check(y, yref, fp32_mode):
+    y = y.double().cpu().numpy()
+    rms = float(np.sqrt(np.mean(yref ** 2)))
+    err = np.abs(y - yref)
+    if fp32_mode:
+        assert err.max() <= 1e-2 * rms, (float(err.max()), rms)
+    else:
+        mag = np.maximum(np.abs(y), np.abs(yref))
+        ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-30))) - 7)
+        bad = ~(err <= 1e-2 * rms + 0.5 * ulp)
+        assert not bad.any(), (int(bad.sum()), float(err.max()), rms)
+
+
+@pytest.mark.parametrize("R,C", [(1, 8), (5, 256), (300, 4096), (64, 11008)])
+def test_quantize_fp8_bit_exact(P, oracle_mod, R, C):
+    g = torch.Generator().manual_seed(R + C)
+    x = torch.randn(R, C, generator=g) * 3
+    x[:, : C // 16] *= 50              # outlier channels
+    if R > 2:
+        x[1] = 0.0                     # a zero row: scale 1, codes 0
+        x[2, ::3] = -0.0               # negative zeros keep their sign
+    xb = x.to(torch.bfloat16)
+    codes, scales = P.patch_quantize_fp8(xb.cuda())
+    torch.cuda.synchronize()
+    ref_s = oracle_mod.fp8_row_scales(bf16_bits(xb))
+    ref_q = oracle_mod.fp8_quantize(bf16_bits(xb), ref_s)
+    assert np.array_equal(scales.cpu().numpy(), ref_s)
+    assert np.array_equal(codes.cpu().numpy(), ref_q)
+
+
+def oracle_fp8(oracle_mod, w, xc, tmap, tn, tk):
+    ref = oracle_mod.score_mask(bf16_bits(w), bf16_bits(xc), tn, tk,
+                                tile_map=tmap.numpy().view(np.uint32))
+    weff = oracle_mod.weff(bf16_bits(w), ref["meta"], ref["map"], tn, tk)
+    sw = oracle_mod.fp8_row_scales(weff)
+    qw = oracle_mod.fp8_quantize(weff, sw)
+    return ref, sw, qw
+
+
+@pytest.mark.parametrize("tn,tk", [(128, 128), (64, 128), (128, 64), (64, 64)])
+@pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
+def test_pack_fp8_bit_exact(P, oracle_mod, tn, tk, frac):
+    N, K = 384, 512
+    w = inputs.weight(N, K, 5 + tn + tk)
+    o = inputs.outlier_channels(K, 5)
+    xc = inputs.activations(64, K, 5, o, role=0)
+    nt = (N // tn) * (K // tk)
+    tmap = inputs.random_map(nt, int(frac * nt), seed=tn + 3 * tk)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), tile_n=tn, tile_k=tk, map_in=tmap.cuda())
+    pk = P.patch_pack_fp8(w.cuda(), r["meta"], r["map"], tile_n=tn, tile_k=tk)
+    packed, table = pk.export()
+    sw = pk.fp8_scales()
+    torch.cuda.synchronize()
+    ref, ref_sw, ref_qw = oracle_fp8(oracle_mod, w, xc, tmap, tn, tk)
+    assert np.array_equal(sw.cpu().numpy(), ref_sw)
+    ref_packed, ref_table = oracle_mod.pack_fp8(ref_qw, ref["meta"], ref["map"], tn, tk)
+    assert pk.packed_bytes == ref_packed.size
+    assert np.array_equal(table.cpu().numpy().view(np.uint64), ref_table)
+    assert np.array_equal(packed.cpu().numpy(), ref_packed)
+    pk.close()
+
+
+def run_fp8_gemm(P, oracle_mod, N, K, M, tn, tk, frac, seed, fp32_mode, sample=None):
+    w = inputs.weight(N, K, seed)
+    o = inputs.outlier_channels(K, seed)
+    xc = inputs.activations(128, K, seed, o, role=0)
+    x = inputs.activations(M, K, seed, o, role=1)
+    nt = (N // tn) * (K // tk)
+    tmap = inputs.random_map(nt, int(frac * nt), seed=seed)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), tile_n=tn, tile_k=tk, map_in=tmap.cuda())
+    pk = P.patch_pack_fp8(w.cuda(), r["meta"], r["map"], tile_n=tn, tile_k=tk)
+    y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=fp32_mode)
+    torch.cuda.synchronize()
+    assert P.patch_get_status(pk) == 0
+    ref, sw, qw = oracle_fp8(oracle_mod, w, xc, tmap, tn, tk)
+    assert np.array_equal(r["meta"].cpu().numpy().view(np.uint32), ref["meta"])
+    sx = oracle_mod.fp8_row_scales(bf16_bits(x))
+    qx = oracle_mod.fp8_quantize(bf16_bits(x), sx)
+    if sample is None:
+        check(y, oracle_mod.gemm_fp8(qx, sx, qw, sw), fp32_mode)
+    else:
+        g = np.random.default_rng(seed)
+        ms, ns = g.integers(0, M, sample), g.integers(0, N, sample)
+        yref = oracle_mod.gemm_fp8_at(qx, sx, qw, sw, ms, ns)
+        check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, fp32_mode)
+        rows = slice(N - 128, N)  # one whole band, every token
+        check(y[:, rows], oracle_mod.gemm_fp8(qx, sx, np.ascontiguousarray(qw[rows]), sw[rows]), fp32_mode)
+    pk.close()
+
+
+@pytest.mark.parametrize("fp32_mode", [True, False])
+@pytest.mark.parametrize("M", [1, 7, 16, 64, 100, 200, 300])
+def test_gemm_fp8_small_shapes(P, oracle_mod, M, fp32_mode):
+    run_fp8_gemm(P, oracle_mod, 384, 512, M, 128, 128, 0.5, seed=M + 60, fp32_mode=fp32_mode)
+
+
+@pytest.mark.parametrize("tn,tk", [(128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("frac", [0.0, 0.5, 1.0])
+def test_gemm_fp8_tiles_and_fractions(P, oracle_mod, tn, tk, frac):
+    run_fp8_gemm(P, oracle_mod, 256, 768, 150, tn, tk, frac, seed=tn + tk + 11, fp32_mode=True)
+
+
+@pytest.mark.parametrize("M", [16, 2048])
+@pytest.mark.parametrize("frac", [0.5, 1.0])
+def test_gemm_fp8_llama_mlp_shape(P, oracle_mod, M, frac):
+    run_fp8_gemm(P, oracle_mod, 11008, 4096, M, 128, 128, frac, seed=91 + M, fp32_mode=False,
+                 sample=4000 if M > 16 else None)
