@@ -311,7 +311,7 @@ def colsq_bytes(T, K):
 
 
 # ----------------------------------------------------------- isolated GEMMs
-def isolated_gemm(P, wl, W, M, frac_map, X, flush, reps=20, seed=0, nm=(2, 4)):
+def isolated_gemm(P, wl, W, M, frac_map, X, flush, reps=20, seed=0, nm=(2, 4), fp8=False):
     """Time one GEMM configuration with L2 flushed before every call.  The
     N:M patterns (2:4, or 4:8) are Wanda's with X as calibration; the map is
     seeded random."""
@@ -319,7 +319,10 @@ def isolated_gemm(P, wl, W, M, frac_map, X, flush, reps=20, seed=0, nm=(2, 4)):
     nt = (N // wl.tile_n) * (K // wl.tile_k)
     tmap = inputs.random_map(nt, inputs.n_sparse_tiles(frac_map, nt), seed).cuda()
     r = P.patch_score_mask(W, X, tile_n=wl.tile_n, tile_k=wl.tile_k, map_in=tmap, nm=nm)
-    pk = P.patch_pack(W, r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k, nm=nm)
+    if fp8:
+        pk = P.patch_pack_fp8(W, r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k)
+    else:
+        pk = P.patch_pack(W, r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k, nm=nm)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     for _ in range(3):
         P.patch_hybrid_gemm(pk, X, out=Y)
@@ -449,9 +452,11 @@ def nm48_isolated(P, flush, peaks):
     for M in (16, 2048):
         Xd = inputs.activations(M, m.K, w.seed, o, role=1).cuda()
         ent = {}
-        for name, f, nm in (("dense", 0.0, (2, 4)), ("2:4 f=0.5", 0.5, (2, 4)), ("4:8 f=0.5", 0.5, (4, 8))):
-            # the same map, the same Wanda ranking; only the pattern differs
-            t_ms, nb = isolated_gemm(P, w, Wd, M, f, Xd, flush, seed=w.seed + 5, nm=nm)
+        for name, f, nm, fp8 in (("dense", 0.0, (2, 4), False), ("2:4 f=0.5", 0.5, (2, 4), False),
+                                 ("4:8 f=0.5", 0.5, (4, 8), False), ("fp8 dense", 0.0, (2, 4), True),
+                                 ("fp8 2:4 f=0.5", 0.5, (2, 4), True), ("fp8 2:4 f=1", 1.0, (2, 4), True)):
+            # the same map, the same Wanda ranking; only the pattern / precision differs
+            t_ms, nb = isolated_gemm(P, w, Wd, M, f, Xd, flush, seed=w.seed + 5, nm=nm, fp8=fp8)
             e = {"us": t_ms * 1e3, "packed_bytes": nb,
                  "effective_tflops": 2.0 * M * m.N * m.K / (t_ms * 1e-3) / 1e12}
             if M <= 16:
@@ -464,7 +469,9 @@ def nm48_isolated(P, flush, peaks):
     return {"by_shape": out,
             "note": "4:8 handles run the one-band kernel whose converter warps expand 4:8 k-steps "
                     "into dense tiles in shared memory (no 4:8 tensor-core mode for 16-bit "
-                    "inputs); L2 flushed before every call"}
+                    "inputs); FP8 handles quantise X per token inside the call and run the "
+                    "kind::f8f6f4 kernel (its time includes that quantisation); effective TFLOP/s "
+                    "count 2MNK; L2 flushed before every call"}
 
 
 def decode_isolated(P, flush, peaks):
@@ -746,7 +753,7 @@ def main():
     if not args.no_extras and rank == 0 and world == 1:
         extras["prefill_gemm_isolated"] = prefill_sweep(P, wl.name, flush, peaks)
         extras["decode_gemm_isolated"] = decode_isolated(P, flush, peaks)
-        extras["nm48_gemm_isolated"] = nm48_isolated(P, flush, peaks)
+        extras["pattern_precision_isolated"] = nm48_isolated(P, flush, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
