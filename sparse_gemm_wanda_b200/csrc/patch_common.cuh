@@ -242,6 +242,22 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
     return d;
 }
 
+// The same descriptor split for a tight issue loop: the constant fields with
+// a zero start address, as two 32-bit halves.  A shared-memory address is
+// below 256 KB, so (address >> 4) fits the 14-bit start field and ORs into
+// the low half without touching the other fields; advancing along K inside a
+// swizzle atom adds (bytes >> 4) to it.
+struct DescBase {
+    uint32_t lo, hi;
+};
+__host__ __device__ constexpr DescBase smem_desc_base(uint32_t lbo_bytes, uint32_t sbo_bytes, SmemLayout layout) {
+    return DescBase{((lbo_bytes >> 4) & 0x3FFFu) << 16,
+                    ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (static_cast<uint32_t>(layout) << 29)};
+}
+__device__ __forceinline__ uint64_t desc_at(DescBase b, uint32_t addr16) {
+    return (static_cast<uint64_t>(b.hi) << 32) | (b.lo | addr16);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B, fp32 D, both K-major,
 // M = 128 and the given N; `sparse` sets the 2:4 flag, `id2` the metadata
 // selector.

@@ -257,6 +257,11 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
             // ------------------------------------------------- MMA (leader)
             const uint32_t e_tmem = tmem_base + static_cast<uint32_t>(2 * bn);
             const uint32_t idesc_dense = idesc_pair(bn, false);
+            const uint32_t idesc_sparse[2] = {idesc_pair(bn, true, 0), idesc_pair(bn, true, 1)};
+            constexpr DescBase kDescDenseA = smem_desc_base(16, 1024, kSwizzle128B);
+            constexpr DescBase kDescSparseA = smem_desc_base(16, 512, kSwizzle64B);
+            constexpr DescBase kDescX = smem_desc_base(16, 1024, kSwizzle128B);
+            constexpr DescBase kDescMeta = smem_desc_base(16, 128, kSwizzleNone);
             int it = 0;
             bool ok = true;
             for (int i = 0; ok; ++i) {
@@ -287,23 +292,20 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
                         const uint32_t a_addr = slot + static_cast<uint32_t>((e & kEntryOffsetMask) - first);
                         const uint32_t b_addr = slot + static_cast<uint32_t>(p.aslot + h * half * kStep * 2);
                         const bool fresh = pr == 0 && h == 0;
+                        // descriptors: constant fields + 16-byte address units
+                        const uint32_t a16 = a_addr >> 4, b16 = b_addr >> 4;
                         if (e & kEntrySparse) {
                             if (e & kEntryMeta)
-                                tmem_cp_pair_128x128b(e_tmem, smem_desc(a_addr - kMetaBlockBytes, 16, 128, kSwizzleNone));
+                                tmem_cp_pair_128x128b(e_tmem, desc_at(kDescMeta, (a_addr - kMetaBlockBytes) >> 4));
 #pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                const uint64_t ad = smem_desc(a_addr + q * 32, 16, 512, kSwizzle64B);
-                                const uint64_t bd = smem_desc(b_addr + q * 64, 16, 1024, kSwizzle128B);
-                                mma_sparse_pair(d_tmem, ad, bd, e_tmem + 2 * h, idesc_pair(bn, true, q),
-                                                (fresh && q == 0) ? 0u : 1u);
-                            }
+                            for (int q = 0; q < 2; ++q)
+                                mma_sparse_pair(d_tmem, desc_at(kDescSparseA, a16 + 2 * q), desc_at(kDescX, b16 + 4 * q),
+                                                e_tmem + 2 * h, idesc_sparse[q], (fresh && q == 0) ? 0u : 1u);
                         } else {
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const uint64_t ad = smem_desc(a_addr + q * 32, 16, 1024, kSwizzle128B);
-                                const uint64_t bd = smem_desc(b_addr + q * 32, 16, 1024, kSwizzle128B);
-                                mma_dense_pair(d_tmem, ad, bd, idesc_dense, (fresh && q == 0) ? 0u : 1u);
-                            }
+                            for (int q = 0; q < 4; ++q)
+                                mma_dense_pair(d_tmem, desc_at(kDescDenseA, a16 + 2 * q), desc_at(kDescX, b16 + 2 * q),
+                                               idesc_dense, (fresh && q == 0) ? 0u : 1u);
                         }
                     }
                     tc_commit_pair(&empty[s]);
