@@ -474,6 +474,48 @@ def nm48_isolated(P, flush, peaks):
                     "count 2MNK; L2 flushed before every call"}
 
 
+def tile_shapes_isolated(P, flush, peaks):
+    """Finer tiles on the Llama-7B MLP shape at M = 2048: 128x128, 128x64,
+    64x128 and 64x64 tiles at f in {0, .5, 1} (seeded random maps).  The GEMM
+    runs 128-row bands with 64-column k-steps; a band's k-step runs the 2:4
+    MMA when every tile it covers is 2:4, so a 64-row tile is fast only where
+    its band partner agrees (M = 64 MMAs run at half the M = 128 rate on this
+    GPU, so splitting a band is no faster than running it dense)."""
+    import types
+
+    import numpy as np
+    w = inputs.workloads()["llama7b-prefill"]
+    m = w.matrices[0]
+    M = w.tokens[0]
+    o = inputs.outlier_channels(m.K, w.seed)
+    Wd = inputs.weight(m.N, m.K, w.seed + m.N).cuda()
+    Xd = inputs.activations(M, m.K, w.seed, o, role=1).cuda()
+    fl = 2.0 * M * m.N * m.K
+    out = {}
+    base = None
+    for tn, tk in ((128, 128), (128, 64), (64, 128), (64, 64)):
+        shape = types.SimpleNamespace(tile_n=tn, tile_k=tk)
+        ent = {}
+        for f in (0.0, 0.5, 1.0):
+            seed = w.seed + 7 * tn + tk + int(f * 100)
+            t_ms, _ = isolated_gemm(P, shape, Wd, M, f, Xd, flush, seed=seed)
+            nt = (m.N // tn) * (m.K // tk)
+            bits = np.unpackbits(inputs.random_map(nt, inputs.n_sparse_tiles(f, nt), seed).numpy()
+                                 .view(np.uint8), bitorder="little")[:nt].reshape(m.N // tn, m.K // tk)
+            # 128-row bands x 64-column k-steps that run the 2:4 MMA
+            b = bits.repeat(tn // 64, axis=0).repeat(tk // 64, axis=1)
+            run_sparse = float((b[0::2] & b[1::2]).mean())
+            if base is None:
+                base = t_ms
+            ent[f"f{f}"] = {"us": t_ms * 1e3, "effective_tflops": fl / (t_ms * 1e-3) / 1e12,
+                            "ksteps_run_sparse": run_sparse, "speedup_vs_128x128_dense": base / t_ms}
+        out[f"{tn}x{tk}"] = ent
+    del Wd, Xd
+    return {"shape": f"M={M} N={m.N} K={m.K}", "by_tile": out,
+            "note": "seeded random maps; L2 flushed before every call; ksteps_run_sparse = share "
+                    "of (128-row band, 64-column k-step) units whose tiles are all 2:4"}
+
+
 def decode_isolated(P, flush, peaks):
     """The decode GEMV on the Llama-7B decode shapes at M in {1, 4, 16}: one
     CUDA graph of back-to-back calls over copies larger than 3x L2, per call."""
@@ -754,6 +796,7 @@ def main():
         extras["prefill_gemm_isolated"] = prefill_sweep(P, wl.name, flush, peaks)
         extras["decode_gemm_isolated"] = decode_isolated(P, flush, peaks)
         extras["pattern_precision_isolated"] = nm48_isolated(P, flush, peaks)
+        extras["tile_shapes_isolated"] = tile_shapes_isolated(P, flush, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:

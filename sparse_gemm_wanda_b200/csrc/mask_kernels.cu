@@ -37,21 +37,35 @@ __global__ void norms_from_colsq_kernel(const double *__restrict__ colsq_in, int
 
 // ----------------------------------------------------------------- scoring
 // Select the two kept positions of one group: q is kept iff fewer than two
-// other candidates come before it in the order (score desc, index asc).
-__device__ __forceinline__ uint32_t top2_code(const double s[4]) {
-    // For p < q, p precedes q iff s_p >= s_q (a tie goes to the lower index).
-    const int b01 = s[0] >= s[1], b02 = s[0] >= s[2], b03 = s[0] >= s[3];
-    const int b12 = s[1] >= s[2], b13 = s[1] >= s[3], b23 = s[2] >= s[3];
+// other candidates come before it in the order (score desc, index asc); for
+// p < q, p precedes q iff s_p >= s_q (a tie goes to the lower index).  As a
+// table over the six comparison bits
+// i = [s0>=s1] | [s0>=s2]<<1 | [s0>=s3]<<2 | [s1>=s2]<<3 | [s1>=s3]<<4 | [s2>=s3]<<5:
+// low nibble the 4-bit code (lowest | highest kept position << 2), high
+// nibble the pruned positions (those not in the code).  Every one of the 64
+// patterns gets the value of the rank formula, reachable or not.
+__host__ __device__ constexpr uint8_t top2_entry(int i) {
+    const int b01 = i & 1, b02 = (i >> 1) & 1, b03 = (i >> 2) & 1;
+    const int b12 = (i >> 3) & 1, b13 = (i >> 4) & 1, b23 = (i >> 5) & 1;
     const int r0 = (1 - b01) + (1 - b02) + (1 - b03);
     const int r1 = b01 + (1 - b12) + (1 - b13);
     const int r2 = b02 + b12 + (1 - b23);
     const int r3 = b03 + b13 + b23;
     const int k0 = r0 < 2, k1 = r1 < 2, k2 = r2 < 2, k3 = r3 < 2;
-    // lowest and highest kept positions
-    const uint32_t lo = k0 ? 0u : (k1 ? 1u : 2u);
-    const uint32_t hi = k3 ? 3u : (k2 ? 2u : 1u);
-    return lo | (hi << 2);
+    const int lo = k0 ? 0 : (k1 ? 1 : 2);
+    const int hi = k3 ? 3 : (k2 ? 2 : 1);
+    const int pruned = 0xF & ~((1 << lo) | (1 << hi));
+    return static_cast<uint8_t>(lo | (hi << 2) | (pruned << 4));
 }
+struct Top2Table {
+    uint32_t w[16];  // entry i in byte i % 4 of word i / 4
+};
+__host__ __device__ constexpr Top2Table make_top2_table() {
+    Top2Table t{};
+    for (int i = 0; i < 64; ++i) t.w[i / 4] |= static_cast<uint32_t>(top2_entry(i)) << (8 * (i % 4));
+    return t;
+}
+__constant__ Top2Table kTop2Table = make_top2_table();
 
 // 4:8 groups: q is kept iff fewer than four other candidates come before it
 // in the order (score desc, index asc); returns the 8-bit keep mask.
@@ -90,14 +104,15 @@ __device__ __forceinline__ double bf16_abs_f64(uint32_t bits16) {
 // word's pruned-score sum (left to right).  The CTA then adds each row's
 // words left to right and the rows as a balanced pairwise tree.
 template <int TN, int TK, int PAT>
-__global__ void __launch_bounds__(TN *(TK / 32))
+__global__ void __launch_bounds__(TN *(TK / 32), PAT == 2 ? 2048 / (TN * (TK / 32)) : 1)
 score_mask_kernel(const uint16_t *__restrict__ W, const double *__restrict__ norm, int64_t N,
                   int64_t K, uint32_t *__restrict__ meta, double *__restrict__ loss,
                   int32_t *__restrict__ rank, uint32_t *__restrict__ done) {
     constexpr int WPR = TK / 32;      // words per tile row
-    constexpr int kNormStride = 33;   // padded: the words' norms sit in different banks
+    constexpr int kNormStride = 34;   // padded: the words' norms sit in different banks (16-B rows)
     constexpr int kWarps = TN / 32;   // warps holding the tile's row sums
-    __shared__ double ns[WPR * kNormStride];
+    __shared__ __align__(16) double ns[WPR * kNormStride];
+    __shared__ uint32_t top2[16];
     __shared__ double wsum[TN * WPR];
     __shared__ double warp_sum[kWarps];
     const int64_t tiles_k = K / TK;
@@ -107,6 +122,7 @@ score_mask_kernel(const uint16_t *__restrict__ W, const double *__restrict__ nor
     const int r = tid / WPR, w = tid % WPR;
 
     for (int u = tid; u < TK; u += TN * WPR) ns[(u / 32) * kNormStride + u % 32] = __ldg(norm + j0 + u);
+    if (PAT == 2 && tid < 16) top2[tid] = kTop2Table.w[tid];
     const uint4 *src = reinterpret_cast<const uint4 *>(W + (i0 + r) * K + j0 + 32 * w);
     uint4 v[4];
 #pragma unroll
@@ -132,26 +148,36 @@ score_mask_kernel(const uint16_t *__restrict__ W, const double *__restrict__ nor
                 if (!((m >> q) & 1u)) acc = __dadd_rn(acc, sc[q]);
             word |= m << (8 * h);
         }
-    } else
+    } else {
+        const uint8_t *tab = reinterpret_cast<const uint8_t *>(top2);
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-        const uint32_t e[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+        for (int h = 0; h < 4; ++h) {
+            const uint32_t e[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
 #pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-            const int col = h * 8 + gg * 4;
-            double sc[4];
+            for (int gg = 0; gg < 2; ++gg) {
+                const int col = h * 8 + gg * 4;
+                const double2 n01 = *reinterpret_cast<const double2 *>(nw + col);
+                const double2 n23 = *reinterpret_cast<const double2 *>(nw + col + 2);
+                // |w| exactly: bf16 -> fp32 (the bits moved up), sign cleared
+                // for both halves of a word at once, fp32 -> fp64 exact
+                const uint32_t a01 = e[gg * 2] & 0x7FFF7FFFu, a23 = e[gg * 2 + 1] & 0x7FFF7FFFu;
+                double sc[4];
+                sc[0] = __dmul_rn(static_cast<double>(__uint_as_float(a01 << 16)), n01.x);
+                sc[1] = __dmul_rn(static_cast<double>(__uint_as_float(a01 & 0xFFFF0000u)), n01.y);
+                sc[2] = __dmul_rn(static_cast<double>(__uint_as_float(a23 << 16)), n23.x);
+                sc[3] = __dmul_rn(static_cast<double>(__uint_as_float(a23 & 0xFFFF0000u)), n23.y);
+                const uint32_t idx = static_cast<uint32_t>(sc[0] >= sc[1]) | (static_cast<uint32_t>(sc[0] >= sc[2]) << 1) |
+                                     (static_cast<uint32_t>(sc[0] >= sc[3]) << 2) |
+                                     (static_cast<uint32_t>(sc[1] >= sc[2]) << 3) |
+                                     (static_cast<uint32_t>(sc[1] >= sc[3]) << 4) |
+                                     (static_cast<uint32_t>(sc[2] >= sc[3]) << 5);
+                const uint32_t ent = tab[idx];
+                // the pruned scores, left to right
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t pairbits = e[gg * 2 + q / 2];
-                const uint32_t bits = (q & 1) ? (pairbits >> 16) : (pairbits & 0xFFFFu);
-                sc[q] = __dmul_rn(bf16_abs_f64(bits), nw[col + q]);
+                for (int q = 0; q < 4; ++q)
+                    if ((ent >> (4 + q)) & 1u) acc = __dadd_rn(acc, sc[q]);
+                word |= (ent & 0xFu) << (4 * (h * 2 + gg));
             }
-            const uint32_t code = top2_code(sc);
-            const int lo = static_cast<int>(code & 3u), hi = static_cast<int>(code >> 2);
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (q != lo && q != hi) acc = __dadd_rn(acc, sc[q]);
-            word |= code << (4 * (h * 2 + gg));
         }
     }
     meta[(i0 + r) * (K / 32) + j0 / 32 + w] = word;
@@ -190,29 +216,66 @@ score_mask_kernel(const uint16_t *__restrict__ W, const double *__restrict__ nor
 
 // ------------------------------------------------------------- tile ranking
 constexpr int kRankThreads = 128;
-constexpr int kRankSlice = 256;
+constexpr int kRankPerThread = 2;                           // tiles t per thread
+constexpr int kRankTiles = kRankThreads * kRankPerThread;   // tiles t per block
+constexpr int kRankSlice = 256;                             // tiles u per block, at most
+
+// slice of u per block: narrower for few tiles, so the comparisons spread over
+// enough blocks to fill the device
+inline int rank_slice(int64_t n_tiles) { return n_tiles <= 4096 ? 64 : kRankSlice; }
 
 // rank[t] += #{u in this block's slice : (L_u, u) < (L_t, t)}.  Integer
 // counts, so the accumulated rank does not depend on the order of atomics.
 // The last block to finish writes the bitmap: bit t set iff rank[t] < n_sparse.
+// For u < t the pair order is L_u <= L_t, for u > t it is L_u < L_t; a slice
+// wholly below or above a thread's tiles takes the one comparison.
 __global__ void __launch_bounds__(kRankThreads)
-rank_tiles_kernel(const double *__restrict__ loss, int64_t n_tiles, int64_t n_sparse,
+rank_tiles_kernel(const double *__restrict__ loss, int64_t n_tiles, int64_t n_sparse, int slice,
                   int32_t *__restrict__ rank, uint32_t *__restrict__ done, uint32_t *__restrict__ map) {
     __shared__ double sl[kRankSlice];
     __shared__ bool last;
-    const int64_t t = static_cast<int64_t>(blockIdx.x) * kRankThreads + threadIdx.x;
-    const int64_t u0 = static_cast<int64_t>(blockIdx.y) * kRankSlice;
-    const int64_t u1 = min(n_tiles, u0 + kRankSlice);
+    const int64_t tb = static_cast<int64_t>(blockIdx.x) * kRankTiles + threadIdx.x;
+    const int64_t u0 = static_cast<int64_t>(blockIdx.y) * slice;
+    const int64_t u1 = min(n_tiles, u0 + slice);
     for (int64_t u = u0 + threadIdx.x; u < u1; u += kRankThreads) sl[u - u0] = loss[u];
     __syncthreads();
-    if (t < n_tiles) {
-        const double lt = loss[t];
-        int32_t r = 0;
-        for (int64_t u = u0; u < u1; ++u) {
-            const double lu = sl[u - u0];
-            r += (lu < lt) || (lu == lt && u < t);
+    double lt[kRankPerThread];
+    int32_t cnt[kRankPerThread];
+#pragma unroll
+    for (int j = 0; j < kRankPerThread; ++j) {
+        const int64_t t = tb + j * kRankThreads;
+        lt[j] = t < n_tiles ? loss[t] : 0.0;
+        cnt[j] = 0;
+    }
+    const int len = static_cast<int>(u1 - u0);
+    const int64_t t_first = tb, t_last = tb + (kRankPerThread - 1) * kRankThreads;
+    if (u1 <= t_first) {
+        for (int i = 0; i < len; ++i) {
+            const double lu = sl[i];
+#pragma unroll
+            for (int j = 0; j < kRankPerThread; ++j) cnt[j] += lu <= lt[j];
         }
-        atomicAdd(rank + t, r);
+    } else if (u0 > t_last) {
+        for (int i = 0; i < len; ++i) {
+            const double lu = sl[i];
+#pragma unroll
+            for (int j = 0; j < kRankPerThread; ++j) cnt[j] += lu < lt[j];
+        }
+    } else {
+        for (int i = 0; i < len; ++i) {
+            const double lu = sl[i];
+            const int64_t u = u0 + i;
+#pragma unroll
+            for (int j = 0; j < kRankPerThread; ++j) {
+                const int64_t t = tb + j * kRankThreads;
+                cnt[j] += (lu < lt[j]) || (lu == lt[j] && u < t);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kRankPerThread; ++j) {
+        const int64_t t = tb + j * kRankThreads;
+        if (t < n_tiles) atomicAdd(rank + t, cnt[j]);
     }
     if (!map) return;  // the caller turns ranks into bitmaps itself
     __threadfence();
@@ -225,6 +288,7 @@ rank_tiles_kernel(const double *__restrict__ loss, int64_t n_tiles, int64_t n_sp
     const int64_t words = (n_tiles + 31) / 32;
     for (int64_t wd = threadIdx.x; wd < words; wd += kRankThreads) {
         uint32_t bits = 0;
+#pragma unroll
         for (int q = 0; q < 32; ++q) {
             const int64_t tt = wd * 32 + q;
             if (tt < n_tiles && __ldcg(rank + tt) < n_sparse) bits |= 1u << q;
@@ -273,9 +337,11 @@ cudaError_t launch_select_maps_global(const double *loss_cat, const int64_t *n_t
         g.word0[m + 1] = g.word0[m] + (n_tiles[m] + 31) / 32;
     }
     const int64_t total = g.offset[count];
-    dim3 grid(static_cast<unsigned>((total + kRankThreads - 1) / kRankThreads),
-              static_cast<unsigned>((total + kRankSlice - 1) / kRankSlice));
-    rank_tiles_kernel<<<grid, kRankThreads, 0, stream>>>(loss_cat, total, n_sparse, rank, nullptr, nullptr);
+    const int slice = rank_slice(total);
+    dim3 grid(static_cast<unsigned>((total + kRankTiles - 1) / kRankTiles),
+              static_cast<unsigned>((total + slice - 1) / slice));
+    rank_tiles_kernel<<<grid, kRankThreads, 0, stream>>>(loss_cat, total, n_sparse, slice, rank, nullptr,
+                                                         nullptr);
     split_maps_kernel<<<static_cast<unsigned>((g.word0[count] + 127) / 128), 128, 0, stream>>>(rank, n_sparse, g);
     note_launches(2);
     return cudaGetLastError();
@@ -318,9 +384,10 @@ cudaError_t launch_score_mask(const void *W, const double *norm, int64_t N, int6
 
 cudaError_t launch_select_map(const double *loss, int64_t n_tiles, int64_t n_sparse, int32_t *rank,
                               uint32_t *done, uint32_t *map, cudaStream_t stream) {
-    dim3 grid(static_cast<unsigned>((n_tiles + kRankThreads - 1) / kRankThreads),
-              static_cast<unsigned>((n_tiles + kRankSlice - 1) / kRankSlice));
-    rank_tiles_kernel<<<grid, kRankThreads, 0, stream>>>(loss, n_tiles, n_sparse, rank, done, map);
+    const int slice = rank_slice(n_tiles);
+    dim3 grid(static_cast<unsigned>((n_tiles + kRankTiles - 1) / kRankTiles),
+              static_cast<unsigned>((n_tiles + slice - 1) / slice));
+    rank_tiles_kernel<<<grid, kRankThreads, 0, stream>>>(loss, n_tiles, n_sparse, slice, rank, done, map);
     note_launches(1);
     return cudaGetLastError();
 }
