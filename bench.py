@@ -629,6 +629,7 @@ def main():
     ap.add_argument("--T", type=int, default=2048)
     ap.add_argument("--frac", type=float, default=0.5)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--fp8", action="store_true", help="--case gemm: FP8 (e4m3) values in the tiles")
     ap.add_argument("--force-kernel", type=int, default=0,
                     help="--case gemm: prefill kernel (library test hook; 0 = the library's choice)")
     args = ap.parse_args()
@@ -865,7 +866,8 @@ def run_case(args):
             for _ in range(args.reps):
                 P.patch_pack(W, r["meta"], r["map"]).close()
         else:
-            pk = P.patch_pack(W, r["meta"], r["map"])
+            pk = (P.patch_pack_fp8(W, r["meta"], r["map"]) if args.fp8
+                  else P.patch_pack(W, r["meta"], r["map"]))
             P.test_prefill_kernel(args.force_kernel)
             for _ in range(args.reps):
                 P.patch_hybrid_gemm(pk, X)
@@ -873,7 +875,7 @@ def run_case(args):
             assert P.patch_get_status(pk) == 0
             pk.close()
     torch.cuda.synchronize()
-    print(f"case {args.case} N={args.N} K={args.K} M={args.M} frac={args.frac} ok")
+    print(f"case {args.case} N={args.N} K={args.K} M={args.M} frac={args.frac}{' fp8' if args.fp8 else ''} ok")
 
 
 def main_reference(args, wl, world, rank):

@@ -336,6 +336,10 @@ patch_status patch_pack_nm(const void *W_bf16, const uint32_t *meta, const uint3
  *     (r/8)*512 + (r%8)*64 + ((v/16) ^ ((r%8)/2))*16 + v%16;
  *   - table[b*(K/128)+c] (uint64): bits 0..47 offset of the k-step's codes,
  *     bit 62 = 2:4.
+ * With an even band count the handle also holds a prefill table for the
+ * two-SM kernel (not exported): bands 2p and 2p+1 take one kind at every
+ * k-step, a 2:4 k-step whose partner band's is dense pointing to a dense
+ * side copy of its W_eff codes (16384 bytes each, after the packed bytes).
  * Errors as patch_pack.
  */
 patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
@@ -394,7 +398,9 @@ void patch_test_stall_first_kstep(int32_t on);
  * uses.  0 = chosen by the library (the default), 1 = one band per CTA,
  * 2 = two bands per CTA sharing each token tile, 3 = two-SM (CTA pair)
  * kernel, 4 = two-SM kernel with two bands per SM; 3 and 4 only where the
- * band count is even (else as 0).  Results are
+ * band count is even (else as 0).  FP8 handles: 1 = one band per CTA, 3 =
+ * the two-SM kernel (even band count and an even number of 128-column
+ * k-steps, else as 1), anything else = chosen by the library.  Results are
  * the same up to fp32 rounding order; this only lets tests reach each kernel.
  */
 void patch_test_prefill_kernel(int32_t which);

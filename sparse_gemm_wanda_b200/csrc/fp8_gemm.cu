@@ -15,9 +15,12 @@
 // overlaps the next tile's main loop.  A stage is one k-step: one bulk copy of
 // its packed bytes (16 KB dense, or 2 KB metadata + 8 KB kept codes) and one
 // TMA load of the BN x 128-byte X tile (128-byte swizzle, rows past M zero).
-// Roles (192 threads): warp 0 lane 0 producer, warp 1 lane 0 MMA (warp 1 also
-// allocates tensor memory), warps 2..5 epilogue.  Every mbarrier wait is
-// bounded by %globaltimer; a wait that runs out raises the handle's status.
+// Roles (224 threads): warp 0 lane 0 weight producer, warp 6 lane 0 X
+// producer (the copies one thread issues are processed largely one after
+// another, so the two streams go through two threads), warp 1 lane 0 MMA
+// (warp 1 also allocates tensor memory), warps 2..5 epilogue.  Every mbarrier
+// wait is bounded by %globaltimer; a wait that runs out raises the handle's
+// status.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -33,7 +36,7 @@ namespace patchk {
 
 namespace {
 
-constexpr int kF8Threads = 192;
+constexpr int kF8Threads = 224;
 constexpr int kF8Step = 128;                 // columns (bytes of codes) per k-step
 constexpr int kF8Aslot = kDenseStepBytes;    // 16 KB: a dense k-step, or metadata + kept codes
 constexpr int kF8SmemLimit = 232448;
@@ -121,7 +124,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 2);  // the weight and X producers
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -151,7 +154,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             for (int i = 0; ok; ++i) {
                 const int tile = cta + i * P;
                 if (tile >= p.tiles) break;
-                const int band = tile / p.ttiles, tt = tile % p.ttiles;
+                const int band = tile / p.ttiles;
                 const uint64_t *tab = p.table + static_cast<int64_t>(band) * p.steps;
                 for (int c = 0; c < p.steps; ++c) {
                     const int s = it % S;
@@ -167,9 +170,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
                     stage_info[s] = e;
                     ++it;
                     uint8_t *st = smem + s * C::kStageBytes;
-                    mbar_arrive_expect_tx(&full[s], bytes + C::kXBytes);
+                    mbar_arrive_expect_tx(&full[s], bytes);
                     bulk_g2s(st, p.packed + first, bytes, &full[s]);
-                    tma_load_2d(st + kF8Aslot, &tmap_x, c * kF8Step, tt * BN, &full[s]);
                 }
             }
             if (!ok) {
@@ -179,6 +181,32 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
             // the last phase issued on every stage lands before the CTA exits
             for (int q = (it > S ? it - S : 0); q < it; ++q)
                 mbar_wait_bounded(&full[q % S], (q / S) & 1u, never_flag, kF8WaitLimitNs / 4);
+        }
+    } else if (warp == 6) {
+        if (lane == 0 && !skip) {
+            // ---------------------------------------------------- X producer
+            int it = 0;
+            bool ok = true;
+            for (int i = 0; ok; ++i) {
+                const int tile = cta + i * P;
+                if (tile >= p.tiles) break;
+                const int tt = tile % p.ttiles;
+                for (int c = 0; c < p.steps; ++c) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (it >= S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kF8WaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    ++it;
+                    mbar_arrive_expect_tx(&full[s], C::kXBytes);
+                    tma_load_2d(smem + s * C::kStageBytes + kF8Aslot, &tmap_x, c * kF8Step, tt * BN, &full[s]);
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1u;
+                atomicOr(p.status, kStatusTimeout);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0 && !skip) {
@@ -349,6 +377,13 @@ cudaError_t run_fp8(const Fp8Launch &g, cudaStream_t stream) {
 
 cudaError_t launch_fp8_gemm(const Fp8Launch &g, cudaStream_t stream) {
     if (g.K % kF8Step != 0 || g.N % kBand != 0 || g.M < 1) return cudaErrorInvalidValue;
+    // more than one token tile: the two-SM kernel, where the bands pair up
+    // (prefill table) and the k-step count is even
+    const bool duo_ok = g.ptable && (g.N / kBand) % 2 == 0 && (g.K / kF8Step) % 2 == 0 && g.K / kF8Step <= 224;
+    if (duo_ok && g.force_kernel != 1 && (g.M > 128 || g.force_kernel == 3)) {
+        const DuoFp8Plan dp = plan_duo_fp8(g.N, g.M, g.num_sms, g.all_sparse != 0);
+        if (dp.bn > 0) return launch_duo_fp8(g, dp, stream);
+    }
     if (g.M <= 64) return run_fp8<64>(g, stream);
     if (g.M <= 128) return run_fp8<128>(g, stream);
     return run_fp8<240>(g, stream);

@@ -127,15 +127,23 @@ fp8_weff_scales_kernel(const uint16_t *__restrict__ W, const uint32_t *__restric
     if (threadIdx.x == 0) scale[i] = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
 }
 
-// One block per (band, 128-column k-step), 128 threads.
+// One block per (band, 128-column k-step), 128 threads; with a prefill
+// table, a second set of blocks writes the dense side copies it names.
 __global__ void __launch_bounds__(128)
 pack_fp8_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
                 const uint32_t *__restrict__ map, int64_t K, int tn, int tk,
                 const float *__restrict__ scale, const uint64_t *__restrict__ table,
-                uint8_t *__restrict__ out) {
+                const uint64_t *__restrict__ ptable, int64_t units, uint8_t *__restrict__ out) {
     const int64_t steps = K / 128;
-    const int64_t b = blockIdx.x / steps, c = blockIdx.x % steps;
-    const uint64_t entry = table[blockIdx.x];
+    const bool side = blockIdx.x >= units;
+    const int64_t unit = side ? blockIdx.x - units : blockIdx.x;
+    const int64_t b = unit / steps, c = unit % steps;
+    uint64_t entry = table[unit];
+    if (side) {
+        entry = ptable[unit];
+        if (!(entry & kEntrySide)) return;
+        entry &= kEntryOffsetMask;  // a dense k-step at the side offset
+    }
     uint8_t *dst = out + (entry & kEntryOffsetMask);
     const int64_t row0 = b * kBand, col0 = c * 128, words_k = K / 32;
     const int tid = threadIdx.x;
@@ -205,14 +213,14 @@ cudaError_t launch_fp8_quantize_rows(const void *x, int64_t R, int64_t C, uint8_
 }
 
 cudaError_t launch_pack_fp8(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
-                            int64_t K, int tn, int tk, const uint64_t *table, float *scale,
-                            uint8_t *out, cudaStream_t stream) {
+                            int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
+                            float *scale, uint8_t *out, cudaStream_t stream) {
     if (N % kBand != 0 || K % 128 != 0 || N > 0x7FFFFFFF) return cudaErrorInvalidValue;
     fp8_weff_scales_kernel<<<static_cast<unsigned>(N), kQuantThreads, 0, stream>>>(
         static_cast<const uint16_t *>(W), meta, map, K, tn, tk, scale);
-    const int64_t blocks = (N / kBand) * (K / 128);
-    pack_fp8_kernel<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(
-        static_cast<const uint16_t *>(W), meta, map, K, tn, tk, scale, table, out);
+    const int64_t units = (N / kBand) * (K / 128);
+    pack_fp8_kernel<<<static_cast<unsigned>(ptable ? 2 * units : units), 128, 0, stream>>>(
+        static_cast<const uint16_t *>(W), meta, map, K, tn, tk, scale, table, ptable, units, out);
     note_launches(2);
     return cudaGetLastError();
 }

@@ -672,6 +672,25 @@ patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint
                 off += patchk::kDenseStepBytes;
             }
         }
+    // prefill table for the two-SM kernel (even band counts): bands 2p and
+    // 2p+1 take the same kind at every k-step; where one is 2:4 and the other
+    // dense, the 2:4 band's k-step gets a dense side copy of its W_eff codes
+    // after the packed bytes
+    const bool duo = bands % 2 == 0;
+    std::vector<uint64_t> ptable(duo ? table.size() : 0);
+    uint64_t side = 0;
+    if (duo)
+        for (int64_t bp = 0; bp < bands / 2; ++bp)
+            for (int64_t c = 0; c < steps; ++c) {
+                const size_t i0 = static_cast<size_t>(2 * bp * steps + c), i1 = i0 + static_cast<size_t>(steps);
+                ptable[i0] = table[i0];
+                ptable[i1] = table[i1];
+                const bool s0 = (table[i0] & patchk::kEntrySparse) != 0, s1 = (table[i1] & patchk::kEntrySparse) != 0;
+                if (s0 != s1) {
+                    ptable[s0 ? i0 : i1] = (off + side) | patchk::kEntrySide;
+                    side += patchk::kDenseStepBytes;
+                }
+            }
     patch_packed *h = new (std::nothrow) patch_packed();
     if (!h) return PATCH_ERR_OOM;
     cudaGetDevice(&h->device);
@@ -680,10 +699,14 @@ patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint
     h->num_sms = num_sms;
     h->bands = bands;
     h->packed_bytes = off;
+    h->side_bytes = side;
+    h->duo_ok = duo ? 1 : 0;
     h->sparse_ksteps = static_cast<int64_t>(n_sparse);
     h->meta_blocks = static_cast<int64_t>(n_sparse);
-    // allocation 1: table | row scales | status; allocation 2: the packed bytes
-    const size_t off_scale = round_up(sizeof(uint64_t) * table.size(), 256);
+    // allocation 1: table | prefill table | row scales | status; allocation
+    // 2: the packed bytes, then the side copies
+    const size_t off_ptable = round_up(sizeof(uint64_t) * table.size(), 256);
+    const size_t off_scale = round_up(off_ptable + sizeof(uint64_t) * ptable.size(), 256);
     const size_t off_status = round_up(off_scale + sizeof(float) * static_cast<size_t>(N), 256);
     const size_t total = off_status + 256;
     e = patchk::device_pool(&h->pool);
@@ -693,20 +716,23 @@ patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint
         return from_cuda(e);
     }
     h->table = reinterpret_cast<uint64_t *>(h->base);
-    h->ptable = h->table;
+    h->ptable = duo ? reinterpret_cast<uint64_t *>(h->base + off_ptable) : nullptr;
     h->fp8_scale = reinterpret_cast<float *>(h->base + off_scale);
     h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
     e = cudaMemsetAsync(h->status, 0, 256, stream);
     if (e == cudaSuccess)
-        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->packed), std::max<size_t>(off, 16), h->pool,
-                                    stream);
-    // pageable source: the call returns once the table has been staged
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->packed), std::max<size_t>(off + side, 16),
+                                    h->pool, stream);
+    // pageable sources: the call returns once the tables have been staged
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(h->table, table.data(), sizeof(uint64_t) * table.size(), cudaMemcpyHostToDevice,
                             stream);
+    if (e == cudaSuccess && duo)
+        e = cudaMemcpyAsync(h->ptable, ptable.data(), sizeof(uint64_t) * ptable.size(), cudaMemcpyHostToDevice,
+                            stream);
     if (e == cudaSuccess)
         e = patchk::launch_pack_fp8(W_bf16, meta, map, N, K, static_cast<int>(tn), static_cast<int>(tk),
-                                    h->table, h->fp8_scale, h->packed, stream);
+                                    h->table, h->ptable, h->fp8_scale, h->packed, stream);
     if (e != cudaSuccess) {
         patch_free(h, stream_v);
         return from_cuda(e);
@@ -737,6 +763,10 @@ static patch_status fp8_gemm(const patch_packed *Wp, const void *X_bf16, int64_t
         patchk::Fp8Launch g;
         g.packed = Wp->packed;
         g.table = Wp->table;
+        g.ptable = Wp->ptable;
+        g.packed_bytes = Wp->packed_bytes + Wp->side_bytes;
+        g.all_sparse = Wp->sparse_ksteps == Wp->bands * (Wp->shp.K / 128) ? 1 : 0;
+        g.force_kernel = g_test_kernel.load(std::memory_order_relaxed);
         g.sw = Wp->fp8_scale;
         g.xq = ws;
         g.sx = sx;

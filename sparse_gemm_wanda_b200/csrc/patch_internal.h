@@ -170,22 +170,40 @@ size_t decode_workspace_bytes(int nchunks);
 cudaError_t launch_fp8_quantize_rows(const void *x, int64_t R, int64_t C, uint8_t *q, float *scale,
                                      cudaStream_t stream);
 // W_eff row scales into `scale` [N] and the packed k-steps at the table's offsets.
+// ptable (nullable): the prefill table; its side entries (kEntrySide) get
+// dense copies of their k-steps' W_eff codes
 cudaError_t launch_pack_fp8(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
-                            int64_t K, int tn, int tk, const uint64_t *table, float *scale,
-                            uint8_t *out, cudaStream_t stream);
+                            int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
+                            float *scale, uint8_t *out, cudaStream_t stream);
 struct Fp8Launch {
     const uint8_t *packed;
-    const uint64_t *table;  // [N/128][K/128]
-    const float *sw;        // [N]
-    const uint8_t *xq;      // [M, K] e4m3 codes of X
-    const float *sx;        // [M]
+    const uint64_t *table;   // [N/128][K/128]
+    const uint64_t *ptable;  // prefill table (even band counts), else null
+    uint64_t packed_bytes;   // packed k-steps + side copies
+    int all_sparse;          // every k-step 2:4 (no dense weight slot needed)
+    const float *sw;         // [N]
+    const uint8_t *xq;       // [M, K] e4m3 codes of X
+    const float *sx;         // [M]
     int64_t N, K, M;
     void *Y;
     int y_fp32;
     uint32_t *status;
     int num_sms;
+    int force_kernel;        // test hook: 1 = one band per CTA, 3 = two-SM kernel, 0 = chosen here
 };
 cudaError_t launch_fp8_gemm(const Fp8Launch &g, cudaStream_t stream);
+
+// Two-SM FP8 prefill GEMM (csrc/prefill_duo_fp8.cu): bands 2p, 2p+1 of the
+// prefill table on a CTA pair, one 128-column k-step per stage.
+struct DuoFp8Plan {
+    int bn;           // tokens per tile (each CTA of the pair holds bn / 2)
+    int ttiles, items;
+    int clusters;     // CTA pairs launched
+    int stages, stage_bytes, smem;
+    int aslot;        // weight slot of a stage
+};
+DuoFp8Plan plan_duo_fp8(int64_t N, int64_t M, int num_sms, bool all_sparse);
+cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStream_t stream);
 
 // The library's stream-ordered memory pool for the current device (cached
 // memory is kept, not returned to the system between calls).

@@ -1,0 +1,517 @@
+// Two-SM FP8 hybrid GEMM for prefill: tcgen05 kind::f8f6f4 with
+// cta_group::2 (sm_100a).  Y = diag(sx) (QX QW^T) diag(sw), the product of
+// the FP8 path ("SparseGPT vs Wanda: one-shot LLM pruning without
+// retraining", FAQ: prune first, then quantise; the tile scheme of "PATCH:
+// Learnable Tile-level Hybrid Sparsity for LLMs", section 2).
+//
+// Why.  The tensor core reads its operands from shared memory and the TMA
+// copies write there too, about 128 B per cycle per SM in all.  With one CTA
+// per MMA every SM writes and reads the whole token tile; with cta_group::2 a
+// CTA pair runs M = 256 MMAs (one 128-row band per SM) and each SM holds
+// HALF of the token tile, which cuts an SM's shared-memory bytes per
+// 128-column k-step from 92 KB to 62 KB at 240 tokens.
+//
+// Work item = (band pair, token tile of BN tokens); clusters of two CTAs take
+// items c, c + C, ...; CTA rank r owns band 2p + r and tokens [r BN/2,
+// (r+1) BN/2) of the tile.  Stage = one 128-column k-step: this SM's band
+// (ONE TMA load of 16 KB dense or 2 KB metadata + 8 KB codes, through tensor
+// maps over the packed buffer in 2 KB rows) and its half of the X codes (ONE
+// TMA load, 128-byte swizzle, rows past M zero), issued by two threads in
+// different warps.  Both CTAs' loads complete on the leader's stage mbarrier.
+// The bands of a pair take one kind at every k-step through the prefill table
+// (a 2:4 k-step whose partner is dense points to a dense side copy).  The
+// leader's MMA thread issues 4 dense K32 or 2 sparse K64 M256 x BN MMAs per
+// stage (the 2:4 metadata of sparse MMA q at tensor-memory column e + 2q);
+// a commit with a CTA mask frees the stage in both CTAs and hands each
+// accumulator to both epilogues, which scale by sw[n] sx[m] and round once.
+// Two accumulators alternate between items (2 x BN + 4 metadata columns).
+//
+// Every mbarrier wait is bounded by %globaltimer; a CTA that gives up raises
+// its own and its peer's abort flag, drains its copies and still meets its
+// peer at the final cluster barrier, so both CTAs free tensor memory together.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "patch_cluster.cuh"
+#include "patch_common.cuh"
+#include "patch_internal.h"
+
+namespace patchk {
+
+namespace {
+
+constexpr int kD8Threads = 288;   // warps 0, 7: weight producers; 6, 8: X producers
+constexpr int kD8Producers = 2;   // issuing threads per copy stream (stage s: producer s % 2)
+constexpr int kD8Step = 128;      // columns (code bytes) per k-step
+constexpr int kD8MaxStages = 8;
+constexpr int kD8TabSteps = 224;  // k-steps per band (K <= 28672)
+constexpr int kD8TabBytes = kD8Producers * 2 * kD8TabSteps * 8;
+constexpr int kD8TmemCols = 512;
+constexpr int kD8SmemLimit = 232448;
+constexpr int kD8TailBytes = 1024 + kD8TabBytes + 512;
+constexpr uint64_t kD8WaitLimitNs = 2000000000ull;
+
+struct D8Params {
+    const uint64_t *table;   // prefill table [bands][steps]
+    const float *sw, *sx;
+    int64_t N, K, M;
+    int steps, ttiles, items;
+    int bn, half, stages, stage_bytes, aslot;
+    void *Y;
+    int y_fp32;
+    uint32_t *status;
+};
+
+struct D8Maps {
+    CUtensorMap x, a_dense, a_sparse;
+};
+
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_f8_sparse_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                   uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// kind::f8f6f4 instruction descriptor: A and B e4m3 (format 0), K-major, fp32
+// D, M = 256, the given N; `sparse` sets the 2:4 flag (selector 0).
+__host__ __device__ constexpr uint32_t idesc_e4m3_pair(int n, bool sparse) {
+    return (sparse ? (1u << 2) : 0u) | (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(256 >> 4) << 24);
+}
+
+__device__ __forceinline__ void store_y(const D8Params &p, int64_t idx, float v) {
+    if (p.y_fp32)
+        static_cast<float *>(p.Y)[idx] = v;
+    else
+        static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
+}
+
+__global__ void __launch_bounds__(kD8Threads, 1)
+duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int S = p.stages;
+    uint64_t *tab_buf = reinterpret_cast<uint64_t *>(smem + S * p.stage_bytes);  // [producer][2][224]
+    uint64_t *full = tab_buf + kD8Producers * 2 * kD8TabSteps;  // leader: all loads of both CTAs
+    uint64_t *empty = full + kD8MaxStages;        // both: freed by the leader's commit
+    uint64_t *acc_full = empty + kD8MaxStages;    // [2] both
+    uint64_t *acc_empty = acc_full + 2;           // [2] leader: 4 warps x 2 CTAs
+    uint64_t *tab_full = acc_empty + 2;           // [producer][2] own table copies
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tab_full + 2 * kD8Producers);
+    volatile uint32_t *abort_flag = tmem_slot + 1;
+    volatile uint32_t *never_flag = tmem_slot + 2;
+    uint64_t *stage_info = reinterpret_cast<uint64_t *>(tmem_slot + 4);  // [S]: the k-step's entry
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_rank();
+    const int cl = blockIdx.x / 2, C = gridDim.x / 2;
+    const int bn = p.bn, half = p.half;
+
+    // weight producer j keeps its own two item tables
+    auto fetch_table = [&](int j, int item, int buf) {
+        const int band = 2 * (item / p.ttiles) + static_cast<int>(rank);
+        const uint32_t nb = static_cast<uint32_t>(p.steps) * 8u;
+        mbar_arrive_expect_tx(&tab_full[2 * j + buf], nb);
+        bulk_g2s(tab_buf + (2 * j + buf) * kD8TabSteps, p.table + static_cast<int64_t>(band) * p.steps, nb,
+                 &tab_full[2 * j + buf]);
+    };
+    auto give_up = [&]() {
+        *abort_flag = 1u;
+        st_cluster_u32(map_to_rank(const_cast<uint32_t *>(abort_flag), rank ^ 1u), 1u);
+        atomicOr(p.status, kStatusTimeout);
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kD8MaxStages; ++s) {
+            mbar_init(&full[s], 2);  // the leader's weight and X producers
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);
+        }
+        for (int b = 0; b < 2 * kD8Producers; ++b) mbar_init(&tab_full[b], 1);
+        *never_flag = 0u;
+        *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
+        fence_mbar_init_cluster();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, kD8TmemCols);
+        tmem_relinquish_pair();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&maps.x);
+        prefetch_tmap(&maps.a_dense);
+        prefetch_tmap(&maps.a_sparse);
+    }
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all();  // both CTAs' barriers and tensor memory exist from here on
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const bool skip = *abort_flag != 0;
+    if (warp == 0 || warp == 7) {
+        const int j = warp == 0 ? 0 : 1;  // stages s with s % 2 == j
+        if (lane == 0 && !skip) {
+            // ----------------------------------------------- weight producer
+            for (int i = 0; i < 2 && cl + i * C < p.items; ++i) fetch_table(j, cl + i * C, i);
+            int it = 0;
+            bool ok = true;
+            int tabs = 0;
+            for (int i = 0; i < 2 && cl + i * C < p.items; ++i) ++tabs;
+            for (int i = 0; ok; ++i) {
+                const int item = cl + i * C;
+                if (item >= p.items) break;
+                const int buf = i & 1;
+                if (!mbar_wait_bounded(&tab_full[2 * j + buf], (i >> 1) & 1u, abort_flag, kD8WaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                const uint64_t *tab = tab_buf + (2 * j + buf) * kD8TabSteps;
+                for (int c = 0; c < p.steps; ++c, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if ((it & 1) != j) continue;
+                    if (it >= S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kD8WaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint64_t e = tab[c];
+                    const bool sp = (e & kEntrySparse) != 0;
+                    const uint64_t first = (e & kEntryOffsetMask) - (sp ? kMetaBlockBytes : 0);
+                    const uint32_t a_bytes = sp ? kMetaBlockBytes + kSparseStepBytes : kDenseStepBytes;
+                    stage_info[s] = e;
+                    // both bands of the pair take this kind: the leader arms
+                    // its barrier for both CTAs' weight bytes
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * a_bytes);
+                    tma2d_pair(smem + s * p.stage_bytes, sp ? &maps.a_sparse : &maps.a_dense, 0,
+                               static_cast<int32_t>(first / 2048), map_to_rank(&full[s], 0));
+                }
+                if (ok && cl + (i + 2) * C < p.items) {
+                    fetch_table(j, cl + (i + 2) * C, buf);
+                    ++tabs;
+                }
+            }
+            for (int q = (tabs > 2 ? tabs - 2 : 0); q < tabs; ++q)
+                mbar_wait_bounded(&tab_full[2 * j + (q & 1)], (q >> 1) & 1u, never_flag, kD8WaitLimitNs / 4);
+            if (!ok) give_up();
+            // drain (this producer's stages): the leader waits for their last
+            // phase (its barrier counts both CTAs' loads); the peer until the
+            // leader's MMAs have released them, or gives up
+            for (int q = (it > S ? it - S : 0); q < it; ++q) {
+                if ((q & 1) != j) continue;
+                if (rank == 0)
+                    mbar_wait_bounded(&full[q % S], (q / S) & 1u, never_flag, kD8WaitLimitNs / 4);
+                else
+                    mbar_wait_bounded(&empty[q % S], (q / S) & 1u, never_flag, kD8WaitLimitNs / 4);
+            }
+        }
+    } else if (warp == 6 || warp == 8) {
+        const int j = warp == 6 ? 0 : 1;
+        if (lane == 0 && !skip) {
+            // ---------------------------------------------------- X producer
+            const uint32_t x_bytes = 2u * static_cast<uint32_t>(half) * kD8Step;  // both CTAs
+            int it = 0;
+            bool ok = true;
+            for (int i = 0; ok; ++i) {
+                const int item = cl + i * C;
+                if (item >= p.items) break;
+                const int tt = item % p.ttiles;
+                for (int c = 0; c < p.steps; ++c, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if ((it & 1) != j) continue;
+                    if (it >= S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kD8WaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], x_bytes);
+                    tma2d_pair(smem + s * p.stage_bytes + p.aslot, &maps.x, c * kD8Step,
+                               tt * bn + static_cast<int>(rank) * half, map_to_rank(&full[s], 0));
+                }
+            }
+            if (!ok) give_up();
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && !skip && rank == 0) {
+            // ------------------------------------------------- MMA (leader)
+            const uint32_t e_tmem = tmem_base + static_cast<uint32_t>(2 * bn);
+            const uint32_t id_dense = idesc_e4m3_pair(bn, false), id_sparse = idesc_e4m3_pair(bn, true);
+            constexpr DescBase kDescDenseA = smem_desc_base(16, 1024, kSwizzle128B);
+            constexpr DescBase kDescSparseA = smem_desc_base(16, 512, kSwizzle64B);
+            constexpr DescBase kDescX = smem_desc_base(16, 1024, kSwizzle128B);
+            constexpr DescBase kDescMeta = smem_desc_base(16, 128, kSwizzleNone);
+            int it = 0;
+            bool ok = true;
+            for (int i = 0; ok; ++i) {
+                const int item = cl + i * C;
+                if (item >= p.items) break;
+                const int buf = i & 1;
+                if (i >= 2 &&
+                    !mbar_wait_bounded(&acc_empty[buf], ((i >> 1) & 1u) ^ 1u, abort_flag, kD8WaitLimitNs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * bn);
+                for (int c = 0; c < p.steps; ++c, ++it) {
+                    const int s = it % S;
+                    const uint32_t ph = (it / S) & 1u;
+                    if (!mbar_wait_bounded(&full[s], ph, abort_flag, kD8WaitLimitNs)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t slot = smem_u32(smem + s * p.stage_bytes);
+                    const uint32_t s16 = slot >> 4, b16 = (slot + static_cast<uint32_t>(p.aslot)) >> 4;
+                    if (stage_info[s] & kEntrySparse) {
+                        tmem_cp_pair_128x128b(e_tmem, desc_at(kDescMeta, s16));
+#pragma unroll
+                        for (int q = 0; q < 2; ++q)
+                            mma_f8_sparse_pair(d_tmem, desc_at(kDescSparseA, s16 + kMetaBlockBytes / 16 + 2 * q),
+                                               desc_at(kDescX, b16 + 4 * q), e_tmem + 2 * q, id_sparse,
+                                               (c == 0 && q == 0) ? 0u : 1u);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            mma_f8_pair(d_tmem, desc_at(kDescDenseA, s16 + 2 * q), desc_at(kDescX, b16 + 2 * q),
+                                        id_dense, (c == 0 && q == 0) ? 0u : 1u);
+                    }
+                    tc_commit_pair(&empty[s]);
+                }
+                // fires once every MMA of the item has completed (also after a
+                // failure, so no epilogue frees tensor memory under a running MMA)
+                tc_commit_pair(&acc_full[buf]);
+            }
+            if (!ok) give_up();
+        }
+    } else if (warp >= 2 && warp <= 5 && !skip) {
+        // ---------------------------------------------- epilogue (both CTAs)
+        const int quad = warp % 4;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+        for (int i = 0;; ++i) {
+            const int item = cl + i * C;
+            if (item >= p.items) break;
+            const int bp = item / p.ttiles, tt = item % p.ttiles;
+            const int buf = i & 1;
+            const bool ok = mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1u, never_flag, kD8WaitLimitNs);
+            tc_fence_after();
+            if (!ok) {
+                give_up();
+                break;
+            }
+            const int64_t n = static_cast<int64_t>(2 * bp + static_cast<int>(rank)) * kBand + row;
+            const int64_t m_base = static_cast<int64_t>(tt) * bn;
+            const int m_valid = static_cast<int>(min(static_cast<int64_t>(bn), p.M - m_base));
+            const float swn = __ldg(p.sw + n);
+            if (*abort_flag == 0) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < m_valid; c0 += 16) {
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(buf * bn + c0), r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        if (c0 + q < m_valid) {
+                            const int64_t m = m_base + c0 + q;
+                            store_y(p, m * p.N + n, __uint_as_float(r[q]) * swn * __ldg(p.sx + m));
+                        }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(map_to_rank(&acc_empty[buf], 0));
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    cluster_sync_all();  // the peer's MMAs and remote arrivals are all done
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem_base, kD8TmemCols);
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// the packed buffer as rows of 2 KB (256 x 8-byte elements), box of `box_rows`
+bool encode_rows(EncodeTiledFn enc, CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {256, rows};
+    const cuuint64_t strides[1] = {2048};
+    const cuuint32_t box[2] = {256, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t ensure_attributes() {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(duo_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kD8SmemLimit);
+    });
+    return attr_err;
+}
+
+// clusters of two CTAs that fit on the device at once with `smem` bytes each
+int max_clusters(int smem) {
+    if (ensure_attributes() != cudaSuccess) return 0;
+    static std::mutex mu;
+    static int cached_smem = -1, cached = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached_smem == smem) return cached;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(kD8Threads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, duo_fp8_kernel, &cfg) != cudaSuccess) n = 0;
+    cached_smem = smem;
+    cached = n;
+    return n;
+}
+
+}  // namespace
+
+DuoFp8Plan plan_duo_fp8(int64_t N, int64_t M, int num_sms, bool all_sparse) {
+    DuoFp8Plan best{};
+    const int64_t bpairs = (N / kBand) / 2;
+    // shared memory per stage: the weight slot (a dense k-step, or metadata +
+    // codes when no k-step of the matrix is dense) + BN/2 X rows of 128 B
+    const int aslot = all_sparse ? kMetaBlockBytes + kSparseStepBytes : kDenseStepBytes;
+    auto smem_for = [aslot](int bn, int *stages, int *stage_bytes) {
+        *stage_bytes = aslot + (bn / 2) * kD8Step;
+        *stages = std::min(kD8MaxStages, (kD8SmemLimit - kD8TailBytes) / *stage_bytes);
+        return *stages * *stage_bytes + kD8TailBytes;
+    };
+    int st = 0, sb = 0;
+    const int clusters_cap = max_clusters(smem_for(128, &st, &sb));
+    if (clusters_cap < 1) return best;
+    const int clusters = std::min(clusters_cap, num_sms / 2);
+    // per SM per dense k-step: max(MMA cycles (4 x BN/2), shared-memory bytes
+    // (weights and X half written by the copies and read by the MMAs) at
+    // 128 B per cycle); the last wave counts whole
+    double best_cost = 0;
+    for (int bn = 240; bn >= 128; bn -= 16) {
+        const int64_t tt = (M + bn - 1) / bn;
+        const int64_t items = bpairs * tt;
+        const int64_t waves = (items + clusters - 1) / clusters;
+        const double kstep = std::max(2.0 * bn, 2.0 * (aslot + 64.0 * bn) / 128.0);
+        const double cost = static_cast<double>(waves) * kstep;
+        if (best.bn == 0 || cost < best_cost) {
+            best_cost = cost;
+            best.bn = bn;
+            best.ttiles = static_cast<int>(tt);
+            best.items = static_cast<int>(items);
+            best.clusters = static_cast<int>(std::min<int64_t>(clusters, items));
+        }
+    }
+    best.smem = smem_for(best.bn, &best.stages, &best.stage_bytes);
+    best.aslot = aslot;
+    return best;
+}
+
+cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStream_t stream) {
+    const cudaError_t attr_err = ensure_attributes();
+    if (attr_err != cudaSuccess) return attr_err;
+    const int64_t steps = g.K / kD8Step;
+    if (plan.bn < 128 || plan.stages < 2 || plan.smem > kD8SmemLimit || plan.clusters < 1)
+        return cudaErrorInvalidValue;
+    if ((g.N / kBand) % 2 != 0 || steps % 2 != 0 || steps > kD8TabSteps || !g.ptable || !g.packed_bytes)
+        return cudaErrorInvalidValue;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorInvalidValue;
+    D8Maps maps;
+    // X codes [M, K] uint8 row-major: box = 128 bytes x this CTA's half of the
+    // token tile, 128-byte swizzle, rows past M read as zero
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(g.K), static_cast<cuuint64_t>(g.M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(g.K)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kD8Step), static_cast<cuuint32_t>(plan.bn / 2)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&maps.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(g.xq), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const uint64_t rows = g.packed_bytes / 2048;  // packed + side copies, in 2 KB rows
+    if (!encode_rows(enc, &maps.a_dense, g.packed, rows, kDenseStepBytes / 2048) ||
+        !encode_rows(enc, &maps.a_sparse, g.packed, rows, (kMetaBlockBytes + kSparseStepBytes) / 2048))
+        return cudaErrorInvalidValue;
+    D8Params p;
+    p.table = g.ptable;
+    p.sw = g.sw;
+    p.sx = g.sx;
+    p.N = g.N;
+    p.K = g.K;
+    p.M = g.M;
+    p.steps = static_cast<int>(steps);
+    p.ttiles = plan.ttiles;
+    p.items = plan.items;
+    p.bn = plan.bn;
+    p.half = plan.bn / 2;
+    p.stages = plan.stages;
+    p.stage_bytes = plan.stage_bytes;
+    p.aslot = plan.aslot;
+    p.Y = g.Y;
+    p.y_fp32 = g.y_fp32;
+    p.status = g.status;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * plan.clusters));
+    cfg.blockDim = dim3(kD8Threads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(plan.smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t err = cudaLaunchKernelEx(&cfg, duo_fp8_kernel, maps, p);
+    if (err == cudaSuccess) note_launches(1);
+    return err;
+}
+
+}  // namespace patchk

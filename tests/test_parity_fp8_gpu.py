@@ -90,6 +90,19 @@ def test_pack_fp8_bit_exact(P, oracle_mod, tn, tk, frac):
     pk.close()
 
 
+class forced_kernel:
+    """Select the prefill kernel for the calls inside the block (test hook)."""
+
+    def __init__(self, P, which):
+        self.P, self.which = P, which
+
+    def __enter__(self):
+        self.P.test_prefill_kernel(self.which)
+
+    def __exit__(self, *exc):
+        self.P.test_prefill_kernel(0)
+
+
 def run_fp8_gemm(P, oracle_mod, N, K, M, tn, tk, frac, seed, fp32_mode, sample=None):
     w = inputs.weight(N, K, seed)
     o = inputs.outlier_channels(K, seed)
@@ -135,3 +148,25 @@ def test_gemm_fp8_tiles_and_fractions(P, oracle_mod, tn, tk, frac):
 def test_gemm_fp8_llama_mlp_shape(P, oracle_mod, M, frac):
     run_fp8_gemm(P, oracle_mod, 11008, 4096, M, 128, 128, frac, seed=91 + M, fp32_mode=False,
                  sample=4000 if M > 16 else None)
+
+
+@pytest.mark.parametrize("N,K,M,tn,tk,frac", [
+    (1024, 1024, 700, 128, 128, 0.5),   # random map: side copies where a band pair differs
+    (1024, 1024, 700, 128, 128, 1.0),   # every k-step 2:4 (the smaller weight slot)
+    (1024, 1024, 700, 128, 128, 0.0),   # every k-step dense
+    (768, 512, 333, 64, 64, 0.5),       # 64-row tiles: halves of a band differ
+    (512, 1536, 1000, 128, 64, 0.75),   # 64-column tiles
+    (256, 768, 129, 128, 128, 0.5),     # one band pair, a ragged second tile
+])
+@pytest.mark.parametrize("kernel", [1, 3])
+def test_gemm_fp8_one_band_and_two_sm(P, oracle_mod, N, K, M, tn, tk, frac, kernel):
+    # the same FP8 handle through the one-band kernel (1) and the two-SM
+    # kernel on the prefill table (3), compared in full with the oracle
+    with forced_kernel(P, kernel):
+        run_fp8_gemm(P, oracle_mod, N, K, M, tn, tk, frac, seed=N + M + tn + tk + kernel, fp32_mode=True)
+
+
+def test_gemm_fp8_odd_kstep_count_falls_back(P, oracle_mod):
+    # an odd number of 128-column k-steps (K = 384) keeps the one-band kernel
+    with forced_kernel(P, 3):
+        run_fp8_gemm(P, oracle_mod, 512, 384, 300, 128, 128, 0.5, seed=17, fp32_mode=False)
