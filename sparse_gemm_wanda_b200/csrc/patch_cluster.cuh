@@ -93,6 +93,36 @@ __device__ __forceinline__ void mma_sparse_pair(uint32_t d_tmem, uint64_t a_desc
         "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// One k-step of MMAs back to back in one asm block (descriptors computed up
+// front): four dense M256 K16 MMAs, or two 2:4 M256 K32 MMAs with metadata
+// selectors 0 and 1.  `accumulate` applies to the first MMA; the others
+// always accumulate.
+__device__ __forceinline__ void mma_dense_pair_x4(uint32_t d_tmem, uint64_t a0, uint64_t a1, uint64_t a2,
+                                                  uint64_t a3, uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3,
+                                                  uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t"
+        "setp.ne.b32 p, %10, 0;\n\t"
+        "setp.eq.b32 t, %9, %9;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %5, %9, p;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %2, %6, %9, t;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %3, %7, %9, t;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %4, %8, %9, t;\n\t}\n" ::"r"(d_tmem),
+        "l"(a0), "l"(a1), "l"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_sparse_pair_x2(uint32_t d_tmem, uint64_t a0, uint64_t a1, uint64_t b0,
+                                                   uint64_t b1, uint32_t e_tmem, uint32_t idesc0, uint32_t idesc1,
+                                                   uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t"
+        "setp.ne.b32 p, %8, 0;\n\t"
+        "setp.eq.b32 t, %6, %6;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %3, [%5], %6, p;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %2, %4, [%5], %7, t;\n\t}\n" ::"r"(d_tmem),
+        "l"(a0), "l"(a1), "l"(b0), "l"(b1), "r"(e_tmem), "r"(idesc0), "r"(idesc1), "r"(accumulate)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_cp_pair_128x128b(uint32_t taddr, uint64_t s_desc) {
     asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");
 }

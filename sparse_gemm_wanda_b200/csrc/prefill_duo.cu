@@ -101,7 +101,11 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tab_full + 2);
     volatile uint32_t *abort_flag = tmem_slot + 1;
     volatile uint32_t *never_flag = tmem_slot + 2;
-    uint64_t *stage_info = reinterpret_cast<uint64_t *>(tmem_slot + 4);  // [S][2]: the pair's entries
+    // [S]: the stage's k-pair for the MMA thread, packed by the weight producer:
+    // bits 0-10 / 11-21 = k-step 0 / 1 values' offset in the stage (16-byte
+    // units), bits 22 / 23 = k-step 0 / 1 is 2:4, bits 24 / 25 = its
+    // metadata block precedes it
+    uint32_t *stage_word = tmem_slot + 4;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cluster_rank();
@@ -192,8 +196,10 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
                     const uint64_t end = (e1 & kEntryOffsetMask) +
                                          ((e1 & kEntrySparse) ? kSparseStepBytes : kDenseStepBytes);
                     const uint32_t a_bytes = static_cast<uint32_t>(end - first);  // 32, 26 or 18 KB
-                    stage_info[2 * s + 0] = e0;
-                    stage_info[2 * s + 1] = e1;
+                    stage_word[s] = static_cast<uint32_t>(((e0 & kEntryOffsetMask) - first) >> 4) |
+                                    (static_cast<uint32_t>(((e1 & kEntryOffsetMask) - first) >> 4) << 11) |
+                                    ((e0 & kEntrySparse) ? 1u << 22 : 0u) | ((e1 & kEntrySparse) ? 1u << 23 : 0u) |
+                                    ((e0 & kEntryMeta) ? 1u << 24 : 0u) | ((e1 & kEntryMeta) ? 1u << 25 : 0u);
                     ++it;
                     if (p.stall_first_kstep && blockIdx.x == 0 && it == 1) continue;  // never lands
                     // the two bands of a pair agree in kind and metadata placement,
@@ -262,7 +268,14 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
             constexpr DescBase kDescSparseA = smem_desc_base(16, 512, kSwizzle64B);
             constexpr DescBase kDescX = smem_desc_base(16, 1024, kSwizzle128B);
             constexpr DescBase kDescMeta = smem_desc_base(16, 128, kSwizzleNone);
-            int it = 0;
+            // the stage and its phase advance without division; a stage's
+            // shared-memory addresses in 16-byte units
+            const uint32_t smem16 = smem_u32(smem) >> 4;
+            const uint32_t stage16 = static_cast<uint32_t>(p.stage_bytes) >> 4;
+            const uint32_t aslot16 = static_cast<uint32_t>(p.aslot) >> 4;
+            const uint32_t xk16 = static_cast<uint32_t>(half * kStep * 2) >> 4;  // one k-step of X rows
+            int s = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int i = 0; ok; ++i) {
                 const int item = cl + i * C;
@@ -275,40 +288,37 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * bn);
-                for (int pr = 0; pr < p.nsteps / 2; ++pr, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1u;
+                for (int pr = 0; pr < p.nsteps / 2; ++pr) {
                     if (!mbar_wait_bounded(&full[s], ph, abort_flag, kDuoWaitLimitNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t slot = smem_u32(smem + s * p.stage_bytes);
-                    const uint64_t e0 = stage_info[2 * s];
-                    const uint64_t first = (e0 & kEntryOffsetMask) - ((e0 & kEntryMeta) ? kMetaBlockBytes : 0);
+                    const uint32_t w = stage_word[s];
+                    const uint32_t slot16 = smem16 + static_cast<uint32_t>(s) * stage16;
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const uint64_t e = stage_info[2 * s + h];
-                        const uint32_t a_addr = slot + static_cast<uint32_t>((e & kEntryOffsetMask) - first);
-                        const uint32_t b_addr = slot + static_cast<uint32_t>(p.aslot + h * half * kStep * 2);
+                        const uint32_t a16 = slot16 + ((w >> (11 * h)) & 0x7FFu);
+                        const uint32_t b16 = slot16 + aslot16 + static_cast<uint32_t>(h) * xk16;
                         const bool fresh = pr == 0 && h == 0;
-                        // descriptors: constant fields + 16-byte address units
-                        const uint32_t a16 = a_addr >> 4, b16 = b_addr >> 4;
-                        if (e & kEntrySparse) {
-                            if (e & kEntryMeta)
-                                tmem_cp_pair_128x128b(e_tmem, desc_at(kDescMeta, (a_addr - kMetaBlockBytes) >> 4));
-#pragma unroll
-                            for (int q = 0; q < 2; ++q)
-                                mma_sparse_pair(d_tmem, desc_at(kDescSparseA, a16 + 2 * q), desc_at(kDescX, b16 + 4 * q),
-                                                e_tmem + 2 * h, idesc_sparse[q], (fresh && q == 0) ? 0u : 1u);
+                        if (w & (1u << (22 + h))) {
+                            if (w & (1u << (24 + h)))
+                                tmem_cp_pair_128x128b(e_tmem, desc_at(kDescMeta, a16 - kMetaBlockBytes / 16));
+                            mma_sparse_pair_x2(d_tmem, desc_at(kDescSparseA, a16), desc_at(kDescSparseA, a16 + 2),
+                                               desc_at(kDescX, b16), desc_at(kDescX, b16 + 4), e_tmem + 2 * h,
+                                               idesc_sparse[0], idesc_sparse[1], fresh ? 0u : 1u);
                         } else {
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                mma_dense_pair(d_tmem, desc_at(kDescDenseA, a16 + 2 * q), desc_at(kDescX, b16 + 2 * q),
-                                               idesc_dense, (fresh && q == 0) ? 0u : 1u);
+                            mma_dense_pair_x4(d_tmem, desc_at(kDescDenseA, a16), desc_at(kDescDenseA, a16 + 2),
+                                              desc_at(kDescDenseA, a16 + 4), desc_at(kDescDenseA, a16 + 6),
+                                              desc_at(kDescX, b16), desc_at(kDescX, b16 + 2), desc_at(kDescX, b16 + 4),
+                                              desc_at(kDescX, b16 + 6), idesc_dense, fresh ? 0u : 1u);
                         }
                     }
                     tc_commit_pair(&empty[s]);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 // fires once every MMA of the item has completed (also after a
                 // failure, so no epilogue frees tensor memory under a running MMA)
