@@ -194,13 +194,14 @@ struct Fp8Launch {
 cudaError_t launch_fp8_gemm(const Fp8Launch &g, cudaStream_t stream);
 
 // Two-SM FP8 prefill GEMM (csrc/prefill_duo_fp8.cu): bands 2p, 2p+1 of the
-// prefill table on a CTA pair, one 128-column k-step per stage.
+// prefill table on a CTA pair, two 128-column k-steps per stage.
 struct DuoFp8Plan {
     int bn;           // tokens per tile (each CTA of the pair holds bn / 2)
     int ttiles, items;
     int clusters;     // CTA pairs launched
     int stages, stage_bytes, smem;
-    int aslot;        // weight slot of a stage
+    int aslot;        // weight slot of a stage (two k-steps)
+    int aslot_step;   // its half for one k-step
 };
 DuoFp8Plan plan_duo_fp8(int64_t N, int64_t M, int num_sms, bool all_sparse);
 cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStream_t stream);

@@ -48,7 +48,7 @@ namespace patchk {
 
 namespace {
 
-constexpr int kDuoThreads = 224;   // + warp 6: the X-tile producer
+constexpr int kDuoThreads = 352;   // warps 0 weights, 1 MMA, 6 X tiles; 2-5 and 7-10 the two epilogue groups
 constexpr int kDuoMaxStages = 8;
 constexpr int kDuoTabSteps = 448;                      // k-steps per band (K <= 28672)
 constexpr int kDuoTabBytes = 2 * kDuoTabSteps * 8;     // two items of one band
@@ -136,7 +136,7 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 8);
+            mbar_init(&acc_empty[b], 16);  // 8 epilogue warps x 2 CTAs
             mbar_init(&tab_full[b], 1);
         }
         *never_flag = 0u;
@@ -328,8 +328,11 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
         }
     } else if (!skip) {
         // ---------------------------------------------- epilogue (both CTAs)
+        // two groups of four warps (one warp per TMEM lane quarter each)
+        // take alternate 16-column chunks of an accumulator
         pdl_wait();  // Y may still be read by an earlier kernel
         const int quad = warp % 4;
+        const int grp = warp >= 7 ? 1 : 0;
         const int row = quad * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
         for (int i = 0;; ++i) {
@@ -348,13 +351,16 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
             const int m_valid = static_cast<int>(min(static_cast<int64_t>(bn), p.M - m_base));
             if (*abort_flag == 0) {
 #pragma unroll 1
-                for (int c0 = 0; c0 < m_valid; c0 += 16) {
+                for (int c0 = 16 * grp; c0 < m_valid; c0 += 32) {
                     uint32_t r[16];
                     tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(buf * bn + c0), r);
                     tmem_ld_wait();
+                    int64_t idx = (m_base + c0) * p.N + n;
 #pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        if (c0 + q < m_valid) store_y(p, (m_base + c0 + q) * p.N + n, __uint_as_float(r[q]));
+                    for (int q = 0; q < 16; ++q) {
+                        if (c0 + q < m_valid) store_y(p, idx, __uint_as_float(r[q]));
+                        idx += p.N;
+                    }
                 }
             }
             tc_fence_before();

@@ -13,18 +13,21 @@
 //
 // Work item = (band pair, token tile of BN tokens); clusters of two CTAs take
 // items c, c + C, ...; CTA rank r owns band 2p + r and tokens [r BN/2,
-// (r+1) BN/2) of the tile.  Stage = one 128-column k-step: this SM's band
-// (ONE TMA load of 16 KB dense or 2 KB metadata + 8 KB codes, through tensor
-// maps over the packed buffer in 2 KB rows) and its half of the X codes (ONE
-// TMA load, 128-byte swizzle, rows past M zero), issued by two threads in
-// different warps.  Both CTAs' loads complete on the leader's stage mbarrier.
+// (r+1) BN/2) of the tile.  Stage = two 128-column k-steps: this SM's band
+// (one TMA load per k-step of 16 KB dense or 2 KB metadata + 8 KB codes,
+// through tensor maps over the packed buffer in 2 KB rows, each into a fixed
+// half of the weight slot) and its half of the X codes for both k-steps (ONE
+// 3-D TMA load, 128-byte swizzle, rows past M zero), from a weight and an X
+// producer thread.  Both CTAs' loads complete on the leader's stage mbarrier.
 // The bands of a pair take one kind at every k-step through the prefill table
 // (a 2:4 k-step whose partner is dense points to a dense side copy).  The
 // leader's MMA thread issues 4 dense K32 or 2 sparse K64 M256 x BN MMAs per
-// stage (the 2:4 metadata of sparse MMA q at tensor-memory column e + 2q);
-// a commit with a CTA mask frees the stage in both CTAs and hands each
-// accumulator to both epilogues, which scale by sw[n] sx[m] and round once.
-// Two accumulators alternate between items (2 x BN + 4 metadata columns).
+// k-step (the 2:4 metadata of k-step h, sparse MMA q at tensor-memory column
+// e + 4h + 2q): two k-steps per stage halve the per-stage work of the issuing
+// thread against the MMAs'.  A commit with a CTA mask frees the stage in both
+// CTAs and hands each accumulator to both epilogues, which scale by sw[n]
+// sx[m] and round once.  Two accumulators alternate between items (2 x BN + 8
+// metadata columns).
 //
 // Every mbarrier wait is bounded by %globaltimer; a CTA that gives up raises
 // its own and its peer's abort flag, drains its copies and still meets its
@@ -45,12 +48,11 @@ namespace patchk {
 
 namespace {
 
-constexpr int kD8Threads = 288;   // warps 0, 7: weight producers; 6, 8: X producers
-constexpr int kD8Producers = 2;   // issuing threads per copy stream (stage s: producer s % 2)
+constexpr int kD8Threads = 352;   // warps 0 weights, 1 MMA, 6 X; 2-5 and 7-10 the two epilogue groups
 constexpr int kD8Step = 128;      // columns (code bytes) per k-step
 constexpr int kD8MaxStages = 8;
 constexpr int kD8TabSteps = 224;  // k-steps per band (K <= 28672)
-constexpr int kD8TabBytes = kD8Producers * 2 * kD8TabSteps * 8;
+constexpr int kD8TabBytes = 2 * kD8TabSteps * 8;
 constexpr int kD8TmemCols = 512;
 constexpr int kD8SmemLimit = 232448;
 constexpr int kD8TailBytes = 1024 + kD8TabBytes + 512;
@@ -62,31 +64,44 @@ struct D8Params {
     int64_t N, K, M;
     int steps, ttiles, items;
     int bn, half, stages, stage_bytes, aslot;
+    int aslot_step;          // weight bytes reserved per k-step in a stage (aslot = 2 x this)
     void *Y;
     int y_fp32;
     uint32_t *status;
 };
 
+// Tensor maps over the packed buffer as rows of 2 KB: one k-step (8 rows
+// dense, 5 rows 2:4) or two contiguous k-steps (16, 13 or 10 rows).
 struct D8Maps {
-    CUtensorMap x, a_dense, a_sparse;
+    CUtensorMap x, a_dense, a_sparse, a_dd, a_mixed, a_ss;
 };
 
-__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
+// one k-step's MMAs back to back: four dense K32, or two 2:4 K64 with the
+// metadata columns e0 and e1; `accumulate` applies to the first only
+__device__ __forceinline__ void mma_f8_pair_x4(uint32_t d_tmem, uint64_t a0, uint64_t a1, uint64_t a2, uint64_t a3,
+                                               uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3, uint32_t idesc,
+                                               uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred p, t;\n\t"
+        "setp.ne.b32 p, %10, 0;\n\t"
+        "setp.eq.b32 t, %9, %9;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %5, %9, p;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %2, %6, %9, t;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %3, %7, %9, t;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %4, %8, %9, t;\n\t}\n" ::"r"(d_tmem),
+        "l"(a0), "l"(a1), "l"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-__device__ __forceinline__ void mma_f8_sparse_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                                   uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+__device__ __forceinline__ void mma_f8_sparse_pair_x2(uint32_t d_tmem, uint64_t a0, uint64_t a1, uint64_t b0,
+                                                      uint64_t b1, uint32_t e0, uint32_t e1, uint32_t idesc,
+                                                      uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred p, t;\n\t"
+        "setp.ne.b32 p, %8, 0;\n\t"
+        "setp.eq.b32 t, %7, %7;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %1, %3, [%5], %7, p;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %2, %4, [%6], %7, t;\n\t}\n" ::"r"(d_tmem),
+        "l"(a0), "l"(a1), "l"(b0), "l"(b1), "r"(e0), "r"(e1), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -110,29 +125,29 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int S = p.stages;
-    uint64_t *tab_buf = reinterpret_cast<uint64_t *>(smem + S * p.stage_bytes);  // [producer][2][224]
-    uint64_t *full = tab_buf + kD8Producers * 2 * kD8TabSteps;  // leader: all loads of both CTAs
+    uint64_t *tab_buf = reinterpret_cast<uint64_t *>(smem + S * p.stage_bytes);  // [2][224]
+    uint64_t *full = tab_buf + 2 * kD8TabSteps;  // leader: all loads of both CTAs
     uint64_t *empty = full + kD8MaxStages;        // both: freed by the leader's commit
     uint64_t *acc_full = empty + kD8MaxStages;    // [2] both
     uint64_t *acc_empty = acc_full + 2;           // [2] leader: 4 warps x 2 CTAs
-    uint64_t *tab_full = acc_empty + 2;           // [producer][2] own table copies
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tab_full + 2 * kD8Producers);
+    uint64_t *tab_full = acc_empty + 2;           // [2] own table copies
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tab_full + 2);
     volatile uint32_t *abort_flag = tmem_slot + 1;
     volatile uint32_t *never_flag = tmem_slot + 2;
-    uint64_t *stage_info = reinterpret_cast<uint64_t *>(tmem_slot + 4);  // [S]: the k-step's entry
+    // [S]: bit h = k-step h of the stage is 2:4; bits 2-12 = where k-step 1's
+    // bytes start in the weight slot (16-byte units)
+    uint32_t *stage_word = tmem_slot + 4;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cluster_rank();
     const int cl = blockIdx.x / 2, C = gridDim.x / 2;
     const int bn = p.bn, half = p.half;
 
-    // weight producer j keeps its own two item tables
-    auto fetch_table = [&](int j, int item, int buf) {
+    auto fetch_table = [&](int item, int buf) {
         const int band = 2 * (item / p.ttiles) + static_cast<int>(rank);
         const uint32_t nb = static_cast<uint32_t>(p.steps) * 8u;
-        mbar_arrive_expect_tx(&tab_full[2 * j + buf], nb);
-        bulk_g2s(tab_buf + (2 * j + buf) * kD8TabSteps, p.table + static_cast<int64_t>(band) * p.steps, nb,
-                 &tab_full[2 * j + buf]);
+        mbar_arrive_expect_tx(&tab_full[buf], nb);
+        bulk_g2s(tab_buf + buf * kD8TabSteps, p.table + static_cast<int64_t>(band) * p.steps, nb, &tab_full[buf]);
     };
     auto give_up = [&]() {
         *abort_flag = 1u;
@@ -147,9 +162,9 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 8);
+            mbar_init(&acc_empty[b], 16);  // 8 epilogue warps x 2 CTAs
+            mbar_init(&tab_full[b], 1);
         }
-        for (int b = 0; b < 2 * kD8Producers; ++b) mbar_init(&tab_full[b], 1);
         *never_flag = 0u;
         *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
         fence_mbar_init_cluster();
@@ -162,6 +177,9 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
         prefetch_tmap(&maps.x);
         prefetch_tmap(&maps.a_dense);
         prefetch_tmap(&maps.a_sparse);
+        prefetch_tmap(&maps.a_dd);
+        prefetch_tmap(&maps.a_mixed);
+        prefetch_tmap(&maps.a_ss);
     }
     __syncwarp();
     tc_fence_before();
@@ -169,11 +187,14 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const bool skip = *abort_flag != 0;
-    if (warp == 0 || warp == 7) {
-        const int j = warp == 0 ? 0 : 1;  // stages s with s % 2 == j
+    if (threadIdx.x == 0 && !skip) {
+        for (int i = 0; i < 2 && cl + i * C < p.items; ++i) fetch_table(cl + i * C, i);
+    }
+    const int pairs = p.steps / 2;
+
+    if (warp == 0) {
         if (lane == 0 && !skip) {
             // ----------------------------------------------- weight producer
-            for (int i = 0; i < 2 && cl + i * C < p.items; ++i) fetch_table(j, cl + i * C, i);
             int it = 0;
             bool ok = true;
             int tabs = 0;
@@ -182,71 +203,82 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
                 const int item = cl + i * C;
                 if (item >= p.items) break;
                 const int buf = i & 1;
-                if (!mbar_wait_bounded(&tab_full[2 * j + buf], (i >> 1) & 1u, abort_flag, kD8WaitLimitNs)) {
+                if (!mbar_wait_bounded(&tab_full[buf], (i >> 1) & 1u, abort_flag, kD8WaitLimitNs)) {
                     ok = false;
                     break;
                 }
-                const uint64_t *tab = tab_buf + (2 * j + buf) * kD8TabSteps;
-                for (int c = 0; c < p.steps; ++c, ++it) {
+                const uint64_t *tab = tab_buf + buf * kD8TabSteps;
+                for (int pr = 0; pr < pairs; ++pr) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
-                    if ((it & 1) != j) continue;
                     if (it >= S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kD8WaitLimitNs)) {
                         ok = false;
                         break;
                     }
-                    const uint64_t e = tab[c];
-                    const bool sp = (e & kEntrySparse) != 0;
-                    const uint64_t first = (e & kEntryOffsetMask) - (sp ? kMetaBlockBytes : 0);
-                    const uint32_t a_bytes = sp ? kMetaBlockBytes + kSparseStepBytes : kDenseStepBytes;
-                    stage_info[s] = e;
-                    // both bands of the pair take this kind: the leader arms
-                    // its barrier for both CTAs' weight bytes
-                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * a_bytes);
-                    tma2d_pair(smem + s * p.stage_bytes, sp ? &maps.a_sparse : &maps.a_dense, 0,
-                               static_cast<int32_t>(first / 2048), map_to_rank(&full[s], 0));
+                    ++it;
+                    const uint64_t e0 = tab[2 * pr], e1 = tab[2 * pr + 1];
+                    const bool sp0 = (e0 & kEntrySparse) != 0, sp1 = (e1 & kEntrySparse) != 0;
+                    const uint32_t b0 = sp0 ? kMetaBlockBytes + kSparseStepBytes : kDenseStepBytes;
+                    const uint32_t b1 = sp1 ? kMetaBlockBytes + kSparseStepBytes : kDenseStepBytes;
+                    const uint64_t f0 = (e0 & kEntryOffsetMask) - (sp0 ? kMetaBlockBytes : 0);
+                    const uint64_t f1 = (e1 & kEntryOffsetMask) - (sp1 ? kMetaBlockBytes : 0);
+                    // k-step 1 right behind k-step 0 in the slot; both bands of
+                    // the pair agree in kinds and, the packer pairing their
+                    // side copies too, in this placement
+                    stage_word[s] = (sp0 ? 1u : 0u) | (sp1 ? 2u : 0u) | ((b0 >> 4) << 2);
+                    // the leader arms its barrier for both CTAs' weight bytes
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (b0 + b1));
+                    uint8_t *st = smem + s * p.stage_bytes;
+                    if (f1 == f0 + b0) {
+                        // contiguous: one copy of both k-steps
+                        const CUtensorMap *am = (sp0 && sp1) ? &maps.a_ss : ((sp0 || sp1) ? &maps.a_mixed : &maps.a_dd);
+                        tma2d_pair(st, am, 0, static_cast<int32_t>(f0 / 2048), map_to_rank(&full[s], 0));
+                    } else {
+                        tma2d_pair(st, sp0 ? &maps.a_sparse : &maps.a_dense, 0, static_cast<int32_t>(f0 / 2048),
+                                   map_to_rank(&full[s], 0));
+                        tma2d_pair(st + b0, sp1 ? &maps.a_sparse : &maps.a_dense, 0, static_cast<int32_t>(f1 / 2048),
+                                   map_to_rank(&full[s], 0));
+                    }
                 }
                 if (ok && cl + (i + 2) * C < p.items) {
-                    fetch_table(j, cl + (i + 2) * C, buf);
+                    fetch_table(cl + (i + 2) * C, buf);
                     ++tabs;
                 }
             }
             for (int q = (tabs > 2 ? tabs - 2 : 0); q < tabs; ++q)
-                mbar_wait_bounded(&tab_full[2 * j + (q & 1)], (q >> 1) & 1u, never_flag, kD8WaitLimitNs / 4);
+                mbar_wait_bounded(&tab_full[q & 1], (q >> 1) & 1u, never_flag, kD8WaitLimitNs / 4);
             if (!ok) give_up();
-            // drain (this producer's stages): the leader waits for their last
-            // phase (its barrier counts both CTAs' loads); the peer until the
-            // leader's MMAs have released them, or gives up
+            // drain: the leader waits for the last phase of every stage (its
+            // barrier counts both CTAs' loads); the peer until the leader's
+            // MMAs have released each of its stages, or gives up
             for (int q = (it > S ? it - S : 0); q < it; ++q) {
-                if ((q & 1) != j) continue;
                 if (rank == 0)
                     mbar_wait_bounded(&full[q % S], (q / S) & 1u, never_flag, kD8WaitLimitNs / 4);
                 else
                     mbar_wait_bounded(&empty[q % S], (q / S) & 1u, never_flag, kD8WaitLimitNs / 4);
             }
         }
-    } else if (warp == 6 || warp == 8) {
-        const int j = warp == 6 ? 0 : 1;
+    } else if (warp == 6) {
         if (lane == 0 && !skip) {
             // ---------------------------------------------------- X producer
-            const uint32_t x_bytes = 2u * static_cast<uint32_t>(half) * kD8Step;  // both CTAs
+            const uint32_t x_bytes = 2u * 2u * static_cast<uint32_t>(half) * kD8Step;  // both CTAs, 2 k-steps
             int it = 0;
             bool ok = true;
             for (int i = 0; ok; ++i) {
                 const int item = cl + i * C;
                 if (item >= p.items) break;
                 const int tt = item % p.ttiles;
-                for (int c = 0; c < p.steps; ++c, ++it) {
+                for (int pr = 0; pr < pairs; ++pr) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
-                    if ((it & 1) != j) continue;
                     if (it >= S && !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, kD8WaitLimitNs)) {
                         ok = false;
                         break;
                     }
+                    ++it;
                     if (rank == 0) mbar_arrive_expect_tx(&full[s], x_bytes);
-                    tma2d_pair(smem + s * p.stage_bytes + p.aslot, &maps.x, c * kD8Step,
-                               tt * bn + static_cast<int>(rank) * half, map_to_rank(&full[s], 0));
+                    tma3d_pair(smem + s * p.stage_bytes + p.aslot, &maps.x, 0,
+                               tt * bn + static_cast<int>(rank) * half, 2 * pr, map_to_rank(&full[s], 0));
                 }
             }
             if (!ok) give_up();
@@ -254,13 +286,20 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
     } else if (warp == 1) {
         if (lane == 0 && !skip && rank == 0) {
             // ------------------------------------------------- MMA (leader)
-            const uint32_t e_tmem = tmem_base + static_cast<uint32_t>(2 * bn);
+            const uint32_t e_tmem = tmem_base + static_cast<uint32_t>(2 * bn);  // 4 columns per k-step
             const uint32_t id_dense = idesc_e4m3_pair(bn, false), id_sparse = idesc_e4m3_pair(bn, true);
             constexpr DescBase kDescDenseA = smem_desc_base(16, 1024, kSwizzle128B);
             constexpr DescBase kDescSparseA = smem_desc_base(16, 512, kSwizzle64B);
             constexpr DescBase kDescX = smem_desc_base(16, 1024, kSwizzle128B);
             constexpr DescBase kDescMeta = smem_desc_base(16, 128, kSwizzleNone);
-            int it = 0;
+            // the stage and its phase advance without division; addresses
+            // in 16-byte units
+            const uint32_t smem16 = smem_u32(smem) >> 4;
+            const uint32_t stage16 = static_cast<uint32_t>(p.stage_bytes) >> 4;
+            const uint32_t aslot16 = static_cast<uint32_t>(p.aslot) >> 4;
+            const uint32_t xk16 = static_cast<uint32_t>(half * kD8Step) >> 4;  // one k-step of X rows
+            int s = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int i = 0; ok; ++i) {
                 const int item = cl + i * C;
@@ -273,30 +312,38 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * bn);
-                for (int c = 0; c < p.steps; ++c, ++it) {
-                    const int s = it % S;
-                    const uint32_t ph = (it / S) & 1u;
+                for (int pr = 0; pr < pairs; ++pr) {
                     if (!mbar_wait_bounded(&full[s], ph, abort_flag, kD8WaitLimitNs)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t slot = smem_u32(smem + s * p.stage_bytes);
-                    const uint32_t s16 = slot >> 4, b16 = (slot + static_cast<uint32_t>(p.aslot)) >> 4;
-                    if (stage_info[s] & kEntrySparse) {
-                        tmem_cp_pair_128x128b(e_tmem, desc_at(kDescMeta, s16));
+                    const uint32_t w = stage_word[s];
+                    const uint32_t slot16 = smem16 + static_cast<uint32_t>(s) * stage16;
 #pragma unroll
-                        for (int q = 0; q < 2; ++q)
-                            mma_f8_sparse_pair(d_tmem, desc_at(kDescSparseA, s16 + kMetaBlockBytes / 16 + 2 * q),
-                                               desc_at(kDescX, b16 + 4 * q), e_tmem + 2 * q, id_sparse,
-                                               (c == 0 && q == 0) ? 0u : 1u);
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            mma_f8_pair(d_tmem, desc_at(kDescDenseA, s16 + 2 * q), desc_at(kDescX, b16 + 2 * q),
-                                        id_dense, (c == 0 && q == 0) ? 0u : 1u);
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t a16 = slot16 + (h ? ((w >> 2) & 0x7FFu) : 0u);
+                        const uint32_t b16 = slot16 + aslot16 + static_cast<uint32_t>(h) * xk16;
+                        const uint32_t acc = (pr == 0 && h == 0) ? 0u : 1u;
+                        if (w & (1u << h)) {
+                            const uint32_t e = e_tmem + 4u * static_cast<uint32_t>(h);
+                            tmem_cp_pair_128x128b(e, desc_at(kDescMeta, a16));
+                            const uint32_t v16 = a16 + kMetaBlockBytes / 16;
+                            mma_f8_sparse_pair_x2(d_tmem, desc_at(kDescSparseA, v16), desc_at(kDescSparseA, v16 + 2),
+                                                  desc_at(kDescX, b16), desc_at(kDescX, b16 + 4), e, e + 2, id_sparse,
+                                                  acc);
+                        } else {
+                            mma_f8_pair_x4(d_tmem, desc_at(kDescDenseA, a16), desc_at(kDescDenseA, a16 + 2),
+                                           desc_at(kDescDenseA, a16 + 4), desc_at(kDescDenseA, a16 + 6),
+                                           desc_at(kDescX, b16), desc_at(kDescX, b16 + 2), desc_at(kDescX, b16 + 4),
+                                           desc_at(kDescX, b16 + 6), id_dense, acc);
+                        }
                     }
                     tc_commit_pair(&empty[s]);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 // fires once every MMA of the item has completed (also after a
                 // failure, so no epilogue frees tensor memory under a running MMA)
@@ -304,9 +351,12 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
             }
             if (!ok) give_up();
         }
-    } else if (warp >= 2 && warp <= 5 && !skip) {
+    } else if (!skip) {
         // ---------------------------------------------- epilogue (both CTAs)
+        // two groups of four warps (one warp per TMEM lane quarter each)
+        // take alternate 16-column chunks of an accumulator
         const int quad = warp % 4;
+        const int grp = warp >= 7 ? 1 : 0;
         const int row = quad * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
         for (int i = 0;; ++i) {
@@ -326,16 +376,20 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
             const float swn = __ldg(p.sw + n);
             if (*abort_flag == 0) {
 #pragma unroll 1
-                for (int c0 = 0; c0 < m_valid; c0 += 16) {
+                for (int c0 = 16 * grp; c0 < m_valid; c0 += 32) {
                     uint32_t r[16];
                     tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(buf * bn + c0), r);
+                    // token scales of the chunk: lane l holds column l % 16's
+                    const int ml = c0 + (lane & 15);
+                    const float sxl = ml < m_valid ? __ldg(p.sx + m_base + ml) : 0.0f;
                     tmem_ld_wait();
+                    int64_t idx = (m_base + c0) * p.N + n;
 #pragma unroll
-                    for (int q = 0; q < 16; ++q)
-                        if (c0 + q < m_valid) {
-                            const int64_t m = m_base + c0 + q;
-                            store_y(p, m * p.N + n, __uint_as_float(r[q]) * swn * __ldg(p.sx + m));
-                        }
+                    for (int q = 0; q < 16; ++q) {
+                        const float sq = __shfl_sync(0xFFFFFFFFu, sxl, q);
+                        if (c0 + q < m_valid) store_y(p, idx, __uint_as_float(r[q]) * swn * sq);
+                        idx += p.N;
+                    }
                 }
             }
             tc_fence_before();
@@ -418,11 +472,13 @@ int max_clusters(int smem) {
 DuoFp8Plan plan_duo_fp8(int64_t N, int64_t M, int num_sms, bool all_sparse) {
     DuoFp8Plan best{};
     const int64_t bpairs = (N / kBand) / 2;
-    // shared memory per stage: the weight slot (a dense k-step, or metadata +
-    // codes when no k-step of the matrix is dense) + BN/2 X rows of 128 B
-    const int aslot = all_sparse ? kMetaBlockBytes + kSparseStepBytes : kDenseStepBytes;
+    // shared memory per stage (two k-steps): the weight slot (two dense
+    // k-steps, or metadata + codes twice when no k-step of the matrix is
+    // dense) + BN/2 X rows of 128 B per k-step
+    const int aslot_step = all_sparse ? kMetaBlockBytes + kSparseStepBytes : kDenseStepBytes;
+    const int aslot = 2 * aslot_step;
     auto smem_for = [aslot](int bn, int *stages, int *stage_bytes) {
-        *stage_bytes = aslot + (bn / 2) * kD8Step;
+        *stage_bytes = aslot + 2 * (bn / 2) * kD8Step;
         *stages = std::min(kD8MaxStages, (kD8SmemLimit - kD8TailBytes) / *stage_bytes);
         return *stages * *stage_bytes + kD8TailBytes;
     };
@@ -450,6 +506,7 @@ DuoFp8Plan plan_duo_fp8(int64_t N, int64_t M, int num_sms, bool all_sparse) {
     }
     best.smem = smem_for(best.bn, &best.stages, &best.stage_bytes);
     best.aslot = aslot;
+    best.aslot_step = aslot_step;
     return best;
 }
 
@@ -464,19 +521,25 @@ cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStrea
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorInvalidValue;
     D8Maps maps;
-    // X codes [M, K] uint8 row-major: box = 128 bytes x this CTA's half of the
-    // token tile, 128-byte swizzle, rows past M read as zero
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(g.K), static_cast<cuuint64_t>(g.M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(g.K)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kD8Step), static_cast<cuuint32_t>(plan.bn / 2)};
-    const cuuint32_t estr[2] = {1, 1};
-    if (enc(&maps.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(g.xq), dims, strides, box, estr,
+    // X codes [M, K] uint8 row-major, viewed as (128 bytes, M rows, K/128
+    // k-steps): box = this CTA's half of the token tile for both k-steps of a
+    // stage, 128-byte swizzle, rows past M read as zero
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD8Step), static_cast<cuuint64_t>(g.M),
+                                static_cast<cuuint64_t>(g.K / kD8Step)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.K), static_cast<cuuint64_t>(kD8Step)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kD8Step), static_cast<cuuint32_t>(plan.bn / 2), 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&maps.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(g.xq), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     const uint64_t rows = g.packed_bytes / 2048;  // packed + side copies, in 2 KB rows
-    if (!encode_rows(enc, &maps.a_dense, g.packed, rows, kDenseStepBytes / 2048) ||
-        !encode_rows(enc, &maps.a_sparse, g.packed, rows, (kMetaBlockBytes + kSparseStepBytes) / 2048))
+    constexpr uint32_t kRowsD = kDenseStepBytes / 2048, kRowsS = (kMetaBlockBytes + kSparseStepBytes) / 2048;
+    if (!encode_rows(enc, &maps.a_dense, g.packed, rows, kRowsD) ||
+        !encode_rows(enc, &maps.a_sparse, g.packed, rows, kRowsS) ||
+        !encode_rows(enc, &maps.a_dd, g.packed, rows, 2 * kRowsD) ||
+        !encode_rows(enc, &maps.a_mixed, g.packed, rows, kRowsD + kRowsS) ||
+        !encode_rows(enc, &maps.a_ss, g.packed, rows, 2 * kRowsS))
         return cudaErrorInvalidValue;
     D8Params p;
     p.table = g.ptable;
@@ -493,6 +556,7 @@ cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStrea
     p.stages = plan.stages;
     p.stage_bytes = plan.stage_bytes;
     p.aslot = plan.aslot;
+    p.aslot_step = plan.aslot_step;
     p.Y = g.Y;
     p.y_fp32 = g.y_fp32;
     p.status = g.status;
