@@ -364,8 +364,10 @@ patch_status patch_packed_fp8_scales(const patch_packed *Wp, float *scales_dst, 
  * memory and one rounding at the end (PATCH page, section 2, inference and
  * deployment: one kernel over mixed dense / 2:4 tiles).  Dense k-steps issue
  * the dense tcgen05 MMA, 2:4 k-steps the sparse tcgen05 MMA, into one
- * accumulator.  M <= 16 runs the split-K decode configuration; larger M the
- * prefill configuration.  The call only enqueues work: it never waits for the
+ * accumulator.  M <= 16, and M <= 64 where K <= 8192, run the split-K
+ * configuration (the weights read once, spread over every SM, with 16-, 32-
+ * or 64-token tiles and an in-order fix-up of the chunk partials); larger M
+ * the prefill configuration.  The call only enqueues work: it never waits for the
  * device (everything it needs from the device was read back by patch_pack).
  *
  *   Wp      handle from patch_pack.
@@ -395,7 +397,8 @@ void patch_test_stall_first_kstep(int32_t on);
 
 /*
  * Test hook: the prefill kernel every later patch_hybrid_gemm with M > 16
- * uses.  0 = chosen by the library (the default), 1 = one band per CTA,
+ * uses.  0 = chosen by the library (the default), 1 = one band per CTA
+ * (64-token tiles up to M = 64),
  * 2 = two bands per CTA sharing each token tile, 3 = two-SM (CTA pair)
  * kernel, 4 = two-SM kernel with two bands per SM; 3 and 4 only where the
  * band count is even (else as 0).  FP8 handles: 1 = one band per CTA, 3 =

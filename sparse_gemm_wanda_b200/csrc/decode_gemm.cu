@@ -60,17 +60,30 @@ namespace patchk {
 namespace {
 
 constexpr int kDecThreads = 224;
-constexpr int kDecBN = 16;                                // token rows of the MMA (N = 16)
-constexpr int kDecStages = 3;
 constexpr int kDecChunkPairs = 4;                         // k-pairs per chunk, at most
 constexpr int kDecWBytes = 4 * kDenseStepBytes;           // two packed k-pairs, at most
-constexpr int kDecXStepBytes = kDecBN * kStep * 2;        // one k-step of X: 16 rows x 64
-constexpr int kDecXBytes = 4 * kDecXStepBytes;            // the stage's four X tiles
-constexpr int kDecStageBytes = kDecWBytes + kDecXBytes;   // 73728
-constexpr int kDecTmemCols = 128;  // 2 chunks x 2 issuers x 16 accumulator | 2 issuers x 2 x 4 metadata
-constexpr uint32_t kDecEcol = 4 * kDecBN;
-constexpr int kDecSmemBytes = kDecStages * kDecStageBytes + 1024 + 512;
 constexpr uint64_t kDecWaitLimitNs = 2000000000ull;       // 2 s per wait
+
+// Per token-tile width BN (the MMA's N: 16, 32 or 64 token rows).  A stage is
+// the packed bytes of two k-pairs plus their four X tiles; three stages fit
+// at BN = 16 (72 KB each), two at 32 and 64 (80 / 96 KB).  Tensor memory:
+// 2 chunks x 2 issuers x BN accumulator columns, then 2 issuers x 2 k-pairs
+// x 4 metadata columns.
+template <int BN>
+struct DecCfg {
+    static_assert(BN == 16 || BN == 32 || BN == 64, "decode token tile");
+    static constexpr int kXStepBytes = BN * kStep * 2;     // one k-step of X: BN rows x 64
+    static constexpr int kXBytes = 4 * kXStepBytes;        // the stage's four X tiles
+    static constexpr int kStageBytes = kDecWBytes + kXBytes;
+    static constexpr int kStages = BN == 16 ? 3 : 2;
+    static constexpr uint32_t kEcol = 4 * BN;
+    static constexpr int kCols = 4 * BN + 16;
+    static constexpr int kTmemCols = kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 512;
+    static_assert(kStageBytes % 1024 == 0, "stage regions stay 1024-B aligned");
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+    static_assert(kStages <= 4, "stage words and drained counters share the control block");
+};
 
 // chunk descriptor: first byte (40 bits) | 2:4 flag of each k-step (16) | pairs (4)
 constexpr uint64_t kDescOffsetMask = (1ull << 40) - 1;
@@ -145,8 +158,14 @@ __device__ __forceinline__ void store_out(const DecodeParams &p, int64_t idx, fl
         static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
 }
 
+template <int BN>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ DecodeParams p) {
+    using C = DecCfg<BN>;
+    constexpr int kDecStages = C::kStages;
+    constexpr int kDecStageBytes = C::kStageBytes;
+    constexpr int kDecXBytes = C::kXBytes;
+    constexpr int kDecXStepBytes = C::kXStepBytes;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -181,7 +200,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, kDecTmemCols);
+        tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) prefetch_tmap(&tmap_x);
@@ -313,13 +332,13 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             // Descriptors: a template per layout plus the operand's shared
             // address in 16-byte units (all addresses here are below 256 KB,
             // so the 14-bit address field never carries into other fields).
-            constexpr uint32_t kIdDense = idesc_bf16(kDecBN, false);
-            constexpr uint32_t kIdSp0 = idesc_bf16(kDecBN, true, 0);
-            constexpr uint32_t kIdSp1 = idesc_bf16(kDecBN, true, 1);
+            constexpr uint32_t kIdDense = idesc_bf16(BN, false);
+            constexpr uint32_t kIdSp0 = idesc_bf16(BN, true, 0);
+            constexpr uint32_t kIdSp1 = idesc_bf16(BN, true, 1);
             const uint64_t t_sw128 = smem_desc(0, 16, 1024, kSwizzle128B);  // dense A, X
             const uint64_t t_sw64 = smem_desc(0, 16, 512, kSwizzle64B);     // 2:4 A
             const uint64_t t_meta = smem_desc(0, 16, 128, kSwizzleNone);    // metadata
-            const uint32_t e_tmem = tmem_base + kDecEcol + 8 * q;
+            const uint32_t e_tmem = tmem_base + C::kEcol + 8 * q;
             const uint32_t smem0 = smem_u32(smem);
             int it = q;       // ring position
             int nch = 0;      // chunks of this CTA (from the done word)
@@ -364,7 +383,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (2 * buf + q) * kDecBN;
+                const uint32_t d_tmem = tmem_base + (2 * buf + q) * BN;
                 const uint32_t st16 = (smem0 + s * kDecStageBytes) >> 4;  // stage, 16-byte units
                 const uint64_t x16 = t_sw128 + st16 + (kDecWBytes >> 4);
                 const int sp = static_cast<int>((w >> kStagePairsShift) & 3u);
@@ -445,17 +464,21 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             const int j = acc_chunk[buf];
             if (j < 0) break;
             const uint32_t mask = acc_mask[buf];  // the same for every lane
-            uint32_t r0[16], r1[16];
-            if (mask & 1u) tmem_ld_32x32b_x16(lane_base + (2 * buf) * kDecBN, r0);
-            if (mask & 2u) tmem_ld_32x32b_x16(lane_base + (2 * buf + 1) * kDecBN, r1);
-            tmem_ld_wait();
-            if (*abort_flag == 0) {
-                float *part = p.partial + static_cast<int64_t>(j) * kDecBN * kBand + row;
+            // 16 token columns at a time (columns past M are never stored)
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN && c0 < p.M; c0 += 16) {
+                uint32_t r0[16], r1[16];
+                if (mask & 1u) tmem_ld_32x32b_x16(lane_base + (2 * buf) * BN + c0, r0);
+                if (mask & 2u) tmem_ld_32x32b_x16(lane_base + (2 * buf + 1) * BN + c0, r1);
+                tmem_ld_wait();
+                if (*abort_flag == 0) {
+                    float *part = p.partial + (static_cast<int64_t>(j) * BN + c0) * kBand + row;
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const float v = (mask == 3u) ? __fadd_rn(__uint_as_float(r0[q]), __uint_as_float(r1[q]))
-                                                 : __uint_as_float(mask & 1u ? r0[q] : r1[q]);
-                    if (q < p.M) part[q * kBand] = v;
+                    for (int q = 0; q < 16; ++q) {
+                        const float v = (mask == 3u) ? __fadd_rn(__uint_as_float(r0[q]), __uint_as_float(r1[q]))
+                                                     : __uint_as_float(mask & 1u ? r0[q] : r1[q]);
+                        if (c0 + q < p.M) part[q * kBand] = v;
+                    }
                 }
             }
             // the accumulator may be reused as soon as every lane has read it
@@ -470,25 +493,26 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, kDecTmemCols);
+    if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
 // Fix-up: Y[m, band*128 + row] = the band's chunk partials added in chunk
 // order.  Block (band, m), one thread per row.  Launched as a programmatic
 // dependent of the GEMM; resets the chunk counter once the GEMM is complete.
+template <int BN>
 __global__ void __launch_bounds__(kBand)
 decode_reduce_kernel(const __grid_constant__ DecodeParams p) {
     if (threadIdx.x == 0) pdl_trigger();  // the next GEMM may start its prologue
     pdl_wait();
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.counter = 0u;
     const int band = blockIdx.x, m = blockIdx.y, row = threadIdx.x;
-    const float *src = p.partial + (static_cast<int64_t>(band) * p.cpb * kDecBN + m) * kBand + row;
+    const float *src = p.partial + (static_cast<int64_t>(band) * p.cpb * BN + m) * kBand + row;
     float acc = 0.0f;
     for (int c0 = 0; c0 < p.cpb; c0 += 8) {
         float v[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-            v[q] = (c0 + q < p.cpb) ? __ldcg(src + static_cast<int64_t>(c0 + q) * kDecBN * kBand) : 0.0f;
+            v[q] = (c0 + q < p.cpb) ? __ldcg(src + static_cast<int64_t>(c0 + q) * BN * kBand) : 0.0f;
 #pragma unroll
         for (int q = 0; q < 8; ++q)
             if (c0 + q < p.cpb) acc = __fadd_rn(acc, v[q]);
@@ -540,40 +564,53 @@ uint64_t decode_chunk_desc(const uint64_t *band_table, int64_t nsteps, int pr0, 
            (static_cast<uint64_t>(np) << kDescPairsShift);
 }
 
-size_t decode_workspace_bytes(int nchunks) {
-    return sizeof(float) * static_cast<size_t>(nchunks) * kDecBN * kBand;
+size_t decode_workspace_bytes(int nchunks, int bn) {
+    return sizeof(float) * static_cast<size_t>(nchunks) * bn * kBand;
 }
 
-cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
+namespace {
+
+template <int BN>
+cudaError_t launch_decode(const GemmLaunch &g, cudaStream_t stream) {
+    using C = DecCfg<BN>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(decode_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kDecSmemBytes);
+        attr_err = cudaFuncSetAttribute(decode_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        C::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorInvalidValue;
     // X [M,K] viewed as (64 columns, M rows, K/64 k-steps); box = the four
-    // k-steps of a stage, 16 rows, 128-byte swizzle, rows past M and k-steps
+    // k-steps of a stage, BN rows, 128-byte swizzle, rows past M and k-steps
     // past K read as zero
     CUtensorMap map;
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kStep), static_cast<cuuint64_t>(g.M),
                                 static_cast<cuuint64_t>(g.K / kStep)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.K) * 2, static_cast<cuuint64_t>(kStep) * 2};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kStep), static_cast<cuuint32_t>(kDecBN), 4};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kStep), static_cast<cuuint32_t>(BN), 4};
     const cuuint32_t estr[3] = {1, 1, 1};
     if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(g.X), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    if (!g.chunk_desc || !g.chunk_desc_host || !g.workspace || !g.counter) return cudaErrorInvalidValue;
+    if (!g.chunk_desc || !g.chunk_desc_host || !g.counter) return cudaErrorInvalidValue;
     if (g.dec_cp < 1 || g.dec_cp > kDecChunkPairs) return cudaErrorInvalidValue;
     const int grid_ctas = std::min(std::min(g.num_sms, g.dec_nchunks), kDecMaxCtas);
     // a CTA's chunk ordinals travel in 16 bits (dynamic claiming could in
     // principle hand one CTA every chunk)
     if (g.dec_nchunks > kDecMaxChunksPerCta) return cudaErrorInvalidValue;
-    if (decode_workspace_bytes(g.dec_nchunks) > g.workspace_bytes) return cudaErrorInvalidValue;
+    // partials: the handle's slots hold 16 token rows per chunk; wider tiles
+    // take theirs from the stream-ordered pool for the call
+    const size_t ws_bytes = decode_workspace_bytes(g.dec_nchunks, BN);
+    float *ws = nullptr;
+    if (g.workspace && ws_bytes <= g.workspace_bytes) {
+        ws = g.workspace;
+    } else {
+        const cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), ws_bytes, g.pool, stream);
+        if (e != cudaSuccess) return e;
+    }
 
     DecodeParams p;
     p.packed = g.packed;
@@ -586,7 +623,7 @@ cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
     p.nchunks = g.dec_nchunks;
     p.Y = g.Y;
     p.y_fp32 = g.y_fp32;
-    p.partial = g.workspace;
+    p.partial = ws;
     p.counter = g.counter;
     p.status = g.status;
     p.ready = g.ready;
@@ -600,22 +637,36 @@ cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kDecThreads);
-    cfg.dynamicSmemBytes = kDecSmemBytes;
+    cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gemm_kernel, map, p);
-    if (err != cudaSuccess) return err;
-    note_launches(1);
-    cfg.gridDim = dim3(static_cast<unsigned>(g.N / kBand), static_cast<unsigned>(g.M));
-    cfg.blockDim = dim3(kBand);
-    cfg.dynamicSmemBytes = 0;
-    err = cudaLaunchKernelEx(&cfg, decode_reduce_kernel, p);
-    if (err == cudaSuccess) note_launches(1);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gemm_kernel<BN>, map, p);
+    if (err == cudaSuccess) {
+        note_launches(1);
+        cfg.gridDim = dim3(static_cast<unsigned>(g.N / kBand), static_cast<unsigned>(g.M));
+        cfg.blockDim = dim3(kBand);
+        cfg.dynamicSmemBytes = 0;
+        err = cudaLaunchKernelEx(&cfg, decode_reduce_kernel<BN>, p);
+        if (err == cudaSuccess) note_launches(1);
+    }
+    if (ws != g.workspace) {
+        const cudaError_t e2 = cudaFreeAsync(ws, stream);
+        if (err == cudaSuccess) err = e2;
+    }
     return err;
+}
+
+}  // namespace
+
+cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
+    if (g.M <= 16) return launch_decode<16>(g, stream);
+    if (g.M <= 32) return launch_decode<32>(g, stream);
+    if (g.M <= kDecodeMaxM) return launch_decode<64>(g, stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace patchk

@@ -794,7 +794,7 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     }
     if (g.M <= 16) return launch_decode_gemm(g, stream);  // split-K GEMV, csrc/decode_gemm.cu
     // test hook: one prefill kernel for every M > 16 (parity of each kernel)
-    if (g.force_kernel == 1) return run<160, 3>(g, 1, stream);
+    if (g.force_kernel == 1) return g.M <= 64 ? run<64, 4>(g, 1, stream) : run<160, 3>(g, 1, stream);
     if (g.force_kernel == 2 && g.K / kStep <= 448) return launch_pair_gemm(g, plan_pair_gemm(g.N, g.M, g.num_sms), stream);
     if (g.force_kernel == 3 && g.duo_ok && g.K / kStep <= 448) {
         const DuoPlan dp = plan_duo_gemm(g.N, g.M, g.num_sms, g.max_pair_bytes);
@@ -804,6 +804,15 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
         const QuadPlan qp = plan_quad_gemm(g.N, g.M, g.num_sms);
         if (qp.bn > 0) return launch_quad_gemm(g, qp, stream);
     }
+    // up to 64 tokens: the split-K kernel of csrc/decode_gemm.cu (32- or
+    // 64-token tiles, four k-pairs per chunk, every chunk's partial added in
+    // order by the fix-up) while a band has at most 16 chunks; for longer K
+    // this file's stream-K kernel, with two partials per CTA, is faster.
+    // Measured on B200, back-to-back calls on the Llama-7B block shapes at
+    // f = 0.6: 4096x4096 M = 32 / 64: 11.6 / 12.5 us against 14.4 / 14.5;
+    // 11008x4096: 20.7 / 24.9 against 24.1 / 25.2; 4096x11008: 21.7 / 23.2
+    // against 20.6 / 21.2.
+    if (g.M <= kDecodeMaxM && g.K <= 8192) return launch_decode_gemm(g, stream);
     if (g.M <= 64) return run<64, 4>(g, 1, stream);   // 48 KB stages
     if (g.M <= 128) return run<128, 3>(g, 1, stream); // 64 KB stages
     // larger token counts: the band-pair kernel (two bands share each X tile)

@@ -152,7 +152,9 @@ QuadPlan plan_quad_gemm(int64_t N, int64_t M, int num_sms);
 cudaError_t launch_quad_gemm(const GemmLaunch &g, const QuadPlan &plan, cudaStream_t stream);
 double quad_kstep_cycles(int bn);
 
-// Decode GEMV for M <= 16 (csrc/decode_gemm.cu).
+// Split-K GEMV / skinny GEMM for M <= kDecodeMaxM (csrc/decode_gemm.cu):
+// token tiles of 16, 32 or 64 rows.
+constexpr int64_t kDecodeMaxM = 64;
 cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream);
 // Chunking of a packed matrix for the decode GEMV: `cp` k-pairs per chunk,
 // `cpb` chunks per band.
@@ -160,8 +162,8 @@ void plan_decode_chunks(int64_t bands, int64_t nsteps, int num_sms, int *cp, int
 // Descriptor of the chunk holding pairs [pr0, pr0 + np) of a band whose
 // k-step table starts at `band_table`: first byte | 2:4 flags << 40 | np << 56.
 uint64_t decode_chunk_desc(const uint64_t *band_table, int64_t nsteps, int pr0, int np);
-// fp32 partial bytes of the decode GEMV (one 16 x 128 slot per chunk).
-size_t decode_workspace_bytes(int nchunks);
+// fp32 partial bytes of the decode GEMV (one bn x 128 slot per chunk).
+size_t decode_workspace_bytes(int nchunks, int bn = 16);
 
 // FP8 handles (csrc/fp8_kernels.cu, csrc/fp8_gemm.cu).
 // Per-row e4m3 quantisation of a bf16 matrix [R, C]: scale[r] = amax / 448

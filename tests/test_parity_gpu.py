@@ -302,6 +302,78 @@ def test_gemm_decode_ragged_pair_counts(P, oracle_mod, N, K, M):
     run_case(P, oracle_mod, N, K, M, 128, 128, 0.5, seed=N + K + M, fp32_mode=True)
 
 
+@pytest.mark.parametrize("N,K", [(128, 128), (128, 384), (256, 640), (384, 896), (128, 1152)])
+@pytest.mark.parametrize("M", [17, 32, 33, 47, 64])
+def test_gemm_skinny_ragged_pair_counts(P, oracle_mod, N, K, M):
+    # the split-K path with 32- and 64-token tiles (17 <= M <= 64): ragged
+    # token tiles, chunks of fewer than four pairs, single-pair stages
+    run_case(P, oracle_mod, N, K, M, 128, 128, 0.5, seed=N + K + M, fp32_mode=True)
+
+
+@pytest.mark.parametrize("tn,tk", [(64, 64), (128, 64)])
+@pytest.mark.parametrize("frac", [0.0, 1.0])
+@pytest.mark.parametrize("M", [24, 64])
+def test_gemm_skinny_tiles_and_fractions(P, oracle_mod, tn, tk, frac, M):
+    run_case(P, oracle_mod, 256, 512, M, tn, tk, frac, seed=tn + tk + M + 7, fp32_mode=False)
+
+
+@pytest.mark.parametrize("N,K", [(4096, 4096), (11008, 4096), (4096, 11008)])
+@pytest.mark.parametrize("M", [32, 64])
+def test_gemm_skinny_config_full(P, oracle_mod, N, K, M):
+    # Llama-7B block shapes at M = 32 / 64, map by least Wanda tile loss at
+    # f = 0.6, every output compared
+    seed = inputs.BASE_SEED + 2
+    w = inputs.weight(N, K, seed + N)
+    o = inputs.outlier_channels(K, seed)
+    xc = inputs.activations(1024, K, seed, o, role=0)
+    x = inputs.activations(M, K, seed, o, role=1 + M)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), fraction=0.6)
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    y16 = P.patch_hybrid_gemm(pk, x.cuda())
+    y32 = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    y32b = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    assert P.patch_get_status(pk) == 0
+    # chunk partials are added in a fixed order: repeated calls agree bit for bit
+    assert torch.equal(y32, y32b)
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, frac=0.6)
+    yref = oracle_mod.gemm(bf16_bits(x), weff)
+    rel_rms_check(y32, yref, True)
+    rel_rms_check(y16, yref, False)
+    pk.close()
+
+
+@pytest.mark.parametrize("M", [40, 64])
+def test_gemm_skinny_one_band_kernel_forced(P, oracle_mod, M):
+    # the one-band stream-K kernel with 64-token tiles (test hook) at the
+    # token counts the split-K path now serves
+    with forced_kernel(P, 1):
+        run_case(P, oracle_mod, 1024, 2048, M, 128, 128, 0.5, seed=M + 9, fp32_mode=True)
+
+
+@pytest.mark.parametrize("M", [20, 64])
+def test_gemm_skinny_bounded_wait_reports_timeout(P, oracle_mod, M):
+    # the failure-detection hook on the 32- / 64-token split-K kernel
+    N, K = 256, 512
+    w, xc, x = make_problem(N, K, 64, M, seed=43 + M)
+    nt = (N // 128) * (K // 128)
+    tmap = inputs.random_map(nt, nt // 2, seed=43)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    P.test_stall_first_kstep(True)
+    try:
+        P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    finally:
+        P.test_stall_first_kstep(False)
+    assert P.patch_get_status(pk) == 5  # PATCH_ERR_TIMEOUT, read and cleared
+    assert P.patch_get_status(pk) == 0
+    y = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap)
+    rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), weff), True)
+    pk.close()
+
+
 def test_gemm_tiny_config(P, oracle_mod):
     # W 256x256, 64x64 tiles, 8 of 16 tiles 2:4, Xcal 64x256, X 8x256, 3 outlier channels
     wl = inputs.workloads()["tiny"]
