@@ -158,8 +158,9 @@ def cpu_cores():
 def make_tensors(wl, rank: int, device="cpu", rows=None, calib_tokens=None):
     """Synthetic weights, calibration sets and inputs of a workload (per-rank seed).
 
-    Calibration sets are keyed by input group: layers that read the same
-    activations (q/k/v; gate/up) share one set and hence one column norm.
+    Calibration sets and the GEMM inputs X are keyed by input group: layers
+    that read the same activations (q/k/v; gate/up) share one calibration set
+    (hence one column norm) and one X per token count.
     `rows` / `calib_tokens` cut a bounded sample (the first rows of every
     matrix, the first tokens of every calibration set: the same values as the
     full draw's)."""
@@ -167,6 +168,7 @@ def make_tensors(wl, rank: int, device="cpu", rows=None, calib_tokens=None):
     mats = []
     outl = {}
     calib = {}
+    group_x = {}
     for mi, m in enumerate(wl.matrices):
         if m.K not in outl:
             outl[m.K] = inputs.outlier_channels(m.K, seed, wl.outlier_count)
@@ -180,10 +182,12 @@ def make_tensors(wl, rank: int, device="cpu", rows=None, calib_tokens=None):
         w = inputs.weight(m.N, m.K, seed + 17 * (mi + 1))
         if rows is not None:
             w = w[:rows].contiguous()
-        xs = {M: inputs.activations(M, m.K, seed, outl[m.K], role=1 + mi * 100 + M)
-              for M in wl.tokens}
+        if g not in group_x:
+            gi = len(group_x)
+            group_x[g] = {M: inputs.activations(M, m.K, seed, outl[m.K], role=1 + gi * 100 + M).to(device)
+                          for M in wl.tokens}
         mats.append({"name": m.name, "N": w.shape[0], "K": m.K, "group": g, "W": w.to(device),
-                     "X": {M: x.to(device) for M, x in xs.items()}})
+                     "X": group_x[g]})
     return mats, calib
 
 
@@ -270,10 +274,24 @@ def run_step(P, wl, mats, calib, maps, ys, ev: StepEvents | None = None, colsq_c
     mark("pack")
     pks = [P.patch_pack(mats[mi]["W"], r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k)
            for (mi, _), r in zip(units, masks)]
+    # matrices that read the same X (one unit per matrix) share one call
+    batches = []
+    for (mi, f), pk in zip(units, pks):
+        g = mats[mi]["group"] if wl.map_rule != "random" else (mi, f)
+        if batches and batches[-1][0] == g:
+            batches[-1][1].append((mi, f, pk))
+        else:
+            batches.append((g, [(mi, f, pk)]))
     for M in sorted(wl.tokens, reverse=True):
         mark(f"gemm_m{M}")
-        for (mi, f), pk in zip(units, pks):
-            P.patch_hybrid_gemm(pk, mats[mi]["X"][M], out=ys[(mi, f, M)])
+        for _, members in batches:
+            x = mats[members[0][0]]["X"][M]
+            if len(members) == 1:
+                mi, f, pk = members[0]
+                P.patch_hybrid_gemm(pk, x, out=ys[(mi, f, M)])
+            else:
+                P.patch_hybrid_gemm_group([pk for _, _, pk in members], x,
+                                          outs=[ys[(mi, f, M)] for mi, f, _ in members])
     mark("end")
     return pks
 
@@ -754,11 +772,14 @@ def main():
     # ------------------------------------------------------- end to end
     e2e = None
     if not args.no_extras or world > 1:
+        gx = {}
+        for m in mats:  # one X per input group and token count
+            gx.setdefault(m["group"], m["X"])
         host = {"W": [m["W"].cpu().pin_memory() for m in mats],
-                "X": [{M: x.cpu().pin_memory() for M, x in m["X"].items()} for m in mats],
+                "X": {g: {M: x.cpu().pin_memory() for M, x in xs.items()} for g, xs in gx.items()},
                 "C": {g: c.cpu().pin_memory() for g, c in calib.items()}}
         h2d = sum(t.numel() * 2 for t in host["W"]) + sum(c.numel() * 2 for c in host["C"].values()) \
-            + sum(x.numel() * 2 for d in host["X"] for x in d.values())
+            + sum(x.numel() * 2 for d in host["X"].values() for x in d.values())
         hy = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in ys.items()}
         d2h = sum(v.numel() * 2 for v in ys.values())
         e2e_ms = []
@@ -768,9 +789,10 @@ def main():
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(s)
+            dx = {g: {M: x.to("cuda", non_blocking=True) for M, x in xs.items()}
+                  for g, xs in host["X"].items()}
             dm = [{"name": m["name"], "N": m["N"], "K": m["K"], "group": m["group"],
-                   "W": host["W"][mi].to("cuda", non_blocking=True),
-                   "X": {M: x.to("cuda", non_blocking=True) for M, x in host["X"][mi].items()}}
+                   "W": host["W"][mi].to("cuda", non_blocking=True), "X": dx[m["group"]]}
                   for mi, m in enumerate(mats)]
             dc = {g: c.to("cuda", non_blocking=True) for g, c in host["C"].items()}
             close_all(run_step(P, wl, dm, dc, maps, ys))
@@ -778,7 +800,7 @@ def main():
                 hy[k].copy_(v, non_blocking=True)
             e1.record(s)
             e1.synchronize()
-            del dm, dc
+            del dm, dc, dx
             if it >= args.warmup:
                 e2e_ms.append(e0.elapsed_time(e1))
         e_ms = max_over_ranks(statistics.fmean(e2e_ms), "cuda")

@@ -387,6 +387,42 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
                                int32_t y_is_fp32, void *stream);
 
 /*
+ * Several hybrid products that read the same activations, in one launch:
+ * Ys[i][M, N_i] = X[M, K] * W_eff_i^T for i < count, each exactly as
+ * patch_hybrid_gemm computes it (bit for bit: the same chunks, added in the
+ * same order).  The layers of a decoder block that share an input (q, k and
+ * v; gate and up) are each one hybrid linear layer of the PATCH page
+ * (section 2, inference and deployment); the pages say nothing about
+ * launching them together.  This entry point exists because at decode token
+ * counts a product is bound by reading its weights once, and the fixed cost
+ * of a launch (its start, the first copies' latency, the tail and the fix-up)
+ * weighs most on the smaller matrices: one launch over the group pays it
+ * once and spreads all the group's chunks over every SM.
+ *
+ *   Wps     count (1..8) handles from patch_pack on the current device, all
+ *           with the same K.
+ *   X_bf16  [M,K] bf16, 16-byte aligned, the input of every product.
+ *   M       tokens, >= 0 (M == 0 returns PATCH_OK without touching anything).
+ *   Ys      count outputs, Ys[i] [M, N_i] bf16 or fp32 (y_is_fp32), 16-byte
+ *           aligned, not overlapping one another or X.
+ *
+ * One launch is made when every handle is bf16 2:4 (not FP8, not 4:8) and M
+ * is in the split-K range (M <= 16, or M <= 64 with K <= 8192); otherwise the
+ * products are enqueued one after another, as count calls of
+ * patch_hybrid_gemm would.  Partial slots come from the library's
+ * stream-ordered pool for the call; the first handle's claim counter serves
+ * the launch, so calls that use a handle must not run concurrently on
+ * different streams (the rule of patch_hybrid_gemm).  A wait that runs out
+ * raises every handle's status word; a raised word on any handle makes the
+ * whole launch skip its work.  The call never waits for the device.
+ * Handles that cannot share a launch (another pattern or K) are not an
+ * error: their products are enqueued one by one.  Errors: INVALID_ARG (null
+ * pointers, count out of range, misalignment, y_is_fp32 not 0 / 1), CUDA.
+ */
+patch_status patch_hybrid_gemm_group(const patch_packed *const *Wps, int32_t count, const void *X_bf16,
+                                     int64_t M, void *const *Ys, int32_t y_is_fp32, void *stream);
+
+/*
  * Failure-detection test hook: while `on` is non-zero, the first CTA of every
  * later patch_hybrid_gemm never loads its first k-step, so that CTA's bounded
  * wait runs out on purpose and patch_get_status reports PATCH_ERR_TIMEOUT.

@@ -103,23 +103,43 @@ constexpr int kStageOrdShift = 40;
 constexpr int kStagePosShift = 56;
 constexpr int kDecMaxChunksPerCta = 65535;
 
+// One launch covers one matrix, or several that read the same X (the same K,
+// hence the same chunking): their bands are numbered one after another
+// (matrix i holds global bands band0[i] .. band0[i+1]-1), chunk j belongs to
+// global band j / cpb, and each matrix keeps its own packed bytes, chunk
+// descriptors, output, status and ready words.
 struct DecodeParams {
-    const uint8_t *packed;
-    const uint64_t *chunk_desc;  // [nchunks]
-    int64_t N, K, M;
-    int cpb;      // chunks per band
+    int64_t K, M;
+    int cpb;      // chunks per band (the same for every matrix of the launch)
     int cp;       // k-pairs per chunk (the last chunk of a band may hold fewer)
-    int nchunks;
-    void *Y;
+    int nchunks;  // all matrices
+    int nmat;     // 1 .. kDecMaxGroup
+    int32_t band0[kDecMaxGroup + 1];
+    const uint8_t *packed[kDecMaxGroup];
+    const uint64_t *chunk_desc[kDecMaxGroup];  // [bands * cpb] of each matrix
+    void *Y[kDecMaxGroup];
+    int64_t N[kDecMaxGroup];
+    uint32_t *status[kDecMaxGroup];
+    const uint32_t *ready[kDecMaxGroup];
     int y_fp32;
-    float *partial;     // [nchunks][16][128]
+    float *partial;     // [nchunks][BN][128]
     uint32_t *counter;  // chunks claimed beyond the first 2 * gridDim.x; zero between calls
-    uint32_t *status;
-    const uint32_t *ready;
     int stall_first_kstep;  // failure-detection test hook
-    uint64_t first_desc[kDecMaxCtas];   // chunk_desc[c] for c < gridDim.x
-    uint64_t second_desc[kDecMaxCtas];  // chunk_desc[c + gridDim.x] where that exists
+    uint64_t first_desc[kDecMaxCtas];   // descriptor of chunk c for c < gridDim.x
+    uint64_t second_desc[kDecMaxCtas];  // of chunk c + gridDim.x where that exists
 };
+
+// matrix holding global band gb
+__device__ __forceinline__ int dec_mat_of_band(const DecodeParams &p, int gb) {
+    int i = 0;
+    while (i + 1 < p.nmat && p.band0[i + 1] <= gb) ++i;
+    return i;
+}
+
+// a wait that ran out: every matrix of the launch reports it
+__device__ __forceinline__ void dec_raise_timeout(const DecodeParams &p) {
+    for (int i = 0; i < p.nmat; ++i) atomicOr(p.status[i], kStatusTimeout);
+}
 
 // Bytes of pair i of a chunk whose k-step flags are `flags`, and whether its
 // metadata block is present.  Mirrors the packer: a 2 KB metadata block
@@ -151,11 +171,11 @@ __device__ __forceinline__ bool wait_count_bounded(volatile uint32_t *ctr, uint3
     }
 }
 
-__device__ __forceinline__ void store_out(const DecodeParams &p, int64_t idx, float v) {
+__device__ __forceinline__ void store_out(const DecodeParams &p, int mi, int64_t idx, float v) {
     if (p.y_fp32)
-        static_cast<float *>(p.Y)[idx] = v;
+        static_cast<float *>(p.Y[mi])[idx] = v;
     else
-        static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
+        static_cast<__nv_bfloat16 *>(p.Y[mi])[idx] = __float2bfloat16_rn(v);
 }
 
 template <int BN>
@@ -187,7 +207,9 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         pdl_trigger();
         // the packed bytes are final once the ready flag is seen; otherwise
         // (the packer may be the kernel just before) wait first
-        if (ld_acquire_gpu(p.ready) == 0u) pdl_wait();
+        bool all_ready = true;
+        for (int i = 0; i < p.nmat; ++i) all_ready = all_ready && ld_acquire_gpu(p.ready[i]) != 0u;
+        if (!all_ready) pdl_wait();
         else waited = false;
         for (int s = 0; s < kDecStages; ++s) {
             mbar_init(&full[s], 1);
@@ -196,7 +218,10 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
         for (int b = 0; b < 2; ++b) mbar_init(&acc_full[b], 4);
         *never_flag = 0u;
         for (int w = 0; w < 4; ++w) drained[w] = 0u;
-        *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
+        // a matrix whose status is raised skips the whole launch
+        uint32_t raised = 0u;
+        for (int i = 0; i < p.nmat; ++i) raised |= *reinterpret_cast<volatile uint32_t *>(p.status[i]);
+        *abort_flag = (raised & kStatusTimeout) ? 1u : 0u;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -264,7 +289,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     if (!(p.stall_first_kstep && blockIdx.x == 0 && it == 1)) {  // else never lands
                         uint8_t *st = smem + s * kDecStageBytes;
                         mbar_arrive_expect_tx(&full[s], bytes + kDecXBytes);
-                        bulk_g2s(st, p.packed + src, bytes, &full[s]);
+                        bulk_g2s(st, p.packed[dec_mat_of_band(p, j / p.cpb)] + src, bytes, &full[s]);
                         if (waited) {
                             tma_load_3d(st + kDecWBytes, &tmap_x, 0, 0, 2 * (pr0 + i), &full[s]);
                         } else {
@@ -290,7 +315,10 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                     }
                     have_tk = false;
                     jnn = 2 * G + static_cast<int>(tk);
-                    if (jnn < p.nchunks) dnn = __ldcg(p.chunk_desc + jnn);
+                    if (jnn < p.nchunks) {
+                        const int mi = dec_mat_of_band(p, jnn / p.cpb);
+                        dnn = __ldcg(p.chunk_desc[mi] + (jnn - p.band0[mi] * p.cpb));
+                    }
                 }
                 j = jn;
                 d = dn;
@@ -315,7 +343,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             }
             if (!ok) {
                 *abort_flag = 1u;
-                atomicOr(p.status, kStatusTimeout);
+                dec_raise_timeout(p);
             }
             // Drain: the last phase armed on every stage must have landed
             // before the CTA exits (a no-op when the MMA thread consumed all).
@@ -430,7 +458,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             }
             if (!ok) {
                 *abort_flag = 1u;
-                atomicOr(p.status, kStatusTimeout);
+                dec_raise_timeout(p);
             }
             // End of work for the epilogue: a phase whose chunk is -1, one
             // commit and one arrive from each issuer.  The commits fire once
@@ -458,7 +486,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             tc_fence_after();
             if (!ok) {
                 *abort_flag = 1u;
-                atomicOr(p.status, kStatusTimeout);
+                dec_raise_timeout(p);
                 break;
             }
             const int j = acc_chunk[buf];
@@ -506,6 +534,7 @@ decode_reduce_kernel(const __grid_constant__ DecodeParams p) {
     pdl_wait();
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.counter = 0u;
     const int band = blockIdx.x, m = blockIdx.y, row = threadIdx.x;
+    const int mi = dec_mat_of_band(p, band);
     const float *src = p.partial + (static_cast<int64_t>(band) * p.cpb * BN + m) * kBand + row;
     float acc = 0.0f;
     for (int c0 = 0; c0 < p.cpb; c0 += 8) {
@@ -517,7 +546,8 @@ decode_reduce_kernel(const __grid_constant__ DecodeParams p) {
         for (int q = 0; q < 8; ++q)
             if (c0 + q < p.cpb) acc = __fadd_rn(acc, v[q]);
     }
-    store_out(p, static_cast<int64_t>(m) * p.N + static_cast<int64_t>(band) * kBand + row, acc);
+    store_out(p, mi, static_cast<int64_t>(m) * p.N[mi] + static_cast<int64_t>(band - p.band0[mi]) * kBand + row,
+              acc);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -571,7 +601,7 @@ size_t decode_workspace_bytes(int nchunks, int bn) {
 namespace {
 
 template <int BN>
-cudaError_t launch_decode(const GemmLaunch &g, cudaStream_t stream) {
+cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) {
     using C = DecCfg<BN>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -580,6 +610,8 @@ cudaError_t launch_decode(const GemmLaunch &g, cudaStream_t stream) {
                                         C::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
+    if (count < 1 || count > kDecMaxGroup) return cudaErrorInvalidValue;
+    const GemmLaunch &g = gs[0];
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorInvalidValue;
     // X [M,K] viewed as (64 columns, M rows, K/64 k-steps); box = the four
@@ -595,15 +627,64 @@ cudaError_t launch_decode(const GemmLaunch &g, cudaStream_t stream) {
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    if (!g.chunk_desc || !g.chunk_desc_host || !g.counter) return cudaErrorInvalidValue;
-    if (g.dec_cp < 1 || g.dec_cp > kDecChunkPairs) return cudaErrorInvalidValue;
-    const int grid_ctas = std::min(std::min(g.num_sms, g.dec_nchunks), kDecMaxCtas);
+    if (!g.counter) return cudaErrorInvalidValue;
+    if (g.dec_cp < 1 || g.dec_cp > kDecChunkPairs || g.dec_cpb < 1) return cudaErrorInvalidValue;
+
+    DecodeParams p;
+    p.K = g.K;
+    p.M = g.M;
+    p.cpb = g.dec_cpb;
+    p.cp = g.dec_cp;
+    p.nmat = count;
+    p.y_fp32 = g.y_fp32;
+    p.counter = g.counter;
+    p.stall_first_kstep = g.stall_first_kstep;
+    int64_t bands = 0;
+    for (int i = 0; i < kDecMaxGroup; ++i) {
+        p.packed[i] = nullptr;
+        p.chunk_desc[i] = nullptr;
+        p.Y[i] = nullptr;
+        p.N[i] = 0;
+        p.status[i] = nullptr;
+        p.ready[i] = nullptr;
+    }
+    for (int i = 0; i < count; ++i) {
+        const GemmLaunch &m = gs[i];
+        // one chunking, one X, one output type for the whole launch
+        if (m.K != g.K || m.M != g.M || m.X != g.X || m.y_fp32 != g.y_fp32 || m.dec_cp != g.dec_cp ||
+            m.dec_cpb != g.dec_cpb || m.N % kBand != 0 || m.dec_nchunks != (m.N / kBand) * g.dec_cpb ||
+            !m.chunk_desc || !m.chunk_desc_host || !m.packed || !m.Y || !m.status || !m.ready)
+            return cudaErrorInvalidValue;
+        p.band0[i] = static_cast<int32_t>(bands);
+        p.packed[i] = m.packed;
+        p.chunk_desc[i] = m.chunk_desc;
+        p.Y[i] = m.Y;
+        p.N[i] = m.N;
+        p.status[i] = m.status;
+        p.ready[i] = m.ready;
+        bands += m.N / kBand;
+    }
+    for (int i = count; i <= kDecMaxGroup; ++i) p.band0[i] = static_cast<int32_t>(bands);
+    const int64_t nchunks = bands * g.dec_cpb;
     // a CTA's chunk ordinals travel in 16 bits (dynamic claiming could in
-    // principle hand one CTA every chunk)
-    if (g.dec_nchunks > kDecMaxChunksPerCta) return cudaErrorInvalidValue;
-    // partials: the handle's slots hold 16 token rows per chunk; wider tiles
-    // take theirs from the stream-ordered pool for the call
-    const size_t ws_bytes = decode_workspace_bytes(g.dec_nchunks, BN);
+    // principle hand one CTA every chunk); chunk numbers in 29 bits
+    if (nchunks > kDecMaxChunksPerCta) return cudaErrorInvalidValue;
+    p.nchunks = static_cast<int>(nchunks);
+    const int grid = static_cast<int>(std::min<int64_t>(std::min<int64_t>(g.num_sms, nchunks), kDecMaxCtas));
+    // host copy of chunk c's descriptor
+    auto desc_of = [&](int64_t c) {
+        int i = 0;
+        while (i + 1 < count && p.band0[i + 1] * static_cast<int64_t>(g.dec_cpb) <= c) ++i;
+        return gs[i].chunk_desc_host[c - static_cast<int64_t>(p.band0[i]) * g.dec_cpb];
+    };
+    for (int c = 0; c < kDecMaxCtas; ++c) {
+        p.first_desc[c] = c < grid ? desc_of(c) : 0ull;
+        p.second_desc[c] = (c < grid && c + grid < nchunks) ? desc_of(c + grid) : 0ull;
+    }
+    // partials: the handle's slots hold 16 token rows per chunk of one
+    // matrix; wider tiles or several matrices take theirs from the
+    // stream-ordered pool for the call
+    const size_t ws_bytes = decode_workspace_bytes(p.nchunks, BN);
     float *ws = nullptr;
     if (g.workspace && ws_bytes <= g.workspace_bytes) {
         ws = g.workspace;
@@ -611,28 +692,7 @@ cudaError_t launch_decode(const GemmLaunch &g, cudaStream_t stream) {
         const cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), ws_bytes, g.pool, stream);
         if (e != cudaSuccess) return e;
     }
-
-    DecodeParams p;
-    p.packed = g.packed;
-    p.chunk_desc = g.chunk_desc;
-    p.N = g.N;
-    p.K = g.K;
-    p.M = g.M;
-    p.cpb = g.dec_cpb;
-    p.cp = g.dec_cp;
-    p.nchunks = g.dec_nchunks;
-    p.Y = g.Y;
-    p.y_fp32 = g.y_fp32;
     p.partial = ws;
-    p.counter = g.counter;
-    p.status = g.status;
-    p.ready = g.ready;
-    p.stall_first_kstep = g.stall_first_kstep;
-    const int grid = grid_ctas;
-    for (int c = 0; c < kDecMaxCtas; ++c) {
-        p.first_desc[c] = c < grid ? g.chunk_desc_host[c] : 0ull;
-        p.second_desc[c] = (c < grid && c + grid < g.dec_nchunks) ? g.chunk_desc_host[c + grid] : 0ull;
-    }
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -647,7 +707,7 @@ cudaError_t launch_decode(const GemmLaunch &g, cudaStream_t stream) {
     cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gemm_kernel<BN>, map, p);
     if (err == cudaSuccess) {
         note_launches(1);
-        cfg.gridDim = dim3(static_cast<unsigned>(g.N / kBand), static_cast<unsigned>(g.M));
+        cfg.gridDim = dim3(static_cast<unsigned>(bands), static_cast<unsigned>(g.M));
         cfg.blockDim = dim3(kBand);
         cfg.dynamicSmemBytes = 0;
         err = cudaLaunchKernelEx(&cfg, decode_reduce_kernel<BN>, p);
@@ -662,11 +722,17 @@ cudaError_t launch_decode(const GemmLaunch &g, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
-    if (g.M <= 16) return launch_decode<16>(g, stream);
-    if (g.M <= 32) return launch_decode<32>(g, stream);
-    if (g.M <= kDecodeMaxM) return launch_decode<64>(g, stream);
+cudaError_t launch_decode_group(const GemmLaunch *gs, int count, cudaStream_t stream) {
+    if (count < 1) return cudaErrorInvalidValue;
+    const int64_t M = gs[0].M;
+    if (M <= 16) return launch_decode<16>(gs, count, stream);
+    if (M <= 32) return launch_decode<32>(gs, count, stream);
+    if (M <= kDecodeMaxM) return launch_decode<64>(gs, count, stream);
     return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
+    return launch_decode_group(&g, 1, stream);
 }
 
 }  // namespace patchk

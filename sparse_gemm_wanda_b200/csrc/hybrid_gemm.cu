@@ -812,7 +812,7 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     // f = 0.6: 4096x4096 M = 32 / 64: 11.6 / 12.5 us against 14.4 / 14.5;
     // 11008x4096: 20.7 / 24.9 against 24.1 / 25.2; 4096x11008: 21.7 / 23.2
     // against 20.6 / 21.2.
-    if (g.M <= kDecodeMaxM && g.K <= 8192) return launch_decode_gemm(g, stream);
+    if (takes_split_k(g.M, g.K, 0)) return launch_decode_gemm(g, stream);
     if (g.M <= 64) return run<64, 4>(g, 1, stream);   // 48 KB stages
     if (g.M <= 128) return run<128, 3>(g, 1, stream); // 64 KB stages
     // larger token counts: the band-pair kernel (two bands share each X tile)

@@ -783,15 +783,9 @@ static patch_status fp8_gemm(const patch_packed *Wp, const void *X_bf16, int64_t
     return from_cuda(e != cudaSuccess ? e : e2);
 }
 
-patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
-                               int32_t y_is_fp32, void *stream_v) {
-    if (!Wp || M < 0) return PATCH_ERR_INVALID_ARG;
-    if (M == 0) return PATCH_OK;  // empty batch: nothing to do
-    if (!X_bf16 || !Y) return PATCH_ERR_INVALID_ARG;
-    if (!aligned16(X_bf16) || !aligned16(Y)) return PATCH_ERR_INVALID_ARG;
-    if (y_is_fp32 != 0 && y_is_fp32 != 1) return PATCH_ERR_INVALID_ARG;
-    if (M > (int64_t(1) << 31)) return PATCH_ERR_INVALID_ARG;
-    if (Wp->pattern == 8) return fp8_gemm(Wp, X_bf16, M, Y, y_is_fp32, static_cast<cudaStream_t>(stream_v));
+// the launch description of one bf16 handle's product
+static patchk::GemmLaunch gemm_launch(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
+                                      int32_t y_is_fp32) {
     patchk::GemmLaunch g;
     g.packed = Wp->packed;
     g.table = Wp->table;
@@ -823,7 +817,50 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
     g.stall_first_kstep = g_test_stall.load(std::memory_order_relaxed);
     g.force_kernel = g_test_kernel.load(std::memory_order_relaxed);
     g.pattern = Wp->pattern;
+    return g;
+}
+
+patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
+                               int32_t y_is_fp32, void *stream_v) {
+    if (!Wp || M < 0) return PATCH_ERR_INVALID_ARG;
+    if (M == 0) return PATCH_OK;  // empty batch: nothing to do
+    if (!X_bf16 || !Y) return PATCH_ERR_INVALID_ARG;
+    if (!aligned16(X_bf16) || !aligned16(Y)) return PATCH_ERR_INVALID_ARG;
+    if (y_is_fp32 != 0 && y_is_fp32 != 1) return PATCH_ERR_INVALID_ARG;
+    if (M > (int64_t(1) << 31)) return PATCH_ERR_INVALID_ARG;
+    if (Wp->pattern == 8) return fp8_gemm(Wp, X_bf16, M, Y, y_is_fp32, static_cast<cudaStream_t>(stream_v));
+    const patchk::GemmLaunch g = gemm_launch(Wp, X_bf16, M, Y, y_is_fp32);
     return from_cuda(patchk::launch_hybrid_gemm(g, static_cast<cudaStream_t>(stream_v)));
+}
+
+patch_status patch_hybrid_gemm_group(const patch_packed *const *Wps, int32_t count, const void *X_bf16,
+                                     int64_t M, void *const *Ys, int32_t y_is_fp32, void *stream_v) {
+    if (!Wps || !Ys || count < 1 || count > patchk::kDecMaxGroup || M < 0) return PATCH_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i)
+        if (!Wps[i]) return PATCH_ERR_INVALID_ARG;
+    if (M == 0) return PATCH_OK;
+    if (!X_bf16 || !aligned16(X_bf16)) return PATCH_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i)
+        if (!Ys[i] || !aligned16(Ys[i])) return PATCH_ERR_INVALID_ARG;
+    if (y_is_fp32 != 0 && y_is_fp32 != 1) return PATCH_ERR_INVALID_ARG;
+    if (M > (int64_t(1) << 31)) return PATCH_ERR_INVALID_ARG;
+    const int64_t K = Wps[0]->shp.K;
+    const int force = g_test_kernel.load(std::memory_order_relaxed);
+    bool one_launch = count > 1 && patchk::takes_split_k(M, K, force);
+    for (int i = 0; i < count && one_launch; ++i)
+        one_launch = Wps[i]->pattern == 2 && Wps[i]->shp.K == K && Wps[i]->num_sms == Wps[0]->num_sms;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    if (!one_launch) {
+        // the products one after another on the stream (the same results)
+        for (int i = 0; i < count; ++i) {
+            const patch_status st = patch_hybrid_gemm(Wps[i], X_bf16, M, Ys[i], y_is_fp32, stream_v);
+            if (st != PATCH_OK) return st;
+        }
+        return PATCH_OK;
+    }
+    patchk::GemmLaunch gs[patchk::kDecMaxGroup];
+    for (int i = 0; i < count; ++i) gs[i] = gemm_launch(Wps[i], X_bf16, M, Ys[i], y_is_fp32);
+    return from_cuda(patchk::launch_decode_group(gs, count, stream));
 }
 
 void patch_free(patch_packed *Wp, void *stream_v) {

@@ -51,6 +51,7 @@ cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map
 // Decode (M <= 16) GEMV: CTAs whose first chunk travels in the kernel
 // parameters, at most.
 constexpr int kDecMaxCtas = 160;
+constexpr int kDecMaxGroup = 8;  // matrices sharing X in one split-K launch
 
 // Layout plan of a packed matrix, computed on the device from the tile map
 // (plan_pack_kernel) and read back once by patch_pack.
@@ -155,7 +156,20 @@ double quad_kstep_cycles(int bn);
 // Split-K GEMV / skinny GEMM for M <= kDecodeMaxM (csrc/decode_gemm.cu):
 // token tiles of 16, 32 or 64 rows.
 constexpr int64_t kDecodeMaxM = 64;
+// above 16 tokens the split-K kernel serves K up to this (longer K: the
+// one-band stream-K kernel)
+constexpr int64_t kSplitKMaxK = 8192;
+// whether a bf16 2:4 product of M tokens runs the split-K kernel (test hook
+// `force_kernel` set: only M <= 16 does)
+inline bool takes_split_k(int64_t M, int64_t K, int force_kernel) {
+    return M <= 16 || (M <= kDecodeMaxM && K <= kSplitKMaxK && force_kernel == 0);
+}
 cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream);
+// One split-K launch over `count` (1..kDecMaxGroup) matrices that read the
+// same X: the same K, M, X, output type and chunking; each member its own
+// handle fields and Y.  The first member's counter (and workspace, when large
+// enough) serve the launch.
+cudaError_t launch_decode_group(const GemmLaunch *gs, int count, cudaStream_t stream);
 // Chunking of a packed matrix for the decode GEMV: `cp` k-pairs per chunk,
 // `cpb` chunks per band.
 void plan_decode_chunks(int64_t bands, int64_t nsteps, int num_sms, int *cp, int *cpb, int *nchunks);

@@ -27,7 +27,7 @@ EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
            "patch_select_maps_global", "patch_test_stall_first_kstep", "patch_pool_usage",
            "patch_colsq", "patch_colsq_partials", "patch_colsq_fold", "patch_test_prefill_kernel",
            "patch_score_mask_nm", "patch_pack_nm", "patch_pack_fp8", "patch_quantize_fp8",
-           "patch_packed_fp8_scales")
+           "patch_packed_fp8_scales", "patch_hybrid_gemm_group")
 
 
 class PatchLibraryError(RuntimeError):
@@ -107,6 +107,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.patch_pack.argtypes = [vp, vp, vp, PatchShape, ctypes.POINTER(vp),
                                ctypes.POINTER(ctypes.c_size_t), vp]
     lib.patch_hybrid_gemm.argtypes = [vp, vp, i64, vp, i32, vp]
+    lib.patch_hybrid_gemm_group.argtypes = [ctypes.POINTER(vp), i32, vp, i64, ctypes.POINTER(vp), i32, vp]
+    lib.patch_hybrid_gemm_group.restype = ctypes.c_int
     lib.patch_free.argtypes = [vp, vp]
     lib.patch_free.restype = None
     lib.patch_get_status.argtypes = [vp]
@@ -400,6 +402,30 @@ def patch_hybrid_gemm(packed: PackedWeight, X: torch.Tensor, out: torch.Tensor |
                                  _dptr(out, want, "out"), 1 if out_fp32 else 0, _stream(stream))
     _check("patch_hybrid_gemm", code)
     return out
+
+
+def patch_hybrid_gemm_group(packed: list, X: torch.Tensor, outs: list | None = None,
+                            out_fp32: bool = False, stream=None) -> list:
+    """Ys[i] = X @ W_eff_i^T for handles that share the input X (same K), in
+    one launch where the library can (see patch_hybrid_gemm_group in
+    include/patch.h); returns the outputs."""
+    lib = load_library()
+    M, K = X.shape
+    n = len(packed)
+    for pk in packed:
+        if pk.K != K:
+            raise ValueError(f"X has {K} columns, a packed weight {pk.K}")
+    want = torch.float32 if out_fp32 else torch.bfloat16
+    if outs is None:
+        outs = [torch.empty((M, pk.N), dtype=want, device=X.device) for pk in packed]
+    if len(outs) != n:
+        raise ValueError("one output per handle")
+    handles = (ctypes.c_void_p * max(n, 1))(*[pk.handle for pk in packed])
+    ys = (ctypes.c_void_p * max(n, 1))(*[_dptr(y, want, "out") for y in outs])
+    code = lib.patch_hybrid_gemm_group(handles, n, _dptr(X, torch.bfloat16, "X"), M, ys,
+                                       1 if out_fp32 else 0, _stream(stream))
+    _check("patch_hybrid_gemm_group", code)
+    return outs
 
 
 def patch_free(packed: PackedWeight, stream=None) -> None:

@@ -374,6 +374,127 @@ def test_gemm_skinny_bounded_wait_reports_timeout(P, oracle_mod, M):
     pk.close()
 
 
+def group_problem(P, oracle_mod, shapes, K, seed, frac=0.5):
+    """Handles for matrices [N_i, K] that share one input, random maps."""
+    pks, weffs = [], []
+    for i, N in enumerate(shapes):
+        w, xc, _ = make_problem(N, K, 64, 1, seed + 7 * i)
+        nt = (N // 128) * (K // 128)
+        tmap = inputs.random_map(nt, int(round(frac * nt)), seed=seed + i)
+        r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+        pks.append(P.patch_pack(w.cuda(), r["meta"], r["map"]))
+        weffs.append(oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap))
+    return pks, weffs
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 24, 64])
+@pytest.mark.parametrize("fp32_mode", [True, False])
+def test_gemm_group_equals_single_calls(P, oracle_mod, M, fp32_mode):
+    # one launch over three matrices that read the same X gives, bit for bit,
+    # what three calls give (the same chunks, added in the same order)
+    K = 1152  # 9 k-pairs per band: a ragged last chunk
+    pks, weffs = group_problem(P, oracle_mod, [512, 768, 256], K, seed=200 + M)
+    x = inputs.activations(M, K, 300 + M, None)
+    xd = x.cuda()
+    ys = P.patch_hybrid_gemm_group(pks, xd, out_fp32=fp32_mode)
+    singles = [P.patch_hybrid_gemm(pk, xd, out_fp32=fp32_mode) for pk in pks]
+    torch.cuda.synchronize()
+    for pk in pks:
+        assert P.patch_get_status(pk) == 0
+    for y, y1, weff in zip(ys, singles, weffs):
+        assert torch.equal(y, y1)
+        rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), weff), fp32_mode)
+    for pk in pks:
+        pk.close()
+
+
+@pytest.mark.parametrize("M", [1, 8, 64])
+def test_gemm_group_block_shapes(P, oracle_mod, M):
+    # q, k, v (3 x 4096x4096) and gate, up (2 x 11008x4096) of the Llama-7B
+    # block, each group in one launch; equal to single calls, and to the
+    # oracle on sampled outputs
+    K = 4096
+    for shapes, seed in (([4096, 4096, 4096], 410), ([11008, 11008], 420)):
+        pks, weffs = group_problem(P, oracle_mod, shapes, K, seed=seed + M, frac=0.6)
+        x = inputs.activations(M, K, seed + M, inputs.outlier_channels(K, seed))
+        xd = x.cuda()
+        ys = P.patch_hybrid_gemm_group(pks, xd, out_fp32=True)
+        singles = [P.patch_hybrid_gemm(pk, xd, out_fp32=True) for pk in pks]
+        torch.cuda.synchronize()
+        g = np.random.default_rng(seed + M)
+        for y, y1, weff, pk in zip(ys, singles, weffs, pks):
+            assert P.patch_get_status(pk) == 0
+            assert torch.equal(y, y1)
+            ms, ns = g.integers(0, M, 3000), g.integers(0, pk.N, 3000)
+            yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
+            rel_rms_check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, True)
+        for pk in pks:
+            pk.close()
+
+
+def test_gemm_group_falls_back_to_single_calls(P, oracle_mod):
+    # handles that cannot share a launch (a 4:8 handle; M above the split-K
+    # range) are run one after another with the same results
+    K, M = 512, 200
+    pks, weffs = group_problem(P, oracle_mod, [256, 384], K, seed=77)
+    x = inputs.activations(M, K, 78, None)
+    ys = P.patch_hybrid_gemm_group(pks, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    for y, weff in zip(ys, weffs):
+        rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), weff), True)
+    w, xc, _ = make_problem(256, K, 64, 1, 79)
+    r48 = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=inputs.random_map(8, 4, seed=79).cuda(), nm=(4, 8))
+    pk48 = P.patch_pack(w.cuda(), r48["meta"], r48["map"], nm=(4, 8))
+    x8 = inputs.activations(8, K, 80, None)
+    mixed = [pks[0], pk48]
+    ys = P.patch_hybrid_gemm_group(mixed, x8.cuda(), out_fp32=True)
+    singles = [P.patch_hybrid_gemm(pk, x8.cuda(), out_fp32=True) for pk in mixed]
+    torch.cuda.synchronize()
+    for y, y1 in zip(ys, singles):
+        assert torch.equal(y, y1)
+    for pk in pks + [pk48]:
+        pk.close()
+
+
+def test_gemm_group_bounded_wait_raises_every_status(P, oracle_mod):
+    K, M = 512, 8
+    pks, weffs = group_problem(P, oracle_mod, [256, 128, 384], K, seed=91)
+    x = inputs.activations(M, K, 92, None)
+    P.test_stall_first_kstep(True)
+    try:
+        P.patch_hybrid_gemm_group(pks, x.cuda(), out_fp32=True)
+    finally:
+        P.test_stall_first_kstep(False)
+    for pk in pks:
+        assert P.patch_get_status(pk) == 5  # PATCH_ERR_TIMEOUT, read and cleared
+    ys = P.patch_hybrid_gemm_group(pks, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    for y, weff, pk in zip(ys, weffs, pks):
+        assert P.patch_get_status(pk) == 0
+        rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), weff), True)
+    for pk in pks:
+        pk.close()
+
+
+def test_gemm_group_bad_arguments(P, oracle_mod):
+    import ctypes
+    lib = P.load_library()
+    pks, _ = group_problem(P, oracle_mod, [128], 256, seed=95)
+    x = torch.zeros((4, 256), dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros((4, 128), dtype=torch.float32, device="cuda")
+    h = (ctypes.c_void_p * 9)(*([pks[0].handle] * 9))
+    ys = (ctypes.c_void_p * 9)(*([ctypes.c_void_p(y.data_ptr())] * 9))
+    xp = ctypes.c_void_p(x.data_ptr())
+    assert lib.patch_hybrid_gemm_group(h, 0, xp, 4, ys, 1, None) == 1
+    assert lib.patch_hybrid_gemm_group(h, 9, xp, 4, ys, 1, None) == 1
+    assert lib.patch_hybrid_gemm_group(None, 1, xp, 4, ys, 1, None) == 1
+    assert lib.patch_hybrid_gemm_group(h, 1, None, 4, ys, 1, None) == 1
+    assert lib.patch_hybrid_gemm_group(h, 1, xp, 4, ys, 2, None) == 1
+    assert lib.patch_hybrid_gemm_group(h, 1, xp, 0, ys, 1, None) == 0  # empty batch
+    torch.cuda.synchronize()
+    pks[0].close()
+
+
 def test_gemm_tiny_config(P, oracle_mod):
     # W 256x256, 64x64 tiles, 8 of 16 tiles 2:4, Xcal 64x256, X 8x256, 3 outlier channels
     wl = inputs.workloads()["tiny"]
