@@ -122,7 +122,7 @@ struct DecodeParams {
     uint32_t *status[kDecMaxGroup];
     const uint32_t *ready[kDecMaxGroup];
     int y_fp32;
-    float *partial;     // [nchunks][BN][128]
+    float *partial[kDecMaxGroup];  // per matrix: [its chunks][BN][128]
     uint32_t *counter;  // chunks claimed beyond the first 2 * gridDim.x; zero between calls
     int stall_first_kstep;  // failure-detection test hook
     uint64_t first_desc[kDecMaxCtas];   // descriptor of chunk c for c < gridDim.x
@@ -500,7 +500,9 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                 if (mask & 2u) tmem_ld_32x32b_x16(lane_base + (2 * buf + 1) * BN + c0, r1);
                 tmem_ld_wait();
                 if (*abort_flag == 0) {
-                    float *part = p.partial + (static_cast<int64_t>(j) * BN + c0) * kBand + row;
+                    const int mi = dec_mat_of_band(p, j / p.cpb);
+                    const int64_t lj = j - static_cast<int64_t>(p.band0[mi]) * p.cpb;  // chunk of matrix mi
+                    float *part = p.partial[mi] + (lj * BN + c0) * kBand + row;
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         const float v = (mask == 3u) ? __fadd_rn(__uint_as_float(r0[q]), __uint_as_float(r1[q]))
@@ -535,7 +537,7 @@ decode_reduce_kernel(const __grid_constant__ DecodeParams p) {
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.counter = 0u;
     const int band = blockIdx.x, m = blockIdx.y, row = threadIdx.x;
     const int mi = dec_mat_of_band(p, band);
-    const float *src = p.partial + (static_cast<int64_t>(band) * p.cpb * BN + m) * kBand + row;
+    const float *src = p.partial[mi] + (static_cast<int64_t>(band - p.band0[mi]) * p.cpb * BN + m) * kBand + row;
     float acc = 0.0f;
     for (int c0 = 0; c0 < p.cpb; c0 += 8) {
         float v[8];
@@ -681,18 +683,23 @@ cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) 
         p.first_desc[c] = c < grid ? desc_of(c) : 0ull;
         p.second_desc[c] = (c < grid && c + grid < nchunks) ? desc_of(c + grid) : 0ull;
     }
-    // partials: the handle's slots hold 16 token rows per chunk of one
-    // matrix; wider tiles or several matrices take theirs from the
-    // stream-ordered pool for the call
-    const size_t ws_bytes = decode_workspace_bytes(p.nchunks, BN);
+    // partials: each handle's own slots (16 token rows per chunk) where they
+    // are large enough; otherwise one block from the stream-ordered pool for
+    // the call, cut per matrix
+    bool own = true;
+    for (int i = 0; i < count; ++i)
+        own = own && gs[i].workspace &&
+              decode_workspace_bytes(gs[i].dec_nchunks, BN) <= gs[i].workspace_bytes;
     float *ws = nullptr;
-    if (g.workspace && ws_bytes <= g.workspace_bytes) {
-        ws = g.workspace;
-    } else {
-        const cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), ws_bytes, g.pool, stream);
+    if (!own) {
+        const cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws),
+                                                      decode_workspace_bytes(p.nchunks, BN), g.pool, stream);
         if (e != cudaSuccess) return e;
     }
-    p.partial = ws;
+    for (int i = 0; i < kDecMaxGroup; ++i)
+        p.partial[i] = i >= count ? nullptr
+                       : own ? gs[i].workspace
+                             : ws + static_cast<int64_t>(p.band0[i]) * g.dec_cpb * BN * kBand;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -713,7 +720,7 @@ cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) 
         err = cudaLaunchKernelEx(&cfg, decode_reduce_kernel<BN>, p);
         if (err == cudaSuccess) note_launches(1);
     }
-    if (ws != g.workspace) {
+    if (ws) {
         const cudaError_t e2 = cudaFreeAsync(ws, stream);
         if (err == cudaSuccess) err = e2;
     }
