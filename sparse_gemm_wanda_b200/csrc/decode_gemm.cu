@@ -729,6 +729,16 @@ cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) 
 
 }  // namespace
 
+void preload_decode_kernels() {
+    cudaFuncAttributes a;
+    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<16>);
+    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<32>);
+    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<64>);
+    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<16>);
+    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<32>);
+    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<64>);
+}
+
 cudaError_t launch_decode_group(const GemmLaunch *gs, int count, cudaStream_t stream) {
     if (count < 1) return cudaErrorInvalidValue;
     const int64_t M = gs[0].M;

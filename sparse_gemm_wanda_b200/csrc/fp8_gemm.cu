@@ -375,6 +375,13 @@ cudaError_t run_fp8(const Fp8Launch &g, cudaStream_t stream) {
 
 }  // namespace
 
+void preload_fp8_gemm_kernels() {
+    cudaFuncAttributes a;
+    (void)cudaFuncGetAttributes(&a, fp8_gemm_kernel<64>);
+    (void)cudaFuncGetAttributes(&a, fp8_gemm_kernel<128>);
+    (void)cudaFuncGetAttributes(&a, fp8_gemm_kernel<240>);
+}
+
 cudaError_t launch_fp8_gemm(const Fp8Launch &g, cudaStream_t stream) {
     if (g.K % kF8Step != 0 || g.N % kBand != 0 || g.M < 1) return cudaErrorInvalidValue;
     // more than one token tile: the two-SM kernel, where the bands pair up

@@ -203,6 +203,11 @@ pack_fp8_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ met
 
 }  // namespace
 
+void preload_fp8_quantize_kernels() {
+    cudaFuncAttributes a;
+    (void)cudaFuncGetAttributes(&a, fp8_quantize_rows_kernel);
+}
+
 cudaError_t launch_fp8_quantize_rows(const void *x, int64_t R, int64_t C, uint8_t *q, float *scale,
                                      cudaStream_t stream) {
     if (R < 1 || C < 8 || C % 8 != 0 || R > 0x7FFFFFFF) return cudaErrorInvalidValue;

@@ -785,6 +785,18 @@ cudaError_t run(const GemmLaunch &g, int ctas_per_sm, cudaStream_t stream) {
 
 }  // namespace
 
+void preload_hybrid_kernels() {
+    cudaFuncAttributes a;
+    (void)cudaFuncGetAttributes(&a, hybrid_gemm_kernel<64, 4, false>);
+    (void)cudaFuncGetAttributes(&a, hybrid_gemm_kernel<128, 3, false>);
+    (void)cudaFuncGetAttributes(&a, hybrid_gemm_kernel<160, 3, false>);
+    (void)cudaFuncGetAttributes(&a, hybrid_gemm_kernel<64, 4, true>);
+    (void)cudaFuncGetAttributes(&a, hybrid_gemm_kernel<128, 3, true>);
+    (void)cudaFuncGetAttributes(&a, streamk_reduce_kernel<64>);
+    (void)cudaFuncGetAttributes(&a, streamk_reduce_kernel<128>);
+    (void)cudaFuncGetAttributes(&a, streamk_reduce_kernel<160>);
+}
+
 cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     if (g.pattern == 4) {
         // 4:8 handles: the one-band kernel with converter warps, every M

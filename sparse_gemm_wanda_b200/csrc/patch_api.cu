@@ -10,6 +10,7 @@
 
 #include <algorithm>
 #include <map>
+#include <set>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -382,6 +383,27 @@ static cudaError_t noalloc_scratch_address(uint8_t **ptr) {
     return cudaSuccess;
 }
 
+// The GEMM kernels, loaded once per context (see preload_* in
+// patch_internal.h); a context the driver cannot name loads them every time
+// (cheap once loaded).
+static void preload_gemm_kernels() {
+    static std::mutex mu;
+    static std::set<unsigned long long> done;
+    unsigned long long id = 0;
+    const bool named = current_context_id(&id);
+    std::lock_guard<std::mutex> lock(mu);
+    if (named && done.count(id)) return;
+    patchk::preload_hybrid_kernels();
+    patchk::preload_decode_kernels();
+    patchk::preload_pair_kernels();
+    patchk::preload_duo_kernels();
+    patchk::preload_quad_kernels();
+    patchk::preload_fp8_gemm_kernels();
+    patchk::preload_duo_fp8_kernels();
+    patchk::preload_fp8_quantize_kernels();
+    if (named) done.insert(id);
+}
+
 patch_status patch_score_mask_noalloc(const void *W_bf16, const void *Xcal_bf16, int64_t T,
                                       const double *colsq_in, patch_shape shp,
                                       double sparse_tile_fraction, const uint32_t *map_in,
@@ -573,6 +595,7 @@ static patch_status pack_impl(const void *W_bf16, const uint32_t *meta, const ui
                                      pattern);
     patchk::PackPlan plan;
     h->pair_prefix.assign(static_cast<size_t>(bands * (Q + 1)), 0);
+    preload_gemm_kernels();  // this call waits for the device below in any case
     if (e == cudaSuccess) e = read_plan(plan_dev, &plan, h->pair_prefix_dev, &h->pair_prefix, stream);
     if (e != cudaSuccess) {
         patch_free(h, stream_v);
@@ -650,6 +673,7 @@ patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint
     // the layout is planned on the host from the map (read back in the one
     // wait of this call): a k-step is 2:4 iff every tile it overlaps is
     std::vector<uint32_t> hmap(static_cast<size_t>((n_tiles + 31) / 32));
+    preload_gemm_kernels();  // this call waits for the device below in any case
     cudaError_t e = cudaMemcpyAsync(hmap.data(), map, sizeof(uint32_t) * hmap.size(), cudaMemcpyDeviceToHost,
                                     stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);

@@ -153,6 +153,19 @@ QuadPlan plan_quad_gemm(int64_t N, int64_t M, int num_sms);
 cudaError_t launch_quad_gemm(const GemmLaunch &g, const QuadPlan &plan, cudaStream_t stream);
 double quad_kstep_cycles(int bn);
 
+// Load every GEMM kernel of the library in the current context (each file
+// its own).  Under lazy module loading the first launch of a kernel loads it,
+// which waits for the device; the pack calls, which synchronise anyway, run
+// these once per context so that no GEMM call ever does.
+void preload_hybrid_kernels();
+void preload_decode_kernels();
+void preload_pair_kernels();
+void preload_duo_kernels();
+void preload_quad_kernels();
+void preload_fp8_gemm_kernels();
+void preload_duo_fp8_kernels();
+void preload_fp8_quantize_kernels();
+
 // Split-K GEMV / skinny GEMM for M <= kDecodeMaxM (csrc/decode_gemm.cu):
 // token tiles of 16, 32 or 64 rows.
 constexpr int64_t kDecodeMaxM = 64;

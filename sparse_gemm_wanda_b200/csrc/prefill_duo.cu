@@ -448,6 +448,11 @@ double duo_kstep_cycles(int bn) {
     return std::max(2.0 * bn, 256.0 + bn);
 }
 
+void preload_duo_kernels() {
+    cudaFuncAttributes a;
+    (void)cudaFuncGetAttributes(&a, duo_gemm_kernel);
+}
+
 DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms, int max_pair_bytes) {
     DuoPlan best{};
     const int64_t bpairs = (N / kBand) / 2;

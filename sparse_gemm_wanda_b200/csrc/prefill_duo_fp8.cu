@@ -469,6 +469,11 @@ int max_clusters(int smem) {
 
 }  // namespace
 
+void preload_duo_fp8_kernels() {
+    cudaFuncAttributes a;
+    (void)cudaFuncGetAttributes(&a, duo_fp8_kernel);
+}
+
 DuoFp8Plan plan_duo_fp8(int64_t N, int64_t M, int num_sms, bool all_sparse) {
     DuoFp8Plan best{};
     const int64_t bpairs = (N / kBand) / 2;

@@ -391,6 +391,11 @@ EncodeTiledFn encode_fn() {
 
 double pair_kstep_cycles(int bn) { return 512.0 + 3.0 * bn; }
 
+void preload_pair_kernels() {
+    cudaFuncAttributes a;
+    (void)cudaFuncGetAttributes(&a, pair_gemm_kernel);
+}
+
 PairPlan plan_pair_gemm(int64_t N, int64_t M, int num_sms) {
     // Token tile: the multiple of 16 in [128, 240] that minimises
     // waves x time per item (the last wave counts whole).  A dense k-step of

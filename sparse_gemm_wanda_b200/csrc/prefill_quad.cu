@@ -457,6 +457,11 @@ double quad_kstep_cycles(int bn) {
     return std::max(4.0 * bn, 512.0 + 1.5 * bn);
 }
 
+void preload_quad_kernels() {
+    cudaFuncAttributes a;
+    (void)cudaFuncGetAttributes(&a, quad_gemm_kernel);
+}
+
 QuadPlan plan_quad_gemm(int64_t N, int64_t M, int num_sms) {
     QuadPlan best{};
     const int64_t bands = N / kBand;

@@ -616,6 +616,47 @@ def test_gemm_first_call_does_not_block_the_host(P, oracle_mod, M):
     pk.close()
 
 
+FIRST_CALL_SCRIPT = r"""
+import sys, time, torch
+sys.path.insert(0, {root!r})
+from sparse_gemm_wanda_b200 import inputs, patch as P
+P.load_library()
+N, K = 1024, 1024
+w = inputs.weight(N, K, 5).cuda()
+xc = inputs.activations(64, K, 5, None).cuda()
+tmap = inputs.random_map(64, 32, seed=5).cuda()
+r = P.patch_score_mask(w, xc, map_in=tmap)
+pk = P.patch_pack(w, r["meta"], r["map"])
+stream = torch.cuda.current_stream()
+for M in (8, 40, 300, 2048):  # split-K 16 / 64 tokens, one-band, two-SM
+    x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    torch.cuda._sleep(1_000_000_000)
+    t0 = time.perf_counter()
+    P.patch_hybrid_gemm(pk, x, out=y, out_fp32=True)
+    dt = time.perf_counter() - t0
+    busy = not stream.query()
+    torch.cuda.synchronize()
+    assert busy and dt < 0.2, (M, busy, dt)
+print("first calls ok")
+"""
+
+
+def test_gemm_first_calls_of_a_process_do_not_block_the_host():
+    # In a fresh process every GEMM kernel is launched for the first time;
+    # under lazy module loading a first launch would load the kernel and wait
+    # for the device, so the pack call (which waits anyway) loads them all.
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", FIRST_CALL_SCRIPT.format(root=root)],
+                         capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert "first calls ok" in out.stdout
+
+
 def test_gemm_repeated_calls_reset_tickets(P, oracle_mod):
     # stream-K tiles shared by several CTAs: every call must find its tickets at zero
     N, K, M = 1024, 2048, 5
@@ -788,6 +829,49 @@ def test_gemm_two_sm_kernel_mixed_maps(P, oracle_mod, N, K, M, tn, tk, frac, fp3
     with forced_kernel(P, 3):
         run_case(P, oracle_mod, N, K, M, tn, tk, frac, seed=N + M + tn + tk, fp32_mode=fp32_mode,
                  sample=6000)
+
+
+@pytest.mark.parametrize("N,K,M,frac", [
+    (1024, 1024, 300, 0.5),    # fewer items than clusters
+    (2048, 2048, 256, 0.6),
+    (4096, 4096, 512, 0.6),    # Llama-7B block shapes at M = 512
+    (11008, 4096, 512, 0.6),
+    (4096, 11008, 512, 0.6),
+    (4096, 1024, 4096, 0.5),   # many waves
+])
+def test_gemm_two_sm_kernel_block_shapes(P, oracle_mod, N, K, M, frac):
+    # the two-SM kernel where its items fill one wave or less (M = 256 / 512
+    # on the Llama-7B block shapes), a problem with fewer items than
+    # clusters, and one of many waves; repeated calls agree bit for bit
+    w, xc, x = make_problem(N, K, 64, M, seed=N + K + M)
+    nt = (N // 128) * (K // 128)
+    tmap = inputs.random_map(nt, int(round(frac * nt)), seed=N + M)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    xd = x.cuda()
+    with forced_kernel(P, 3):
+        y16 = P.patch_hybrid_gemm(pk, xd)
+        y32 = P.patch_hybrid_gemm(pk, xd, out_fp32=True)
+        y32b = P.patch_hybrid_gemm(pk, xd, out_fp32=True)
+    torch.cuda.synchronize()
+    assert P.patch_get_status(pk) == 0
+    assert torch.equal(y32, y32b)
+    weff = oracle_weff_checked(oracle_mod, r, w, xc, 128, 128, tmap=tmap)
+    if M * N <= 300 * 1024:
+        yref = oracle_mod.gemm(bf16_bits(x), weff)
+        rel_rms_check(y32, yref, True)
+        rel_rms_check(y16, yref, False)
+    else:
+        g = np.random.default_rng(N + M)
+        # every row of the first band pair and the last, and random outputs
+        ms = np.concatenate([g.integers(0, M, 3000), np.repeat(np.arange(M)[:: max(1, M // 16)], 4)])
+        ns = np.concatenate([g.integers(0, N, 3000),
+                             np.tile(np.array([0, 255, N - 256, N - 1]), len(np.arange(M)[:: max(1, M // 16)]))])
+        yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
+        mi, ni = torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()
+        rel_rms_check(y32[mi, ni], yref, True)
+        rel_rms_check(y16[mi, ni], yref, False)
+    pk.close()
 
 
 @pytest.mark.parametrize("fp32_mode", [True, False])
