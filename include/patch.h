@@ -147,8 +147,8 @@ patch_status patch_colsq(const void *Xcal_bf16, int64_t T, int64_t K, double *co
  *   patch_colsq_partials: partials_out [ceil(T/128), K] fp64 (16-byte
  *     aligned, written): row c is the sum of x_tj^2 over tokens 128c ..
  *     128c+127 of this Xcal, added token by token from 0.0.
- *   patch_colsq_fold: colsq_out[j] = the rows of partials [chunks, K] added
- *     row by row from 0.0.
+ *   patch_colsq_fold: colsq_out[j] = the rows of partials [chunks, K]
+ *     (16-byte aligned) added row by row from 0.0.
  * The partials of consecutive pieces, stacked in token order and folded, give
  * bit for bit patch_colsq's result for the whole set.  No scratch.  Errors:
  * INVALID_ARG (null pointers, T or chunks < 1, K not a multiple of 64,

@@ -316,7 +316,8 @@ patch_status patch_colsq_partials(const void *Xcal_bf16, int64_t T, int64_t K,
 
 patch_status patch_colsq_fold(const double *partials, int64_t chunks, int64_t K, double *colsq_out,
                               void *stream_v) {
-    if (!partials || !colsq_out || chunks < 1 || K < 64 || K % 64 != 0) return PATCH_ERR_INVALID_ARG;
+    if (!partials || !colsq_out || chunks < 1 || K < 64 || K % 64 != 0 || !aligned16(partials))
+        return PATCH_ERR_INVALID_ARG;
     patch_status st = check_device(nullptr);
     if (st != PATCH_OK) return st;
     return from_cuda(patchk::launch_colsq_fold(partials, chunks, K, colsq_out, nullptr,
