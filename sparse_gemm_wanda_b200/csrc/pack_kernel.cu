@@ -56,7 +56,10 @@ __device__ __forceinline__ uint32_t kept_pair(uint32_t a, uint32_t b, uint32_t c
 }
 
 // One CTA per (band, k-step); every thread writes whole 16-byte chunks of the
-// swizzled output straight from global W (no shared-memory staging).
+// swizzled output straight from global W (no shared-memory staging), its
+// loads issued before its stores.  Where the prefill table points the k-step
+// to a dense side copy (bands of a pair that differ in type), the same CTA
+// also writes that copy: the k-step's W_eff in the dense layout.
 __global__ void __launch_bounds__(kPackThreads)
 pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
             const uint32_t *__restrict__ map, int64_t N, int64_t K, int tn, int tk,
@@ -65,20 +68,20 @@ pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
             int pattern) {
     const int64_t nsteps = K / kStep;
     const int64_t steps_all = (N / kBand) * nsteps;
-    // blocks [0, steps_all): the packed k-steps; blocks [steps_all, 2 steps_all)
-    // (launched only with a prefill table): the dense side copies it points to
-    const bool side = static_cast<int64_t>(blockIdx.x) >= steps_all;
-    const int64_t idx = side ? blockIdx.x - steps_all : blockIdx.x;
+    (void)steps_all;
+    const int64_t idx = blockIdx.x;
     const int64_t b = idx / nsteps, c = idx % nsteps;
-    const uint64_t entry = side ? ptable[idx] : table[idx];
+    const uint64_t entry = table[idx];
     const int64_t off = static_cast<int64_t>(entry & kEntryOffsetMask);
+    // the dense side copy of this k-step, if the prefill table has one
+    const uint64_t sentry = ptable ? ptable[idx] : 0ull;
+    const bool side = (sentry & kEntrySide) != 0;
+    const int64_t soff = static_cast<int64_t>(sentry & kEntryOffsetMask);
     const int tid = threadIdx.x;
     const int64_t row0 = b * kBand, col0 = c * kStep;
     const int64_t words_k = K / 32;
 
-    if (side && !(entry & kEntrySide)) {
-        // the prefill table reuses the packed k-step here: nothing to write
-    } else if (entry & kEntryNM48) {
+    if (entry & kEntryNM48) {
         // 4:8: thread = row; its 32 kept values (in column order, four per
         // group of 8) at r*64, its 8 keep masks at 8192 + r*8
         const int r = tid;
@@ -114,36 +117,64 @@ pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
     } else if (!(entry & kEntrySparse)) {
         // dense: chunk u = r*8 + ((k/8) ^ (r%8)); W_eff, i.e. pruned entries of
         // a 2:4 tile (64-row tiles sharing a band with a dense tile) are zeroed
-#pragma unroll 4
-        for (int u = tid; u < kBand * 8; u += kPackThreads) {
+        constexpr int kPer = kBand * 8 / kPackThreads;
+        uint4 v[kPer];
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int u = tid + q * kPackThreads;
+            const int r = u / 8, k8 = (u % 8) ^ (r % 8);
+            v[q] = __ldg(reinterpret_cast<const uint4 *>(W + (row0 + r) * K + col0 + 8 * k8));
+        }
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int u = tid + q * kPackThreads;
             const int r = u / 8, k8 = (u % 8) ^ (r % 8);
             const int64_t i = row0 + r, j = col0 + 8 * k8;
-            uint4 v = __ldg(reinterpret_cast<const uint4 *>(W + i * K + j));
             const int64_t tile = (i / tn) * (K / tk) + j / tk;
             if ((__ldg(map + tile / 32) >> (tile % 32)) & 1u) {
                 const uint32_t mw = __ldg(meta + i * words_k + j / 32);
                 if (pattern == 4)
-                    v = mask_eight(v, (mw >> (8 * ((j % 32) / 8))) & 0xFFu);
+                    v[q] = mask_eight(v[q], (mw >> (8 * ((j % 32) / 8))) & 0xFFu);
                 else
-                    v = mask_two_groups(v, mw >> (4 * ((j % 32) / 4)));
+                    v[q] = mask_two_groups(v[q], mw >> (4 * ((j % 32) / 4)));
             }
-            reinterpret_cast<uint4 *>(out + off)[u] = v;
+            reinterpret_cast<uint4 *>(out + off)[u] = v[q];
+            if (side) reinterpret_cast<uint4 *>(out + soff)[u] = v[q];
         }
     } else {
         // 2:4: chunk u = r*4 + ((v/8) ^ ((r%8)/2)) holds the kept values of groups
         // 4*(v/8) .. 4*(v/8)+3 of the row, two per group in column order
-#pragma unroll 4
-        for (int u = tid; u < kBand * 4; u += kPackThreads) {
+        constexpr int kPer = kBand * 4 / kPackThreads;
+        uint4 a[kPer], bq[kPer];
+        uint32_t mw[kPer];
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int u = tid + q * kPackThreads;
             const int r = u / 4, v8 = (u % 4) ^ ((r % 8) / 2);
             const int64_t i = row0 + r, j = col0 + 16 * v8;
             const uint4 *src = reinterpret_cast<const uint4 *>(W + i * K + j);
-            const uint4 a = __ldg(src), bq = __ldg(src + 1);
-            const uint32_t e[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
-            const uint32_t codes = __ldg(meta + i * words_k + j / 32) >> (4 * ((j % 32) / 4));
+            a[q] = __ldg(src);
+            bq[q] = __ldg(src + 1);
+            mw[q] = __ldg(meta + i * words_k + j / 32);
+        }
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int u = tid + q * kPackThreads;
+            const int r = u / 4, v8 = (u % 4) ^ ((r % 8) / 2);
+            const int64_t j = col0 + 16 * v8;
+            const uint32_t e[8] = {a[q].x, a[q].y, a[q].z, a[q].w, bq[q].x, bq[q].y, bq[q].z, bq[q].w};
+            const uint32_t codes = mw[q] >> (4 * ((j % 32) / 4));
             uint32_t o[4];
 #pragma unroll
             for (int g = 0; g < 4; ++g) o[g] = kept_pair(e[2 * g], e[2 * g + 1], (codes >> (4 * g)) & 0xFu);
             reinterpret_cast<uint4 *>(out + off)[u] = make_uint4(o[0], o[1], o[2], o[3]);
+            if (side) {
+                // the same 16 columns as W_eff in the dense layout: chunks
+                // 2 v8 and 2 v8 + 1 of row r, at (k8 ^ (r % 8))
+                uint4 *d = reinterpret_cast<uint4 *>(out + soff) + r * 8;
+                d[(2 * v8) ^ (r % 8)] = mask_two_groups(a[q], codes);
+                d[(2 * v8 + 1) ^ (r % 8)] = mask_two_groups(bq[q], codes >> 8);
+            }
         }
         if (entry & kEntryMeta) {
             // The metadata block of k-pair p: line l = m0 + 8*k1 + 16*m2 holds, in
@@ -510,7 +541,7 @@ cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, 
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                         int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
                         uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream, int pattern) {
-    const int64_t blocks = (N / kBand) * (K / kStep) * (ptable ? 2 : 1);
+    const int64_t blocks = (N / kBand) * (K / kStep);
     if (blocks > 0x7FFFFFFF || (pattern != 2 && pattern != 4)) return cudaErrorInvalidValue;
     pack_kernel<<<static_cast<unsigned>(blocks), kPackThreads, 0, stream>>>(
         static_cast<const uint16_t *>(W), meta, map, N, K, tn, tk, table, ptable, out, done, ready,
