@@ -57,10 +57,15 @@ __device__ __forceinline__ float block_max(float v, float *red) {
 }
 
 // One block per row of a bf16 matrix [R, C] (C a multiple of 8): scale and codes.
+// Launched as a programmatic dependent: it lets the next kernel (the FP8 GEMM)
+// start its prologue at once, and touches memory only after the kernel
+// before it has completed.
 __global__ void __launch_bounds__(kQuantThreads)
 fp8_quantize_rows_kernel(const uint16_t *__restrict__ x, int64_t C, uint8_t *__restrict__ q,
                          float *__restrict__ scale) {
     __shared__ float red[kQuantThreads / 32];
+    if (threadIdx.x == 0) pdl_trigger();
+    pdl_wait();
     const int64_t r = blockIdx.x;
     const uint4 *row = reinterpret_cast<const uint4 *>(x + r * C);
     const int64_t chunks = C / 8;
@@ -211,10 +216,19 @@ void preload_fp8_quantize_kernels() {
 cudaError_t launch_fp8_quantize_rows(const void *x, int64_t R, int64_t C, uint8_t *q, float *scale,
                                      cudaStream_t stream) {
     if (R < 1 || C < 8 || C % 8 != 0 || R > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    fp8_quantize_rows_kernel<<<static_cast<unsigned>(R), kQuantThreads, 0, stream>>>(
-        static_cast<const uint16_t *>(x), C, q, scale);
-    note_launches(1);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(R));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_quantize_rows_kernel, static_cast<const uint16_t *>(x), C,
+                                             q, scale);
+    if (e == cudaSuccess) note_launches(1);
+    return e;
 }
 
 cudaError_t launch_pack_fp8(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,

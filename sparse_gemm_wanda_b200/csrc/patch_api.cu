@@ -23,6 +23,7 @@ struct patch_packed {
     int device;
     int pattern;               // 2: dense / 2:4 tiles; 4: dense / 4:8 tiles; 8: FP8 dense / 2:4
     float *fp8_scale;          // FP8 handles: W_eff row scales [N]
+    uint8_t *fp8_xscratch;     // FP8 handles: X codes and token scales of calls with M <= kFp8ScratchRows
     uint8_t *base;             // pool allocation: table, descriptors, prefix, plan, workspace, status
     patch_shape shp;
     uint8_t *packed;           // packed k-steps, then the side copies (a pool allocation of its own, exact size)
@@ -655,6 +656,13 @@ patch_status patch_quantize_fp8(const void *X_bf16, int64_t R, int64_t C, uint8_
                                                       static_cast<cudaStream_t>(stream_v)));
 }
 
+// Decode-sized FP8 calls quantise X into the handle's own scratch (no pool
+// allocation on the call); larger ones take a pool block for the call.
+constexpr int64_t kFp8ScratchRows = 64;
+static size_t fp8_xscratch_bytes(int64_t rows, int64_t K) {
+    return round_up(static_cast<size_t>(rows * K), 256) + sizeof(float) * static_cast<size_t>(rows);
+}
+
 patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
                             patch_shape shp, patch_packed **out, size_t *packed_bytes,
                             void *stream_v) {
@@ -728,11 +736,13 @@ patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint
     h->duo_ok = duo ? 1 : 0;
     h->sparse_ksteps = static_cast<int64_t>(n_sparse);
     h->meta_blocks = static_cast<int64_t>(n_sparse);
-    // allocation 1: table | prefill table | row scales | status; allocation
-    // 2: the packed bytes, then the side copies
+    // allocation 1: table | prefill table | row scales | X scratch of
+    // decode-sized calls | status; allocation 2: the packed bytes, then the
+    // side copies
     const size_t off_ptable = round_up(sizeof(uint64_t) * table.size(), 256);
     const size_t off_scale = round_up(off_ptable + sizeof(uint64_t) * ptable.size(), 256);
-    const size_t off_status = round_up(off_scale + sizeof(float) * static_cast<size_t>(N), 256);
+    const size_t off_xs = round_up(off_scale + sizeof(float) * static_cast<size_t>(N), 256);
+    const size_t off_status = round_up(off_xs + fp8_xscratch_bytes(kFp8ScratchRows, K), 256);
     const size_t total = off_status + 256;
     e = patchk::device_pool(&h->pool);
     if (e == cudaSuccess) e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->base), total, h->pool, stream);
@@ -743,6 +753,7 @@ patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint
     h->table = reinterpret_cast<uint64_t *>(h->base);
     h->ptable = duo ? reinterpret_cast<uint64_t *>(h->base + off_ptable) : nullptr;
     h->fp8_scale = reinterpret_cast<float *>(h->base + off_scale);
+    h->fp8_xscratch = h->base + off_xs;
     h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
     e = cudaMemsetAsync(h->status, 0, 256, stream);
     if (e == cudaSuccess)
@@ -776,11 +787,16 @@ patch_status patch_packed_fp8_scales(const patch_packed *Wp, float *scales_dst, 
 static patch_status fp8_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
                              int32_t y_is_fp32, cudaStream_t stream) {
     const int64_t K = Wp->shp.K;
-    // the activations' codes and token scales, for this call only
+    // the activations' codes and token scales
     const size_t off_sx = round_up(static_cast<size_t>(M * K), 256);
     const size_t bytes = off_sx + sizeof(float) * static_cast<size_t>(M);
     uint8_t *ws = nullptr;
-    cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), bytes, Wp->pool, stream);
+    const bool own = M <= kFp8ScratchRows && Wp->fp8_xscratch;
+    cudaError_t e = cudaSuccess;
+    if (own)
+        ws = Wp->fp8_xscratch;
+    else
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws), bytes, Wp->pool, stream);
     if (e != cudaSuccess) return from_cuda(e);
     float *sx = reinterpret_cast<float *>(ws + off_sx);
     e = patchk::launch_fp8_quantize_rows(X_bf16, M, K, ws, sx, stream);
@@ -802,9 +818,10 @@ static patch_status fp8_gemm(const patch_packed *Wp, const void *X_bf16, int64_t
         g.y_fp32 = y_is_fp32;
         g.status = Wp->status;
         g.num_sms = Wp->num_sms;
+        g.pool = Wp->pool;
         e = patchk::launch_fp8_gemm(g, stream);
     }
-    cudaError_t e2 = cudaFreeAsync(ws, stream);
+    const cudaError_t e2 = own ? cudaSuccess : cudaFreeAsync(ws, stream);
     return from_cuda(e != cudaSuccess ? e : e2);
 }
 

@@ -219,6 +219,7 @@ struct Fp8Launch {
     uint32_t *status;
     int num_sms;
     int force_kernel;        // test hook: 1 = one band per CTA, 3 = two-SM kernel, 0 = chosen here
+    cudaMemPool_t pool;      // split-K partials of the one-band kernel (null: no split)
 };
 cudaError_t launch_fp8_gemm(const Fp8Launch &g, cudaStream_t stream);
 
