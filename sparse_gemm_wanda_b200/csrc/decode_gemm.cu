@@ -77,7 +77,9 @@ struct DecCfg {
     static constexpr int kStageBytes = kDecWBytes + kXBytes;
     static constexpr int kStages = BN == 16 ? 3 : 2;
     static constexpr uint32_t kEcol = 4 * BN;
-    static constexpr int kCols = 4 * BN + 16;
+    // metadata: per issuer 2 pairs x 2 k-steps x 4 columns (FP8 k-steps each
+    // carry their own block; bf16 pairs use the first 4 of each 8)
+    static constexpr int kCols = 4 * BN + 32;
     static constexpr int kTmemCols = kCols <= 128 ? 128 : kCols <= 256 ? 256 : 512;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 512;
     static_assert(kStageBytes % 1024 == 0, "stage regions stay 1024-B aligned");
@@ -122,6 +124,8 @@ struct DecodeParams {
     uint32_t *status[kDecMaxGroup];
     const uint32_t *ready[kDecMaxGroup];
     int y_fp32;
+    const float *f8_sw;  // FP8: [N] row scales (one matrix)
+    const float *f8_sx;  // FP8: [M] token scales
     float *partial[kDecMaxGroup];  // per matrix: [its chunks][BN][128]
     uint32_t *counter;  // chunks claimed beyond the first 2 * gridDim.x; zero between calls
     int stall_first_kstep;  // failure-detection test hook
@@ -144,8 +148,14 @@ __device__ __forceinline__ void dec_raise_timeout(const DecodeParams &p) {
 // Bytes of pair i of a chunk whose k-step flags are `flags`, and whether its
 // metadata block is present.  Mirrors the packer: a 2 KB metadata block
 // precedes the first 2:4 k-step of every k-pair.
+// FP8 (e4m3): every 2:4 k-step carries its own 2 KB metadata block.
+template <bool F8>
 __device__ __forceinline__ uint32_t pair_bytes(uint32_t flags, int i) {
     const uint32_t f = (flags >> (2 * i)) & 3u;
+    if constexpr (F8) {
+        const uint32_t sp = kMetaBlockBytes + kSparseStepBytes;
+        return ((f & 1u) ? sp : kDenseStepBytes) + ((f & 2u) ? sp : kDenseStepBytes);
+    }
     return (f == 0u) ? 2u * kDenseStepBytes
                      : (f == 3u) ? kMetaBlockBytes + 2u * kSparseStepBytes
                                  : kMetaBlockBytes + kDenseStepBytes + kSparseStepBytes;
@@ -178,7 +188,7 @@ __device__ __forceinline__ void store_out(const DecodeParams &p, int mi, int64_t
         static_cast<__nv_bfloat16 *>(p.Y[mi])[idx] = __float2bfloat16_rn(v);
 }
 
-template <int BN>
+template <int BN, bool F8>
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ DecodeParams p) {
     using C = DecCfg<BN>;
@@ -276,7 +286,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
                         break;
                     }
                     const int sp = min(2, np - i);
-                    const uint32_t bytes = pair_bytes(flags, i) + (sp == 2 ? pair_bytes(flags, i + 1) : 0u);
+                    const uint32_t bytes = pair_bytes<F8>(flags, i) + (sp == 2 ? pair_bytes<F8>(flags, i + 1) : 0u);
                     const uint32_t sflags = (flags >> (2 * i)) & (sp == 2 ? 0xFu : 0x3u);
                     stage_word[s] = static_cast<uint64_t>(j) | (np > 2 ? kStageTwo : 0ull) |
                                     (static_cast<uint64_t>(sp) << kStagePairsShift) |
@@ -360,13 +370,13 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
             // Descriptors: a template per layout plus the operand's shared
             // address in 16-byte units (all addresses here are below 256 KB,
             // so the 14-bit address field never carries into other fields).
-            constexpr uint32_t kIdDense = idesc_bf16(BN, false);
-            constexpr uint32_t kIdSp0 = idesc_bf16(BN, true, 0);
+            constexpr uint32_t kIdDense = F8 ? idesc_e4m3(BN, false) : idesc_bf16(BN, false);
+            constexpr uint32_t kIdSp0 = F8 ? idesc_e4m3(BN, true) : idesc_bf16(BN, true, 0);
             constexpr uint32_t kIdSp1 = idesc_bf16(BN, true, 1);
             const uint64_t t_sw128 = smem_desc(0, 16, 1024, kSwizzle128B);  // dense A, X
             const uint64_t t_sw64 = smem_desc(0, 16, 512, kSwizzle64B);     // 2:4 A
             const uint64_t t_meta = smem_desc(0, 16, 128, kSwizzleNone);    // metadata
-            const uint32_t e_tmem = tmem_base + C::kEcol + 8 * q;
+            const uint32_t e_tmem = tmem_base + C::kEcol + 16 * q;
             const uint32_t smem0 = smem_u32(smem);
             int it = q;       // ring position
             int nch = 0;      // chunks of this CTA (from the done word)
@@ -425,24 +435,48 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const uint64_t bx = x16 + (2 * t + h) * (kDecXStepBytes >> 4);
-                        if ((f >> h) & 1u) {
-                            // the pair's metadata block precedes its first 2:4 k-step
-                            if (h == 0 || !(f & 1u)) {
-                                tmem_cp_128x128b(e_tmem + 4 * t, t_meta + st16 + off16);
+                        if constexpr (F8) {
+                            // a 128-column e4m3 k-step: the byte shape of a bf16
+                            // 64-column one (128-byte rows dense, 64-byte rows of
+                            // kept codes), K32 dense / K64 sparse per MMA; a 2:4
+                            // k-step's own metadata block precedes it, sparse MMA
+                            // j reads columns e + 2j with selector 0
+                            if ((f >> h) & 1u) {
+                                const uint32_t e = e_tmem + 8 * t + 4 * h;
+                                tmem_cp_128x128b(e, t_meta + st16 + off16);
                                 off16 += kMetaBlockBytes >> 4;
+                                const uint64_t a = t_sw64 + st16 + off16;
+                                mma_f8_sparse(d_tmem, a, bx, e, kIdSp0, acc);
+                                mma_f8_sparse(d_tmem, a + 2, bx + 4, e + 2, kIdSp0, 1u);
+                                off16 += kSparseStepBytes >> 4;
+                            } else {
+                                const uint64_t a = t_sw128 + st16 + off16;
+                                mma_f8(d_tmem, a, bx, kIdDense, acc);
+                                mma_f8(d_tmem, a + 2, bx + 2, kIdDense, 1u);
+                                mma_f8(d_tmem, a + 4, bx + 4, kIdDense, 1u);
+                                mma_f8(d_tmem, a + 6, bx + 6, kIdDense, 1u);
+                                off16 += kDenseStepBytes >> 4;
                             }
-                            const uint64_t a = t_sw64 + st16 + off16;
-                            const uint32_t e = e_tmem + 4 * t + 2 * h;
-                            mma_sparse(d_tmem, a, bx, e, kIdSp0, acc);
-                            mma_sparse(d_tmem, a + 2, bx + 4, e, kIdSp1, 1u);
-                            off16 += kSparseStepBytes >> 4;
                         } else {
-                            const uint64_t a = t_sw128 + st16 + off16;
-                            mma_dense(d_tmem, a, bx, kIdDense, acc);
-                            mma_dense(d_tmem, a + 2, bx + 2, kIdDense, 1u);
-                            mma_dense(d_tmem, a + 4, bx + 4, kIdDense, 1u);
-                            mma_dense(d_tmem, a + 6, bx + 6, kIdDense, 1u);
-                            off16 += kDenseStepBytes >> 4;
+                            if ((f >> h) & 1u) {
+                                // the pair's metadata block precedes its first 2:4 k-step
+                                if (h == 0 || !(f & 1u)) {
+                                    tmem_cp_128x128b(e_tmem + 8 * t, t_meta + st16 + off16);
+                                    off16 += kMetaBlockBytes >> 4;
+                                }
+                                const uint64_t a = t_sw64 + st16 + off16;
+                                const uint32_t e = e_tmem + 8 * t + 2 * h;
+                                mma_sparse(d_tmem, a, bx, e, kIdSp0, acc);
+                                mma_sparse(d_tmem, a + 2, bx + 4, e, kIdSp1, 1u);
+                                off16 += kSparseStepBytes >> 4;
+                            } else {
+                                const uint64_t a = t_sw128 + st16 + off16;
+                                mma_dense(d_tmem, a, bx, kIdDense, acc);
+                                mma_dense(d_tmem, a + 2, bx + 2, kIdDense, 1u);
+                                mma_dense(d_tmem, a + 4, bx + 4, kIdDense, 1u);
+                                mma_dense(d_tmem, a + 6, bx + 6, kIdDense, 1u);
+                                off16 += kDenseStepBytes >> 4;
+                            }
                         }
                         acc = 1u;
                     }
@@ -529,7 +563,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_cons
 // Fix-up: Y[m, band*128 + row] = the band's chunk partials added in chunk
 // order.  Block (band, m), one thread per row.  Launched as a programmatic
 // dependent of the GEMM; resets the chunk counter once the GEMM is complete.
-template <int BN>
+template <int BN, bool F8>
 __global__ void __launch_bounds__(kBand)
 decode_reduce_kernel(const __grid_constant__ DecodeParams p) {
     if (threadIdx.x == 0) pdl_trigger();  // the next GEMM may start its prologue
@@ -548,8 +582,9 @@ decode_reduce_kernel(const __grid_constant__ DecodeParams p) {
         for (int q = 0; q < 8; ++q)
             if (c0 + q < p.cpb) acc = __fadd_rn(acc, v[q]);
     }
-    store_out(p, mi, static_cast<int64_t>(m) * p.N[mi] + static_cast<int64_t>(band - p.band0[mi]) * kBand + row,
-              acc);
+    const int64_t n = static_cast<int64_t>(band - p.band0[mi]) * kBand + row;
+    if constexpr (F8) acc = acc * __ldg(p.f8_sw + n) * __ldg(p.f8_sx + m);
+    store_out(p, mi, static_cast<int64_t>(m) * p.N[mi] + n, acc);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -602,32 +637,36 @@ size_t decode_workspace_bytes(int nchunks, int bn) {
 
 namespace {
 
-template <int BN>
+template <int BN, bool F8>
 cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) {
     using C = DecCfg<BN>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(decode_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(decode_gemm_kernel<BN, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    if (count < 1 || count > kDecMaxGroup) return cudaErrorInvalidValue;
+    if (count < 1 || count > kDecMaxGroup || (F8 && count != 1)) return cudaErrorInvalidValue;
     const GemmLaunch &g = gs[0];
+    if (F8 && (!g.f8_sw || !g.f8_sx)) return cudaErrorInvalidValue;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorInvalidValue;
-    // X [M,K] viewed as (64 columns, M rows, K/64 k-steps); box = the four
-    // k-steps of a stage, BN rows, 128-byte swizzle, rows past M and k-steps
-    // past K read as zero
+    // X [M,K] viewed as (128-byte column blocks, M rows, K-steps): 64 bf16
+    // columns or 128 e4m3 codes per k-step; box = the four k-steps of a
+    // stage, BN rows, 128-byte swizzle, rows past M and k-steps past K read
+    // as zero
+    const int64_t kstep_cols = F8 ? 128 : kStep, elem = F8 ? 1 : 2;
     CUtensorMap map;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kStep), static_cast<cuuint64_t>(g.M),
-                                static_cast<cuuint64_t>(g.K / kStep)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.K) * 2, static_cast<cuuint64_t>(kStep) * 2};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kStep), static_cast<cuuint32_t>(BN), 4};
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kstep_cols), static_cast<cuuint64_t>(g.M),
+                                static_cast<cuuint64_t>(g.K / kstep_cols)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.K * elem), static_cast<cuuint64_t>(kstep_cols * elem)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kstep_cols), static_cast<cuuint32_t>(BN), 4};
     const cuuint32_t estr[3] = {1, 1, 1};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(g.X), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    if (enc(&map, F8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+            const_cast<void *>(g.X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     if (!g.counter) return cudaErrorInvalidValue;
     if (g.dec_cp < 1 || g.dec_cp > kDecChunkPairs || g.dec_cpb < 1) return cudaErrorInvalidValue;
@@ -639,6 +678,8 @@ cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) 
     p.cp = g.dec_cp;
     p.nmat = count;
     p.y_fp32 = g.y_fp32;
+    p.f8_sw = g.f8_sw;
+    p.f8_sx = g.f8_sx;
     p.counter = g.counter;
     p.stall_first_kstep = g.stall_first_kstep;
     int64_t bands = 0;
@@ -711,13 +752,13 @@ cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gemm_kernel<BN>, map, p);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, decode_gemm_kernel<BN, F8>, map, p);
     if (err == cudaSuccess) {
         note_launches(1);
         cfg.gridDim = dim3(static_cast<unsigned>(bands), static_cast<unsigned>(g.M));
         cfg.blockDim = dim3(kBand);
         cfg.dynamicSmemBytes = 0;
-        err = cudaLaunchKernelEx(&cfg, decode_reduce_kernel<BN>, p);
+        err = cudaLaunchKernelEx(&cfg, decode_reduce_kernel<BN, F8>, p);
         if (err == cudaSuccess) note_launches(1);
     }
     if (ws) {
@@ -731,25 +772,38 @@ cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) 
 
 void preload_decode_kernels() {
     cudaFuncAttributes a;
-    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<16>);
-    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<32>);
-    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<64>);
-    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<16>);
-    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<32>);
-    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<64>);
+    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<16, false>);
+    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<32, false>);
+    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<64, false>);
+    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<16, false>);
+    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<32, false>);
+    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<64, false>);
+    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<16, true>);
+    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<32, true>);
+    (void)cudaFuncGetAttributes(&a, decode_gemm_kernel<64, true>);
+    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<16, true>);
+    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<32, true>);
+    (void)cudaFuncGetAttributes(&a, decode_reduce_kernel<64, true>);
 }
 
 cudaError_t launch_decode_group(const GemmLaunch *gs, int count, cudaStream_t stream) {
     if (count < 1) return cudaErrorInvalidValue;
     const int64_t M = gs[0].M;
-    if (M <= 16) return launch_decode<16>(gs, count, stream);
-    if (M <= 32) return launch_decode<32>(gs, count, stream);
-    if (M <= kDecodeMaxM) return launch_decode<64>(gs, count, stream);
+    if (M <= 16) return launch_decode<16, false>(gs, count, stream);
+    if (M <= 32) return launch_decode<32, false>(gs, count, stream);
+    if (M <= kDecodeMaxM) return launch_decode<64, false>(gs, count, stream);
     return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
     return launch_decode_group(&g, 1, stream);
+}
+
+cudaError_t launch_decode_f8(const GemmLaunch &g, cudaStream_t stream) {
+    if (g.M <= 16) return launch_decode<16, true>(&g, 1, stream);
+    if (g.M <= 32) return launch_decode<32, true>(&g, 1, stream);
+    if (g.M <= kDecodeMaxM) return launch_decode<64, true>(&g, 1, stream);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace patchk

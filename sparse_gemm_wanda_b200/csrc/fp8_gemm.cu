@@ -71,32 +71,6 @@ __device__ __forceinline__ void f8_item(const F8Params &p, int w, int &tile, int
     c1 = min(p.steps, c0 + p.kper);
 }
 
-__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void mma_f8_sparse(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                              uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// kind::f8f6f4 instruction descriptor: A and B e4m3 (format 0), K-major, fp32
-// D, M = 128, the given N; `sparse` sets the 2:4 flag (selector 0).
-__host__ __device__ constexpr uint32_t idesc_e4m3(int n, bool sparse) {
-    return (sparse ? (1u << 2) : 0u) | (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) |
-           (static_cast<uint32_t>(128 >> 4) << 24);
-}
-
 __device__ __forceinline__ void store_y(const F8Params &p, int64_t idx, float v) {
     if (p.y_fp32)
         static_cast<float *>(p.Y)[idx] = v;

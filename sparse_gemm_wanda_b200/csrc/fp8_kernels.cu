@@ -208,9 +208,12 @@ pack_fp8_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ met
 
 }  // namespace
 
+__global__ void publish_ready_kernel(uint32_t *ready) { st_release_gpu(ready, 1u); }
+
 void preload_fp8_quantize_kernels() {
     cudaFuncAttributes a;
     (void)cudaFuncGetAttributes(&a, fp8_quantize_rows_kernel);
+    (void)cudaFuncGetAttributes(&a, publish_ready_kernel);
 }
 
 cudaError_t launch_fp8_quantize_rows(const void *x, int64_t R, int64_t C, uint8_t *q, float *scale,
@@ -233,7 +236,7 @@ cudaError_t launch_fp8_quantize_rows(const void *x, int64_t R, int64_t C, uint8_
 
 cudaError_t launch_pack_fp8(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                             int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
-                            float *scale, uint8_t *out, cudaStream_t stream) {
+                            float *scale, uint8_t *out, uint32_t *ready, cudaStream_t stream) {
     if (N % kBand != 0 || K % 128 != 0 || N > 0x7FFFFFFF) return cudaErrorInvalidValue;
     fp8_weff_scales_kernel<<<static_cast<unsigned>(N), kQuantThreads, 0, stream>>>(
         static_cast<const uint16_t *>(W), meta, map, K, tn, tk, scale);
@@ -241,6 +244,13 @@ cudaError_t launch_pack_fp8(const void *W, const uint32_t *meta, const uint32_t 
     pack_fp8_kernel<<<static_cast<unsigned>(ptable ? 2 * units : units), 128, 0, stream>>>(
         static_cast<const uint16_t *>(W), meta, map, K, tn, tk, scale, table, ptable, units, out);
     note_launches(2);
+    // the packed codes and scales are final once the kernels above have
+    // completed (stream order): the split-K GEMM may then fetch them ahead of
+    // its griddepcontrol.wait
+    if (ready) {
+        publish_ready_kernel<<<1, 1, 0, stream>>>(ready);
+        note_launches(1);
+    }
     return cudaGetLastError();
 }
 

@@ -724,6 +724,29 @@ patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint
                     side += patchk::kDenseStepBytes;
                 }
             }
+    // split-K chunks for decode token counts (an even k-step count: two
+    // 128-column k-steps per pair): per chunk the first byte (a 2:4 k-step's
+    // metadata block precedes it), each k-step's 2:4 flag and the pair count
+    int dec_cp = 0, dec_cpb = 0, dec_nchunks = 0;
+    std::vector<uint64_t> chunk_desc;
+    if (steps % 2 == 0) {
+        patchk::plan_decode_chunks(bands, steps, num_sms, &dec_cp, &dec_cpb, &dec_nchunks);
+        chunk_desc.resize(static_cast<size_t>(dec_nchunks));
+        const int64_t Q = steps / 2;
+        for (int64_t b = 0; b < bands; ++b)
+            for (int64_t q = 0; q < dec_cpb; ++q) {
+                const int64_t pr0 = q * dec_cp, np = std::min<int64_t>(dec_cp, Q - pr0);
+                const uint64_t e0 = table[static_cast<size_t>(b * steps + 2 * pr0)];
+                const uint64_t first = (e0 & patchk::kEntryOffsetMask) -
+                                       ((e0 & patchk::kEntrySparse) ? patchk::kMetaBlockBytes : 0);
+                uint64_t flags = 0;
+                for (int64_t i = 0; i < 2 * np; ++i)
+                    if (table[static_cast<size_t>(b * steps + 2 * pr0 + i)] & patchk::kEntrySparse) flags |= 1ull << i;
+                chunk_desc[static_cast<size_t>(b * dec_cpb + q)] =
+                    (first & ((1ull << 40) - 1)) | (flags << 40) | (static_cast<uint64_t>(np) << 56);
+            }
+        if (off >= (1ull << 40)) dec_nchunks = 0;  // descriptors hold 40-bit offsets
+    }
     patch_packed *h = new (std::nothrow) patch_packed();
     if (!h) return PATCH_ERR_OOM;
     cudaGetDevice(&h->device);
@@ -739,10 +762,13 @@ patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint
     // allocation 1: table | prefill table | row scales | X scratch of
     // decode-sized calls | status; allocation 2: the packed bytes, then the
     // side copies
+    const size_t ws_bytes = dec_nchunks ? patchk::decode_workspace_bytes(dec_nchunks) : 0;
     const size_t off_ptable = round_up(sizeof(uint64_t) * table.size(), 256);
     const size_t off_scale = round_up(off_ptable + sizeof(uint64_t) * ptable.size(), 256);
     const size_t off_xs = round_up(off_scale + sizeof(float) * static_cast<size_t>(N), 256);
-    const size_t off_status = round_up(off_xs + fp8_xscratch_bytes(kFp8ScratchRows, K), 256);
+    const size_t off_chunks = round_up(off_xs + fp8_xscratch_bytes(kFp8ScratchRows, K), 256);
+    const size_t off_ws = round_up(off_chunks + sizeof(uint64_t) * chunk_desc.size(), 256);
+    const size_t off_status = round_up(off_ws + ws_bytes, 256);
     const size_t total = off_status + 256;
     e = patchk::device_pool(&h->pool);
     if (e == cudaSuccess) e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->base), total, h->pool, stream);
@@ -755,6 +781,16 @@ patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint
     h->fp8_scale = reinterpret_cast<float *>(h->base + off_scale);
     h->fp8_xscratch = h->base + off_xs;
     h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
+    if (dec_nchunks) {
+        h->dec_cp = dec_cp;
+        h->dec_cpb = dec_cpb;
+        h->dec_nchunks = dec_nchunks;
+        h->chunk_desc = reinterpret_cast<uint64_t *>(h->base + off_chunks);
+        h->chunk_desc_host.assign(chunk_desc.begin(),
+                                  chunk_desc.begin() + std::min<int64_t>(dec_nchunks, 2 * patchk::kDecMaxCtas));
+        h->workspace = reinterpret_cast<float *>(h->base + off_ws);
+        h->workspace_bytes = ws_bytes;
+    }
     e = cudaMemsetAsync(h->status, 0, 256, stream);
     if (e == cudaSuccess)
         e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->packed), std::max<size_t>(off + side, 16),
@@ -766,9 +802,12 @@ patch_status patch_pack_fp8(const void *W_bf16, const uint32_t *meta, const uint
     if (e == cudaSuccess && duo)
         e = cudaMemcpyAsync(h->ptable, ptable.data(), sizeof(uint64_t) * ptable.size(), cudaMemcpyHostToDevice,
                             stream);
+    if (e == cudaSuccess && dec_nchunks)
+        e = cudaMemcpyAsync(h->chunk_desc, chunk_desc.data(), sizeof(uint64_t) * chunk_desc.size(),
+                            cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess)
         e = patchk::launch_pack_fp8(W_bf16, meta, map, N, K, static_cast<int>(tn), static_cast<int>(tk),
-                                    h->table, h->ptable, h->fp8_scale, h->packed, stream);
+                                    h->table, h->ptable, h->fp8_scale, h->packed, h->status + 2, stream);
     if (e != cudaSuccess) {
         patch_free(h, stream_v);
         return from_cuda(e);
@@ -800,7 +839,36 @@ static patch_status fp8_gemm(const patch_packed *Wp, const void *X_bf16, int64_t
     if (e != cudaSuccess) return from_cuda(e);
     float *sx = reinterpret_cast<float *>(ws + off_sx);
     e = patchk::launch_fp8_quantize_rows(X_bf16, M, K, ws, sx, stream);
-    if (e == cudaSuccess) {
+    const int force = g_test_kernel.load(std::memory_order_relaxed);
+    if (e == cudaSuccess && M <= patchk::kDecodeMaxM && Wp->dec_nchunks > 0 && force == 0) {
+        // decode token counts: the split-K kernel on the e4m3 codes, the weights
+        // read once over every SM; the fix-up applies the row and token scales
+        patchk::GemmLaunch g = {};
+        g.packed = Wp->packed;
+        g.table = Wp->table;
+        g.N = Wp->shp.N;
+        g.K = K;
+        g.X = ws;
+        g.M = M;
+        g.Y = Y;
+        g.y_fp32 = y_is_fp32;
+        g.workspace = Wp->workspace;
+        g.workspace_bytes = Wp->workspace_bytes;
+        g.pool = Wp->pool;
+        g.status = Wp->status;
+        g.ready = Wp->status + 2;  // raised once the pack's kernels have completed
+        g.counter = Wp->status + 3;
+        g.chunk_desc = Wp->chunk_desc;
+        g.chunk_desc_host = Wp->chunk_desc_host.data();
+        g.dec_cp = Wp->dec_cp;
+        g.dec_cpb = Wp->dec_cpb;
+        g.dec_nchunks = Wp->dec_nchunks;
+        g.num_sms = Wp->num_sms;
+        g.stall_first_kstep = g_test_stall.load(std::memory_order_relaxed);
+        g.f8_sw = Wp->fp8_scale;
+        g.f8_sx = sx;
+        e = patchk::launch_decode_f8(g, stream);
+    } else if (e == cudaSuccess) {
         patchk::Fp8Launch g;
         g.packed = Wp->packed;
         g.table = Wp->table;

@@ -207,6 +207,33 @@ __device__ __forceinline__ void mma_sparse(uint32_t d_tmem, uint64_t a_desc, uin
         : "memory");
 }
 
+// kind::f8f6f4 (e4m3 x e4m3 -> fp32), one CTA: dense and 2:4.
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_f8_sparse(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// kind::f8f6f4 instruction descriptor: A and B e4m3 (format 0), K-major, fp32
+// D, M = 128, the given N; `sparse` sets the 2:4 flag (selector 0).
+__host__ __device__ constexpr uint32_t idesc_e4m3(int n, bool sparse) {
+    return (sparse ? (1u << 2) : 0u) | (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(128 >> 4) << 24);
+}
+
 // Copy 128 rows x 128 bits from shared memory into 128 TMEM lanes x 4 columns.
 __device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t s_desc) {
     asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(s_desc) : "memory");

@@ -103,6 +103,9 @@ struct GemmLaunch {
     int force_kernel;        // test hook: 0 auto, 1 one-band, 2 band-pair, 3 two-SM, 4 two-SM four-band (M > 16)
     int pattern;             // 2: dense / 2:4 tiles; 4: dense / 4:8 tiles
     const int64_t *pair_prefix;  // host: per band, cumulative packed bytes of its k-pairs
+    // FP8 handles (split-K path only): X holds the e4m3 codes, Y = acc * sw[n] * sx[m]
+    const float *f8_sw;      // [N] W_eff row scales
+    const float *f8_sx;      // [M] token scales
 };
 
 // Picks the configuration (token tile, schedule) for M and launches.
@@ -183,6 +186,10 @@ cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream);
 // handle fields and Y.  The first member's counter (and workspace, when large
 // enough) serve the launch.
 cudaError_t launch_decode_group(const GemmLaunch *gs, int count, cudaStream_t stream);
+// The same split-K kernel on an FP8 handle (one matrix): 128-column e4m3
+// k-steps taken two per "pair", kind::f8f6f4 MMAs, the fix-up applying the
+// row and token scales.  g.X is the e4m3 code matrix [M, K], M <= kDecodeMaxM.
+cudaError_t launch_decode_f8(const GemmLaunch &g, cudaStream_t stream);
 // Chunking of a packed matrix for the decode GEMV: `cp` k-pairs per chunk,
 // `cpb` chunks per band.
 void plan_decode_chunks(int64_t bands, int64_t nsteps, int num_sms, int *cp, int *cpb, int *nchunks);
@@ -203,7 +210,7 @@ cudaError_t launch_fp8_quantize_rows(const void *x, int64_t R, int64_t C, uint8_
 // dense copies of their k-steps' W_eff codes
 cudaError_t launch_pack_fp8(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                             int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
-                            float *scale, uint8_t *out, cudaStream_t stream);
+                            float *scale, uint8_t *out, uint32_t *ready, cudaStream_t stream);
 struct Fp8Launch {
     const uint8_t *packed;
     const uint64_t *table;   // [N/128][K/128]
