@@ -170,3 +170,48 @@ def test_gemm_fp8_odd_kstep_count_falls_back(P, oracle_mod):
     # an odd number of 128-column k-steps (K = 384) keeps the one-band kernel
     with forced_kernel(P, 3):
         run_fp8_gemm(P, oracle_mod, 512, 384, 300, 128, 128, 0.5, seed=17, fp32_mode=False)
+
+
+@pytest.mark.parametrize("N,K", [(128, 256), (256, 1280), (384, 2304), (128, 3072)])
+@pytest.mark.parametrize("M", [1, 5, 16, 33, 64])
+def test_gemm_fp8_split_k_ragged_chunks(P, oracle_mod, N, K, M):
+    # M <= 64 on FP8 handles with an even count of 128-column k-steps: the
+    # split-K kernel; pairs per band 1, 5, 9, 12 (chunks of fewer than four
+    # pairs, single-pair stages, single-band matrices), 16 / 32 / 64-token tiles
+    run_fp8_gemm(P, oracle_mod, N, K, M, 128, 128, 0.5, seed=N + K + M, fp32_mode=True)
+
+
+@pytest.mark.parametrize("M", [1, 16, 64])
+def test_gemm_fp8_split_k_full_shapes(P, oracle_mod, M):
+    # the Llama-7B decode shapes on FP8 handles: every output of one band and
+    # sampled outputs everywhere; repeated calls agree bit for bit
+    for N, K in ((4096, 4096), (11008, 4096), (4096, 11008)):
+        run_fp8_gemm(P, oracle_mod, N, K, M, 128, 128, 0.5, seed=N + M, fp32_mode=False, sample=4000)
+
+
+def test_gemm_fp8_split_k_repeatable_and_bounded_wait(P, oracle_mod):
+    N, K, M = 512, 1024, 8
+    w = inputs.weight(N, K, 71)
+    xc = inputs.activations(128, K, 71, None, role=0)
+    x = inputs.activations(M, K, 72, None, role=1)
+    nt = (N // 128) * (K // 128)
+    tmap = inputs.random_map(nt, nt // 2, seed=71)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pk = P.patch_pack_fp8(w.cuda(), r["meta"], r["map"])
+    y0 = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    y1 = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)  # chunks added in a fixed order
+    # failure detection: the first CTA never receives its first k-step; its
+    # bounded wait runs out and the status word reports it
+    P.test_stall_first_kstep(True)
+    try:
+        P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    finally:
+        P.test_stall_first_kstep(False)
+    assert P.patch_get_status(pk) == 5
+    assert P.patch_get_status(pk) == 0
+    y2 = P.patch_hybrid_gemm(pk, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y2)
+    pk.close()
