@@ -313,11 +313,14 @@ patch_status patch_pack_nm(const void *W_bf16, const uint32_t *meta, const uint3
  * prune first, then quantise).  The Wanda 2:4 codes and the tile map come
  * from patch_score_mask as for bf16; W_eff is then quantised to e4m3 with one
  * fp32 scale per output row, and patch_hybrid_gemm on the handle quantises X
- * with one fp32 scale per token (each call, into pool scratch of M*K + 4*M
- * bytes) and computes
+ * with one fp32 scale per token (each call: into the handle's own scratch for
+ * M <= 64, else into pool scratch of M*K + 4*M bytes) and computes
  *     Y[m,n] = sx[m] * sw[n] * sum_k dec(qx[m,k]) * dec(qw[n,k])
  * on the tensor cores (tcgen05 kind::f8f6f4: dense MMAs for dense k-steps,
- * the sparse MMA for 2:4 k-steps), fp32 accumulation, one rounding.
+ * the sparse MMA for 2:4 k-steps), fp32 accumulation, one rounding.  M <= 64
+ * with an even number of 128-column k-steps runs the split-K configuration
+ * (chunk partials added in a fixed order, scales applied at the end); the
+ * handle then also holds the chunk descriptors and partial slots.
  * Quantisation of a row: s = amax / 448 in fp32 (1 for an all-zero row);
  * q = e4m3(x / s) with the quotient in fp32, rounded to nearest with ties to
  * the even code, saturating at +-448.
