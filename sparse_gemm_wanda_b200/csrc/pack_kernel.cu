@@ -225,6 +225,9 @@ pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kPlanMaxWords = 14;  // 448 k-steps (K <= 28672) / 32
+// bands whose k-step types the planner keeps in shared memory after its first
+// pass (the later passes then read them there instead of the map again)
+constexpr int kPlanCacheBands = 512;
 
 // Bit c % 32 of word c / 32 of `bits`: k-step c of band b is 2:4.
 __device__ __forceinline__ void band_types(const uint32_t *__restrict__ map, int b, int nsteps,
@@ -267,11 +270,20 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
                  PackPlan *__restrict__ plan, int pattern) {
     __shared__ unsigned long long warp_sum[kPlanWarps];
     __shared__ uint32_t types[kPlanWarps][2][kPlanMaxWords];
+    __shared__ uint32_t tcache[kPlanCacheBands * kPlanMaxWords];
     __shared__ unsigned long long carry, n_sparse, n_meta, side_carry;
     __shared__ unsigned int duo_ok, max_pair, pmax_pair;
     const int tid = threadIdx.x, lane = tid % 32, wid = tid / 32;
     const int Q = nsteps / 2, tiles_k = (nsteps * kStep) >> log_tk;
     uint32_t *mine = types[wid][0], *next = types[wid][1];
+    const bool cached = bands <= kPlanCacheBands;
+    const int words = (nsteps + 31) / 32;
+    // band b's k-step types: the cache after pass 1, else gathered into buf
+    auto types_of = [&](int b, uint32_t *buf) -> const uint32_t * {
+        if (cached) return tcache + b * kPlanMaxWords;
+        band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, buf);
+        return buf;
+    };
     if (tid == 0) {
         carry = 0;
         n_sparse = 0;
@@ -288,6 +300,7 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
         unsigned int mp = 0;
         for (int b = wid; b < bands; b += kPlanWarps) {
             band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
+            if (cached && lane < words) tcache[b * kPlanMaxWords + lane] = mine[lane];
             int64_t *pre = pair_prefix + static_cast<int64_t>(b) * (Q + 1);
             if (lane == 0) pre[0] = 0;
             unsigned long long run = 0;
@@ -357,12 +370,12 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
     }
     // pass 3: k-step entries and decode chunk descriptors
     for (int b = wid; b < bands; b += kPlanWarps) {
-        band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
+        const uint32_t *tb = types_of(b, mine);
         const uint64_t start = band_start[b];
         const int64_t *pre = pair_prefix + static_cast<int64_t>(b) * (Q + 1);
         uint64_t *row = table + static_cast<int64_t>(b) * nsteps;
         for (int q = lane; q < Q; q += 32) {
-            const bool s0 = bit_of(mine, 2 * q), s1 = bit_of(mine, 2 * q + 1);
+            const bool s0 = bit_of(tb, 2 * q), s1 = bit_of(tb, 2 * q + 1);
             uint64_t off = start + static_cast<uint64_t>(pre[q]);
             uint64_t e0, e1;
             if (pattern == 4) {
@@ -398,7 +411,7 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
             const int np = min(cp, Q - pr0);
             uint64_t flags = 0;
             for (int i = 0; i < 2 * np; ++i)
-                if (bit_of(mine, 2 * pr0 + i)) flags |= 1ull << i;
+                if (bit_of(tb, 2 * pr0 + i)) flags |= 1ull << i;
             const uint64_t first = start + static_cast<uint64_t>(pre[pr0]);
             chunk_desc[static_cast<int64_t>(b) * cpb + q] =
                 (first & ((1ull << 40) - 1)) | (flags << 40) | (static_cast<uint64_t>(np) << 56);
@@ -415,15 +428,15 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
     for (int pb = wid; 2 * pb < bands; pb += kPlanWarps) {
         const int b = 2 * pb;
         const bool paired = b + 1 < bands && pattern == 2;
-        band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
-        if (paired) band_types(map, b + 1, nsteps, log_tn, log_tk, tiles_k, lane, next);
+        const uint32_t *tb = types_of(b, mine);
+        const uint32_t *tn1 = paired ? types_of(b + 1, next) : next;
         unsigned int n0 = 0, n1 = 0, mp = 0;
         for (int q0 = 0; q0 < Q; q0 += 32) {
             const int q = q0 + lane;
             bool d0 = false, d1 = false;
             if (q < Q) {
-                const bool s0 = bit_of(mine, 2 * q), s1 = bit_of(mine, 2 * q + 1);
-                const bool t0 = paired && bit_of(next, 2 * q), t1 = paired && bit_of(next, 2 * q + 1);
+                const bool s0 = bit_of(tb, 2 * q), s1 = bit_of(tb, 2 * q + 1);
+                const bool t0 = paired && bit_of(tn1, 2 * q), t1 = paired && bit_of(tn1, 2 * q + 1);
                 const bool mis = paired && (s0 != t0 || s1 != t1);
                 d0 = mis && (s0 || s1);
                 d1 = mis && (t0 || t1);
@@ -477,8 +490,8 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
     for (int b = wid; b < bands; b += kPlanWarps) {
         const int partner = b ^ 1;
         const bool paired = partner < bands && pattern == 2;
-        band_types(map, b, nsteps, log_tn, log_tk, tiles_k, lane, mine);
-        if (paired) band_types(map, partner, nsteps, log_tn, log_tk, tiles_k, lane, next);
+        const uint32_t *tb = types_of(b, mine);
+        const uint32_t *tp = paired ? types_of(partner, next) : next;
         const uint64_t *row = table + static_cast<int64_t>(b) * nsteps;
         uint64_t *prow = ptable + static_cast<int64_t>(b) * nsteps;
         unsigned int run = 0;
@@ -486,8 +499,8 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
             const int q = q0 + lane;
             bool d = false;
             if (q < Q) {
-                const bool s0 = bit_of(mine, 2 * q), s1 = bit_of(mine, 2 * q + 1);
-                const bool t0 = paired && bit_of(next, 2 * q), t1 = paired && bit_of(next, 2 * q + 1);
+                const bool s0 = bit_of(tb, 2 * q), s1 = bit_of(tb, 2 * q + 1);
+                const bool t0 = paired && bit_of(tp, 2 * q), t1 = paired && bit_of(tp, 2 * q + 1);
                 d = paired && (s0 != t0 || s1 != t1) && (s0 || s1);
             }
             const uint32_t ball = __ballot_sync(0xFFFFFFFFu, d);
