@@ -1,9 +1,12 @@
-// Split-K hybrid GEMV for decode (M <= 16 tokens) on the sm_100a tensor cores.
+// Split-K hybrid GEMV / skinny GEMM for decode token counts (M <= 64; token
+// tiles of 16, 32 or 64 rows) on the sm_100a tensor cores.
 //
 // Same product as the prefill kernel, Y = X * W_eff^T with dense k-steps on
 // tcgen05.mma and 2:4 k-steps on tcgen05.mma.sp ("PATCH: Learnable Tile-level
 // Hybrid Sparsity for LLMs", section 2, inference and deployment), shaped for
-// the case where the weights are read once and the run is bound by HBM.
+// the case where the weights are read once and the run is bound by HBM.  The
+// same kernel serves FP8 handles (e4m3 codes, kind::f8f6f4, scales applied by
+// the fix-up) and launches over several matrices that read one X.
 //
 // Work.  Every 128-row band of W is cut into chunks of `cp` consecutive
 // k-pairs (128 input columns each).  CTA c first runs chunks c and c + G (G

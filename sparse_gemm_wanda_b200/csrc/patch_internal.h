@@ -48,7 +48,7 @@ cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map
                         uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream,
                         int pattern = 2);
 
-// Decode (M <= 16) GEMV: CTAs whose first chunk travels in the kernel
+// Split-K decode kernel: CTAs whose first chunks travel in the kernel
 // parameters, at most.
 constexpr int kDecMaxCtas = 160;
 constexpr int kDecMaxGroup = 8;  // matrices sharing X in one split-K launch
