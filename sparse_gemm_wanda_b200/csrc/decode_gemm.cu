@@ -14,7 +14,7 @@
 // stream faster take more chunks and no CTA's static share decides the end
 // of the kernel.  A claim is made one chunk ahead, while the current chunk's
 // copies are in flight, so its round trip is off the copy path.  Each
-// chunk leaves its 16 x 128 fp32 partial in its own slot; a fix-up kernel adds
+// chunk leaves its BN x 128 fp32 partial in its own slot; a fix-up kernel adds
 // the chunks of a band in chunk order, so Y does not depend on which CTA ran
 // which chunk.  No CTA ever waits for another.
 //
@@ -24,12 +24,12 @@
 // chunks travel in the kernel parameters and the first copies start at once.
 // A pipeline stage holds two consecutive k-pairs of a chunk (a k-quad, 256
 // input columns): one bulk copy of their packed bytes (36-64 KB) and one 3-D
-// TMA load of their four X tiles (16 rows, rows past M read as zero).  Few,
+// TMA load of their four X tiles (BN rows, rows past M read as zero).  Few,
 // large copies matter: an SM's copy engine spends about as long on a small
 // copy as on a 16 KB one.
 //
 // Issue.  On B200 each tcgen05.mma costs the issuing thread about 75 cycles
-// whatever N is (N = 16 here), a metadata copy about 180 and a commit about
+// whatever N is (N = 16 measured), a metadata copy about 180 and a commit about
 // 140, while instructions from two threads overlap.  So two issuer warps
 // share the work: ring positions alternate between them, each with its own
 // accumulator per chunk (a chunk's two stages always land on different
@@ -44,7 +44,7 @@
 //
 // Roles (224 threads): warp 0 lane 0 producer, lane 0 of warps 1 and 6 MMA
 // issuers (even and odd ring positions), warps 2..5 epilogue (tcgen05.ld of
-// the 16-column accumulators, fp32 partial stores).  Two accumulator sets
+// the BN-column accumulators, fp32 partial stores).  Two accumulator sets
 // alternate between consecutive chunks.  Every mbarrier wait is bounded by
 // %globaltimer.
 #include <cuda.h>
