@@ -409,10 +409,12 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
  *   Ys      count outputs, Ys[i] [M, N_i] bf16 or fp32 (y_is_fp32), 16-byte
  *           aligned, not overlapping one another or X.
  *
- * One launch is made when every handle is bf16 2:4 (not FP8, not 4:8) and M
- * is in the split-K range (M <= 16, or M <= 64 with K <= 8192); otherwise the
- * products are enqueued one after another, as count calls of
- * patch_hybrid_gemm would.  Partial slots come from the library's
+ * One launch is made when every handle is bf16 2:4 and M is in the split-K
+ * range (M <= 16, or M <= 64 with K <= 8192), or when every handle is FP8
+ * with an even number of 128-column k-steps and M <= 64 (X is then quantised
+ * once, into the first handle's scratch); otherwise (mixed kinds, 4:8
+ * handles, larger M) the products are enqueued one after another, as count
+ * calls of patch_hybrid_gemm would.  Partial slots come from the library's
  * stream-ordered pool for the call; the first handle's claim counter serves
  * the launch, so calls that use a handle must not run concurrently on
  * different streams (the rule of patch_hybrid_gemm).  A wait that runs out

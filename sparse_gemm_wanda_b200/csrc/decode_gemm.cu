@@ -127,8 +127,8 @@ struct DecodeParams {
     uint32_t *status[kDecMaxGroup];
     const uint32_t *ready[kDecMaxGroup];
     int y_fp32;
-    const float *f8_sw;  // FP8: [N] row scales (one matrix)
-    const float *f8_sx;  // FP8: [M] token scales
+    const float *f8_sw[kDecMaxGroup];  // FP8: [N] row scales of each matrix
+    const float *f8_sx;                // FP8: [M] token scales (the shared X)
     float *partial[kDecMaxGroup];  // per matrix: [its chunks][BN][128]
     uint32_t *counter;  // chunks claimed beyond the first 2 * gridDim.x; zero between calls
     int stall_first_kstep;  // failure-detection test hook
@@ -586,7 +586,7 @@ decode_reduce_kernel(const __grid_constant__ DecodeParams p) {
             if (c0 + q < p.cpb) acc = __fadd_rn(acc, v[q]);
     }
     const int64_t n = static_cast<int64_t>(band - p.band0[mi]) * kBand + row;
-    if constexpr (F8) acc = acc * __ldg(p.f8_sw + n) * __ldg(p.f8_sx + m);
+    if constexpr (F8) acc = acc * __ldg(p.f8_sw[mi] + n) * __ldg(p.f8_sx + m);
     store_out(p, mi, static_cast<int64_t>(m) * p.N[mi] + n, acc);
 }
 
@@ -650,9 +650,9 @@ cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) 
                                         C::kSmemBytes);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    if (count < 1 || count > kDecMaxGroup || (F8 && count != 1)) return cudaErrorInvalidValue;
+    if (count < 1 || count > kDecMaxGroup) return cudaErrorInvalidValue;
     const GemmLaunch &g = gs[0];
-    if (F8 && (!g.f8_sw || !g.f8_sx)) return cudaErrorInvalidValue;
+    if (F8 && !g.f8_sx) return cudaErrorInvalidValue;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorInvalidValue;
     // X [M,K] viewed as (128-byte column blocks, M rows, K-steps): 64 bf16
@@ -681,13 +681,13 @@ cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) 
     p.cp = g.dec_cp;
     p.nmat = count;
     p.y_fp32 = g.y_fp32;
-    p.f8_sw = g.f8_sw;
     p.f8_sx = g.f8_sx;
     p.counter = g.counter;
     p.stall_first_kstep = g.stall_first_kstep;
     int64_t bands = 0;
     for (int i = 0; i < kDecMaxGroup; ++i) {
         p.packed[i] = nullptr;
+        p.f8_sw[i] = nullptr;
         p.chunk_desc[i] = nullptr;
         p.Y[i] = nullptr;
         p.N[i] = 0;
@@ -699,10 +699,12 @@ cudaError_t launch_decode(const GemmLaunch *gs, int count, cudaStream_t stream) 
         // one chunking, one X, one output type for the whole launch
         if (m.K != g.K || m.M != g.M || m.X != g.X || m.y_fp32 != g.y_fp32 || m.dec_cp != g.dec_cp ||
             m.dec_cpb != g.dec_cpb || m.N % kBand != 0 || m.dec_nchunks != (m.N / kBand) * g.dec_cpb ||
-            !m.chunk_desc || !m.chunk_desc_host || !m.packed || !m.Y || !m.status || !m.ready)
+            !m.chunk_desc || !m.chunk_desc_host || !m.packed || !m.Y || !m.status || !m.ready ||
+            (F8 && (!m.f8_sw || m.f8_sx != g.f8_sx)))
             return cudaErrorInvalidValue;
         p.band0[i] = static_cast<int32_t>(bands);
         p.packed[i] = m.packed;
+        p.f8_sw[i] = m.f8_sw;
         p.chunk_desc[i] = m.chunk_desc;
         p.Y[i] = m.Y;
         p.N[i] = m.N;
@@ -802,10 +804,12 @@ cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream) {
     return launch_decode_group(&g, 1, stream);
 }
 
-cudaError_t launch_decode_f8(const GemmLaunch &g, cudaStream_t stream) {
-    if (g.M <= 16) return launch_decode<16, true>(&g, 1, stream);
-    if (g.M <= 32) return launch_decode<32, true>(&g, 1, stream);
-    if (g.M <= kDecodeMaxM) return launch_decode<64, true>(&g, 1, stream);
+cudaError_t launch_decode_f8(const GemmLaunch *gs, int count, cudaStream_t stream) {
+    if (count < 1) return cudaErrorInvalidValue;
+    const int64_t M = gs[0].M;
+    if (M <= 16) return launch_decode<16, true>(gs, count, stream);
+    if (M <= 32) return launch_decode<32, true>(gs, count, stream);
+    if (M <= kDecodeMaxM) return launch_decode<64, true>(gs, count, stream);
     return cudaErrorInvalidValue;
 }
 

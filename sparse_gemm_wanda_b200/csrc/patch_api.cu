@@ -823,6 +823,37 @@ patch_status patch_packed_fp8_scales(const patch_packed *Wp, float *scales_dst, 
                                      cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream_v)));
 }
 
+// The split-K launch description of one FP8 handle's product on X codes xq
+// with token scales sx.
+static patchk::GemmLaunch fp8_split_launch(const patch_packed *Wp, const uint8_t *xq, const float *sx, int64_t M,
+                                           void *Y, int32_t y_is_fp32) {
+    patchk::GemmLaunch g = {};
+    g.packed = Wp->packed;
+    g.table = Wp->table;
+    g.N = Wp->shp.N;
+    g.K = Wp->shp.K;
+    g.X = xq;
+    g.M = M;
+    g.Y = Y;
+    g.y_fp32 = y_is_fp32;
+    g.workspace = Wp->workspace;
+    g.workspace_bytes = Wp->workspace_bytes;
+    g.pool = Wp->pool;
+    g.status = Wp->status;
+    g.ready = Wp->status + 2;  // raised once the pack's kernels have completed
+    g.counter = Wp->status + 3;
+    g.chunk_desc = Wp->chunk_desc;
+    g.chunk_desc_host = Wp->chunk_desc_host.data();
+    g.dec_cp = Wp->dec_cp;
+    g.dec_cpb = Wp->dec_cpb;
+    g.dec_nchunks = Wp->dec_nchunks;
+    g.num_sms = Wp->num_sms;
+    g.stall_first_kstep = g_test_stall.load(std::memory_order_relaxed);
+    g.f8_sw = Wp->fp8_scale;
+    g.f8_sx = sx;
+    return g;
+}
+
 static patch_status fp8_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
                              int32_t y_is_fp32, cudaStream_t stream) {
     const int64_t K = Wp->shp.K;
@@ -843,31 +874,8 @@ static patch_status fp8_gemm(const patch_packed *Wp, const void *X_bf16, int64_t
     if (e == cudaSuccess && M <= patchk::kDecodeMaxM && Wp->dec_nchunks > 0 && force == 0) {
         // decode token counts: the split-K kernel on the e4m3 codes, the weights
         // read once over every SM; the fix-up applies the row and token scales
-        patchk::GemmLaunch g = {};
-        g.packed = Wp->packed;
-        g.table = Wp->table;
-        g.N = Wp->shp.N;
-        g.K = K;
-        g.X = ws;
-        g.M = M;
-        g.Y = Y;
-        g.y_fp32 = y_is_fp32;
-        g.workspace = Wp->workspace;
-        g.workspace_bytes = Wp->workspace_bytes;
-        g.pool = Wp->pool;
-        g.status = Wp->status;
-        g.ready = Wp->status + 2;  // raised once the pack's kernels have completed
-        g.counter = Wp->status + 3;
-        g.chunk_desc = Wp->chunk_desc;
-        g.chunk_desc_host = Wp->chunk_desc_host.data();
-        g.dec_cp = Wp->dec_cp;
-        g.dec_cpb = Wp->dec_cpb;
-        g.dec_nchunks = Wp->dec_nchunks;
-        g.num_sms = Wp->num_sms;
-        g.stall_first_kstep = g_test_stall.load(std::memory_order_relaxed);
-        g.f8_sw = Wp->fp8_scale;
-        g.f8_sx = sx;
-        e = patchk::launch_decode_f8(g, stream);
+        const patchk::GemmLaunch g = fp8_split_launch(Wp, ws, sx, M, Y, y_is_fp32);
+        e = patchk::launch_decode_f8(&g, 1, stream);
     } else if (e == cudaSuccess) {
         patchk::Fp8Launch g;
         g.packed = Wp->packed;
@@ -956,10 +964,25 @@ patch_status patch_hybrid_gemm_group(const patch_packed *const *Wps, int32_t cou
     if (M > (int64_t(1) << 31)) return PATCH_ERR_INVALID_ARG;
     const int64_t K = Wps[0]->shp.K;
     const int force = g_test_kernel.load(std::memory_order_relaxed);
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    // FP8 handles: X is quantised once (into the first handle's scratch) and
+    // the group's products run as one split-K launch on the codes
+    bool f8_group = count > 1 && M <= kFp8ScratchRows && M <= patchk::kDecodeMaxM && force == 0;
+    for (int i = 0; i < count && f8_group; ++i)
+        f8_group = Wps[i]->pattern == 8 && Wps[i]->shp.K == K && Wps[i]->dec_nchunks > 0 &&
+                   Wps[i]->num_sms == Wps[0]->num_sms && Wps[0]->fp8_xscratch;
+    if (f8_group) {
+        uint8_t *xq = Wps[0]->fp8_xscratch;
+        float *sx = reinterpret_cast<float *>(xq + round_up(static_cast<size_t>(M * K), 256));
+        cudaError_t e = patchk::launch_fp8_quantize_rows(X_bf16, M, K, xq, sx, stream);
+        if (e != cudaSuccess) return from_cuda(e);
+        patchk::GemmLaunch gs[patchk::kDecMaxGroup];
+        for (int i = 0; i < count; ++i) gs[i] = fp8_split_launch(Wps[i], xq, sx, M, Ys[i], y_is_fp32);
+        return from_cuda(patchk::launch_decode_f8(gs, count, stream));
+    }
     bool one_launch = count > 1 && patchk::takes_split_k(M, K, force);
     for (int i = 0; i < count && one_launch; ++i)
         one_launch = Wps[i]->pattern == 2 && Wps[i]->shp.K == K && Wps[i]->num_sms == Wps[0]->num_sms;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
     if (!one_launch) {
         // the products one after another on the stream (the same results)
         for (int i = 0; i < count; ++i) {

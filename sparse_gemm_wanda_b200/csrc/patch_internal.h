@@ -186,10 +186,12 @@ cudaError_t launch_decode_gemm(const GemmLaunch &g, cudaStream_t stream);
 // handle fields and Y.  The first member's counter (and workspace, when large
 // enough) serve the launch.
 cudaError_t launch_decode_group(const GemmLaunch *gs, int count, cudaStream_t stream);
-// The same split-K kernel on an FP8 handle (one matrix): 128-column e4m3
-// k-steps taken two per "pair", kind::f8f6f4 MMAs, the fix-up applying the
-// row and token scales.  g.X is the e4m3 code matrix [M, K], M <= kDecodeMaxM.
-cudaError_t launch_decode_f8(const GemmLaunch &g, cudaStream_t stream);
+// The same split-K kernel on FP8 handles (one matrix, or a group reading the
+// same X): 128-column e4m3 k-steps taken two per "pair", kind::f8f6f4 MMAs,
+// the fix-up applying each matrix's row scales and the token scales.  X holds
+// the e4m3 code matrix [M, K] (the same for every member, as is f8_sx),
+// M <= kDecodeMaxM.
+cudaError_t launch_decode_f8(const GemmLaunch *gs, int count, cudaStream_t stream);
 // Chunking of a packed matrix for the decode GEMV: `cp` k-pairs per chunk,
 // `cpb` chunks per band.
 void plan_decode_chunks(int64_t bands, int64_t nsteps, int num_sms, int *cp, int *cpb, int *nchunks);

@@ -215,3 +215,44 @@ def test_gemm_fp8_split_k_repeatable_and_bounded_wait(P, oracle_mod):
     torch.cuda.synchronize()
     assert torch.equal(y0, y2)
     pk.close()
+
+
+@pytest.mark.parametrize("M", [1, 16, 64])
+def test_gemm_fp8_group_equals_single_calls(P, oracle_mod, M):
+    # FP8 handles that read one X: X quantised once, one split-K launch over
+    # the group; every output equals its single call bit for bit
+    K = 1024
+    pks, refs = [], []
+    x = inputs.activations(M, K, 500 + M, None, role=1)
+    for i, N in enumerate((512, 256, 384)):
+        w = inputs.weight(N, K, 510 + i)
+        xc = inputs.activations(128, K, 510 + i, None, role=0)
+        nt = (N // 128) * (K // 128)
+        tmap = inputs.random_map(nt, nt // 2, seed=520 + i)
+        r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+        pks.append(P.patch_pack_fp8(w.cuda(), r["meta"], r["map"]))
+        refs.append(oracle_fp8(oracle_mod, w, xc, tmap, 128, 128))
+    xd = x.cuda()
+    ys = P.patch_hybrid_gemm_group(pks, xd, out_fp32=True)
+    singles = [P.patch_hybrid_gemm(pk, xd, out_fp32=True) for pk in pks]
+    torch.cuda.synchronize()
+    sx = oracle_mod.fp8_row_scales(bf16_bits(x))
+    qx = oracle_mod.fp8_quantize(bf16_bits(x), sx)
+    for y, y1, (ref, sw, qw), pk in zip(ys, singles, refs, pks):
+        assert P.patch_get_status(pk) == 0
+        assert torch.equal(y, y1)
+        check(y, oracle_mod.gemm_fp8(qx, sx, qw, sw), True)
+    # a group mixing an FP8 and a bf16 handle runs as single calls
+    w = inputs.weight(256, K, 530)
+    xc = inputs.activations(128, K, 530, None, role=0)
+    tmap = inputs.random_map(16, 8, seed=530)
+    r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+    pkb = P.patch_pack(w.cuda(), r["meta"], r["map"])
+    mixed = [pks[0], pkb]
+    ym = P.patch_hybrid_gemm_group(mixed, xd, out_fp32=True)
+    ys1 = [P.patch_hybrid_gemm(pk, xd, out_fp32=True) for pk in mixed]
+    torch.cuda.synchronize()
+    for y, y1 in zip(ym, ys1):
+        assert torch.equal(y, y1)
+    for pk in pks + [pkb]:
+        pk.close()
