@@ -492,6 +492,70 @@ def nm48_isolated(P, flush, peaks):
                     "count 2MNK; L2 flushed before every call"}
 
 
+def fp8_block_gemms(P, wl, mats, calib, flush, reps=5):
+    """The block's GEMM phase on FP8 handles: the same least-loss masks and maps
+    as the bf16 step, W_eff quantised per output row (patch_pack_fp8), every
+    token count, q/k/v and gate/up as grouped calls; device time per token
+    count (median of `reps` phases, L2 flushed before each), beside the same
+    phase on the bf16 handles."""
+    units = units_of(wl, mats)
+    if wl.map_rule == "random" or not wl.calib_tokens:
+        return None
+    colsq = {g: P.patch_colsq(xc) for g, xc in calib.items()}
+    masks = [P.patch_score_mask(mats[mi]["W"], None, tile_n=wl.tile_n, tile_k=wl.tile_k, fraction=f,
+                                colsq_in=colsq[mats[mi]["group"]]) for mi, f in units]
+    out = {}
+    for kind in ("bf16", "fp8"):
+        if kind == "fp8":
+            pks = [P.patch_pack_fp8(mats[mi]["W"], r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k)
+                   for (mi, _), r in zip(units, masks)]
+        else:
+            pks = [P.patch_pack(mats[mi]["W"], r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k)
+                   for (mi, _), r in zip(units, masks)]
+        batches = []
+        for (mi, f), pk in zip(units, pks):
+            g = mats[mi]["group"]
+            if batches and batches[-1][0] == g:
+                batches[-1][1].append((mi, pk))
+            else:
+                batches.append((g, [(mi, pk)]))
+        ys = {(mi, M): torch.empty((M, mats[mi]["N"]), dtype=torch.bfloat16, device="cuda")
+              for mi, _ in units for M in wl.tokens}
+        res = {}
+        for M in sorted(wl.tokens, reverse=True):
+            def phase():
+                for _, members in batches:
+                    x = mats[members[0][0]]["X"][M]
+                    if len(members) == 1:
+                        P.patch_hybrid_gemm(members[0][1], x, out=ys[(members[0][0], M)])
+                    else:
+                        P.patch_hybrid_gemm_group([pk for _, pk in members], x,
+                                                  outs=[ys[(mi, M)] for mi, _ in members])
+            phase()
+            ts = []
+            for _ in range(reps):
+                flush()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                phase()
+                e1.record()
+                e1.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            t = statistics.median(ts)
+            fl = sum(2.0 * M * mats[mi]["N"] * mats[mi]["K"] for mi, _ in units)
+            res[f"m{M}"] = {"ms": t, "effective_tflops": fl / (t * 1e-3) / 1e12}
+        status = [P.patch_get_status(pk) for pk in pks]
+        packed = sum(pk.packed_bytes for pk in pks)
+        close_all(pks)
+        if any(status):
+            raise RuntimeError(f"GEMM status {status}")
+        out[kind] = {"by_m": res, "packed_bytes": packed}
+    return {**out, "note": "the block's GEMM phase per token count on bf16 and on FP8 (e4m3) handles "
+                           "built from the same masks and maps; FP8 calls quantise X per token "
+                           "inside the call; L2 flushed before each phase"}
+
+
 def tile_shapes_isolated(P, flush, peaks):
     """Finer tiles on the Llama-7B MLP shape at M = 2048: 128x128, 128x64,
     64x128 and 64x64 tiles at f in {0, .5, 1} (seeded random maps).  The GEMM
@@ -889,6 +953,9 @@ def main():
         extras["decode_gemm_isolated"] = decode_isolated(P, flush, peaks)
         extras["pattern_precision_isolated"] = nm48_isolated(P, flush, peaks)
         extras["tile_shapes_isolated"] = tile_shapes_isolated(P, flush, peaks)
+        fb = fp8_block_gemms(P, wl, mats, calib, flush)
+        if fb is not None:
+            extras["block_gemms_fp8_vs_bf16"] = fb
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
