@@ -60,7 +60,7 @@ __device__ __forceinline__ uint32_t kept_pair(uint32_t a, uint32_t b, uint32_t c
 // loads issued before its stores.  Where the prefill table points the k-step
 // to a dense side copy (bands of a pair that differ in type), the same CTA
 // also writes that copy: the k-step's W_eff in the dense layout.
-__global__ void __launch_bounds__(kPackThreads)
+__global__ void __launch_bounds__(kPackThreads, 8)
 pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
             const uint32_t *__restrict__ map, int64_t N, int64_t K, int tn, int tk,
             const uint64_t *__restrict__ table, const uint64_t *__restrict__ ptable,
