@@ -850,4 +850,47 @@ cudaError_t launch_hybrid_gemm(const GemmLaunch &g, cudaStream_t stream) {
     return run<160, 3>(g, 1, stream);                 // 72 KB stages
 }
 
+namespace {
+
+// The estimate launch_hybrid_gemm acts on for one bf16 2:4 matrix above 128
+// tokens: the lowest of the one-band, band-pair and two-SM estimates.
+double own_prefill_cost(const GemmLaunch &g) {
+    const PairPlan pp = plan_pair_gemm(g.N, g.M, g.num_sms);
+    const int64_t items1 = (g.N / kBand) * ((g.M + 159) / 160);
+    double cost = static_cast<double>((items1 + g.num_sms - 1) / g.num_sms) * 576.0;
+    if (g.K / kStep <= 448) cost = std::min(cost, pp.cost);
+    if (g.duo_ok && g.K / kStep <= 448) {
+        const DuoPlan dp = plan_duo_gemm(g.N, g.M, g.num_sms, g.max_pair_bytes);
+        if (dp.bn > 0) cost = std::min(cost, dp.cost);
+    }
+    return cost;
+}
+
+}  // namespace
+
+bool plan_hybrid_group(const GemmLaunch *gs, int count, DuoPlan *plan) {
+    if (count < 2 || count > kDuoGroupMax) return false;
+    const GemmLaunch &g = gs[0];
+    if (g.M <= 128 || g.K / kStep > 448) return false;
+    int64_t sum_n = 0;
+    int max_pair = 0;
+    double own = 0;
+    for (int i = 0; i < count; ++i) {
+        const GemmLaunch &m = gs[i];
+        if (m.pattern != 2 || !m.duo_ok || m.K != g.K || m.M != g.M || m.num_sms != g.num_sms ||
+            m.force_kernel != g.force_kernel || (m.N / kBand) % 2 != 0)
+            return false;
+        sum_n += m.N;
+        max_pair = std::max(max_pair, m.max_pair_bytes);
+        own += own_prefill_cost(m);
+    }
+    // test hook 3 (two-SM kernel for every M) takes the grouped launch too
+    if (g.force_kernel != 0 && g.force_kernel != 3) return false;
+    const DuoPlan dp = plan_duo_gemm(sum_n, g.M, g.num_sms, max_pair);
+    if (dp.bn == 0) return false;
+    if (g.force_kernel == 0 && dp.cost > own) return false;
+    *plan = dp;
+    return true;
+}
+
 }  // namespace patchk

@@ -980,6 +980,19 @@ patch_status patch_hybrid_gemm_group(const patch_packed *const *Wps, int32_t cou
         for (int i = 0; i < count; ++i) gs[i] = fp8_split_launch(Wps[i], xq, sx, M, Ys[i], y_is_fp32);
         return from_cuda(patchk::launch_decode_f8(gs, count, stream));
     }
+    if (count > 1 && M > 128 && !patchk::takes_split_k(M, K, force)) {
+        // prefill: one two-SM launch over every matrix's band pairs when the
+        // estimate says it finishes first (fills the SMs that one matrix's
+        // items leave idle in its last wave)
+        bool same = true;
+        for (int i = 0; i < count && same; ++i) same = Wps[i]->shp.K == K;
+        if (same) {
+            patchk::GemmLaunch gs[patchk::kDecMaxGroup];
+            for (int i = 0; i < count; ++i) gs[i] = gemm_launch(Wps[i], X_bf16, M, Ys[i], y_is_fp32);
+            patchk::DuoPlan dp;
+            if (patchk::plan_hybrid_group(gs, count, &dp)) return from_cuda(patchk::launch_duo_group(gs, count, dp, stream));
+        }
+    }
     bool one_launch = count > 1 && patchk::takes_split_k(M, K, force);
     for (int i = 0; i < count && one_launch; ++i)
         one_launch = Wps[i]->pattern == 2 && Wps[i]->shp.K == K && Wps[i]->num_sms == Wps[0]->num_sms;

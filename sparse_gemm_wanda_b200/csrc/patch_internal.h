@@ -140,6 +140,14 @@ struct DuoPlan {
 };
 DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms, int max_pair_bytes);
 cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream_t stream);
+// One launch over up to kDuoGroupMax matrices that read the same X (same K,
+// M and output type); the plan is made for the sum of their N.
+constexpr int kDuoGroupMax = 8;
+cudaError_t launch_duo_group(const GemmLaunch *gs, int count, const DuoPlan &plan, cudaStream_t stream);
+// Whether one two-SM launch over the group (bf16 2:4 handles with paired
+// band types, the same X, more than 128 tokens) is estimated to finish before
+// the matrices' own launches one after another; fills *plan when it is.
+bool plan_hybrid_group(const GemmLaunch *gs, int count, DuoPlan *plan);
 double duo_kstep_cycles(int bn);
 
 // Two-SM, four-band prefill GEMM (csrc/prefill_quad.cu): each SM of a CTA

@@ -48,6 +48,7 @@ namespace patchk {
 
 namespace {
 
+constexpr int kDuoMaxGroup = kDuoGroupMax;     // matrices sharing X in one launch
 constexpr int kDuoThreads = 352;   // warps 0 weights, 1 MMA, 6 X tiles; 2-5 and 7-10 the two epilogue groups
 constexpr int kDuoMaxStages = 8;
 constexpr int kDuoTabSteps = 448;                      // k-steps per band (K <= 28672)
@@ -58,24 +59,38 @@ constexpr int kDuoSmemLimit = 232448;
 constexpr int kDuoTailBytes = 1024 + kDuoTabBytes + 512;
 constexpr uint64_t kDuoWaitLimitNs = 2000000000ull;
 
+// One launch covers one matrix, or several that read the same X (the same K):
+// their band pairs are numbered one after another (matrix i holds global
+// pairs pair0[i] .. pair0[i+1]-1) and each keeps its own prefill table,
+// packed bytes (tensor maps), output, status and ready words.
 struct DuoParams {
-    const uint64_t *table;
-    int64_t N, K, M;
-    int nsteps, bands, ttiles, items;
+    const uint64_t *table[kDuoMaxGroup];  // prefill tables
+    int64_t N[kDuoMaxGroup];
+    void *Y[kDuoMaxGroup];
+    uint32_t *status[kDuoMaxGroup];
+    const uint32_t *ready[kDuoMaxGroup];
+    int32_t pair0[kDuoMaxGroup + 1];
+    int nmat;
+    int64_t K, M;
+    int nsteps, ttiles, items;
     int bn, half, stages, stage_bytes;
-    int aslot;  // bytes of a stage's weight slot: the largest k-pair of this matrix
-    void *Y;
+    int aslot;  // bytes of a stage's weight slot: the largest k-pair of the matrices
     int y_fp32;
-    uint32_t *status;
-    const uint32_t *ready;
     int stall_first_kstep;  // failure-detection test hook
 };
 
-__device__ __forceinline__ void store_y(const DuoParams &p, int64_t idx, float v) {
+// matrix holding global band pair gp
+__device__ __forceinline__ int duo_mat_of_pair(const DuoParams &p, int gp) {
+    int i = 0;
+    while (i + 1 < p.nmat && p.pair0[i + 1] <= gp) ++i;
+    return i;
+}
+
+__device__ __forceinline__ void store_y(const DuoParams &p, int mi, int64_t idx, float v) {
     if (p.y_fp32)
-        static_cast<float *>(p.Y)[idx] = v;
+        static_cast<float *>(p.Y[mi])[idx] = v;
     else
-        static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
+        static_cast<__nv_bfloat16 *>(p.Y[mi])[idx] = __float2bfloat16_rn(v);
 }
 
 // Tensor maps over the packed buffer viewed as rows of 2 KB (256 x 8-byte
@@ -83,7 +98,8 @@ __device__ __forceinline__ void store_y(const DuoParams &p, int64_t idx, float v
 // (one dense + metadata + one 2:4) or 9 (metadata + two 2:4).  X is viewed
 // as (64 columns, M rows, K/64 k-steps) with a box of both k-steps of a pair.
 struct DuoMaps {
-    CUtensorMap x, a_dd, a_mixed, a_ss;
+    CUtensorMap x;
+    CUtensorMap a_dd[kDuoMaxGroup], a_mixed[kDuoMaxGroup], a_ss[kDuoMaxGroup];
 };
 
 __global__ void __launch_bounds__(kDuoThreads, 1)
@@ -113,23 +129,26 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
     const int bn = p.bn, half = p.half;
 
     auto fetch_table = [&](int item, int buf) {
-        const int band = 2 * (item / p.ttiles) + static_cast<int>(rank);
+        const int gp = item / p.ttiles, mi = duo_mat_of_pair(p, gp);
+        const int band = 2 * (gp - p.pair0[mi]) + static_cast<int>(rank);
         const uint32_t nb = static_cast<uint32_t>(p.nsteps) * 8u;
         mbar_arrive_expect_tx(&tab_full[buf], nb);
-        bulk_g2s(tab_buf + buf * kDuoTabSteps, p.table + static_cast<int64_t>(band) * p.nsteps, nb,
+        bulk_g2s(tab_buf + buf * kDuoTabSteps, p.table[mi] + static_cast<int64_t>(band) * p.nsteps, nb,
                  &tab_full[buf]);
     };
     auto give_up = [&]() {
         *abort_flag = 1u;
         st_cluster_u32(map_to_rank(const_cast<uint32_t *>(abort_flag), rank ^ 1u), 1u);
-        atomicOr(p.status, kStatusTimeout);
+        for (int i = 0; i < p.nmat; ++i) atomicOr(p.status[i], kStatusTimeout);
     };
 
     if (threadIdx.x == 0) {
         pdl_trigger();
         // weights are final once the packer's ready flag is seen; otherwise
         // (the packer may be the kernel just before) wait first
-        if (ld_acquire_gpu(p.ready) == 0u) pdl_wait();
+        bool all_ready = true;
+        for (int i = 0; i < p.nmat; ++i) all_ready = all_ready && ld_acquire_gpu(p.ready[i]) != 0u;
+        if (!all_ready) pdl_wait();
         for (int s = 0; s < kDuoMaxStages; ++s) {
             mbar_init(&full[s], 2);  // the leader's weight and X producers
             mbar_init(&empty[s], 1);
@@ -140,7 +159,10 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
             mbar_init(&tab_full[b], 1);
         }
         *never_flag = 0u;
-        *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
+        // a matrix whose status is raised skips the whole launch
+        uint32_t raised = 0u;
+        for (int i = 0; i < p.nmat; ++i) raised |= *reinterpret_cast<volatile uint32_t *>(p.status[i]);
+        *abort_flag = (raised & kStatusTimeout) ? 1u : 0u;
         fence_mbar_init_cluster();
     }
     if (warp == 1) {
@@ -149,9 +171,11 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&maps.x);
-        prefetch_tmap(&maps.a_dd);
-        prefetch_tmap(&maps.a_mixed);
-        prefetch_tmap(&maps.a_ss);
+        for (int i = 0; i < p.nmat; ++i) {
+            prefetch_tmap(&maps.a_dd[i]);
+            prefetch_tmap(&maps.a_mixed[i]);
+            prefetch_tmap(&maps.a_ss[i]);
+        }
     }
     __syncwarp();
     tc_fence_before();
@@ -184,6 +208,7 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
                     break;
                 }
                 const uint64_t *tab = tab_buf + buf * kDuoTabSteps;
+                const int mi = duo_mat_of_pair(p, item / p.ttiles);  // the item's matrix
                 for (int pr = 0; pr < p.nsteps / 2; ++pr) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
@@ -205,9 +230,9 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
                     // the two bands of a pair agree in kind and metadata placement,
                     // so the leader arms the barrier for both CTAs' weight bytes
                     if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * a_bytes);
-                    const CUtensorMap *am = a_bytes == 2u * kDenseStepBytes ? &maps.a_dd
-                                          : (a_bytes == 2u * kSparseStepBytes + kMetaBlockBytes ? &maps.a_ss
-                                                                                               : &maps.a_mixed);
+                    const CUtensorMap *am = a_bytes == 2u * kDenseStepBytes ? &maps.a_dd[mi]
+                                          : (a_bytes == 2u * kSparseStepBytes + kMetaBlockBytes ? &maps.a_ss[mi]
+                                                                                               : &maps.a_mixed[mi]);
                     tma2d_pair(smem + s * p.stage_bytes, am, 0, static_cast<int32_t>(first / 2048),
                                map_to_rank(&full[s], 0));
                 }
@@ -338,7 +363,9 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
         for (int i = 0;; ++i) {
             const int item = cl + i * C;
             if (item >= p.items) break;
-            const int bp = item / p.ttiles, tt = item % p.ttiles;
+            const int gp = item / p.ttiles, tt = item % p.ttiles;
+            const int mi = duo_mat_of_pair(p, gp);
+            const int bp = gp - p.pair0[mi];
             const int buf = i & 1;
             const bool ok = mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1u, never_flag, kDuoWaitLimitNs);
             tc_fence_after();
@@ -355,11 +382,12 @@ duo_gemm_kernel(const __grid_constant__ DuoMaps maps, const __grid_constant__ Du
                     uint32_t r[16];
                     tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(buf * bn + c0), r);
                     tmem_ld_wait();
-                    int64_t idx = (m_base + c0) * p.N + n;
+                    const int64_t ld = p.N[mi];
+                    int64_t idx = (m_base + c0) * ld + n;
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
-                        if (c0 + q < m_valid) store_y(p, idx, __uint_as_float(r[q]));
-                        idx += p.N;
+                        if (c0 + q < m_valid) store_y(p, mi, idx, __uint_as_float(r[q]));
+                        idx += ld;
                     }
                 }
             }
@@ -473,6 +501,7 @@ DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms, int max_pair_bytes) {
     for (int bn = 240; bn >= 128; bn -= 16) {
         const int64_t tt = (M + bn - 1) / bn;
         const int64_t items = bpairs * tt;
+        if (items > INT32_MAX) continue;  // items are counted in 32 bits
         const int64_t waves = (items + clusters - 1) / clusters;
         const double cost = static_cast<double>(waves) * duo_kstep_cycles(bn);
         if (best.bn == 0 || cost < best_cost) {
@@ -491,11 +520,13 @@ DuoPlan plan_duo_gemm(int64_t N, int64_t M, int num_sms, int max_pair_bytes) {
     return best;
 }
 
-cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream_t stream) {
+cudaError_t launch_duo_group(const GemmLaunch *gs, int count, const DuoPlan &plan, cudaStream_t stream) {
     const cudaError_t attr_err = ensure_duo_attributes();
     if (attr_err != cudaSuccess) return attr_err;
+    if (count < 1 || count > kDuoMaxGroup) return cudaErrorInvalidValue;
     if (plan.stages < 2 || plan.smem > kDuoSmemLimit || plan.clusters < 1) return cudaErrorInvalidValue;
-    if ((g.N / kBand) % 2 != 0 || g.K / kStep > kDuoTabSteps || !g.packed_rows) return cudaErrorInvalidValue;
+    const GemmLaunch &g = gs[0];
+    if (g.K / kStep > kDuoTabSteps) return cudaErrorInvalidValue;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorInvalidValue;
     DuoMaps maps;
@@ -510,30 +541,52 @@ cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const uint64_t rows = g.packed_rows / 16;  // 2 KB rows
-    if (!encode_rows(enc, &maps.a_dd, g.packed, rows, 2 * kDenseStepBytes / 2048) ||
-        !encode_rows(enc, &maps.a_mixed, g.packed, rows,
-                     (kDenseStepBytes + kMetaBlockBytes + kSparseStepBytes) / 2048) ||
-        !encode_rows(enc, &maps.a_ss, g.packed, rows, (kMetaBlockBytes + 2 * kSparseStepBytes) / 2048))
-        return cudaErrorInvalidValue;
     DuoParams p;
-    p.table = g.ptable;  // the prefill table: the bands of every pair agree in type
-    p.N = g.N;
+    int64_t pairs = 0;
+    for (int i = 0; i < count; ++i) {
+        const GemmLaunch &m = gs[i];
+        // one X, one K, one output type; every matrix pairs its bands
+        if (m.K != g.K || m.M != g.M || m.X != g.X || m.y_fp32 != g.y_fp32 || (m.N / kBand) % 2 != 0 ||
+            !m.packed_rows || !m.ptable || !m.Y || !m.status || !m.ready)
+            return cudaErrorInvalidValue;
+        const uint64_t rows = m.packed_rows / 16;  // 2 KB rows
+        if (!encode_rows(enc, &maps.a_dd[i], m.packed, rows, 2 * kDenseStepBytes / 2048) ||
+            !encode_rows(enc, &maps.a_mixed[i], m.packed, rows,
+                         (kDenseStepBytes + kMetaBlockBytes + kSparseStepBytes) / 2048) ||
+            !encode_rows(enc, &maps.a_ss[i], m.packed, rows, (kMetaBlockBytes + 2 * kSparseStepBytes) / 2048))
+            return cudaErrorInvalidValue;
+        p.table[i] = m.ptable;  // the prefill table: the bands of every pair agree in type
+        p.N[i] = m.N;
+        p.Y[i] = m.Y;
+        p.status[i] = m.status;
+        p.ready[i] = m.ready;
+        p.pair0[i] = static_cast<int32_t>(pairs);
+        pairs += m.N / (2 * kBand);
+    }
+    for (int i = count; i < kDuoMaxGroup; ++i) {
+        maps.a_dd[i] = maps.a_dd[0];
+        maps.a_mixed[i] = maps.a_mixed[0];
+        maps.a_ss[i] = maps.a_ss[0];
+        p.table[i] = nullptr;
+        p.N[i] = 0;
+        p.Y[i] = nullptr;
+        p.status[i] = nullptr;
+        p.ready[i] = nullptr;
+    }
+    for (int i = count; i <= kDuoMaxGroup; ++i) p.pair0[i] = static_cast<int32_t>(pairs);
+    p.nmat = count;
     p.K = g.K;
     p.M = g.M;
     p.nsteps = static_cast<int>(g.K / kStep);
-    p.bands = static_cast<int>(g.N / kBand);
     p.ttiles = plan.ttiles;
     p.items = plan.items;
+    if (static_cast<int64_t>(p.items) != pairs * plan.ttiles) return cudaErrorInvalidValue;
     p.bn = plan.bn;
     p.half = plan.bn / 2;
     p.stages = plan.stages;
     p.stage_bytes = plan.stage_bytes;
     p.aslot = plan.aslot;
-    p.Y = g.Y;
     p.y_fp32 = g.y_fp32;
-    p.status = g.status;
-    p.ready = g.ready;
     p.stall_first_kstep = g.stall_first_kstep;
 
     cudaLaunchConfig_t cfg = {};
@@ -553,6 +606,10 @@ cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream
     cudaError_t err = cudaLaunchKernelEx(&cfg, duo_gemm_kernel, maps, p);
     if (err == cudaSuccess) note_launches(1);
     return err;
+}
+
+cudaError_t launch_duo_gemm(const GemmLaunch &g, const DuoPlan &plan, cudaStream_t stream) {
+    return launch_duo_group(&g, 1, plan, stream);
 }
 
 }  // namespace patchk

@@ -432,6 +432,60 @@ def test_gemm_group_block_shapes(P, oracle_mod, M):
             pk.close()
 
 
+@pytest.mark.parametrize("M", [200, 700, 1300])
+@pytest.mark.parametrize("forced", [False, True])
+def test_gemm_group_prefill_one_launch(P, oracle_mod, M, forced):
+    # above 128 tokens a group of handles whose band pairs agree in type runs
+    # as one two-SM launch over all their band pairs (test hook 3 takes it at
+    # every size; otherwise the estimate decides); each output against the
+    # oracle, every element
+    K = 1152
+    pks, weffs = group_problem(P, oracle_mod, [512, 768, 256], K, seed=230 + M)
+    x = inputs.activations(M, K, 330 + M, None)
+    xd = x.cuda()
+    if forced:
+        with forced_kernel(P, 3):
+            ys = P.patch_hybrid_gemm_group(pks, xd, out_fp32=True)
+            ys16 = P.patch_hybrid_gemm_group(pks, xd, out_fp32=False)
+            ys2 = P.patch_hybrid_gemm_group(pks, xd, out_fp32=True)
+    else:
+        ys = P.patch_hybrid_gemm_group(pks, xd, out_fp32=True)
+        ys16 = P.patch_hybrid_gemm_group(pks, xd, out_fp32=False)
+        ys2 = P.patch_hybrid_gemm_group(pks, xd, out_fp32=True)
+    torch.cuda.synchronize()
+    for y, y16, yb, weff, pk in zip(ys, ys16, ys2, weffs, pks):
+        assert P.patch_get_status(pk) == 0
+        assert torch.equal(y, yb)  # repeatable
+        yref = oracle_mod.gemm(bf16_bits(x), weff)
+        rel_rms_check(y, yref, True)
+        rel_rms_check(y16, yref, False)
+    for pk in pks:
+        pk.close()
+
+
+@pytest.mark.parametrize("M", [512, 4096])
+def test_gemm_group_prefill_block_shapes(P, oracle_mod, M):
+    # q/k/v and gate/up of the Llama-7B block at prefill token counts, each
+    # group through the grouped entry point; sampled outputs (every band
+    # pair's edge rows included) against the oracle
+    K = 4096
+    for shapes, seed in (([4096, 4096, 4096], 510), ([11008, 11008], 520)):
+        pks, weffs = group_problem(P, oracle_mod, shapes, K, seed=seed + M, frac=0.6)
+        x = inputs.activations(M, K, seed + M, inputs.outlier_channels(K, seed))
+        ys = P.patch_hybrid_gemm_group(pks, x.cuda(), out_fp32=True)
+        torch.cuda.synchronize()
+        g = np.random.default_rng(seed + M)
+        for y, weff, pk in zip(ys, weffs, pks):
+            assert P.patch_get_status(pk) == 0
+            N = pk.N
+            ms = np.concatenate([g.integers(0, M, 2000), np.array([0, M - 1, M // 2, 0, M - 1, 0])])
+            ns = np.concatenate([g.integers(0, N, 2000), np.array([0, N - 1, 255, N - 256, 0, 128])])
+            yref = oracle_mod.gemm_at(bf16_bits(x), weff, ms, ns)
+            rel_rms_check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, True)
+        for pk in pks:
+            pk.close()
+
+
 def test_gemm_group_falls_back_to_single_calls(P, oracle_mod):
     # handles that cannot share a launch (a 4:8 handle; M above the split-K
     # range) are run one after another with the same results
@@ -468,6 +522,30 @@ def test_gemm_group_bounded_wait_raises_every_status(P, oracle_mod):
     for pk in pks:
         assert P.patch_get_status(pk) == 5  # PATCH_ERR_TIMEOUT, read and cleared
     ys = P.patch_hybrid_gemm_group(pks, x.cuda(), out_fp32=True)
+    torch.cuda.synchronize()
+    for y, weff, pk in zip(ys, weffs, pks):
+        assert P.patch_get_status(pk) == 0
+        rel_rms_check(y, oracle_mod.gemm(bf16_bits(x), weff), True)
+    for pk in pks:
+        pk.close()
+
+
+def test_gemm_group_prefill_bounded_wait_raises_every_status(P, oracle_mod):
+    # the grouped two-SM launch: a k-pair that never lands ends the launch
+    # through its bounded waits and raises every member's status word
+    K, M = 512, 300
+    pks, weffs = group_problem(P, oracle_mod, [256, 512], K, seed=93)
+    x = inputs.activations(M, K, 94, None)
+    P.test_stall_first_kstep(True)
+    try:
+        with forced_kernel(P, 3):
+            P.patch_hybrid_gemm_group(pks, x.cuda(), out_fp32=True)
+    finally:
+        P.test_stall_first_kstep(False)
+    for pk in pks:
+        assert P.patch_get_status(pk) == 5  # PATCH_ERR_TIMEOUT, read and cleared
+    with forced_kernel(P, 3):
+        ys = P.patch_hybrid_gemm_group(pks, x.cuda(), out_fp32=True)
     torch.cuda.synchronize()
     for y, weff, pk in zip(ys, weffs, pks):
         assert P.patch_get_status(pk) == 0
