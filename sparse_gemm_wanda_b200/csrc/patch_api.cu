@@ -854,6 +854,30 @@ static patchk::GemmLaunch fp8_split_launch(const patch_packed *Wp, const uint8_t
     return g;
 }
 
+// the launch description of one FP8 handle's product on quantised X
+static patchk::Fp8Launch fp8_launch(const patch_packed *Wp, const uint8_t *xq, const float *sx, int64_t M,
+                                    void *Y, int32_t y_is_fp32) {
+    patchk::Fp8Launch g;
+    g.packed = Wp->packed;
+    g.table = Wp->table;
+    g.ptable = Wp->ptable;
+    g.packed_bytes = Wp->packed_bytes + Wp->side_bytes;
+    g.all_sparse = Wp->sparse_ksteps == Wp->bands * (Wp->shp.K / 128) ? 1 : 0;
+    g.force_kernel = g_test_kernel.load(std::memory_order_relaxed);
+    g.sw = Wp->fp8_scale;
+    g.xq = xq;
+    g.sx = sx;
+    g.N = Wp->shp.N;
+    g.K = Wp->shp.K;
+    g.M = M;
+    g.Y = Y;
+    g.y_fp32 = y_is_fp32;
+    g.status = Wp->status;
+    g.num_sms = Wp->num_sms;
+    g.pool = Wp->pool;
+    return g;
+}
+
 static patch_status fp8_gemm(const patch_packed *Wp, const void *X_bf16, int64_t M, void *Y,
                              int32_t y_is_fp32, cudaStream_t stream) {
     const int64_t K = Wp->shp.K;
@@ -877,25 +901,7 @@ static patch_status fp8_gemm(const patch_packed *Wp, const void *X_bf16, int64_t
         const patchk::GemmLaunch g = fp8_split_launch(Wp, ws, sx, M, Y, y_is_fp32);
         e = patchk::launch_decode_f8(&g, 1, stream);
     } else if (e == cudaSuccess) {
-        patchk::Fp8Launch g;
-        g.packed = Wp->packed;
-        g.table = Wp->table;
-        g.ptable = Wp->ptable;
-        g.packed_bytes = Wp->packed_bytes + Wp->side_bytes;
-        g.all_sparse = Wp->sparse_ksteps == Wp->bands * (Wp->shp.K / 128) ? 1 : 0;
-        g.force_kernel = g_test_kernel.load(std::memory_order_relaxed);
-        g.sw = Wp->fp8_scale;
-        g.xq = ws;
-        g.sx = sx;
-        g.N = Wp->shp.N;
-        g.K = K;
-        g.M = M;
-        g.Y = Y;
-        g.y_fp32 = y_is_fp32;
-        g.status = Wp->status;
-        g.num_sms = Wp->num_sms;
-        g.pool = Wp->pool;
-        e = patchk::launch_fp8_gemm(g, stream);
+        e = patchk::launch_fp8_gemm(fp8_launch(Wp, ws, sx, M, Y, y_is_fp32), stream);
     }
     const cudaError_t e2 = own ? cudaSuccess : cudaFreeAsync(ws, stream);
     return from_cuda(e != cudaSuccess ? e : e2);
@@ -979,6 +985,46 @@ patch_status patch_hybrid_gemm_group(const patch_packed *const *Wps, int32_t cou
         patchk::GemmLaunch gs[patchk::kDecMaxGroup];
         for (int i = 0; i < count; ++i) gs[i] = fp8_split_launch(Wps[i], xq, sx, M, Ys[i], y_is_fp32);
         return from_cuda(patchk::launch_decode_f8(gs, count, stream));
+    }
+    if (count > 1 && M > 128 && (force == 0 || force == 3)) {
+        // FP8 prefill: X quantised once, then one two-SM launch over every
+        // matrix's band pairs when the estimate says it finishes first
+        const int64_t steps = K / 128;
+        bool ok = steps % 2 == 0 && steps <= 224;
+        bool all_sparse = true;
+        int64_t sum_n = 0;
+        double own = 0;
+        for (int i = 0; i < count && ok; ++i) {
+            const patch_packed *h = Wps[i];
+            ok = h->pattern == 8 && h->shp.K == K && h->ptable && (h->shp.N / 128) % 2 == 0 &&
+                 h->num_sms == Wps[0]->num_sms;
+            if (!ok) break;
+            const bool sp = h->sparse_ksteps == h->bands * steps;
+            all_sparse = all_sparse && sp;
+            sum_n += h->shp.N;
+            const patchk::DuoFp8Plan one = patchk::plan_duo_fp8(h->shp.N, M, h->num_sms, sp);
+            ok = one.bn > 0;
+            own += one.cost;
+        }
+        patchk::DuoFp8Plan dp{};
+        if (ok) dp = patchk::plan_duo_fp8(sum_n, M, Wps[0]->num_sms, all_sparse);
+        if (ok && dp.bn > 0 && (force == 3 || dp.cost <= own)) {
+            const size_t off_sx = round_up(static_cast<size_t>(M * K), 256);
+            uint8_t *ws = nullptr;
+            cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&ws),
+                                                    off_sx + sizeof(float) * static_cast<size_t>(M),
+                                                    Wps[0]->pool, stream);
+            if (e != cudaSuccess) return from_cuda(e);
+            float *sx = reinterpret_cast<float *>(ws + off_sx);
+            e = patchk::launch_fp8_quantize_rows(X_bf16, M, K, ws, sx, stream);
+            if (e == cudaSuccess) {
+                patchk::Fp8Launch gs[patchk::kDecMaxGroup];
+                for (int i = 0; i < count; ++i) gs[i] = fp8_launch(Wps[i], ws, sx, M, Ys[i], y_is_fp32);
+                e = patchk::launch_duo_fp8_group(gs, count, dp, stream);
+            }
+            const cudaError_t e2 = cudaFreeAsync(ws, stream);
+            return from_cuda(e != cudaSuccess ? e : e2);
+        }
     }
     if (count > 1 && M > 128 && !patchk::takes_split_k(M, K, force)) {
         // prefill: one two-SM launch over every matrix's band pairs when the

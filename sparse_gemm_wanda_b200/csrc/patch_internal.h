@@ -249,9 +249,14 @@ struct DuoFp8Plan {
     int stages, stage_bytes, smem;
     int aslot;        // weight slot of a stage (two k-steps)
     int aslot_step;   // its half for one k-step
+    double cost;      // waves x estimated cycles per k-step of an item
 };
 DuoFp8Plan plan_duo_fp8(int64_t N, int64_t M, int num_sms, bool all_sparse);
 cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStream_t stream);
+// One launch over up to kDuoGroupMax FP8 matrices that read the same X codes
+// and scales (same K, M and output type); the plan is made for the sum of
+// their N, with all_sparse only if every matrix is.
+cudaError_t launch_duo_fp8_group(const Fp8Launch *gs, int count, const DuoFp8Plan &plan, cudaStream_t stream);
 
 // The library's stream-ordered memory pool for the current device (cached
 // memory is kept, not returned to the system between calls).

@@ -58,22 +58,41 @@ constexpr int kD8SmemLimit = 232448;
 constexpr int kD8TailBytes = 1024 + kD8TabBytes + 512;
 constexpr uint64_t kD8WaitLimitNs = 2000000000ull;
 
+constexpr int kD8MaxGroup = kDuoGroupMax;  // matrices sharing X in one launch
+
+// One launch covers one matrix, or several that read the same X codes (the
+// same K): their band pairs are numbered one after another (matrix i holds
+// global pairs pair0[i] .. pair0[i+1]-1) and each keeps its own prefill
+// table, packed bytes (tensor maps), row scales, output and status word.
 struct D8Params {
-    const uint64_t *table;   // prefill table [bands][steps]
-    const float *sw, *sx;
-    int64_t N, K, M;
+    const uint64_t *table[kD8MaxGroup];  // prefill tables [bands][steps]
+    const float *sw[kD8MaxGroup];
+    int64_t N[kD8MaxGroup];
+    void *Y[kD8MaxGroup];
+    uint32_t *status[kD8MaxGroup];
+    int32_t pair0[kD8MaxGroup + 1];
+    int nmat;
+    const float *sx;
+    int64_t K, M;
     int steps, ttiles, items;
     int bn, half, stages, stage_bytes, aslot;
     int aslot_step;          // weight bytes reserved per k-step in a stage (aslot = 2 x this)
-    void *Y;
     int y_fp32;
-    uint32_t *status;
 };
 
-// Tensor maps over the packed buffer as rows of 2 KB: one k-step (8 rows
+// matrix holding global band pair gp
+__device__ __forceinline__ int d8_mat_of_pair(const D8Params &p, int gp) {
+    int i = 0;
+    while (i + 1 < p.nmat && p.pair0[i + 1] <= gp) ++i;
+    return i;
+}
+
+// Tensor maps over each packed buffer as rows of 2 KB: one k-step (8 rows
 // dense, 5 rows 2:4) or two contiguous k-steps (16, 13 or 10 rows).
 struct D8Maps {
-    CUtensorMap x, a_dense, a_sparse, a_dd, a_mixed, a_ss;
+    CUtensorMap x;
+    CUtensorMap a_dense[kD8MaxGroup], a_sparse[kD8MaxGroup], a_dd[kD8MaxGroup], a_mixed[kD8MaxGroup],
+        a_ss[kD8MaxGroup];
 };
 
 // one k-step's MMAs back to back: four dense K32, or two 2:4 K64 with the
@@ -112,11 +131,11 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_pair(int n, bool sparse) {
            (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
-__device__ __forceinline__ void store_y(const D8Params &p, int64_t idx, float v) {
+__device__ __forceinline__ void store_y(const D8Params &p, int mi, int64_t idx, float v) {
     if (p.y_fp32)
-        static_cast<float *>(p.Y)[idx] = v;
+        static_cast<float *>(p.Y[mi])[idx] = v;
     else
-        static_cast<__nv_bfloat16 *>(p.Y)[idx] = __float2bfloat16_rn(v);
+        static_cast<__nv_bfloat16 *>(p.Y[mi])[idx] = __float2bfloat16_rn(v);
 }
 
 __global__ void __launch_bounds__(kD8Threads, 1)
@@ -144,15 +163,17 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
     const int bn = p.bn, half = p.half;
 
     auto fetch_table = [&](int item, int buf) {
-        const int band = 2 * (item / p.ttiles) + static_cast<int>(rank);
+        const int gp = item / p.ttiles, mi = d8_mat_of_pair(p, gp);
+        const int band = 2 * (gp - p.pair0[mi]) + static_cast<int>(rank);
         const uint32_t nb = static_cast<uint32_t>(p.steps) * 8u;
         mbar_arrive_expect_tx(&tab_full[buf], nb);
-        bulk_g2s(tab_buf + buf * kD8TabSteps, p.table + static_cast<int64_t>(band) * p.steps, nb, &tab_full[buf]);
+        bulk_g2s(tab_buf + buf * kD8TabSteps, p.table[mi] + static_cast<int64_t>(band) * p.steps, nb,
+                 &tab_full[buf]);
     };
     auto give_up = [&]() {
         *abort_flag = 1u;
         st_cluster_u32(map_to_rank(const_cast<uint32_t *>(abort_flag), rank ^ 1u), 1u);
-        atomicOr(p.status, kStatusTimeout);
+        for (int i = 0; i < p.nmat; ++i) atomicOr(p.status[i], kStatusTimeout);
     };
 
     if (threadIdx.x == 0) {
@@ -166,7 +187,10 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
             mbar_init(&tab_full[b], 1);
         }
         *never_flag = 0u;
-        *abort_flag = (*reinterpret_cast<volatile uint32_t *>(p.status) & kStatusTimeout) ? 1u : 0u;
+        // a matrix whose status is raised skips the whole launch
+        uint32_t raised = 0u;
+        for (int i = 0; i < p.nmat; ++i) raised |= *reinterpret_cast<volatile uint32_t *>(p.status[i]);
+        *abort_flag = (raised & kStatusTimeout) ? 1u : 0u;
         fence_mbar_init_cluster();
     }
     if (warp == 1) {
@@ -175,11 +199,13 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
     }
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&maps.x);
-        prefetch_tmap(&maps.a_dense);
-        prefetch_tmap(&maps.a_sparse);
-        prefetch_tmap(&maps.a_dd);
-        prefetch_tmap(&maps.a_mixed);
-        prefetch_tmap(&maps.a_ss);
+        for (int i = 0; i < p.nmat; ++i) {
+            prefetch_tmap(&maps.a_dense[i]);
+            prefetch_tmap(&maps.a_sparse[i]);
+            prefetch_tmap(&maps.a_dd[i]);
+            prefetch_tmap(&maps.a_mixed[i]);
+            prefetch_tmap(&maps.a_ss[i]);
+        }
     }
     __syncwarp();
     tc_fence_before();
@@ -208,6 +234,7 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
                     break;
                 }
                 const uint64_t *tab = tab_buf + buf * kD8TabSteps;
+                const int mi = d8_mat_of_pair(p, item / p.ttiles);  // the item's matrix
                 for (int pr = 0; pr < pairs; ++pr) {
                     const int s = it % S;
                     const uint32_t ph = (it / S) & 1u;
@@ -231,13 +258,14 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
                     uint8_t *st = smem + s * p.stage_bytes;
                     if (f1 == f0 + b0) {
                         // contiguous: one copy of both k-steps
-                        const CUtensorMap *am = (sp0 && sp1) ? &maps.a_ss : ((sp0 || sp1) ? &maps.a_mixed : &maps.a_dd);
+                        const CUtensorMap *am = (sp0 && sp1) ? &maps.a_ss[mi]
+                                              : ((sp0 || sp1) ? &maps.a_mixed[mi] : &maps.a_dd[mi]);
                         tma2d_pair(st, am, 0, static_cast<int32_t>(f0 / 2048), map_to_rank(&full[s], 0));
                     } else {
-                        tma2d_pair(st, sp0 ? &maps.a_sparse : &maps.a_dense, 0, static_cast<int32_t>(f0 / 2048),
-                                   map_to_rank(&full[s], 0));
-                        tma2d_pair(st + b0, sp1 ? &maps.a_sparse : &maps.a_dense, 0, static_cast<int32_t>(f1 / 2048),
-                                   map_to_rank(&full[s], 0));
+                        tma2d_pair(st, sp0 ? &maps.a_sparse[mi] : &maps.a_dense[mi], 0,
+                                   static_cast<int32_t>(f0 / 2048), map_to_rank(&full[s], 0));
+                        tma2d_pair(st + b0, sp1 ? &maps.a_sparse[mi] : &maps.a_dense[mi], 0,
+                                   static_cast<int32_t>(f1 / 2048), map_to_rank(&full[s], 0));
                     }
                 }
                 if (ok && cl + (i + 2) * C < p.items) {
@@ -362,7 +390,9 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
         for (int i = 0;; ++i) {
             const int item = cl + i * C;
             if (item >= p.items) break;
-            const int bp = item / p.ttiles, tt = item % p.ttiles;
+            const int gp = item / p.ttiles, tt = item % p.ttiles;
+            const int mi = d8_mat_of_pair(p, gp);
+            const int bp = gp - p.pair0[mi];
             const int buf = i & 1;
             const bool ok = mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1u, never_flag, kD8WaitLimitNs);
             tc_fence_after();
@@ -373,7 +403,8 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
             const int64_t n = static_cast<int64_t>(2 * bp + static_cast<int>(rank)) * kBand + row;
             const int64_t m_base = static_cast<int64_t>(tt) * bn;
             const int m_valid = static_cast<int>(min(static_cast<int64_t>(bn), p.M - m_base));
-            const float swn = __ldg(p.sw + n);
+            const float swn = __ldg(p.sw[mi] + n);
+            const int64_t ld = p.N[mi];
             if (*abort_flag == 0) {
 #pragma unroll 1
                 for (int c0 = 16 * grp; c0 < m_valid; c0 += 32) {
@@ -383,12 +414,12 @@ duo_fp8_kernel(const __grid_constant__ D8Maps maps, const __grid_constant__ D8Pa
                     const int ml = c0 + (lane & 15);
                     const float sxl = ml < m_valid ? __ldg(p.sx + m_base + ml) : 0.0f;
                     tmem_ld_wait();
-                    int64_t idx = (m_base + c0) * p.N + n;
+                    int64_t idx = (m_base + c0) * ld + n;
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         const float sq = __shfl_sync(0xFFFFFFFFu, sxl, q);
-                        if (c0 + q < m_valid) store_y(p, idx, __uint_as_float(r[q]) * swn * sq);
-                        idx += p.N;
+                        if (c0 + q < m_valid) store_y(p, mi, idx, __uint_as_float(r[q]) * swn * sq);
+                        idx += ld;
                     }
                 }
             }
@@ -498,6 +529,7 @@ DuoFp8Plan plan_duo_fp8(int64_t N, int64_t M, int num_sms, bool all_sparse) {
     for (int bn = 240; bn >= 128; bn -= 16) {
         const int64_t tt = (M + bn - 1) / bn;
         const int64_t items = bpairs * tt;
+        if (items > INT32_MAX) continue;  // items are counted in 32 bits
         const int64_t waves = (items + clusters - 1) / clusters;
         const double kstep = std::max(2.0 * bn, 2.0 * (aslot + 64.0 * bn) / 128.0);
         const double cost = static_cast<double>(waves) * kstep;
@@ -512,17 +544,19 @@ DuoFp8Plan plan_duo_fp8(int64_t N, int64_t M, int num_sms, bool all_sparse) {
     best.smem = smem_for(best.bn, &best.stages, &best.stage_bytes);
     best.aslot = aslot;
     best.aslot_step = aslot_step;
+    best.cost = best_cost;
     return best;
 }
 
-cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStream_t stream) {
+cudaError_t launch_duo_fp8_group(const Fp8Launch *gs, int count, const DuoFp8Plan &plan, cudaStream_t stream) {
     const cudaError_t attr_err = ensure_attributes();
     if (attr_err != cudaSuccess) return attr_err;
+    if (count < 1 || count > kD8MaxGroup) return cudaErrorInvalidValue;
+    const Fp8Launch &g = gs[0];
     const int64_t steps = g.K / kD8Step;
     if (plan.bn < 128 || plan.stages < 2 || plan.smem > kD8SmemLimit || plan.clusters < 1)
         return cudaErrorInvalidValue;
-    if ((g.N / kBand) % 2 != 0 || steps % 2 != 0 || steps > kD8TabSteps || !g.ptable || !g.packed_bytes)
-        return cudaErrorInvalidValue;
+    if (steps % 2 != 0 || steps > kD8TabSteps) return cudaErrorInvalidValue;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorInvalidValue;
     D8Maps maps;
@@ -538,19 +572,48 @@ cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStrea
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const uint64_t rows = g.packed_bytes / 2048;  // packed + side copies, in 2 KB rows
     constexpr uint32_t kRowsD = kDenseStepBytes / 2048, kRowsS = (kMetaBlockBytes + kSparseStepBytes) / 2048;
-    if (!encode_rows(enc, &maps.a_dense, g.packed, rows, kRowsD) ||
-        !encode_rows(enc, &maps.a_sparse, g.packed, rows, kRowsS) ||
-        !encode_rows(enc, &maps.a_dd, g.packed, rows, 2 * kRowsD) ||
-        !encode_rows(enc, &maps.a_mixed, g.packed, rows, kRowsD + kRowsS) ||
-        !encode_rows(enc, &maps.a_ss, g.packed, rows, 2 * kRowsS))
-        return cudaErrorInvalidValue;
     D8Params p;
-    p.table = g.ptable;
-    p.sw = g.sw;
+    int64_t pairs = 0;
+    for (int i = 0; i < count; ++i) {
+        const Fp8Launch &m = gs[i];
+        // one X (codes and scales), one K, one output type; every matrix pairs its bands
+        if (m.K != g.K || m.M != g.M || m.xq != g.xq || m.sx != g.sx || m.y_fp32 != g.y_fp32 ||
+            (m.N / kBand) % 2 != 0 || !m.ptable || !m.packed_bytes || !m.sw || !m.Y || !m.status)
+            return cudaErrorInvalidValue;
+        // a matrix without dense k-steps only fits a plan sized for that
+        if (!m.all_sparse && plan.aslot_step != kDenseStepBytes) return cudaErrorInvalidValue;
+        const uint64_t rows = m.packed_bytes / 2048;  // packed + side copies, in 2 KB rows
+        if (!encode_rows(enc, &maps.a_dense[i], m.packed, rows, kRowsD) ||
+            !encode_rows(enc, &maps.a_sparse[i], m.packed, rows, kRowsS) ||
+            !encode_rows(enc, &maps.a_dd[i], m.packed, rows, 2 * kRowsD) ||
+            !encode_rows(enc, &maps.a_mixed[i], m.packed, rows, kRowsD + kRowsS) ||
+            !encode_rows(enc, &maps.a_ss[i], m.packed, rows, 2 * kRowsS))
+            return cudaErrorInvalidValue;
+        p.table[i] = m.ptable;
+        p.sw[i] = m.sw;
+        p.N[i] = m.N;
+        p.Y[i] = m.Y;
+        p.status[i] = m.status;
+        p.pair0[i] = static_cast<int32_t>(pairs);
+        pairs += m.N / (2 * kBand);
+    }
+    for (int i = count; i < kD8MaxGroup; ++i) {
+        maps.a_dense[i] = maps.a_dense[0];
+        maps.a_sparse[i] = maps.a_sparse[0];
+        maps.a_dd[i] = maps.a_dd[0];
+        maps.a_mixed[i] = maps.a_mixed[0];
+        maps.a_ss[i] = maps.a_ss[0];
+        p.table[i] = nullptr;
+        p.sw[i] = nullptr;
+        p.N[i] = 0;
+        p.Y[i] = nullptr;
+        p.status[i] = nullptr;
+    }
+    for (int i = count; i <= kD8MaxGroup; ++i) p.pair0[i] = static_cast<int32_t>(pairs);
+    if (static_cast<int64_t>(plan.items) != pairs * plan.ttiles) return cudaErrorInvalidValue;
+    p.nmat = count;
     p.sx = g.sx;
-    p.N = g.N;
     p.K = g.K;
     p.M = g.M;
     p.steps = static_cast<int>(steps);
@@ -562,9 +625,7 @@ cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStrea
     p.stage_bytes = plan.stage_bytes;
     p.aslot = plan.aslot;
     p.aslot_step = plan.aslot_step;
-    p.Y = g.Y;
     p.y_fp32 = g.y_fp32;
-    p.status = g.status;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(2 * plan.clusters));
@@ -581,6 +642,10 @@ cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStrea
     cudaError_t err = cudaLaunchKernelEx(&cfg, duo_fp8_kernel, maps, p);
     if (err == cudaSuccess) note_launches(1);
     return err;
+}
+
+cudaError_t launch_duo_fp8(const Fp8Launch &g, const DuoFp8Plan &plan, cudaStream_t stream) {
+    return launch_duo_fp8_group(&g, 1, plan, stream);
 }
 
 }  // namespace patchk

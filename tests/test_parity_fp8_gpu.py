@@ -256,3 +256,77 @@ def test_gemm_fp8_group_equals_single_calls(P, oracle_mod, M):
         assert torch.equal(y, y1)
     for pk in pks + [pkb]:
         pk.close()
+
+
+def fp8_group_problem(P, oracle_mod, shapes, K, fracs, seed):
+    """FP8 handles for matrices [N_i, K] that share one input, random maps."""
+    pks, refs = [], []
+    for i, (N, frac) in enumerate(zip(shapes, fracs)):
+        w = inputs.weight(N, K, seed + i)
+        xc = inputs.activations(128, K, seed + i, None, role=0)
+        nt = (N // 128) * (K // 128)
+        tmap = inputs.random_map(nt, int(round(frac * nt)), seed=seed + 50 + i)
+        r = P.patch_score_mask(w.cuda(), xc.cuda(), map_in=tmap.cuda())
+        pks.append(P.patch_pack_fp8(w.cuda(), r["meta"], r["map"]))
+        ref = oracle_fp8(oracle_mod, w, xc, tmap, 128, 128)
+        assert np.array_equal(r["meta"].cpu().numpy().view(np.uint32), ref[0]["meta"])
+        refs.append(ref)
+    return pks, refs
+
+
+@pytest.mark.parametrize("M", [200, 700])
+@pytest.mark.parametrize("fracs", [(0.5, 1.0, 0.25), (1.0, 1.0, 1.0)])
+@pytest.mark.parametrize("forced", [False, True])
+def test_gemm_fp8_group_prefill_one_launch(P, oracle_mod, M, fracs, forced):
+    # above 128 tokens FP8 handles that read one X: X quantised once and,
+    # when the estimate takes it (always under test hook 3), one two-SM
+    # launch over every matrix's band pairs; every element against the oracle
+    # (a group whose matrices are all 2:4 gets the smaller weight slot)
+    K = 1024
+    pks, refs = fp8_group_problem(P, oracle_mod, (512, 768, 256), K, fracs, seed=600 + M)
+    x = inputs.activations(M, K, 640 + M, None, role=1)
+    xd = x.cuda()
+    if forced:
+        with forced_kernel(P, 3):
+            ys = P.patch_hybrid_gemm_group(pks, xd, out_fp32=True)
+            ys16 = P.patch_hybrid_gemm_group(pks, xd, out_fp32=False)
+            ys2 = P.patch_hybrid_gemm_group(pks, xd, out_fp32=True)
+    else:
+        ys = P.patch_hybrid_gemm_group(pks, xd, out_fp32=True)
+        ys16 = P.patch_hybrid_gemm_group(pks, xd, out_fp32=False)
+        ys2 = P.patch_hybrid_gemm_group(pks, xd, out_fp32=True)
+    torch.cuda.synchronize()
+    sx = oracle_mod.fp8_row_scales(bf16_bits(x))
+    qx = oracle_mod.fp8_quantize(bf16_bits(x), sx)
+    for y, y16, yb, (ref, sw, qw), pk in zip(ys, ys16, ys2, refs, pks):
+        assert P.patch_get_status(pk) == 0
+        assert torch.equal(y, yb)  # repeatable
+        yref = oracle_mod.gemm_fp8(qx, sx, qw, sw)
+        check(y, yref, True)
+        check(y16, yref, False)
+    for pk in pks:
+        pk.close()
+
+
+def test_gemm_fp8_group_prefill_block_shapes(P, oracle_mod):
+    # q/k/v and gate/up of the Llama-7B block on FP8 handles at M = 512
+    # through the grouped entry point; sampled outputs (edge rows of the
+    # first and last band pair included) against the oracle
+    K, M = 4096, 512
+    for shapes, seed in (((4096, 4096, 4096), 700), ((11008, 11008), 710)):
+        pks, refs = fp8_group_problem(P, oracle_mod, shapes, K, (0.6,) * len(shapes), seed=seed)
+        x = inputs.activations(M, K, seed + 5, inputs.outlier_channels(K, seed), role=1)
+        ys = P.patch_hybrid_gemm_group(pks, x.cuda(), out_fp32=True)
+        torch.cuda.synchronize()
+        sx = oracle_mod.fp8_row_scales(bf16_bits(x))
+        qx = oracle_mod.fp8_quantize(bf16_bits(x), sx)
+        g = np.random.default_rng(seed)
+        for y, (ref, sw, qw), pk in zip(ys, refs, pks):
+            assert P.patch_get_status(pk) == 0
+            N = pk.N
+            ms = np.concatenate([g.integers(0, M, 2000), np.array([0, M - 1, M // 2, 0, M - 1, 0])])
+            ns = np.concatenate([g.integers(0, N, 2000), np.array([0, N - 1, 255, N - 256, 0, 128])])
+            yref = oracle_mod.gemm_fp8_at(qx, sx, qw, sw, ms, ns)
+            check(y[torch.from_numpy(ms).cuda(), torch.from_numpy(ns).cuda()], yref, True)
+        for pk in pks:
+            pk.close()
