@@ -413,11 +413,13 @@ patch_status patch_hybrid_gemm(const patch_packed *Wp, const void *X_bf16, int64
  * range (M <= 16, or M <= 64 with K <= 8192), or when every handle is FP8
  * with an even number of 128-column k-steps and M <= 64 (X is then quantised
  * once, into the first handle's scratch), or, above 128 tokens, when every
- * handle is bf16 2:4 with an even band count and K <= 28672 and the library
- * estimates one two-SM launch over all their band pairs to finish no later
- * than their own launches; otherwise (mixed kinds, 4:8 handles, 64 < M <=
- * 128) the products are enqueued one after another, as count calls of
- * patch_hybrid_gemm would.  In the split-K launches each output is
+ * handle is bf16 2:4 with an even band count and K <= 28672, or every handle
+ * is FP8 with an even band count and an even number of 128-column k-steps
+ * (at most 224; X quantised once, into a pool allocation of M*K + 4*M bytes
+ * freed on the stream), and the library estimates one two-SM launch over all
+ * their band pairs to finish no later than their own launches; otherwise
+ * (mixed kinds, 4:8 handles, 64 < M <= 128) the products are enqueued one
+ * after another, as count calls of patch_hybrid_gemm would.  In the split-K launches each output is
  * bit-identical to its single call; the grouped prefill launch may tile the
  * tokens differently from a single call, which changes fp32 rounding order
  * only.  Partial slots come from the library's
