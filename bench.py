@@ -781,6 +781,8 @@ def main():
     ap.add_argument("--frac", type=float, default=0.5)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--fp8", action="store_true", help="--case gemm: FP8 (e4m3) values in the tiles")
+    ap.add_argument("--group", type=int, default=1,
+                    help="--case gemm: this many [N, K] matrices reading one X, one grouped call")
     ap.add_argument("--force-kernel", type=int, default=0,
                     help="--case gemm: prefill kernel (library test hook; 0 = the library's choice)")
     args = ap.parse_args()
@@ -1024,16 +1026,25 @@ def run_case(args):
             for _ in range(args.reps):
                 P.patch_pack(W, r["meta"], r["map"]).close()
         else:
-            pk = (P.patch_pack_fp8(W, r["meta"], r["map"]) if args.fp8
-                  else P.patch_pack(W, r["meta"], r["map"]))
+            pack = P.patch_pack_fp8 if args.fp8 else P.patch_pack
+            pks = [pack(W, r["meta"], r["map"])]
+            for i in range(1, args.group):
+                Wi = (torch.randn(args.N, args.K, generator=g) * 0.02).to(torch.bfloat16).cuda()
+                ri = P.patch_score_mask(Wi, Xcal, map_in=inputs.random_map(nt, int(round(args.frac * nt)), 7 + i).cuda())
+                pks.append(pack(Wi, ri["meta"], ri["map"]))
             P.test_prefill_kernel(args.force_kernel)
             for _ in range(args.reps):
-                P.patch_hybrid_gemm(pk, X)
+                if args.group > 1:
+                    P.patch_hybrid_gemm_group(pks, X)
+                else:
+                    P.patch_hybrid_gemm(pks[0], X)
             torch.cuda.synchronize()
-            assert P.patch_get_status(pk) == 0
-            pk.close()
+            for pk in pks:
+                assert P.patch_get_status(pk) == 0
+                pk.close()
     torch.cuda.synchronize()
-    print(f"case {args.case} N={args.N} K={args.K} M={args.M} frac={args.frac}{' fp8' if args.fp8 else ''} ok")
+    print(f"case {args.case} N={args.N} K={args.K} M={args.M} frac={args.frac}{' fp8' if args.fp8 else ''}"
+          f"{f' group={args.group}' if args.group > 1 else ''} ok")
 
 
 def main_reference(args, wl, world, rank):
