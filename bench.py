@@ -272,8 +272,12 @@ def run_step(P, wl, mats, calib, maps, ys, ev: StepEvents | None = None, colsq_c
                                    map_in=maps[(mi, f)])
         masks.append(r)
     mark("pack")
-    pks = [P.patch_pack(mats[mi]["W"], r["meta"], r["map"], tile_n=wl.tile_n, tile_k=wl.tile_k)
-           for (mi, _), r in zip(units, masks)]
+    # up to eight matrices per call: one host wait for each call's layouts
+    pks = []
+    for b in range(0, len(units), 8):
+        chunk = list(zip(units[b:b + 8], masks[b:b + 8]))
+        pks += P.patch_pack_group([mats[mi]["W"] for (mi, _), _ in chunk], [r["meta"] for _, r in chunk],
+                                  [r["map"] for _, r in chunk], tile_n=wl.tile_n, tile_k=wl.tile_k)
     # matrices that read the same X (one unit per matrix) share one call
     batches = []
     for (mi, f), pk in zip(units, pks):

@@ -289,6 +289,25 @@ patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t
                         void *stream);
 
 /*
+ * patch_pack for several matrices with ONE wait (no counterpart on the pages:
+ * the compressor above, batched).  Matrix i is (Ws_bf16[i], metas[i],
+ * maps[i], shps[i]), each under patch_pack's preconditions; shapes may
+ * differ.  Every layout is planned in one launch (a block per matrix), the
+ * plan summaries and k-pair prefixes are read back in one wait of `stream`,
+ * then every packed buffer is allocated and packed.  Each outs[i] is then
+ * exactly the handle patch_pack would give for matrix i (the same packed
+ * bytes and tables).
+ *   count         1..8.
+ *   outs          count handle slots (host array); all null on any error.
+ *   packed_bytes  optional host array of count: compressed bytes per handle.
+ * Errors: as patch_pack, for any member (every member's arguments are
+ * checked before anything is allocated); on an error no handle is left.
+ */
+patch_status patch_pack_group(const void *const *Ws_bf16, const uint32_t *const *metas,
+                              const uint32_t *const *maps, const patch_shape *shps, int32_t count,
+                              patch_packed **outs, size_t *packed_bytes, void *stream);
+
+/*
  * Compressor for another N:M pattern (see patch_score_mask_nm).  (2, 4) is
  * exactly patch_pack.  (4, 8): the 4:8 handle's packed format (normative):
  *   - bands of 128 rows, k-steps of 64 columns; a k-step is 4:8-compressed

@@ -262,12 +262,31 @@ __device__ __forceinline__ uint32_t kpair_bytes(bool s0, bool s1, int pattern = 
            (s1 ? (s0 ? 0 : kMetaBlockBytes) + kSparseStepBytes : kDenseStepBytes);
 }
 
-__global__ void __launch_bounds__(kPlanThreads, 1)
-plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int log_tn, int log_tk, int cp,
-                 int cpb, uint64_t *__restrict__ table, uint64_t *__restrict__ chunk_desc,
-                 int64_t *__restrict__ pair_prefix, uint64_t *__restrict__ band_start,
-                 uint64_t *__restrict__ ptable, uint64_t *__restrict__ side_start,
-                 PackPlan *__restrict__ plan, int pattern) {
+// The plans of up to kPlanMaxGroup matrices, one block each.
+struct PlanGroup {
+    const uint32_t *map[kPlanMaxGroup];
+    int bands[kPlanMaxGroup], nsteps[kPlanMaxGroup], log_tn[kPlanMaxGroup], log_tk[kPlanMaxGroup];
+    int cp[kPlanMaxGroup], cpb[kPlanMaxGroup];
+    uint64_t *table[kPlanMaxGroup], *chunk_desc[kPlanMaxGroup];
+    int64_t *pair_prefix[kPlanMaxGroup];
+    uint64_t *band_start[kPlanMaxGroup], *ptable[kPlanMaxGroup], *side_start[kPlanMaxGroup];
+    PackPlan *plan[kPlanMaxGroup];
+    int pattern[kPlanMaxGroup];
+};
+
+__global__ void __launch_bounds__(kPlanThreads, 1) plan_pack_kernel(const __grid_constant__ PlanGroup grp) {
+    // this block's matrix
+    const int gi = blockIdx.x;
+    const uint32_t *__restrict__ map = grp.map[gi];
+    const int bands = grp.bands[gi], nsteps = grp.nsteps[gi], log_tn = grp.log_tn[gi], log_tk = grp.log_tk[gi];
+    const int cp = grp.cp[gi], cpb = grp.cpb[gi], pattern = grp.pattern[gi];
+    uint64_t *__restrict__ table = grp.table[gi];
+    uint64_t *__restrict__ chunk_desc = grp.chunk_desc[gi];
+    int64_t *__restrict__ pair_prefix = grp.pair_prefix[gi];
+    uint64_t *__restrict__ band_start = grp.band_start[gi];
+    uint64_t *__restrict__ ptable = grp.ptable[gi];
+    uint64_t *__restrict__ side_start = grp.side_start[gi];
+    PackPlan *__restrict__ plan = grp.plan[gi];
     __shared__ unsigned long long warp_sum[kPlanWarps];
     __shared__ uint32_t types[kPlanWarps][2][kPlanMaxWords];
     __shared__ uint32_t tcache[kPlanCacheBands * kPlanMaxWords];
@@ -535,20 +554,42 @@ plan_pack_kernel(const uint32_t *__restrict__ map, int bands, int nsteps, int lo
     }
 }
 
+cudaError_t launch_plan_pack_group(const PlanArgs *args, int count, cudaStream_t stream) {
+    if (count < 1 || count > kPlanMaxGroup) return cudaErrorInvalidValue;
+    PlanGroup grp{};
+    for (int i = 0; i < count; ++i) {
+        const PlanArgs &a = args[i];
+        const int64_t nsteps = a.K / kStep;
+        if (nsteps > 32 * kPlanMaxWords || (a.N / kBand) > (int64_t(1) << 24)) return cudaErrorInvalidValue;
+        if (a.pattern != 2 && a.pattern != 4) return cudaErrorInvalidValue;
+        grp.map[i] = a.map;
+        grp.bands[i] = static_cast<int>(a.N / kBand);
+        grp.nsteps[i] = static_cast<int>(nsteps);
+        grp.log_tn[i] = a.tn == 64 ? 6 : 7;
+        grp.log_tk[i] = a.tk == 64 ? 6 : 7;
+        grp.cp[i] = a.cp;
+        grp.cpb[i] = a.cpb;
+        grp.table[i] = a.table;
+        grp.chunk_desc[i] = a.chunk_desc;
+        grp.pair_prefix[i] = a.pair_prefix;
+        grp.band_start[i] = a.band_start;
+        grp.ptable[i] = a.ptable;
+        grp.side_start[i] = a.side_start;
+        grp.plan[i] = a.plan;
+        grp.pattern[i] = a.pattern;
+    }
+    plan_pack_kernel<<<count, kPlanThreads, 0, stream>>>(grp);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, int tk, int cp,
                              int cpb, uint64_t *table, uint64_t *chunk_desc, int64_t *pair_prefix,
                              uint64_t *band_start, uint64_t *ptable, uint64_t *side_start,
                              PackPlan *plan, cudaStream_t stream, int pattern) {
-    const int64_t nsteps = K / kStep;
-    if (nsteps > 32 * kPlanMaxWords || (N / kBand) > (int64_t(1) << 24)) return cudaErrorInvalidValue;
-    if (pattern != 2 && pattern != 4) return cudaErrorInvalidValue;
-    const int log_tn = tn == 64 ? 6 : 7, log_tk = tk == 64 ? 6 : 7;
-    plan_pack_kernel<<<1, kPlanThreads, 0, stream>>>(map, static_cast<int>(N / kBand), static_cast<int>(nsteps),
-                                                     log_tn, log_tk, cp, cpb, table, chunk_desc,
-                                                     pair_prefix, band_start, ptable, side_start, plan,
-                                                     pattern);
-    note_launches(1);
-    return cudaGetLastError();
+    const PlanArgs a{map, N, K, tn, tk, cp, cpb, table, chunk_desc, pair_prefix, band_start, ptable, side_start,
+                     plan, pattern};
+    return launch_plan_pack_group(&a, 1, stream);
 }
 
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,

@@ -96,33 +96,38 @@ patch_status check_device(int *num_sms) {
     return PATCH_OK;
 }
 
-// The plan summary written by plan_pack_kernel, read back into page-locked
-// memory (one buffer per device, held under the lock until the copy landed),
-// and the per-band k-pair prefix the prefill kernels balance their work with
-// (into `prefix`, pageable: that copy returns once it has landed).  The
-// stream is waited for once, here; no later call on the handle waits.
-cudaError_t read_plan(const patchk::PackPlan *src, patchk::PackPlan *dst, const int64_t *prefix_src,
-                      std::vector<int64_t> *prefix, cudaStream_t stream) {
+// The plan summaries written by plan_pack_kernel, read back into page-locked
+// memory (one buffer of kPlanMaxGroup plans per device, held under the lock
+// until the copies landed), and each matrix's per-band k-pair prefix the
+// prefill kernels balance their work with (into `prefix[i]`, pageable: that
+// copy returns once it has landed).  The stream is waited for once, here; no
+// later call on the handles waits.
+cudaError_t read_plans(const patchk::PackPlan *const *src, patchk::PackPlan *dst, const int64_t *const *prefix_src,
+                       std::vector<int64_t> *const *prefix, int count, cudaStream_t stream) {
     static std::mutex mu;
     static std::map<int, patchk::PackPlan *> bufs;
+    if (count < 1 || count > patchk::kPlanMaxGroup) return cudaErrorInvalidValue;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
     patchk::PackPlan *&buf = bufs[dev];
     if (!buf) {
-        e = cudaMallocHost(reinterpret_cast<void **>(&buf), sizeof(patchk::PackPlan));
+        e = cudaMallocHost(reinterpret_cast<void **>(&buf), sizeof(patchk::PackPlan) * patchk::kPlanMaxGroup);
         if (e != cudaSuccess) {
             buf = nullptr;
             return e;
         }
     }
-    e = cudaMemcpyAsync(buf, src, sizeof(patchk::PackPlan), cudaMemcpyDeviceToHost, stream);
-    if (e == cudaSuccess && !prefix->empty())
-        e = cudaMemcpyAsync(prefix->data(), prefix_src, sizeof(int64_t) * prefix->size(),
-                            cudaMemcpyDeviceToHost, stream);
+    for (int i = 0; i < count && e == cudaSuccess; ++i) {
+        e = cudaMemcpyAsync(buf + i, src[i], sizeof(patchk::PackPlan), cudaMemcpyDeviceToHost, stream);
+        if (e == cudaSuccess && !prefix[i]->empty())
+            e = cudaMemcpyAsync(prefix[i]->data(), prefix_src[i], sizeof(int64_t) * prefix[i]->size(),
+                                cudaMemcpyDeviceToHost, stream);
+    }
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-    if (e == cudaSuccess) *dst = *buf;
+    if (e == cudaSuccess)
+        for (int i = 0; i < count; ++i) dst[i] = buf[i];
     return e;
 }
 
@@ -530,110 +535,142 @@ void patch_test_prefill_kernel(int32_t which) {
     g_test_kernel.store((which >= 0 && which <= 4) ? which : 0, std::memory_order_relaxed);
 }
 
+// Up to kPlanMaxGroup matrices packed with one wait: every handle is made and
+// its plan launched (one plan launch for all), the plans are read back in one
+// wait, then every packed buffer is allocated and packed.  On an error no
+// handle is left: those made so far are freed and every out[i] is null.
+static patch_status pack_group_impl(const void *const *Ws, const uint32_t *const *metas,
+                                    const uint32_t *const *maps, const patch_shape *shps, int count,
+                                    patch_packed **outs, size_t *packed_bytes, void *stream_v, int pattern) {
+    if (!outs || count < 1 || count > patchk::kPlanMaxGroup) return PATCH_ERR_INVALID_ARG;
+    for (int i = 0; i < count; ++i) outs[i] = nullptr;
+    if (!Ws || !metas || !maps || !shps) return PATCH_ERR_INVALID_ARG;
+    // every argument is checked before anything is allocated
+    for (int i = 0; i < count; ++i) {
+        const patch_status st = check_shape(shps[i]);
+        if (st != PATCH_OK) return st;
+        if (shps[i].N % kBand != 0 || shps[i].K % (2 * kStep) != 0) return PATCH_ERR_INVALID_ARG;
+        if (shps[i].K > 28672) return PATCH_ERR_INVALID_ARG;  // one segment's table must fit on chip
+        if (!Ws[i] || !metas[i] || !maps[i] || !aligned16(Ws[i])) return PATCH_ERR_INVALID_ARG;
+    }
+    int num_sms = 0;
+    patch_status st = check_device(&num_sms);
+    if (st != PATCH_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+
+    patch_packed *hs[patchk::kPlanMaxGroup] = {};
+    patchk::PlanArgs pa[patchk::kPlanMaxGroup];
+    const patchk::PackPlan *plan_dev[patchk::kPlanMaxGroup];
+    const int64_t *prefix_dev[patchk::kPlanMaxGroup];
+    std::vector<int64_t> *prefix_host[patchk::kPlanMaxGroup];
+    auto fail = [&](patch_status why) {
+        for (int i = 0; i < count; ++i)
+            if (hs[i]) patch_free(hs[i], stream_v);
+        return why;
+    };
+    for (int i = 0; i < count; ++i) {
+        const patch_shape shp = shps[i];
+        const int64_t N = shp.N, K = shp.K;
+        const int64_t bands = N / kBand, nsteps = K / kStep, Q = nsteps / 2;
+        patch_packed *h = new (std::nothrow) patch_packed();
+        if (!h) return fail(PATCH_ERR_OOM);
+        hs[i] = h;
+        cudaGetDevice(&h->device);
+        h->pattern = pattern;
+        h->shp = shp;
+        h->num_sms = num_sms;
+        h->bands = bands;
+        patchk::plan_decode_chunks(bands, nsteps, num_sms, &h->dec_cp, &h->dec_cpb, &h->dec_nchunks);
+        h->workspace_bytes = patchk::decode_workspace_bytes(h->dec_nchunks);
+
+        // The layout is planned on the device from the map (no map read-back,
+        // no table upload); only the plan summary comes back, to size the
+        // packed buffer.  Allocation 1: table | chunk descriptors | k-pair
+        // prefix | band starts | plan | workspace | status.  Allocation 2: the
+        // packed bytes.
+        const size_t off_table = 0;
+        const size_t off_chunks = off_table + sizeof(uint64_t) * static_cast<size_t>(bands * nsteps);
+        const size_t off_prefix = round_up(off_chunks + sizeof(uint64_t) * static_cast<size_t>(h->dec_nchunks), 256);
+        const size_t off_bstart = round_up(off_prefix + sizeof(int64_t) * static_cast<size_t>(bands * (Q + 1)), 256);
+        const size_t off_ptable = round_up(off_bstart + sizeof(uint64_t) * static_cast<size_t>(bands), 256);
+        const size_t off_sstart = round_up(off_ptable + sizeof(uint64_t) * static_cast<size_t>(bands * nsteps), 256);
+        const size_t off_plan = round_up(off_sstart + sizeof(uint64_t) * static_cast<size_t>(bands), 256);
+        const size_t off_ws = round_up(off_plan + sizeof(patchk::PackPlan), 256);
+        const size_t off_status = round_up(off_ws + h->workspace_bytes, 256);
+        const size_t status_bytes = 256;
+        const size_t total = off_status + status_bytes;
+        cudaError_t e = patchk::device_pool(&h->pool);
+        if (e == cudaSuccess)
+            e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->base), total, h->pool, stream);
+        if (e != cudaSuccess) return fail(from_cuda(e));
+        h->table = reinterpret_cast<uint64_t *>(h->base + off_table);
+        h->chunk_desc = reinterpret_cast<uint64_t *>(h->base + off_chunks);
+        h->pair_prefix_dev = reinterpret_cast<int64_t *>(h->base + off_prefix);
+        h->ptable = reinterpret_cast<uint64_t *>(h->base + off_ptable);
+        patchk::PackPlan *pd = reinterpret_cast<patchk::PackPlan *>(h->base + off_plan);
+        h->workspace = reinterpret_cast<float *>(h->base + off_ws);
+        // status word | pack completion counter | ready flag | decode chunk counter
+        h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
+        e = cudaMemsetAsync(h->status, 0, status_bytes, stream);
+        if (e != cudaSuccess) return fail(from_cuda(e));
+        pa[i] = patchk::PlanArgs{maps[i], N, K, static_cast<int>(shp.tile_n), static_cast<int>(shp.tile_k),
+                                 h->dec_cp, h->dec_cpb, h->table, h->chunk_desc, h->pair_prefix_dev,
+                                 reinterpret_cast<uint64_t *>(h->base + off_bstart), h->ptable,
+                                 reinterpret_cast<uint64_t *>(h->base + off_sstart), pd, pattern};
+        plan_dev[i] = pd;
+        prefix_dev[i] = h->pair_prefix_dev;
+        h->pair_prefix.assign(static_cast<size_t>(bands * (Q + 1)), 0);
+        prefix_host[i] = &h->pair_prefix;
+    }
+    cudaError_t e = patchk::launch_plan_pack_group(pa, count, stream);
+    preload_gemm_kernels();  // this call waits for the device below in any case
+    patchk::PackPlan plans[patchk::kPlanMaxGroup];
+    if (e == cudaSuccess) e = read_plans(plan_dev, plans, prefix_dev, prefix_host, count, stream);
+    if (e != cudaSuccess) return fail(from_cuda(e));
+    for (int i = 0; i < count; ++i) {
+        patch_packed *h = hs[i];
+        const patchk::PackPlan &plan = plans[i];
+        h->packed_bytes = static_cast<size_t>(plan.packed_bytes);
+        h->side_bytes = static_cast<size_t>(plan.side_bytes);
+        if (plan.packed_bytes >= (1ull << 40) || plan.packed_bytes + plan.side_bytes >= (1ull << 47))
+            return fail(PATCH_ERR_UNSUPPORTED);  // chunk descriptors hold 40-bit offsets, table entries 48-bit ones
+        h->sparse_ksteps = static_cast<int64_t>(plan.sparse_ksteps);
+        h->meta_blocks = static_cast<int64_t>(plan.meta_blocks);
+        h->duo_ok = plan.duo_ok ? 1 : 0;
+        h->max_pair_bytes = static_cast<int>(plan.pair_max_bytes);
+        h->chunk_desc_host.assign(plan.first_desc,
+                                  plan.first_desc + std::min<int64_t>(h->dec_nchunks, 2 * patchk::kDecMaxCtas));
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->packed),
+                                    std::max<size_t>(h->packed_bytes + h->side_bytes, 16), h->pool, stream);
+        if (e == cudaSuccess)
+            e = patchk::launch_pack(Ws[i], metas[i], maps[i], h->shp.N, h->shp.K, static_cast<int>(h->shp.tile_n),
+                                    static_cast<int>(h->shp.tile_k), h->table, h->side_bytes ? h->ptable : nullptr,
+                                    h->packed, h->status + 1, h->status + 2, stream, pattern);
+        if (e != cudaSuccess) return fail(from_cuda(e));
+    }
+    for (int i = 0; i < count; ++i) {
+        if (packed_bytes) packed_bytes[i] = hs[i]->packed_bytes;
+        outs[i] = hs[i];
+    }
+    return PATCH_OK;
+}
+
 static patch_status pack_impl(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
                               patch_shape shp, patch_packed **out, size_t *packed_bytes,
                               void *stream_v, int pattern) {
     if (!out) return PATCH_ERR_INVALID_ARG;
-    *out = nullptr;
-    patch_status st = check_shape(shp);
-    if (st != PATCH_OK) return st;
-    if (shp.N % kBand != 0 || shp.K % (2 * kStep) != 0) return PATCH_ERR_INVALID_ARG;
-    if (shp.K > 28672) return PATCH_ERR_INVALID_ARG;  // one segment's table must fit on chip
-    if (!W_bf16 || !meta || !map || !aligned16(W_bf16)) return PATCH_ERR_INVALID_ARG;
-    int num_sms = 0;
-    st = check_device(&num_sms);
-    if (st != PATCH_OK) return st;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
-
-    const int64_t N = shp.N, K = shp.K, tn = shp.tile_n, tk = shp.tile_k;
-    const int64_t bands = N / kBand, nsteps = K / kStep, Q = nsteps / 2;
-
-    patch_packed *h = new (std::nothrow) patch_packed();
-    if (!h) return PATCH_ERR_OOM;
-    cudaGetDevice(&h->device);
-    h->pattern = pattern;
-    h->shp = shp;
-    h->num_sms = num_sms;
-    h->bands = bands;
-    patchk::plan_decode_chunks(bands, nsteps, num_sms, &h->dec_cp, &h->dec_cpb, &h->dec_nchunks);
-    h->workspace_bytes = patchk::decode_workspace_bytes(h->dec_nchunks);
-
-    // The layout is planned on the device from the map (no map read-back, no
-    // table upload); only the plan summary comes back, to size the packed
-    // buffer.  Allocation 1: table | chunk descriptors | k-pair prefix | band
-    // starts | plan | workspace | status.  Allocation 2: the packed bytes.
-    const size_t off_table = 0;
-    const size_t off_chunks = off_table + sizeof(uint64_t) * static_cast<size_t>(bands * nsteps);
-    const size_t off_prefix = round_up(off_chunks + sizeof(uint64_t) * static_cast<size_t>(h->dec_nchunks), 256);
-    const size_t off_bstart = round_up(off_prefix + sizeof(int64_t) * static_cast<size_t>(bands * (Q + 1)), 256);
-    const size_t off_ptable = round_up(off_bstart + sizeof(uint64_t) * static_cast<size_t>(bands), 256);
-    const size_t off_sstart = round_up(off_ptable + sizeof(uint64_t) * static_cast<size_t>(bands * nsteps), 256);
-    const size_t off_plan = round_up(off_sstart + sizeof(uint64_t) * static_cast<size_t>(bands), 256);
-    const size_t off_ws = round_up(off_plan + sizeof(patchk::PackPlan), 256);
-    const size_t off_status = round_up(off_ws + h->workspace_bytes, 256);
-    const size_t status_bytes = 256;
-    const size_t total = off_status + status_bytes;
-    cudaError_t e = patchk::device_pool(&h->pool);
-    if (e == cudaSuccess)
-        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->base), total, h->pool, stream);
-    if (e != cudaSuccess) {
-        delete h;
-        return from_cuda(e);
-    }
-    h->table = reinterpret_cast<uint64_t *>(h->base + off_table);
-    h->chunk_desc = reinterpret_cast<uint64_t *>(h->base + off_chunks);
-    h->pair_prefix_dev = reinterpret_cast<int64_t *>(h->base + off_prefix);
-    h->ptable = reinterpret_cast<uint64_t *>(h->base + off_ptable);
-    patchk::PackPlan *plan_dev = reinterpret_cast<patchk::PackPlan *>(h->base + off_plan);
-    h->workspace = reinterpret_cast<float *>(h->base + off_ws);
-    // status word | pack completion counter | ready flag | decode chunk counter
-    h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
-    e = cudaMemsetAsync(h->status, 0, status_bytes, stream);
-    if (e == cudaSuccess)
-        e = patchk::launch_plan_pack(map, N, K, static_cast<int>(tn), static_cast<int>(tk), h->dec_cp,
-                                     h->dec_cpb, h->table, h->chunk_desc, h->pair_prefix_dev,
-                                     reinterpret_cast<uint64_t *>(h->base + off_bstart), h->ptable,
-                                     reinterpret_cast<uint64_t *>(h->base + off_sstart), plan_dev, stream,
-                                     pattern);
-    patchk::PackPlan plan;
-    h->pair_prefix.assign(static_cast<size_t>(bands * (Q + 1)), 0);
-    preload_gemm_kernels();  // this call waits for the device below in any case
-    if (e == cudaSuccess) e = read_plan(plan_dev, &plan, h->pair_prefix_dev, &h->pair_prefix, stream);
-    if (e != cudaSuccess) {
-        patch_free(h, stream_v);
-        return from_cuda(e);
-    }
-    h->packed_bytes = static_cast<size_t>(plan.packed_bytes);
-    h->side_bytes = static_cast<size_t>(plan.side_bytes);
-    if (plan.packed_bytes >= (1ull << 40) || plan.packed_bytes + plan.side_bytes >= (1ull << 47)) {
-        // chunk descriptors hold 40-bit offsets, table entries 48-bit ones
-        patch_free(h, stream_v);
-        return PATCH_ERR_UNSUPPORTED;
-    }
-    h->sparse_ksteps = static_cast<int64_t>(plan.sparse_ksteps);
-    h->meta_blocks = static_cast<int64_t>(plan.meta_blocks);
-    h->duo_ok = plan.duo_ok ? 1 : 0;
-    h->max_pair_bytes = static_cast<int>(plan.pair_max_bytes);
-    h->chunk_desc_host.assign(plan.first_desc,
-                              plan.first_desc + std::min<int64_t>(h->dec_nchunks, 2 * patchk::kDecMaxCtas));
-    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&h->packed),
-                                std::max<size_t>(h->packed_bytes + h->side_bytes, 16), h->pool, stream);
-    if (e == cudaSuccess)
-        e = patchk::launch_pack(W_bf16, meta, map, N, K, static_cast<int>(tn), static_cast<int>(tk),
-                                h->table, h->side_bytes ? h->ptable : nullptr, h->packed,
-                                h->status + 1, h->status + 2, stream, pattern);
-    if (e != cudaSuccess) {
-        patch_free(h, stream_v);
-        return from_cuda(e);
-    }
-    if (packed_bytes) *packed_bytes = h->packed_bytes;
-    *out = h;
-    return PATCH_OK;
+    return pack_group_impl(&W_bf16, &meta, &map, &shp, 1, out, packed_bytes, stream_v, pattern);
 }
 
 patch_status patch_pack(const void *W_bf16, const uint32_t *meta, const uint32_t *map,
                         patch_shape shp, patch_packed **out, size_t *packed_bytes, void *stream_v) {
     return pack_impl(W_bf16, meta, map, shp, out, packed_bytes, stream_v, 2);
+}
+
+patch_status patch_pack_group(const void *const *Ws_bf16, const uint32_t *const *metas,
+                              const uint32_t *const *maps, const patch_shape *shps, int32_t count,
+                              patch_packed **outs, size_t *packed_bytes, void *stream_v) {
+    return pack_group_impl(Ws_bf16, metas, maps, shps, count, outs, packed_bytes, stream_v, 2);
 }
 
 patch_status patch_pack_nm(const void *W_bf16, const uint32_t *meta, const uint32_t *map,

@@ -75,6 +75,19 @@ cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, 
                              int cpb, uint64_t *table, uint64_t *chunk_desc, int64_t *pair_prefix,
                              uint64_t *band_start, uint64_t *ptable, uint64_t *side_start,
                              PackPlan *plan, cudaStream_t stream, int pattern = 2);
+// The same for up to kPlanMaxGroup matrices in one launch (a block each).
+constexpr int kPlanMaxGroup = 8;
+struct PlanArgs {
+    const uint32_t *map;
+    int64_t N, K;
+    int tn, tk, cp, cpb;
+    uint64_t *table, *chunk_desc;
+    int64_t *pair_prefix;
+    uint64_t *band_start, *ptable, *side_start;
+    PackPlan *plan;
+    int pattern;
+};
+cudaError_t launch_plan_pack_group(const PlanArgs *args, int count, cudaStream_t stream);
 
 struct GemmLaunch {
     const uint8_t *packed;

@@ -27,7 +27,7 @@ EXPORTS = ("patch_score_mask", "patch_pack", "patch_hybrid_gemm", "patch_free",
            "patch_select_maps_global", "patch_test_stall_first_kstep", "patch_pool_usage",
            "patch_colsq", "patch_colsq_partials", "patch_colsq_fold", "patch_test_prefill_kernel",
            "patch_score_mask_nm", "patch_pack_nm", "patch_pack_fp8", "patch_quantize_fp8",
-           "patch_packed_fp8_scales", "patch_hybrid_gemm_group")
+           "patch_packed_fp8_scales", "patch_hybrid_gemm_group", "patch_pack_group")
 
 
 class PatchLibraryError(RuntimeError):
@@ -106,6 +106,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.patch_pool_usage.restype = ctypes.c_int
     lib.patch_pack.argtypes = [vp, vp, vp, PatchShape, ctypes.POINTER(vp),
                                ctypes.POINTER(ctypes.c_size_t), vp]
+    lib.patch_pack_group.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                     ctypes.POINTER(PatchShape), i32, ctypes.POINTER(vp),
+                                     ctypes.POINTER(ctypes.c_size_t), vp]
+    lib.patch_pack_group.restype = ctypes.c_int
     lib.patch_hybrid_gemm.argtypes = [vp, vp, i64, vp, i32, vp]
     lib.patch_hybrid_gemm_group.argtypes = [ctypes.POINTER(vp), i32, vp, i64, ctypes.POINTER(vp), i32, vp]
     lib.patch_hybrid_gemm_group.restype = ctypes.c_int
@@ -402,6 +406,25 @@ def patch_hybrid_gemm(packed: PackedWeight, X: torch.Tensor, out: torch.Tensor |
                                  _dptr(out, want, "out"), 1 if out_fp32 else 0, _stream(stream))
     _check("patch_hybrid_gemm", code)
     return out
+
+
+def patch_pack_group(Ws: list, metas: list, tile_maps: list, *, tile_n: int = 128, tile_k: int = 128,
+                     stream=None) -> list:
+    """patch_pack for several matrices (2:4 tiles) with one host wait; one
+    handle per matrix, each equal to its patch_pack handle."""
+    lib = load_library()
+    n = len(Ws)
+    if len(metas) != n or len(tile_maps) != n:
+        raise ValueError("one meta and one map per weight")
+    w_p = (ctypes.c_void_p * max(n, 1))(*[_dptr(w, torch.bfloat16, "W") for w in Ws])
+    m_p = (ctypes.c_void_p * max(n, 1))(*[_dptr(m, (torch.int32, torch.uint32), "meta") for m in metas])
+    t_p = (ctypes.c_void_p * max(n, 1))(*[_dptr(t, (torch.int32, torch.uint32), "map") for t in tile_maps])
+    shps = (PatchShape * max(n, 1))(*[PatchShape(w.shape[0], w.shape[1], tile_n, tile_k) for w in Ws])
+    outs = (ctypes.c_void_p * max(n, 1))()
+    nbytes = (ctypes.c_size_t * max(n, 1))()
+    code = lib.patch_pack_group(w_p, m_p, t_p, shps, n, outs, nbytes, _stream(stream))
+    _check("patch_pack_group", code)
+    return [PackedWeight(outs[i], (Ws[i].shape[0], Ws[i].shape[1], tile_n, tile_k), nbytes[i]) for i in range(n)]
 
 
 def patch_hybrid_gemm_group(packed: list, X: torch.Tensor, outs: list | None = None,

@@ -136,3 +136,24 @@ def test_binding_fails_loudly_without_library(tmp_path):
             patch.load_library(str(tmp_path / "missing.so"))
         finally:
             patch._lib = saved
+
+
+def test_pack_group_argument_checks(lib):
+    # every member is checked before anything is allocated; no handle is left
+    from sparse_gemm_wanda_b200.patch import PatchShape
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)  # never dereferenced: checks fail first
+    ws = (vp * 2)(fake, fake)
+    outs = (vp * 2)(vp(0x55), vp(0x66))
+    good = PatchShape(256, 256, 128, 128)
+    shps = (PatchShape * 2)(good, PatchShape(256, 256, 32, 128))  # second: unsupported tile
+    assert lib.patch_pack_group(ws, ws, ws, shps, 2, outs, None, None) == 2
+    assert not outs[0] and not outs[1]
+    shps = (PatchShape * 2)(good, PatchShape(200, 256, 64, 128))  # N not a multiple of 128
+    assert lib.patch_pack_group(ws, ws, ws, shps, 2, outs, None, None) == 1
+    shps = (PatchShape * 2)(good, good)
+    nulls = (vp * 2)(fake, None)
+    assert lib.patch_pack_group(nulls, ws, ws, shps, 2, outs, None, None) == 1
+    assert lib.patch_pack_group(ws, ws, ws, shps, 0, outs, None, None) == 1
+    assert lib.patch_pack_group(ws, ws, ws, shps, 9, outs, None, None) == 1
+    assert lib.patch_pack_group(ws, ws, ws, shps, 2, None, None, None) == 1

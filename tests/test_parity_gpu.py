@@ -254,6 +254,55 @@ def test_pack_bit_exact(P, oracle_mod, tn, tk, frac):
     pk.close()
 
 
+@pytest.mark.parametrize("tn,tk", [(128, 128), (64, 64)])
+def test_pack_group_bit_exact(P, oracle_mod, tn, tk):
+    # several matrices of different shapes (an odd band count among them)
+    # packed with one wait: every packed buffer and k-step table equal to the
+    # oracle's, and the products equal to those of single-call handles
+    shapes = [(512, 768, 0.5), (384, 1024, 1.0), (1024, 512, 0.3), (256, 256, 0.0)]
+    ws, rs, tmaps = [], [], []
+    for i, (N, K, frac) in enumerate(shapes):
+        w, xc, _ = make_problem(N, K, 64, 1, seed=900 + i + tn)
+        nt = (N // tn) * (K // tk)
+        tmap = inputs.random_map(nt, int(frac * nt), seed=910 + i + tk)
+        r = P.patch_score_mask(w.cuda(), xc.cuda(), tile_n=tn, tile_k=tk, map_in=tmap.cuda())
+        ref_meta = oracle_mask(oracle_mod, w, xc, tn, tk, tmap=tmap.numpy().view(np.uint32))["meta"]
+        assert np.array_equal(r["meta"].cpu().numpy().view(np.uint32), ref_meta)
+        ws.append(w)
+        rs.append((r, ref_meta))
+        tmaps.append(tmap)
+    pks = P.patch_pack_group([w.cuda() for w in ws], [r["meta"] for r, _ in rs], [r["map"] for r, _ in rs],
+                             tile_n=tn, tile_k=tk)
+    singles = [P.patch_pack(w.cuda(), r["meta"], r["map"], tile_n=tn, tile_k=tk) for w, (r, _) in zip(ws, rs)]
+    for (N, K, _), w, (r, ref_meta), tmap, pk, pk1 in zip(shapes, ws, rs, tmaps, pks, singles):
+        packed, table = pk.export()
+        torch.cuda.synchronize()
+        ref_packed, ref_table = oracle_mod.pack(bf16_bits(w), ref_meta, tmap.numpy().view(np.uint32), tn, tk)
+        assert pk.packed_bytes == ref_packed.size
+        assert np.array_equal(table.cpu().numpy().view(np.uint64), ref_table)
+        assert np.array_equal(packed.cpu().numpy(), ref_packed)
+        for M in (8, 300):
+            x = inputs.activations(M, K, 920 + M, None).cuda()
+            y = P.patch_hybrid_gemm(pk, x, out_fp32=True)
+            y1 = P.patch_hybrid_gemm(pk1, x, out_fp32=True)
+            torch.cuda.synchronize()
+            assert torch.equal(y, y1)
+        assert P.patch_get_status(pk) == 0
+    for pk in pks + singles:
+        pk.close()
+
+
+def test_pack_group_bad_member_leaves_no_handle(P):
+    # a member that fails its checks fails the call before anything is made
+    w = torch.zeros(256, 256, dtype=torch.bfloat16, device="cuda")
+    meta = torch.zeros(256, 8, dtype=torch.int32, device="cuda")
+    tmap = torch.zeros(1, dtype=torch.int32, device="cuda")
+    w_bad = torch.zeros(200, 256, dtype=torch.bfloat16, device="cuda")  # N not a multiple of 128
+    with pytest.raises(P.PatchError) as e:
+        P.patch_pack_group([w, w_bad], [meta, meta], [tmap, tmap])
+    assert e.value.code == 1
+
+
 # ----------------------------------------------------------------------- GEMM
 
 def run_case(P, oracle_mod, N, K, M, tn, tk, frac, seed, fp32_mode, sample=None):
