@@ -583,15 +583,6 @@ cudaError_t launch_plan_pack_group(const PlanArgs *args, int count, cudaStream_t
     return cudaGetLastError();
 }
 
-cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, int tk, int cp,
-                             int cpb, uint64_t *table, uint64_t *chunk_desc, int64_t *pair_prefix,
-                             uint64_t *band_start, uint64_t *ptable, uint64_t *side_start,
-                             PackPlan *plan, cudaStream_t stream, int pattern) {
-    const PlanArgs a{map, N, K, tn, tk, cp, cpb, table, chunk_desc, pair_prefix, band_start, ptable, side_start,
-                     plan, pattern};
-    return launch_plan_pack_group(&a, 1, stream);
-}
-
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                         int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
                         uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream, int pattern) {

@@ -66,16 +66,12 @@ struct PackPlan {
     uint32_t pad_;
     uint64_t first_desc[2 * kDecMaxCtas];  // decode chunk descriptors 0 .. 2*kDecMaxCtas-1
 };
-// Writes the k-step table [bands][nsteps], the decode chunk descriptors
-// [bands][cpb], the per-band cumulative k-pair bytes [bands][nsteps/2 + 1],
-// the first byte of each band (scratch [bands]), the prefill table
-// [bands][nsteps] with the side-region offsets of its dense copies (scratch
-// side_start [bands]) and the plan summary; one block.
-cudaError_t launch_plan_pack(const uint32_t *map, int64_t N, int64_t K, int tn, int tk, int cp,
-                             int cpb, uint64_t *table, uint64_t *chunk_desc, int64_t *pair_prefix,
-                             uint64_t *band_start, uint64_t *ptable, uint64_t *side_start,
-                             PackPlan *plan, cudaStream_t stream, int pattern = 2);
-// The same for up to kPlanMaxGroup matrices in one launch (a block each).
+// Plans the packed layout of up to kPlanMaxGroup matrices, one block each:
+// writes each matrix's k-step table [bands][nsteps], decode chunk
+// descriptors [bands][cpb], per-band cumulative k-pair bytes
+// [bands][nsteps/2 + 1], the first byte of each band (scratch [bands]), the
+// prefill table [bands][nsteps] with the side-region offsets of its dense
+// copies (scratch side_start [bands]) and the plan summary.
 constexpr int kPlanMaxGroup = 8;
 struct PlanArgs {
     const uint32_t *map;
