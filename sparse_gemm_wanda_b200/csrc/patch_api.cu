@@ -96,39 +96,53 @@ patch_status check_device(int *num_sms) {
     return PATCH_OK;
 }
 
-// The plan summaries written by plan_pack_kernel, read back into page-locked
-// memory (one buffer of kPlanMaxGroup plans per device, held under the lock
-// until the copies landed), and each matrix's per-band k-pair prefix the
-// prefill kernels balance their work with (into `prefix[i]`, pageable: that
-// copy returns once it has landed).  The stream is waited for once, here; no
+// The plan summaries written by plan_pack_kernel and each matrix's per-band
+// k-pair prefix (the prefill kernels balance their work with it), read back
+// into one page-locked buffer per device (grown on demand, held under the
+// lock until the copies landed) and from there into `dst` and `prefix[i]`.
+// Every copy is asynchronous; the stream is waited for once, here, and no
 // later call on the handles waits.
 cudaError_t read_plans(const patchk::PackPlan *const *src, patchk::PackPlan *dst, const int64_t *const *prefix_src,
                        std::vector<int64_t> *const *prefix, int count, cudaStream_t stream) {
     static std::mutex mu;
-    static std::map<int, patchk::PackPlan *> bufs;
+    static std::map<int, std::pair<uint8_t *, size_t>> bufs;
     if (count < 1 || count > patchk::kPlanMaxGroup) return cudaErrorInvalidValue;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    size_t need = sizeof(patchk::PackPlan) * static_cast<size_t>(count);
+    for (int i = 0; i < count; ++i) need += sizeof(int64_t) * prefix[i]->size();
     std::lock_guard<std::mutex> lock(mu);
-    patchk::PackPlan *&buf = bufs[dev];
-    if (!buf) {
-        e = cudaMallocHost(reinterpret_cast<void **>(&buf), sizeof(patchk::PackPlan) * patchk::kPlanMaxGroup);
+    std::pair<uint8_t *, size_t> &buf = bufs[dev];
+    if (buf.second < need) {
+        if (buf.first) cudaFreeHost(buf.first);  // no copy into it is in flight: each call waits for its own
+        buf = {nullptr, 0};
+        e = cudaMallocHost(reinterpret_cast<void **>(&buf.first), need);
         if (e != cudaSuccess) {
-            buf = nullptr;
+            buf = {nullptr, 0};
             return e;
         }
+        buf.second = need;
     }
+    patchk::PackPlan *plans = reinterpret_cast<patchk::PackPlan *>(buf.first);
+    int64_t *pre = reinterpret_cast<int64_t *>(buf.first + sizeof(patchk::PackPlan) * static_cast<size_t>(count));
+    size_t at = 0;
     for (int i = 0; i < count && e == cudaSuccess; ++i) {
-        e = cudaMemcpyAsync(buf + i, src[i], sizeof(patchk::PackPlan), cudaMemcpyDeviceToHost, stream);
+        e = cudaMemcpyAsync(plans + i, src[i], sizeof(patchk::PackPlan), cudaMemcpyDeviceToHost, stream);
         if (e == cudaSuccess && !prefix[i]->empty())
-            e = cudaMemcpyAsync(prefix[i]->data(), prefix_src[i], sizeof(int64_t) * prefix[i]->size(),
-                                cudaMemcpyDeviceToHost, stream);
+            e = cudaMemcpyAsync(pre + at, prefix_src[i], sizeof(int64_t) * prefix[i]->size(), cudaMemcpyDeviceToHost,
+                                stream);
+        at += prefix[i]->size();
     }
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-    if (e == cudaSuccess)
-        for (int i = 0; i < count; ++i) dst[i] = buf[i];
-    return e;
+    if (e != cudaSuccess) return e;
+    at = 0;
+    for (int i = 0; i < count; ++i) {
+        dst[i] = plans[i];
+        std::copy(pre + at, pre + at + prefix[i]->size(), prefix[i]->begin());
+        at += prefix[i]->size();
+    }
+    return cudaSuccess;
 }
 
 // Failure-detection test hook (see patch_test_stall_first_kstep): read from
