@@ -271,6 +271,7 @@ struct PlanGroup {
     int64_t *pair_prefix[kPlanMaxGroup];
     uint64_t *band_start[kPlanMaxGroup], *ptable[kPlanMaxGroup], *side_start[kPlanMaxGroup];
     PackPlan *plan[kPlanMaxGroup];
+    uint32_t *status[kPlanMaxGroup];  // the handle's 64 status words, zeroed here
     int pattern[kPlanMaxGroup];
 };
 
@@ -287,6 +288,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) plan_pack_kernel(const __grid
     uint64_t *__restrict__ ptable = grp.ptable[gi];
     uint64_t *__restrict__ side_start = grp.side_start[gi];
     PackPlan *__restrict__ plan = grp.plan[gi];
+    if (grp.status[gi] && threadIdx.x < kStatusWords) grp.status[gi][threadIdx.x] = 0u;
     __shared__ unsigned long long warp_sum[kPlanWarps];
     __shared__ uint32_t types[kPlanWarps][2][kPlanMaxWords];
     __shared__ uint32_t tcache[kPlanCacheBands * kPlanMaxWords];
@@ -576,6 +578,7 @@ cudaError_t launch_plan_pack_group(const PlanArgs *args, int count, cudaStream_t
         grp.ptable[i] = a.ptable;
         grp.side_start[i] = a.side_start;
         grp.plan[i] = a.plan;
+        grp.status[i] = a.status;
         grp.pattern[i] = a.pattern;
     }
     plan_pack_kernel<<<count, kPlanThreads, 0, stream>>>(grp);

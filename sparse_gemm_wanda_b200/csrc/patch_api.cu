@@ -611,7 +611,7 @@ static patch_status pack_group_impl(const void *const *Ws, const uint32_t *const
         const size_t off_plan = round_up(off_sstart + sizeof(uint64_t) * static_cast<size_t>(bands), 256);
         const size_t off_ws = round_up(off_plan + sizeof(patchk::PackPlan), 256);
         const size_t off_status = round_up(off_ws + h->workspace_bytes, 256);
-        const size_t status_bytes = 256;
+        const size_t status_bytes = sizeof(uint32_t) * patchk::kStatusWords;
         const size_t total = off_status + status_bytes;
         cudaError_t e = patchk::device_pool(&h->pool);
         if (e == cudaSuccess)
@@ -624,13 +624,12 @@ static patch_status pack_group_impl(const void *const *Ws, const uint32_t *const
         patchk::PackPlan *pd = reinterpret_cast<patchk::PackPlan *>(h->base + off_plan);
         h->workspace = reinterpret_cast<float *>(h->base + off_ws);
         // status word | pack completion counter | ready flag | decode chunk counter
+        // (zeroed by the plan launch, before any kernel reads them)
         h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
-        e = cudaMemsetAsync(h->status, 0, status_bytes, stream);
-        if (e != cudaSuccess) return fail(from_cuda(e));
         pa[i] = patchk::PlanArgs{maps[i], N, K, static_cast<int>(shp.tile_n), static_cast<int>(shp.tile_k),
                                  h->dec_cp, h->dec_cpb, h->table, h->chunk_desc, h->pair_prefix_dev,
                                  reinterpret_cast<uint64_t *>(h->base + off_bstart), h->ptable,
-                                 reinterpret_cast<uint64_t *>(h->base + off_sstart), pd, pattern};
+                                 reinterpret_cast<uint64_t *>(h->base + off_sstart), pd, pattern, h->status};
         plan_dev[i] = pd;
         prefix_dev[i] = h->pair_prefix_dev;
         h->pair_prefix.assign(static_cast<size_t>(bands * (Q + 1)), 0);

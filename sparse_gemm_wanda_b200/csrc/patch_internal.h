@@ -82,7 +82,9 @@ struct PlanArgs {
     uint64_t *band_start, *ptable, *side_start;
     PackPlan *plan;
     int pattern;
+    uint32_t *status;  // the handle's kStatusWords status words (zeroed by the plan launch), or null
 };
+constexpr int kStatusWords = 64;
 cudaError_t launch_plan_pack_group(const PlanArgs *args, int count, cudaStream_t stream);
 
 struct GemmLaunch {
