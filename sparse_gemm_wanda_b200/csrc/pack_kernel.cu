@@ -64,8 +64,7 @@ __global__ void __launch_bounds__(kPackThreads, 8)
 pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
             const uint32_t *__restrict__ map, int64_t N, int64_t K, int tn, int tk,
             const uint64_t *__restrict__ table, const uint64_t *__restrict__ ptable,
-            uint8_t *__restrict__ out, uint32_t *__restrict__ done, uint32_t *__restrict__ ready,
-            int pattern) {
+            uint8_t *__restrict__ out, int pattern) {
     const int64_t nsteps = K / kStep;
     const int64_t steps_all = (N / kBand) * nsteps;
     (void)steps_all;
@@ -197,18 +196,17 @@ pack_kernel(const uint16_t *__restrict__ W, const uint32_t *__restrict__ meta,
                 make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
     }
-    // completion: every thread's stores are ordered before the block's ticket;
-    // the last block publishes the ready flag the GEMM reads before its
-    // griddepcontrol.wait
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const uint32_t v = atomicAdd(done, 1u);
-        if (v == gridDim.x - 1) {
-            __threadfence();
-            st_release_gpu(ready, 1u);
-        }
-    }
+}
+
+// The ready flags of up to kPlanMaxGroup handles, set (release) by one
+// thread each once every kernel before this one on the stream has completed:
+// the packed bytes are then final, and a GEMM that reads its flag as set may
+// fetch weights before its griddepcontrol.wait.
+struct ReadyList {
+    uint32_t *ready[kPlanMaxGroup];
+};
+__global__ void publish_ready_list_kernel(const __grid_constant__ ReadyList list, int count) {
+    if (static_cast<int>(threadIdx.x) < count) st_release_gpu(list.ready[threadIdx.x], 1u);
 }
 
 // ------------------------------------------------------------------- plan
@@ -588,14 +586,28 @@ cudaError_t launch_plan_pack_group(const PlanArgs *args, int count, cudaStream_t
 
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                         int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
-                        uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream, int pattern) {
+                        uint8_t *out, cudaStream_t stream, int pattern) {
     const int64_t blocks = (N / kBand) * (K / kStep);
     if (blocks > 0x7FFFFFFF || (pattern != 2 && pattern != 4)) return cudaErrorInvalidValue;
     pack_kernel<<<static_cast<unsigned>(blocks), kPackThreads, 0, stream>>>(
-        static_cast<const uint16_t *>(W), meta, map, N, K, tn, tk, table, ptable, out, done, ready,
-        pattern);
+        static_cast<const uint16_t *>(W), meta, map, N, K, tn, tk, table, ptable, out, pattern);
     note_launches(1);
     return cudaGetLastError();
+}
+
+cudaError_t launch_publish_ready(uint32_t *const *ready, int count, cudaStream_t stream) {
+    if (count < 1 || count > kPlanMaxGroup) return cudaErrorInvalidValue;
+    ReadyList list{};
+    for (int i = 0; i < count; ++i) list.ready[i] = ready[i];
+    publish_ready_list_kernel<<<1, 32, 0, stream>>>(list, count);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+void preload_pack_kernels() {
+    cudaFuncAttributes a;
+    (void)cudaFuncGetAttributes(&a, pack_kernel);
+    (void)cudaFuncGetAttributes(&a, publish_ready_list_kernel);
 }
 
 }  // namespace patchk

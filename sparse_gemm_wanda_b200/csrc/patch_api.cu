@@ -422,6 +422,7 @@ static void preload_gemm_kernels() {
     patchk::preload_fp8_gemm_kernels();
     patchk::preload_duo_fp8_kernels();
     patchk::preload_fp8_quantize_kernels();
+    patchk::preload_pack_kernels();
     if (named) done.insert(id);
 }
 
@@ -623,7 +624,7 @@ static patch_status pack_group_impl(const void *const *Ws, const uint32_t *const
         h->ptable = reinterpret_cast<uint64_t *>(h->base + off_ptable);
         patchk::PackPlan *pd = reinterpret_cast<patchk::PackPlan *>(h->base + off_plan);
         h->workspace = reinterpret_cast<float *>(h->base + off_ws);
-        // status word | pack completion counter | ready flag | decode chunk counter
+        // status word | (unused) | ready flag | decode chunk counter
         // (zeroed by the plan launch, before any kernel reads them)
         h->status = reinterpret_cast<uint32_t *>(h->base + off_status);
         pa[i] = patchk::PlanArgs{maps[i], N, K, static_cast<int>(shp.tile_n), static_cast<int>(shp.tile_k),
@@ -658,9 +659,14 @@ static patch_status pack_group_impl(const void *const *Ws, const uint32_t *const
         if (e == cudaSuccess)
             e = patchk::launch_pack(Ws[i], metas[i], maps[i], h->shp.N, h->shp.K, static_cast<int>(h->shp.tile_n),
                                     static_cast<int>(h->shp.tile_k), h->table, h->side_bytes ? h->ptable : nullptr,
-                                    h->packed, h->status + 1, h->status + 2, stream, pattern);
+                                    h->packed, stream, pattern);
         if (e != cudaSuccess) return fail(from_cuda(e));
     }
+    // every handle's ready flag (status word 2), once all the packs above completed
+    uint32_t *ready[patchk::kPlanMaxGroup];
+    for (int i = 0; i < count; ++i) ready[i] = hs[i]->status + 2;
+    e = patchk::launch_publish_ready(ready, count, stream);
+    if (e != cudaSuccess) return fail(from_cuda(e));
     for (int i = 0; i < count; ++i) {
         if (packed_bytes) packed_bytes[i] = hs[i]->packed_bytes;
         outs[i] = hs[i];

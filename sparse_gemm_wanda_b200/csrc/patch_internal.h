@@ -39,14 +39,16 @@ cudaError_t launch_select_maps_global(const double *loss_cat, const int64_t *n_t
                                       int64_t n_sparse, int32_t *rank, uint32_t *const *maps,
                                       cudaStream_t stream);
 
-// `done` (a zeroed counter) and `ready` (zeroed) live in the handle: the last
-// block to finish publishes ready = 1 with release semantics.
 // `ptable` (may be null) adds the dense copies of the prefill table's side
 // entries, written after the packed bytes.
 cudaError_t launch_pack(const void *W, const uint32_t *meta, const uint32_t *map, int64_t N,
                         int64_t K, int tn, int tk, const uint64_t *table, const uint64_t *ptable,
-                        uint8_t *out, uint32_t *done, uint32_t *ready, cudaStream_t stream,
-                        int pattern = 2);
+                        uint8_t *out, cudaStream_t stream, int pattern = 2);
+// Sets each handle's ready flag (zeroed, in the handle) to 1 with release
+// semantics once the kernels queued before it on the stream (the packs) have
+// completed; up to kPlanMaxGroup flags, one launch.
+cudaError_t launch_publish_ready(uint32_t *const *ready, int count, cudaStream_t stream);
+void preload_pack_kernels();
 
 // Split-K decode kernel: CTAs whose first chunks travel in the kernel
 // parameters, at most.
